@@ -1,0 +1,157 @@
+"""CPU oracle for the frame recurrences (fp64), as a ctypes binding of oracle.c.
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the CPU
+baseline leg of ``bench.py`` may import this package; the library path
+(``linear_attention_video_gdn_b200``) never does.  It shares no code with the
+CUDA path.
+
+What is computed, and the passages it follows, is stated at the top of
+``oracle.c``.  Parity is pinned by the ``-m "not gpu"`` tests in
+``tests/test_oracle_pins.py`` (brute-force dense products, closed forms,
+invariants, O(N^2) masked attention).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+KEY_NORM_EPS = 1e-6
+
+
+def build(force: bool = False) -> str:
+    """Compile liboracle.so in place (gcc -O2, strict IEEE double: no -ffast-math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        subprocess.check_call(["gcc", "-O2", "-fno-fast-math", "-ffp-contract=off", "-fPIC", "-shared",
+                               "-o", _LIB, _SRC, "-lm", "-lpthread"])
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB)
+        P = ctypes.c_void_p
+        I64 = ctypes.c_int64
+        lib.oracle_gdn.argtypes = [P, P, P, P, P, ctypes.c_int, P, P, P, I64, I64, I64, I64, I64, I64,
+                                   I64, I64, P, I64, I64, ctypes.c_int]
+        lib.oracle_gdn.restype = ctypes.c_int
+        lib.oracle_relu_la.argtypes = [P, P, P, P, P, P, P, P, I64, I64, I64, I64, I64, I64, ctypes.c_double]
+        lib.oracle_relu_la.restype = ctypes.c_int
+        lib.oracle_gate_alpha.argtypes = [ctypes.c_double]
+        lib.oracle_gate_alpha.restype = ctypes.c_double
+        lib.oracle_gate_beta.argtypes = [ctypes.c_double]
+        lib.oracle_gate_beta.restype = ctypes.c_double
+        _lib = lib
+    return _lib
+
+
+def _f32(x):
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float32))
+
+
+def _f64(x):
+    return None if x is None else np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data
+
+
+def gate_alpha(a: float) -> float:
+    """alpha = exp(-softplus(a)) in double."""
+    return float(_load().oracle_gate_alpha(float(a)))
+
+
+def gate_beta(b: float) -> float:
+    """beta = sigmoid(b) in double."""
+    return float(_load().oracle_gate_beta(float(b)))
+
+
+def gdn(q, k, v, alpha, beta, *, F: int, L: int, gates_are_logits: bool = True, state_in=None,
+        cols=None, heads=None, want_o: bool = True, nthreads: int | None = None):
+    """Gated DeltaNet frame recurrence in fp64.
+
+    q, k: [..., F*L, dk]; v: [..., F*L, dv]; alpha: [..., F]; beta: [..., F*L];
+    leading dims are flattened into heads.  state_in: [..., dk, dv] or None.
+    cols: (lo, hi) range of d_v columns to compute (others left as NaN).
+    heads: optional subset of flat head indices (outputs still full-sized,
+    other heads NaN).  Returns (o, state_out) as float64 arrays.
+    """
+    q, k, v, alpha, beta = map(_f32, (q, k, v, alpha, beta))
+    lead = q.shape[:-2]
+    N, dk = q.shape[-2:]
+    dv = v.shape[-1]
+    assert N == F * L and k.shape == q.shape and v.shape[:-1] == q.shape[:-1]
+    nh = int(np.prod(lead)) if lead else 1
+    assert alpha.size == nh * F and beta.size == nh * N
+    s_in = _f64(state_in)
+    if s_in is not None:
+        assert s_in.size == nh * dk * dv
+    lo, hi = (0, dv) if cols is None else cols
+    o = np.full(lead + (N, dv), np.nan) if want_o else None
+    s_out = np.full(lead + (dk, dv), np.nan)
+    hl = None if heads is None else np.ascontiguousarray(np.asarray(heads, dtype=np.int64))
+    nthreads = nthreads or (os.cpu_count() or 1)
+    col_block = max(1, min(hi - lo, 16)) if hi > lo else 1
+    rc = _load().oracle_gdn(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), int(gates_are_logits),
+                            _ptr(s_in), _ptr(s_out), _ptr(o), 1, nh, F, L, dk, dv, lo, hi,
+                            _ptr(hl), 0 if hl is None else hl.size, col_block, nthreads)
+    if rc != 0:
+        raise ValueError("oracle_gdn: invalid arguments")
+    return o, s_out
+
+
+def relu_la(q, k, v, *, F: int, L: int, kv_in=None, z_in=None, eps: float = 1e-6):
+    """Block-causal ReLU linear attention in fp64.  Returns (o, kv_out, z_out)."""
+    q, k, v = map(_f32, (q, k, v))
+    lead = q.shape[:-2]
+    N, dk = q.shape[-2:]
+    dv = v.shape[-1]
+    assert N == F * L
+    nh = int(np.prod(lead)) if lead else 1
+    kv_in, z_in = _f64(kv_in), _f64(z_in)
+    o = np.empty(lead + (N, dv))
+    kv_out = np.empty(lead + (dk, dv))
+    z_out = np.empty(lead + (dk,))
+    rc = _load().oracle_relu_la(_ptr(q), _ptr(k), _ptr(v), _ptr(kv_in), _ptr(z_in), _ptr(kv_out),
+                                _ptr(z_out), _ptr(o), 1, nh, F, L, dk, dv, float(eps))
+    if rc != 0:
+        raise ValueError("oracle_relu_la: invalid arguments")
+    return o, kv_out, z_out
+
+
+def gdn_stream(step_inputs, *, steps: int, L: int, state_in=None, cols=None):
+    """Streaming block-cache decode: frames of ``steps`` calls each.
+
+    step_inputs(call) -> dict(q, k, v, a, b) for one frame (F=1) of fresh
+    inputs.  Every step of frame f starts from the committed state S_{f-1};
+    the state after the last step of the frame is committed.  Returns the
+    list of per-call outputs o and the final committed state.
+    """
+    S = None if state_in is None else np.asarray(state_in, np.float64)
+    outs = []
+    call = 0
+    frames = 0
+    while True:
+        x0 = step_inputs(call)
+        if x0 is None:
+            break
+        last_state = None
+        for s in range(steps):
+            x = x0 if s == 0 else step_inputs(call)
+            o, s_out = gdn(x["q"], x["k"], x["v"], x["a"], x["b"], F=1, L=L, state_in=S, cols=cols)
+            outs.append(o)
+            last_state = s_out
+            call += 1
+        S = last_state
+        frames += 1
+    return outs, S

@@ -1,0 +1,235 @@
+/*
+ * CPU oracle for the frame-wise linear-attention recurrences (fp64).
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the CPU
+ * baseline leg of the benchmark may load this library.  It shares no code
+ * with the CUDA path and is deliberately plain: per-token loops in double,
+ * in the order the method states them, with no chunking, no blocking and no
+ * re-association.  Inputs are read as float (bf16 inputs are passed as the
+ * exact float values of the bf16 numbers) and widened to double.
+ *
+ * Sources for what is computed:
+ *  - "SANA-WM, an open-source 2.6B world model for 1-minute 720p video"
+ *    (GeekNews, vi.news.hada.io/topic?id=29572 and its Turkish twin
+ *    tr.news.hada.io/topic?id=29572), section "Core design and generation
+ *    pipeline": attention is a frame-wise (frame-level) Gated DeltaNet.
+ *  - "How NVIDIA SANA-WM generates 60-second 720p video on one GPU"
+ *    (dothoosh.com): the Gated DeltaNet keeps a fixed-size recurrent state,
+ *    independent of video length.
+ *  - "SANA-Video: Efficient Video Generation with Block Linear Diffusion
+ *    Transformer (ICLR 2026 oral)" talk transcript (shadowingenglish.com),
+ *    block KV cache passage: the linear-attention state is a fixed D x D
+ *    matrix; block i adds its own KV contribution to the cached state of
+ *    block i-1, and every token of a block reads that state.
+ *
+ * The pages print no equation.  The update rules below are the library's
+ * definition of the two modes (the plainest reading consistent with the
+ * pages), written in the stored layout S[i][j], i over d_k, j over d_v:
+ *
+ *  Gated DeltaNet, per (b, h), S starts at state_in (or 0):
+ *    for each frame f:  alpha_f = exp(-softplus(a_f))   (or given)
+ *                       S <- alpha_f * S
+ *      for each token t of f, in order:
+ *                       khat = k_t / max(||k_t||_2, 1e-6)
+ *                       beta = sigmoid(b_t)              (or given)
+ *                       r    = S^T khat - v_t            (length d_v)
+ *                       S   <- S - beta * khat r^T
+ *      for each token t of f:  o_t = S^T q_t  (state after the whole frame)
+ *    state_out = S.
+ *
+ *  Block-causal ReLU linear attention, per (b, h), S = kv_in (or 0),
+ *  z = z_in (or 0):
+ *    for each frame f:  S += sum_{t in f} relu(k_t) v_t^T
+ *                       z += sum_{t in f} relu(k_t)
+ *      for each token t of f:
+ *        o_t = relu(q_t)^T S / (relu(q_t)^T z + eps)
+ *
+ * Threads split the work over independent (b, h) heads and blocks of d_v
+ * columns (column j of S and o depends only on column j of v and S0), which
+ * changes no arithmetic.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define GDN_KEY_NORM_EPS 1e-6
+
+/* alpha = exp(-softplus(a)) with softplus(a) = log(1 + exp(a)). */
+static double gate_alpha(double a) { return exp(-log1p(exp(a))); }
+/* beta = sigmoid(b) = 1 / (1 + exp(-b)). */
+static double gate_beta(double b) { return 1.0 / (1.0 + exp(-b)); }
+
+double oracle_gate_alpha(double a) { return gate_alpha(a); }
+double oracle_gate_beta(double b) { return gate_beta(b); }
+
+typedef struct {
+  const float *q, *k, *v, *alpha, *beta;
+  int logits;
+  const double *s_in;
+  double *s_out, *o;
+  int64_t F, L, dk, dv;
+  int64_t bh;          /* flat head index */
+  int64_t c0, c1;      /* column range [c0, c1) of d_v */
+} gdn_unit_t;
+
+static void gdn_unit(const gdn_unit_t *u) {
+  const int64_t F = u->F, L = u->L, dk = u->dk, dv = u->dv, N = F * L;
+  const int64_t nc = u->c1 - u->c0;
+  const float *q = u->q + u->bh * N * dk;
+  const float *k = u->k + u->bh * N * dk;
+  const float *v = u->v + u->bh * N * dv;
+  const float *al = u->alpha + u->bh * F;
+  const float *be = u->beta + u->bh * N;
+  double *S = (double *)calloc((size_t)(dk * nc), sizeof(double)); /* S[i][j - c0] */
+  double *kh = (double *)malloc(sizeof(double) * (size_t)dk);
+  double *r = (double *)malloc(sizeof(double) * (size_t)nc);
+  if (u->s_in)
+    for (int64_t i = 0; i < dk; ++i)
+      for (int64_t j = 0; j < nc; ++j) S[i * nc + j] = u->s_in[u->bh * dk * dv + i * dv + u->c0 + j];
+  for (int64_t f = 0; f < F; ++f) {
+    const double alpha = u->logits ? gate_alpha((double)al[f]) : (double)al[f];
+    for (int64_t e = 0; e < dk * nc; ++e) S[e] *= alpha;
+    for (int64_t t = f * L; t < (f + 1) * L; ++t) {
+      double ss = 0.0;
+      for (int64_t i = 0; i < dk; ++i) ss += (double)k[t * dk + i] * (double)k[t * dk + i];
+      double nrm = sqrt(ss);
+      double den = nrm > GDN_KEY_NORM_EPS ? nrm : GDN_KEY_NORM_EPS;
+      for (int64_t i = 0; i < dk; ++i) kh[i] = (double)k[t * dk + i] / den;
+      const double beta = u->logits ? gate_beta((double)be[t]) : (double)be[t];
+      for (int64_t j = 0; j < nc; ++j) {
+        double p = 0.0;
+        for (int64_t i = 0; i < dk; ++i) p += S[i * nc + j] * kh[i];
+        r[j] = p - (double)v[t * dv + u->c0 + j];
+      }
+      for (int64_t i = 0; i < dk; ++i)
+        for (int64_t j = 0; j < nc; ++j) S[i * nc + j] -= beta * kh[i] * r[j];
+    }
+    if (u->o)
+      for (int64_t t = f * L; t < (f + 1) * L; ++t)
+        for (int64_t j = 0; j < nc; ++j) {
+          double acc = 0.0;
+          for (int64_t i = 0; i < dk; ++i) acc += S[i * nc + j] * (double)q[t * dk + i];
+          u->o[(u->bh * N + t) * dv + u->c0 + j] = acc;
+        }
+  }
+  if (u->s_out)
+    for (int64_t i = 0; i < dk; ++i)
+      for (int64_t j = 0; j < nc; ++j) u->s_out[u->bh * dk * dv + i * dv + u->c0 + j] = S[i * nc + j];
+  free(S);
+  free(kh);
+  free(r);
+}
+
+typedef struct {
+  gdn_unit_t *units;
+  int64_t n;
+  int64_t next;
+  pthread_mutex_t mu;
+} pool_t;
+
+static void *gdn_worker(void *p) {
+  pool_t *pl = (pool_t *)p;
+  for (;;) {
+    pthread_mutex_lock(&pl->mu);
+    int64_t i = pl->next++;
+    pthread_mutex_unlock(&pl->mu);
+    if (i >= pl->n) return NULL;
+    gdn_unit(&pl->units[i]);
+  }
+}
+
+/*
+ * Gated DeltaNet frame recurrence.  Layouts (row-major, contiguous):
+ *   q, k [B,H,F*L,dk]; v [B,H,F*L,dv]; alpha [B,H,F]; beta [B,H,F*L];
+ *   state_in/state_out [B,H,dk,dv] (nullable); o [B,H,F*L,dv] (nullable).
+ * Only d_v columns [col_lo, col_hi) of o and state_out are written.
+ * heads: optional list of nheads flat head indices to compute (NULL = all).
+ */
+int oracle_gdn(const float *q, const float *k, const float *v, const float *alpha, const float *beta,
+               int gates_are_logits, const double *state_in, double *state_out, double *o,
+               int64_t B, int64_t H, int64_t F, int64_t L, int64_t dk, int64_t dv,
+               int64_t col_lo, int64_t col_hi, const int64_t *heads, int64_t nheads,
+               int64_t col_block, int nthreads) {
+  if (B < 0 || H < 0 || F < 0 || L < 0 || dk <= 0 || dv <= 0) return 1;
+  if (col_lo < 0 || col_hi > dv || col_lo > col_hi) return 1;
+  if (col_block <= 0) col_block = dv;
+  int64_t nh = heads ? nheads : B * H;
+  int64_t nb = (col_hi - col_lo + col_block - 1) / col_block;
+  int64_t n = nh * nb;
+  if (n == 0) return 0;
+  gdn_unit_t *units = (gdn_unit_t *)calloc((size_t)n, sizeof(gdn_unit_t));
+  for (int64_t h = 0; h < nh; ++h)
+    for (int64_t c = 0; c < nb; ++c) {
+      gdn_unit_t *u = &units[h * nb + c];
+      u->q = q; u->k = k; u->v = v; u->alpha = alpha; u->beta = beta;
+      u->logits = gates_are_logits; u->s_in = state_in; u->s_out = state_out; u->o = o;
+      u->F = F; u->L = L; u->dk = dk; u->dv = dv;
+      u->bh = heads ? heads[h] : h;
+      u->c0 = col_lo + c * col_block;
+      u->c1 = u->c0 + col_block < col_hi ? u->c0 + col_block : col_hi;
+    }
+  pool_t pl;
+  pl.units = units; pl.n = n; pl.next = 0;
+  pthread_mutex_init(&pl.mu, NULL);
+  if (nthreads < 1) nthreads = 1;
+  if (nthreads > n) nthreads = (int)n;
+  if (nthreads > 512) nthreads = 512;
+  pthread_t th[512];
+  for (int t = 1; t < nthreads; ++t) pthread_create(&th[t], NULL, gdn_worker, &pl);
+  gdn_worker(&pl);
+  for (int t = 1; t < nthreads; ++t) pthread_join(th[t], NULL);
+  pthread_mutex_destroy(&pl.mu);
+  free(units);
+  return 0;
+}
+
+/*
+ * Block-causal ReLU linear attention.  Layouts: q, k [B,H,F*L,dk];
+ * v [B,H,F*L,dv]; kv_in/kv_out [B,H,dk,dv]; z_in/z_out [B,H,dk] (nullable);
+ * o [B,H,F*L,dv].  Single-threaded per call; callers split heads.
+ */
+int oracle_relu_la(const float *q, const float *k, const float *v, const double *kv_in,
+                   const double *z_in, double *kv_out, double *z_out, double *o,
+                   int64_t B, int64_t H, int64_t F, int64_t L, int64_t dk, int64_t dv, double eps) {
+  if (B < 0 || H < 0 || F < 0 || L < 0 || dk <= 0 || dv <= 0) return 1;
+  const int64_t N = F * L;
+  double *S = (double *)malloc(sizeof(double) * (size_t)(dk * dv));
+  double *z = (double *)malloc(sizeof(double) * (size_t)dk);
+  double *rq = (double *)malloc(sizeof(double) * (size_t)dk);
+  for (int64_t bh = 0; bh < B * H; ++bh) {
+    const float *qh = q + bh * N * dk, *kh = k + bh * N * dk, *vh = v + bh * N * dv;
+    for (int64_t e = 0; e < dk * dv; ++e) S[e] = kv_in ? kv_in[bh * dk * dv + e] : 0.0;
+    for (int64_t i = 0; i < dk; ++i) z[i] = z_in ? z_in[bh * dk + i] : 0.0;
+    for (int64_t f = 0; f < F; ++f) {
+      for (int64_t t = f * L; t < (f + 1) * L; ++t)
+        for (int64_t i = 0; i < dk; ++i) {
+          double rk = (double)kh[t * dk + i];
+          if (rk < 0.0) rk = 0.0;
+          z[i] += rk;
+          for (int64_t j = 0; j < dv; ++j) S[i * dv + j] += rk * (double)vh[t * dv + j];
+        }
+      for (int64_t t = f * L; t < (f + 1) * L; ++t) {
+        double den = 0.0;
+        for (int64_t i = 0; i < dk; ++i) {
+          double x = (double)qh[t * dk + i];
+          rq[i] = x > 0.0 ? x : 0.0;
+          den += rq[i] * z[i];
+        }
+        den += eps;
+        for (int64_t j = 0; j < dv; ++j) {
+          double num = 0.0;
+          for (int64_t i = 0; i < dk; ++i) num += rq[i] * S[i * dv + j];
+          o[(bh * N + t) * dv + j] = num / den;
+        }
+      }
+    }
+    if (kv_out) memcpy(kv_out + bh * dk * dv, S, sizeof(double) * (size_t)(dk * dv));
+    if (z_out) memcpy(z_out + bh * dk, z, sizeof(double) * (size_t)dk);
+  }
+  free(S);
+  free(z);
+  free(rq);
+  return 0;
+}

@@ -1,0 +1,385 @@
+"""Pins of the CPU oracle to things other than itself (no GPU needed).
+
+Each test checks the oracle against a closed form, a hand-derived worked case,
+an invariant of the recurrence, or an independent brute-force construction
+(explicit dense matrix products, O(N^2) masked attention), chosen so that a
+dropped term, a wrong sign or index, or a transposed operand in the oracle
+fails at least one of them.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+RNG = np.random.default_rng(12345)
+
+
+def _rand_case(nh, F, L, dk, dv, rng, unit=True):
+    q = rng.standard_normal((nh, F * L, dk)).astype(np.float32)
+    k = rng.standard_normal((nh, F * L, dk)).astype(np.float32)
+    if unit:
+        k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    v = rng.standard_normal((nh, F * L, dv)).astype(np.float32)
+    a = rng.standard_normal((nh, F)).astype(np.float32)
+    b = rng.standard_normal((nh, F * L)).astype(np.float32)
+    return q, k, v, a, b
+
+
+# ---------------------------------------------------------------- gates
+
+def test_gate_closed_forms():
+    # exp(-softplus(a)) == 1/(1+e^a) == sigmoid(-a); sigmoid(b) == 1/(1+e^-b)
+    for a in [-30.0, -5.0, -2.0, -0.5, 0.0, 0.3, 1.0, 4.0, 20.0]:
+        assert oracle.gate_alpha(a) == pytest.approx(1.0 / (1.0 + np.exp(a)), rel=1e-14, abs=1e-300)
+        assert oracle.gate_beta(a) == pytest.approx(1.0 / (1.0 + np.exp(-a)), rel=1e-14)
+    assert oracle.gate_alpha(0.0) == 0.5 and oracle.gate_beta(0.0) == 0.5
+    # alpha in (0,1], beta in (0,1): limits
+    assert oracle.gate_alpha(-800.0) == 1.0
+    assert oracle.gate_alpha(800.0) == 0.0
+
+
+# ---------------------------------------------------------------- worked cases
+
+def test_gdn_worked_2d_golden():
+    g = json.load(open(os.path.join(GOLDEN, "gdn_worked_2d.json")))
+    q, k, v = (np.array(g[x], np.float32)[None] for x in ("q", "k", "v"))
+    al = np.array(g["alpha"], np.float32)[None]
+    be = np.array(g["beta"], np.float32)[None]
+    o, s = oracle.gdn(q, k, v, al, be, F=g["F"], L=g["L"], gates_are_logits=False)
+    np.testing.assert_allclose(o[0], np.array(g["o"]), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(s[0], np.array(g["state_out"]), rtol=0, atol=1e-12)
+
+
+def test_relu_la_worked_2d_golden():
+    g = json.load(open(os.path.join(GOLDEN, "relu_la_worked_2d.json")))
+    q, k, v = (np.array(g[x], np.float32)[None] for x in ("q", "k", "v"))
+    o, kv, z = oracle.relu_la(q, k, v, F=g["F"], L=g["L"], eps=g["eps"])
+    np.testing.assert_allclose(o[0], np.array(g["o"]), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(kv[0], np.array(g["kv_out"]), rtol=0, atol=0)
+    np.testing.assert_allclose(z[0], np.array(g["z_out"]), rtol=0, atol=0)
+
+
+# ---------------------------------------------------------------- brute force
+
+def _bruteforce_gdn(q, k, v, alpha, beta, F, L, S0):
+    """Independent construction: S_F as explicit products of dense factors.
+
+    With M_t = I - beta_t khat_t khat_t^T and scalar decays alpha_f at frame
+    starts, S after step n is  P(0..n) S0 + sum_t P(t+1..n) beta_t khat_t v_t^T,
+    where P(i..n) is the ordered product (latest factor on the left) of every
+    factor after position i.  Each frame's outputs use the state at its end.
+    """
+    dk, dv = k.shape[-1], v.shape[-1]
+    ops = []  # sequence of ("decay", alpha) / ("tok", t)
+    for f in range(F):
+        ops.append(("decay", float(alpha[f])))
+        for t in range(f * L, (f + 1) * L):
+            ops.append(("tok", t))
+
+    def factor(op):
+        kind, x = op
+        if kind == "decay":
+            return x * np.eye(dk)
+        kk = k[x].astype(np.float64)
+        nrm = max(np.sqrt(kk @ kk), 1e-6)
+        kh = kk / nrm
+        return np.eye(dk) - float(beta[x]) * np.outer(kh, kh)
+
+    def state_after(n):  # state after ops[0..n] inclusive
+        P = np.eye(dk)
+        for op in ops[: n + 1]:
+            P = factor(op) @ P
+        S = P @ S0
+        for i in range(n + 1):
+            kind, t = ops[i]
+            if kind != "tok":
+                continue
+            Q = np.eye(dk)
+            for op in ops[i + 1: n + 1]:
+                Q = factor(op) @ Q
+            kk = k[t].astype(np.float64)
+            kh = kk / max(np.sqrt(kk @ kk), 1e-6)
+            S = S + Q @ (float(beta[t]) * np.outer(kh, v[t].astype(np.float64)))
+        return S
+
+    o = np.zeros((F * L, dv))
+    idx = -1
+    for f in range(F):
+        idx += 1 + L
+        Sf = state_after(idx)
+        for t in range(f * L, (f + 1) * L):
+            o[t] = Sf.T @ q[t].astype(np.float64)
+    return o, state_after(len(ops) - 1)
+
+
+@pytest.mark.parametrize("F,L,dk,dv,unit", [(1, 1, 3, 2, True), (2, 3, 4, 3, True), (3, 4, 4, 4, False),
+                                             (3, 2, 2, 4, True)])
+def test_gdn_bruteforce_products(F, L, dk, dv, unit):
+    rng = np.random.default_rng(F * 100 + L * 10 + dk)
+    q, k, v, a, b = _rand_case(1, F, L, dk, dv, rng, unit=unit)
+    S0 = rng.standard_normal((dk, dv))
+    al = np.array([oracle.gate_alpha(x) for x in a[0]], np.float32)
+    be = np.array([oracle.gate_beta(x) for x in b[0]], np.float32)
+    o, s = oracle.gdn(q, k, v, al[None], be[None], F=F, L=L, gates_are_logits=False, state_in=S0[None])
+    o_ref, s_ref = _bruteforce_gdn(q[0], k[0], v[0], al, be, F, L, S0)
+    np.testing.assert_allclose(o[0], o_ref, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(s[0], s_ref, rtol=0, atol=1e-12)
+    # the same run through the logit path must agree with the value path
+    o2, s2 = oracle.gdn(q, k, v, a, b, F=F, L=L, gates_are_logits=True, state_in=S0[None])
+    np.testing.assert_allclose(o2[0], o_ref, rtol=0, atol=1e-6)
+
+
+# ---------------------------------------------------------------- closed forms
+
+def test_gdn_identity_gates_leave_state():
+    # alpha = 1, beta = 0: S never changes and o_t = S0^T q_t
+    rng = np.random.default_rng(1)
+    F, L, dk, dv = 3, 5, 6, 4
+    q, k, v, _, _ = _rand_case(2, F, L, dk, dv, rng)
+    S0 = rng.standard_normal((2, dk, dv))
+    o, s = oracle.gdn(q, k, v, np.ones((2, F), np.float32), np.zeros((2, F * L), np.float32),
+                      F=F, L=L, gates_are_logits=False, state_in=S0)
+    np.testing.assert_allclose(s, S0, rtol=0, atol=0)
+    np.testing.assert_allclose(o, np.einsum("hnd,hde->hne", q.astype(np.float64), S0), rtol=0, atol=1e-12)
+
+
+def test_gdn_single_token_orthonormal():
+    # S0 = 0, one token with unit key: S = beta khat v^T; o = S^T q
+    dk, dv = 5, 3
+    for i in range(dk):
+        k = np.zeros((1, 1, dk), np.float32)
+        k[0, 0, i] = 1.0
+        v = np.array([[[1.5, -2.0, 0.25]]], np.float32)
+        q = np.arange(dk, dtype=np.float32).reshape(1, 1, dk)
+        beta = 0.375
+        o, s = oracle.gdn(q, k, v, np.ones((1, 1), np.float32), np.full((1, 1), beta, np.float32),
+                          F=1, L=1, gates_are_logits=False)
+        expect = beta * np.outer(k[0, 0], v[0, 0])
+        np.testing.assert_allclose(s[0], expect, rtol=0, atol=1e-15)
+        np.testing.assert_allclose(o[0, 0], expect.T @ q[0, 0], rtol=0, atol=1e-15)
+
+
+def test_gdn_exact_recall_orthonormal_keys():
+    # beta = 1 and L <= dk orthonormal keys: S^T khat_i = v_i for every key written
+    rng = np.random.default_rng(7)
+    dk, dv, L = 8, 5, 6
+    Qm, _ = np.linalg.qr(rng.standard_normal((dk, dk)))
+    k = Qm[:, :L].T.astype(np.float32)[None]  # rows orthonormal (up to fp32 rounding)
+    v = rng.standard_normal((1, L, dv)).astype(np.float32)
+    q = rng.standard_normal((1, L, dk)).astype(np.float32)
+    S0 = rng.standard_normal((1, dk, dv))
+    o, s = oracle.gdn(q, k, v, np.ones((1, 1), np.float32), np.ones((1, L), np.float32),
+                      F=1, L=L, gates_are_logits=False, state_in=S0)
+    kh = k[0].astype(np.float64)
+    kh /= np.linalg.norm(kh, axis=1, keepdims=True)
+    np.testing.assert_allclose(kh @ s[0], v[0], rtol=0, atol=1e-6)  # limited by fp32 orthogonality of k
+    # directions orthogonal to every key keep their original read-out
+    P = np.eye(dk) - kh.T @ kh
+    np.testing.assert_allclose(P @ s[0], P @ S0[0], rtol=0, atol=1e-6)
+
+
+def test_gdn_zero_key_is_a_no_op():
+    rng = np.random.default_rng(3)
+    F, L, dk, dv = 2, 4, 4, 3
+    q, k, v, a, b = _rand_case(1, F, L, dk, dv, rng)
+    o, s = oracle.gdn(q, k, v, a, b, F=F, L=L)
+    k2 = k.copy()
+    k2[0, 2] = 0.0
+    k2[0, 5] = 0.0
+    o2, s2 = oracle.gdn(q, k2, v, a, b, F=F, L=L)
+    # compare against a run with those tokens removed (beta forced to 0)
+    b3 = b.copy()
+    b3[0, 2] = -1e4
+    b3[0, 5] = -1e4
+    o3, s3 = oracle.gdn(q, k, v, a, b3, F=F, L=L)
+    np.testing.assert_allclose(s2, s3, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(o2, o3, rtol=0, atol=1e-12)
+    assert not np.allclose(s, s2)
+
+
+# ---------------------------------------------------------------- invariants
+
+def test_gdn_key_scale_invariance():
+    # khat is invariant to positive rescaling of k_t
+    rng = np.random.default_rng(4)
+    F, L, dk, dv = 2, 3, 5, 4
+    q, k, v, a, b = _rand_case(1, F, L, dk, dv, rng, unit=False)
+    o, s = oracle.gdn(q, k, v, a, b, F=F, L=L)
+    scale = np.array([0.5, 2.0, 8.0, 0.25, 4.0, 1.0], np.float32)[None, :, None]
+    o2, s2 = oracle.gdn(q, k * scale, v, a, b, F=F, L=L)
+    np.testing.assert_allclose(o2, o, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(s2, s, rtol=0, atol=1e-12)
+
+
+def test_gdn_affine_in_state_and_linear_in_values():
+    rng = np.random.default_rng(5)
+    F, L, dk, dv = 3, 4, 5, 4
+    q, k, v, a, b = _rand_case(1, F, L, dk, dv, rng)
+    S1 = rng.standard_normal((1, dk, dv))
+    S2 = rng.standard_normal((1, dk, dv))
+    run = lambda vv, S: oracle.gdn(q, k, vv, a, b, F=F, L=L, state_in=S)
+    o0, s0 = run(v, None)
+    oa, sa = run(v, S1)
+    ob, sb = run(v, S2)
+    oab, sab = run(v, S1 + S2)
+    np.testing.assert_allclose(sab - s0, (sa - s0) + (sb - s0), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(oab - o0, (oa - o0) + (ob - o0), rtol=0, atol=1e-12)
+    # linear in v when S0 = 0 (v values kept exactly representable in fp32)
+    v1 = np.round(rng.standard_normal(v.shape) * 64).astype(np.float32) / 64
+    v2 = np.round(rng.standard_normal(v.shape) * 64).astype(np.float32) / 64
+    o1, t1 = run(v1, None)
+    o2, t2 = run(v2, None)
+    o12, t12 = run(v1 + v2, None)
+    np.testing.assert_allclose(t12, t1 + t2, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(o12, o1 + o2, rtol=0, atol=1e-12)
+
+
+def test_gdn_column_permutation_equivariance_and_column_subsets():
+    rng = np.random.default_rng(6)
+    F, L, dk, dv = 2, 5, 6, 7
+    q, k, v, a, b = _rand_case(2, F, L, dk, dv, rng)
+    S0 = rng.standard_normal((2, dk, dv))
+    o, s = oracle.gdn(q, k, v, a, b, F=F, L=L, state_in=S0)
+    perm = rng.permutation(dv)
+    o2, s2 = oracle.gdn(q, k, v[..., perm], a, b, F=F, L=L, state_in=S0[..., perm])
+    np.testing.assert_array_equal(o2, o[..., perm])
+    np.testing.assert_array_equal(s2, s[..., perm])
+    # computing a subset of columns gives bit-identical values for those columns
+    o3, s3 = oracle.gdn(q, k, v, a, b, F=F, L=L, state_in=S0, cols=(2, 5))
+    np.testing.assert_array_equal(o3[..., 2:5], o[..., 2:5])
+    np.testing.assert_array_equal(s3[..., 2:5], s[..., 2:5])
+    assert np.isnan(o3[..., :2]).all()
+
+
+def test_gdn_contraction():
+    # each factor has spectral norm <= 1 (unit keys, beta in (0,1), alpha <= 1)
+    rng = np.random.default_rng(8)
+    F, L, dk, dv = 3, 6, 6, 5
+    q, k, v, a, b = _rand_case(1, F, L, dk, dv, rng)
+    for _ in range(5):
+        S1 = rng.standard_normal((1, dk, dv)) * 3
+        S2 = rng.standard_normal((1, dk, dv)) * 3
+        _, s1 = oracle.gdn(q, k, v, a, b, F=F, L=L, state_in=S1)
+        _, s2 = oracle.gdn(q, k, v, a, b, F=F, L=L, state_in=S2)
+        assert np.linalg.norm(s1[0] - s2[0], 2) <= np.linalg.norm(S1[0] - S2[0], 2) * (1 + 1e-12)
+
+
+def test_gdn_readout_uses_end_of_frame_state_and_split_resume():
+    rng = np.random.default_rng(9)
+    F, L, dk, dv = 4, 3, 5, 4
+    q, k, v, a, b = _rand_case(1, F, L, dk, dv, rng)
+    o, s = oracle.gdn(q, k, v, a, b, F=F, L=L)
+    for f in range(F):
+        n = (f + 1) * L
+        _, sf = oracle.gdn(q[:, :n], k[:, :n], v[:, :n], a[:, :f + 1], b[:, :n], F=f + 1, L=L)
+        np.testing.assert_allclose(o[0, f * L:n], q[0, f * L:n].astype(np.float64) @ sf[0], rtol=0, atol=1e-12)
+    # resume from the state after 2 frames == one run over all frames
+    _, s2 = oracle.gdn(q[:, :2 * L], k[:, :2 * L], v[:, :2 * L], a[:, :2], b[:, :2 * L], F=2, L=L)
+    o_r, s_r = oracle.gdn(q[:, 2 * L:], k[:, 2 * L:], v[:, 2 * L:], a[:, 2:], b[:, 2 * L:], F=2, L=L,
+                          state_in=s2)
+    np.testing.assert_allclose(o_r, o[:, 2 * L:], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(s_r, s, rtol=0, atol=1e-12)
+
+
+def test_gdn_frames_are_block_causal():
+    # changing a later frame's inputs never changes an earlier frame's outputs
+    rng = np.random.default_rng(10)
+    F, L, dk, dv = 3, 4, 4, 4
+    q, k, v, a, b = _rand_case(1, F, L, dk, dv, rng)
+    o, _ = oracle.gdn(q, k, v, a, b, F=F, L=L)
+    v2 = v.copy()
+    v2[0, 2 * L:] += 1.0
+    o2, _ = oracle.gdn(q, k, v2, a, b, F=F, L=L)
+    np.testing.assert_array_equal(o2[0, :2 * L], o[0, :2 * L])
+    assert not np.allclose(o2[0, 2 * L:], o[0, 2 * L:])
+    # but a change inside the frame reaches every token of that frame (bidirectional within a frame)
+    v3 = v.copy()
+    v3[0, 2 * L + L - 1] += 1.0
+    o3, _ = oracle.gdn(q, k, v3, a, b, F=F, L=L)
+    assert (np.abs(o3[0, 2 * L:] - o[0, 2 * L:]).max(axis=1) > 0).all()
+
+
+# ---------------------------------------------------------------- ReLU mode
+
+def _quadratic_masked_attention(q, k, v, F, L, eps):
+    """O(N^2) block-causal masked attention with ReLU features (independent route)."""
+    N = F * L
+    rq = np.maximum(q.astype(np.float64), 0)
+    rk = np.maximum(k.astype(np.float64), 0)
+    frame = np.arange(N) // L
+    mask = frame[None, :] <= frame[:, None]  # key frame <= query frame
+    A = (rq @ rk.T) * mask
+    return (A @ v.astype(np.float64)) / (A.sum(axis=1, keepdims=True) + eps)
+
+
+@pytest.mark.parametrize("F,L,dk,dv", [(1, 7, 4, 3), (4, 5, 6, 5), (8, 8, 8, 8)])
+def test_relu_la_equals_quadratic_masked_attention(F, L, dk, dv):
+    rng = np.random.default_rng(F * L)
+    q = rng.standard_normal((1, F * L, dk)).astype(np.float32)
+    k = rng.standard_normal((1, F * L, dk)).astype(np.float32)
+    v = rng.standard_normal((1, F * L, dv)).astype(np.float32)
+    o, kv, z = oracle.relu_la(q, k, v, F=F, L=L, eps=1e-6)
+    ref = _quadratic_masked_attention(q[0], k[0], v[0], F, L, 1e-6)
+    np.testing.assert_allclose(o[0], ref, rtol=1e-12, atol=1e-12)
+    rk = np.maximum(k[0].astype(np.float64), 0)
+    np.testing.assert_allclose(kv[0], rk.T @ v[0].astype(np.float64), rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(z[0], rk.sum(axis=0), rtol=1e-12, atol=1e-12)
+
+
+def test_relu_la_state_carry_and_zero_query():
+    rng = np.random.default_rng(11)
+    F, L, dk, dv = 4, 3, 5, 4
+    q = rng.standard_normal((2, F * L, dk)).astype(np.float32)
+    k = rng.standard_normal((2, F * L, dk)).astype(np.float32)
+    v = rng.standard_normal((2, F * L, dv)).astype(np.float32)
+    q[0, 1] = -np.abs(q[0, 1])  # relu(q) == 0 -> o == 0
+    o, kv, z = oracle.relu_la(q, k, v, F=F, L=L)
+    assert np.all(o[0, 1] == 0.0)
+    o1, kv1, z1 = oracle.relu_la(q[:, :2 * L], k[:, :2 * L], v[:, :2 * L], F=2, L=L)
+    o2, kv2, z2 = oracle.relu_la(q[:, 2 * L:], k[:, 2 * L:], v[:, 2 * L:], F=2, L=L, kv_in=kv1, z_in=z1)
+    np.testing.assert_allclose(o2, o[:, 2 * L:], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(kv2, kv, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(z2, z, rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------- planted mistakes
+
+def test_pins_catch_planted_mistakes():
+    """The brute-force pin distinguishes the correct rule from plausible wrong ones."""
+    rng = np.random.default_rng(13)
+    F, L, dk, dv = 2, 3, 4, 4
+    q, k, v, a, b = _rand_case(1, F, L, dk, dv, rng)
+    al = np.array([oracle.gate_alpha(x) for x in a[0]], np.float32)
+    be = np.array([oracle.gate_beta(x) for x in b[0]], np.float32)
+    S0 = rng.standard_normal((dk, dv))
+    o_ref, s_ref = _bruteforce_gdn(q[0], k[0], v[0], al, be, F, L, S0)
+
+    def variant(sign=1.0, transpose_read=False, per_token_read=False, decay_after=False):
+        S = S0.copy()
+        o = np.zeros((F * L, dv))
+        for f in range(F):
+            if not decay_after:
+                S = al[f] * S
+            for t in range(f * L, (f + 1) * L):
+                kh = k[0, t].astype(np.float64)
+                kh /= np.linalg.norm(kh)
+                r = (S @ kh if transpose_read else S.T @ kh) - v[0, t]
+                S = S - sign * be[t] * np.outer(kh, r)
+                if per_token_read:
+                    o[t] = S.T @ q[0, t]
+            if decay_after:
+                S = al[f] * S
+            if not per_token_read:
+                for t in range(f * L, (f + 1) * L):
+                    o[t] = S.T @ q[0, t]
+        return o, S
+
+    o_ok, s_ok = variant()
+    np.testing.assert_allclose(o_ok, o_ref, atol=1e-6)
+    for kw in [dict(sign=-1.0), dict(transpose_read=True), dict(per_token_read=True), dict(decay_after=True)]:
+        o_bad, s_bad = variant(**kw)
+        assert np.abs(o_bad - o_ref).max() > 1e-3, kw
