@@ -1,0 +1,176 @@
+/*
+ * gdn_b200.h -- C ABI of the B200 (sm_100a) frame-recurrence library.
+ *
+ * Two recurrences that replace softmax attention in linear video diffusion
+ * transformers, both block-causal over latent frames:
+ *
+ *  1. Frame-wise Gated DeltaNet ("SANA-WM, an open-source 2.6B world model for
+ *     1-minute 720p video", GeekNews vi.news.hada.io/topic?id=29572, section
+ *     "Core design and generation pipeline": a hybrid linear diffusion
+ *     transformer with frame-wise Gated DeltaNet; dothoosh.com, "How NVIDIA
+ *     SANA-WM generates 60-second 720p video on one GPU": most attention
+ *     blocks are Gated DeltaNet with a fixed-size recurrent state).
+ *  2. Block-causal ReLU linear attention with a constant-memory block KV cache
+ *     ("SANA-Video: Efficient Video Generation with Block Linear Diffusion
+ *     Transformer", ICLR 2026 oral talk transcript, block KV cache passage:
+ *     the state is a fixed D x D matrix; block i adds its KV contribution to
+ *     the cached state of block i-1, and each block reads that state).
+ *
+ * The pages give no equations; the update rules stated per entry point are
+ * this library's definition (the plainest reading consistent with them).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - All tensor pointers are DEVICE pointers owned by the caller, except in
+ *    gdn_frame_fwd_host(), whose tensor pointers are HOST pointers.
+ *  - Layouts are row-major and contiguous.  N = F * L tokens per head.
+ *      q, k : [B, H, N, dk]   (element type opts->in_dtype)
+ *      v    : [B, H, N, dv]   (element type opts->in_dtype)
+ *      o    : [B, H, N, dv]   float32
+ *      state: [B, H, dk, dv]  float32, S[i][j] with i over d_k, j over d_v
+ *  - Every pointer must be 16-byte aligned.
+ *  - Calls are asynchronous on opts->stream (stream-ordered) and return after
+ *    launch; errors found on the host are returned at once, errors found on
+ *    the device (a bounded wait that ran out) are written to *opts->status.
+ *  - The library allocates no memory.  Kernels that need scratch take it
+ *    from opts->workspace (size from gdn_workspace_bytes()).  Two calls that
+ *    share a workspace must be ordered on the GPU (same stream).
+ *  - Thread-safe: no global mutable state besides a per-device cache of the
+ *    SM count and of the driver's tensor-map encoder entry point.
+ */
+#ifndef GDN_B200_H_
+#define GDN_B200_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define GDN_API __attribute__((visibility("default")))
+#else
+#define GDN_API
+#endif
+
+#define GDN_ABI_VERSION 1
+
+/* return / status codes */
+#define GDN_OK 0
+#define GDN_ERR_INVALID_ARG 1   /* null pointer, bad size, misaligned pointer, bad workspace */
+#define GDN_ERR_UNSUPPORTED 2   /* valid arguments this build does not handle (e.g. dk > 128) */
+#define GDN_ERR_CUDA 3          /* a CUDA runtime/driver call failed */
+#define GDN_ERR_TIMEOUT 4       /* device: a bounded in-kernel wait expired (outputs invalid) */
+#define GDN_ERR_NO_DEVICE 5     /* no usable sm_100 device for this call */
+
+/* element types of q, k, v */
+#define GDN_DTYPE_F32 0
+#define GDN_DTYPE_BF16 1
+
+/* kernel selection (GDN_IMPL_AUTO picks the fastest valid one) */
+#define GDN_IMPL_AUTO 0
+#define GDN_IMPL_SEQ 1          /* per-token SIMT recurrence, one CTA per head (reference-simple) */
+#define GDN_IMPL_FRAME_SIMT 2   /* frame maps + ticketed frame chain, CUDA cores, fp32 arithmetic */
+#define GDN_IMPL_TC 3           /* frame maps + chain on tcgen05/TMEM tensor cores (bf16 inputs) */
+
+/* operation ids for gdn_workspace_bytes() */
+#define GDN_OP_GDN 0
+#define GDN_OP_RELU_LA 1
+
+typedef struct gdn_opts {
+  int in_dtype;           /* GDN_DTYPE_F32 or GDN_DTYPE_BF16: element type of q, k, v */
+  int gates_are_logits;   /* gdn only. 1: alpha[] holds logits a, alpha_f = exp(-softplus(a));
+                             beta[] holds logits b, beta_t = sigmoid(b).  0: the gate values */
+  int impl;               /* GDN_IMPL_* */
+  void *stream;           /* cudaStream_t; NULL = legacy default stream */
+  void *workspace;        /* device scratch of >= gdn_workspace_bytes() bytes, 256-byte aligned */
+  size_t workspace_bytes;
+  int *status;            /* optional device int; kernels write a GDN_ERR_* code on a device-side
+                             failure and never clear it (caller zeroes it) */
+  int max_ctas;           /* 0 = one persistent CTA per SM; else an upper bound (testing) */
+  int spin_limit_us;      /* bound on any in-kernel wait; 0 = 2,000,000 us */
+  int test_withhold_unit; /* testing only.  0: off.  u + 1: frame unit u (u = f*B*H + b*H + h) never
+                             publishes its state, so the wait of unit u + B*H expires and the
+                             kernel reports GDN_ERR_TIMEOUT through *status */
+} gdn_opts_t;
+
+/*
+ * gdn_frame_fwd -- frame-wise Gated DeltaNet forward.
+ *
+ * Per head (b, h), with S starting at state_in (zero if state_in == NULL):
+ *   for each frame f = 0..F-1:
+ *     S <- alpha_f * S                       (decay once, at the frame start)
+ *     for each token t of frame f, in increasing t:
+ *       khat = k_t / max(||k_t||_2, 1e-6)
+ *       S    <- S - beta_t * khat (S^T khat - v_t)^T        (delta rule)
+ *     for each token t of frame f:  o_t = S^T q_t            (end-of-frame state)
+ *   state_out <- S                           (skipped if state_out == NULL)
+ *
+ * alpha: [B, H, F] float32; beta: [B, H, N] float32 (logits or values, see
+ * opts->gates_are_logits).  state_in may equal state_out (in-place carry).
+ * q, k, v, o must not overlap each other or the states.
+ *
+ * Sizes: B, H, F, L >= 1; 1 <= dk, dv <= 128; dk and dv multiples of 16 for
+ * GDN_IMPL_TC (others: any size up to 128).  Streaming decode is this call with
+ * F = 1, state_in = the cached state and state_out = NULL until the step that
+ * commits the frame.
+ *
+ * Precision: fp32 inputs use fp32 arithmetic throughout (GDN_IMPL_SEQ /
+ * FRAME_SIMT).  bf16 inputs on GDN_IMPL_TC multiply on tensor cores with
+ * fp16 operands (11-bit significands) and fp32 accumulation; state and
+ * outputs are fp32.  Its fp16 operands need |q|, |v| and |S| below 6.5e4.
+ *
+ * Returns GDN_OK or GDN_ERR_*.
+ */
+GDN_API int gdn_frame_fwd(const void *q, const void *k, const void *v, const float *alpha, const float *beta,
+                  const float *state_in, float *state_out, float *o, int B, int H, int F, int L,
+                  int dk, int dv, const gdn_opts_t *opts);
+
+/*
+ * relu_la_block_fwd -- block-causal ReLU linear attention forward.
+ *
+ * Per head (b, h), with S = kv_in (zero if NULL) [dk x dv] and z = z_in (zero
+ * if NULL) [dk]:
+ *   for each frame f:
+ *     S <- S + sum_{t in f} relu(k_t) v_t^T;   z <- z + sum_{t in f} relu(k_t)
+ *     for each token t of f:  o_t = relu(q_t)^T S / (relu(q_t)^T z + eps)
+ *   kv_out <- S, z_out <- z                  (each skipped if NULL)
+ *
+ * kv_in/kv_out: [B, H, dk, dv] float32; z_in/z_out: [B, H, dk] float32.
+ * In-place carry (kv_in == kv_out, z_in == z_out) is allowed.
+ */
+GDN_API int relu_la_block_fwd(const void *q, const void *k, const void *v, const float *kv_in, const float *z_in,
+                      float *kv_out, float *z_out, float *o, int B, int H, int F, int L, int dk, int dv,
+                      float eps, const gdn_opts_t *opts);
+
+/*
+ * gdn_frame_fwd_host -- gdn_frame_fwd with HOST tensors.
+ *
+ * Same semantics and layouts as gdn_frame_fwd, but q, k, v, alpha, beta,
+ * state_in (inputs) and o, state_out (outputs) are host pointers (pinned
+ * memory gives full PCIe bandwidth).  The call copies the inputs into the
+ * caller's device workspace, runs the recurrence there, copies the outputs
+ * back and synchronises opts->stream before returning.
+ * opts->workspace must hold gdn_workspace_bytes_host() bytes.
+ */
+GDN_API int gdn_frame_fwd_host(const void *q, const void *k, const void *v, const float *alpha, const float *beta,
+                       const float *state_in, float *state_out, float *o, int B, int H, int F, int L,
+                       int dk, int dv, const gdn_opts_t *opts);
+
+/* Device scratch bytes that op (GDN_OP_*) needs for these sizes and options. */
+GDN_API size_t gdn_workspace_bytes(int op, int B, int H, int F, int L, int dk, int dv, const gdn_opts_t *opts);
+
+/* Device scratch bytes that gdn_frame_fwd_host() needs (staging + workspace). */
+GDN_API size_t gdn_workspace_bytes_host(int B, int H, int F, int L, int dk, int dv, const gdn_opts_t *opts);
+
+/* Static description of a status code (never NULL). */
+GDN_API const char *gdn_status_string(int status);
+
+/* GDN_ABI_VERSION of the loaded library. */
+GDN_API int gdn_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_B200_H_ */

@@ -1,0 +1,235 @@
+"""B200 (sm_100a) frame-wise linear-attention recurrences: Python binding.
+
+A thin ctypes layer over ``libgdn_b200.so`` (the C ABI declared in
+``include/gdn_b200.h``).  It only marshals arguments: every step of the
+recurrences runs in the library's CUDA kernels.  PyTorch supplies device
+memory and streams.  There is no CPU fallback: importing this package fails
+loudly when the library has not been built.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libgdn_b200.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m linear_attention_video_gdn_b200.build` "
+        "(there is no CPU fallback)")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_NO_DEVICE = range(6)
+DTYPE_F32, DTYPE_BF16 = 0, 1
+IMPL_AUTO, IMPL_SEQ, IMPL_FRAME_SIMT, IMPL_TC = 0, 1, 2, 3
+OP_GDN, OP_RELU_LA = 0, 1
+IMPLS = {"auto": IMPL_AUTO, "seq": IMPL_SEQ, "frame_simt": IMPL_FRAME_SIMT, "tc": IMPL_TC}
+
+EXPORTED = ("gdn_frame_fwd", "relu_la_block_fwd", "gdn_frame_fwd_host", "gdn_workspace_bytes",
+            "gdn_workspace_bytes_host", "gdn_status_string", "gdn_abi_version")
+
+
+class GdnOpts(ctypes.Structure):
+    _fields_ = [("in_dtype", ctypes.c_int), ("gates_are_logits", ctypes.c_int), ("impl", ctypes.c_int),
+                ("stream", ctypes.c_void_p), ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+                ("status", ctypes.c_void_p), ("max_ctas", ctypes.c_int), ("spin_limit_us", ctypes.c_int),
+                ("test_withhold_unit", ctypes.c_int)]
+
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_lib.gdn_frame_fwd.argtypes = [_P] * 8 + [_I] * 6 + [ctypes.POINTER(GdnOpts)]
+_lib.gdn_frame_fwd.restype = _I
+_lib.gdn_frame_fwd_host.argtypes = [_P] * 8 + [_I] * 6 + [ctypes.POINTER(GdnOpts)]
+_lib.gdn_frame_fwd_host.restype = _I
+_lib.relu_la_block_fwd.argtypes = [_P] * 8 + [_I] * 6 + [ctypes.c_float, ctypes.POINTER(GdnOpts)]
+_lib.relu_la_block_fwd.restype = _I
+_lib.gdn_workspace_bytes.argtypes = [_I] * 7 + [ctypes.POINTER(GdnOpts)]
+_lib.gdn_workspace_bytes.restype = ctypes.c_size_t
+_lib.gdn_workspace_bytes_host.argtypes = [_I] * 6 + [ctypes.POINTER(GdnOpts)]
+_lib.gdn_workspace_bytes_host.restype = ctypes.c_size_t
+_lib.gdn_status_string.argtypes = [_I]
+_lib.gdn_status_string.restype = ctypes.c_char_p
+_lib.gdn_abi_version.argtypes = []
+_lib.gdn_abi_version.restype = _I
+
+
+class GdnError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {status_string(code)} (code {code})")
+
+
+def status_string(code: int) -> str:
+    return _lib.gdn_status_string(int(code)).decode()
+
+
+def abi_version() -> int:
+    return int(_lib.gdn_abi_version())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return DTYPE_F32
+    if t.dtype == torch.bfloat16:
+        return DTYPE_BF16
+    raise TypeError(f"q/k/v must be float32 or bfloat16, got {t.dtype}")
+
+
+def _stream_handle(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def make_opts(in_dtype: int, *, gates_are_logits: bool = True, impl="auto", stream=None, workspace=None,
+              status=None, max_ctas: int = 0, spin_limit_us: int = 0, test_withhold_unit: int = -1) -> GdnOpts:
+    o = GdnOpts()
+    o.in_dtype = in_dtype
+    o.gates_are_logits = int(bool(gates_are_logits))
+    o.impl = IMPLS[impl] if isinstance(impl, str) else int(impl)
+    o.stream = _stream_handle(stream)
+    if workspace is not None:
+        o.workspace = workspace.data_ptr()
+        o.workspace_bytes = workspace.numel() * workspace.element_size()
+    o.status = None if status is None else status.data_ptr()
+    o.max_ctas = int(max_ctas)
+    o.spin_limit_us = int(spin_limit_us)
+    o.test_withhold_unit = int(test_withhold_unit) + 1 if test_withhold_unit >= 0 else 0
+    return o
+
+
+def workspace_bytes(op: int, B, H, F, L, dk, dv, opts: GdnOpts) -> int:
+    return int(_lib.gdn_workspace_bytes(op, B, H, F, L, dk, dv, ctypes.byref(opts)))
+
+
+def alloc_workspace(nbytes: int, device) -> torch.Tensor:
+    """Caller-owned device scratch (256-byte aligned by the caching allocator)."""
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def _check(t, name, shape, dtype, device, allow_none=False):
+    if t is None:
+        if allow_none:
+            return
+        raise ValueError(f"{name} is required")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name}: expected device {device}, got {t.device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def gdn_frame_fwd(q, k, v, alpha, beta, *, F: int, state_in=None, state_out=None, o=None,
+                  gates_are_logits: bool = True, impl="auto", workspace=None, stream=None, status=None,
+                  max_ctas: int = 0, spin_limit_us: int = 0, test_withhold_unit: int = -1):
+    """Frame-wise Gated DeltaNet forward on the GPU (see include/gdn_b200.h).
+
+    q, k: [B, H, F*L, dk]; v: [B, H, F*L, dv] (float32 or bfloat16, same dtype);
+    alpha: [B, H, F] float32; beta: [B, H, F*L] float32; state_in/state_out:
+    [B, H, dk, dv] float32 or None.  Returns o [B, H, F*L, dv] float32.
+    """
+    B, H, N, dk = q.shape
+    dv = v.shape[-1]
+    if N % F:
+        raise ValueError(f"token count {N} is not a multiple of F={F}")
+    L = N // F
+    dev = q.device
+    _check(k, "k", (B, H, N, dk), q.dtype, dev)
+    _check(v, "v", (B, H, N, dv), q.dtype, dev)
+    _check(q, "q", (B, H, N, dk), q.dtype, dev)
+    _check(alpha, "alpha", (B, H, F), torch.float32, dev)
+    _check(beta, "beta", (B, H, N), torch.float32, dev)
+    _check(state_in, "state_in", (B, H, dk, dv), torch.float32, dev, allow_none=True)
+    _check(state_out, "state_out", (B, H, dk, dv), torch.float32, dev, allow_none=True)
+    if o is None:
+        o = torch.empty((B, H, N, dv), dtype=torch.float32, device=dev)
+    _check(o, "o", (B, H, N, dv), torch.float32, dev)
+    opts = make_opts(_dtype_code(q), gates_are_logits=gates_are_logits, impl=impl, stream=stream,
+                     status=status, max_ctas=max_ctas, spin_limit_us=spin_limit_us,
+                     test_withhold_unit=test_withhold_unit)
+    need = workspace_bytes(OP_GDN, B, H, F, L, dk, dv, opts)
+    if workspace is None and need > 0:
+        workspace = alloc_workspace(need, dev)
+    if workspace is not None:
+        opts.workspace = workspace.data_ptr()
+        opts.workspace_bytes = workspace.numel() * workspace.element_size()
+    rc = _lib.gdn_frame_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(state_in), _ptr(state_out),
+                            _ptr(o), B, H, F, L, dk, dv, ctypes.byref(opts))
+    if rc != OK:
+        raise GdnError(rc, "gdn_frame_fwd")
+    return o
+
+
+def relu_la_block_fwd(q, k, v, *, F: int, kv_in=None, z_in=None, kv_out=None, z_out=None, o=None,
+                      eps: float = 1e-6, impl="auto", workspace=None, stream=None, status=None,
+                      max_ctas: int = 0, spin_limit_us: int = 0, test_withhold_unit: int = -1):
+    """Block-causal ReLU linear attention forward on the GPU (see include/gdn_b200.h)."""
+    B, H, N, dk = q.shape
+    dv = v.shape[-1]
+    if N % F:
+        raise ValueError(f"token count {N} is not a multiple of F={F}")
+    L = N // F
+    dev = q.device
+    _check(k, "k", (B, H, N, dk), q.dtype, dev)
+    _check(v, "v", (B, H, N, dv), q.dtype, dev)
+    _check(q, "q", (B, H, N, dk), q.dtype, dev)
+    for t, nm, shp in ((kv_in, "kv_in", (B, H, dk, dv)), (kv_out, "kv_out", (B, H, dk, dv)),
+                       (z_in, "z_in", (B, H, dk)), (z_out, "z_out", (B, H, dk))):
+        _check(t, nm, shp, torch.float32, dev, allow_none=True)
+    if o is None:
+        o = torch.empty((B, H, N, dv), dtype=torch.float32, device=dev)
+    _check(o, "o", (B, H, N, dv), torch.float32, dev)
+    opts = make_opts(_dtype_code(q), impl=impl, stream=stream, status=status, max_ctas=max_ctas,
+                     spin_limit_us=spin_limit_us, test_withhold_unit=test_withhold_unit)
+    need = workspace_bytes(OP_RELU_LA, B, H, F, L, dk, dv, opts)
+    if workspace is None:
+        workspace = alloc_workspace(need, dev)
+    opts.workspace = workspace.data_ptr()
+    opts.workspace_bytes = workspace.numel() * workspace.element_size()
+    rc = _lib.relu_la_block_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(kv_in), _ptr(z_in), _ptr(kv_out), _ptr(z_out),
+                                _ptr(o), B, H, F, L, dk, dv, float(eps), ctypes.byref(opts))
+    if rc != OK:
+        raise GdnError(rc, "relu_la_block_fwd")
+    return o
+
+
+def gdn_frame_fwd_host(q, k, v, alpha, beta, *, F: int, o, state_in=None, state_out=None,
+                       gates_are_logits: bool = True, impl="auto", workspace=None, stream=None, status=None):
+    """gdn_frame_fwd with HOST (CPU, ideally pinned) tensors; synchronous.
+
+    Copies inputs into ``workspace`` (a device uint8 tensor of at least
+    ``host_workspace_bytes(...)`` bytes), runs, and copies o/state_out back.
+    """
+    B, H, N, dk = q.shape
+    dv = v.shape[-1]
+    L = N // F
+    for t in (q, k, v, alpha, beta, o, state_in, state_out):
+        if t is not None and (t.device.type != "cpu" or not t.is_contiguous()):
+            raise ValueError("gdn_frame_fwd_host takes contiguous CPU tensors")
+    opts = make_opts(_dtype_code(q), gates_are_logits=gates_are_logits, impl=impl, stream=stream, status=status)
+    need = host_workspace_bytes(B, H, F, L, dk, dv, opts)
+    if workspace is None:
+        workspace = alloc_workspace(need, torch.device("cuda", torch.cuda.current_device()))
+    opts.workspace = workspace.data_ptr()
+    opts.workspace_bytes = workspace.numel() * workspace.element_size()
+    rc = _lib.gdn_frame_fwd_host(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(state_in),
+                                 _ptr(state_out), _ptr(o), B, H, F, L, dk, dv, ctypes.byref(opts))
+    if rc != OK:
+        raise GdnError(rc, "gdn_frame_fwd_host")
+    return o
+
+
+def host_workspace_bytes(B, H, F, L, dk, dv, opts: GdnOpts) -> int:
+    return int(_lib.gdn_workspace_bytes_host(B, H, F, L, dk, dv, ctypes.byref(opts)))

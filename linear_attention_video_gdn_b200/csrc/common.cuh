@@ -1,0 +1,120 @@
+// Shared device-side helpers: workspace layout, bounded waits, element loads.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/gdn_b200.h"
+
+namespace gdn {
+
+// Key normalisation floor: khat = k / max(||k||, kKeyNormEps).
+constexpr float kKeyNormEps = 1e-6f;
+
+// Workspace of the frame-chain kernels:
+//   [0, 256)                 : int counters (ticket counter at [0])
+//   [256, 256 + 4*units)     : int flag per (b, h, f) unit: 1 once its state is published
+//   then, 256-byte aligned   : float published state per unit, transposed: St[j][i] (dv rows of dk)
+struct Workspace {
+  int *counter;
+  int *flags;
+  float *states;
+};
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+inline size_t chain_workspace_bytes(long units, long state_elems) {
+  size_t b = 256;
+  b += align_up(sizeof(int) * (size_t)units, 256);
+  b += align_up(sizeof(float) * (size_t)units * (size_t)state_elems, 256);
+  return b;
+}
+
+inline Workspace chain_workspace(void *base, long units) {
+  char *p = (char *)base;
+  Workspace w;
+  w.counter = (int *)p;
+  w.flags = (int *)(p + 256);
+  w.states = (float *)(p + 256 + align_up(sizeof(int) * (size_t)units, 256));
+  return w;
+}
+
+// Bytes of the zero-initialised head of the workspace (counter + flags).
+inline size_t chain_workspace_zero_bytes(long units) { return 256 + align_up(sizeof(int) * (size_t)units, 256); }
+
+__device__ __forceinline__ unsigned long long global_timer_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ int ld_acquire(const int *p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void st_release(int *p, int v) {
+  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Latch the first device-side error code into *status (if given).
+__device__ __forceinline__ void latch_status(int *status, int code) {
+  if (status) atomicCAS(status, 0, code);
+}
+
+// Spin (with back-off) until *flag >= target or limit_ns elapses.  Returns
+// false on timeout.  Called by one thread.
+__device__ __forceinline__ bool wait_flag(const int *flag, int target, unsigned long long limit_ns) {
+  if (ld_acquire(flag) >= target) return true;
+  const unsigned long long t0 = global_timer_ns();
+  unsigned ns = 32;
+  while (true) {
+    __nanosleep(ns);
+    if (ld_acquire(flag) >= target) return true;
+    if (global_timer_ns() - t0 > limit_ns) return false;
+    if (ns < 256) ns *= 2;
+  }
+}
+
+template <typename T>
+__device__ __forceinline__ float to_f32(T x);
+template <>
+__device__ __forceinline__ float to_f32<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+// Gate activations (fp32): alpha = exp(-softplus(a)) = 1 / (1 + e^a); beta = sigmoid(b).
+__device__ __forceinline__ float gate_alpha(float a) { return 1.0f / (1.0f + expf(a)); }
+__device__ __forceinline__ float gate_beta(float b) { return 1.0f / (1.0f + expf(-b)); }
+
+struct GdnParams {
+  const void *q, *k, *v;
+  const float *alpha, *beta;
+  const float *state_in;
+  float *state_out;
+  float *o;
+  int B, H, F, L, dk, dv;
+  int gates_are_logits;
+  int *status;
+  unsigned long long spin_limit_ns;
+  long withhold;  // unit that never publishes (testing), -1 = none
+  Workspace ws;
+};
+
+struct ReluParams {
+  const void *q, *k, *v;
+  const float *kv_in, *z_in;
+  float *kv_out, *z_out;
+  float *o;
+  int B, H, F, L, dk, dv;
+  float eps;
+  int *status;
+  unsigned long long spin_limit_ns;
+  long withhold;  // unit that never publishes (testing), -1 = none
+  Workspace ws;
+};
+
+}  // namespace gdn

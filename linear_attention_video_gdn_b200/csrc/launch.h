@@ -1,0 +1,19 @@
+// Internal kernel launchers (host side), one per kernel family.
+#pragma once
+
+#include "common.cuh"
+
+namespace gdn {
+
+cudaError_t launch_gdn_seq(const GdnParams &p, int in_dtype, cudaStream_t st);
+cudaError_t launch_gdn_frame_simt(const GdnParams &p, int in_dtype, int grid, cudaStream_t st);
+cudaError_t launch_relu_frame_simt(const ReluParams &p, int in_dtype, int grid, cudaStream_t st);
+
+// tcgen05 / TMEM / TMA kernels (bf16 inputs, dk = dv in {16..128} multiples of 16).
+bool gdn_tc_supported(int dk, int dv);
+size_t gdn_tc_state_elems(int dk, int dv);
+cudaError_t launch_gdn_tc(const GdnParams &p, int grid, cudaStream_t st);
+bool relu_tc_supported(int dk, int dv);
+cudaError_t launch_relu_tc(const ReluParams &p, int grid, cudaStream_t st);
+
+}  // namespace gdn

@@ -1,0 +1,108 @@
+"""The C-ABI library: loads, exports every declared symbol, validates arguments on the host.
+
+No compute call runs here (this file needs no GPU): calls that pass host
+validation stop at the device query, which reports GDN_ERR_NO_DEVICE on a
+machine without an sm_100 GPU.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gdn_b200.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from linear_attention_video_gdn_b200 import build
+    build.build()
+    import linear_attention_video_gdn_b200 as lib
+    return lib
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"GDN_API\s+[\w\s\*]+?\b(\w+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_symbols()
+    assert "gdn_frame_fwd" in names and "relu_la_block_fwd" in names
+    raw = ctypes.CDLL(lib.LIB_PATH)
+    for n in names:
+        assert hasattr(raw, n), n
+    assert set(names) == set(lib.EXPORTED)
+
+
+def test_header_constants_match_binding(lib):
+    text = open(HEADER).read()
+    consts = dict((k, int(v)) for k, v in re.findall(r"#define (GDN_\w+) (\d+)", text))
+    assert consts["GDN_ABI_VERSION"] == lib.abi_version()
+    assert consts["GDN_ERR_TIMEOUT"] == lib.ERR_TIMEOUT and consts["GDN_IMPL_TC"] == lib.IMPL_TC
+    assert consts["GDN_DTYPE_BF16"] == lib.DTYPE_BF16 and consts["GDN_OP_RELU_LA"] == lib.OP_RELU_LA
+    # the ctypes mirror of gdn_opts_t has the C layout (ints, pointers, size_t in declaration order)
+    fields = re.search(r"typedef struct gdn_opts \{(.*?)\} gdn_opts_t;", text, re.S).group(1)
+    names = re.findall(r"^\s*(?:int|void|size_t)\s*\*?\s*(\w+);", fields, re.M)
+    assert names == [f[0] for f in lib.GdnOpts._fields_]
+
+
+def test_status_strings(lib):
+    for code in range(6):
+        assert isinstance(lib.status_string(code), str) and lib.status_string(code)
+    assert lib.status_string(99) == "unknown status"
+
+
+def test_workspace_sizes(lib):
+    o = lib.make_opts(lib.DTYPE_BF16, impl="frame_simt", stream=0)
+    B, H, F, L, d = 1, 20, 240, 920, 112
+    n = lib.workspace_bytes(lib.OP_GDN, B, H, F, L, d, d, o)
+    units = B * H * F
+    assert n >= units * d * d * 4 + units * 4
+    assert n % 256 == 0
+    assert lib.workspace_bytes(lib.OP_GDN, 0, H, F, L, d, d, o) == 0  # invalid sizes
+    assert lib.workspace_bytes(lib.OP_GDN, B, H, F, L, 129, d, o) == 0
+    r = lib.workspace_bytes(lib.OP_RELU_LA, 2, 20, 81, 920, d, d, o)
+    assert r >= 2 * 20 * 81 * (d + 1) * d * 4
+    seq = lib.make_opts(lib.DTYPE_F32, impl="seq", stream=0)
+    assert lib.workspace_bytes(lib.OP_GDN, B, H, F, L, d, d, seq) == 0
+
+
+def test_host_argument_validation(lib):
+    raw = lib._lib
+    o = lib.make_opts(lib.DTYPE_BF16, stream=0)
+    P = ctypes.c_void_p
+    p16 = P(0x10000)  # aligned, never dereferenced: validation fails first
+    p_odd = P(0x10001)
+    call = lambda *a: raw.gdn_frame_fwd(*a, ctypes.byref(o))
+    # null required pointer
+    assert call(None, p16, p16, p16, p16, None, None, p16, 1, 1, 1, 1, 16, 16) == lib.ERR_INVALID_ARG
+    # misaligned pointer
+    assert call(p_odd, p16, p16, p16, p16, None, None, p16, 1, 1, 1, 1, 16, 16) == lib.ERR_INVALID_ARG
+    # bad sizes
+    assert call(p16, p16, p16, p16, p16, None, None, p16, 1, 1, 0, 1, 16, 16) == lib.ERR_INVALID_ARG
+    assert call(p16, p16, p16, p16, p16, None, None, p16, 1, 1, 1, 1, 256, 16) == lib.ERR_UNSUPPORTED
+    # bad dtype / impl
+    o.in_dtype = 7
+    assert call(p16, p16, p16, p16, p16, None, None, p16, 1, 1, 1, 1, 16, 16) == lib.ERR_INVALID_ARG
+    o.in_dtype = lib.DTYPE_BF16
+    o.impl = 9
+    assert call(p16, p16, p16, p16, p16, None, None, p16, 1, 1, 1, 1, 16, 16) == lib.ERR_INVALID_ARG
+    # null opts
+    assert raw.gdn_frame_fwd(p16, p16, p16, p16, p16, None, None, p16, 1, 1, 1, 1, 16, 16, None) == \
+        lib.ERR_INVALID_ARG
+    # negative eps for the ReLU mode
+    o.impl = 0
+    assert raw.relu_la_block_fwd(p16, p16, p16, None, None, None, None, p16, 1, 1, 1, 1, 16, 16,
+                                 ctypes.c_float(-1.0), ctypes.byref(o)) == lib.ERR_INVALID_ARG
+
+
+def test_no_device_is_reported_without_gpu(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("GPU present")
+    o = lib.make_opts(lib.DTYPE_BF16, stream=0)
+    p16 = ctypes.c_void_p(0x10000)
+    rc = lib._lib.gdn_frame_fwd(p16, p16, p16, p16, p16, None, None, p16, 1, 1, 1, 1, 16, 16, ctypes.byref(o))
+    assert rc == lib.ERR_NO_DEVICE

@@ -1,0 +1,258 @@
+"""GPU parity of the Gated DeltaNet frame recurrence against the fp64 CPU oracle.
+
+Every case compares the CUDA path (called through the C ABI) with the oracle
+element by element on the same seeded inputs; the bar is
+max|gpu - oracle| <= tol * max|oracle| for o and for the output state, with
+tol = 2e-3 for bf16 inputs and 1e-5 for fp32 inputs.
+"""
+import numpy as np
+import pytest
+
+from helpers import device_inputs, oracle_gdn, rel_err, synth, tol_for
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+W = synth.WORKLOADS
+
+
+@pytest.fixture(scope="module")
+def lib():
+    import linear_attention_video_gdn_b200 as lib
+    return lib
+
+
+@pytest.fixture(scope="module")
+def dev():
+    return torch.device("cuda", 0)
+
+
+def run_gdn(lib, w, t, dev, impl, state_in=None, want_state=True, **kw):
+    s_out = torch.empty((w.B, w.H, w.dk, w.dv), dtype=torch.float32, device=dev) if want_state else None
+    s_in = None if state_in is None else torch.from_numpy(np.asarray(state_in, np.float32)).to(dev)
+    o = lib.gdn_frame_fwd(t["q"], t["k"], t["v"], t["a"], t["b"], F=w.F, state_in=s_in, state_out=s_out,
+                          impl=impl, **kw)
+    torch.cuda.synchronize()
+    return o.cpu().numpy(), (None if s_out is None else s_out.cpu().numpy())
+
+
+def impls_for(w):
+    out = ["seq", "frame_simt"]
+    if w.dtype == "bf16" and w.dk % 16 == 0 and w.dv % 16 == 0:
+        out.append("tc")
+    return out
+
+
+# ------------------------------------------------------------------ the workloads
+
+@pytest.mark.parametrize("impl", ["seq", "frame_simt"])
+def test_tiny_fp32(lib, dev, impl):
+    w = W["tiny_fp32"]
+    x = synth.inputs(w)
+    t, h = device_inputs(w, x, dev, torch)
+    o, s = run_gdn(lib, w, t, dev, impl)
+    o_ref, s_ref = oracle_gdn(h, w)
+    assert rel_err(o, o_ref) <= 1e-5
+    assert rel_err(s, s_ref) <= 1e-5
+
+
+@pytest.mark.parametrize("impl", ["frame_simt", "tc"])
+def test_480p_5s(lib, dev, impl):
+    w = W["gdn_480p_5s"]
+    x = synth.inputs(w)
+    t, h = device_inputs(w, x, dev, torch)
+    o, s = run_gdn(lib, w, t, dev, impl)
+    o_ref, s_ref = oracle_gdn(h, w)
+    eo, es = rel_err(o, o_ref), rel_err(s, s_ref)
+    print(f"480p {impl}: err_o={eo:.3e} err_s={es:.3e}")
+    assert eo <= 2e-3 and es <= 2e-3
+
+
+@pytest.mark.parametrize("impl", ["frame_simt", "tc"])
+def test_720p_60s_sampled(lib, dev, impl):
+    """Full 720p-60s size in the benchmark's launch configuration; the oracle
+    recomputes two heads on a subset of d_v columns (columns evolve independently)."""
+    w = W["gdn_720p_60s"]
+    x = synth.inputs(w)
+    t, h = device_inputs(w, x, dev, torch)
+    o, s = run_gdn(lib, w, t, dev, impl)
+    heads = [0, 13]
+    cols = (40, 56)
+    sub = {n: h[n].reshape((w.B * w.H,) + h[n].shape[2:])[heads] for n in "qkvab"}
+    o_ref, s_ref = synth_free_oracle(sub, w, cols)
+    o_g = o.reshape((w.B * w.H,) + o.shape[2:])[heads]
+    s_g = s.reshape((w.B * w.H,) + s.shape[2:])[heads]
+    eo, es = rel_err(o_g[..., cols[0]:cols[1]], o_ref[..., cols[0]:cols[1]]), \
+        rel_err(s_g[..., cols[0]:cols[1]], s_ref[..., cols[0]:cols[1]])
+    print(f"720p {impl}: err_o={eo:.3e} err_s={es:.3e}")
+    assert eo <= 2e-3 and es <= 2e-3
+    assert np.isfinite(o).all() and np.isfinite(s).all()
+
+
+def synth_free_oracle(sub, w, cols):
+    from helpers import oracle
+    return oracle.gdn(sub["q"], sub["k"], sub["v"], sub["a"], sub["b"], F=w.F, L=w.L, cols=cols)
+
+
+# ------------------------------------------------------------------ shapes and tails
+
+SHAPES = [  # (F, L, dk, dv, H)
+    (1, 1, 32, 32, 1), (2, 16, 64, 64, 2), (3, 63, 112, 112, 1), (2, 64, 112, 112, 2), (2, 65, 112, 112, 1),
+    (7, 20, 128, 128, 1), (1, 390, 112, 112, 2), (2, 129, 48, 80, 1), (3, 37, 16, 16, 3),
+]
+
+
+@pytest.mark.parametrize("F,L,dk,dv,H", SHAPES)
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_shapes_all_impls(lib, dev, F, L, dk, dv, H, dtype):
+    w = W["gdn_480p_5s"].with_(F=F, L=L, dk=dk, dv=dv, H=H, B=1 + (H == 1), dtype=dtype, seed=100 + F + L)
+    x = synth.inputs(w)
+    t, h = device_inputs(w, x, dev, torch)
+    S0 = np.random.default_rng(L).standard_normal((w.B, w.H, dk, dv)).astype(np.float32)
+    o_ref, s_ref = oracle_gdn(h, w, state_in=S0)
+    tol = tol_for(w)
+    for impl in impls_for(w):
+        o, s = run_gdn(lib, w, t, dev, impl, state_in=S0)
+        assert rel_err(o, o_ref) <= tol, impl
+        assert rel_err(s, s_ref) <= tol, impl
+
+
+def test_streaming_equals_whole_sequence(lib, dev):
+    """F=1 calls that carry the state reproduce one call over all frames."""
+    w = W["gdn_480p_5s"].with_(F=4, L=90, H=3)
+    x = synth.inputs(w)
+    t, h = device_inputs(w, x, dev, torch)
+    for impl in impls_for(w):
+        o_all, s_all = run_gdn(lib, w, t, dev, impl)
+        S = None
+        outs = []
+        for f in range(w.F):
+            sl = slice(f * w.L, (f + 1) * w.L)
+            s_out = torch.empty((w.B, w.H, w.dk, w.dv), dtype=torch.float32, device=dev)
+            o = lib.gdn_frame_fwd(t["q"][:, :, sl].contiguous(), t["k"][:, :, sl].contiguous(),
+                                  t["v"][:, :, sl].contiguous(), t["a"][:, :, f:f + 1].contiguous(),
+                                  t["b"][:, :, sl].contiguous(), F=1, state_in=S, state_out=s_out, impl=impl)
+            outs.append(o)
+            S = s_out
+        torch.cuda.synchronize()
+        o_str = torch.cat(outs, dim=2).cpu().numpy()
+        assert rel_err(o_str, o_all) <= 1e-5, impl
+        assert rel_err(S.cpu().numpy(), s_all) <= 1e-5, impl
+
+
+def test_in_place_state_carry(lib, dev):
+    w = W["gdn_480p_5s"].with_(F=2, L=50, H=2)
+    x = synth.inputs(w)
+    t, h = device_inputs(w, x, dev, torch)
+    S0 = np.random.default_rng(5).standard_normal((w.B, w.H, w.dk, w.dv)).astype(np.float32)
+    o_ref, s_ref = oracle_gdn(h, w, state_in=S0)
+    for impl in impls_for(w):
+        S = torch.from_numpy(S0).to(dev)
+        o = lib.gdn_frame_fwd(t["q"], t["k"], t["v"], t["a"], t["b"], F=w.F, state_in=S, state_out=S, impl=impl)
+        torch.cuda.synchronize()
+        assert rel_err(o.cpu().numpy(), o_ref) <= 2e-3, impl
+        assert rel_err(S.cpu().numpy(), s_ref) <= 2e-3, impl
+
+
+def test_gate_values_and_edge_gates(lib, dev):
+    """Gates passed as values; alpha = 1 with beta = 0 leaves the state unchanged."""
+    w = W["gdn_480p_5s"].with_(F=3, L=40, H=2)
+    x = synth.inputs(w)
+    t, h = device_inputs(w, x, dev, torch)
+    S0 = np.random.default_rng(2).standard_normal((w.B, w.H, w.dk, w.dv)).astype(np.float32)
+    ones = torch.ones_like(t["a"])
+    zeros = torch.zeros_like(t["b"])
+    for impl in impls_for(w):
+        s_out = torch.empty((w.B, w.H, w.dk, w.dv), dtype=torch.float32, device=dev)
+        o = lib.gdn_frame_fwd(t["q"], t["k"], t["v"], ones, zeros, F=w.F, gates_are_logits=False,
+                              state_in=torch.from_numpy(S0).to(dev), state_out=s_out, impl=impl)
+        torch.cuda.synchronize()
+        assert rel_err(s_out.cpu().numpy(), S0) <= 2e-3, impl
+        expect = np.einsum("bhnd,bhde->bhne", h["q"].astype(np.float64), S0.astype(np.float64))
+        assert rel_err(o.cpu().numpy(), expect) <= 2e-3, impl
+    # value gates agree with the logit gates
+    al = torch.sigmoid(-t["a"])
+    be = torch.sigmoid(t["b"])
+    o_ref, s_ref = oracle_gdn(h, w)
+    for impl in impls_for(w):
+        s_out = torch.empty((w.B, w.H, w.dk, w.dv), dtype=torch.float32, device=dev)
+        o = lib.gdn_frame_fwd(t["q"], t["k"], t["v"], al, be, F=w.F, gates_are_logits=False, state_out=s_out,
+                              impl=impl)
+        torch.cuda.synchronize()
+        assert rel_err(o.cpu().numpy(), o_ref) <= 2e-3, impl
+
+
+def test_zero_keys_and_large_values(lib, dev):
+    w = W["gdn_480p_5s"].with_(F=2, L=70, H=2, unit_keys=False)
+    x = synth.inputs(w)
+    x["k"][:, :, 5] = 0.0
+    x["k"][:, :, 69:75] = 0.0
+    x["k"] *= 7.0   # unnormalised keys
+    x["v"] *= 50.0  # larger values
+    t, h = device_inputs(w, x, dev, torch)
+    o_ref, s_ref = oracle_gdn(h, w)
+    for impl in impls_for(w):
+        o, s = run_gdn(lib, w, t, dev, impl)
+        assert rel_err(o, o_ref) <= 2e-3, impl
+        assert rel_err(s, s_ref) <= 2e-3, impl
+
+
+def test_few_ctas_many_frames(lib, dev):
+    """A persistent grid far smaller than the frame count still completes the chain."""
+    w = W["gdn_480p_5s"].with_(F=30, L=33, H=3)
+    x = synth.inputs(w)
+    t, h = device_inputs(w, x, dev, torch)
+    o_ref, s_ref = oracle_gdn(h, w)
+    for impl in impls_for(w):
+        if impl == "seq":
+            continue
+        for ctas in (1, 2, 7):
+            o, s = run_gdn(lib, w, t, dev, impl, max_ctas=ctas)
+            assert rel_err(o, o_ref) <= 2e-3, (impl, ctas)
+            assert rel_err(s, s_ref) <= 2e-3, (impl, ctas)
+
+
+def test_deterministic(lib, dev):
+    w = W["gdn_480p_5s"].with_(F=5, L=100, H=4)
+    x = synth.inputs(w)
+    t, _ = device_inputs(w, x, dev, torch)
+    for impl in impls_for(w):
+        o1, s1 = run_gdn(lib, w, t, dev, impl)
+        o2, s2 = run_gdn(lib, w, t, dev, impl)
+        np.testing.assert_array_equal(o1, o2)
+        np.testing.assert_array_equal(s1, s2)
+
+
+def test_host_entry_point(lib, dev):
+    w = W["gdn_480p_5s"].with_(F=3, L=64, H=2)
+    x = synth.inputs(w)
+    t, h = device_inputs(w, x, dev, torch)
+    o_dev, s_dev = run_gdn(lib, w, t, dev, "auto")
+    qh, kh, vh = (t[n].cpu().pin_memory() for n in "qkv")
+    ah, bh = t["a"].cpu().pin_memory(), t["b"].cpu().pin_memory()
+    o_h = torch.empty((w.B, w.H, w.N, w.dv), dtype=torch.float32).pin_memory()
+    s_h = torch.empty((w.B, w.H, w.dk, w.dv), dtype=torch.float32).pin_memory()
+    lib.gdn_frame_fwd_host(qh, kh, vh, ah, bh, F=w.F, o=o_h, state_out=s_h)
+    np.testing.assert_array_equal(o_h.numpy(), o_dev)
+    np.testing.assert_array_equal(s_h.numpy(), s_dev)
+
+
+def test_device_timeout_status_is_reported(lib, dev):
+    """A chain wait that is never satisfied ends with GDN_ERR_TIMEOUT in *status.
+
+    The test asks the kernel to withhold the publish of frame 0 of head 0, so
+    the wait of frame 1 of that head runs out after 2 ms; the kernel returns
+    cleanly and the context stays usable for the next call.
+    """
+    w = W["gdn_480p_5s"].with_(F=3, L=16, H=1)
+    x = synth.inputs(w)
+    t, h = device_inputs(w, x, dev, torch)
+    for impl in [i for i in impls_for(w) if i != "seq"]:
+        status = torch.zeros(4, dtype=torch.int32, device=dev)
+        run_gdn(lib, w, t, dev, impl, spin_limit_us=2000, status=status, test_withhold_unit=0)
+        assert int(status[0].item()) == lib.ERR_TIMEOUT, impl
+        status.zero_()
+        o, s = run_gdn(lib, w, t, dev, impl, status=status)
+        assert int(status[0].item()) == 0
+        o_ref, s_ref = oracle_gdn(h, w)
+        assert rel_err(o, o_ref) <= 2e-3
