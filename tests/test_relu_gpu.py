@@ -34,7 +34,7 @@ def prep(w, x, dev):
 
 def impls_for(w):
     out = ["frame_simt"]
-    if w.dtype == "bf16" and w.dk % 16 == 0 and w.dv % 16 == 0:
+    if w.dtype == "bf16" and w.dk % 16 == 0 and w.dv % 16 == 0 and w.dv <= 112:
         out.append("tc")
     return out
 
