@@ -67,7 +67,7 @@ struct Bars {
   uint32_t tmem_base;
   int abort;
   int ticket_ring[4];
-  float beta[2][64];
+  __align__(16) float beta[2][64];
 };
 constexpr size_t kGdnSmemBytes = OFF_BAR + sizeof(Bars) + 1024;
 
@@ -266,11 +266,11 @@ __global__ void __launch_bounds__(kGThreads, 1)
         break;
       }
       tc_fence_after();
-      // 4. N[t][u] = beta_t G[t][u] for u < t (rows t = TMEM lanes 0..63: warps 8, 9)
-      float *Ns = reinterpret_cast<float *>(sm + OFF_N);
+      // 4. Nt[u][t] = N[t][u] = beta_t G[t][u] for t > u (G is symmetric, so lane u
+      //    reads row u of G); TMEM lanes 0..63 live in warps 8 and 9.
+      float *Nt = reinterpret_cast<float *>(sm + OFF_N);
       if (warp < 10) {
-        const int t = pt;  // lane
-        const float bt = bar.beta[s][t];
+        const int u = pt;  // lane
 #pragma unroll
         for (int cb = 0; cb < 4; ++cb) {
           float r[16];
@@ -278,40 +278,46 @@ __global__ void __launch_bounds__(kGThreads, 1)
           tmem_ld_wait();
 #pragma unroll
           for (int e = 0; e < 16; e += 4) {
-            const int u = cb * 16 + e;
+            const int t = cb * 16 + e;
+            const float4 b4 = *reinterpret_cast<const float4 *>(&bar.beta[s][t]);
             float4 o4;
-            o4.x = (u + 0 < t) ? bt * r[e + 0] : 0.f;
-            o4.y = (u + 1 < t) ? bt * r[e + 1] : 0.f;
-            o4.z = (u + 2 < t) ? bt * r[e + 2] : 0.f;
-            o4.w = (u + 3 < t) ? bt * r[e + 3] : 0.f;
-            *reinterpret_cast<float4 *>(Ns + t * N_STRIDE + u) = o4;
+            o4.x = (t + 0 > u) ? b4.x * r[e + 0] : 0.f;
+            o4.y = (t + 1 > u) ? b4.y * r[e + 1] : 0.f;
+            o4.z = (t + 2 > u) ? b4.z * r[e + 2] : 0.f;
+            o4.w = (t + 3 > u) ? b4.w * r[e + 3] : 0.f;
+            *reinterpret_cast<float4 *>(Nt + u * N_STRIDE + t) = o4;
           }
         }
       }
       tc_fence_before();
       named_bar(2, 128);
-      // 5. T = (I + N)^-1 diag(beta): thread s' < 64 solves column s' by forward substitution
+      // 5. T = (I + N)^-1 diag(beta): thread `col` < 64 solves column col of
+      //    X = (I + N)^-1 by forward substitution in axpy form: once x_u is
+      //    final, acc[t] += N[t][u] x_u for every later t (independent FMAs),
+      //    and x_t = -acc[t].  The critical path is one FMA per step.
       if (pt < 64) {
         const int col = pt;
-        float x[64];
+        float acc[64];
 #pragma unroll
-        for (int t = 0; t < 64; ++t) {
-          float acc = 0.f;
+        for (int t = 0; t < 64; ++t) acc[t] = 0.f;
 #pragma unroll
-          for (int u = 0; u < t; u += 4) {
-            const float4 n4 = *reinterpret_cast<const float4 *>(Ns + t * N_STRIDE + u);
-            acc += n4.x * x[u];
-            if (u + 1 < t) acc += n4.y * x[u + 1];
-            if (u + 2 < t) acc += n4.z * x[u + 2];
-            if (u + 3 < t) acc += n4.w * x[u + 3];
+        for (int u = 0; u < 64; ++u) {
+          const float xu = (u == col) ? 1.f : (u < col ? 0.f : -acc[u]);
+          acc[u] = xu;
+#pragma unroll
+          for (int t4 = ((u + 1) >> 2) << 2; t4 < 64; t4 += 4) {
+            const float4 n4 = *reinterpret_cast<const float4 *>(Nt + u * N_STRIDE + t4);
+            if (t4 + 0 > u) acc[t4 + 0] = fmaf(n4.x, xu, acc[t4 + 0]);
+            if (t4 + 1 > u) acc[t4 + 1] = fmaf(n4.y, xu, acc[t4 + 1]);
+            if (t4 + 2 > u) acc[t4 + 2] = fmaf(n4.z, xu, acc[t4 + 2]);
+            if (t4 + 3 > u) acc[t4 + 3] = fmaf(n4.w, xu, acc[t4 + 3]);
           }
-          x[t] = (t == col) ? 1.f : (t < col ? 0.f : -acc);
         }
         const float bc = bar.beta[s][col];
         uint8_t *Tt = sm + OFF_T + s * 8192;
 #pragma unroll
         for (int t = 0; t < 64; ++t)
-          *reinterpret_cast<__half *>(Tt + sw128_offset(t, col)) = __float2half_rn(x[t] * bc);
+          *reinterpret_cast<__half *>(Tt + sw128_offset(t, col)) = __float2half_rn(acc[t] * bc);
       }
       fence_async_smem();
       named_bar(2, 128);

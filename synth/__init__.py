@@ -132,7 +132,7 @@ WORKLOADS = {
 }
 
 
-def inputs(w: Workload, heads=None, call: int = 0) -> dict:
+def inputs(w: Workload, heads=None, call: int = 0, frames: int | None = None) -> dict:
     """Draw q, k, v, a, b for workload ``w`` (float32 numpy arrays).
 
     ``heads``: None for all B*H heads (arrays shaped [B, H, ...]); else a list
@@ -140,9 +140,13 @@ def inputs(w: Workload, heads=None, call: int = 0) -> dict:
     ``call``: streaming call index (frame * steps + step); each call has its
     own fresh inputs.  For streaming workloads one call covers one frame, so
     the token count per head is L (not F*L) and a has one entry per head.
+    ``frames``: draw only the first ``frames`` frames of every head (same
+    values as the full draw; arrays hold frames * L tokens).
     """
-    N = w.L if w.mode == "gdn_stream" else w.N
-    F = 1 if w.mode == "gdn_stream" else w.F
+    Nfull = w.L if w.mode == "gdn_stream" else w.N
+    Ffull = 1 if w.mode == "gdn_stream" else w.F
+    F = Ffull if frames is None else min(frames, Ffull)
+    N = F * w.L
     off = TID_STRIDE_PER_CALL * call
     hl = list(range(w.B * w.H)) if heads is None else list(heads)
     n = len(hl)
@@ -152,14 +156,14 @@ def inputs(w: Workload, heads=None, call: int = 0) -> dict:
     a = np.empty((n, F), np.float32)
     b = np.empty((n, N), np.float32)
     for i, bh in enumerate(hl):
-        normal(w.seed, TID_Q + off, bh * N * w.dk, N * w.dk, out=q[i].reshape(-1))
+        normal(w.seed, TID_Q + off, bh * Nfull * w.dk, N * w.dk, out=q[i].reshape(-1))
         if w.unit_keys:
-            unit_rows(w.seed, TID_K + off, bh * N, N, w.dk, out=k[i])
+            unit_rows(w.seed, TID_K + off, bh * Nfull, N, w.dk, out=k[i])
         else:
-            normal(w.seed, TID_K + off, bh * N * w.dk, N * w.dk, out=k[i].reshape(-1))
-        normal(w.seed, TID_V + off, bh * N * w.dv, N * w.dv, out=v[i].reshape(-1))
-        normal(w.seed, TID_A + off, bh * F, F, mean=w.a_mean, out=a[i])
-        normal(w.seed, TID_B + off, bh * N, N, out=b[i])
+            normal(w.seed, TID_K + off, bh * Nfull * w.dk, N * w.dk, out=k[i].reshape(-1))
+        normal(w.seed, TID_V + off, bh * Nfull * w.dv, N * w.dv, out=v[i].reshape(-1))
+        normal(w.seed, TID_A + off, bh * Ffull, F, mean=w.a_mean, out=a[i])
+        normal(w.seed, TID_B + off, bh * Nfull, N, out=b[i])
     if heads is None:
         q = q.reshape(w.B, w.H, N, w.dk)
         k = k.reshape(w.B, w.H, N, w.dk)

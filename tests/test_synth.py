@@ -57,3 +57,12 @@ def test_workload_inputs_heads_slice():
     s0 = synth.inputs(synth.WORKLOADS["gdn_stream_720p"].with_(L=5, H=2), call=0)
     s1 = synth.inputs(synth.WORKLOADS["gdn_stream_720p"].with_(L=5, H=2), call=1)
     assert s0["q"].shape == (1, 2, 5, 112) and not np.array_equal(s0["q"], s1["q"])
+
+
+def test_leading_frames_match_full_draw():
+    w = synth.WORKLOADS["gdn_480p_5s"].with_(F=4, L=5, H=3)
+    full = synth.inputs(w)
+    part = synth.inputs(w, frames=2)
+    for key in "qkvb":
+        np.testing.assert_array_equal(part[key], full[key][:, :, :10])
+    np.testing.assert_array_equal(part["a"], full["a"][:, :, :2])
