@@ -157,6 +157,32 @@ GDN_API int gdn_frame_fwd_host(const void *q, const void *k, const void *v, cons
                        const float *state_in, float *state_out, float *o, int B, int H, int F, int L,
                        int dk, int dv, const gdn_opts_t *opts);
 
+/*
+ * gdn_frame_fwd_noalloc -- gdn_frame_fwd without a caller-provided workspace.
+ *
+ * The pages describe no counterpart of this call; it exists for callers that
+ * cannot allocate device memory at all (for example a plugin inside a host
+ * program that owns every device allocation and passes the plugin only its
+ * input and output buffers, or a runtime with a fixed memory plan that allows
+ * no allocation after start-up).  Arguments, semantics and layouts are those of
+ * gdn_frame_fwd; opts->workspace and opts->workspace_bytes are ignored.
+ *
+ * The frame-chain scratch comes from a fixed array inside the library, of
+ * GDN_NOALLOC_SCRATCH_BYTES on every GPU that loads the library, kept until
+ * the process exits.  Calls whose gdn_workspace_bytes(GDN_OP_GDN, ...) exceeds
+ * that size return GDN_ERR_UNSUPPORTED without launching anything.  The first
+ * call on a device looks up the array's device address; make that first call
+ * before any stream capture.  All calls share the array: calls that may run
+ * at the same time on the GPU (other streams, unordered host threads) race on
+ * it and must be serialised by the caller.  Each call clears the part of the
+ * array that must start at zero before its kernel runs.  The call allocates
+ * no memory.
+ */
+#define GDN_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+GDN_API int gdn_frame_fwd_noalloc(const void *q, const void *k, const void *v, const float *alpha,
+                                  const float *beta, const float *state_in, float *state_out, float *o, int B,
+                                  int H, int F, int L, int dk, int dv, const gdn_opts_t *opts);
+
 /* Device scratch bytes that op (GDN_OP_*) needs for these sizes and options. */
 GDN_API size_t gdn_workspace_bytes(int op, int B, int H, int F, int L, int dk, int dv, const gdn_opts_t *opts);
 

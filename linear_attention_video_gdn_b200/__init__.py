@@ -18,7 +18,7 @@ LIB_PATH = os.path.join(_HERE, "libgdn_b200.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m linear_attention_video_gdn_b200.build` "
+        f"{LIB_PATH} is missing: build it with `python linear_attention_video_gdn_b200/build.py` "
         "(there is no CPU fallback)")
 
 _lib = ctypes.CDLL(LIB_PATH)
@@ -29,8 +29,9 @@ IMPL_AUTO, IMPL_SEQ, IMPL_FRAME_SIMT, IMPL_TC = 0, 1, 2, 3
 OP_GDN, OP_RELU_LA = 0, 1
 IMPLS = {"auto": IMPL_AUTO, "seq": IMPL_SEQ, "frame_simt": IMPL_FRAME_SIMT, "tc": IMPL_TC}
 
-EXPORTED = ("gdn_frame_fwd", "relu_la_block_fwd", "gdn_frame_fwd_host", "gdn_workspace_bytes",
-            "gdn_workspace_bytes_host", "gdn_status_string", "gdn_abi_version")
+EXPORTED = ("gdn_frame_fwd", "relu_la_block_fwd", "gdn_frame_fwd_host", "gdn_frame_fwd_noalloc",
+            "gdn_workspace_bytes", "gdn_workspace_bytes_host", "gdn_status_string", "gdn_abi_version")
+NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 
 class GdnOpts(ctypes.Structure):
@@ -46,6 +47,8 @@ _lib.gdn_frame_fwd.argtypes = [_P] * 8 + [_I] * 6 + [ctypes.POINTER(GdnOpts)]
 _lib.gdn_frame_fwd.restype = _I
 _lib.gdn_frame_fwd_host.argtypes = [_P] * 8 + [_I] * 6 + [ctypes.POINTER(GdnOpts)]
 _lib.gdn_frame_fwd_host.restype = _I
+_lib.gdn_frame_fwd_noalloc.argtypes = [_P] * 8 + [_I] * 6 + [ctypes.POINTER(GdnOpts)]
+_lib.gdn_frame_fwd_noalloc.restype = _I
 _lib.relu_la_block_fwd.argtypes = [_P] * 8 + [_I] * 6 + [ctypes.c_float, ctypes.POINTER(GdnOpts)]
 _lib.relu_la_block_fwd.restype = _I
 _lib.gdn_workspace_bytes.argtypes = [_I] * 7 + [ctypes.POINTER(GdnOpts)]
@@ -233,3 +236,37 @@ def gdn_frame_fwd_host(q, k, v, alpha, beta, *, F: int, o, state_in=None, state_
 
 def host_workspace_bytes(B, H, F, L, dk, dv, opts: GdnOpts) -> int:
     return int(_lib.gdn_workspace_bytes_host(B, H, F, L, dk, dv, ctypes.byref(opts)))
+
+
+def gdn_frame_fwd_noalloc(q, k, v, alpha, beta, *, F: int, state_in=None, state_out=None, o=None,
+                          gates_are_logits: bool = True, impl="auto", stream=None, status=None):
+    """gdn_frame_fwd for callers that cannot allocate device memory.
+
+    Same arguments and result as gdn_frame_fwd, but the frame-chain scratch is
+    a fixed array inside the library (NOALLOC_SCRATCH_BYTES per GPU) instead of
+    a caller workspace; sizes that need more scratch raise GdnError
+    (ERR_UNSUPPORTED).  Calls share that array, so calls that could overlap on
+    the GPU must be serialised.  ``o`` should be passed by callers that cannot
+    allocate; when it is None this wrapper (not the library) creates it.
+    """
+    B, H, N, dk = q.shape
+    dv = v.shape[-1]
+    if N % F:
+        raise ValueError(f"token count {N} is not a multiple of F={F}")
+    L = N // F
+    dev = q.device
+    _check(k, "k", (B, H, N, dk), q.dtype, dev)
+    _check(v, "v", (B, H, N, dv), q.dtype, dev)
+    _check(alpha, "alpha", (B, H, F), torch.float32, dev)
+    _check(beta, "beta", (B, H, N), torch.float32, dev)
+    _check(state_in, "state_in", (B, H, dk, dv), torch.float32, dev, allow_none=True)
+    _check(state_out, "state_out", (B, H, dk, dv), torch.float32, dev, allow_none=True)
+    if o is None:
+        o = torch.empty((B, H, N, dv), dtype=torch.float32, device=dev)
+    _check(o, "o", (B, H, N, dv), torch.float32, dev)
+    opts = make_opts(_dtype_code(q), gates_are_logits=gates_are_logits, impl=impl, stream=stream, status=status)
+    rc = _lib.gdn_frame_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(state_in),
+                                    _ptr(state_out), _ptr(o), B, H, F, L, dk, dv, ctypes.byref(opts))
+    if rc != OK:
+        raise GdnError(rc, "gdn_frame_fwd_noalloc")
+    return o

@@ -1,6 +1,7 @@
 """Build libgdn_b200.so in place: every csrc/*.cu for sm_100a with nvcc.
 
-Usage: python -m linear_attention_video_gdn_b200.build [--force]
+Usage: python linear_attention_video_gdn_b200/build.py [--force] [-v]
+(run by path: importing the package would load the library it builds)
 """
 from __future__ import annotations
 

@@ -16,8 +16,8 @@ HEADER = os.path.join(ROOT, "include", "gdn_b200.h")
 
 @pytest.fixture(scope="module")
 def lib():
-    from linear_attention_video_gdn_b200 import build
-    build.build()
+    import __graft_entry__
+    __graft_entry__.build()
     import linear_attention_video_gdn_b200 as lib
     return lib
 
