@@ -12,26 +12,32 @@
 // A_f = ordered product of (I - beta_t khat_t khat_t^T), B_f = the frame's
 // update from a zero state, by running the delta rule on Y = [A | B] from
 // [I | 0] with targets [0 | V], chunked 64 tokens at a time in the UT form
-//     R = [0 | V] - Khat Y,   Y <- Y + Khat^T T R = Y + W^T R,
+//     Y <- Y + W^T ([0 | V] - Khat Y),   W^T = Khat^T T,
 //     T = (I + N)^-1 diag(beta),  N = strict_lower(diag(beta) Khat Khat^T),
-//     W = T^T Khat = diag(beta) Z,  (I + N^T) Z = Khat  (back substitution),
 // kept transposed in TMEM (lanes = columns of A and B, fp32).  Only the
 // d x d chain step S_f = ... waits on the previous frame's published state.
 // Then O_f = Q_f S_f.
 //
-// Warp roles (384 threads):
-//   warps 0-3  "tile A" and warps 4-7 "tile B": two independent chains, one
-//              per 128-lane TMEM tile of Y^T (A^T rows, B^T rows).  Per chunk
-//              each runs R^T = [0 ; V^T] - Y^T Khat^T and Y^T += R^T W on
-//              tcgen05 with a TMEM -> fp16 shared-memory conversion after
-//              each; the first thread of each issues its MMAs.  Together they
-//              run the chain step, the read-out MMAs and the fp32 epilogue.
-//   warps 8-11 "prep": TMA loads of k, v; key normalisation (fp16 khat);
-//              Gram matrix Khat Khat^T on tcgen05; the back substitution for
-//              W on CUDA cores (one thread per d_k column).  Runs up to two
-//              chunks ahead.
-// Operands that are not exact in bf16 (khat, Y, R, U, T, S, q) enter the
-// tensor cores as fp16 (11-bit significands); all accumulation is fp32.
+// Warp roles (512 threads):
+//   warps 0-3, 4-7  tile chains A and B, one per 128-lane TMEM tile of Y^T
+//                   (rows of A^T, rows of B^T).  Per chunk: R^T = -Y^T Khat^T
+//                   on tcgen05, R^T back into TMEM as fp16 pairs, Y^T += R^T W
+//                   (+ V^T W for tile B, the [0 | V] target) with R^T read from
+//                   TMEM, and an fp16 copy of Y^T in shared memory for the next
+//                   chunk.  The first chunk of a frame starts from Y = [I | 0],
+//                   so its R^T is -Khat^T and [0 | V] directly.  Together the
+//                   eight warps run the chain step, publish S_f and read out.
+//   warps 8-11, 12-15  two prep groups for even and odd chunks: gates beta,
+//                   key normalisation (fp16 khat), v to fp16, Gram matrix Khat
+//                   Khat^T on tcgen05, T by blocked inversion of the unit lower
+//                   triangular I + N (16 x 16 fp32 blocks on CUDA cores), W^T =
+//                   Khat^T T on tcgen05, fp16 W for the chains.
+// k and v reach a 3-slot ring by TMA, issued by the chains as soon as a slot's
+// last MMA has completed (chunk c + 3 after chunk c; a frame's first three
+// chunks as soon as its ticket is taken).
+// Operands that are not exact in bf16 (khat, v after the cast, Y, R, T, W, S,
+// q) enter the tensor cores as fp16 (11-bit significands); all accumulation is
+// fp32.
 #include "launch.h"
 #include "tc_host.h"
 #include "tc_ptx.cuh"
@@ -39,49 +45,51 @@
 namespace gdn {
 namespace tc {
 
-constexpr int kGThreads = 384;  // 8 chain warps + 1 prep warpgroup
-constexpr int kChain = 256;  // warps 0-7
-constexpr int kC = 64;       // tokens per chunk
+constexpr int kChain = 256;      // warps 0-7
+constexpr int kGThreads = 512;   // + two prep warpgroups
+constexpr int kC = 64;           // tokens per chunk
+constexpr int kSlots = 3;        // chunks in flight (k, v, W)
+constexpr int kQTok = 64;        // tokens per read-out tile
 
 // shared memory map (bytes from the 1024-aligned base)
-constexpr uint32_t OFF_MIRROR = 0;         // 64 KB: Y^T as fp16, [tile][k-block][128 rows][128 B]
-constexpr uint32_t OFF_RU = 65536;         // 32 KB: R^T fp16, [tile][128 rows][128 B]
-constexpr uint32_t OFF_KHAT = 98304;       // 48 KB: khat ring, [k-block][3 slots][64 rows][128 B]
-constexpr uint32_t KHAT_KB_STRIDE = 24576;
-constexpr uint32_t OFF_V = 147456;         // 32 KB: v ring (bf16, raw), [slot][dv-block][64 rows][128 B]
-constexpr uint32_t OFF_W = 180224;         // 32 KB: W ring fp16, [slot][128 rows i][128 B (64 tokens)];
-                                           //        while the prep group works on a slot it first holds
-                                           //        N (fp32 64 x 64, float4-XOR-swizzled rows)
-constexpr uint32_t OFF_I = 212992;         // 8 KB: identity 64 x 64 bf16 (K-major)
-constexpr uint32_t OFF_NHL = 221184;       // 4 KB: fp16 block N[32 + u][t] (t, u < 32), rows t, K-major
-constexpr uint32_t OFF_BAR = 225280;       // barriers and small state
-// read-out phase aliases
-constexpr uint32_t OFF_S16 = OFF_MIRROR;           // S_f as fp16 B operand [k-block][128 rows j][128 B]
-constexpr uint32_t OFF_SPREV = OFF_MIRROR + 32768; // alpha S_{f-1}^T fp16 A operand (mirror tile-B region)
-constexpr uint32_t OFF_Q0 = OFF_RU;                // q tile buffer 0 (32 KB)
-constexpr uint32_t OFF_Q1 = OFF_MIRROR + 32768;    // q tile buffer 1 (32 KB, after the chain MMA)
+constexpr uint32_t OFF_MIRROR = 0;       // 64 KB: Y^T as fp16, [tile][k-block][128 rows][128 B]
+constexpr uint32_t OFF_SLOT = 65536;     // 3 slots of 48 KB:
+constexpr uint32_t SLOT_BYTES = 49152;
+constexpr uint32_t SL_KHAT = 0;          //   khat fp16 (TMA'd bf16 k, normalised in place) [k-block][64 t][128 B]
+constexpr uint32_t SL_V = 16384;         //   v fp16 (TMA'd bf16, cast in place) [j-block][64 t][128 B]
+constexpr uint32_t SL_W = 32768;         //   W fp16, [128 rows i][128 B (64 t)]; fp32 16 x 16 blocks of the
+                                         //   inversion while the prep group works on the slot
+constexpr uint32_t OFF_T = OFF_SLOT + kSlots * SLOT_BYTES;  // 2 x 8 KB: T fp16 [64 rows u][128 B (64 t)]
+constexpr uint32_t OFF_BAR = OFF_T + 2 * 8192;              // barriers and small state
+// read-out aliases (the mirror is free once the chain step has read A_f^T)
+constexpr uint32_t OFF_S16 = OFF_MIRROR;          // S_f^T fp16 [k-block][128 rows j][128 B]
+constexpr uint32_t OFF_QB = OFF_MIRROR + 32768;   // two q tiles [k-block][64 t][128 B]
 
 struct Bars {
-  uint64_t kv_full[2];
-  uint64_t khat_ready[2];
-  uint64_t w_ready[2];
-  uint64_t slot_free[2];  // two arrivals: the last MMA of each tile chain on the slot
-  uint64_t g_bar;
-  uint64_t mma_bar[2];    // per tile chain
-  uint64_t fr_bar;        // frame-level MMAs (chain step, read-out)
+  uint64_t kv_full[kSlots];     // TMA bytes of k and v
+  uint64_t khat_ready[kSlots];  // prep: khat normalised
+  uint64_t w_ready[kSlots];     // prep: W written
+  uint64_t slot_free[kSlots];   // the last MMA of each tile chain on the slot (2 arrivals)
+  uint64_t g_bar[2];            // per prep group: its MMAs
+  uint64_t mma_bar[2];          // per tile chain
+  uint64_t fr_bar;              // frame-level MMAs (chain step)
   uint64_t q_full[2];
-  uint64_t tkt_bar[2];    // chain group -> prep group: the next frame's ticket is in ticket_ring
+  uint64_t o_bar[2];            // read-out MMA into O buffer b
+  uint64_t tkt_bar[2];          // chain group -> prep groups: next frame's ticket
   uint32_t tmem_base;
   int abort;
+  uint32_t loads;               // chunks whose k, v loads have been issued
   int ticket_ring[4];
-  __align__(16) float beta[2][64];
+  __align__(16) float beta[kSlots][64];
 };
 constexpr size_t kGdnSmemBytes = OFF_BAR + sizeof(Bars) + 1024;
+static_assert(kGdnSmemBytes <= 232448, "shared memory budget");
 
 // TMEM columns
-constexpr uint32_t TM_Y = 0;     // tile A [0,128), tile B [128,256)
-constexpr uint32_t TM_RU = 256;  // R^T: tile A [256,320), tile B [320,384); read-out O uses [256,384)
-constexpr uint32_t TM_G = 384;   // Gram matrix, 64 columns
+constexpr uint32_t TM_Y = 0;     // Y^T: tile A [0,128), tile B [128,256)
+constexpr uint32_t TM_R = 256;   // R^T: tile A [256,320), tile B [320,384); chain step: alpha S^T pairs
+                                 // [256,320); read-out: O buffers [256,320), [320,384)
+constexpr uint32_t TM_P = 384;   // prep group g: [384 + 64 g, 448 + 64 g): Gram matrix, then W^T
 
 __device__ __forceinline__ void named_bar(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
@@ -100,6 +108,74 @@ __device__ __forceinline__ void store_row16_f16(uint8_t *tile, uint32_t row, uin
   *reinterpret_cast<uint4 *>(tile + sw128_offset(row, col0 + 8)) = b;
 }
 
+// bf16 x 8 -> fp16 x 8 (one 16-byte chunk)
+__device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 u) {
+  const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+  uint32_t o[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 v2 = __bfloat1622float2(h[e]);
+    o[e] = pack_h2(v2.x, v2.y);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// ---------------------------------------------------------------- blocked inversion
+// The 64 x 64 unit lower triangular I + N is handled as 4 x 4 blocks of 16 x 16.
+// Shared-memory scratch (the slot's W area, 16 KB): blocks of 1 KB, fp32,
+// row r = 16 floats whose four float4 groups are permuted by q ^ ((r >> 1) & 3)
+// (eight consecutive rows of one group fall in distinct bank groups).
+//   lblk(i, j), i >= j (10 blocks): N's block (i, j); the diagonal ones are
+//              replaced by D_i = (I + N_ii)^-1, the others by E_ij = D_i N_ij;
+//   iblk(i, j), i > j (6 blocks): block (i, j) of (I + N)^-1.
+// With Linv_jj = D_j, block (i, j) of the inverse is -sum_{k=j}^{i-1} E_ik Linv_kj
+// (forward block substitution), computed by distance i - j = 1, 2, 3.
+__device__ __forceinline__ int bofs(int r, int q) { return r * 16 + ((q ^ ((r >> 1) & 3)) << 2); }
+__device__ __forceinline__ float *lblk(float *scr, int i, int j) { return scr + (i * (i + 1) / 2 + j) * 256; }
+__device__ __forceinline__ float *iblk(float *scr, int i, int j) {
+  const int d = i - j;
+  return scr + (10 + (d - 1) * (8 - d) / 2 + j) * 256;
+}
+__device__ __forceinline__ float4 ld_blk4(const float *b, int r, int q) {
+  return *reinterpret_cast<const float4 *>(b + bofs(r, q));
+}
+__device__ __forceinline__ void st_blk4(float *b, int r, int q, float4 v) {
+  *reinterpret_cast<float4 *>(b + bofs(r, q)) = v;
+}
+__device__ __forceinline__ void fma4(float4 &acc, float a, float4 b) {
+  acc.x = fmaf(a, b.x, acc.x);
+  acc.y = fmaf(a, b.y, acc.y);
+  acc.z = fmaf(a, b.z, acc.z);
+  acc.w = fmaf(a, b.w, acc.w);
+}
+// acc += (row r of A) x (columns 4q .. 4q+3 of B), 16 x 16 blocks.  The rows of
+// B are loaded eight at a time ahead of their FMAs, into two accumulators, so
+// that one thread keeps several shared-memory loads in flight.
+__device__ __forceinline__ void blk_row_mul(float4 &acc, const float *A, const float *B, int r, int q) {
+  float4 a4[4], b[8];
+#pragma unroll
+  for (int g = 0; g < 4; ++g) a4[g] = ld_blk4(A, r, g);
+  float4 acc1 = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+#pragma unroll
+    for (int s = 0; s < 8; ++s) b[s] = ld_blk4(B, 8 * h + s, q);
+#pragma unroll
+    for (int s = 0; s < 8; s += 4) {
+      const float4 a = a4[2 * h + s / 4];
+      fma4(acc, a.x, b[s]);
+      fma4(acc1, a.y, b[s + 1]);
+      fma4(acc, a.z, b[s + 2]);
+      fma4(acc1, a.w, b[s + 3]);
+    }
+  }
+  acc.x += acc1.x;
+  acc.y += acc1.y;
+  acc.z += acc1.z;
+  acc.w += acc1.w;
+}
+__device__ __forceinline__ float4 neg4(float4 v) { return make_float4(-v.x, -v.y, -v.z, -v.w); }
+
 __global__ void __launch_bounds__(kGThreads, 1)
     gdn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                   const __grid_constant__ CUtensorMap tmap_v, GdnParams p) {
@@ -113,39 +189,33 @@ __global__ void __launch_bounds__(kGThreads, 1)
   const long units = (long)BH * F;
   const long N = (long)F * L;
   const unsigned long long lim = p.spin_limit_ns;
-  const int nkd = dk / 16;          // k-steps over d_k
+  const int nkd = dk / 16;            // k-steps over d_k
   const int nch = (L + kC - 1) / kC;  // chunks per frame
+  volatile int *abort_flag = &bar.abort;
 
   // ---------------------------------------------------------------- set-up
   if (tid == 0) {
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kSlots; ++s) {
       mbar_init(&bar.kv_full[s], 1);
       mbar_init(&bar.khat_ready[s], 1);
       mbar_init(&bar.w_ready[s], 1);
       mbar_init(&bar.slot_free[s], 2);
-      mbar_init(&bar.q_full[s], 1);
-      mbar_init(&bar.mma_bar[s], 1);
     }
-    mbar_init(&bar.g_bar, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bar.g_bar[s], 1);
+      mbar_init(&bar.mma_bar[s], 1);
+      mbar_init(&bar.q_full[s], 1);
+      mbar_init(&bar.o_bar[s], 1);
+      mbar_init(&bar.tkt_bar[s], 1);
+    }
     mbar_init(&bar.fr_bar, 1);
-    mbar_init(&bar.tkt_bar[0], 1);
-    mbar_init(&bar.tkt_bar[1], 1);
     bar.abort = 0;
+    bar.loads = 0;
     mbar_fence_init();
     tma_prefetch_desc(&tmap_q);
     tma_prefetch_desc(&tmap_k);
     tma_prefetch_desc(&tmap_v);
   }
-  // identity (bf16, K-major 64 x 64) and zero pad slot of the khat ring
-  for (int e = tid; e < 64 * 64; e += kGThreads) {
-    const int r = e / 64, c = e % 64;
-    *reinterpret_cast<__nv_bfloat16 *>(sm + OFF_I + sw128_offset(r, c)) = __float2bfloat16(r == c ? 1.f : 0.f);
-  }
-  for (int e = tid; e < 2 * 8192 / 16; e += kGThreads) {
-    const int kb = e / 512, w = e % 512;
-    *reinterpret_cast<uint4 *>(sm + OFF_KHAT + kb * KHAT_KB_STRIDE + 2 * 8192 + w * 16) = make_uint4(0, 0, 0, 0);
-  }
-  fence_async_smem();
   if (warp == 0) {
     tmem_alloc(&bar.tmem_base, 512);
     tmem_relinquish();
@@ -155,429 +225,495 @@ __global__ void __launch_bounds__(kGThreads, 1)
   tc_fence_after();
   const uint32_t tmem = bar.tmem_base;
 
+  // Issue the k, v loads of chunk c of frame (f, bh), the g-th chunk of this
+  // CTA, into slot g % 3 once the slot's previous chunk is done with it.
+  // Called by one thread; false on a timeout.
+  auto issue_kv = [&](uint32_t gg, int f, int bh, int c) -> bool {
+    const int s = (int)(gg % kSlots);
+    if (!mbar_wait(&bar.slot_free[s], ((gg / kSlots) & 1u) ^ 1u, lim)) return false;
+    uint8_t *slot = sm + OFF_SLOT + s * SLOT_BYTES;
+    const int t0 = c * kC;
+    mbar_expect_tx(&bar.kv_full[s], 32768);
+    tma_load_4d(slot + SL_KHAT, &tmap_k, &bar.kv_full[s], 0, t0, f, bh);
+    tma_load_4d(slot + SL_KHAT + 8192, &tmap_k, &bar.kv_full[s], 64, t0, f, bh);
+    tma_load_4d(slot + SL_V, &tmap_v, &bar.kv_full[s], 0, t0, f, bh);
+    tma_load_4d(slot + SL_V + 8192, &tmap_v, &bar.kv_full[s], 64, t0, f, bh);
+    bar.loads = gg + 1;
+    return true;
+  };
+  // the first (up to) three chunks of the frame of ticket tk, the g0-th chunk on
+  auto issue_frame_kv = [&](int tk, uint32_t g0) -> bool {
+    if (tk < 0) return true;
+    for (int c = 0; c < nch && c < kSlots; ++c)
+      if (!issue_kv(g0 + c, tk / BH, tk % BH, c)) return false;
+    return true;
+  };
+
   if (warp >= 8) {
-    // ============================================================ prep group
-    regs_inc<232>();  // the back substitution keeps 64 values per thread live
-    const int pt = tid - kChain;  // 0..127
-    const int pbar = 2;           // named barrier of the prep group
-    const uint32_t tmG = tmem + TM_G;
+    // ============================================================ prep groups
+    regs_dec<120>();  // the block launches with 512 x 128; the chains take 2 x 128 x 136
+    const int grp = (warp - 8) >> 2;     // 0: even chunks, 1: odd chunks
+    const int pt = tid - kChain - 128 * grp;  // 0..127
+    const int pbar = 2 + grp;            // named barrier of the group
+    const uint32_t tmP = tmem + TM_P + 64 * grp;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    uint32_t g_phase = 0;
-    uint32_t g = 0;          // chunks processed so far (all frames)
-    float bnext = 0.f;       // gate input of token pt of the chunk whose loads are in flight
-    bool bvalid = false;     // token pt exists in that chunk
-    bool loaded = false;     // loads of chunk g already issued
+    uint8_t *tbuf = sm + OFF_T + grp * 8192;
+    uint32_t gph = 0;  // phase of g_bar[grp]
+    uint32_t g = 0;
     bool stop = false;
-    // Issue the TMA loads of chunk c of frame (f, bh) into slot gg & 1 once the
-    // chain group has released it, and prefetch its gates into bnext.
-    auto issue_loads = [&](uint32_t gg, int f, int bh, int c) -> int {
-      const int s = gg & 1;
-      int bad = 0;
-      if (pt == 0) {
-        if (!mbar_wait(&bar.slot_free[s], ((gg >> 1) & 1u) ^ 1u, lim)) {
-          bad = 1;
-        } else {
-          const int t0 = c * kC;
-          mbar_expect_tx(&bar.kv_full[s], 32768);
-          tma_load_4d(sm + OFF_KHAT + s * 8192, &tmap_k, &bar.kv_full[s], 0, t0, f, bh);
-          tma_load_4d(sm + OFF_KHAT + KHAT_KB_STRIDE + s * 8192, &tmap_k, &bar.kv_full[s], 64, t0, f, bh);
-          tma_load_4d(sm + OFF_V + s * 16384, &tmap_v, &bar.kv_full[s], 0, t0, f, bh);
-          tma_load_4d(sm + OFF_V + s * 16384 + 8192, &tmap_v, &bar.kv_full[s], 64, t0, f, bh);
-        }
-      }
-      if (pt < 64) {  // raw gate of the token; activated when stored (keeps the load latency off this path)
-        const int t = c * kC + pt;
-        bnext = t < L ? p.beta[(long)bh * N + (long)f * L + t] : 0.f;
-        bvalid = t < L;
-      }
-      return bad;
+    auto group_fail = [&](int timed_out) {
+      if (pt == 0 && timed_out && !*abort_flag) latch_status(p.status, GDN_ERR_TIMEOUT);
+      *abort_flag = 1;
+      stop = true;
     };
     for (int k = 0; !stop; ++k) {
-      // the chain group takes each frame's ticket and hands it over
       {
-        const int bad = (pt == 0) ? !mbar_wait(&bar.tkt_bar[k & 1], (k >> 1) & 1u, lim) : 0;
-        if (bar_sync_or(pbar, 128, bad || *((volatile int *)&bar.abort))) {
-          if (pt == 0 && bad) latch_status(p.status, GDN_ERR_TIMEOUT);
-          bar.abort = 1;
+        const int bad = pt == 0 ? !mbar_wait(&bar.tkt_bar[k & 1], (k >> 1) & 1u, lim) : 0;
+        if (bar_sync_or(pbar, 128, bad || *abort_flag)) {
+          group_fail(bad);
           break;
         }
       }
       const int tk = bar.ticket_ring[k & 3];
       if (tk < 0) break;
-      const int f = tk / BH;
-      const int bh = tk % BH;
       for (int c = 0; c < nch; ++c, ++g) {
-      const int s = g & 1;
-      const uint32_t ph = (g >> 1) & 1u;
-      int pbad = 0;
-      if (!loaded) pbad = issue_loads(g, f, bh, c);
-      if (pt < 64) bar.beta[s][pt] = bvalid ? (p.gates_are_logits ? gate_beta(bnext) : bnext) : 0.f;
-      if (bar_sync_or(pbar, 128, pbad || *((volatile int *)&bar.abort))) {
-        if (pt == 0 && pbad) latch_status(p.status, GDN_ERR_TIMEOUT);
-        bar.abort = 1;
-        stop = true;
-        break;
-      }
-      if (bar_sync_or(pbar, 128, pt == 0 ? !mbar_wait(&bar.kv_full[s], ph, lim) : 0)) {
-        if (pt == 0) latch_status(p.status, GDN_ERR_TIMEOUT);
-        bar.abort = 1;
-        stop = true;
-        break;
-      }
-      // 2. normalise keys in place: thread pt -> token pt/2, k-block pt%2
-      {
-        const int t = pt >> 1, kb = pt & 1;
-        uint8_t *row = sm + OFF_KHAT + kb * KHAT_KB_STRIDE + s * 8192;
-        float x[64];
-        float ss = 0.f;
-#pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-          const uint4 u = *reinterpret_cast<const uint4 *>(row + sw128_offset(t, ch * 8));
-          const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 v2 = __bfloat1622float2(h[e]);
-            x[ch * 8 + 2 * e] = v2.x;
-            x[ch * 8 + 2 * e + 1] = v2.y;
-            ss += v2.x * v2.x + v2.y * v2.y;
+        if ((int)(g & 1u) != grp) continue;
+        const int s = (int)(g % kSlots);
+        const uint32_t ph = (g / kSlots) & 1u;
+        uint8_t *slot = sm + OFF_SLOT + s * SLOT_BYTES;
+        // gate of token pt of the chunk (used from step 3 on, so its load latency is hidden)
+        float braw = 0.f;
+        const bool bvalid = pt < 64 && c * kC + pt < L;
+        if (bvalid) braw = p.beta[(long)(tk % BH) * N + (long)(tk / BH) * L + c * kC + pt];
+        {
+          const int bad = pt == 0 ? !mbar_wait(&bar.kv_full[s], ph, lim) : 0;
+          if (bar_sync_or(pbar, 128, bad || *abort_flag)) {
+            group_fail(bad);
+            break;
           }
         }
-        ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-        const float inv = 1.0f / fmaxf(sqrtf(ss), kKeyNormEps);
+        // 1. normalise keys in place (fp16), v to fp16 in place: thread -> token pt/2, block pt%2
+        {
+          const int t = pt >> 1, kb = pt & 1;
+          uint8_t *krow = slot + SL_KHAT + kb * 8192;
+          uint8_t *vrow = slot + SL_V + kb * 8192;
+          uint4 ku[8];
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-          const uint4 u = make_uint4(pack_h2(x[ch * 8] * inv, x[ch * 8 + 1] * inv),
-                                     pack_h2(x[ch * 8 + 2] * inv, x[ch * 8 + 3] * inv),
-                                     pack_h2(x[ch * 8 + 4] * inv, x[ch * 8 + 5] * inv),
-                                     pack_h2(x[ch * 8 + 6] * inv, x[ch * 8 + 7] * inv));
-          *reinterpret_cast<uint4 *>(row + sw128_offset(t, ch * 8)) = u;
-        }
-      }
-      fence_async_smem();
-      tc_fence_before();
-      named_bar(pbar, 128);
-      // 3. khat ready; Gram matrix G = Khat Khat^T (rows: this chunk and the next slot)
-      if (pt == 0) {
-        mbar_arrive_only(&bar.khat_ready[s]);
-        tc_fence_after();
-        const uint32_t idg = idesc_f16(128, 64, 0, 0, 0);
-        for (int kk = 0; kk < nkd; ++kk) {
-          const uint32_t a = smem_u32(sm + OFF_KHAT + (kk >> 2) * KHAT_KB_STRIDE + s * 8192 + (kk & 3) * 32);
-          mma_f16_ss(tmG, sdesc_sw128(a, 16, 1024), sdesc_sw128(a, 16, 1024), idg, kk > 0 ? 1u : 0u);
-        }
-        mma_commit(&bar.g_bar);
-      }
-      // prefetch the next chunk of this frame while the Gram matrix is computed
-      loaded = c + 1 < nch;
-      const int nbad = loaded ? issue_loads(g + 1, f, bh, c + 1) : 0;
-      const int gbad = pt == 0 ? !mbar_wait(&bar.g_bar, g_phase, lim) : 0;
-      g_phase ^= 1u;
-      if (bar_sync_or(pbar, 128, gbad || nbad)) {
-        if (pt == 0) latch_status(p.status, GDN_ERR_TIMEOUT);
-        bar.abort = 1;
-        stop = true;
-        break;
-      }
-      tc_fence_after();
-      // 4. Nt[t][u] = N[u][t] = beta_u G[u][t] for u > t.  G is symmetric, so lane
-      //    t (the group's first two warps) reads row t of G and writes row t of Nt (fp32, float4
-      //    index XOR (t & 15)); Nt occupies the W slot until step 5.
-      float *Nt = reinterpret_cast<float *>(sm + OFF_W + s * 16384);
-      if (pt < 64) {  // the group's first two warps hold TMEM lanes 0..63
-        const int t = pt;  // lane
-        float r[4][16];
+          for (int ch = 0; ch < 8; ++ch) ku[ch] = *reinterpret_cast<const uint4 *>(krow + sw128_offset(t, ch * 8));
+          float ssp[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int cb = 0; cb < 4; ++cb) tmem_ld16(tmG + lane_off + cb * 16, r[cb]);
-        tmem_ld_wait();
-#pragma unroll
-        for (int cb = 0; cb < 4; ++cb)
-#pragma unroll
-          for (int e = 0; e < 16; e += 4) {
-            const int u = cb * 16 + e;
-            const float4 b4 = *reinterpret_cast<const float4 *>(&bar.beta[s][u]);
-            float4 o4;
-            o4.x = (u + 0 > t) ? b4.x * r[cb][e + 0] : 0.f;
-            o4.y = (u + 1 > t) ? b4.y * r[cb][e + 1] : 0.f;
-            o4.z = (u + 2 > t) ? b4.z * r[cb][e + 2] : 0.f;
-            o4.w = (u + 3 > t) ? b4.w * r[cb][e + 3] : 0.f;
-            *reinterpret_cast<float4 *>(Nt + t * 64 + (((u >> 2) ^ (t & 15)) << 2)) = o4;
-          }
-        if (t < 32) {
-          // B operand of the cross-term MMA: row t holds N[32 + u][t] = beta_{32+u} G[t][32+u]
-#pragma unroll
-          for (int ch = 0; ch < 4; ++ch) {
-            uint32_t h4[4];
+          for (int ch = 0; ch < 8; ++ch) {
+            const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&ku[ch]);
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const int u = 32 + ch * 8 + 2 * e;
-              h4[e] = pack_h2(bar.beta[s][u] * r[u >> 4][u & 15], bar.beta[s][u + 1] * r[(u + 1) >> 4][(u + 1) & 15]);
-            }
-            *reinterpret_cast<uint4 *>(sm + OFF_NHL + sw128_offset(t, ch * 8)) = make_uint4(h4[0], h4[1], h4[2], h4[3]);
-          }
-        }
-      }
-      tc_fence_before();
-      named_bar(pbar, 128);
-      // 5. W = diag(beta) Z with (I + N^T) Z = Khat: thread i < d_k owns column i
-      //    of Z and back-substitutes from the last token,
-      //        z[t] = khat[t][i] - sum_{u > t} N[u][t] z[u],
-      //    in two halves: rows 63..32 on CUDA cores; the hi -> lo coupling
-      //    sum_{u >= 32} N[u][t] z[u] for t < 32 as one tcgen05 MMA (z_hi^T in
-      //    TMEM as A, the fp16 N block as B); then rows 31..0.
-      float z[64];
-      const bool solver = pt < dk;
-      if (solver) {
-        const int i = pt;
-        const uint8_t *kt = sm + OFF_KHAT + (i >> 6) * KHAT_KB_STRIDE + s * 8192;
-#pragma unroll
-        for (int t = 0; t < 64; ++t) z[t] = __half2float(*reinterpret_cast<const __half *>(kt + sw128_offset(t, i & 63)));
-      }
-      // rows in blocks of four: the four rows' sums over already final z[u] are
-      // independent (two partial sums each), then the 4 x 4 triangle in order
-      auto solve_rows = [&](int hi_block, int u_end) {
-#pragma unroll
-        for (int tb = 60; tb >= 0; tb -= 4) {
-          if ((tb >= 32) != (hi_block != 0)) continue;
-          float a[4][2];
-#pragma unroll
-          for (int r = 0; r < 4; ++r) {
-            a[r][0] = z[tb + r];
-            a[r][1] = 0.f;
-          }
-#pragma unroll
-          for (int u4 = tb + 4; u4 < 64; u4 += 4) {
-            if (u4 >= u_end) continue;
-#pragma unroll
-            for (int r = 0; r < 4; ++r) {
-              const int t = tb + r;
-              const float4 n4 = *reinterpret_cast<const float4 *>(Nt + t * 64 + (((u4 >> 2) ^ (t & 15)) << 2));
-              a[r][0] = fmaf(-n4.x, z[u4 + 0], a[r][0]);
-              a[r][1] = fmaf(-n4.y, z[u4 + 1], a[r][1]);
-              a[r][0] = fmaf(-n4.z, z[u4 + 2], a[r][0]);
-              a[r][1] = fmaf(-n4.w, z[u4 + 3], a[r][1]);
+              const float2 v2 = __bfloat1622float2(h[e]);
+              ssp[e] = fmaf(v2.x, v2.x, fmaf(v2.y, v2.y, ssp[e]));
             }
           }
+          float ss = (ssp[0] + ssp[1]) + (ssp[2] + ssp[3]);
+          ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+          const float inv = 1.0f / fmaxf(sqrtf(ss), kKeyNormEps);
 #pragma unroll
-          for (int r = 3; r >= 0; --r) {
-            const int t = tb + r;
-            const float4 n4 = *reinterpret_cast<const float4 *>(Nt + t * 64 + (((tb >> 2) ^ (t & 15)) << 2));
-            float v = a[r][0] + a[r][1];
-            if (r < 3) v = fmaf(-n4.w, z[tb + 3], v);
-            if (r < 2) v = fmaf(-n4.z, z[tb + 2], v);
-            if (r < 1) v = fmaf(-n4.y, z[tb + 1], v);
-            z[t] = v;
+          for (int ch = 0; ch < 8; ++ch) {
+            const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&ku[ch]);
+            uint32_t o[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 v2 = __bfloat1622float2(h[e]);
+              o[e] = pack_h2(v2.x * inv, v2.y * inv);
+            }
+            *reinterpret_cast<uint4 *>(krow + sw128_offset(t, ch * 8)) = make_uint4(o[0], o[1], o[2], o[3]);
+          }
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch) ku[ch] = *reinterpret_cast<const uint4 *>(vrow + sw128_offset(t, ch * 8));
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch)
+            *reinterpret_cast<uint4 *>(vrow + sw128_offset(t, ch * 8)) = bf16x8_to_f16x8(ku[ch]);
+        }
+        fence_async_smem();
+        tc_fence_before();
+        named_bar(pbar, 128);
+        // 2. khat ready for the chains; Gram matrix G = Khat Khat^T (lanes 0..63 = tokens)
+        if (pt == 0) {
+          mbar_arrive_only(&bar.khat_ready[s]);
+          tc_fence_after();
+          const uint32_t idg = idesc_f16(128, 64, 0, 0, 0);
+          for (int kk = 0; kk < nkd; ++kk) {
+            const uint32_t a = smem_u32(slot + SL_KHAT + (kk >> 2) * 8192 + (kk & 3) * 32);
+            mma_f16_ss(tmP, sdesc_sw128(a, 16, 1024), sdesc_sw128(a, 16, 1024), idg, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(&bar.g_bar[grp]);
+        }
+        {
+          const int bad = pt == 0 ? !mbar_wait(&bar.g_bar[grp], gph, lim) : 0;
+          gph ^= 1u;
+          if (bar_sync_or(pbar, 128, bad)) {
+            group_fail(bad);
+            break;
           }
         }
-      };
-      if (solver) solve_rows(1, 64);
-      {
-        // z_hi^T as the MMA's A operand: lane i, 16 columns of packed fp16 (zeros past d_k)
-        uint32_t hz[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) hz[e] = solver ? pack_h2(z[32 + 2 * e], z[33 + 2 * e]) : 0u;
-        tmem_st16u(tmG + lane_off, hz);
-        tmem_st_wait();
-      }
-      tc_fence_before();
-      named_bar(pbar, 128);
-      if (pt == 0) {
         tc_fence_after();
-        const uint32_t idc = idesc_f16(128, 32, 0, 0, 0);
-        const uint32_t nb = smem_u32(sm + OFF_NHL);
-        for (int kk = 0; kk < 2; ++kk)
-          mma_f16_ts(tmG + 32, tmG + kk * 8, sdesc_sw128(nb + kk * 32, 16, 1024), idc, kk > 0 ? 1u : 0u);
-        mma_commit(&bar.g_bar);
-      }
-      {
-        const int cbad = pt == 0 ? !mbar_wait(&bar.g_bar, g_phase, lim) : 0;
-        g_phase ^= 1u;
-        if (bar_sync_or(pbar, 128, cbad)) {
-          if (pt == 0) latch_status(p.status, GDN_ERR_TIMEOUT);
-          bar.abort = 1;
-          stop = true;
-          break;
-        }
-      }
-      tc_fence_after();
-      {
-        float cr[2][16];
-        tmem_ld16(tmG + 32 + lane_off, cr[0]);
-        tmem_ld16(tmG + 48 + lane_off, cr[1]);
-        tmem_ld_wait();
-        if (solver) {
+        float *scr = reinterpret_cast<float *>(slot + SL_W);
+        const float *bet = bar.beta[s];
+        // 3. N's blocks: row t of N = beta_t G[t][u] for u < t (warps 0-1 hold TMEM lanes 0..63)
+        if (pt < 64) {
+          const int t = pt;
+          const float bt = bvalid ? (p.gates_are_logits ? gate_beta(braw) : braw) : 0.f;
+          bar.beta[s][t] = bt;
+          const int ib = t >> 4, r = t & 15;
+          float gr[4][16];
 #pragma unroll
-          for (int t = 0; t < 32; ++t) z[t] -= cr[t >> 4][t & 15];
-          solve_rows(0, 32);
-        }
-      }
-      named_bar(pbar, 128);  // every read of N is done before W overwrites it
-      if (solver) {
-        // row i of the K-major B operand W^T-as-(K = token, N = i): W[t][i] = beta_t z[t]
-        uint8_t *wrow = sm + OFF_W + s * 16384;
+          for (int jb = 0; jb < 4; ++jb) tmem_ld16(tmP + lane_off + jb * 16, gr[jb]);
+          tmem_ld_wait();
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-          uint32_t w4[4];
+          for (int jb = 0; jb < 4; ++jb) {
+            if (jb > ib) continue;
+            float *dst = lblk(scr, ib, jb);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int t = ch * 8 + 2 * e;
-            w4[e] = pack_h2(bar.beta[s][t] * z[t], bar.beta[s][t + 1] * z[t + 1]);
+            for (int q = 0; q < 4; ++q) {
+              const int u = jb * 16 + q * 4;
+              float4 v;
+              v.x = (u + 0 < t) ? bt * gr[jb][q * 4 + 0] : 0.f;
+              v.y = (u + 1 < t) ? bt * gr[jb][q * 4 + 1] : 0.f;
+              v.z = (u + 2 < t) ? bt * gr[jb][q * 4 + 2] : 0.f;
+              v.w = (u + 3 < t) ? bt * gr[jb][q * 4 + 3] : 0.f;
+              st_blk4(dst, r, q, v);
+            }
           }
-          *reinterpret_cast<uint4 *>(wrow + sw128_offset(pt, ch * 8)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
         }
-      }
-      fence_async_smem();
-      named_bar(pbar, 128);
-      if (pt == 0) mbar_arrive_only(&bar.w_ready[s]);
+        tc_fence_before();
+        named_bar(pbar, 128);
+        // 4. D_k = (I + N_kk)^-1: thread (k, c) solves column c by forward substitution
+        if (pt < 64) {
+          const int kq = pt >> 4, c = pt & 15;
+          float *Dk = lblk(scr, kq, kq);
+          float x[16];
+#pragma unroll
+          for (int r = 0; r < 16; ++r) x[r] = (r == c) ? 1.f : 0.f;
+          float4 cur[4], nxt[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) cur[q] = ld_blk4(Dk, 1, q);
+#pragma unroll
+          for (int r = 1; r < 16; ++r) {
+            if (r + 1 < 16) {  // the next row's loads do not depend on x
+#pragma unroll
+              for (int q = 0; q < 4; ++q)
+                if (4 * q < r + 1) nxt[q] = ld_blk4(Dk, r + 1, q);
+            }
+            float a[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              if (4 * q < r) a[0] = fmaf(cur[q].x, x[4 * q], a[0]);
+              if (4 * q + 1 < r) a[1] = fmaf(cur[q].y, x[4 * q + 1], a[1]);
+              if (4 * q + 2 < r) a[2] = fmaf(cur[q].z, x[4 * q + 2], a[2]);
+              if (4 * q + 3 < r) a[3] = fmaf(cur[q].w, x[4 * q + 3], a[3]);
+            }
+            x[r] = (r > c) ? -((a[0] + a[1]) + (a[2] + a[3])) : x[r];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) cur[q] = nxt[q];
+          }
+          __syncwarp();  // the block's 16 threads share this warp: all reads of N_kk are done
+#pragma unroll
+          for (int r = 0; r < 16; ++r) Dk[bofs(r, c >> 2) + (c & 3)] = x[r];
+        }
+        named_bar(pbar, 128);
+        // 5. E_ik = D_i N_ik for the six blocks below the diagonal (in place)
+        {
+          float4 acc[3];
+          int ei[3], ek[3], er[3], eq[3];
+#pragma unroll
+          for (int ps = 0; ps < 3; ++ps) {
+            const int it = pt + 128 * ps;
+            const int e = it >> 6, rem = it & 63;
+            eq[ps] = rem >> 4;
+            er[ps] = rem & 15;
+            ei[ps] = e < 3 ? e + 1 : (e < 5 ? e - 1 : 3);
+            ek[ps] = e < 3 ? e : (e < 5 ? e - 3 : 0);
+            acc[ps] = make_float4(0.f, 0.f, 0.f, 0.f);
+            blk_row_mul(acc[ps], lblk(scr, ei[ps], ei[ps]), lblk(scr, ei[ps], ek[ps]), er[ps], eq[ps]);
+          }
+          named_bar(pbar, 128);
+#pragma unroll
+          for (int ps = 0; ps < 3; ++ps) st_blk4(lblk(scr, ei[ps], ek[ps]), er[ps], eq[ps], acc[ps]);
+        }
+        named_bar(pbar, 128);
+        // 6. distance 1: Linv_{k+1,k} = -E_{k+1,k} D_k
+#pragma unroll
+        for (int ps = 0; ps < 2; ++ps) {
+          const int it = pt + 128 * ps;
+          if (it < 192) {
+            const int e = it >> 6, rem = it & 63, q = rem >> 4, r = rem & 15;
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            blk_row_mul(acc, lblk(scr, e + 1, e), lblk(scr, e, e), r, q);
+            st_blk4(iblk(scr, e + 1, e), r, q, neg4(acc));
+          }
+        }
+        named_bar(pbar, 128);
+        // 7. distance 2: Linv_{k+2,k} = -(E_{k+2,k} D_k + E_{k+2,k+1} Linv_{k+1,k})
+        {
+          const int e = pt >> 6, rem = pt & 63, q = rem >> 4, r = rem & 15;
+          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+          blk_row_mul(acc, lblk(scr, e + 2, e), lblk(scr, e, e), r, q);
+          blk_row_mul(acc, lblk(scr, e + 2, e + 1), iblk(scr, e + 1, e), r, q);
+          st_blk4(iblk(scr, e + 2, e), r, q, neg4(acc));
+        }
+        named_bar(pbar, 128);
+        // 8. distance 3: Linv_30 = -(E_30 D_0 + E_31 Linv_10 + E_32 Linv_20)
+        if (pt < 64) {
+          const int q = pt >> 4, r = pt & 15;
+          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+          blk_row_mul(acc, lblk(scr, 3, 0), lblk(scr, 0, 0), r, q);
+          blk_row_mul(acc, lblk(scr, 3, 1), iblk(scr, 1, 0), r, q);
+          blk_row_mul(acc, lblk(scr, 3, 2), iblk(scr, 2, 0), r, q);
+          st_blk4(iblk(scr, 3, 0), r, q, neg4(acc));
+        }
+        named_bar(pbar, 128);
+        // 9. T[u][t] = Linv[u][t] beta_t as fp16, rows u (MN-major B operand: N = t, K = u)
+        {
+          const int u = pt >> 1, half = pt & 1;
+          const int ub = u >> 4, r = u & 15;
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const int tb = half * 2 + h2;
+            float v[16];
+            if (tb > ub) {
+#pragma unroll
+              for (int e = 0; e < 16; ++e) v[e] = 0.f;
+            } else {
+              const float *src = tb == ub ? lblk(scr, ub, ub) : iblk(scr, ub, tb);
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const float4 t4 = ld_blk4(src, r, q);
+                const float4 b4 = *reinterpret_cast<const float4 *>(bet + tb * 16 + q * 4);
+                v[4 * q] = t4.x * b4.x;
+                v[4 * q + 1] = t4.y * b4.y;
+                v[4 * q + 2] = t4.z * b4.z;
+                v[4 * q + 3] = t4.w * b4.w;
+              }
+            }
+            store_row16_f16(tbuf, u, tb * 16, v);
+          }
+        }
+        fence_async_smem();
+        named_bar(pbar, 128);
+        // 10. W^T = Khat^T T (lanes i, columns t): A = khat read MN-major, B = T MN-major
+        if (pt == 0) {
+          tc_fence_after();
+          const uint32_t kb0 = smem_u32(slot + SL_KHAT), tb0 = smem_u32(tbuf);
+          const uint32_t idw = idesc_f16(128, 64, 0, 1, 1);
+          for (int kk = 0; kk < 4; ++kk)
+            mma_f16_ss(tmP, sdesc_sw128(kb0 + kk * 2048, 8192, 1024), sdesc_sw128(tb0 + kk * 2048, 8192, 1024), idw,
+                       kk > 0 ? 1u : 0u);
+          mma_commit(&bar.g_bar[grp]);
+        }
+        {
+          const int bad = pt == 0 ? !mbar_wait(&bar.g_bar[grp], gph, lim) : 0;
+          gph ^= 1u;
+          if (bar_sync_or(pbar, 128, bad)) {
+            group_fail(bad);
+            break;
+          }
+        }
+        tc_fence_after();
+        // 11. row i of the K-major B operand W (N = i, K = t); the scratch blocks are dead
+        {
+#pragma unroll
+          for (int hb = 0; hb < 2; ++hb) {
+            float r[2][16];
+            tmem_ld16(tmP + lane_off + hb * 32, r[0]);
+            tmem_ld16(tmP + lane_off + hb * 32 + 16, r[1]);
+            tmem_ld_wait();
+            if (pt < dk) {
+              store_row16_f16(slot + SL_W, pt, hb * 32, r[0]);
+              store_row16_f16(slot + SL_W, pt, hb * 32 + 16, r[1]);
+            }
+          }
+        }
+        fence_async_smem();
+        tc_fence_before();
+        named_bar(pbar, 128);
+        if (pt == 0) mbar_arrive_only(&bar.w_ready[s]);
       }
     }
   } else {
-    // ============================================================ chain group
-    regs_dec<128>();
+    // ============================================================ tile chains
+    regs_inc<136>();
     const int tile = warp >> 2;           // 0: tile A (rows of A^T), 1: tile B (rows of B^T)
     const int row = tid & 127;            // TMEM lane / operand row within the tile
     const bool issuer = row == 0;         // threads 0 and 128 issue their tile's MMAs
-    const int tbar = 3 + tile;            // named barrier of one tile chain (128 threads)
+    const int tbar = 4 + tile;            // named barrier of one tile chain (128 threads)
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t tmY = tmem + TM_Y + tile * 128;
+    const uint32_t tmR = tmem + TM_R + tile * 64;
+    uint8_t *mir = sm + OFF_MIRROR + tile * 32768;
     uint32_t tphase = 0;                  // phase of mma_bar[tile]
     uint32_t fphase = 0;                  // phase of fr_bar
-    uint32_t qcount[2] = {0, 0};
+    // read-out tiles over the CTA's lifetime: q loads issued / waited for, MMAs
+    // issued / waited for; tile n uses q buffer n & 1 and O buffer n & 1
+    uint32_t qi = 0, qw = 0, oi = 0, ow = 0;
     int frames = 0;
     bool failed = false;
     uint32_t g = 0;
-    const uint32_t id_vi = idesc_f16(128, 64, 1, 1, 0);          // V^T (MN) x I (K), bf16
-    const uint32_t id_r = idesc_f16(128, 64, 0, 0, 0, 1, 0);     // -(Y^T) x Khat^T, fp16
-    const uint32_t id_y = idesc_f16(128, dk, 0, 0, 0);           // R^T x W (both K-major)
-    const uint32_t id_s = idesc_f16(128, dk, 0, 0, 1);           // (alpha S^T) x A^T (MN)
-    const uint32_t id_o = idesc_f16(128, 128, 0, 0, 0);          // S^T x Q^T (128 tokens)
+    const uint32_t id_r = idesc_f16(128, 64, 0, 0, 0, 1, 0);   // -(Y^T) x Khat^T
+    const uint32_t id_y = idesc_f16(128, dk, 0, 0, 0);          // R^T (TMEM) x W
+    const uint32_t id_vw = idesc_f16(128, dk, 0, 1, 0);         // V^T (MN) x W
+    const uint32_t id_kw = idesc_f16(128, dk, 0, 1, 0, 1, 0);   // -(Khat^T) (MN) x W
+    const uint32_t id_s = idesc_f16(128, dk, 0, 0, 1);          // (alpha S^T, TMEM) x A^T (MN)
+    const uint32_t id_o = idesc_f16(128, kQTok, 0, 0, 0);       // S^T x Q^T
 
     // Wait for this tile's MMAs: the issuing thread polls the mbarrier, the
     // others wait on the named barrier (which takes no issue slots from the
     // warps doing work).  False, for all 128 threads of the tile, on a
-    // timeout, on `extra` from any of them, or once the prep group gave up.
+    // timeout, on `extra` from any of them, or once another role gave up.
     auto tile_wait = [&](int extra) -> bool {
       int bad = extra;
       if (issuer) bad |= !mbar_wait(&bar.mma_bar[tile], tphase, lim);
       tphase ^= 1u;
-      return !bar_sync_or(tbar, 128, bad || *((volatile int *)&bar.abort));
+      return !bar_sync_or(tbar, 128, bad || *abort_flag);
     };
-    // the same for frame-level MMAs, over all 256 chain threads
-    auto frame_wait = [&](int extra) -> bool {
-      int bad = extra;
-      if (tid == 0) bad |= !mbar_wait(&bar.fr_bar, fphase, lim);
-      fphase ^= 1u;
-      return !bar_sync_or(1, kChain, bad || *((volatile int *)&bar.abort));
+    // the same for one thread's mbarrier over all 256 chain threads
+    auto group_wait = [&](uint64_t *b, uint32_t parity) -> bool {
+      int bad = 0;
+      if (tid == 0) bad = !mbar_wait(b, parity, lim);
+      return !bar_sync_or(1, kChain, bad || *abort_flag);
+    };
+    auto issue_q = [&](int f, int bh, int t0) {  // thread 0
+      const int bq = qi & 1;
+      mbar_expect_tx(&bar.q_full[bq], 16384);
+      uint8_t *qb = sm + OFF_QB + bq * 16384;
+      tma_load_4d(qb, &tmap_q, &bar.q_full[bq], 0, t0, f, bh);
+      tma_load_4d(qb + 8192, &tmap_q, &bar.q_full[bq], 64, t0, f, bh);
+      ++qi;
     };
 
     // The chain group takes the tickets: the first here, each next one right
     // after the current frame's state is published (before its read-out), and
-    // hands each to the prep group.  A ticket is thus started a fixed read-out
-    // time after it is taken, whatever the frame chain's waits were.
+    // hands each to the loader and the prep groups.  A ticket is thus started a
+    // fixed read-out time after it is taken, whatever the frame chain's waits were.
     if (tid == 0) {
       const long t = atomicAdd(p.ws.counter, 1);
-      bar.ticket_ring[0] = (int)(t < units ? t : -1);
+      const int tk0 = (int)(t < units ? t : -1);
+      bar.ticket_ring[0] = tk0;
       mbar_arrive_only(&bar.tkt_bar[0]);
+      if (!issue_frame_kv(tk0, 0)) failed = true;
     }
-    named_bar(1, kChain);
-    for (;;) {
+    if (bar_sync_or(1, kChain, failed ? 1 : 0)) failed = true;
+    for (; !failed;) {
       const int tk = bar.ticket_ring[frames & 3];
       ++frames;
       if (tk < 0) break;
-      {
-        const int s = g & 1;
-        const uint32_t ph = (g >> 1) & 1u;
-        const int kbad = tid == 0 ? !mbar_wait(&bar.khat_ready[s], ph, lim) : 0;
-        if (bar_sync_or(1, kChain, kbad)) {
-          failed = true;
-          break;
-        }
-      }
       const long ticket = tk;
       const int f = (int)(ticket / BH);
       const int bh = (int)(ticket % BH);
 
-      // Y = [I | 0] in TMEM (fp32) and in the fp16 mirror, rows of this tile
-      {
-        const int rdim = tile == 0 ? dk : dv;
+      // Y_A^T = I in TMEM (the first chunk accumulates onto it); Y_B^T starts
+      // from the first chunk's product
+      if (tile == 0) {
 #pragma unroll 1
         for (int cb = 0; cb < nkd; ++cb) {
           float r[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) r[e] = (tile == 0 && cb * 16 + e == row && row < rdim) ? 1.f : 0.f;
-          tmem_st16(tmem + TM_Y + tile * 128 + lane_off + cb * 16, r);
-          store_row16_f16(sm + OFF_MIRROR + tile * 32768 + (cb >> 2) * 16384, row, (cb & 3) * 16, r);
+          for (int e = 0; e < 16; ++e) r[e] = (cb * 16 + e == row) ? 1.f : 0.f;
+          tmem_st16(tmY + lane_off + cb * 16, r);
         }
         tmem_st_wait();
       }
-      fence_async_smem();
       tc_fence_before();
       named_bar(tbar, 128);
 
       // ---- the frame's chunks, one independent chain per tile
       for (int c = 0; c < nch; ++c, ++g) {
-        const int s = g & 1;
-        const uint32_t ph = (g >> 1) & 1u;
+        const int s = (int)(g % kSlots);
+        const uint32_t ph = (g / kSlots) & 1u;
+        uint8_t *slot = sm + OFF_SLOT + s * SLOT_BYTES;
         int cbad = 0;
-        // R^T = [0 ; V^T] - Y^T Khat^T  (the V^T part for tile B only)
-        if (issuer) {
-          if (c > 0 && !mbar_wait(&bar.khat_ready[s], ph, lim)) cbad = 1;
-          tc_fence_after();
-          const uint32_t kh = smem_u32(sm + OFF_KHAT + s * 8192);
-          const uint32_t mb = smem_u32(sm + OFF_MIRROR + tile * 32768);
-          const uint32_t dR = tmem + TM_RU + tile * 64;
-          if (tile == 1) {
-            const uint32_t vb = smem_u32(sm + OFF_V + s * 16384);
-            const uint32_t ib = smem_u32(sm + OFF_I);
-            for (int kk = 0; kk < 4; ++kk)
-              mma_f16_ss(dR, sdesc_sw128(vb + kk * 2048, 8192, 1024), sdesc_sw128(ib + kk * 32, 16, 1024), id_vi,
+        if (c > 0) {
+          // R^T = -Y^T Khat^T (the [0 ; V^T] target enters with the W product)
+          if (issuer) {
+            if (!mbar_wait(&bar.khat_ready[s], ph, lim)) cbad = 1;
+            tc_fence_after();
+            const uint32_t kh = smem_u32(slot + SL_KHAT);
+            const uint32_t mb = smem_u32(mir);
+            for (int kk = 0; kk < nkd; ++kk) {
+              const uint32_t ko = (kk >> 2) * 16384 + (kk & 3) * 32;
+              const uint32_t kho = (kk >> 2) * 8192 + (kk & 3) * 32;
+              mma_f16_ss(tmR, sdesc_sw128(mb + ko, 16, 1024), sdesc_sw128(kh + kho, 16, 1024), id_r,
                          kk > 0 ? 1u : 0u);
+            }
+            mma_commit(&bar.mma_bar[tile]);
           }
-          for (int kk = 0; kk < nkd; ++kk) {
-            const uint32_t ko = (kk >> 2) * 16384 + (kk & 3) * 32;
-            const uint32_t kho = (kk >> 2) * KHAT_KB_STRIDE + (kk & 3) * 32;
-            mma_f16_ss(dR, sdesc_sw128(mb + ko, 16, 1024), sdesc_sw128(kh + kho, 16, 1024), id_r,
-                       (tile == 1 || kk > 0) ? 1u : 0u);
+          if (!tile_wait(cbad)) {
+            failed = true;
+            break;
           }
-          mma_commit(&bar.mma_bar[tile]);
-        }
-        if (!tile_wait(cbad)) { failed = true; break; }
-        tc_fence_after();
-        {
-          float r[4][16];
+          tc_fence_after();
+          {
+            // row of R^T -> fp16 pairs in the first 32 columns (A operand of the next MMA)
+            float r[4][16];
 #pragma unroll
-          for (int cb = 0; cb < 4; ++cb) tmem_ld16(tmem + TM_RU + tile * 64 + lane_off + cb * 16, r[cb]);
-          tmem_ld_wait();
+            for (int cb = 0; cb < 4; ++cb) tmem_ld16(tmR + lane_off + cb * 16, r[cb]);
+            tmem_ld_wait();
 #pragma unroll
-          for (int cb = 0; cb < 4; ++cb) store_row16_f16(sm + OFF_RU + tile * 16384, row, cb * 16, r[cb]);
+            for (int hp = 0; hp < 2; ++hp) {
+              uint32_t h[16];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                h[e] = pack_h2(r[2 * hp][2 * e], r[2 * hp][2 * e + 1]);
+                h[8 + e] = pack_h2(r[2 * hp + 1][2 * e], r[2 * hp + 1][2 * e + 1]);
+              }
+              tmem_st16u(tmR + lane_off + hp * 16, h);
+            }
+            tmem_st_wait();
+          }
+          tc_fence_before();
+          named_bar(tbar, 128);
         }
-        fence_async_smem();
-        tc_fence_before();
-        named_bar(tbar, 128);
-        // Y^T += R^T W ; the last MMA of this tile on slot s releases it
+        // Y^T += R^T W  (tile B also + V^T W); the last MMA of this tile on slot s releases it
         if (issuer) {
           if (!mbar_wait(&bar.w_ready[s], ph, lim)) cbad = 1;
           tc_fence_after();
-          const uint32_t rb = smem_u32(sm + OFF_RU + tile * 16384);
-          const uint32_t wb = smem_u32(sm + OFF_W + s * 16384);
-          for (int kk = 0; kk < 4; ++kk)
-            mma_f16_ss(tmem + TM_Y + tile * 128, sdesc_sw128(rb + kk * 32, 16, 1024),
-                       sdesc_sw128(wb + kk * 32, 16, 1024), id_y, 1u);
+          const uint32_t wb = smem_u32(slot + SL_W);
+          if (c > 0) {
+            for (int kk = 0; kk < 4; ++kk)
+              mma_f16_ts(tmY, tmR + kk * 8, sdesc_sw128(wb + kk * 32, 16, 1024), id_y, 1u);
+          } else if (tile == 0) {
+            const uint32_t kb = smem_u32(slot + SL_KHAT);
+            for (int kk = 0; kk < 4; ++kk)
+              mma_f16_ss(tmY, sdesc_sw128(kb + kk * 2048, 8192, 1024), sdesc_sw128(wb + kk * 32, 16, 1024), id_kw,
+                         1u);
+          }
+          if (tile == 1) {
+            const uint32_t vb = smem_u32(slot + SL_V);
+            for (int kk = 0; kk < 4; ++kk)
+              mma_f16_ss(tmY, sdesc_sw128(vb + kk * 2048, 8192, 1024), sdesc_sw128(wb + kk * 32, 16, 1024), id_vw,
+                         (c > 0 || kk > 0) ? 1u : 0u);
+          }
           mma_commit(&bar.mma_bar[tile]);
           mma_commit(&bar.slot_free[s]);
         }
-        if (!tile_wait(cbad)) { failed = true; break; }
+        if (!tile_wait(cbad)) {
+          failed = true;
+          break;
+        }
         tc_fence_after();
+        // slot s is free once both tiles' last MMAs on it are done: chunk c + 3 goes there
+        if (tile == 1 && issuer && c + kSlots < nch && !issue_kv(g + kSlots, f, bh, c + kSlots)) {
+          *abort_flag = 1;
+          latch_status(p.status, GDN_ERR_TIMEOUT);
+        }
         // Y^T rows -> fp16 mirror (tile B's rows are not needed after the last chunk)
         if (c + 1 < nch || tile == 0) {
+#pragma unroll
 #pragma unroll
           for (int hb = 0; hb < 2; ++hb) {  // two batches of up to 4 column blocks
             float r[4][16];
 #pragma unroll
             for (int e = 0; e < 4; ++e)
-              if (hb * 4 + e < nkd) tmem_ld16(tmem + TM_Y + tile * 128 + lane_off + (hb * 4 + e) * 16, r[e]);
+              if (hb * 4 + e < nkd) tmem_ld16(tmY + lane_off + (hb * 4 + e) * 16, r[e]);
             tmem_ld_wait();
 #pragma unroll
             for (int e = 0; e < 4; ++e)
-              if (hb * 4 + e < nkd) store_row16_f16(sm + OFF_MIRROR + tile * 32768 + hb * 16384, row, e * 16, r[e]);
+              if (hb * 4 + e < nkd) store_row16_f16(mir + hb * 16384, row, e * 16, r[e]);
           }
         }
         fence_async_smem();
@@ -590,62 +726,68 @@ __global__ void __launch_bounds__(kGThreads, 1)
       }
 
       // ---- chain step: S_f^T = B_f^T + (alpha S_{f-1}^T) A_f^T
-      const int n3 = (L + 127) / 128;
-      if (tid == 0) {
-        // q tile 0 -> the R/U region (free now)
-        mbar_expect_tx(&bar.q_full[0], 32768);
-        tma_load_4d(sm + OFF_Q0, &tmap_q, &bar.q_full[0], 0, 0, f, bh);
-        tma_load_4d(sm + OFF_Q0 + 16384, &tmap_q, &bar.q_full[0], 64, 0, f, bh);
+      const int nq = (L + kQTok - 1) / kQTok;
+      if (tid == 0) {  // first read-out q tiles -> the tile-B half of the mirror (free now)
+        issue_q(f, bh, 0);
+        if (nq > 1) issue_q(f, bh, kQTok);
       }
       const float a_raw = p.alpha[(long)bh * F + f];
       const float alpha = p.gates_are_logits ? gate_alpha(a_raw) : a_raw;
       const bool have_prev = f > 0 || p.state_in != nullptr;
-      int bad = 0;
-      if (tid == 0 && f > 0) bad = !wait_flag(p.ws.flags + (long)bh * F + (f - 1), 1, lim);
-      if (bar_sync_or(1, kChain, bad)) {
-        if (tid == 0) mbar_wait(&bar.q_full[0], qcount[0] & 1u, lim);  // drain the q load in flight
-        failed = true;
-        break;
+      {
+        int bad = 0;
+        if (tid == 0 && f > 0) bad = !wait_flag(p.ws.flags + (long)bh * F + (f - 1), 1, lim);
+        if (bar_sync_or(1, kChain, bad || *abort_flag)) {
+          failed = true;
+          break;
+        }
       }
       if (have_prev) {
-        // rows j of alpha * S_{f-1}^T (threads of both tiles split the d_k
-        // columns); states are stored S[l][j] (d_v contiguous), so lanes j read
-        // consecutive addresses
+        // alpha S_{f-1}^T as fp16 pairs in TMEM (A operand): lane j, column l/2.
+        // States are stored S[l][j] (d_v contiguous), so lanes j read
+        // consecutive addresses.  Tile A covers l < 64, tile B l >= 64.
         const int j = row;
-        const int half = tile;  // 0: k-block 0, 1: k-block 1
         const float *prev = f > 0 ? p.ws.states + ((long)bh * F + (f - 1)) * (long)dk * dv
                                   : p.state_in + (long)bh * dk * dv;
-#pragma unroll 1
-        for (int cb = half * 4; cb < half * 4 + 4; ++cb) {
-          if (cb >= nkd) break;
-          float r[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) r[e] = j < dv ? alpha * __ldcg(prev + (long)(cb * 16 + e) * dv + j) : 0.f;
-          store_row16_f16(sm + OFF_SPREV + (cb >> 2) * 16384, j, (cb & 3) * 16, r);
+        for (int pp = tile * 2; pp < tile * 2 + 2; ++pp) {
+          if (2 * pp >= nkd) break;
+          uint32_t h[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int l0 = pp * 32 + 2 * e;
+            const float v0 = (j < dv && l0 < dk) ? alpha * __ldcg(prev + (long)l0 * dv + j) : 0.f;
+            const float v1 = (j < dv && l0 + 1 < dk) ? alpha * __ldcg(prev + (long)(l0 + 1) * dv + j) : 0.f;
+            h[e] = pack_h2(v0, v1);
+          }
+          tmem_st16u(tmem + TM_R + lane_off + pp * 16, h);
         }
-        fence_async_smem();
+        tmem_st_wait();
+        tc_fence_before();
         named_bar(1, kChain);
         if (tid == 0) {
           tc_fence_after();
-          const uint32_t sb = smem_u32(sm + OFF_SPREV);
           const uint32_t ab = smem_u32(sm + OFF_MIRROR);  // tile A of the mirror = A_f^T rows, read MN-major
           for (int kk = 0; kk < nkd; ++kk)
-            mma_f16_ss(tmem + TM_Y + 128, sdesc_sw128(sb + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                       sdesc_sw128(ab + kk * 2048, 16384, 1024), id_s, 1u);
+            mma_f16_ts(tmem + TM_Y + 128, tmem + TM_R + kk * 8, sdesc_sw128(ab + kk * 2048, 16384, 1024), id_s, 1u);
           mma_commit(&bar.fr_bar);
         }
-        if (!frame_wait(0)) { failed = true; break; }
+        const bool ok = group_wait(&bar.fr_bar, fphase);
+        fphase ^= 1u;
+        if (!ok) {
+          failed = true;
+          break;
+        }
         tc_fence_after();
       }
-      // S_f^T rows: publish fp32 as S[i][j] (lanes j write consecutive
-      // addresses), state_out, fp16 operand for the read-out
+      // S_f^T rows: publish fp32 as S[l][j] (lanes j write consecutive
+      // addresses), state_out, fp16 A operand of the read-out
       {
         const int j = row;
-        const int half = tile;
         float *cur = p.ws.states + ((long)bh * F + f) * (long)dk * dv;
         float *sout = (f == F - 1 && p.state_out) ? p.state_out + (long)bh * dk * dv : nullptr;
 #pragma unroll 1
-        for (int cb = half * 4; cb < half * 4 + 4; ++cb) {
+        for (int cb = tile * 4; cb < tile * 4 + 4; ++cb) {
           if (cb >= nkd) break;
           float r[16];
           tmem_ld16(tmem + TM_Y + 128 + lane_off + cb * 16, r);
@@ -673,71 +815,73 @@ __global__ void __launch_bounds__(kGThreads, 1)
           st_release(p.ws.flags + (long)bh * F + f, 1);
         }
         const long t = atomicAdd(p.ws.counter, 1);
-        bar.ticket_ring[frames & 3] = (int)(t < units ? t : -1);
+        const int tkn = (int)(t < units ? t : -1);
+        bar.ticket_ring[frames & 3] = tkn;
         mbar_arrive_only(&bar.tkt_bar[frames & 1]);
-        if (n3 > 1) {
-          mbar_expect_tx(&bar.q_full[1], 32768);
-          tma_load_4d(sm + OFF_Q1, &tmap_q, &bar.q_full[1], 0, 128, f, bh);
-          tma_load_4d(sm + OFF_Q1 + 16384, &tmap_q, &bar.q_full[1], 64, 128, f, bh);
+        if (!issue_frame_kv(tkn, g)) {
+          *abort_flag = 1;
+          latch_status(p.status, GDN_ERR_TIMEOUT);
         }
       }
 
-      // ---- read-out: O_f = Q_f S_f, 128 tokens per tile
-      for (int qc = 0; qc < n3; ++qc) {
-        const int b = qc & 1;
-        uint8_t *qb = sm + (b == 0 ? OFF_Q0 : OFF_Q1);
-        const int qbad = tid == 0 ? !mbar_wait(&bar.q_full[b], qcount[b] & 1u, lim) : 0;
-        ++qcount[b];
-        if (bar_sync_or(1, kChain, qbad)) { failed = true; break; }
-        // bf16 -> fp16 in place
-        for (int i = tid * 16; i < 32768; i += kChain * 16) {
-          uint4 u = *reinterpret_cast<uint4 *>(qb + i);
-          __nv_bfloat162 *h = reinterpret_cast<__nv_bfloat162 *>(&u);
-          uint32_t o[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 v2 = __bfloat1622float2(h[e]);
-            o[e] = pack_h2(v2.x, v2.y);
-          }
-          *reinterpret_cast<uint4 *>(qb + i) = make_uint4(o[0], o[1], o[2], o[3]);
+      // ---- read-out: O_f = Q_f S_f, 64 tokens per tile, O^T in TMEM (lanes j).
+      // Tile q + 1's MMA runs while tile q's results are stored.
+      auto q_mma = [&]() -> bool {  // all 256 chain threads
+        const int b = qw & 1;
+        if (!group_wait(&bar.q_full[b], (qw >> 1) & 1u)) return false;
+        ++qw;
+        uint8_t *qb = sm + OFF_QB + b * 16384;
+        for (int i = tid * 16; i < 16384; i += kChain * 16) {  // bf16 -> fp16 in place
+          uint4 *a = reinterpret_cast<uint4 *>(qb + i);
+          *a = bf16x8_to_f16x8(*a);
         }
         fence_async_smem();
         named_bar(1, kChain);
         if (tid == 0) {
           tc_fence_after();
-          // O^T = S_f^T Q^T: lanes = output columns j, TMEM columns = tokens
           const uint32_t a0 = smem_u32(sm + OFF_S16), b0 = smem_u32(qb);
-          for (int kk = 0; kk < nkd; ++kk) {
-            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-            mma_f16_ss(tmem + TM_RU, sdesc_sw128(a0 + off, 16, 1024), sdesc_sw128(b0 + off, 16, 1024), id_o,
-                       kk > 0 ? 1u : 0u);
-          }
-          mma_commit(&bar.fr_bar);
+          const int bo = oi & 1;
+          for (int kk = 0; kk < nkd; ++kk)
+            mma_f16_ss(tmem + TM_R + bo * 64, sdesc_sw128(a0 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                       sdesc_sw128(b0 + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), id_o, kk > 0 ? 1u : 0u);
+          mma_commit(&bar.o_bar[bo]);
         }
-        if (!frame_wait(0)) { failed = true; break; }
+        ++oi;
+        return true;
+      };
+      if (!q_mma()) {
+        failed = true;
+        break;
+      }
+      for (int qc = 0; qc < nq; ++qc) {
+        if (qc + 1 < nq && !q_mma()) {
+          failed = true;
+          break;
+        }
+        const int b = ow & 1;
+        if (!group_wait(&bar.o_bar[b], (ow >> 1) & 1u)) {
+          failed = true;
+          break;
+        }
+        ++ow;
         tc_fence_after();
-        if (tid == 0 && qc + 2 < n3) {
-          mbar_expect_tx(&bar.q_full[b], 32768);
-          tma_load_4d(qb, &tmap_q, &bar.q_full[b], 0, (qc + 2) * 128, f, bh);
-          tma_load_4d(qb + 16384, &tmap_q, &bar.q_full[b], 64, (qc + 2) * 128, f, bh);
-        }
-        // epilogue: lane j holds O[t][j] for the tile's tokens t; warps 0-3
-        // store tokens [0, 64), warps 4-7 tokens [64, 128); for each token a
-        // warp writes 32 consecutive floats of row t
+        if (tid == 0 && qc + 2 < nq) issue_q(f, bh, (qc + 2) * kQTok);
+        // epilogue: lane j holds O[t][j]; warps 0-3 store tokens [0, 32), warps
+        // 4-7 tokens [32, 64) of the tile; per token a warp writes 32
+        // consecutive floats of row t
         {
           const int j = row;
-          float *obase = p.o + ((long)bh * N + (long)f * L + (long)qc * 128) * dv + j;
-          const int tl = L - qc * 128;  // tokens of this tile
-#pragma unroll 1
-          for (int tb = tile * 4; tb < tile * 4 + 4; ++tb) {
-            float r[16];
-            tmem_ld16(tmem + TM_RU + lane_off + tb * 16, r);
-            tmem_ld_wait();
-            if (j < dv) {
+          const int t0 = qc * kQTok + tile * 32;
+          float *obase = p.o + ((long)bh * N + (long)f * L + t0) * dv + j;
+          const int tl = L - t0;  // tokens left from t0
+          float r[2][16];
+          tmem_ld16(tmem + TM_R + b * 64 + lane_off + tile * 32, r[0]);
+          tmem_ld16(tmem + TM_R + b * 64 + lane_off + tile * 32 + 16, r[1]);
+          tmem_ld_wait();
+          if (j < dv) {
 #pragma unroll
-              for (int e = 0; e < 16; ++e)
-                if (tb * 16 + e < tl) obase[(long)(tb * 16 + e) * dv] = r[e];
-            }
+            for (int e = 0; e < 32; ++e)
+              if (e < tl) obase[(long)e * dv] = r[e >> 4][e & 15];
           }
         }
         tc_fence_before();
@@ -746,8 +890,19 @@ __global__ void __launch_bounds__(kGThreads, 1)
       if (failed) break;
     }
     if (failed) {
-      if (tid == 0) latch_status(p.status, GDN_ERR_TIMEOUT);
-      bar.abort = 1;
+      if (tid == 0 && !*abort_flag) latch_status(p.status, GDN_ERR_TIMEOUT);
+      *abort_flag = 1;
+    }
+    // loads and MMAs issued by thread 0 complete before the CTA exits
+    if (tid == 0) {
+      for (; qw < qi; ++qw) mbar_wait(&bar.q_full[qw & 1], (qw >> 1) & 1u, lim);
+      for (; ow < oi; ++ow) mbar_wait(&bar.o_bar[ow & 1], (ow >> 1) & 1u, lim);
+    }
+    named_bar(1, kChain);
+    if (tid == 0) {  // the last k, v loads issued (earlier ones were waited for by the prep groups)
+      const uint32_t n = bar.loads;
+      for (uint32_t gg = n > (uint32_t)kSlots ? n - kSlots : 0u; gg < n; ++gg)
+        mbar_wait(&bar.kv_full[gg % kSlots], (gg / kSlots) & 1u, lim);
     }
   }
   tc_fence_before();
@@ -768,7 +923,7 @@ cudaError_t launch_gdn_tc(const GdnParams &p, int grid, cudaStream_t st) {
   using namespace tc;
   CUtensorMap mq, mk, mv;
   const int BH = p.B * p.H;
-  if (!make_bf16_map(&mq, p.q, p.dk, p.L, p.F, BH, 128) || !make_bf16_map(&mk, p.k, p.dk, p.L, p.F, BH, 64) ||
+  if (!make_bf16_map(&mq, p.q, p.dk, p.L, p.F, BH, kQTok) || !make_bf16_map(&mk, p.k, p.dk, p.L, p.F, BH, 64) ||
       !make_bf16_map(&mv, p.v, p.dv, p.L, p.F, BH, 64))
     return cudaErrorInvalidValue;
   cudaError_t e =
