@@ -35,9 +35,13 @@
 // k and v reach a 3-slot ring by TMA, issued by the chains as soon as a slot's
 // last MMA has completed (chunk c + 3 after chunk c; a frame's first three
 // chunks as soon as its ticket is taken).
-// Operands that are not exact in bf16 (khat, v after the cast, Y, R, T, W, S,
-// q) enter the tensor cores as fp16 (11-bit significands); all accumulation is
-// fp32.
+// The frame chain passes S_f between CTAs as fp16 rows S_f^T[j][l] (one bulk
+// store out, 16-byte loads in); alpha_f is folded into the fp16 copy of A_f.
+// The read-out takes S_f as a bf16 high/low pair (two MMAs on bf16 q) and
+// leaves through shared memory with bulk stores.
+// Operands that are not exact in bf16 (khat, v after the cast, Y, R, T, W, A_f,
+// S_{f-1}) enter the tensor cores as fp16 (11-bit significands); all
+// accumulation is fp32.
 #include "launch.h"
 #include "tc_host.h"
 #include "tc_ptx.cuh"
@@ -61,9 +65,10 @@ constexpr uint32_t SL_W = 32768;         //   W fp16, [128 rows i][128 B (64 t)]
                                          //   inversion while the prep group works on the slot
 constexpr uint32_t OFF_T = OFF_SLOT + kSlots * SLOT_BYTES;  // 2 x 8 KB: T fp16 [64 rows u][128 B (64 t)]
 constexpr uint32_t OFF_BAR = OFF_T + 2 * 8192;              // barriers and small state
-// read-out aliases (the mirror is free once the chain step has read A_f^T)
-constexpr uint32_t OFF_S16 = OFF_MIRROR;          // S_f^T fp16 [k-block][128 rows j][128 B]
-constexpr uint32_t OFF_QB = OFF_MIRROR + 32768;   // two q tiles [k-block][64 t][128 B]
+// frame-end aliases: the tile-B half of the mirror is free after the last
+// chunk, the tile-A half once the chain step has read alpha A_f^T
+constexpr uint32_t OFF_STAGE = OFF_MIRROR;        // 28 KB: fp16 rows of S_f, then fp32 rows of O, for bulk stores
+constexpr uint32_t OFF_QB = OFF_MIRROR + 32768;   // two q tiles (bf16) [k-block][64 t][128 B]
 
 struct Bars {
   uint64_t kv_full[kSlots];     // TMA bytes of k and v
@@ -86,7 +91,8 @@ constexpr size_t kGdnSmemBytes = OFF_BAR + sizeof(Bars) + 1024;
 static_assert(kGdnSmemBytes <= 232448, "shared memory budget");
 
 // TMEM columns
-constexpr uint32_t TM_Y = 0;     // Y^T: tile A [0,128), tile B [128,256)
+constexpr uint32_t TM_Y = 0;     // Y^T: tile A [0,128), tile B [128,256); read-out: S_f^T as bf16 pairs,
+                                 // high parts [0,64), low parts [64,128)
 constexpr uint32_t TM_R = 256;   // R^T: tile A [256,320), tile B [320,384); chain step: alpha S^T pairs
                                  // [256,320); read-out: O buffers [256,320), [320,384)
 constexpr uint32_t TM_P = 384;   // prep group g: [384 + 64 g, 448 + 64 g): Gram matrix, then W^T
@@ -126,8 +132,9 @@ __device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 u) {
 // row r = 16 floats whose four float4 groups are permuted by q ^ ((r >> 1) & 3)
 // (eight consecutive rows of one group fall in distinct bank groups).
 //   lblk(i, j), i >= j (10 blocks): N's block (i, j); the diagonal ones are
-//              replaced by D_i = (I + N_ii)^-1, the others by E_ij = D_i N_ij;
-//   iblk(i, j), i > j (6 blocks): block (i, j) of (I + N)^-1.
+//              replaced by D_i = (I + N_ii)^-1, the others (once E is formed)
+//              by block (i, j) of (I + N)^-1;
+//   iblk(i, j), i > j (6 blocks): E_ij = D_i N_ij.
 // With Linv_jj = D_j, block (i, j) of the inverse is -sum_{k=j}^{i-1} E_ik Linv_kj
 // (forward block substitution), computed by distance i - j = 1, 2, 3.
 __device__ __forceinline__ int bofs(int r, int q) { return r * 16 + ((q ^ ((r >> 1) & 3)) << 2); }
@@ -417,57 +424,31 @@ __global__ void __launch_bounds__(kGThreads, 1)
           for (int r = 0; r < 16; ++r) Dk[bofs(r, c >> 2) + (c & 3)] = x[r];
         }
         named_bar(pbar, 128);
-        // 5. E_ik = D_i N_ik for the six blocks below the diagonal (in place)
-        {
-          float4 acc[3];
-          int ei[3], ek[3], er[3], eq[3];
-#pragma unroll
-          for (int ps = 0; ps < 3; ++ps) {
-            const int it = pt + 128 * ps;
-            const int e = it >> 6, rem = it & 63;
-            eq[ps] = rem >> 4;
-            er[ps] = rem & 15;
-            ei[ps] = e < 3 ? e + 1 : (e < 5 ? e - 1 : 3);
-            ek[ps] = e < 3 ? e : (e < 5 ? e - 3 : 0);
-            acc[ps] = make_float4(0.f, 0.f, 0.f, 0.f);
-            blk_row_mul(acc[ps], lblk(scr, ei[ps], ei[ps]), lblk(scr, ei[ps], ek[ps]), er[ps], eq[ps]);
+        // 5. E_ik = D_i N_ik for the six blocks below the diagonal; item = (block,
+        //    float4 column group q, row r), 64 per block
+#pragma unroll 1
+        for (int it = pt; it < 6 * 64; it += 128) {
+          const int e = it >> 6, q = (it >> 4) & 3, r = it & 15;
+          const int d = e < 3 ? 1 : (e < 5 ? 2 : 3), kq = e < 3 ? e : (e < 5 ? e - 3 : 0);
+          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+          blk_row_mul(acc, lblk(scr, kq + d, kq + d), lblk(scr, kq + d, kq), r, q);
+          st_blk4(iblk(scr, kq + d, kq), r, q, acc);
+        }
+        named_bar(pbar, 128);
+        // 6-8. distance d = 1, 2, 3: Linv_{k+d,k} = -(E_{k+d,k} D_k + sum_{m=1}^{d-1}
+        //      E_{k+d,k+m} Linv_{k+m,k}), written over N's (dead) block
+#pragma unroll 1
+        for (int d = 1; d <= 3; ++d) {
+#pragma unroll 1
+          for (int it = pt; it < (4 - d) * 64; it += 128) {
+            const int kq = it >> 6, q = (it >> 4) & 3, r = it & 15;
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 1
+            for (int m = 0; m < d; ++m) blk_row_mul(acc, iblk(scr, kq + d, kq + m), lblk(scr, kq + m, kq), r, q);
+            st_blk4(lblk(scr, kq + d, kq), r, q, neg4(acc));
           }
           named_bar(pbar, 128);
-#pragma unroll
-          for (int ps = 0; ps < 3; ++ps) st_blk4(lblk(scr, ei[ps], ek[ps]), er[ps], eq[ps], acc[ps]);
         }
-        named_bar(pbar, 128);
-        // 6. distance 1: Linv_{k+1,k} = -E_{k+1,k} D_k
-#pragma unroll
-        for (int ps = 0; ps < 2; ++ps) {
-          const int it = pt + 128 * ps;
-          if (it < 192) {
-            const int e = it >> 6, rem = it & 63, q = rem >> 4, r = rem & 15;
-            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-            blk_row_mul(acc, lblk(scr, e + 1, e), lblk(scr, e, e), r, q);
-            st_blk4(iblk(scr, e + 1, e), r, q, neg4(acc));
-          }
-        }
-        named_bar(pbar, 128);
-        // 7. distance 2: Linv_{k+2,k} = -(E_{k+2,k} D_k + E_{k+2,k+1} Linv_{k+1,k})
-        {
-          const int e = pt >> 6, rem = pt & 63, q = rem >> 4, r = rem & 15;
-          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-          blk_row_mul(acc, lblk(scr, e + 2, e), lblk(scr, e, e), r, q);
-          blk_row_mul(acc, lblk(scr, e + 2, e + 1), iblk(scr, e + 1, e), r, q);
-          st_blk4(iblk(scr, e + 2, e), r, q, neg4(acc));
-        }
-        named_bar(pbar, 128);
-        // 8. distance 3: Linv_30 = -(E_30 D_0 + E_31 Linv_10 + E_32 Linv_20)
-        if (pt < 64) {
-          const int q = pt >> 4, r = pt & 15;
-          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-          blk_row_mul(acc, lblk(scr, 3, 0), lblk(scr, 0, 0), r, q);
-          blk_row_mul(acc, lblk(scr, 3, 1), iblk(scr, 1, 0), r, q);
-          blk_row_mul(acc, lblk(scr, 3, 2), iblk(scr, 2, 0), r, q);
-          st_blk4(iblk(scr, 3, 0), r, q, neg4(acc));
-        }
-        named_bar(pbar, 128);
         // 9. T[u][t] = Linv[u][t] beta_t as fp16, rows u (MN-major B operand: N = t, K = u)
         {
           const int u = pt >> 1, half = pt & 1;
@@ -480,7 +461,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
 #pragma unroll
               for (int e = 0; e < 16; ++e) v[e] = 0.f;
             } else {
-              const float *src = tb == ub ? lblk(scr, ub, ub) : iblk(scr, ub, tb);
+              const float *src = lblk(scr, ub, tb);  // D_ub on the diagonal, the inverse's block below it
 #pragma unroll
               for (int q = 0; q < 4; ++q) {
                 const float4 t4 = ld_blk4(src, r, q);
@@ -559,7 +540,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
     const uint32_t id_vw = idesc_f16(128, dk, 0, 1, 0);         // V^T (MN) x W
     const uint32_t id_kw = idesc_f16(128, dk, 0, 1, 0, 1, 0);   // -(Khat^T) (MN) x W
     const uint32_t id_s = idesc_f16(128, dk, 0, 0, 1);          // (alpha S^T, TMEM) x A^T (MN)
-    const uint32_t id_o = idesc_f16(128, kQTok, 0, 0, 0);       // S^T x Q^T
+    const uint32_t id_o = idesc_f16(128, kQTok, 1, 0, 0);       // S^T (bf16 pairs, TMEM) x Q^T (bf16)
 
     // Wait for this tile's MMAs: the issuing thread polls the mbarrier, the
     // others wait on the named barrier (which takes no issue slots from the
@@ -605,6 +586,8 @@ __global__ void __launch_bounds__(kGThreads, 1)
       const long ticket = tk;
       const int f = (int)(ticket / BH);
       const int bh = (int)(ticket % BH);
+      const float a_raw = p.alpha[(long)bh * F + f];
+      const float alpha = p.gates_are_logits ? gate_alpha(a_raw) : a_raw;
 
       // Y_A^T = I in TMEM (the first chunk accumulates onto it); Y_B^T starts
       // from the first chunk's product
@@ -701,19 +684,26 @@ __global__ void __launch_bounds__(kGThreads, 1)
           *abort_flag = 1;
           latch_status(p.status, GDN_ERR_TIMEOUT);
         }
-        // Y^T rows -> fp16 mirror (tile B's rows are not needed after the last chunk)
+        // Y^T rows -> fp16 mirror (tile B's rows are not needed after the last
+        // chunk; tile A's last copy is alpha_f A_f^T for the chain step)
         if (c + 1 < nch || tile == 0) {
+          const float sc = c + 1 < nch ? 1.f : alpha;
 #pragma unroll
+          for (int hb = 0; hb < 4; ++hb) {  // batches of up to 2 column blocks
+            if (2 * hb >= nkd) break;
+            float r[2][16];
 #pragma unroll
-          for (int hb = 0; hb < 2; ++hb) {  // two batches of up to 4 column blocks
-            float r[4][16];
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-              if (hb * 4 + e < nkd) tmem_ld16(tmY + lane_off + (hb * 4 + e) * 16, r[e]);
+            for (int e = 0; e < 2; ++e)
+              if (2 * hb + e < nkd) tmem_ld16(tmY + lane_off + (2 * hb + e) * 16, r[e]);
             tmem_ld_wait();
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-              if (hb * 4 + e < nkd) store_row16_f16(mir + hb * 16384, row, e * 16, r[e]);
+            for (int e = 0; e < 2; ++e)
+              if (2 * hb + e < nkd) {
+                const int cb = 2 * hb + e;
+#pragma unroll
+                for (int x = 0; x < 16; ++x) r[e][x] *= sc;
+                store_row16_f16(mir + (cb >> 2) * 16384, row, (cb & 3) * 16, r[e]);
+              }
           }
         }
         fence_async_smem();
@@ -725,14 +715,12 @@ __global__ void __launch_bounds__(kGThreads, 1)
         break;
       }
 
-      // ---- chain step: S_f^T = B_f^T + (alpha S_{f-1}^T) A_f^T
+      // ---- chain step: S_f^T = B_f^T + S_{f-1}^T (alpha A_f^T)
       const int nq = (L + kQTok - 1) / kQTok;
       if (tid == 0) {  // first read-out q tiles -> the tile-B half of the mirror (free now)
         issue_q(f, bh, 0);
         if (nq > 1) issue_q(f, bh, kQTok);
       }
-      const float a_raw = p.alpha[(long)bh * F + f];
-      const float alpha = p.gates_are_logits ? gate_alpha(a_raw) : a_raw;
       const bool have_prev = f > 0 || p.state_in != nullptr;
       {
         int bad = 0;
@@ -742,32 +730,55 @@ __global__ void __launch_bounds__(kGThreads, 1)
           break;
         }
       }
+      const int j = row;
+      const int l0 = tile * 64;                                        // this thread's half of the d_k columns
+      const int nl = dk - l0 < 64 ? (dk - l0 > 0 ? dk - l0 : 0) : 64;  // columns in it (a multiple of 16)
       if (have_prev) {
-        // alpha S_{f-1}^T as fp16 pairs in TMEM (A operand): lane j, column l/2.
-        // States are stored S[l][j] (d_v contiguous), so lanes j read
-        // consecutive addresses.  Tile A covers l < 64, tile B l >= 64.
-        const int j = row;
-        const float *prev = f > 0 ? p.ws.states + ((long)bh * F + (f - 1)) * (long)dk * dv
-                                  : p.state_in + (long)bh * dk * dv;
+        // S_{f-1}^T row j as fp16 pairs into TMEM columns [256, 256 + d_k / 2) (A operand)
+        if (nl > 0) {
+          if (f > 0) {
+            // published rows S^T[j][l] (fp16, d_k per row): the pairs are the loaded words
+            const uint4 *src = reinterpret_cast<const uint4 *>(
+                reinterpret_cast<const __half *>(p.ws.states) + ((long)bh * F + (f - 1)) * (long)dk * dv +
+                (long)j * dk + l0);
+            uint4 u[8];
 #pragma unroll
-        for (int pp = tile * 2; pp < tile * 2 + 2; ++pp) {
-          if (2 * pp >= nkd) break;
-          uint32_t h[16];
+            for (int e = 0; e < 8; ++e)
+              u[e] = (j < dv && 8 * e < nl) ? __ldcg(src + e) : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int l0 = pp * 32 + 2 * e;
-            const float v0 = (j < dv && l0 < dk) ? alpha * __ldcg(prev + (long)l0 * dv + j) : 0.f;
-            const float v1 = (j < dv && l0 + 1 < dk) ? alpha * __ldcg(prev + (long)(l0 + 1) * dv + j) : 0.f;
-            h[e] = pack_h2(v0, v1);
+            for (int h2 = 0; h2 < 2; ++h2) {
+              if (32 * h2 < nl) {
+                const uint32_t w[16] = {u[4 * h2].x,     u[4 * h2].y,     u[4 * h2].z,     u[4 * h2].w,
+                                        u[4 * h2 + 1].x, u[4 * h2 + 1].y, u[4 * h2 + 1].z, u[4 * h2 + 1].w,
+                                        u[4 * h2 + 2].x, u[4 * h2 + 2].y, u[4 * h2 + 2].z, u[4 * h2 + 2].w,
+                                        u[4 * h2 + 3].x, u[4 * h2 + 3].y, u[4 * h2 + 3].z, u[4 * h2 + 3].w};
+                tmem_st16u(tmem + TM_R + lane_off + (l0 + 32 * h2) / 2, w);
+              }
+            }
+          } else {
+            // the caller's fp32 state S[l][j] (d_v contiguous: lanes j read consecutive addresses)
+            const float *prev = p.state_in + (long)bh * dk * dv;
+#pragma unroll 1
+            for (int h2 = 0; h2 < 2; ++h2) {
+              if (32 * h2 >= nl) break;
+              uint32_t w[16];
+#pragma unroll
+              for (int e = 0; e < 16; ++e) {
+                const int l = l0 + 32 * h2 + 2 * e;
+                const float v0 = (j < dv && l < dk) ? __ldcg(prev + (long)l * dv + j) : 0.f;
+                const float v1 = (j < dv && l + 1 < dk) ? __ldcg(prev + (long)(l + 1) * dv + j) : 0.f;
+                w[e] = pack_h2(v0, v1);
+              }
+              tmem_st16u(tmem + TM_R + lane_off + (l0 + 32 * h2) / 2, w);
+            }
           }
-          tmem_st16u(tmem + TM_R + lane_off + pp * 16, h);
         }
         tmem_st_wait();
         tc_fence_before();
         named_bar(1, kChain);
         if (tid == 0) {
           tc_fence_after();
-          const uint32_t ab = smem_u32(sm + OFF_MIRROR);  // tile A of the mirror = A_f^T rows, read MN-major
+          const uint32_t ab = smem_u32(sm + OFF_MIRROR);  // tile A of the mirror = alpha A_f^T rows, read MN-major
           for (int kk = 0; kk < nkd; ++kk)
             mma_f16_ts(tmem + TM_Y + 128, tmem + TM_R + kk * 8, sdesc_sw128(ab + kk * 2048, 16384, 1024), id_s, 1u);
           mma_commit(&bar.fr_bar);
@@ -780,37 +791,55 @@ __global__ void __launch_bounds__(kGThreads, 1)
         }
         tc_fence_after();
       }
-      // S_f^T rows: publish fp32 as S[l][j] (lanes j write consecutive
-      // addresses), state_out, fp16 A operand of the read-out
+      // S_f^T row j (this thread's half of l): an fp16 row into the staging
+      // area (one bulk store to the workspace, for the next frame), bf16
+      // high/low pairs into TMEM [0, 128) (the read-out's A operand), and the
+      // fp32 state_out after the last frame
       {
-        const int j = row;
-        float *cur = p.ws.states + ((long)bh * F + f) * (long)dk * dv;
         float *sout = (f == F - 1 && p.state_out) ? p.state_out + (long)bh * dk * dv : nullptr;
+        __half *srow = reinterpret_cast<__half *>(sm + OFF_STAGE) + (long)j * dk + l0;
 #pragma unroll 1
-        for (int cb = tile * 4; cb < tile * 4 + 4; ++cb) {
-          if (cb >= nkd) break;
+        for (int h2 = 0; h2 < 4; ++h2) {  // 16 columns l at a time
+          if (16 * h2 >= nl) break;
+          const int lb = l0 + 16 * h2;
           float r[16];
-          tmem_ld16(tmem + TM_Y + 128 + lane_off + cb * 16, r);
+          tmem_ld16(tmem + TM_Y + 128 + lane_off + lb, r);
           tmem_ld_wait();
-          if (j < dv) {
+          uint32_t hi[8], lo[8], hf[8];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) cur[(long)(cb * 16 + e) * dv + j] = r[e];
+          for (int e = 0; e < 8; ++e) {
+            const float a = j < dv ? r[2 * e] : 0.f;
+            const float b = j < dv ? r[2 * e + 1] : 0.f;
+            const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+            const float2 hb = __bfloat1622float2(h);
+            const __nv_bfloat162 lw = __floats2bfloat162_rn(a - hb.x, b - hb.y);
+            hi[e] = *reinterpret_cast<const uint32_t *>(&h);
+            lo[e] = *reinterpret_cast<const uint32_t *>(&lw);
+            hf[e] = pack_h2(a, b);
+          }
+          tmem_st8u(tmem + TM_Y + lane_off + lb / 2, hi);
+          tmem_st8u(tmem + TM_Y + 64 + lane_off + lb / 2, lo);
+          if (j < dv) {
+            *reinterpret_cast<uint4 *>(srow + 16 * h2) = make_uint4(hf[0], hf[1], hf[2], hf[3]);
+            *reinterpret_cast<uint4 *>(srow + 16 * h2 + 8) = make_uint4(hf[4], hf[5], hf[6], hf[7]);
             if (sout) {
 #pragma unroll
-              for (int e = 0; e < 16; ++e) sout[(long)(cb * 16 + e) * dv + j] = r[e];
+              for (int e = 0; e < 16; ++e) sout[(long)(lb + e) * dv + j] = r[e];
             }
-          } else {
-#pragma unroll
-            for (int e = 0; e < 16; ++e) r[e] = 0.f;
           }
-          store_row16_f16(sm + OFF_S16 + (cb >> 2) * 16384, j, (cb & 3) * 16, r);
         }
       }
+      tmem_st_wait();
       fence_async_smem();
       tc_fence_before();
       named_bar(1, kChain);
       if (tid == 0) {
+        __half *dst = reinterpret_cast<__half *>(p.ws.states) + ((long)bh * F + f) * (long)dk * dv;
+        bulk_store(dst, sm + OFF_STAGE, (uint32_t)(dk * dv * 2));
+        bulk_commit();
+        bulk_wait_all();
         if (ticket != p.withhold) {
+          fence_async_global();
           __threadfence();
           st_release(p.ws.flags + (long)bh * F + f, 1);
         }
@@ -824,69 +853,70 @@ __global__ void __launch_bounds__(kGThreads, 1)
         }
       }
 
-      // ---- read-out: O_f = Q_f S_f, 64 tokens per tile, O^T in TMEM (lanes j).
-      // Tile q + 1's MMA runs while tile q's results are stored.
-      auto q_mma = [&]() -> bool {  // all 256 chain threads
+      // ---- read-out: O_f = Q_f S_f, 64 tokens per tile.  Thread 0 issues
+      // O^T = S_f^T Q^T (bf16 high and low parts of S_f from TMEM, bf16 q from
+      // shared memory) into TMEM buffer n & 1, one tile ahead; the epilogue
+      // moves O^T through shared memory into O's own row-major layout and each
+      // tile chain's first thread bulk-stores its 32 tokens.
+      auto q_mma = [&]() -> bool {  // thread 0
         const int b = qw & 1;
-        if (!group_wait(&bar.q_full[b], (qw >> 1) & 1u)) return false;
+        if (!mbar_wait(&bar.q_full[b], (qw >> 1) & 1u, lim)) return false;
         ++qw;
-        uint8_t *qb = sm + OFF_QB + b * 16384;
-        for (int i = tid * 16; i < 16384; i += kChain * 16) {  // bf16 -> fp16 in place
-          uint4 *a = reinterpret_cast<uint4 *>(qb + i);
-          *a = bf16x8_to_f16x8(*a);
-        }
-        fence_async_smem();
-        named_bar(1, kChain);
-        if (tid == 0) {
-          tc_fence_after();
-          const uint32_t a0 = smem_u32(sm + OFF_S16), b0 = smem_u32(qb);
-          const int bo = oi & 1;
+        tc_fence_after();
+        const uint32_t b0 = smem_u32(sm + OFF_QB + b * 16384);
+        const int bo = oi & 1;
+        for (int hl = 0; hl < 2; ++hl)
           for (int kk = 0; kk < nkd; ++kk)
-            mma_f16_ss(tmem + TM_R + bo * 64, sdesc_sw128(a0 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                       sdesc_sw128(b0 + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), id_o, kk > 0 ? 1u : 0u);
-          mma_commit(&bar.o_bar[bo]);
-        }
+            mma_f16_ts(tmem + TM_R + bo * 64, tmem + TM_Y + hl * 64 + kk * 8,
+                       sdesc_sw128(b0 + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), id_o,
+                       (hl > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&bar.o_bar[bo]);
         ++oi;
         return true;
       };
-      if (!q_mma()) {
-        failed = true;
-        break;
-      }
+      int qbad = 0;
+      if (tid == 0) qbad = !q_mma();
       for (int qc = 0; qc < nq; ++qc) {
-        if (qc + 1 < nq && !q_mma()) {
-          failed = true;
-          break;
-        }
+        if (tid == 0 && !qbad && qc + 1 < nq) qbad = !q_mma();
         const int b = ow & 1;
-        if (!group_wait(&bar.o_bar[b], (ow >> 1) & 1u)) {
-          failed = true;
-          break;
+        {
+          int bad = qbad;
+          if (tid == 0 && !bad) bad = !mbar_wait(&bar.o_bar[b], (ow >> 1) & 1u, lim);
+          if (bar_sync_or(1, kChain, bad || *abort_flag)) {
+            failed = true;
+            break;
+          }
         }
         ++ow;
         tc_fence_after();
         if (tid == 0 && qc + 2 < nq) issue_q(f, bh, (qc + 2) * kQTok);
-        // epilogue: lane j holds O[t][j]; warps 0-3 store tokens [0, 32), warps
-        // 4-7 tokens [32, 64) of the tile; per token a warp writes 32
-        // consecutive floats of row t
+        // epilogue: lane j holds O[t][j] for the tile's tokens t; tile A's
+        // threads take tokens [0, 32), tile B's [32, 64)
         {
-          const int j = row;
           const int t0 = qc * kQTok + tile * 32;
-          float *obase = p.o + ((long)bh * N + (long)f * L + t0) * dv + j;
-          const int tl = L - t0;  // tokens left from t0
+          const int tl = L - t0 < 32 ? L - t0 : 32;  // tokens of this half (may be <= 0)
+          float *stg = reinterpret_cast<float *>(sm + OFF_STAGE) + tile * 32 * dv;
           float r[2][16];
           tmem_ld16(tmem + TM_R + b * 64 + lane_off + tile * 32, r[0]);
           tmem_ld16(tmem + TM_R + b * 64 + lane_off + tile * 32 + 16, r[1]);
           tmem_ld_wait();
+          if (issuer) bulk_wait_read();  // the previous tile's bulk store has read the staging rows
+          named_bar(tbar, 128);
           if (j < dv) {
 #pragma unroll
-            for (int e = 0; e < 32; ++e)
-              if (e < tl) obase[(long)e * dv] = r[e >> 4][e & 15];
+            for (int e = 0; e < 32; ++e) stg[e * dv + j] = r[e >> 4][e & 15];
           }
+          fence_async_smem();
+          named_bar(tbar, 128);
+          if (issuer && tl > 0)
+            bulk_store(p.o + ((long)bh * N + (long)f * L + t0) * dv, stg, (uint32_t)(tl * dv * 4));
+          if (issuer) bulk_commit();
         }
         tc_fence_before();
         named_bar(1, kChain);
       }
+      // the staging rows (the tile-A half of the mirror) are rewritten by the next frame
+      if (issuer) bulk_wait_read();
       if (failed) break;
     }
     if (failed) {
@@ -898,6 +928,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
       for (; qw < qi; ++qw) mbar_wait(&bar.q_full[qw & 1], (qw >> 1) & 1u, lim);
       for (; ow < oi; ++ow) mbar_wait(&bar.o_bar[ow & 1], (ow >> 1) & 1u, lim);
     }
+    if (issuer) bulk_wait_all();
     named_bar(1, kChain);
     if (tid == 0) {  // the last k, v loads issued (earlier ones were waited for by the prep groups)
       const uint32_t n = bar.loads;
@@ -917,7 +948,8 @@ bool gdn_tc_supported(int dk, int dv) {
   return dk % 16 == 0 && dv % 16 == 0 && dk >= 16 && dk <= 128 && dv >= 16 && dv <= 128;
 }
 
-size_t gdn_tc_state_elems(int dk, int dv) { return (size_t)dk * dv; }
+// published frame states are fp16 rows S^T[j][l]: d_k * d_v halves = d_k * d_v / 2 floats
+size_t gdn_tc_state_elems(int dk, int dv) { return (size_t)dk * dv / 2; }
 
 cudaError_t launch_gdn_tc(const GdnParams &p, int grid, cudaStream_t st) {
   using namespace tc;

@@ -43,14 +43,16 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 // The bound is counted in SM clock cycles (2 per ns, i.e. at most limit_ns at
 // clocks up to 2 GHz and proportionally longer at lower clocks): clock64 is
 // cheap enough to read on every spin, unlike %globaltimer.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, unsigned long long limit_ns) {
-  if (mbar_try_wait(bar, parity)) return true;
+__device__ __forceinline__ bool mbar_wait_slow(uint64_t *bar, uint32_t parity, unsigned long long limit_ns) {
   const long long t0 = clock64();
   const long long lim = (long long)(limit_ns * 2ull);
   while (!mbar_try_wait(bar, parity)) {
     if (clock64() - t0 > lim) return false;
   }
   return true;
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, unsigned long long limit_ns) {
+  return mbar_try_wait(bar, parity) || mbar_wait_slow(bar, parity, limit_ns);
 }
 
 // Named barrier over `n` threads that also ORs a predicate across them.
@@ -80,6 +82,21 @@ __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map) {
 }
 // Make generic-proxy writes to shared memory visible to the async proxy (MMA / TMA).
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+// Order the async proxy's global writes (bulk stores) with later generic-proxy accesses.
+__device__ __forceinline__ void fence_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
+
+// 1-D bulk copy shared -> global (both addresses 16-byte aligned, bytes a
+// multiple of 16), tracked in this thread's bulk async-group.
+__device__ __forceinline__ void bulk_store(void *gdst, const void *ssrc, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst), "r"(smem_u32(ssrc)),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// This thread's bulk groups have finished reading shared memory (the source may be reused).
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// This thread's bulk groups have completed (their global writes are performed).
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // ---------------------------------------------------------------- TMEM
 __device__ __forceinline__ void tmem_alloc(uint32_t *dst_smem, uint32_t ncols) {
@@ -149,11 +166,16 @@ __device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t (&u)[1
       "r"(u[10]), "r"(u[11]), "r"(u[12]), "r"(u[13]), "r"(u[14]), "r"(u[15])
       : "memory");
 }
+__device__ __forceinline__ void tmem_st8u(uint32_t taddr, const uint32_t (&u)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(u[0]),
+               "r"(u[1]), "r"(u[2]), "r"(u[3]), "r"(u[4]), "r"(u[5]), "r"(u[6]), "r"(u[7])
+               : "memory");
+}
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // Per-warpgroup register budget (all 128 threads of the warpgroup execute it).
-// The block launches with 384 x 168 = 64,512 registers; the splits used here
-// (2 x 128 x 128 + 128 x 232 = 62,464) stay within that.
+// The budgets of all warpgroups, 128 x N each, must add up to no more than the
+// block's threads x registers at launch, or an increase waits forever.
 template <int N>
 __device__ __forceinline__ void regs_inc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N)); }
 template <int N>
