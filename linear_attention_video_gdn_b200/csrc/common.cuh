@@ -16,7 +16,9 @@ constexpr float kKeyNormEps = 1e-6f;
 // Workspace of the frame-chain kernels:
 //   [0, 256)                 : int counters (ticket counter at [0])
 //   [256, 256 + 4*units)     : int flag per (b, h, f) unit: 1 once its state is published
-//   then, 256-byte aligned   : float published state per unit, transposed: St[j][i] (dv rows of dk)
+//   then, 256-byte aligned   : published state per unit, in the layout of the kernel that runs:
+//                              the SIMT frame kernel fp32 St[j][i] (dv rows of dk), the tcgen05
+//                              kernel fp16 rows S^T[j][l] (half the bytes; sized in floats)
 struct Workspace {
   int *counter;
   int *flags;

@@ -53,7 +53,7 @@ constexpr int kChain = 256;      // warps 0-7
 constexpr int kGThreads = 512;   // + two prep warpgroups
 constexpr int kC = 64;           // tokens per chunk
 constexpr int kSlots = 3;        // chunks in flight (k, v, W)
-constexpr int kQTok = 64;        // tokens per read-out tile
+constexpr int kQTok = 32;        // tokens per read-out tile (tile chain A takes even tiles, B odd ones)
 
 // shared memory map (bytes from the 1024-aligned base)
 constexpr uint32_t OFF_MIRROR = 0;       // 64 KB: Y^T as fp16, [tile][k-block][128 rows][128 B]
@@ -68,7 +68,7 @@ constexpr uint32_t OFF_BAR = OFF_T + 2 * 8192;              // barriers and smal
 // frame-end aliases: the tile-B half of the mirror is free after the last
 // chunk, the tile-A half once the chain step has read alpha A_f^T
 constexpr uint32_t OFF_STAGE = OFF_MIRROR;        // 28 KB: fp16 rows of S_f, then fp32 rows of O, for bulk stores
-constexpr uint32_t OFF_QB = OFF_MIRROR + 32768;   // two q tiles (bf16) [k-block][64 t][128 B]
+constexpr uint32_t OFF_QB = OFF_MIRROR + 32768;   // per tile chain two q tiles (bf16) [k-block][32 t][128 B]
 
 struct Bars {
   uint64_t kv_full[kSlots];     // TMA bytes of k and v
@@ -78,8 +78,8 @@ struct Bars {
   uint64_t g_bar[2];            // per prep group: its MMAs
   uint64_t mma_bar[2];          // per tile chain
   uint64_t fr_bar;              // frame-level MMAs (chain step)
-  uint64_t q_full[2];
-  uint64_t o_bar[2];            // read-out MMA into O buffer b
+  uint64_t q_full[2][2];        // [tile chain][buffer]
+  uint64_t o_bar[2][2];         // [tile chain][buffer]: read-out MMA into that O buffer
   uint64_t tkt_bar[2];          // chain group -> prep groups: next frame's ticket
   uint32_t tmem_base;
   int abort;
@@ -93,8 +93,9 @@ static_assert(kGdnSmemBytes <= 232448, "shared memory budget");
 // TMEM columns
 constexpr uint32_t TM_Y = 0;     // Y^T: tile A [0,128), tile B [128,256); read-out: S_f^T as bf16 pairs,
                                  // high parts [0,64), low parts [64,128)
-constexpr uint32_t TM_R = 256;   // R^T: tile A [256,320), tile B [320,384); chain step: alpha S^T pairs
-                                 // [256,320); read-out: O buffers [256,320), [320,384)
+constexpr uint32_t TM_R = 256;   // R^T: tile A [256,320), tile B [320,384); chain step: S^T pairs
+                                 // [256,320); read-out: O buffers, 32 columns each, tile A [256,320),
+                                 // tile B [320,384)
 constexpr uint32_t TM_P = 384;   // prep group g: [384 + 64 g, 448 + 64 g): Gram matrix, then W^T
 
 __device__ __forceinline__ void named_bar(int id, int n) {
@@ -211,8 +212,10 @@ __global__ void __launch_bounds__(kGThreads, 1)
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bar.g_bar[s], 1);
       mbar_init(&bar.mma_bar[s], 1);
-      mbar_init(&bar.q_full[s], 1);
-      mbar_init(&bar.o_bar[s], 1);
+      mbar_init(&bar.q_full[0][s], 1);
+      mbar_init(&bar.q_full[1][s], 1);
+      mbar_init(&bar.o_bar[0][s], 1);
+      mbar_init(&bar.o_bar[1][s], 1);
       mbar_init(&bar.tkt_bar[s], 1);
     }
     mbar_init(&bar.fr_bar, 1);
@@ -269,7 +272,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
     uint32_t g = 0;
     bool stop = false;
     auto group_fail = [&](int timed_out) {
-      if (pt == 0 && timed_out && !*abort_flag) latch_status(p.status, GDN_ERR_TIMEOUT);
+      if (pt == 0 && timed_out) latch_status(p.status, GDN_ERR_TIMEOUT);  // the first code latched wins
       *abort_flag = 1;
       stop = true;
     };
@@ -529,8 +532,9 @@ __global__ void __launch_bounds__(kGThreads, 1)
     uint8_t *mir = sm + OFF_MIRROR + tile * 32768;
     uint32_t tphase = 0;                  // phase of mma_bar[tile]
     uint32_t fphase = 0;                  // phase of fr_bar
-    // read-out tiles over the CTA's lifetime: q loads issued / waited for, MMAs
-    // issued / waited for; tile n uses q buffer n & 1 and O buffer n & 1
+    // this tile chain's read-out tiles over the CTA's lifetime: q loads issued /
+    // waited for, MMAs issued / waited for; tile n uses q buffer n & 1 and O
+    // buffer n & 1
     uint32_t qi = 0, qw = 0, oi = 0, ow = 0;
     int frames = 0;
     bool failed = false;
@@ -541,6 +545,8 @@ __global__ void __launch_bounds__(kGThreads, 1)
     const uint32_t id_kw = idesc_f16(128, dk, 0, 1, 0, 1, 0);   // -(Khat^T) (MN) x W
     const uint32_t id_s = idesc_f16(128, dk, 0, 0, 1);          // (alpha S^T, TMEM) x A^T (MN)
     const uint32_t id_o = idesc_f16(128, kQTok, 1, 0, 0);       // S^T (bf16 pairs, TMEM) x Q^T (bf16)
+    uint8_t *qbuf = sm + OFF_QB + tile * 16384;                  // this chain's q buffers, 8 KB each
+    const uint32_t tmO = tmem + TM_R + tile * 64;                // this chain's O buffers, 32 columns each
 
     // Wait for this tile's MMAs: the issuing thread polls the mbarrier, the
     // others wait on the named barrier (which takes no issue slots from the
@@ -558,19 +564,21 @@ __global__ void __launch_bounds__(kGThreads, 1)
       if (tid == 0) bad = !mbar_wait(b, parity, lim);
       return !bar_sync_or(1, kChain, bad || *abort_flag);
     };
-    auto issue_q = [&](int f, int bh, int t0) {  // thread 0
+    auto issue_q = [&](int f, int bh, int t0) {  // the tile's issuer
       const int bq = qi & 1;
-      mbar_expect_tx(&bar.q_full[bq], 16384);
-      uint8_t *qb = sm + OFF_QB + bq * 16384;
-      tma_load_4d(qb, &tmap_q, &bar.q_full[bq], 0, t0, f, bh);
-      tma_load_4d(qb + 8192, &tmap_q, &bar.q_full[bq], 64, t0, f, bh);
+      mbar_expect_tx(&bar.q_full[tile][bq], 8192);
+      uint8_t *qb = qbuf + bq * 8192;
+      tma_load_4d(qb, &tmap_q, &bar.q_full[tile][bq], 0, t0, f, bh);
+      tma_load_4d(qb + 4096, &tmap_q, &bar.q_full[tile][bq], 64, t0, f, bh);
       ++qi;
     };
 
     // The chain group takes the tickets: the first here, each next one right
     // after the current frame's state is published (before its read-out), and
-    // hands each to the loader and the prep groups.  A ticket is thus started a
-    // fixed read-out time after it is taken, whatever the frame chain's waits were.
+    // hands each to the prep groups.  A ticket is thus started a fixed read-out
+    // time after it is taken, whatever the frame chain's waits were; taking it
+    // earlier (for the prep groups to run on across the frame boundary) was
+    // measured slower, the longer hold lengthening the frame chain's waits.
     if (tid == 0) {
       const long t = atomicAdd(p.ws.counter, 1);
       const int tk0 = (int)(t < units ? t : -1);
@@ -716,10 +724,11 @@ __global__ void __launch_bounds__(kGThreads, 1)
       }
 
       // ---- chain step: S_f^T = B_f^T + S_{f-1}^T (alpha A_f^T)
-      const int nq = (L + kQTok - 1) / kQTok;
-      if (tid == 0) {  // first read-out q tiles -> the tile-B half of the mirror (free now)
-        issue_q(f, bh, 0);
-        if (nq > 1) issue_q(f, bh, kQTok);
+      // read-out tiles of this chain: tile-chain A takes tiles 0, 2, 4, ...; B 1, 3, 5, ...
+      const int nq = ((L + kQTok - 1) / kQTok - tile + 1) / 2;
+      if (issuer) {  // its first q tiles -> the tile-B half of the mirror (free now)
+        if (nq > 0) issue_q(f, bh, tile * kQTok);
+        if (nq > 1) issue_q(f, bh, (2 + tile) * kQTok);
       }
       const bool have_prev = f > 0 || p.state_in != nullptr;
       {
@@ -853,80 +862,91 @@ __global__ void __launch_bounds__(kGThreads, 1)
         }
       }
 
-      // ---- read-out: O_f = Q_f S_f, 64 tokens per tile.  Thread 0 issues
-      // O^T = S_f^T Q^T (bf16 high and low parts of S_f from TMEM, bf16 q from
-      // shared memory) into TMEM buffer n & 1, one tile ahead; the epilogue
-      // moves O^T through shared memory into O's own row-major layout and each
-      // tile chain's first thread bulk-stores its 32 tokens.
-      auto q_mma = [&]() -> bool {  // thread 0
+      // ---- read-out: O_f = Q_f S_f in 32-token tiles, two independent
+      // pipelines (tile chain A: even tiles, B: odd tiles).  Each chain's
+      // issuer runs O^T = S_f^T Q^T (bf16 high and low parts of S_f from TMEM,
+      // bf16 q) into its TMEM buffer n & 1 one tile ahead; the epilogue moves
+      // O^T through shared memory into O's row-major layout and the issuer
+      // bulk-stores the 32 tokens.
+      named_bar(1, kChain);  // thread 0's bulk store of S_f has read the staging area
+      auto q_mma = [&](bool poll) -> int {  // the tile's issuer; with `poll` only if the q tile is in (else 2)
         const int b = qw & 1;
-        if (!mbar_wait(&bar.q_full[b], (qw >> 1) & 1u, lim)) return false;
+        if (poll) {
+          if (!mbar_try_wait(&bar.q_full[tile][b], (qw >> 1) & 1u)) return 2;
+        } else if (!mbar_wait(&bar.q_full[tile][b], (qw >> 1) & 1u, lim)) {
+          return 0;
+        }
         ++qw;
         tc_fence_after();
-        const uint32_t b0 = smem_u32(sm + OFF_QB + b * 16384);
+        const uint32_t b0 = smem_u32(qbuf + b * 8192);
         const int bo = oi & 1;
         for (int hl = 0; hl < 2; ++hl)
           for (int kk = 0; kk < nkd; ++kk)
-            mma_f16_ts(tmem + TM_R + bo * 64, tmem + TM_Y + hl * 64 + kk * 8,
-                       sdesc_sw128(b0 + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), id_o,
+            mma_f16_ts(tmO + bo * 32, tmem + TM_Y + hl * 64 + kk * 8,
+                       sdesc_sw128(b0 + (kk >> 2) * 4096 + (kk & 3) * 32, 16, 1024), id_o,
                        (hl > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&bar.o_bar[bo]);
+        mma_commit(&bar.o_bar[tile][bo]);
         ++oi;
-        return true;
+        return 1;
       };
       int qbad = 0;
-      if (tid == 0) qbad = !q_mma();
+      if (issuer && nq > 0) qbad = !q_mma(false);
+      float *stg = reinterpret_cast<float *>(sm + OFF_STAGE) + tile * kQTok * dv;
       for (int qc = 0; qc < nq; ++qc) {
-        if (tid == 0 && !qbad && qc + 1 < nq) qbad = !q_mma();
         const int b = ow & 1;
         {
           int bad = qbad;
-          if (tid == 0 && !bad) bad = !mbar_wait(&bar.o_bar[b], (ow >> 1) & 1u, lim);
-          if (bar_sync_or(1, kChain, bad || *abort_flag)) {
+          if (issuer && !bad) bad = !mbar_wait(&bar.o_bar[tile][b], (ow >> 1) & 1u, lim);
+          if (bar_sync_or(tbar, 128, bad || *abort_flag)) {
             failed = true;
             break;
           }
         }
         ++ow;
         tc_fence_after();
-        if (tid == 0 && qc + 2 < nq) issue_q(f, bh, (qc + 2) * kQTok);
-        // epilogue: lane j holds O[t][j] for the tile's tokens t; tile A's
-        // threads take tokens [0, 32), tile B's [32, 64)
-        {
-          const int t0 = qc * kQTok + tile * 32;
-          const int tl = L - t0 < 32 ? L - t0 : 32;  // tokens of this half (may be <= 0)
-          float *stg = reinterpret_cast<float *>(sm + OFF_STAGE) + tile * 32 * dv;
-          float r[2][16];
-          tmem_ld16(tmem + TM_R + b * 64 + lane_off + tile * 32, r[0]);
-          tmem_ld16(tmem + TM_R + b * 64 + lane_off + tile * 32 + 16, r[1]);
-          tmem_ld_wait();
-          if (issuer) bulk_wait_read();  // the previous tile's bulk store has read the staging rows
-          named_bar(tbar, 128);
-          if (j < dv) {
-#pragma unroll
-            for (int e = 0; e < 32; ++e) stg[e * dv + j] = r[e >> 4][e & 15];
-          }
-          fence_async_smem();
-          named_bar(tbar, 128);
-          if (issuer && tl > 0)
-            bulk_store(p.o + ((long)bh * N + (long)f * L + t0) * dv, stg, (uint32_t)(tl * dv * 4));
-          if (issuer) bulk_commit();
+        const int t0 = (2 * qc + tile) * kQTok;
+        const int tl = L - t0 < kQTok ? L - t0 : kQTok;  // tokens of this tile
+        float r[2][16];
+        tmem_ld16(tmO + b * 32 + lane_off, r[0]);
+        tmem_ld16(tmO + b * 32 + lane_off + 16, r[1]);
+        tmem_ld_wait();
+        // this tile's q buffer is free: tile qc + 2 goes there; tile qc + 1's MMA
+        // starts now if its q tile is in, else after this epilogue
+        bool next_pending = false;
+        if (issuer) {
+          if (qc + 2 < nq) issue_q(f, bh, (2 * (qc + 2) + tile) * kQTok);
+          if (qc + 1 < nq) next_pending = q_mma(true) == 2;
+          bulk_wait_read();  // the previous tile's bulk store has read the staging rows
         }
+        named_bar(tbar, 128);
+        if (j < dv) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) stg[e * dv + j] = r[e >> 4][e & 15];
+        }
+        fence_async_smem();
         tc_fence_before();
-        named_bar(1, kChain);
+        named_bar(tbar, 128);
+        if (issuer) {
+          bulk_store(p.o + ((long)bh * N + (long)f * L + t0) * dv, stg, (uint32_t)(tl * dv * 4));
+          bulk_commit();
+          if (next_pending) qbad = !q_mma(false);
+        }
       }
       // the staging rows (the tile-A half of the mirror) are rewritten by the next frame
       if (issuer) bulk_wait_read();
-      if (failed) break;
+      if (bar_sync_or(1, kChain, failed ? 1 : 0)) {
+        failed = true;
+        break;
+      }
     }
     if (failed) {
-      if (tid == 0 && !*abort_flag) latch_status(p.status, GDN_ERR_TIMEOUT);
+      if (tid == 0) latch_status(p.status, GDN_ERR_TIMEOUT);  // the first code latched wins
       *abort_flag = 1;
     }
     // loads and MMAs issued by thread 0 complete before the CTA exits
-    if (tid == 0) {
-      for (; qw < qi; ++qw) mbar_wait(&bar.q_full[qw & 1], (qw >> 1) & 1u, lim);
-      for (; ow < oi; ++ow) mbar_wait(&bar.o_bar[ow & 1], (ow >> 1) & 1u, lim);
+    if (issuer) {
+      for (; qw < qi; ++qw) mbar_wait(&bar.q_full[tile][qw & 1], (qw >> 1) & 1u, lim);
+      for (; ow < oi; ++ow) mbar_wait(&bar.o_bar[tile][ow & 1], (ow >> 1) & 1u, lim);
     }
     if (issuer) bulk_wait_all();
     named_bar(1, kChain);
