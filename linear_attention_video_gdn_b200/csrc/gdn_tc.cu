@@ -302,11 +302,10 @@ __global__ void __launch_bounds__(kGThreads, 1)
             break;
           }
         }
-        // 1. normalise keys in place (fp16), v to fp16 in place: thread -> token pt/2, block pt%2
+        // 1. normalise keys in place (fp16): thread -> token pt/2, block pt%2
         {
           const int t = pt >> 1, kb = pt & 1;
           uint8_t *krow = slot + SL_KHAT + kb * 8192;
-          uint8_t *vrow = slot + SL_V + kb * 8192;
           uint4 ku[8];
 #pragma unroll
           for (int ch = 0; ch < 8; ++ch) ku[ch] = *reinterpret_cast<const uint4 *>(krow + sw128_offset(t, ch * 8));
@@ -334,11 +333,6 @@ __global__ void __launch_bounds__(kGThreads, 1)
             }
             *reinterpret_cast<uint4 *>(krow + sw128_offset(t, ch * 8)) = make_uint4(o[0], o[1], o[2], o[3]);
           }
-#pragma unroll
-          for (int ch = 0; ch < 8; ++ch) ku[ch] = *reinterpret_cast<const uint4 *>(vrow + sw128_offset(t, ch * 8));
-#pragma unroll
-          for (int ch = 0; ch < 8; ++ch)
-            *reinterpret_cast<uint4 *>(vrow + sw128_offset(t, ch * 8)) = bf16x8_to_f16x8(ku[ch]);
         }
         fence_async_smem();
         tc_fence_before();
@@ -353,6 +347,18 @@ __global__ void __launch_bounds__(kGThreads, 1)
             mma_f16_ss(tmP, sdesc_sw128(a, 16, 1024), sdesc_sw128(a, 16, 1024), idg, kk > 0 ? 1u : 0u);
           }
           mma_commit(&bar.g_bar[grp]);
+        }
+        // v to fp16 in place while the Gram matrix is computed (the chains read
+        // it after w_ready, which follows the fence below)
+        {
+          const int t = pt >> 1, kb = pt & 1;
+          uint8_t *vrow = slot + SL_V + kb * 8192;
+          uint4 vu[8];
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch) vu[ch] = *reinterpret_cast<const uint4 *>(vrow + sw128_offset(t, ch * 8));
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch)
+            *reinterpret_cast<uint4 *>(vrow + sw128_offset(t, ch * 8)) = bf16x8_to_f16x8(vu[ch]);
         }
         {
           const int bad = pt == 0 ? !mbar_wait(&bar.g_bar[grp], gph, lim) : 0;
