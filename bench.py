@@ -201,6 +201,24 @@ def run_reference(args, rank: int):
     print(json.dumps(line), flush=True)
 
 
+def max_over_ranks(value: float, device, world: int) -> float:
+    """The largest per-rank value (the step time of the slowest rank); every rank
+    gets it.  With one rank, the value itself."""
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tokens_per_s(tokens_per_rank: int, world: int, ms_max: float) -> float:
+    """Weak scaling: every rank processes its own copy of the workload, so the job
+    processes world x tokens in the slowest rank's step time."""
+    return world * tokens_per_rank / (ms_max / 1e3)
+
+
 def run_ours(args, rank: int, world: int, local_rank: int):
     import torch
     import torch.distributed as dist
@@ -240,11 +258,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
             step()
         e1.record(stream)
         torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / args.steps
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dev, world)
     if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
         dist.barrier()
     torch.cuda.synchronize()
 
@@ -260,7 +275,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     tr = ncu_traffic() if w.F == 240 else None
     line = {
         "metric": METRIC,
-        "value": world * tokens / (ms / 1e3),
+        "value": whole_job_tokens_per_s(tokens, world, ms),
         "unit": "tokens/s",
         "n_gpus": world,
         "steps": args.steps,
@@ -286,7 +301,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "clocks": clk.summary(),
     }
     if ms_e2e is not None:
-        line["e2e"] = {"value": world * tokens / (ms_e2e / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+        line["e2e"] = {"value": whole_job_tokens_per_s(tokens, world, ms_e2e), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                        "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e,
                        "call": "gdn_frame_fwd_host (C ABI, pinned host buffers, copies + kernel + sync)"}
     if relu is not None:
@@ -313,11 +328,7 @@ def end_to_end_and_relu(args, lib, synth, torch, dist, w, dev, stream, world, ra
         lib.gdn_frame_fwd_host(hq, hk, hv, ha, hb, F=w.F, o=ho, workspace=hws)
     t1.record(stream)
     torch.cuda.synchronize()
-    ms_e2e = t0.elapsed_time(t1) / n_e2e
-    if world > 1:
-        t = torch.tensor([ms_e2e], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_e2e = float(t.item())
+    ms_e2e = max_over_ranks(t0.elapsed_time(t1) / n_e2e, dev, world)
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, ha, hb))
     d2h = ho.numel() * ho.element_size()
     del hws
