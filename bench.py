@@ -46,6 +46,7 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-streaming", action="store_true", help="skip the streaming-call leg")
     ap.add_argument("--frames", type=int, default=0,
                     help="use only the first N latent frames (a smaller case of the same kernel, for profiling)")
     ap.add_argument("--quick", action="store_true",
@@ -305,7 +306,10 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                        "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e,
                        "call": "gdn_frame_fwd_host (C ABI, pinned host buffers, copies + kernel + sync)"}
     if relu is not None:
+        streaming = relu.pop("streaming", None)
         line["relu_la"] = relu
+        if streaming is not None:
+            line["streaming"] = streaming
     if world == 1 and not args.no_cpu_baseline and not args.quick:
         line["cpu_baseline"] = cpu_baseline(w)
     print(json.dumps(line), flush=True)
@@ -358,7 +362,56 @@ def end_to_end_and_relu(args, lib, synth, torch, dist, w, dev, stream, world, ra
         relu = {"workload": "relu_720p_81f", "ms": rms, "tokens_per_s": wr.B * wr.N / (rms / 1e3),
                 "achieved_gbs": rbytes / (rms / 1e3) / 1e9, "frac_hbm": rbytes / (rms / 1e3) / 1e9 / peak}
         del rq, rk, rv, ro, rws
+        relu["streaming"] = None
+        if not args.no_streaming:
+            relu["streaming"] = streaming_leg(lib, synth, torch, dev, stream)
     return ms_e2e, h2d, d2h, relu
+
+
+def streaming_leg(lib, synth, torch, dev, stream):
+    """Streaming decode at the 720p shape: one frame per call (F = 1, 20 heads,
+    920 tokens), 4 calls per frame with fresh q, k, v and gates, the state
+    committed by the 4th.  Timed over 20 frames with the automatic chunk
+    segments and with one CTA per frame (segments = 1)."""
+    ws_ = synth.WORKLOADS["gdn_stream_720p"].with_(F=1)
+    calls = []
+    for c in range(8):  # 8 calls' inputs, cycled (about 100 MB)
+        x = synth.inputs(ws_, call=c)
+        calls.append([torch.from_numpy(x[n]).to(torch.bfloat16).to(dev) for n in "qkv"] +
+                     [torch.from_numpy(x[n]).to(dev) for n in "ab"])
+    o = torch.empty((ws_.B, ws_.H, ws_.L, ws_.dv), dtype=torch.float32, device=dev)
+    s_in = torch.zeros((ws_.B, ws_.H, ws_.dk, ws_.dv), dtype=torch.float32, device=dev)
+    s_out = torch.empty_like(s_in)
+    out = {"workload": "gdn_stream_720p (F=1 per call, 4 calls per frame)", "frames_timed": 20}
+    for tag, segs in (("auto", 0), ("one_cta_per_frame", 1)):
+        o_ = lib.make_opts(lib.DTYPE_BF16, segments=segs)
+        wsb = lib.alloc_workspace(lib.workspace_bytes(lib.OP_GDN, ws_.B, ws_.H, 1, ws_.L, ws_.dk, ws_.dv, o_), dev)
+
+        def frame(i):
+            for st in range(4):
+                q_, k_, v_, a_, b_ = calls[(4 * i + st) % 8]
+                lib.gdn_frame_fwd(q_, k_, v_, a_, b_, F=1, state_in=s_in, state_out=(s_out if st == 3 else None),
+                                  o=o, workspace=wsb, segments=segs)
+
+        for i in range(3):
+            frame(i)
+        torch.cuda.synchronize()
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for i in range(20):
+            frame(i)
+        t1.record(stream)
+        torch.cuda.synchronize()
+        out[f"us_per_call_{tag}"] = t0.elapsed_time(t1) / 80 * 1e3
+    us = out["us_per_call_auto"]
+    # bytes per call: q, k, v (bf16), gates, o (fp32), state in (fp32); +state out on one call in 4
+    nb = ws_.B * ws_.H * (ws_.L * (3 * ws_.dk * 2 + 4 + ws_.dv * 4) + 4 + ws_.dk * ws_.dv * 4 * 1.25)
+    peak, _ = measured_peaks()
+    out.update({"frame_tokens_per_s": ws_.B * ws_.L / (us / 1e6), "alg_bytes_per_call": nb,
+                "achieved_gbs": nb / (us / 1e6) / 1e9, "frac_hbm": nb / (us / 1e6) / 1e9 / peak,
+                "l2": "not flushed; the call is latency-bound (its bytes take about 3 us of HBM time)"})
+    return out
 
 
 def main():

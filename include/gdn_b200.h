@@ -53,7 +53,7 @@ extern "C" {
 #define GDN_API
 #endif
 
-#define GDN_ABI_VERSION 1
+#define GDN_ABI_VERSION 2
 
 /* return / status codes */
 #define GDN_OK 0
@@ -89,9 +89,13 @@ typedef struct gdn_opts {
                              failure and never clear it (caller zeroes it) */
   int max_ctas;           /* 0 = one persistent CTA per SM; else an upper bound (testing) */
   int spin_limit_us;      /* bound on any in-kernel wait; 0 = 2,000,000 us */
-  int test_withhold_unit; /* testing only.  0: off.  u + 1: frame unit u (u = f*B*H + b*H + h) never
-                             publishes its state, so the wait of unit u + B*H expires and the
+  int test_withhold_unit; /* testing only.  0: off.  u + 1: unit u (u = (f*P + s)*B*H + b*H + h,
+                             P segments, P = 1 unless segments are in use) never publishes its
+                             state, so the wait of the unit after it in its chain expires and the
                              kernel reports GDN_ERR_TIMEOUT through *status */
+  int segments;           /* gdn on GDN_IMPL_TC.  0 = automatic; P >= 1: split every frame into P
+                             runs of whole 64-token chunks handled by P CTAs (see gdn_frame_fwd);
+                             P is lowered to the chunk count and to what fits one resident grid */
 } gdn_opts_t;
 
 /*
@@ -114,6 +118,16 @@ typedef struct gdn_opts {
  * GDN_IMPL_TC (others: any size up to 128).  Streaming decode is this call with
  * F = 1, state_in = the cached state and state_out = NULL until the step that
  * commits the frame.
+ *
+ * Segments (GDN_IMPL_TC): when the B*H*F frames are few (streaming calls), a
+ * frame is split into P segments of consecutive 64-token chunks, one CTA each.
+ * Segment s builds its own map (A_s, B_s) over its tokens, so that the frame
+ * state is S = A_{P-1}(...(A_0 (alpha_f S_{f-1}) + B_0)...) + B_{P-1}, the
+ * chain running through the segments in order; every segment then reads out
+ * its tokens against the state after the frame's last segment.  Segments are
+ * used only when all B*H*F*P CTAs fit on the device at once (one cooperative
+ * launch), so no CTA waits for work that has not started.  The automatic
+ * choice takes P > 1 only when at most half the SMs would otherwise be busy.
  *
  * Precision: fp32 inputs use fp32 arithmetic throughout (GDN_IMPL_SEQ /
  * FRAME_SIMT).  bf16 inputs on GDN_IMPL_TC multiply on tensor cores with

@@ -38,7 +38,7 @@ class GdnOpts(ctypes.Structure):
     _fields_ = [("in_dtype", ctypes.c_int), ("gates_are_logits", ctypes.c_int), ("impl", ctypes.c_int),
                 ("stream", ctypes.c_void_p), ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
                 ("status", ctypes.c_void_p), ("max_ctas", ctypes.c_int), ("spin_limit_us", ctypes.c_int),
-                ("test_withhold_unit", ctypes.c_int)]
+                ("test_withhold_unit", ctypes.c_int), ("segments", ctypes.c_int)]
 
 
 _P = ctypes.c_void_p
@@ -94,7 +94,8 @@ def _stream_handle(stream) -> int:
 
 
 def make_opts(in_dtype: int, *, gates_are_logits: bool = True, impl="auto", stream=None, workspace=None,
-              status=None, max_ctas: int = 0, spin_limit_us: int = 0, test_withhold_unit: int = -1) -> GdnOpts:
+              status=None, max_ctas: int = 0, spin_limit_us: int = 0, test_withhold_unit: int = -1,
+              segments: int = 0) -> GdnOpts:
     o = GdnOpts()
     o.in_dtype = in_dtype
     o.gates_are_logits = int(bool(gates_are_logits))
@@ -107,6 +108,7 @@ def make_opts(in_dtype: int, *, gates_are_logits: bool = True, impl="auto", stre
     o.max_ctas = int(max_ctas)
     o.spin_limit_us = int(spin_limit_us)
     o.test_withhold_unit = int(test_withhold_unit) + 1 if test_withhold_unit >= 0 else 0
+    o.segments = int(segments)
     return o
 
 
@@ -136,7 +138,7 @@ def _check(t, name, shape, dtype, device, allow_none=False):
 
 def gdn_frame_fwd(q, k, v, alpha, beta, *, F: int, state_in=None, state_out=None, o=None,
                   gates_are_logits: bool = True, impl="auto", workspace=None, stream=None, status=None,
-                  max_ctas: int = 0, spin_limit_us: int = 0, test_withhold_unit: int = -1):
+                  max_ctas: int = 0, spin_limit_us: int = 0, test_withhold_unit: int = -1, segments: int = 0):
     """Frame-wise Gated DeltaNet forward on the GPU (see include/gdn_b200.h).
 
     q, k: [B, H, F*L, dk]; v: [B, H, F*L, dv] (float32 or bfloat16, same dtype);
@@ -161,7 +163,7 @@ def gdn_frame_fwd(q, k, v, alpha, beta, *, F: int, state_in=None, state_out=None
     _check(o, "o", (B, H, N, dv), torch.float32, dev)
     opts = make_opts(_dtype_code(q), gates_are_logits=gates_are_logits, impl=impl, stream=stream,
                      status=status, max_ctas=max_ctas, spin_limit_us=spin_limit_us,
-                     test_withhold_unit=test_withhold_unit)
+                     test_withhold_unit=test_withhold_unit, segments=segments)
     need = workspace_bytes(OP_GDN, B, H, F, L, dk, dv, opts)
     if workspace is None and need > 0:
         workspace = alloc_workspace(need, dev)

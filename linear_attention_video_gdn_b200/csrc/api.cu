@@ -62,9 +62,58 @@ size_t gdn_state_elems(int impl, int dk, int dv) {
   return (size_t)dk * dv;
 }
 
-size_t gdn_ws_bytes(int impl, int B, int H, int F, int dk, int dv) {
+// Chunk segments per frame (GDN_IMPL_TC).  The automatic choice considers
+// segments only for launches of at most kSegUnitsMax frames, and at most
+// kMaxSegs of them.
+constexpr long kSegUnitsMax = 128;
+constexpr int kMaxSegs = 8;
+
+// The most segments a launch with these sizes and options may use; sizes the
+// workspace without asking the device.
+int gdn_seg_bound(int impl, const gdn_opts_t *o, long units, int L) {
+  if (impl != GDN_IMPL_TC) return 1;
+  const int nch = (L + 63) / 64;
+  if (o->segments > 0) return o->segments < nch ? o->segments : nch;
+  if (units > kSegUnitsMax) return 1;
+  return nch < kMaxSegs ? nch : kMaxSegs;
+}
+
+// The segments of a launch on `sms` SMs: all units * P CTAs must be resident
+// at once.  Automatic: P > 1 only when the frames alone would fill at most
+// half the grid, and then about sqrt(chunks per frame) of them.  A call's time
+// grows by one chunk's latency per chunk in a segment and by one chain step's
+// per segment, and the two were measured about equal (~5.5-6 us each for one
+// 920-token frame of 20 heads: 109 us at P = 1, 74 at 2, 62 at 4, 69 at 8).
+int gdn_segs(int impl, const gdn_opts_t *o, int sms, long units, int L) {
+  int bound = gdn_seg_bound(impl, o, units, L);
+  if (bound <= 1) return 1;
+  long g = sms;
+  if (o->max_ctas > 0 && o->max_ctas < g) g = o->max_ctas;
+  if (o->segments <= 0) {
+    if (2 * units > g) return 1;
+    const int nch = (L + 63) / 64;
+    int want = 1;
+    while (want * want < nch) ++want;
+    if (want < bound) bound = want;
+  }
+  const long fit = g / units;
+  const long P = fit < bound ? fit : bound;
+  return (int)(P < 1 ? 1 : P);
+}
+
+// Workspace of gdn with P segments: the chain scratch over units * P segment
+// units, then (P > 1) each frame's end state as bf16 high/low pairs, d_k
+// words per row of S^T.
+size_t gdn_ws_bytes_p(int impl, int B, int H, int F, int dk, int dv, int P) {
   if (impl == GDN_IMPL_SEQ) return 0;
-  return chain_workspace_bytes((long)B * H * F, (long)gdn_state_elems(impl, dk, dv));
+  const long units = (long)B * H * F;
+  size_t b = chain_workspace_bytes(units * P, (long)gdn_state_elems(impl, dk, dv));
+  if (P > 1) b += align_up(sizeof(uint32_t) * (size_t)units * dk * dv, 256);
+  return b;
+}
+
+size_t gdn_ws_bytes(int impl, const gdn_opts_t *o, int B, int H, int F, int L, int dk, int dv) {
+  return gdn_ws_bytes_p(impl, B, H, F, dk, dv, gdn_seg_bound(impl, o, (long)B * H * F, L));
 }
 
 size_t relu_ws_bytes(int B, int H, int F, int dk, int dv) {
@@ -104,7 +153,7 @@ extern "C" const char *gdn_status_string(int s) {
 
 extern "C" size_t gdn_workspace_bytes(int op, int B, int H, int F, int L, int dk, int dv, const gdn_opts_t *opts) {
   if (!opts || check_sizes(B, H, F, L, dk, dv) != GDN_OK) return 0;
-  if (op == GDN_OP_GDN) return gdn_ws_bytes(pick_gdn_impl(opts, dk, dv), B, H, F, dk, dv);
+  if (op == GDN_OP_GDN) return gdn_ws_bytes(pick_gdn_impl(opts, dk, dv), opts, B, H, F, L, dk, dv);
   if (op == GDN_OP_RELU_LA) return relu_ws_bytes(B, H, F, dk, dv);
   return 0;
 }
@@ -139,20 +188,27 @@ extern "C" int gdn_frame_fwd(const void *q, const void *k, const void *v, const 
   p.status = opts->status;
   p.spin_limit_ns = spin_ns(opts);
   p.withhold = opts->test_withhold_unit > 0 ? (long)opts->test_withhold_unit - 1 : -1;
+  p.segs = 1;
 
   cudaError_t e;
   if (impl == GDN_IMPL_SEQ) {
     e = launch_gdn_seq(p, opts->in_dtype, st);
   } else {
     const long units = (long)B * H * F;
-    const size_t need = gdn_ws_bytes(impl, B, H, F, dk, dv);
+    const int P = gdn_segs(impl, opts, sms, units, L);
+    const size_t need = gdn_ws_bytes_p(impl, B, H, F, dk, dv, P);
     if (!opts->workspace || opts->workspace_bytes < need) return GDN_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(opts->workspace) & 255u) != 0) return GDN_ERR_INVALID_ARG;
-    p.ws = chain_workspace(opts->workspace, units);
-    e = cudaMemsetAsync(opts->workspace, 0, chain_workspace_zero_bytes(units), st);
+    p.ws = chain_workspace(opts->workspace, units * P);
+    p.segs = P;
+    if (P > 1)
+      p.ro_states = reinterpret_cast<uint32_t *>(
+          (char *)opts->workspace + chain_workspace_bytes(units * P, (long)gdn_state_elems(impl, dk, dv)));
+    e = cudaMemsetAsync(opts->workspace, 0, chain_workspace_zero_bytes(units * P), st);
     if (e != cudaSuccess) return GDN_ERR_CUDA;
-    const int grid = grid_for(opts, sms, units);
-    e = impl == GDN_IMPL_TC ? launch_gdn_tc(p, grid, st) : launch_gdn_frame_simt(p, opts->in_dtype, grid, st);
+    const int grid = P > 1 ? (int)(units * P) : grid_for(opts, sms, units);
+    e = impl == GDN_IMPL_TC ? launch_gdn_tc(p, grid, P > 1, st)
+                            : launch_gdn_frame_simt(p, opts->in_dtype, grid, st);
   }
   return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
@@ -232,7 +288,7 @@ HostLayout host_layout(int B, int H, int F, int L, int dk, int dv, int in_dtype,
 
 extern "C" size_t gdn_workspace_bytes_host(int B, int H, int F, int L, int dk, int dv, const gdn_opts_t *opts) {
   if (!opts || check_sizes(B, H, F, L, dk, dv) != GDN_OK) return 0;
-  const size_t ws = gdn_ws_bytes(pick_gdn_impl(opts, dk, dv), B, H, F, dk, dv);
+  const size_t ws = gdn_ws_bytes(pick_gdn_impl(opts, dk, dv), opts, B, H, F, L, dk, dv);
   return host_layout(B, H, F, L, dk, dv, opts->in_dtype, ws).total;
 }
 
@@ -243,7 +299,7 @@ extern "C" int gdn_frame_fwd_host(const void *q, const void *k, const void *v, c
   if (opts->in_dtype != GDN_DTYPE_F32 && opts->in_dtype != GDN_DTYPE_BF16) return GDN_ERR_INVALID_ARG;
   int rc = check_sizes(B, H, F, L, dk, dv);
   if (rc != GDN_OK) return rc;
-  const size_t ws = gdn_ws_bytes(pick_gdn_impl(opts, dk, dv), B, H, F, dk, dv);
+  const size_t ws = gdn_ws_bytes(pick_gdn_impl(opts, dk, dv), opts, B, H, F, L, dk, dv);
   const HostLayout h = host_layout(B, H, F, L, dk, dv, opts->in_dtype, ws);
   if (!opts->workspace || opts->workspace_bytes < h.total) return GDN_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(opts->workspace) & 255u) != 0) return GDN_ERR_INVALID_ARG;

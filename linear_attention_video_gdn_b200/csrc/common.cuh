@@ -103,7 +103,9 @@ struct GdnParams {
   int *status;
   unsigned long long spin_limit_ns;
   long withhold;  // unit that never publishes (testing), -1 = none
-  Workspace ws;
+  Workspace ws;   // flags and published states per segment unit ((b, h, f), then segment)
+  int segs;       // chunk segments per frame (tcgen05 kernel; 1 elsewhere)
+  uint32_t *ro_states;  // segs > 1: per (b, h, f) the end-of-frame S^T rows as bf16 high/low pairs
 };
 
 struct ReluParams {

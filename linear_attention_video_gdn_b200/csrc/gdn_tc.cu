@@ -7,7 +7,11 @@
 // o = S^T q with the state after the whole frame.
 //
 // Work unit = one (b, h, f) frame, taken from a ticket counter (f-major) by a
-// persistent CTA.  For its frame the CTA builds the frame map
+// persistent CTA; with P segments per frame (few frames, e.g. a streaming
+// call) a unit is one run of consecutive chunks of a frame, and the map below
+// is the segment's, chained through the frame's segments in order (alpha_f on
+// the first only), every segment reading out against the frame's last state.
+// For its frame the CTA builds the frame map
 //     S_f = A_f (alpha_f S_{f-1}) + B_f,
 // A_f = ordered product of (I - beta_t khat_t khat_t^T), B_f = the frame's
 // update from a zero state, by running the delta rule on Y = [A | B] from
@@ -184,6 +188,9 @@ __device__ __forceinline__ void blk_row_mul(float4 &acc, const float *A, const f
 }
 __device__ __forceinline__ float4 neg4(float4 v) { return make_float4(-v.x, -v.y, -v.z, -v.w); }
 
+// kSeg: frames split into p.segs chunk segments (else one unit per frame; the
+// segment arithmetic folds away)
+template <bool kSeg>
 __global__ void __launch_bounds__(kGThreads, 1)
     gdn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                   const __grid_constant__ CUtensorMap tmap_v, GdnParams p) {
@@ -194,12 +201,36 @@ __global__ void __launch_bounds__(kGThreads, 1)
   const int warp = tid >> 5;
   const int dk = p.dk, dv = p.dv, L = p.L, F = p.F;
   const int BH = p.B * p.H;
-  const long units = (long)BH * F;
+  const int P = kSeg ? p.segs : 1;     // chunk segments per frame
+  const long units = (long)BH * F * P; // tickets
   const long N = (long)F * L;
   const unsigned long long lim = p.spin_limit_ns;
   const int nkd = dk / 16;            // k-steps over d_k
   const int nch = (L + kC - 1) / kC;  // chunks per frame
   volatile int *abort_flag = &bar.abort;
+  // ticket (f-major, then segment, then b*H + h) -> frame, segment, head and
+  // the segment's chunks [c0, c1)
+  struct Unit {
+    int f, s, bh, c0, c1;
+  };
+  auto unit_of = [&](int tk) -> Unit {
+    Unit u;
+    if (!kSeg) {
+      u.f = tk / BH;
+      u.s = 0;
+      u.bh = tk - u.f * BH;
+      u.c0 = 0;
+      u.c1 = nch;
+      return u;
+    }
+    u.f = tk / (BH * P);
+    const int r = tk - u.f * BH * P;
+    u.s = r / BH;
+    u.bh = r - u.s * BH;
+    u.c0 = u.s * nch / P;
+    u.c1 = (u.s + 1) * nch / P;
+    return u;
+  };
 
   // ---------------------------------------------------------------- set-up
   if (tid == 0) {
@@ -251,11 +282,12 @@ __global__ void __launch_bounds__(kGThreads, 1)
     bar.loads = gg + 1;
     return true;
   };
-  // the first (up to) three chunks of the frame of ticket tk, the g0-th chunk on
+  // the first (up to) three chunks of ticket tk's unit, the g0-th chunk on
   auto issue_frame_kv = [&](int tk, uint32_t g0) -> bool {
     if (tk < 0) return true;
-    for (int c = 0; c < nch && c < kSlots; ++c)
-      if (!issue_kv(g0 + c, tk / BH, tk % BH, c)) return false;
+    const Unit u = unit_of(tk);
+    for (int c = u.c0; c < u.c1 && c < u.c0 + kSlots; ++c)
+      if (!issue_kv(g0 + (c - u.c0), u.f, u.bh, c)) return false;
     return true;
   };
 
@@ -286,7 +318,8 @@ __global__ void __launch_bounds__(kGThreads, 1)
       }
       const int tk = bar.ticket_ring[k & 3];
       if (tk < 0) break;
-      for (int c = 0; c < nch; ++c, ++g) {
+      const int c0 = unit_of(tk).c0, c1 = unit_of(tk).c1;
+      for (int c = c0; c < c1; ++c, ++g) {
         if ((int)(g & 1u) != grp) continue;
         const int s = (int)(g % kSlots);
         const uint32_t ph = (g / kSlots) & 1u;
@@ -294,7 +327,10 @@ __global__ void __launch_bounds__(kGThreads, 1)
         // gate of token pt of the chunk (used from step 3 on, so its load latency is hidden)
         float braw = 0.f;
         const bool bvalid = pt < 64 && c * kC + pt < L;
-        if (bvalid) braw = p.beta[(long)(tk % BH) * N + (long)(tk / BH) * L + c * kC + pt];
+        if (bvalid) {  // the unit decoded again here keeps fewer registers live across the loop
+          const Unit un = unit_of(tk);
+          braw = p.beta[(long)un.bh * N + (long)un.f * L + c * kC + pt];
+        }
         {
           const int bad = pt == 0 ? !mbar_wait(&bar.kv_full[s], ph, lim) : 0;
           if (bar_sync_or(pbar, 128, bad || *abort_flag)) {
@@ -598,10 +634,12 @@ __global__ void __launch_bounds__(kGThreads, 1)
       ++frames;
       if (tk < 0) break;
       const long ticket = tk;
-      const int f = (int)(ticket / BH);
-      const int bh = (int)(ticket % BH);
+      const Unit un = unit_of(tk);
+      // (one unit per frame: the 64-bit forms, which leave the register allocation as it was)
+      const int f = kSeg ? un.f : (int)(ticket / BH), bh = kSeg ? un.bh : (int)(ticket % BH);
+      const int seg = un.s, c0 = un.c0, c1 = un.c1;
       const float a_raw = p.alpha[(long)bh * F + f];
-      const float alpha = p.gates_are_logits ? gate_alpha(a_raw) : a_raw;
+      const float alpha = seg > 0 ? 1.f : (p.gates_are_logits ? gate_alpha(a_raw) : a_raw);
 
       // Y_A^T = I in TMEM (the first chunk accumulates onto it); Y_B^T starts
       // from the first chunk's product
@@ -619,12 +657,12 @@ __global__ void __launch_bounds__(kGThreads, 1)
       named_bar(tbar, 128);
 
       // ---- the frame's chunks, one independent chain per tile
-      for (int c = 0; c < nch; ++c, ++g) {
+      for (int c = c0; c < c1; ++c, ++g) {
         const int s = (int)(g % kSlots);
         const uint32_t ph = (g / kSlots) & 1u;
         uint8_t *slot = sm + OFF_SLOT + s * SLOT_BYTES;
         int cbad = 0;
-        if (c > 0) {
+        if (c > c0) {
           // R^T = -Y^T Khat^T (the [0 ; V^T] target enters with the W product)
           if (issuer) {
             if (!mbar_wait(&bar.khat_ready[s], ph, lim)) cbad = 1;
@@ -670,7 +708,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
           if (!mbar_wait(&bar.w_ready[s], ph, lim)) cbad = 1;
           tc_fence_after();
           const uint32_t wb = smem_u32(slot + SL_W);
-          if (c > 0) {
+          if (c > c0) {
             for (int kk = 0; kk < 4; ++kk)
               mma_f16_ts(tmY, tmR + kk * 8, sdesc_sw128(wb + kk * 32, 16, 1024), id_y, 1u);
           } else if (tile == 0) {
@@ -683,7 +721,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
             const uint32_t vb = smem_u32(slot + SL_V);
             for (int kk = 0; kk < 4; ++kk)
               mma_f16_ss(tmY, sdesc_sw128(vb + kk * 2048, 8192, 1024), sdesc_sw128(wb + kk * 32, 16, 1024), id_vw,
-                         (c > 0 || kk > 0) ? 1u : 0u);
+                         (c > c0 || kk > 0) ? 1u : 0u);
           }
           mma_commit(&bar.mma_bar[tile]);
           mma_commit(&bar.slot_free[s]);
@@ -694,14 +732,14 @@ __global__ void __launch_bounds__(kGThreads, 1)
         }
         tc_fence_after();
         // slot s is free once both tiles' last MMAs on it are done: chunk c + 3 goes there
-        if (tile == 1 && issuer && c + kSlots < nch && !issue_kv(g + kSlots, f, bh, c + kSlots)) {
+        if (tile == 1 && issuer && c + kSlots < c1 && !issue_kv(g + kSlots, f, bh, c + kSlots)) {
           *abort_flag = 1;
           latch_status(p.status, GDN_ERR_TIMEOUT);
         }
         // Y^T rows -> fp16 mirror (tile B's rows are not needed after the last
         // chunk; tile A's last copy is alpha_f A_f^T for the chain step)
-        if (c + 1 < nch || tile == 0) {
-          const float sc = c + 1 < nch ? 1.f : alpha;
+        if (c + 1 < c1 || tile == 0) {
+          const float sc = c + 1 < c1 ? 1.f : alpha;
 #pragma unroll
           for (int hb = 0; hb < 4; ++hb) {  // batches of up to 2 column blocks
             if (2 * hb >= nkd) break;
@@ -730,16 +768,21 @@ __global__ void __launch_bounds__(kGThreads, 1)
       }
 
       // ---- chain step: S_f^T = B_f^T + S_{f-1}^T (alpha A_f^T)
+      const long uidx = ((long)bh * F + f) * P + seg;  // this unit's flag and published state
       // read-out tiles of this chain: tile-chain A takes tiles 0, 2, 4, ...; B 1, 3, 5, ...
-      const int nq = ((L + kQTok - 1) / kQTok - tile + 1) / 2;
+      const int tb0 = c0 * kC, tb1 = (kSeg && c1 * kC < L) ? c1 * kC : L;  // the unit's tokens
+      const int nq = ((tb1 - tb0 + kQTok - 1) / kQTok - tile + 1) / 2;
       if (issuer) {  // its first q tiles -> the tile-B half of the mirror (free now)
-        if (nq > 0) issue_q(f, bh, tile * kQTok);
-        if (nq > 1) issue_q(f, bh, (2 + tile) * kQTok);
+        if (nq > 0) issue_q(f, bh, tb0 + tile * kQTok);
+        if (nq > 1) issue_q(f, bh, tb0 + (2 + tile) * kQTok);
       }
-      const bool have_prev = f > 0 || p.state_in != nullptr;
+      // the state before this unit: the previous segment's, or the previous
+      // frame's last segment's (unit uidx - 1 either way), else state_in
+      const bool chained = f > 0 || seg > 0;
+      const bool have_prev = chained || p.state_in != nullptr;
       {
         int bad = 0;
-        if (tid == 0 && f > 0) bad = !wait_flag(p.ws.flags + (long)bh * F + (f - 1), 1, lim);
+        if (tid == 0 && chained) bad = !wait_flag(p.ws.flags + uidx - 1, 1, lim);
         if (bar_sync_or(1, kChain, bad || *abort_flag)) {
           failed = true;
           break;
@@ -751,11 +794,10 @@ __global__ void __launch_bounds__(kGThreads, 1)
       if (have_prev) {
         // S_{f-1}^T row j as fp16 pairs into TMEM columns [256, 256 + d_k / 2) (A operand)
         if (nl > 0) {
-          if (f > 0) {
+          if (chained) {
             // published rows S^T[j][l] (fp16, d_k per row): the pairs are the loaded words
             const uint4 *src = reinterpret_cast<const uint4 *>(
-                reinterpret_cast<const __half *>(p.ws.states) + ((long)bh * F + (f - 1)) * (long)dk * dv +
-                (long)j * dk + l0);
+                reinterpret_cast<const __half *>(p.ws.states) + (uidx - 1) * (long)dk * dv + (long)j * dk + l0);
             uint4 u[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e)
@@ -807,11 +849,14 @@ __global__ void __launch_bounds__(kGThreads, 1)
         tc_fence_after();
       }
       // S_f^T row j (this thread's half of l): an fp16 row into the staging
-      // area (one bulk store to the workspace, for the next frame), bf16
-      // high/low pairs into TMEM [0, 128) (the read-out's A operand), and the
-      // fp32 state_out after the last frame
+      // area (one bulk store to the workspace, for the next unit), bf16
+      // high/low pairs into TMEM [0, 128) (the read-out's A operand) and, from
+      // a frame's last segment of several, to the workspace for the others'
+      // read-outs, and the fp32 state_out after the last frame
+      const bool last_seg = seg == P - 1;
+      uint32_t *ro = (P > 1 && last_seg && j < dv) ? p.ro_states + (((long)bh * F + f) * dv + j) * dk : nullptr;
       {
-        float *sout = (f == F - 1 && p.state_out) ? p.state_out + (long)bh * dk * dv : nullptr;
+        float *sout = (f == F - 1 && last_seg && p.state_out) ? p.state_out + (long)bh * dk * dv : nullptr;
         __half *srow = reinterpret_cast<__half *>(sm + OFF_STAGE) + (long)j * dk + l0;
 #pragma unroll 1
         for (int h2 = 0; h2 < 4; ++h2) {  // 16 columns l at a time
@@ -841,22 +886,31 @@ __global__ void __launch_bounds__(kGThreads, 1)
 #pragma unroll
               for (int e = 0; e < 16; ++e) sout[(long)(lb + e) * dv + j] = r[e];
             }
+            if (ro) {  // row j: high pairs in words [0, d_k / 2), low pairs in [d_k / 2, d_k)
+              uint4 *rh = reinterpret_cast<uint4 *>(ro + lb / 2);
+              uint4 *rl = reinterpret_cast<uint4 *>(ro + dk / 2 + lb / 2);
+              rh[0] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+              rh[1] = make_uint4(hi[4], hi[5], hi[6], hi[7]);
+              rl[0] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+              rl[1] = make_uint4(lo[4], lo[5], lo[6], lo[7]);
+            }
           }
         }
       }
+      if (ro) __threadfence();  // before thread 0 releases the flag
       tmem_st_wait();
       fence_async_smem();
       tc_fence_before();
       named_bar(1, kChain);
       if (tid == 0) {
-        __half *dst = reinterpret_cast<__half *>(p.ws.states) + ((long)bh * F + f) * (long)dk * dv;
+        __half *dst = reinterpret_cast<__half *>(p.ws.states) + uidx * (long)dk * dv;
         bulk_store(dst, sm + OFF_STAGE, (uint32_t)(dk * dv * 2));
         bulk_commit();
         bulk_wait_all();
         if (ticket != p.withhold) {
           fence_async_global();
           __threadfence();
-          st_release(p.ws.flags + (long)bh * F + f, 1);
+          st_release(p.ws.flags + uidx, 1);
         }
         const long t = atomicAdd(p.ws.counter, 1);
         const int tkn = (int)(t < units ? t : -1);
@@ -875,6 +929,35 @@ __global__ void __launch_bounds__(kGThreads, 1)
       // O^T through shared memory into O's row-major layout and the issuer
       // bulk-stores the 32 tokens.
       named_bar(1, kChain);  // thread 0's bulk store of S_f has read the staging area
+      if (!last_seg) {
+        // the frame's state is the last segment's: its bf16 high/low rows
+        // replace this unit's in TMEM [0, 128)
+        int bad = 0;
+        if (tid == 0) bad = !wait_flag(p.ws.flags + uidx - seg + (P - 1), 1, lim);
+        if (bar_sync_or(1, kChain, bad || *abort_flag)) {
+          failed = true;
+          break;
+        }
+        const uint4 *src = reinterpret_cast<const uint4 *>(p.ro_states + (((long)bh * F + f) * dv + j) * dk);
+#pragma unroll 1
+        for (int h2 = 0; h2 < 4; ++h2) {
+          if (16 * h2 >= nl) break;
+          const int lb = l0 + 16 * h2;
+          uint4 a[4];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            a[e] = j < dv ? __ldcg(src + lb / 8 + e) : make_uint4(0u, 0u, 0u, 0u);
+            a[2 + e] = j < dv ? __ldcg(src + dk / 8 + lb / 8 + e) : make_uint4(0u, 0u, 0u, 0u);
+          }
+          const uint32_t hi[8] = {a[0].x, a[0].y, a[0].z, a[0].w, a[1].x, a[1].y, a[1].z, a[1].w};
+          const uint32_t lo[8] = {a[2].x, a[2].y, a[2].z, a[2].w, a[3].x, a[3].y, a[3].z, a[3].w};
+          tmem_st8u(tmem + TM_Y + lane_off + lb / 2, hi);
+          tmem_st8u(tmem + TM_Y + 64 + lane_off + lb / 2, lo);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        named_bar(1, kChain);
+      }
       auto q_mma = [&](bool poll) -> int {  // the tile's issuer; with `poll` only if the q tile is in (else 2)
         const int b = qw & 1;
         if (poll) {
@@ -910,8 +993,8 @@ __global__ void __launch_bounds__(kGThreads, 1)
         }
         ++ow;
         tc_fence_after();
-        const int t0 = (2 * qc + tile) * kQTok;
-        const int tl = L - t0 < kQTok ? L - t0 : kQTok;  // tokens of this tile
+        const int t0 = tb0 + (2 * qc + tile) * kQTok;
+        const int tl = tb1 - t0 < kQTok ? tb1 - t0 : kQTok;  // tokens of this tile
         float r[2][16];
         tmem_ld16(tmO + b * 32 + lane_off, r[0]);
         tmem_ld16(tmO + b * 32 + lane_off + 16, r[1]);
@@ -920,7 +1003,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
         // starts now if its q tile is in, else after this epilogue
         bool next_pending = false;
         if (issuer) {
-          if (qc + 2 < nq) issue_q(f, bh, (2 * (qc + 2) + tile) * kQTok);
+          if (qc + 2 < nq) issue_q(f, bh, tb0 + (2 * (qc + 2) + tile) * kQTok);
           if (qc + 1 < nq) next_pending = q_mma(true) == 2;
           bulk_wait_read();  // the previous tile's bulk store has read the staging rows
         }
@@ -977,18 +1060,34 @@ bool gdn_tc_supported(int dk, int dv) {
 // published frame states are fp16 rows S^T[j][l]: d_k * d_v halves = d_k * d_v / 2 floats
 size_t gdn_tc_state_elems(int dk, int dv) { return (size_t)dk * dv / 2; }
 
-cudaError_t launch_gdn_tc(const GdnParams &p, int grid, cudaStream_t st) {
+cudaError_t launch_gdn_tc(const GdnParams &p, int grid, bool cooperative, cudaStream_t st) {
   using namespace tc;
   CUtensorMap mq, mk, mv;
   const int BH = p.B * p.H;
   if (!make_bf16_map(&mq, p.q, p.dk, p.L, p.F, BH, kQTok) || !make_bf16_map(&mk, p.k, p.dk, p.L, p.F, BH, 64) ||
       !make_bf16_map(&mv, p.v, p.dv, p.L, p.F, BH, 64))
     return cudaErrorInvalidValue;
+  if (!cooperative) {  // one unit per frame
+    cudaError_t e =
+        cudaFuncSetAttribute(gdn_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGdnSmemBytes);
+    if (e != cudaSuccess) return e;
+    gdn_tc_kernel<false><<<grid, kGThreads, kGdnSmemBytes, st>>>(mq, mk, mv, p);
+    return cudaGetLastError();
+  }
   cudaError_t e =
-      cudaFuncSetAttribute(gdn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGdnSmemBytes);
+      cudaFuncSetAttribute(gdn_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGdnSmemBytes);
   if (e != cudaSuccess) return e;
-  gdn_tc_kernel<<<grid, kGThreads, kGdnSmemBytes, st>>>(mq, mk, mv, p);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(kGThreads);
+  cfg.dynamicSmemBytes = kGdnSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeCooperative;
+  at[0].val.cooperative = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, gdn_tc_kernel<true>, mq, mk, mv, p);
 }
 
 }  // namespace gdn

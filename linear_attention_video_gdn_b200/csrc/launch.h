@@ -12,7 +12,8 @@ cudaError_t launch_relu_frame_simt(const ReluParams &p, int in_dtype, int grid, 
 // tcgen05 / TMEM / TMA kernels (bf16 inputs, dk = dv in {16..128} multiples of 16).
 bool gdn_tc_supported(int dk, int dv);
 size_t gdn_tc_state_elems(int dk, int dv);
-cudaError_t launch_gdn_tc(const GdnParams &p, int grid, cudaStream_t st);
+// cooperative: p.segs > 1; all CTAs resident at once (segments wait across CTAs both ways)
+cudaError_t launch_gdn_tc(const GdnParams &p, int grid, bool cooperative, cudaStream_t st);
 bool relu_tc_supported(int dk, int dv);
 cudaError_t launch_relu_tc(const ReluParams &p, int grid, cudaStream_t st);
 

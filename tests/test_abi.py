@@ -69,6 +69,31 @@ def test_workspace_sizes(lib):
     assert lib.workspace_bytes(lib.OP_GDN, B, H, F, L, d, d, seq) == 0
 
 
+def test_workspace_sizes_with_segments(lib):
+    """The tcgen05 path sizes its scratch for the most chunk segments a launch
+    may use: fp16 states and flags per segment unit, plus one bf16 high/low
+    end state per frame; one segment for many frames or one-chunk frames."""
+    d = 112
+
+    def need(B, H, F, L, **kw):
+        return lib.workspace_bytes(lib.OP_GDN, B, H, F, L, d, d, lib.make_opts(lib.DTYPE_BF16, impl="tc", stream=0,
+                                                                               **kw))
+
+    def layout(units, P):  # counter block, flags, fp16 states, then the end states (P > 1)
+        up = lambda x: (x + 255) // 256 * 256
+        return 256 + up(4 * units * P) + up(units * P * d * d * 2) + (up(units * d * d * 4) if P > 1 else 0)
+
+    nch = (920 + 63) // 64
+    assert need(1, 20, 1, 920) == layout(20, min(nch, 8))                 # a streaming call: auto bound
+    assert need(1, 20, 1, 920, segments=1) == layout(20, 1)
+    assert need(1, 20, 1, 920, segments=3) == layout(20, 3)
+    assert need(1, 20, 1, 920, segments=99) == layout(20, nch)             # at most one chunk each
+    assert need(1, 20, 240, 920) == layout(4800, 1)                        # many frames: one segment
+    assert need(1, 20, 1, 64) == layout(20, 1)                             # one chunk per frame
+    simt = lib.make_opts(lib.DTYPE_BF16, impl="frame_simt", stream=0, segments=4)
+    assert lib.workspace_bytes(lib.OP_GDN, 1, 20, 1, 920, d, d, simt) == 256 + 256 + 20 * d * d * 4
+
+
 def test_host_argument_validation(lib):
     raw = lib._lib
     o = lib.make_opts(lib.DTYPE_BF16, stream=0)

@@ -256,3 +256,64 @@ def test_device_timeout_status_is_reported(lib, dev):
         assert int(status[0].item()) == 0
         o_ref, s_ref = oracle_gdn(h, w)
         assert rel_err(o, o_ref) <= 2e-3
+
+
+# ------------------------------------------------------------------ frames split into chunk segments
+
+SEG_SHAPES = [  # (B, H, F, L, dk, dv): several chunks per frame, ragged last chunk, dk != dv
+    (1, 2, 1, 390, 112, 112), (2, 3, 3, 300, 112, 112), (1, 1, 2, 200, 48, 80), (1, 4, 1, 129, 128, 128),
+]
+
+
+@pytest.mark.parametrize("B,H,F,L,dk,dv", SEG_SHAPES)
+def test_segments_match_oracle(lib, dev, B, H, F, L, dk, dv):
+    """A frame split into P segments (each its own CTA, chained in order, all
+    reading out against the frame's last state) matches the oracle for every P."""
+    w = W["gdn_480p_5s"].with_(B=B, H=H, F=F, L=L, dk=dk, dv=dv, seed=7 + L)
+    x = synth.inputs(w)
+    t, h = device_inputs(w, x, dev, torch)
+    S0 = np.random.default_rng(L + 1).standard_normal((B, H, dk, dv)).astype(np.float32)
+    o_ref, s_ref = oracle_gdn(h, w, state_in=S0)
+    nch = (L + 63) // 64
+    outs = {}
+    for P in sorted({0, 1, 2, 3, nch}):
+        o, s = run_gdn(lib, w, t, dev, "tc", state_in=S0, segments=P)
+        assert rel_err(o, o_ref) <= 2e-3, P
+        assert rel_err(s, s_ref) <= 2e-3, P
+        outs[P] = o
+    # the automatic choice splits these frames (few frames, several chunks)
+    assert not np.array_equal(outs[0], outs[1]) or nch == 1
+
+
+def test_streaming_frame_720p_segments(lib, dev):
+    """One 720p frame of 20 heads (the streaming call) against the oracle, with
+    the automatic segment count, one segment, and state_out left unwritten."""
+    w = W["gdn_720p_60s"].with_(F=1, seed=11)
+    x = synth.inputs(w)
+    t, h = device_inputs(w, x, dev, torch)
+    S0 = 0.1 * np.random.default_rng(3).standard_normal((w.B, w.H, w.dk, w.dv)).astype(np.float32)
+    o_ref, s_ref = oracle_gdn(h, w, state_in=S0)
+    for P in (0, 1):
+        o, s = run_gdn(lib, w, t, dev, "tc", state_in=S0, segments=P)
+        assert rel_err(o, o_ref) <= 2e-3, P
+        assert rel_err(s, s_ref) <= 2e-3, P
+        o2, _ = run_gdn(lib, w, t, dev, "tc", state_in=S0, want_state=False, segments=P)
+        np.testing.assert_array_equal(o2, o)
+
+
+def test_segment_timeout_status_is_reported(lib, dev):
+    """In segment mode a withheld segment state makes the next segment's chain
+    wait and the earlier segment's read-out wait run out; both end cleanly."""
+    w = W["gdn_480p_5s"].with_(B=2, H=1, F=1, L=200)
+    x = synth.inputs(w)
+    t, h = device_inputs(w, x, dev, torch)
+    status = torch.zeros(4, dtype=torch.int32, device=dev)
+    # tickets (f, segment, b*H + h): ticket 0 = segment 0 of head 0
+    run_gdn(lib, w, t, dev, "tc", spin_limit_us=2000, status=status, test_withhold_unit=0, segments=2)
+    assert int(status[0].item()) == lib.ERR_TIMEOUT
+    status.zero_()
+    o, s = run_gdn(lib, w, t, dev, "tc", status=status, segments=2)
+    assert int(status[0].item()) == 0
+    o_ref, s_ref = oracle_gdn(h, w)
+    assert rel_err(o, o_ref) <= 2e-3
+    assert rel_err(s, s_ref) <= 2e-3
