@@ -30,7 +30,8 @@
 //                   TMEM, and an fp16 copy of Y^T in shared memory for the next
 //                   chunk.  The first chunk of a frame starts from Y = [I | 0],
 //                   so its R^T is -Khat^T and [0 | V] directly.  Together the
-//                   eight warps run the chain step, publish S_f and read out.
+//                   eight warps run the chain step and publish S_f; in the
+//                   read-out thread 0 issues the MMAs and warps 4-7 store O.
 //   warps 8-11, 12-15  two prep groups for even and odd chunks: gates beta,
 //                   key normalisation (fp16 khat), v to fp16, Gram matrix Khat
 //                   Khat^T on tcgen05, T by blocked inversion of the unit lower
@@ -41,8 +42,9 @@
 // chunks as soon as its ticket is taken).
 // The frame chain passes S_f between CTAs as fp16 rows S_f^T[j][l] (one bulk
 // store out, 16-byte loads in); alpha_f is folded into the fp16 copy of A_f.
-// The read-out takes S_f as a bf16 high/low pair (two MMAs on bf16 q) and
-// leaves through shared memory with bulk stores.
+// The read-out takes S_f as a bf16 high/low pair (two MMAs on bf16 q) in
+// 64-token tiles: thread 0 issues the MMAs one tile ahead while warps 4-7 move
+// the previous tile through shared memory to a bulk store.
 // Operands that are not exact in bf16 (khat, v after the cast, Y, R, T, W, A_f,
 // S_{f-1}) enter the tensor cores as fp16 (11-bit significands); all
 // accumulation is fp32.
@@ -57,7 +59,7 @@ constexpr int kChain = 256;      // warps 0-7
 constexpr int kGThreads = 512;   // + two prep warpgroups
 constexpr int kC = 64;           // tokens per chunk
 constexpr int kSlots = 3;        // chunks in flight (k, v, W)
-constexpr int kQTok = 32;        // tokens per read-out tile (tile chain A takes even tiles, B odd ones)
+constexpr int kQTok = 64;        // tokens per read-out tile
 
 // shared memory map (bytes from the 1024-aligned base)
 constexpr uint32_t OFF_MIRROR = 0;       // 64 KB: Y^T as fp16, [tile][k-block][128 rows][128 B]
@@ -71,8 +73,8 @@ constexpr uint32_t OFF_T = OFF_SLOT + kSlots * SLOT_BYTES;  // 2 x 8 KB: T fp16 
 constexpr uint32_t OFF_BAR = OFF_T + 2 * 8192;              // barriers and small state
 // frame-end aliases: the tile-B half of the mirror is free after the last
 // chunk, the tile-A half once the chain step has read alpha A_f^T
-constexpr uint32_t OFF_STAGE = OFF_MIRROR;        // 28 KB: fp16 rows of S_f, then fp32 rows of O, for bulk stores
-constexpr uint32_t OFF_QB = OFF_MIRROR + 32768;   // per tile chain two q tiles (bf16) [k-block][32 t][128 B]
+constexpr uint32_t OFF_STAGE = OFF_MIRROR;        // 32 KB: fp16 rows of S_f, then fp32 rows of O (64 tokens)
+constexpr uint32_t OFF_QB = OFF_MIRROR + 32768;   // two q tiles (bf16) [k-block][64 t][128 B], 16 KB each
 
 struct Bars {
   uint64_t kv_full[kSlots];     // TMA bytes of k and v
@@ -82,8 +84,9 @@ struct Bars {
   uint64_t g_bar[2];            // per prep group: its MMAs
   uint64_t mma_bar[2];          // per tile chain
   uint64_t fr_bar;              // frame-level MMAs (chain step)
-  uint64_t q_full[2][2];        // [tile chain][buffer]
-  uint64_t o_bar[2][2];         // [tile chain][buffer]: read-out MMA into that O buffer
+  uint64_t q_full[2];           // read-out: q tile in buffer b
+  uint64_t o_full[2];           // read-out: the MMAs into O buffer b are done
+  uint64_t o_free[2];           // read-out: the epilogue has read O buffer b
   uint64_t tkt_bar[2];          // chain group -> prep groups: next frame's ticket
   uint32_t tmem_base;
   int abort;
@@ -98,8 +101,8 @@ static_assert(kGdnSmemBytes <= 232448, "shared memory budget");
 constexpr uint32_t TM_Y = 0;     // Y^T: tile A [0,128), tile B [128,256); read-out: S_f^T as bf16 pairs,
                                  // high parts [0,64), low parts [64,128)
 constexpr uint32_t TM_R = 256;   // R^T: tile A [256,320), tile B [320,384); chain step: S^T pairs
-                                 // [256,320); read-out: O buffers, 32 columns each, tile A [256,320),
-                                 // tile B [320,384)
+                                 // [256,320); read-out: O buffers, 64 columns each, [256,320) and
+                                 // [320,384)
 constexpr uint32_t TM_P = 384;   // prep group g: [384 + 64 g, 448 + 64 g): Gram matrix, then W^T
 
 __device__ __forceinline__ void named_bar(int id, int n) {
@@ -243,10 +246,9 @@ __global__ void __launch_bounds__(kGThreads, 1)
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bar.g_bar[s], 1);
       mbar_init(&bar.mma_bar[s], 1);
-      mbar_init(&bar.q_full[0][s], 1);
-      mbar_init(&bar.q_full[1][s], 1);
-      mbar_init(&bar.o_bar[0][s], 1);
-      mbar_init(&bar.o_bar[1][s], 1);
+      mbar_init(&bar.q_full[s], 1);
+      mbar_init(&bar.o_full[s], 1);
+      mbar_init(&bar.o_free[s], 1);
       mbar_init(&bar.tkt_bar[s], 1);
     }
     mbar_init(&bar.fr_bar, 1);
@@ -574,10 +576,11 @@ __global__ void __launch_bounds__(kGThreads, 1)
     uint8_t *mir = sm + OFF_MIRROR + tile * 32768;
     uint32_t tphase = 0;                  // phase of mma_bar[tile]
     uint32_t fphase = 0;                  // phase of fr_bar
-    // this tile chain's read-out tiles over the CTA's lifetime: q loads issued /
+    // read-out tiles over the CTA's lifetime (thread 0): q loads issued /
     // waited for, MMAs issued / waited for; tile n uses q buffer n & 1 and O
     // buffer n & 1
     uint32_t qi = 0, qw = 0, oi = 0, ow = 0;
+    uint32_t rt = 0;  // read-out tiles of earlier units
     int frames = 0;
     bool failed = false;
     uint32_t g = 0;
@@ -587,8 +590,8 @@ __global__ void __launch_bounds__(kGThreads, 1)
     const uint32_t id_kw = idesc_f16(128, dk, 0, 1, 0, 1, 0);   // -(Khat^T) (MN) x W
     const uint32_t id_s = idesc_f16(128, dk, 0, 0, 1);          // (alpha S^T, TMEM) x A^T (MN)
     const uint32_t id_o = idesc_f16(128, kQTok, 1, 0, 0);       // S^T (bf16 pairs, TMEM) x Q^T (bf16)
-    uint8_t *qbuf = sm + OFF_QB + tile * 16384;                  // this chain's q buffers, 8 KB each
-    const uint32_t tmO = tmem + TM_R + tile * 64;                // this chain's O buffers, 32 columns each
+    uint8_t *qbuf = sm + OFF_QB;                                 // q buffers, 16 KB each
+    const uint32_t tmO = tmem + TM_R;                            // O buffers, 64 columns each
 
     // Wait for this tile's MMAs: the issuing thread polls the mbarrier, the
     // others wait on the named barrier (which takes no issue slots from the
@@ -606,12 +609,12 @@ __global__ void __launch_bounds__(kGThreads, 1)
       if (tid == 0) bad = !mbar_wait(b, parity, lim);
       return !bar_sync_or(1, kChain, bad || *abort_flag);
     };
-    auto issue_q = [&](int f, int bh, int t0) {  // the tile's issuer
+    auto issue_q = [&](int f, int bh, int t0) {  // thread 0
       const int bq = qi & 1;
-      mbar_expect_tx(&bar.q_full[tile][bq], 8192);
-      uint8_t *qb = qbuf + bq * 8192;
-      tma_load_4d(qb, &tmap_q, &bar.q_full[tile][bq], 0, t0, f, bh);
-      tma_load_4d(qb + 4096, &tmap_q, &bar.q_full[tile][bq], 64, t0, f, bh);
+      mbar_expect_tx(&bar.q_full[bq], 16384);
+      uint8_t *qb = qbuf + bq * 16384;
+      tma_load_4d(qb, &tmap_q, &bar.q_full[bq], 0, t0, f, bh);
+      tma_load_4d(qb + 8192, &tmap_q, &bar.q_full[bq], 64, t0, f, bh);
       ++qi;
     };
 
@@ -771,10 +774,10 @@ __global__ void __launch_bounds__(kGThreads, 1)
       const long uidx = ((long)bh * F + f) * P + seg;  // this unit's flag and published state
       // read-out tiles of this chain: tile-chain A takes tiles 0, 2, 4, ...; B 1, 3, 5, ...
       const int tb0 = c0 * kC, tb1 = (kSeg && c1 * kC < L) ? c1 * kC : L;  // the unit's tokens
-      const int nq = ((tb1 - tb0 + kQTok - 1) / kQTok - tile + 1) / 2;
-      if (issuer) {  // its first q tiles -> the tile-B half of the mirror (free now)
-        if (nq > 0) issue_q(f, bh, tb0 + tile * kQTok);
-        if (nq > 1) issue_q(f, bh, tb0 + (2 + tile) * kQTok);
+      const int nt = (tb1 - tb0 + kQTok - 1) / kQTok;  // read-out tiles
+      if (tid == 0) {  // the first q tiles -> the tile-B half of the mirror (free now)
+        issue_q(f, bh, tb0);
+        if (nt > 1) issue_q(f, bh, tb0 + kQTok);
       }
       // the state before this unit: the previous segment's, or the previous
       // frame's last segment's (unit uidx - 1 either way), else state_in
@@ -922,12 +925,12 @@ __global__ void __launch_bounds__(kGThreads, 1)
         }
       }
 
-      // ---- read-out: O_f = Q_f S_f in 32-token tiles, two independent
-      // pipelines (tile chain A: even tiles, B: odd tiles).  Each chain's
-      // issuer runs O^T = S_f^T Q^T (bf16 high and low parts of S_f from TMEM,
-      // bf16 q) into its TMEM buffer n & 1 one tile ahead; the epilogue moves
-      // O^T through shared memory into O's row-major layout and the issuer
-      // bulk-stores the 32 tokens.
+      // ---- read-out: O_f = Q_f S_f in 64-token tiles.  Thread 0 runs
+      // O^T = S_f^T Q^T (bf16 high and low parts of S_f from TMEM, bf16 q) into
+      // TMEM buffer n & 1 while warps 4-7 (all 128 TMEM lanes) move tile n - 1
+      // through shared memory into O's row-major layout and bulk-store it.  An
+      // MMA's issue holds its thread for its whole duration, so the issuing
+      // thread takes no part in the epilogue.
       named_bar(1, kChain);  // thread 0's bulk store of S_f has read the staging area
       if (!last_seg) {
         // the frame's state is the last segment's: its bf16 high/low rows
@@ -958,71 +961,82 @@ __global__ void __launch_bounds__(kGThreads, 1)
         tc_fence_before();
         named_bar(1, kChain);
       }
-      auto q_mma = [&](bool poll) -> int {  // the tile's issuer; with `poll` only if the q tile is in (else 2)
-        const int b = qw & 1;
-        if (poll) {
-          if (!mbar_try_wait(&bar.q_full[tile][b], (qw >> 1) & 1u)) return 2;
-        } else if (!mbar_wait(&bar.q_full[tile][b], (qw >> 1) & 1u, lim)) {
-          return 0;
-        }
-        ++qw;
-        tc_fence_after();
-        const uint32_t b0 = smem_u32(qbuf + b * 8192);
-        const int bo = oi & 1;
-        for (int hl = 0; hl < 2; ++hl)
-          for (int kk = 0; kk < nkd; ++kk)
-            mma_f16_ts(tmO + bo * 32, tmem + TM_Y + hl * 64 + kk * 8,
-                       sdesc_sw128(b0 + (kk >> 2) * 4096 + (kk & 3) * 32, 16, 1024), id_o,
-                       (hl > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&bar.o_bar[tile][bo]);
-        ++oi;
-        return 1;
-      };
-      int qbad = 0;
-      if (issuer && nq > 0) qbad = !q_mma(false);
-      float *stg = reinterpret_cast<float *>(sm + OFF_STAGE) + tile * kQTok * dv;
-      for (int qc = 0; qc < nq; ++qc) {
-        const int b = ow & 1;
-        {
-          int bad = qbad;
-          if (issuer && !bad) bad = !mbar_wait(&bar.o_bar[tile][b], (ow >> 1) & 1u, lim);
-          if (bar_sync_or(tbar, 128, bad || *abort_flag)) {
-            failed = true;
+      if (tid == 0) {
+        int bad = 0;
+        for (int n = 0; n < nt; ++n) {
+          const uint32_t gt = rt + n, b = gt & 1u, ph = (gt >> 1) & 1u;
+          if (!mbar_wait(&bar.q_full[b], ph, lim)) {
+            bad = 1;
             break;
           }
+          ++qw;
+          if (gt >= 2 && !mbar_wait(&bar.o_free[b], ph ^ 1u, lim)) {  // tile n - 2 has left O buffer b
+            bad = 1;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t b0 = smem_u32(qbuf + b * 16384);
+          for (int hl = 0; hl < 2; ++hl)
+            for (int kk = 0; kk < nkd; ++kk)
+              mma_f16_ts(tmO + b * 64, tmem + TM_Y + hl * 64 + kk * 8,
+                         sdesc_sw128(b0 + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), id_o,
+                         (hl > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(&bar.o_full[b]);
+          ++oi;
+          // q buffer b is free once these MMAs are done: tile n + 2 goes there
+          if (!mbar_wait(&bar.o_full[b], ph, lim)) {
+            bad = 1;
+            break;
+          }
+          ++ow;
+          if (n + 2 < nt) issue_q(f, bh, tb0 + (n + 2) * kQTok);
         }
-        ++ow;
-        tc_fence_after();
-        const int t0 = tb0 + (2 * qc + tile) * kQTok;
-        const int tl = tb1 - t0 < kQTok ? tb1 - t0 : kQTok;  // tokens of this tile
-        float r[2][16];
-        tmem_ld16(tmO + b * 32 + lane_off, r[0]);
-        tmem_ld16(tmO + b * 32 + lane_off + 16, r[1]);
-        tmem_ld_wait();
-        // this tile's q buffer is free: tile qc + 2 goes there; tile qc + 1's MMA
-        // starts now if its q tile is in, else after this epilogue
-        bool next_pending = false;
-        if (issuer) {
-          if (qc + 2 < nq) issue_q(f, bh, tb0 + (2 * (qc + 2) + tile) * kQTok);
-          if (qc + 1 < nq) next_pending = q_mma(true) == 2;
-          bulk_wait_read();  // the previous tile's bulk store has read the staging rows
+        if (bad) {
+          *abort_flag = 1;
+          latch_status(p.status, GDN_ERR_TIMEOUT);
+          failed = true;
         }
-        named_bar(tbar, 128);
-        if (j < dv) {
+      } else if (tile == 1) {
+        float *stg = reinterpret_cast<float *>(sm + OFF_STAGE);
+        for (int n = 0; n < nt; ++n) {
+          const uint32_t gt = rt + n, b = gt & 1u, ph = (gt >> 1) & 1u;
+          {
+            int bad = 0;
+            if (issuer) bad = !mbar_wait(&bar.o_full[b], ph, lim);
+            if (bar_sync_or(tbar, 128, bad || *abort_flag)) {
+              failed = true;
+              break;
+            }
+          }
+          tc_fence_after();
+          if (issuer) bulk_wait_read();  // the previous tile's bulk store has read the staging rows
+          named_bar(tbar, 128);
+#pragma unroll 1
+          for (int hh = 0; hh < 2; ++hh) {  // 32 tokens at a time
+            float r[2][16];
+            tmem_ld16(tmO + b * 64 + lane_off + 32 * hh, r[0]);
+            tmem_ld16(tmO + b * 64 + lane_off + 32 * hh + 16, r[1]);
+            tmem_ld_wait();
+            if (j < dv) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) stg[e * dv + j] = r[e >> 4][e & 15];
-        }
-        fence_async_smem();
-        tc_fence_before();
-        named_bar(tbar, 128);
-        if (issuer) {
-          bulk_store(p.o + ((long)bh * N + (long)f * L + t0) * dv, stg, (uint32_t)(tl * dv * 4));
-          bulk_commit();
-          if (next_pending) qbad = !q_mma(false);
+              for (int e = 0; e < 32; ++e) stg[(32 * hh + e) * dv + j] = r[e >> 4][e & 15];
+            }
+          }
+          tc_fence_before();
+          fence_async_smem();
+          named_bar(tbar, 128);
+          if (issuer) {
+            mbar_arrive_only(&bar.o_free[b]);
+            const int t0 = tb0 + n * kQTok;
+            const int tl = tb1 - t0 < kQTok ? tb1 - t0 : kQTok;  // tokens of this tile
+            bulk_store(p.o + ((long)bh * N + (long)f * L + t0) * dv, stg, (uint32_t)(tl * dv * 4));
+            bulk_commit();
+          }
         }
       }
+      rt += (uint32_t)nt;
       // the staging rows (the tile-A half of the mirror) are rewritten by the next frame
-      if (issuer) bulk_wait_read();
+      if (tid == 128) bulk_wait_read();
       if (bar_sync_or(1, kChain, failed ? 1 : 0)) {
         failed = true;
         break;
@@ -1033,9 +1047,9 @@ __global__ void __launch_bounds__(kGThreads, 1)
       *abort_flag = 1;
     }
     // loads and MMAs issued by thread 0 complete before the CTA exits
-    if (issuer) {
-      for (; qw < qi; ++qw) mbar_wait(&bar.q_full[tile][qw & 1], (qw >> 1) & 1u, lim);
-      for (; ow < oi; ++ow) mbar_wait(&bar.o_bar[tile][ow & 1], (ow >> 1) & 1u, lim);
+    if (tid == 0) {
+      for (; qw < qi; ++qw) mbar_wait(&bar.q_full[qw & 1], (qw >> 1) & 1u, lim);
+      for (; ow < oi; ++ow) mbar_wait(&bar.o_full[ow & 1], (ow >> 1) & 1u, lim);
     }
     if (issuer) bulk_wait_all();
     named_bar(1, kChain);
