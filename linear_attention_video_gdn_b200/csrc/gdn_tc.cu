@@ -915,14 +915,6 @@ __global__ void __launch_bounds__(kGThreads, 1)
           __threadfence();
           st_release(p.ws.flags + uidx, 1);
         }
-        const long t = atomicAdd(p.ws.counter, 1);
-        const int tkn = (int)(t < units ? t : -1);
-        bar.ticket_ring[frames & 3] = tkn;
-        mbar_arrive_only(&bar.tkt_bar[frames & 1]);
-        if (!issue_frame_kv(tkn, g)) {
-          *abort_flag = 1;
-          latch_status(p.status, GDN_ERR_TIMEOUT);
-        }
       }
 
       // ---- read-out: O_f = Q_f S_f in 64-token tiles.  Thread 0 runs
@@ -960,6 +952,18 @@ __global__ void __launch_bounds__(kGThreads, 1)
         tmem_st_wait();
         tc_fence_before();
         named_bar(1, kChain);
+      }
+      // the next ticket, and its first k, v loads, from a thread that is idle in
+      // the read-out (thread 0 issues the read-out MMAs)
+      if (tid == 32) {
+        const long t = atomicAdd(p.ws.counter, 1);
+        const int tkn = (int)(t < units ? t : -1);
+        bar.ticket_ring[frames & 3] = tkn;
+        mbar_arrive_only(&bar.tkt_bar[frames & 1]);
+        if (!issue_frame_kv(tkn, g)) {
+          *abort_flag = 1;
+          latch_status(p.status, GDN_ERR_TIMEOUT);
+        }
       }
       if (tid == 0) {
         int bad = 0;
