@@ -436,7 +436,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
           }
         }
         tc_fence_before();
-        named_bar(pbar, 128);
+        __syncwarp();  // block k's rows of N come from the 16 threads that invert it, in one warp
         // 4. D_k = (I + N_kk)^-1: thread (k, c) solves column c by forward substitution
         if (pt < 64) {
           const int kq = pt >> 4, c = pt & 15;
@@ -851,13 +851,13 @@ __global__ void __launch_bounds__(kGThreads, 1)
         }
         tc_fence_after();
       }
-      // S_f^T row j (this thread's half of l): an fp16 row into the staging
-      // area (one bulk store to the workspace, for the next unit), bf16
-      // high/low pairs into TMEM [0, 128) (the read-out's A operand) and, from
-      // a frame's last segment of several, to the workspace for the others'
-      // read-outs, and the fp32 state_out after the last frame
+      // S_f^T row j (this thread's half of l), in two passes over TMEM: first an
+      // fp16 row into the staging area (one bulk store to the workspace, for
+      // the next unit) and the fp32 state_out after the last frame; then, while
+      // that store drains, bf16 high/low pairs into TMEM [0, 128) (the
+      // read-out's A operand) and, from a frame's last segment of several, to
+      // the workspace for the others' read-outs.  The flag follows both.
       const bool last_seg = seg == P - 1;
-      uint32_t *ro = (P > 1 && last_seg && j < dv) ? p.ro_states + (((long)bh * F + f) * dv + j) * dk : nullptr;
       {
         float *sout = (f == F - 1 && last_seg && p.state_out) ? p.state_out + (long)bh * dk * dv : nullptr;
         __half *srow = reinterpret_cast<__half *>(sm + OFF_STAGE) + (long)j * dk + l0;
@@ -868,47 +868,61 @@ __global__ void __launch_bounds__(kGThreads, 1)
           float r[16];
           tmem_ld16(tmem + TM_Y + 128 + lane_off + lb, r);
           tmem_ld_wait();
-          uint32_t hi[8], lo[8], hf[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float a = j < dv ? r[2 * e] : 0.f;
-            const float b = j < dv ? r[2 * e + 1] : 0.f;
-            const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-            const float2 hb = __bfloat1622float2(h);
-            const __nv_bfloat162 lw = __floats2bfloat162_rn(a - hb.x, b - hb.y);
-            hi[e] = *reinterpret_cast<const uint32_t *>(&h);
-            lo[e] = *reinterpret_cast<const uint32_t *>(&lw);
-            hf[e] = pack_h2(a, b);
-          }
-          tmem_st8u(tmem + TM_Y + lane_off + lb / 2, hi);
-          tmem_st8u(tmem + TM_Y + 64 + lane_off + lb / 2, lo);
           if (j < dv) {
+            uint32_t hf[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) hf[e] = pack_h2(r[2 * e], r[2 * e + 1]);
             *reinterpret_cast<uint4 *>(srow + 16 * h2) = make_uint4(hf[0], hf[1], hf[2], hf[3]);
             *reinterpret_cast<uint4 *>(srow + 16 * h2 + 8) = make_uint4(hf[4], hf[5], hf[6], hf[7]);
             if (sout) {
 #pragma unroll
               for (int e = 0; e < 16; ++e) sout[(long)(lb + e) * dv + j] = r[e];
             }
-            if (ro) {  // row j: high pairs in words [0, d_k / 2), low pairs in [d_k / 2, d_k)
-              uint4 *rh = reinterpret_cast<uint4 *>(ro + lb / 2);
-              uint4 *rl = reinterpret_cast<uint4 *>(ro + dk / 2 + lb / 2);
-              rh[0] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-              rh[1] = make_uint4(hi[4], hi[5], hi[6], hi[7]);
-              rl[0] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-              rl[1] = make_uint4(lo[4], lo[5], lo[6], lo[7]);
-            }
           }
         }
       }
-      if (ro) __threadfence();  // before thread 0 releases the flag
-      tmem_st_wait();
       fence_async_smem();
-      tc_fence_before();
       named_bar(1, kChain);
       if (tid == 0) {
         __half *dst = reinterpret_cast<__half *>(p.ws.states) + uidx * (long)dk * dv;
         bulk_store(dst, sm + OFF_STAGE, (uint32_t)(dk * dv * 2));
         bulk_commit();
+      }
+      uint32_t *ro = (P > 1 && last_seg && j < dv) ? p.ro_states + (((long)bh * F + f) * dv + j) * dk : nullptr;
+#pragma unroll 1
+      for (int h2 = 0; h2 < 4; ++h2) {
+        if (16 * h2 >= nl) break;
+        const int lb = l0 + 16 * h2;
+        float r[16];
+        tmem_ld16(tmem + TM_Y + 128 + lane_off + lb, r);
+        tmem_ld_wait();
+        uint32_t hi[8], lo[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float a = j < dv ? r[2 * e] : 0.f;
+          const float b = j < dv ? r[2 * e + 1] : 0.f;
+          const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+          const float2 hb = __bfloat1622float2(h);
+          const __nv_bfloat162 lw = __floats2bfloat162_rn(a - hb.x, b - hb.y);
+          hi[e] = *reinterpret_cast<const uint32_t *>(&h);
+          lo[e] = *reinterpret_cast<const uint32_t *>(&lw);
+        }
+        tmem_st8u(tmem + TM_Y + lane_off + lb / 2, hi);
+        tmem_st8u(tmem + TM_Y + 64 + lane_off + lb / 2, lo);
+        if (ro) {  // row j: high pairs in words [0, d_k / 2), low pairs in [d_k / 2, d_k)
+          uint4 *rh = reinterpret_cast<uint4 *>(ro + lb / 2);
+          uint4 *rl = reinterpret_cast<uint4 *>(ro + dk / 2 + lb / 2);
+          rh[0] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+          rh[1] = make_uint4(hi[4], hi[5], hi[6], hi[7]);
+          rl[0] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+          rl[1] = make_uint4(lo[4], lo[5], lo[6], lo[7]);
+        }
+      }
+      if (ro) __threadfence();  // before thread 0 releases the flag
+      tmem_st_wait();
+      tc_fence_before();
+      named_bar(1, kChain);
+      if (tid == 0) {
         bulk_wait_all();
         if (ticket != p.withhold) {
           fence_async_global();
