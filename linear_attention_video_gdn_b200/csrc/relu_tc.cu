@@ -14,7 +14,10 @@
 //     once its producer's flag is set (bounded wait), S_f published.
 //  3. Read-out: [num | den] = relu(Q_f) [S_f | z_f] as bf16 hi + lo halves of
 //     the fp32 state (two MMAs, ~16 significant bits), M=128 tokens x N=128;
-//     o = num / (den + eps) in the epilogue, stored as fp32.
+//     o = num / (den + eps) in the epilogue, stored as fp32.  Warps 0-3 apply
+//     relu to each q tile and thread 0 issues its MMAs into TMEM buffer n & 1
+//     (D1's columns are free by then) while warps 4-7 run the epilogue of the
+//     tile before.
 #include "launch.h"
 #include "tc_host.h"
 #include "tc_ptx.cuh"
@@ -32,19 +35,25 @@ struct __align__(1024) ReluSmem {
   uint8_t blo[32768];
   uint64_t full[kStages];
   uint64_t mma_bar;
+  uint64_t d2_full[2];  // read-out: the MMAs into accumulator buffer b are done
+  uint64_t d2_free[2];  // read-out: the epilogue has read buffer b
   uint32_t tmem_base;
   int ticket;
 };
 
-__device__ __forceinline__ void relu_inplace(uint8_t *p, int nbytes, int tid) {
+__device__ __forceinline__ void relu_inplace(uint8_t *p, int nbytes, int tid, int nthreads) {
   const __nv_bfloat162 zero = __float2bfloat162_rn(0.f);
-  for (int i = tid * 16; i < nbytes; i += kThreads * 16) {
+  for (int i = tid * 16; i < nbytes; i += nthreads * 16) {
     uint4 x = *reinterpret_cast<uint4 *>(p + i);
     __nv_bfloat162 *h = reinterpret_cast<__nv_bfloat162 *>(&x);
 #pragma unroll
     for (int e = 0; e < 4; ++e) h[e] = __hmax2(h[e], zero);
     *reinterpret_cast<uint4 *>(p + i) = x;
   }
+}
+
+__device__ __forceinline__ void named_bar(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
@@ -69,6 +78,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) mbar_init(&sm.full[s], 1);
     mbar_init(&sm.mma_bar, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sm.d2_full[b], 1);
+      mbar_init(&sm.d2_free[b], 1);
+    }
     mbar_fence_init();
     tma_prefetch_desc(&tmap_q);
     tma_prefetch_desc(&tmap_k);
@@ -93,6 +106,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t loads = 0;     // loads issued (all threads track the same count)
   uint32_t consumed = 0;  // loads consumed
   uint32_t mma_phase = 0;
+  uint32_t rt = 0;        // read-out tiles of earlier units (buffer n & 1 and its phases)
   bool failed = false;
 
   auto issue_kv = [&](int chunk, int f, int bh) {
@@ -146,7 +160,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int s = consumed % kStages;
       if (!wait_load()) { failed = true; break; }
       ++consumed;
-      relu_inplace(sm.ring[s], 16384, tid);
+      relu_inplace(sm.ring[s], 16384, tid, kThreads);
       if (tid < 64) {
         const uint32_t off = 16384u + (uint32_t)(dv / 64) * 8192u + sw128_offset((uint32_t)tid, (uint32_t)(dv % 64));
         *reinterpret_cast<__nv_bfloat16 *>(sm.ring[s] + off) = __float2bfloat16(1.0f);
@@ -263,46 +277,77 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid != 0) loads += (uint32_t)min(n3, kStages);
 
     // ---- 3. read-out: o = relu(Q) S / (relu(Q) z + eps) ----
-    for (int c = 0; c < n3; ++c) {
-      const int s = consumed % kStages;
-      if (!wait_load()) { failed = true; break; }
-      ++consumed;
-      relu_inplace(sm.ring[s], 32768, tid);
-      fence_async_smem();
-      __syncthreads();
-      if (tid == 0) {
+    if (warp < 4) {
+      for (int c = 0; c < n3; ++c) {
+        const int s = consumed % kStages;
+        {
+          int bad = 0;
+          if (tid == 0) bad = !mbar_wait(&sm.full[s], (consumed / kStages) & 1u, lim);
+          if (bar_sync_or(1, 128, bad)) {
+            failed = true;
+            break;
+          }
+        }
+        ++consumed;
+        relu_inplace(sm.ring[s], 32768, tid, 128);
+        fence_async_smem();
+        named_bar(1, 128);
+        int bad = 0;
+        if (tid == 0) {
+          const uint32_t gt = rt + c, b = gt & 1u, ph = (gt >> 1) & 1u;
+          const uint32_t tD = b ? tD1 : tD2;
+          bad = gt >= 2 && !mbar_wait(&sm.d2_free[b], ph ^ 1u, lim);  // tile n - 2 has left buffer b
+          if (!bad) {
+            tc_fence_after();
+            const uint32_t a0 = smem_u32(sm.ring[s]), bh0 = smem_u32(sm.bhi), bl0 = smem_u32(sm.blo);
+            for (int kk = 0; kk < nk3; ++kk) {
+              const uint32_t off = (uint32_t)(kk / 4) * 16384u + (uint32_t)(kk % 4) * 32u;
+              mma_f16_ss(tD, sdesc_sw128(a0 + off, 16, 1024), sdesc_sw128(bh0 + off, 16, 1024), idesc3,
+                         kk > 0 ? 1u : 0u);
+            }
+            for (int kk = 0; kk < nk3; ++kk) {
+              const uint32_t off = (uint32_t)(kk / 4) * 16384u + (uint32_t)(kk % 4) * 32u;
+              mma_f16_ss(tD, sdesc_sw128(a0 + off, 16, 1024), sdesc_sw128(bl0 + off, 16, 1024), idesc3, 1u);
+            }
+            mma_commit(&sm.d2_full[b]);
+            // the ring stage is free once these MMAs are done: q tile c + 3 goes there
+            if (c + kStages < n3) {
+              bad = !mbar_wait(&sm.d2_full[b], ph, lim);
+              if (!bad) issue_q(c + kStages, f, bh);
+            }
+          }
+        }
+        if (c + kStages < n3) ++loads;
+        if (bar_sync_or(1, 128, bad)) {
+          failed = true;
+          break;
+        }
+      }
+    } else {
+      for (int c = 0; c < n3; ++c) {
+        const uint32_t gt = rt + c, b = gt & 1u;
+        const uint32_t tD = b ? tD1 : tD2;
+        {
+          int bad = 0;
+          if (tid == 128) bad = !mbar_wait(&sm.d2_full[b], (gt >> 1) & 1u, lim);
+          if (bar_sync_or(2, 128, bad)) {
+            failed = true;
+            break;
+          }
+        }
         tc_fence_after();
-        const uint32_t a0 = smem_u32(sm.ring[s]), bh0 = smem_u32(sm.bhi), bl0 = smem_u32(sm.blo);
-        for (int kk = 0; kk < nk3; ++kk) {
-          const uint32_t off = (uint32_t)(kk / 4) * 16384u + (uint32_t)(kk % 4) * 32u;
-          mma_f16_ss(tD2, sdesc_sw128(a0 + off, 16, 1024), sdesc_sw128(bh0 + off, 16, 1024), idesc3,
-                     kk > 0 ? 1u : 0u);
-        }
-        for (int kk = 0; kk < nk3; ++kk) {
-          const uint32_t off = (uint32_t)(kk / 4) * 16384u + (uint32_t)(kk % 4) * 32u;
-          mma_f16_ss(tD2, sdesc_sw128(a0 + off, 16, 1024), sdesc_sw128(bl0 + off, 16, 1024), idesc3, 1u);
-        }
-        mma_commit(&sm.mma_bar);
-      }
-      if (!wait_mma()) { failed = true; break; }
-      tc_fence_after();
-      if (c + kStages < n3) {
-        if (tid == 0) issue_q(c + kStages, f, bh);
-        ++loads;
-      }
-      if (warp >= 4) {
         const int t = c * 128 + (tid - 128);
         float den;
         {
           float r[16];
-          tmem_ld16(tD2 + lane_off + (uint32_t)(dv & ~15), r);
+          tmem_ld16(tD + lane_off + (uint32_t)(dv & ~15), r);
           tmem_ld_wait();
           den = r[dv & 15] + p.eps;
         }
         float *orow = p.o + ((long)bh * N + (long)f * L + t) * dv;
         for (int cb = 0; cb < dv / 16; ++cb) {
           float r[16];
-          tmem_ld16(tD2 + lane_off + cb * 16, r);
+          tmem_ld16(tD + lane_off + cb * 16, r);
           tmem_ld_wait();
           if (t < L) {
             float4 *dst = reinterpret_cast<float4 *>(orow + cb * 16);
@@ -311,11 +356,18 @@ __global__ void __launch_bounds__(kThreads, 1)
               dst[e] = make_float4(r[4 * e] / den, r[4 * e + 1] / den, r[4 * e + 2] / den, r[4 * e + 3] / den);
           }
         }
+        tc_fence_before();
+        named_bar(2, 128);
+        if (tid == 128) mbar_arrive_only(&sm.d2_free[b]);
       }
-      tc_fence_before();
-      __syncthreads();
+      consumed += (uint32_t)n3;
+      loads += (uint32_t)(n3 > kStages ? n3 - kStages : 0);
     }
-    if (failed) break;
+    rt += (uint32_t)n3;
+    if (__syncthreads_or(failed ? 1 : 0)) {
+      failed = true;
+      break;
+    }
   }
   if (failed && tid == 0) latch_status(p.status, GDN_ERR_TIMEOUT);
   tc_fence_before();
