@@ -337,23 +337,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         const int t = c * 128 + (tid - 128);
-        float den;
+        float inv;  // 1 / (relu(q)^T z + eps), one division per token
         {
           float r[16];
           tmem_ld16(tD + lane_off + (uint32_t)(dv & ~15), r);
           tmem_ld_wait();
-          den = r[dv & 15] + p.eps;
+          inv = 1.0f / (r[dv & 15] + p.eps);
         }
         float *orow = p.o + ((long)bh * N + (long)f * L + t) * dv;
-        for (int cb = 0; cb < dv / 16; ++cb) {
-          float r[16];
-          tmem_ld16(tD + lane_off + cb * 16, r);
+#pragma unroll 1
+        for (int cb = 0; cb < dv / 16; cb += 2) {  // 32 columns per TMEM wait
+          float r[2][16];
+          tmem_ld16(tD + lane_off + cb * 16, r[0]);
+          if (cb + 1 < dv / 16) tmem_ld16(tD + lane_off + (cb + 1) * 16, r[1]);
           tmem_ld_wait();
           if (t < L) {
-            float4 *dst = reinterpret_cast<float4 *>(orow + cb * 16);
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-              dst[e] = make_float4(r[4 * e] / den, r[4 * e + 1] / den, r[4 * e + 2] / den, r[4 * e + 3] / den);
+            for (int h = 0; h < 2; ++h) {
+              if (cb + h >= dv / 16) break;
+              float4 *dst = reinterpret_cast<float4 *>(orow + (cb + h) * 16);
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                dst[e] = make_float4(r[h][4 * e] * inv, r[h][4 * e + 1] * inv, r[h][4 * e + 2] * inv,
+                                     r[h][4 * e + 3] * inv);
+            }
           }
         }
         tc_fence_before();
