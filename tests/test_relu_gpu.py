@@ -128,3 +128,18 @@ def test_relu_timeout_status(lib, dev):
         assert int(status[0].item()) == 0
         o_ref, _, _ = oracle.relu_la(h["q"], h["k"], h["v"], F=w.F, L=w.L)
         assert rel_err(o, o_ref) <= 2e-3
+
+
+@pytest.mark.parametrize("ctas", [1, 2, 3])
+def test_relu_few_ctas_odd_tiles(lib, dev, ctas):
+    """One persistent CTA runs many frames whose read-out has an odd number of
+    128-token tiles (L=300: 3 tiles), so its two accumulator buffers change
+    roles from one frame to the next."""
+    w = W["relu_720p_81f"].with_(F=5, L=300, H=2, B=1, seed=77)
+    x = synth.inputs(w)
+    t, h = prep(w, x, dev)
+    o_ref, kv_ref, z_ref = oracle.relu_la(h["q"], h["k"], h["v"], F=w.F, L=w.L)
+    o, kv, z = run(lib, w, t, dev, "tc", max_ctas=ctas)
+    assert rel_err(o, o_ref) <= 2e-3
+    assert rel_err(kv, kv_ref) <= 2e-3
+    assert rel_err(z, z_ref) <= 2e-3
