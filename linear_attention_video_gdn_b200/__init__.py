@@ -144,6 +144,8 @@ def gdn_frame_fwd(q, k, v, alpha, beta, *, F: int, state_in=None, state_out=None
     q, k: [B, H, F*L, dk]; v: [B, H, F*L, dv] (float32 or bfloat16, same dtype);
     alpha: [B, H, F] float32; beta: [B, H, F*L] float32; state_in/state_out:
     [B, H, dk, dv] float32 or None.  Returns o [B, H, F*L, dv] float32.
+    ``segments``: chunk segments per frame for the tensor-core kernel (0 =
+    automatic; see ``gdn_opts.segments``).
     """
     B, H, N, dk = q.shape
     dv = v.shape[-1]
