@@ -285,6 +285,41 @@ def test_gdn_readout_uses_end_of_frame_state_and_split_resume():
     np.testing.assert_allclose(s_r, s, rtol=0, atol=1e-12)
 
 
+def test_gdn_frame_map_composes_from_chunk_segments():
+    """A frame's update is affine in the incoming state, S_out = A S_in + B, and
+    the maps of consecutive runs of tokens compose: the frame decay belongs to
+    the first run only.  This is the algebra that lets a frame be built in
+    pieces (one per run of chunks) and chained; here each piece's map is taken
+    from a short oracle run (A from state I with zero values, B from a zero
+    state), and the composition must reproduce the whole-sequence states and
+    read-outs."""
+    F, L, dk, dv = 2, 10, 4, 3
+    rng = np.random.default_rng(77)
+    q, k, v, a, b = _rand_case(1, F, L, dk, dv, rng, unit=False)
+    al = np.array([oracle.gate_alpha(x) for x in a[0]], np.float64)
+    be = np.array([oracle.gate_beta(x) for x in b[0]], np.float32)
+    S0 = rng.standard_normal((dk, dv))
+    o_ref, s_ref = oracle.gdn(q, k, v, al[None].astype(np.float32), be[None], F=F, L=L, gates_are_logits=False,
+                              state_in=S0[None])
+    for cuts in ([0, 10], [0, 3, 10], [0, 3, 6, 10], [0, 1, 2, 9, 10]):
+        S = S0.copy()
+        o = np.zeros((F * L, dv))
+        for f in range(F):
+            for s_i, (t0, t1) in enumerate(zip(cuts[:-1], cuts[1:])):
+                sl = slice(f * L + t0, f * L + t1)
+                n = t1 - t0
+                decay = np.array([[al[f] if s_i == 0 else 1.0]], np.float32)
+                zeros_v = np.zeros((1, n, dk), np.float32)
+                _, A = oracle.gdn(q[:, sl], k[:, sl], zeros_v, decay, be[None, sl], F=1, L=n,
+                                  gates_are_logits=False, state_in=np.eye(dk)[None], want_o=False)
+                _, B = oracle.gdn(q[:, sl], k[:, sl], v[:, sl], decay, be[None, sl], F=1, L=n,
+                                  gates_are_logits=False, state_in=np.zeros((1, dk, dv)), want_o=False)
+                S = A[0] @ S + B[0]
+            o[f * L:(f + 1) * L] = q[0, f * L:(f + 1) * L].astype(np.float64) @ S
+        np.testing.assert_allclose(S, s_ref[0], rtol=0, atol=1e-10)
+        np.testing.assert_allclose(o, o_ref[0], rtol=0, atol=1e-10)
+
+
 def test_gdn_frames_are_block_causal():
     # changing a later frame's inputs never changes an earlier frame's outputs
     rng = np.random.default_rng(10)
