@@ -44,7 +44,8 @@ def _load():
         lib.oracle_gdn.argtypes = [P, P, P, P, P, ctypes.c_int, P, P, P, I64, I64, I64, I64, I64, I64,
                                    I64, I64, P, I64, I64, ctypes.c_int]
         lib.oracle_gdn.restype = ctypes.c_int
-        lib.oracle_relu_la.argtypes = [P, P, P, P, P, P, P, P, I64, I64, I64, I64, I64, I64, ctypes.c_double]
+        lib.oracle_relu_la.argtypes = [P, P, P, P, P, P, P, P, I64, I64, I64, I64, I64, I64, ctypes.c_double,
+                                       ctypes.c_int]
         lib.oracle_relu_la.restype = ctypes.c_int
         lib.oracle_gate_alpha.argtypes = [ctypes.c_double]
         lib.oracle_gate_alpha.restype = ctypes.c_double
@@ -110,8 +111,11 @@ def gdn(q, k, v, alpha, beta, *, F: int, L: int, gates_are_logits: bool = True, 
     return o, s_out
 
 
-def relu_la(q, k, v, *, F: int, L: int, kv_in=None, z_in=None, eps: float = 1e-6):
-    """Block-causal ReLU linear attention in fp64.  Returns (o, kv_out, z_out)."""
+def relu_la(q, k, v, *, F: int, L: int, kv_in=None, z_in=None, eps: float = 1e-6, nthreads: int | None = None):
+    """Block-causal ReLU linear attention in fp64.  Returns (o, kv_out, z_out).
+
+    Heads are independent; ``nthreads`` threads (default: all host cores) take
+    whole heads, which changes no arithmetic."""
     q, k, v = map(_f32, (q, k, v))
     lead = q.shape[:-2]
     N, dk = q.shape[-2:]
@@ -122,8 +126,9 @@ def relu_la(q, k, v, *, F: int, L: int, kv_in=None, z_in=None, eps: float = 1e-6
     o = np.empty(lead + (N, dv))
     kv_out = np.empty(lead + (dk, dv))
     z_out = np.empty(lead + (dk,))
+    nthreads = nthreads or (os.cpu_count() or 1)
     rc = _load().oracle_relu_la(_ptr(q), _ptr(k), _ptr(v), _ptr(kv_in), _ptr(z_in), _ptr(kv_out),
-                                _ptr(z_out), _ptr(o), 1, nh, F, L, dk, dv, float(eps))
+                                _ptr(z_out), _ptr(o), 1, nh, F, L, dk, dv, float(eps), int(nthreads))
     if rc != 0:
         raise ValueError("oracle_relu_la: invalid arguments")
     return o, kv_out, z_out
@@ -132,26 +137,37 @@ def relu_la(q, k, v, *, F: int, L: int, kv_in=None, z_in=None, eps: float = 1e-6
 def gdn_stream(step_inputs, *, steps: int, L: int, state_in=None, cols=None):
     """Streaming block-cache decode: frames of ``steps`` calls each.
 
-    step_inputs(call) -> dict(q, k, v, a, b) for one frame (F=1) of fresh
-    inputs.  Every step of frame f starts from the committed state S_{f-1};
-    the state after the last step of the frame is committed.  Returns the
-    list of per-call outputs o and the final committed state.
+    Follows the SANA-Video talk's block KV cache passage (the cache made after
+    block i is what every pass over block i+1 reads): ``step_inputs(call)``
+    returns dict(q, k, v, a, b) for one frame (F=1) of fresh inputs, or None
+    once the stream ends (only at a frame boundary).  Every step of frame f
+    starts from the committed state S_{f-1} (``state_in``, or zero, before the
+    first frame); the state after the LAST step of the frame is committed and
+    the other steps' states are discarded.
+
+    Returns (outs, S, committed): the per-call outputs o in call order, the
+    final committed state, and the list of committed states, one per frame.
     """
+    if steps < 1:
+        raise ValueError("steps must be >= 1")
     S = None if state_in is None else np.asarray(state_in, np.float64)
-    outs = []
+    outs, committed = [], []
     call = 0
-    frames = 0
     while True:
-        x0 = step_inputs(call)
-        if x0 is None:
+        x = step_inputs(call)
+        if x is None:
             break
         last_state = None
         for s in range(steps):
-            x = x0 if s == 0 else step_inputs(call)
+            if s > 0:
+                x = step_inputs(call)
+                if x is None:
+                    raise ValueError(f"step_inputs({call}) returned None inside a frame "
+                                     f"(step {s + 1} of {steps}): a frame needs all of its steps")
             o, s_out = gdn(x["q"], x["k"], x["v"], x["a"], x["b"], F=1, L=L, state_in=S, cols=cols)
             outs.append(o)
             last_state = s_out
             call += 1
         S = last_state
-        frames += 1
-    return outs, S
+        committed.append(S)
+    return outs, S, committed

@@ -186,50 +186,104 @@ int oracle_gdn(const float *q, const float *k, const float *v, const float *alph
 }
 
 /*
- * Block-causal ReLU linear attention.  Layouts: q, k [B,H,F*L,dk];
- * v [B,H,F*L,dv]; kv_in/kv_out [B,H,dk,dv]; z_in/z_out [B,H,dk] (nullable);
- * o [B,H,F*L,dv].  Single-threaded per call; callers split heads.
+ * Block-causal ReLU linear attention, one (b, h) head.  Layouts: q, k
+ * [B,H,F*L,dk]; v [B,H,F*L,dv]; kv_in/kv_out [B,H,dk,dv]; z_in/z_out [B,H,dk]
+ * (nullable); o [B,H,F*L,dv].
  */
-int oracle_relu_la(const float *q, const float *k, const float *v, const double *kv_in,
-                   const double *z_in, double *kv_out, double *z_out, double *o,
-                   int64_t B, int64_t H, int64_t F, int64_t L, int64_t dk, int64_t dv, double eps) {
-  if (B < 0 || H < 0 || F < 0 || L < 0 || dk <= 0 || dv <= 0) return 1;
-  const int64_t N = F * L;
+typedef struct {
+  const float *q, *k, *v;
+  const double *kv_in, *z_in;
+  double *kv_out, *z_out, *o;
+  int64_t F, L, dk, dv;
+  double eps;
+  int64_t bh;
+} relu_unit_t;
+
+static void relu_unit(const relu_unit_t *u) {
+  const int64_t F = u->F, L = u->L, dk = u->dk, dv = u->dv, N = F * L, bh = u->bh;
   double *S = (double *)malloc(sizeof(double) * (size_t)(dk * dv));
   double *z = (double *)malloc(sizeof(double) * (size_t)dk);
   double *rq = (double *)malloc(sizeof(double) * (size_t)dk);
-  for (int64_t bh = 0; bh < B * H; ++bh) {
-    const float *qh = q + bh * N * dk, *kh = k + bh * N * dk, *vh = v + bh * N * dv;
-    for (int64_t e = 0; e < dk * dv; ++e) S[e] = kv_in ? kv_in[bh * dk * dv + e] : 0.0;
-    for (int64_t i = 0; i < dk; ++i) z[i] = z_in ? z_in[bh * dk + i] : 0.0;
-    for (int64_t f = 0; f < F; ++f) {
-      for (int64_t t = f * L; t < (f + 1) * L; ++t)
-        for (int64_t i = 0; i < dk; ++i) {
-          double rk = (double)kh[t * dk + i];
-          if (rk < 0.0) rk = 0.0;
-          z[i] += rk;
-          for (int64_t j = 0; j < dv; ++j) S[i * dv + j] += rk * (double)vh[t * dv + j];
-        }
-      for (int64_t t = f * L; t < (f + 1) * L; ++t) {
-        double den = 0.0;
-        for (int64_t i = 0; i < dk; ++i) {
-          double x = (double)qh[t * dk + i];
-          rq[i] = x > 0.0 ? x : 0.0;
-          den += rq[i] * z[i];
-        }
-        den += eps;
-        for (int64_t j = 0; j < dv; ++j) {
-          double num = 0.0;
-          for (int64_t i = 0; i < dk; ++i) num += rq[i] * S[i * dv + j];
-          o[(bh * N + t) * dv + j] = num / den;
-        }
+  const float *qh = u->q + bh * N * dk, *kh = u->k + bh * N * dk, *vh = u->v + bh * N * dv;
+  for (int64_t e = 0; e < dk * dv; ++e) S[e] = u->kv_in ? u->kv_in[bh * dk * dv + e] : 0.0;
+  for (int64_t i = 0; i < dk; ++i) z[i] = u->z_in ? u->z_in[bh * dk + i] : 0.0;
+  for (int64_t f = 0; f < F; ++f) {
+    for (int64_t t = f * L; t < (f + 1) * L; ++t)
+      for (int64_t i = 0; i < dk; ++i) {
+        double rk = (double)kh[t * dk + i];
+        if (rk < 0.0) rk = 0.0;
+        z[i] += rk;
+        for (int64_t j = 0; j < dv; ++j) S[i * dv + j] += rk * (double)vh[t * dv + j];
+      }
+    for (int64_t t = f * L; t < (f + 1) * L; ++t) {
+      double den = 0.0;
+      for (int64_t i = 0; i < dk; ++i) {
+        double x = (double)qh[t * dk + i];
+        rq[i] = x > 0.0 ? x : 0.0;
+        den += rq[i] * z[i];
+      }
+      den += u->eps;
+      for (int64_t j = 0; j < dv; ++j) {
+        double num = 0.0;
+        for (int64_t i = 0; i < dk; ++i) num += rq[i] * S[i * dv + j];
+        u->o[(bh * N + t) * dv + j] = num / den;
       }
     }
-    if (kv_out) memcpy(kv_out + bh * dk * dv, S, sizeof(double) * (size_t)(dk * dv));
-    if (z_out) memcpy(z_out + bh * dk, z, sizeof(double) * (size_t)dk);
   }
+  if (u->kv_out) memcpy(u->kv_out + bh * dk * dv, S, sizeof(double) * (size_t)(dk * dv));
+  if (u->z_out) memcpy(u->z_out + bh * dk, z, sizeof(double) * (size_t)dk);
   free(S);
   free(z);
   free(rq);
+}
+
+typedef struct {
+  relu_unit_t *units;
+  int64_t n;
+  int64_t next;
+  pthread_mutex_t mu;
+} relu_pool_t;
+
+static void *relu_worker(void *p) {
+  relu_pool_t *pl = (relu_pool_t *)p;
+  for (;;) {
+    pthread_mutex_lock(&pl->mu);
+    int64_t i = pl->next++;
+    pthread_mutex_unlock(&pl->mu);
+    if (i >= pl->n) return NULL;
+    relu_unit(&pl->units[i]);
+  }
+}
+
+/*
+ * Block-causal ReLU linear attention over all B*H heads; nthreads threads take
+ * whole heads (heads are independent, so this changes no arithmetic).
+ */
+int oracle_relu_la(const float *q, const float *k, const float *v, const double *kv_in,
+                   const double *z_in, double *kv_out, double *z_out, double *o,
+                   int64_t B, int64_t H, int64_t F, int64_t L, int64_t dk, int64_t dv, double eps,
+                   int nthreads) {
+  if (B < 0 || H < 0 || F < 0 || L < 0 || dk <= 0 || dv <= 0) return 1;
+  const int64_t n = B * H;
+  if (n == 0) return 0;
+  relu_unit_t *units = (relu_unit_t *)calloc((size_t)n, sizeof(relu_unit_t));
+  for (int64_t bh = 0; bh < n; ++bh) {
+    relu_unit_t *u = &units[bh];
+    u->q = q; u->k = k; u->v = v; u->kv_in = kv_in; u->z_in = z_in;
+    u->kv_out = kv_out; u->z_out = z_out; u->o = o;
+    u->F = F; u->L = L; u->dk = dk; u->dv = dv; u->eps = eps; u->bh = bh;
+  }
+  relu_pool_t pl;
+  pl.units = units; pl.n = n; pl.next = 0;
+  pthread_mutex_init(&pl.mu, NULL);
+  if (nthreads < 1) nthreads = 1;
+  if (nthreads > n) nthreads = (int)n;
+  if (nthreads > 512) nthreads = 512;
+  pthread_t th[512];
+  for (int t = 1; t < nthreads; ++t) pthread_create(&th[t], NULL, relu_worker, &pl);
+  relu_worker(&pl);
+  for (int t = 1; t < nthreads; ++t) pthread_join(th[t], NULL);
+  pthread_mutex_destroy(&pl.mu);
+  free(units);
   return 0;
 }

@@ -338,6 +338,91 @@ def test_gdn_frames_are_block_causal():
     assert (np.abs(o3[0, 2 * L:] - o[0, 2 * L:]).max(axis=1) > 0).all()
 
 
+# ---------------------------------------------------------------- streaming (block cache, several steps per frame)
+
+def _stream_calls(nframes, steps, L, dk, dv, seed):
+    """Fresh inputs per call (one frame each), as value gates, for streaming pins."""
+    rng = np.random.default_rng(seed)
+    calls = []
+    for _ in range(nframes * steps):
+        q, k, v, a, b = _rand_case(1, 1, L, dk, dv, rng)
+        calls.append(dict(q=q, k=k, v=v, a=a, b=b))
+    return calls
+
+
+def _feeder(calls):
+    return lambda c: calls[c] if c < len(calls) else None
+
+
+def test_gdn_stream_one_step_equals_whole_sequence():
+    """With one step per frame, streaming is the whole-sequence recurrence over
+    the same frames: every output and the final state are bit-identical."""
+    F, L, dk, dv = 4, 5, 6, 4
+    calls = _stream_calls(F, 1, L, dk, dv, 31)
+    S0 = np.random.default_rng(3).standard_normal((1, dk, dv))
+    outs, S, committed = oracle.gdn_stream(_feeder(calls), steps=1, L=L, state_in=S0)
+    cat = {n: np.concatenate([c[n] for c in calls], axis=1) for n in "qkvab"}
+    o_ref, s_ref = oracle.gdn(cat["q"], cat["k"], cat["v"], cat["a"], cat["b"], F=F, L=L, state_in=S0)
+    np.testing.assert_array_equal(np.concatenate(outs, axis=1), o_ref)
+    np.testing.assert_array_equal(S, s_ref)
+    assert len(committed) == F
+
+
+def test_gdn_stream_commits_only_the_last_step():
+    """Steps 1..3 of a frame leave no trace: changing their inputs changes
+    neither any committed state nor any last-step output; and the committed
+    state after frame f is the whole-sequence state over the last-step inputs
+    of frames 0..f."""
+    nf, steps, L, dk, dv = 3, 4, 6, 5, 4
+    calls = _stream_calls(nf, steps, L, dk, dv, 41)
+    outs, S, committed = oracle.gdn_stream(_feeder(calls), steps=steps, L=L)
+    rng = np.random.default_rng(5)
+    changed = [dict(c) for c in calls]
+    for c in range(len(calls)):
+        if c % steps != steps - 1:
+            changed[c] = {n: (x + rng.standard_normal(x.shape).astype(np.float32)) for n, x in calls[c].items()}
+    outs2, S2, committed2 = oracle.gdn_stream(_feeder(changed), steps=steps, L=L)
+    for f in range(nf):
+        np.testing.assert_array_equal(committed2[f], committed[f])
+        last = f * steps + steps - 1
+        np.testing.assert_array_equal(outs2[last], outs[last])
+        # a non-committing step's output does depend on its own inputs
+        assert not np.array_equal(outs2[f * steps], outs[f * steps])
+    for f in range(nf):
+        lasts = [calls[g * steps + steps - 1] for g in range(f + 1)]
+        cat = {n: np.concatenate([c[n] for c in lasts], axis=1) for n in "qkvab"}
+        _, s_ref = oracle.gdn(cat["q"], cat["k"], cat["v"], cat["a"], cat["b"], F=f + 1, L=L)
+        np.testing.assert_array_equal(committed[f], s_ref)
+
+
+def test_gdn_stream_every_step_matches_bruteforce():
+    """Each step's output, and each committed state, equals the brute-force
+    dense-product result started from the state committed by the previous
+    frame (an independent construction, not the oracle's own loop)."""
+    nf, steps, L, dk, dv = 2, 3, 3, 4, 3
+    calls = _stream_calls(nf, steps, L, dk, dv, 51)
+    outs, S, committed = oracle.gdn_stream(_feeder(calls), steps=steps, L=L)
+    S_prev = np.zeros((dk, dv))
+    for f in range(nf):
+        for s_i in range(steps):
+            c = calls[f * steps + s_i]
+            al = np.array([oracle.gate_alpha(x) for x in c["a"][0]], np.float64)  # gates from logits, in double
+            be = np.array([oracle.gate_beta(x) for x in c["b"][0]], np.float64)
+            o_b, s_b = _bruteforce_gdn(c["q"][0], c["k"][0], c["v"][0], al, be, 1, L, S_prev)
+            np.testing.assert_allclose(outs[f * steps + s_i][0], o_b, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(committed[f][0], s_b, rtol=0, atol=1e-12)
+        S_prev = s_b
+    np.testing.assert_array_equal(S, committed[-1])
+
+
+def test_gdn_stream_refuses_a_frame_cut_short():
+    calls = _stream_calls(1, 4, 3, 4, 3, 61)[:3]  # three of a frame's four steps
+    with pytest.raises(ValueError, match="inside a frame"):
+        oracle.gdn_stream(_feeder(calls), steps=4, L=3)
+    outs, S, committed = oracle.gdn_stream(_feeder([]), steps=4, L=3)
+    assert outs == [] and S is None and committed == []
+
+
 # ---------------------------------------------------------------- ReLU mode
 
 def _quadratic_masked_attention(q, k, v, F, L, eps):
