@@ -27,15 +27,20 @@ import sys
 import threading
 import time
 
+import numpy as np
+
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "GDN frame-recurrence tokens/s (720p-60s shape, bf16) and % of roofline"
 WORKLOAD = "gdn_720p_60s"
 FALLBACK_HBM_GBS = 6650.0
+SPEC_HBM_GBS = 8000.0  # B200 HBM3e figure quoted as "about 8 TB/s"
 # algorithmic bytes per token-head: q, k, v bf16 (3 * 112 * 2) + o fp32 (112 * 4) + beta fp32
 BYTES_PER_TOKEN_HEAD = 3 * 112 * 2 + 112 * 4 + 4
 FLOPS_PER_TOKEN_HEAD = 6 * 112 * 112
+PRECISION = ("bf16 q/k/v; fp16 tensor-core operands with fp32 accumulation; the state is carried from frame to "
+             "frame, and taken from state_in, as fp16; fp32 o and state_out")
 
 
 def parse():
@@ -264,12 +269,19 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         dist.barrier()
     torch.cuda.synchronize()
 
-    ms_e2e, h2d, d2h, relu = None, 0, 0, None
+    ms_e2e, h2d, d2h = None, 0, 0
     if not args.quick:
-        ms_e2e, h2d, d2h, relu = end_to_end_and_relu(args, lib, synth, torch, dist, w, dev, stream, world, rank,
-                                                     (hq, hk, hv, ha, hb), opts)
+        ms_e2e, h2d, d2h = end_to_end_leg(args, lib, torch, dist, w, dev, stream, world, (hq, hk, hv, ha, hb))
     if rank != 0:
         return
+    cpu_on = world == 1 and not args.no_cpu_baseline
+    del q, k, v, a, b, o, ws
+    extra = {}
+    if not args.quick:
+        extra["relu_la"] = relu_leg(args, lib, synth, torch, dev, stream, cpu_on)
+        if not args.no_streaming:
+            extra["streaming"] = streaming_leg(args, lib, synth, torch, dev, stream, cpu_on)
+        extra["configs_other"] = small_configs_leg(args, lib, synth, torch, dev, stream, cpu_on)
     peak, peak_src = measured_peaks()
     alg_bytes = token_heads * BYTES_PER_TOKEN_HEAD + w.B * w.H * (w.F * 4 + w.dk * w.dv * 4)
     achieved = alg_bytes / (ms / 1e3) / 1e9
@@ -286,7 +298,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "bf16",
-        "precision": "bf16 q/k/v, fp16 tensor-core operands, fp32 accumulation, fp32 state and output",
+        "precision": PRECISION,
         "data": "synthetic",
         "config": {"workload": WORKLOAD if w.F == 240 else f"{WORKLOAD} first {w.F} frames",
                    "B": w.B, "H": w.H, "F": w.F, "L": w.L, "dk": w.dk, "dv": w.dv,
@@ -294,7 +306,9 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                    "parallelism": f"dp{world} (independent batch per GPU, no exchange)",
                    "l2": "inputs larger than the 126 MB L2 (2.97 GB per GPU at F=240); no flush needed"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "peak_source": f"{peak_src} hbm_gbs", "alg_bytes_per_launch": alg_bytes,
+                     "peak_source": f"{peak_src} hbm_gbs (headline fraction); frac_vs_8tbs_spec is against the "
+                                    f"8 TB/s HBM3e figure", "frac_vs_8tbs_spec": achieved / SPEC_HBM_GBS,
+                     "alg_bytes_per_launch": alg_bytes,
                      "traffic": None if tr is None else tr["dram_bytes_per_launch"],
                      "traffic_source": None if tr is None else tr["source"]},
         "gpu_launches": args.steps,
@@ -305,17 +319,53 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         line["e2e"] = {"value": whole_job_tokens_per_s(tokens, world, ms_e2e), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                        "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e,
                        "call": "gdn_frame_fwd_host (C ABI, pinned host buffers, copies + kernel + sync)"}
-    if relu is not None:
-        streaming = relu.pop("streaming", None)
-        line["relu_la"] = relu
-        if streaming is not None:
-            line["streaming"] = streaming
-    if world == 1 and not args.no_cpu_baseline and not args.quick:
+    line.update(extra)
+    if cpu_on and not args.quick:
         line["cpu_baseline"] = cpu_baseline(w)
     print(json.dumps(line), flush=True)
 
 
-def end_to_end_and_relu(args, lib, synth, torch, dist, w, dev, stream, world, rank, host, opts):
+def _events_ms(fn, n, stream):
+    """Mean device time of fn() over n calls, CUDA events on `stream`."""
+    import torch
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / n
+
+
+def _roofline(alg_bytes, ms, peak, peak_src):
+    ach = alg_bytes / (ms / 1e3) / 1e9
+    return {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
+            "peak_source": f"{peak_src} hbm_gbs", "frac_vs_8tbs_spec": ach / SPEC_HBM_GBS,
+            "alg_bytes_per_launch": alg_bytes}
+
+
+def _gdn_alg_bytes(w, esz=2):
+    """Algorithmic bytes of one gdn_frame_fwd call: q, k, v read once, o (fp32)
+    written once, gates and the output state."""
+    th = w.B * w.H * w.N
+    return th * (esz * (2 * w.dk + w.dv) + 4 * w.dv + 4) + w.B * w.H * (w.F * 4 + w.dk * w.dv * 4)
+
+
+def _oracle_tokens_per_s(fn, tokens, target_s=2.0):
+    """Run fn() (one oracle call over `tokens` sequence tokens) until about
+    target_s seconds have passed; tokens per second."""
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        fn()
+        n += 1
+        dt = time.perf_counter() - t0
+        if dt >= target_s:
+            return tokens * n / dt, n, dt
+
+
+def end_to_end_leg(args, lib, torch, dist, w, dev, stream, world, host):
     hq, hk, hv, ha, hb = host
     # end to end through the host-buffer C-ABI call (copies inside the timed region)
     ho = torch.empty((w.B, w.H, w.N, w.dv), dtype=torch.float32).pin_memory()
@@ -325,92 +375,167 @@ def end_to_end_and_relu(args, lib, synth, torch, dist, w, dev, stream, world, ra
     if world > 1:
         dist.barrier()
     n_e2e = max(1, args.e2e_steps)
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
-    for _ in range(n_e2e):
-        lib.gdn_frame_fwd_host(hq, hk, hv, ha, hb, F=w.F, o=ho, workspace=hws)
-    t1.record(stream)
-    torch.cuda.synchronize()
-    ms_e2e = max_over_ranks(t0.elapsed_time(t1) / n_e2e, dev, world)
+    ms_e2e = _events_ms(lambda: lib.gdn_frame_fwd_host(hq, hk, hv, ha, hb, F=w.F, o=ho, workspace=hws), n_e2e,
+                        stream)
+    ms_e2e = max_over_ranks(ms_e2e, dev, world)
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, ha, hb))
     d2h = ho.numel() * ho.element_size()
     del hws
+    return ms_e2e, h2d, d2h
 
-    # the ReLU block-causal mode at its own workload (reported beside the headline)
-    relu = None
-    if rank == 0:
-        wr = synth.WORKLOADS["relu_720p_81f"]
-        xr = synth.inputs(wr)
-        rq, rk, rv = (torch.from_numpy(xr[n]).to(torch.bfloat16).to(dev) for n in "qkv")
-        ro = torch.empty((wr.B, wr.H, wr.N, wr.dv), dtype=torch.float32, device=dev)
-        rws = lib.alloc_workspace(lib.workspace_bytes(lib.OP_RELU_LA, wr.B, wr.H, wr.F, wr.L, wr.dk, wr.dv, opts), dev)
-        for _ in range(3):
-            lib.relu_la_block_fwd(rq, rk, rv, F=wr.F, o=ro, workspace=rws)
+
+def relu_leg(args, lib, synth, torch, dev, stream, cpu_baseline_on):
+    """The ReLU block-causal mode at its own workload (B=2, H=20, F=81, L=920)."""
+    wr = synth.WORKLOADS["relu_720p_81f"]
+    xr = synth.inputs(wr)
+    rq, rk, rv = (torch.from_numpy(xr[n]).to(torch.bfloat16).to(dev) for n in "qkv")
+    ro = torch.empty((wr.B, wr.H, wr.N, wr.dv), dtype=torch.float32, device=dev)
+    opts = lib.make_opts(lib.DTYPE_BF16)
+    rws = lib.alloc_workspace(lib.workspace_bytes(lib.OP_RELU_LA, wr.B, wr.H, wr.F, wr.L, wr.dk, wr.dv, opts), dev)
+    call = lambda: lib.relu_la_block_fwd(rq, rk, rv, F=wr.F, o=ro, workspace=rws)
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    rms = _events_ms(call, max(5, args.steps // 2), stream)
+    rbytes = wr.B * wr.H * wr.N * (3 * wr.dk * 2 + wr.dv * 4) + wr.B * wr.H * wr.dk * (wr.dv + 1) * 4
+    peak, src = measured_peaks()
+    out = {"workload": "relu_720p_81f", "B": wr.B, "H": wr.H, "F": wr.F, "L": wr.L, "d": wr.dk, "ms": rms,
+           "tokens_per_s": wr.B * wr.N / (rms / 1e3), "roofline": _roofline(rbytes, rms, peak, src),
+           "achieved_gbs": rbytes / (rms / 1e3) / 1e9, "frac_hbm": rbytes / (rms / 1e3) / 1e9 / peak,
+           "l2": "inputs 2.0 GB, larger than L2; no flush needed"}
+    del rq, rk, rv, ro, rws
+    if cpu_baseline_on:
+        import oracle
+        frames = 2
+        xs = synth.inputs(wr, frames=frames)
+        hx = {n: torch.from_numpy(xs[n]).to(torch.bfloat16).float().numpy() for n in "qkv"}
+        nthreads = os.cpu_count() or 1
+        tps, n, dt = _oracle_tokens_per_s(
+            lambda: oracle.relu_la(hx["q"], hx["k"], hx["v"], F=frames, L=wr.L, nthreads=nthreads),
+            wr.B * frames * wr.L)
+        out["cpu_baseline"] = {"value": tps, "unit": "tokens/s", "cores": min(nthreads, wr.B * wr.H),
+                               "kind": "oracle", "sample": f"all {wr.B * wr.H} heads x first {frames} of {wr.F} "
+                                                           f"frames, {n} runs in {dt:.1f} s"}
+    return out
+
+
+def small_configs_leg(args, lib, synth, torch, dev, stream, cpu_baseline_on):
+    """The tiny fp32 case (launch latency) and the 480p 5 s shape, each timed
+    on its own with CUDA events, with its roofline and the oracle beside it."""
+    import oracle
+    out = {}
+    peak, src = measured_peaks()
+    for name in ("tiny_fp32", "gdn_480p_5s"):
+        w = synth.WORKLOADS[name]
+        x = synth.inputs(w)
+        dt = torch.float32 if w.dtype == "f32" else torch.bfloat16
+        q, k, v = (torch.from_numpy(x[n]).to(dt).to(dev) for n in "qkv")
+        a, b = (torch.from_numpy(x[n]).to(dev) for n in "ab")
+        o = torch.empty((w.B, w.H, w.N, w.dv), dtype=torch.float32, device=dev)
+        s_out = torch.empty((w.B, w.H, w.dk, w.dv), dtype=torch.float32, device=dev)
+        opts = lib.make_opts(lib.DTYPE_F32 if w.dtype == "f32" else lib.DTYPE_BF16)
+        ws = lib.alloc_workspace(lib.workspace_bytes(lib.OP_GDN, w.B, w.H, w.F, w.L, w.dk, w.dv, opts), dev)
+        call = lambda: lib.gdn_frame_fwd(q, k, v, a, b, F=w.F, o=o, state_out=s_out, workspace=ws)
+        for _ in range(5):
+            call()
         torch.cuda.synchronize()
-        r0 = torch.cuda.Event(enable_timing=True)
-        r1 = torch.cuda.Event(enable_timing=True)
-        nr = max(5, args.steps // 2)
-        r0.record(stream)
-        for _ in range(nr):
-            lib.relu_la_block_fwd(rq, rk, rv, F=wr.F, o=ro, workspace=rws)
-        r1.record(stream)
-        torch.cuda.synchronize()
-        rms = r0.elapsed_time(r1) / nr
-        rbytes = wr.B * wr.H * wr.N * (3 * wr.dk * 2 + wr.dv * 4)
-        peak, _ = measured_peaks()
-        relu = {"workload": "relu_720p_81f", "ms": rms, "tokens_per_s": wr.B * wr.N / (rms / 1e3),
-                "achieved_gbs": rbytes / (rms / 1e3) / 1e9, "frac_hbm": rbytes / (rms / 1e3) / 1e9 / peak}
-        del rq, rk, rv, ro, rws
-        relu["streaming"] = None
-        if not args.no_streaming:
-            relu["streaming"] = streaming_leg(lib, synth, torch, dev, stream)
-    return ms_e2e, h2d, d2h, relu
+        n = 200 if name == "tiny_fp32" else 50
+        # L2 flush between timed calls for the 480p shape (its 184 MB of bytes are close to L2's 126 MB)
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if name != "tiny_fp32" else None
+        if flush is None:
+            ms = _events_ms(call, n, stream)
+            l2 = "not flushed (launch-latency case)"
+        else:
+            tot = 0.0
+            for _ in range(n):
+                flush.zero_()
+                tot += _events_ms(call, 1, stream)
+            ms = tot / n
+            l2 = "256 MB buffer written between timed calls (L2 flushed)"
+        nb = _gdn_alg_bytes(w, 4 if w.dtype == "f32" else 2)
+        d = {"workload": name, "B": w.B, "H": w.H, "F": w.F, "L": w.L, "dk": w.dk, "dv": w.dv, "dtype": w.dtype,
+             "ms": ms, "us_per_call": ms * 1e3, "tokens_per_s": w.B * w.N / (ms / 1e3),
+             "roofline": _roofline(nb, ms, peak, src), "l2": l2}
+        if name == "tiny_fp32":
+            d["roofline"]["bound"] = "latency"
+        if cpu_baseline_on:
+            hx = {n_: t.float().cpu().numpy() for n_, t in (("q", q), ("k", k), ("v", v))}
+            nthreads = os.cpu_count() or 1
+            frames = w.F if name == "tiny_fp32" else 3
+            sl = slice(0, frames * w.L)
+            tps, runs, secs = _oracle_tokens_per_s(
+                lambda: oracle.gdn(hx["q"][:, :, sl], hx["k"][:, :, sl], hx["v"][:, :, sl], x["a"][:, :, :frames],
+                                   x["b"][:, :, sl], F=frames, L=w.L, nthreads=nthreads), w.B * frames * w.L)
+            d["cpu_baseline"] = {"value": tps, "unit": "tokens/s", "cores": nthreads, "kind": "oracle",
+                                 "sample": f"all {w.B * w.H} heads x first {frames} of {w.F} frames, {runs} runs "
+                                           f"in {secs:.1f} s"}
+        out[name] = d
+        del q, k, v, a, b, o, s_out, ws, flush
+    return out
 
 
-def streaming_leg(lib, synth, torch, dev, stream):
-    """Streaming decode at the 720p shape: one frame per call (F = 1, 20 heads,
-    920 tokens), 4 calls per frame with fresh q, k, v and gates, the state
-    committed by the 4th.  Timed over 20 frames with the automatic chunk
+def streaming_leg(args, lib, synth, torch, dev, stream, cpu_baseline_on):
+    """The streaming block-cache decode at the 720p shape, run as the protocol:
+    240 frames x 4 denoising steps = 960 calls of one frame (F = 1, 20 heads,
+    920 tokens); every step reads the committed state of the previous frame,
+    state_out is NULL on steps 1-3 and the 4th step commits the state that the
+    next frame reads.  Fresh inputs per call come from a pool of 16 distinct
+    calls (200 MB, more than L2), cycled.  Timed with the automatic chunk
     segments and with one CTA per frame (segments = 1)."""
-    ws_ = synth.WORKLOADS["gdn_stream_720p"].with_(F=1)
-    calls = []
-    for c in range(8):  # 8 calls' inputs, cycled (about 100 MB)
-        x = synth.inputs(ws_, call=c)
-        calls.append([torch.from_numpy(x[n]).to(torch.bfloat16).to(dev) for n in "qkv"] +
-                     [torch.from_numpy(x[n]).to(dev) for n in "ab"])
-    o = torch.empty((ws_.B, ws_.H, ws_.L, ws_.dv), dtype=torch.float32, device=dev)
-    s_in = torch.zeros((ws_.B, ws_.H, ws_.dk, ws_.dv), dtype=torch.float32, device=dev)
-    s_out = torch.empty_like(s_in)
-    out = {"workload": "gdn_stream_720p (F=1 per call, 4 calls per frame)", "frames_timed": 20}
+    w = synth.WORKLOADS["gdn_stream_720p"]
+    steps, frames, pool_n = w.steps, w.F, 16
+    pool = []
+    for c in range(pool_n):
+        x = synth.inputs(w, call=c)
+        pool.append([torch.from_numpy(x[n]).to(torch.bfloat16).to(dev) for n in "qkv"] +
+                    [torch.from_numpy(x[n]).to(dev) for n in "ab"])
+    o = torch.empty((w.B, w.H, w.L, w.dv), dtype=torch.float32, device=dev)
+    sbuf = [torch.zeros((w.B, w.H, w.dk, w.dv), dtype=torch.float32, device=dev) for _ in range(2)]
+    calls = frames * steps
+    out = {"workload": "gdn_stream_720p", "B": w.B, "H": w.H, "L": w.L, "d": w.dk, "frames": frames,
+           "steps_per_frame": steps, "calls_timed": calls,
+           "protocol": "state_in = committed state of the previous frame; state_out NULL on steps 1-3, committed "
+                       "on step 4",
+           "l2": f"inputs cycled from a pool of {pool_n} distinct calls (about 200 MB, more than L2)"}
+    peak, src = measured_peaks()
     for tag, segs in (("auto", 0), ("one_cta_per_frame", 1)):
         o_ = lib.make_opts(lib.DTYPE_BF16, segments=segs)
-        wsb = lib.alloc_workspace(lib.workspace_bytes(lib.OP_GDN, ws_.B, ws_.H, 1, ws_.L, ws_.dk, ws_.dv, o_), dev)
+        wsb = lib.alloc_workspace(lib.workspace_bytes(lib.OP_GDN, w.B, w.H, 1, w.L, w.dk, w.dv, o_), dev)
 
-        def frame(i):
-            for st in range(4):
-                q_, k_, v_, a_, b_ = calls[(4 * i + st) % 8]
-                lib.gdn_frame_fwd(q_, k_, v_, a_, b_, F=1, state_in=s_in, state_out=(s_out if st == 3 else None),
-                                  o=o, workspace=wsb, segments=segs)
+        def protocol(nf):
+            cur = 0
+            for f in range(nf):
+                for st in range(steps):
+                    q_, k_, v_, a_, b_ = pool[(f * steps + st) % pool_n]
+                    lib.gdn_frame_fwd(q_, k_, v_, a_, b_, F=1, state_in=None if f == 0 else sbuf[cur],
+                                      state_out=(sbuf[cur ^ 1] if st == steps - 1 else None), o=o, workspace=wsb,
+                                      segments=segs)
+                cur ^= 1
 
-        for i in range(3):
-            frame(i)
+        protocol(4)
         torch.cuda.synchronize()
-        t0 = torch.cuda.Event(enable_timing=True)
-        t1 = torch.cuda.Event(enable_timing=True)
-        t0.record(stream)
-        for i in range(20):
-            frame(i)
-        t1.record(stream)
-        torch.cuda.synchronize()
-        out[f"us_per_call_{tag}"] = t0.elapsed_time(t1) / 80 * 1e3
+        ms = _events_ms(lambda: protocol(frames), 1, stream)
+        out[f"us_per_call_{tag}"] = ms * 1e3 / calls
+        out[f"ms_protocol_{tag}"] = ms
+        del wsb
     us = out["us_per_call_auto"]
-    # bytes per call: q, k, v (bf16), gates, o (fp32), state in (fp32); +state out on one call in 4
-    nb = ws_.B * ws_.H * (ws_.L * (3 * ws_.dk * 2 + 4 + ws_.dv * 4) + 4 + ws_.dk * ws_.dv * 4 * 1.25)
-    peak, _ = measured_peaks()
-    out.update({"frame_tokens_per_s": ws_.B * ws_.L / (us / 1e6), "alg_bytes_per_call": nb,
-                "achieved_gbs": nb / (us / 1e6) / 1e9, "frac_hbm": nb / (us / 1e6) / 1e9 / peak,
-                "l2": "not flushed; the call is latency-bound (its bytes take about 3 us of HBM time)"})
+    # bytes per call: q, k, v (bf16), gates, o (fp32), state in (fp32); + state out on one call in 4
+    nb = w.B * w.H * (w.L * (3 * w.dk * 2 + 4 + w.dv * 4) + 4 + w.dk * w.dv * 4 * (1 + 1 / steps))
+    out.update({"step_tokens_per_s": w.B * w.L / (us / 1e6), "frames_committed_per_s": 1e6 / (us * steps),
+                "roofline": _roofline(nb, us / 1e3, peak, src)})
+    out["roofline"]["alg_bytes_per_call"] = nb
+    if cpu_baseline_on:
+        import oracle
+        x = synth.inputs(w, call=0)
+        hx = {n: torch.from_numpy(x[n]).to(torch.bfloat16).float().numpy() for n in "qkv"}
+        S = np.zeros((w.B, w.H, w.dk, w.dv))
+        nthreads = os.cpu_count() or 1
+        tps, runs, secs = _oracle_tokens_per_s(
+            lambda: oracle.gdn(hx["q"], hx["k"], hx["v"], x["a"], x["b"], F=1, L=w.L, state_in=S,
+                               nthreads=nthreads), w.B * w.L)
+        out["cpu_baseline"] = {"value": tps, "unit": "step tokens/s", "cores": nthreads, "kind": "oracle",
+                               "sample": f"one streaming call (20 heads, 920 tokens) repeated {runs} times in "
+                                         f"{secs:.1f} s"}
     return out
 
 

@@ -35,8 +35,11 @@
  *  - The library allocates no memory.  Kernels that need scratch take it
  *    from opts->workspace (size from gdn_workspace_bytes()).  Two calls that
  *    share a workspace must be ordered on the GPU (same stream).
- *  - Thread-safe: no global mutable state besides a per-device cache of the
- *    SM count and of the driver's tensor-map encoder entry point.
+ *  - Thread-safe, with one exception: the only global mutable state is a
+ *    per-device cache of the SM count, of the driver's tensor-map encoder
+ *    entry point and of the no-allocation scratch address, and the device
+ *    scratch array of gdn_frame_fwd_noalloc(), which all of that entry
+ *    point's calls share (see there).
  */
 #ifndef GDN_B200_H_
 #define GDN_B200_H_
@@ -53,7 +56,7 @@ extern "C" {
 #define GDN_API
 #endif
 
-#define GDN_ABI_VERSION 2
+#define GDN_ABI_VERSION 3
 
 /* return / status codes */
 #define GDN_OK 0
@@ -62,6 +65,8 @@ extern "C" {
 #define GDN_ERR_CUDA 3          /* a CUDA runtime/driver call failed */
 #define GDN_ERR_TIMEOUT 4       /* device: a bounded in-kernel wait expired (outputs invalid) */
 #define GDN_ERR_NO_DEVICE 5     /* no usable sm_100 device for this call */
+#define GDN_ERR_RANGE 6         /* device: a value met the fp16 range of the tensor-core operands
+                                   (|q|, |v| or |S| >= 65504, or NaN); outputs invalid */
 
 /* element types of q, k, v */
 #define GDN_DTYPE_F32 0
@@ -71,7 +76,11 @@ extern "C" {
 #define GDN_IMPL_AUTO 0
 #define GDN_IMPL_SEQ 1          /* per-token SIMT recurrence, one CTA per head (reference-simple) */
 #define GDN_IMPL_FRAME_SIMT 2   /* frame maps + ticketed frame chain, CUDA cores, fp32 arithmetic */
-#define GDN_IMPL_TC 3           /* frame maps + chain on tcgen05/TMEM tensor cores (bf16 inputs) */
+#define GDN_IMPL_TC 3           /* frame maps + chain on tcgen05/TMEM tensor cores (bf16 inputs): the
+                                   product-form kernel where its sizes allow it and frames are not
+                                   split into segments, else the residual-form kernel */
+#define GDN_IMPL_TC_RESIDUAL 4  /* the residual-form tensor-core kernel only (any d_k, d_v multiple of
+                                   16 up to 128; also splits frames into chunk segments) */
 
 /* operation ids for gdn_workspace_bytes() */
 #define GDN_OP_GDN 0
@@ -162,10 +171,15 @@ GDN_API int relu_la_block_fwd(const void *q, const void *k, const void *v, const
  *
  * Same semantics and layouts as gdn_frame_fwd, but q, k, v, alpha, beta,
  * state_in (inputs) and o, state_out (outputs) are host pointers (pinned
- * memory gives full PCIe bandwidth).  The call copies the inputs into the
- * caller's device workspace, runs the recurrence there, copies the outputs
- * back and synchronises opts->stream before returning.
- * opts->workspace must hold gdn_workspace_bytes_host() bytes.
+ * memory gives full PCIe bandwidth).  The call streams the sequence through
+ * the caller's device workspace in groups of frames: the inputs of the next
+ * group are copied in and the output of the previous group is copied out
+ * while a group runs, on two streams the call creates and destroys, ordered
+ * after the work already queued on opts->stream.  The state passes from group
+ * to group in fp32, so the result equals that of gdn_frame_fwd over the whole
+ * sequence.  The call synchronises opts->stream before returning.
+ * opts->workspace must hold gdn_workspace_bytes_host() bytes (two groups'
+ * inputs and outputs, four states and one group's kernel workspace).
  */
 GDN_API int gdn_frame_fwd_host(const void *q, const void *k, const void *v, const float *alpha, const float *beta,
                        const float *state_in, float *state_out, float *o, int B, int H, int F, int L,
@@ -186,11 +200,12 @@ GDN_API int gdn_frame_fwd_host(const void *q, const void *k, const void *v, cons
  * the process exits.  Calls whose gdn_workspace_bytes(GDN_OP_GDN, ...) exceeds
  * that size return GDN_ERR_UNSUPPORTED without launching anything.  The first
  * call on a device looks up the array's device address; make that first call
- * before any stream capture.  All calls share the array: calls that may run
- * at the same time on the GPU (other streams, unordered host threads) race on
- * it and must be serialised by the caller.  Each call clears the part of the
- * array that must start at zero before its kernel runs.  The call allocates
- * no memory.
+ * before any stream capture.  Later calls made outside stream capture look it
+ * up again, so the address stays right after a device reset.  All calls share
+ * the array: calls that may run at the same time on the GPU (other streams,
+ * unordered host threads) race on it and must be serialised by the caller.
+ * Each call clears the part of the array that must start at zero before its
+ * kernel runs.  The call allocates no memory.
  */
 #define GDN_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
 GDN_API int gdn_frame_fwd_noalloc(const void *q, const void *k, const void *v, const float *alpha,
@@ -203,8 +218,10 @@ GDN_API size_t gdn_workspace_bytes(int op, int B, int H, int F, int L, int dk, i
 /* Device scratch bytes that gdn_frame_fwd_host() needs (staging + workspace). */
 GDN_API size_t gdn_workspace_bytes_host(int B, int H, int F, int L, int dk, int dv, const gdn_opts_t *opts);
 
-/* Static description of a status code (never NULL). */
+/* Static description of a status code (never NULL).  gdn_status_str is the
+ * same function under a shorter name. */
 GDN_API const char *gdn_status_string(int status);
+GDN_API const char *gdn_status_str(int status);
 
 /* GDN_ABI_VERSION of the loaded library. */
 GDN_API int gdn_abi_version(void);

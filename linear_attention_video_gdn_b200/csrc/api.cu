@@ -46,6 +46,7 @@ int check_sizes(int B, int H, int F, int L, int dk, int dv) {
 }
 
 int pick_gdn_impl(const gdn_opts_t *o, int dk, int dv) {
+  if (o->impl == GDN_IMPL_TC_RESIDUAL) return GDN_IMPL_TC;
   if (o->impl != GDN_IMPL_AUTO) return o->impl;
   if (o->in_dtype == GDN_DTYPE_BF16 && gdn_tc_supported(dk, dv)) return GDN_IMPL_TC;
   return GDN_IMPL_FRAME_SIMT;
@@ -57,9 +58,17 @@ int pick_relu_impl(const gdn_opts_t *o, int dk, int dv) {
   return GDN_IMPL_FRAME_SIMT;
 }
 
+// Floats of scratch per published frame state of the frame-chain kernels other
+// than the product-form one (which gdn_ws_bytes_p sizes on its own).
 size_t gdn_state_elems(int impl, int dk, int dv) {
   if (impl == GDN_IMPL_TC) return gdn_tc_state_elems(dk, dv);
   return (size_t)dk * dv;
+}
+
+// The product-form tensor-core kernel runs for GDN_IMPL_TC launches with one
+// segment per frame whose sizes it supports.
+bool use_pform(int impl, const gdn_opts_t *o, int P, int dk, int dv) {
+  return impl == GDN_IMPL_TC && P == 1 && o->impl != GDN_IMPL_TC_RESIDUAL && gdn_pform_supported(dk, dv);
 }
 
 // Chunk segments per frame (GDN_IMPL_TC).  The automatic choice considers
@@ -104,16 +113,27 @@ int gdn_segs(int impl, const gdn_opts_t *o, int sms, long units, int L) {
 // Workspace of gdn with P segments: the chain scratch over units * P segment
 // units, then (P > 1) each frame's end state as bf16 high/low pairs, d_k
 // words per row of S^T.
-size_t gdn_ws_bytes_p(int impl, int B, int H, int F, int dk, int dv, int P) {
+size_t gdn_ws_bytes_p(int impl, const gdn_opts_t *o, int B, int H, int F, int dk, int dv, int P) {
   if (impl == GDN_IMPL_SEQ) return 0;
   const long units = (long)B * H * F;
+  if (use_pform(impl, o, P, dk, dv))
+    return chain_workspace_bytes(units, (long)(gdn_pform_state_bytes(dk, dv) / sizeof(float)));
   size_t b = chain_workspace_bytes(units * P, (long)gdn_state_elems(impl, dk, dv));
   if (P > 1) b += align_up(sizeof(uint32_t) * (size_t)units * dk * dv, 256);
   return b;
 }
 
+// Workspace for any launch these sizes and options may lead to: the segment
+// count is chosen on the device, so both the most segments and one segment
+// (the product-form kernel) are covered.
 size_t gdn_ws_bytes(int impl, const gdn_opts_t *o, int B, int H, int F, int L, int dk, int dv) {
-  return gdn_ws_bytes_p(impl, B, H, F, dk, dv, gdn_seg_bound(impl, o, (long)B * H * F, L));
+  const int bound = gdn_seg_bound(impl, o, (long)B * H * F, L);
+  size_t b = gdn_ws_bytes_p(impl, o, B, H, F, dk, dv, bound);
+  if (bound > 1) {
+    const size_t b1 = gdn_ws_bytes_p(impl, o, B, H, F, dk, dv, 1);
+    if (b1 > b) b = b1;
+  }
+  return b;
 }
 
 size_t relu_ws_bytes(int B, int H, int F, int dk, int dv) {
@@ -147,9 +167,14 @@ extern "C" const char *gdn_status_string(int s) {
     case GDN_ERR_CUDA: return "CUDA runtime error";
     case GDN_ERR_TIMEOUT: return "device: a bounded in-kernel wait expired; outputs are invalid";
     case GDN_ERR_NO_DEVICE: return "no usable sm_100 device";
+    case GDN_ERR_RANGE:
+      return "device: a value met the fp16 range of the tensor-core operands (|q|, |v| or |S| >= 65504, or "
+             "NaN); outputs are invalid";
     default: return "unknown status";
   }
 }
+
+extern "C" const char *gdn_status_str(int s) { return gdn_status_string(s); }
 
 extern "C" size_t gdn_workspace_bytes(int op, int B, int H, int F, int L, int dk, int dv, const gdn_opts_t *opts) {
   if (!opts || check_sizes(B, H, F, L, dk, dv) != GDN_OK) return 0;
@@ -164,7 +189,7 @@ extern "C" int gdn_frame_fwd(const void *q, const void *k, const void *v, const 
   if (!opts) return GDN_ERR_INVALID_ARG;
   if (!q || !k || !v || !alpha || !beta || !o) return GDN_ERR_INVALID_ARG;
   if (opts->in_dtype != GDN_DTYPE_F32 && opts->in_dtype != GDN_DTYPE_BF16) return GDN_ERR_INVALID_ARG;
-  if (opts->impl < GDN_IMPL_AUTO || opts->impl > GDN_IMPL_TC) return GDN_ERR_INVALID_ARG;
+  if (opts->impl < GDN_IMPL_AUTO || opts->impl > GDN_IMPL_TC_RESIDUAL) return GDN_ERR_INVALID_ARG;
   int rc = check_sizes(B, H, F, L, dk, dv);
   if (rc != GDN_OK) return rc;
   const void *ptrs[] = {q, k, v, alpha, beta, state_in, state_out, o, opts->workspace, opts->status};
@@ -196,7 +221,7 @@ extern "C" int gdn_frame_fwd(const void *q, const void *k, const void *v, const 
   } else {
     const long units = (long)B * H * F;
     const int P = gdn_segs(impl, opts, sms, units, L);
-    const size_t need = gdn_ws_bytes_p(impl, B, H, F, dk, dv, P);
+    const size_t need = gdn_ws_bytes_p(impl, opts, B, H, F, dk, dv, P);
     if (!opts->workspace || opts->workspace_bytes < need) return GDN_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(opts->workspace) & 255u) != 0) return GDN_ERR_INVALID_ARG;
     p.ws = chain_workspace(opts->workspace, units * P);
@@ -207,8 +232,12 @@ extern "C" int gdn_frame_fwd(const void *q, const void *k, const void *v, const 
     e = cudaMemsetAsync(opts->workspace, 0, chain_workspace_zero_bytes(units * P), st);
     if (e != cudaSuccess) return GDN_ERR_CUDA;
     const int grid = P > 1 ? (int)(units * P) : grid_for(opts, sms, units);
-    e = impl == GDN_IMPL_TC ? launch_gdn_tc(p, grid, P > 1, st)
-                            : launch_gdn_frame_simt(p, opts->in_dtype, grid, st);
+    if (use_pform(impl, opts, P, dk, dv))
+      e = launch_gdn_pform(p, grid, st);
+    else if (impl == GDN_IMPL_TC)
+      e = launch_gdn_tc(p, grid, P > 1, st);
+    else
+      e = launch_gdn_frame_simt(p, opts->in_dtype, grid, st);
   }
   return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
@@ -256,40 +285,84 @@ extern "C" int relu_la_block_fwd(const void *q, const void *k, const void *v, co
 }
 
 // ---------------------------------------------------------------- host I/O
+//
+// gdn_frame_fwd_host streams the sequence through the device in groups of
+// frames: while group g runs, the inputs of group g + 1 are copied in and the
+// output of group g - 1 is copied out, on three streams.  The state passes
+// from group to group through state_out / state_in in fp32, which is how the
+// kernels hand it from frame to frame inside one call, so the result equals
+// that of one gdn_frame_fwd over the whole sequence.
 
 namespace {
+
+// Frames per group: about 16 groups, so the first copy in and the last copy
+// out (the parts that cannot overlap) are short.
+int host_group_frames(int F) { return F <= 16 ? 1 : (F + 15) / 16; }
+
 struct HostLayout {
-  size_t q, k, v, alpha, beta, s_in, o, s_out, ws, total;
+  int Fg;                          // frames per group (the last group may have fewer)
+  size_t slot;                     // bytes of one staging slot
+  size_t q, k, v, alpha, beta, o;  // offsets inside a slot
+  size_t s_in, s_out, s_a, s_b;    // fp32 states: caller's in / out, the two group hand-off buffers
+  size_t ws;                       // kernel workspace (sized for Fg frames)
+  size_t ws_bytes, total;
 };
 
-HostLayout host_layout(int B, int H, int F, int L, int dk, int dv, int in_dtype, size_t ws_bytes) {
-  const size_t esz = in_dtype == GDN_DTYPE_F32 ? 4 : 2;
-  const size_t N = (size_t)F * L, BH = (size_t)B * H;
+HostLayout host_layout(const gdn_opts_t *opts, int B, int H, int F, int L, int dk, int dv) {
+  const size_t esz = opts->in_dtype == GDN_DTYPE_F32 ? 4 : 2;
   HostLayout h;
+  h.Fg = host_group_frames(F);
+  const size_t BH = (size_t)B * H, Ng = (size_t)h.Fg * L;
   size_t off = 0;
   auto take = [&](size_t bytes) {
     size_t at = off;
     off = align_up(off + bytes, 256);
     return at;
   };
-  h.q = take(BH * N * dk * esz);
-  h.k = take(BH * N * dk * esz);
-  h.v = take(BH * N * dv * esz);
-  h.alpha = take(BH * F * 4);
-  h.beta = take(BH * N * 4);
-  h.s_in = take(BH * dk * dv * 4);
-  h.o = take(BH * N * dv * 4);
-  h.s_out = take(BH * dk * dv * 4);
-  h.ws = take(ws_bytes);
+  h.q = take(BH * Ng * dk * esz);
+  h.k = take(BH * Ng * dk * esz);
+  h.v = take(BH * Ng * dv * esz);
+  h.alpha = take(BH * h.Fg * 4);
+  h.beta = take(BH * Ng * 4);
+  h.o = take(BH * Ng * dv * 4);
+  h.slot = off;
+  off = 2 * h.slot;
+  const size_t sb = BH * dk * dv * 4;
+  h.s_in = take(sb);
+  h.s_out = take(sb);
+  h.s_a = take(sb);
+  h.s_b = take(sb);
+  h.ws_bytes = gdn_ws_bytes(pick_gdn_impl(opts, dk, dv), opts, B, H, h.Fg, L, dk, dv);
+  h.ws = take(h.ws_bytes);
   h.total = off;
   return h;
 }
+
+// Streams and events of one host call, released on every path out.
+struct HostStreams {
+  cudaStream_t up = nullptr, down = nullptr;
+  cudaEvent_t ev[4][2] = {};  // per slot: inputs in, group computed, output out, (spare)
+  bool ok = true;
+  HostStreams() {
+    ok = cudaStreamCreateWithFlags(&up, cudaStreamNonBlocking) == cudaSuccess &&
+         cudaStreamCreateWithFlags(&down, cudaStreamNonBlocking) == cudaSuccess;
+    for (auto &pair : ev)
+      for (auto &e : pair) ok = ok && cudaEventCreateWithFlags(&e, cudaEventDisableTiming) == cudaSuccess;
+  }
+  ~HostStreams() {
+    for (auto &pair : ev)
+      for (auto &e : pair)
+        if (e) cudaEventDestroy(e);
+    if (up) cudaStreamDestroy(up);
+    if (down) cudaStreamDestroy(down);
+  }
+};
+
 }  // namespace
 
 extern "C" size_t gdn_workspace_bytes_host(int B, int H, int F, int L, int dk, int dv, const gdn_opts_t *opts) {
   if (!opts || check_sizes(B, H, F, L, dk, dv) != GDN_OK) return 0;
-  const size_t ws = gdn_ws_bytes(pick_gdn_impl(opts, dk, dv), opts, B, H, F, L, dk, dv);
-  return host_layout(B, H, F, L, dk, dv, opts->in_dtype, ws).total;
+  return host_layout(opts, B, H, F, L, dk, dv).total;
 }
 
 extern "C" int gdn_frame_fwd_host(const void *q, const void *k, const void *v, const float *alpha,
@@ -299,34 +372,70 @@ extern "C" int gdn_frame_fwd_host(const void *q, const void *k, const void *v, c
   if (opts->in_dtype != GDN_DTYPE_F32 && opts->in_dtype != GDN_DTYPE_BF16) return GDN_ERR_INVALID_ARG;
   int rc = check_sizes(B, H, F, L, dk, dv);
   if (rc != GDN_OK) return rc;
-  const size_t ws = gdn_ws_bytes(pick_gdn_impl(opts, dk, dv), opts, B, H, F, L, dk, dv);
-  const HostLayout h = host_layout(B, H, F, L, dk, dv, opts->in_dtype, ws);
+  const HostLayout h = host_layout(opts, B, H, F, L, dk, dv);
   if (!opts->workspace || opts->workspace_bytes < h.total) return GDN_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(opts->workspace) & 255u) != 0) return GDN_ERR_INVALID_ARG;
   char *base = (char *)opts->workspace;
   cudaStream_t st = (cudaStream_t)opts->stream;
   const size_t esz = opts->in_dtype == GDN_DTYPE_F32 ? 4 : 2;
   const size_t N = (size_t)F * L, BH = (size_t)B * H;
-  struct Cp { void *dst; const void *src; size_t n; };
-  const Cp in[] = {{base + h.q, q, BH * N * dk * esz}, {base + h.k, k, BH * N * dk * esz},
-                   {base + h.v, v, BH * N * dv * esz}, {base + h.alpha, alpha, BH * F * 4},
-                   {base + h.beta, beta, BH * N * 4},  {base + h.s_in, state_in, BH * dk * dv * 4}};
-  for (const Cp &c : in) {
-    if (!c.src) continue;
-    if (cudaMemcpyAsync(c.dst, c.src, c.n, cudaMemcpyHostToDevice, st) != cudaSuccess) return GDN_ERR_CUDA;
-  }
+  const size_t sbytes = BH * dk * dv * 4;
+  HostStreams hs;
+  if (!hs.ok) return GDN_ERR_CUDA;
+  // the up and down streams start after whatever the caller queued on opts->stream
+  if (cudaEventRecord(hs.ev[3][0], st) != cudaSuccess || cudaStreamWaitEvent(hs.up, hs.ev[3][0], 0) != cudaSuccess ||
+      cudaStreamWaitEvent(hs.down, hs.ev[3][0], 0) != cudaSuccess)
+    return GDN_ERR_CUDA;
+  if (state_in && cudaMemcpyAsync(base + h.s_in, state_in, sbytes, cudaMemcpyHostToDevice, hs.up) != cudaSuccess)
+    return GDN_ERR_CUDA;
+  const int G = (F + h.Fg - 1) / h.Fg;
   gdn_opts_t inner = *opts;
   inner.workspace = base + h.ws;
-  inner.workspace_bytes = ws;
-  rc = gdn_frame_fwd(base + h.q, base + h.k, base + h.v, (const float *)(base + h.alpha),
-                     (const float *)(base + h.beta), state_in ? (const float *)(base + h.s_in) : nullptr,
-                     state_out ? (float *)(base + h.s_out) : nullptr, (float *)(base + h.o), B, H, F, L, dk, dv,
-                     &inner);
-  if (rc != GDN_OK) return rc;
-  if (cudaMemcpyAsync(o, base + h.o, BH * N * dv * 4, cudaMemcpyDeviceToHost, st) != cudaSuccess)
-    return GDN_ERR_CUDA;
+  inner.workspace_bytes = h.ws_bytes;
+  for (int gi = 0; gi < G; ++gi) {
+    const int f0 = gi * h.Fg, Fn = F - f0 < h.Fg ? F - f0 : h.Fg;
+    const int sl = gi & 1;
+    char *slot = base + (size_t)sl * h.slot;
+    const size_t t0 = (size_t)f0 * L, nt = (size_t)Fn * L;
+    cudaEvent_t in_done = hs.ev[sl][0], computed = hs.ev[sl][1], out_done = hs.ev[2][sl];
+    // inputs of group gi (the slot's previous group must have been computed)
+    if (gi >= 2 && cudaStreamWaitEvent(hs.up, computed, 0) != cudaSuccess) return GDN_ERR_CUDA;
+    struct Cp2 { void *dst; const void *src; size_t row, pitch; };
+    const Cp2 ins[] = {
+        {slot + h.q, (const char *)q + t0 * dk * esz, nt * dk * esz, N * dk * esz},
+        {slot + h.k, (const char *)k + t0 * dk * esz, nt * dk * esz, N * dk * esz},
+        {slot + h.v, (const char *)v + t0 * dv * esz, nt * dv * esz, N * dv * esz},
+        {slot + h.alpha, (const char *)alpha + (size_t)f0 * 4, (size_t)Fn * 4, (size_t)F * 4},
+        {slot + h.beta, (const char *)beta + t0 * 4, nt * 4, N * 4}};
+    for (const Cp2 &c : ins)
+      if (cudaMemcpy2DAsync(c.dst, c.row, c.src, c.pitch, c.row, BH, cudaMemcpyHostToDevice, hs.up) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    if (cudaEventRecord(in_done, hs.up) != cudaSuccess) return GDN_ERR_CUDA;
+    // the group on the caller's stream, once its inputs are in and the slot's previous
+    // output has been copied out
+    if (cudaStreamWaitEvent(st, in_done, 0) != cudaSuccess) return GDN_ERR_CUDA;
+    if (gi >= 2 && cudaStreamWaitEvent(st, out_done, 0) != cudaSuccess) return GDN_ERR_CUDA;
+    const float *sin = gi == 0 ? (state_in ? (const float *)(base + h.s_in) : nullptr)
+                               : (const float *)(base + ((gi - 1) & 1 ? h.s_b : h.s_a));
+    float *sout = gi == G - 1 ? (state_out ? (float *)(base + h.s_out) : nullptr)
+                              : (float *)(base + (gi & 1 ? h.s_b : h.s_a));
+    rc = gdn_frame_fwd(slot + h.q, slot + h.k, slot + h.v, (const float *)(slot + h.alpha),
+                       (const float *)(slot + h.beta), sin, sout, (float *)(slot + h.o), B, H, Fn, L, dk, dv,
+                       &inner);
+    if (rc != GDN_OK) return rc;
+    if (cudaEventRecord(computed, st) != cudaSuccess) return GDN_ERR_CUDA;
+    // output of group gi
+    if (cudaStreamWaitEvent(hs.down, computed, 0) != cudaSuccess) return GDN_ERR_CUDA;
+    if (cudaMemcpy2DAsync((char *)o + t0 * dv * 4, N * dv * 4, slot + h.o, nt * dv * 4, nt * dv * 4, BH,
+                          cudaMemcpyDeviceToHost, hs.down) != cudaSuccess)
+      return GDN_ERR_CUDA;
+    if (cudaEventRecord(out_done, hs.down) != cudaSuccess) return GDN_ERR_CUDA;
+  }
   if (state_out &&
-      cudaMemcpyAsync(state_out, base + h.s_out, BH * dk * dv * 4, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+      cudaMemcpyAsync(state_out, base + h.s_out, sbytes, cudaMemcpyDeviceToHost, hs.down) != cudaSuccess)
+    return GDN_ERR_CUDA;
+  // the caller's stream waits for the last copy out, then the call returns
+  if (cudaEventRecord(hs.ev[3][1], hs.down) != cudaSuccess || cudaStreamWaitEvent(st, hs.ev[3][1], 0) != cudaSuccess)
     return GDN_ERR_CUDA;
   return cudaStreamSynchronize(st) == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }

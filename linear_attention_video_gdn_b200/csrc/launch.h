@@ -14,6 +14,11 @@ bool gdn_tc_supported(int dk, int dv);
 size_t gdn_tc_state_elems(int dk, int dv);
 // cooperative: p.segs > 1; all CTAs resident at once (segments wait across CTAs both ways)
 cudaError_t launch_gdn_tc(const GdnParams &p, int grid, bool cooperative, cudaStream_t st);
+// product-form tensor-core kernel: one CTA per frame, sizes where its shared memory and
+// TMEM maps fit (make_layout in gdn_pform.cu)
+bool gdn_pform_supported(int dk, int dv);
+size_t gdn_pform_state_bytes(int dk, int dv);  // published bytes per frame
+cudaError_t launch_gdn_pform(const GdnParams &p, int grid, cudaStream_t st);
 bool relu_tc_supported(int dk, int dv);
 cudaError_t launch_relu_tc(const ReluParams &p, int grid, cudaStream_t st);
 

@@ -27,16 +27,27 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[GDN_NOALLOC_SCR
 constexpr int kMaxDev = 64;
 std::atomic<void *> g_scratch_addr[kMaxDev];
 
-// Device address of g_noalloc_scratch on the current device, looked up once per
-// device with that device current.  The host-side name is only a stand-in, so
-// kernels must be given this address, never &g_noalloc_scratch.
-int scratch_address(void **out) {
+// Device address of g_noalloc_scratch on the current device.  The host-side
+// name is only a stand-in, so kernels must be given this address, never
+// &g_noalloc_scratch.  The address is looked up with the device current on
+// every call made outside stream capture (after a device reset the runtime
+// loads the module again, possibly elsewhere, so a cached address could be
+// stale) and remembered per device for calls made while `st` is being
+// captured, which do not look it up; so the first call on a device must come
+// before any capture.
+int scratch_address(cudaStream_t st, void **out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return GDN_ERR_NO_DEVICE;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) return GDN_ERR_CUDA;
   void *p = g_scratch_addr[dev].load(std::memory_order_acquire);
-  if (!p) {
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return GDN_ERR_CUDA;
-    g_scratch_addr[dev].store(p, std::memory_order_release);
+  if (cs == cudaStreamCaptureStatusNone) {
+    void *fresh = nullptr;
+    if (cudaGetSymbolAddress(&fresh, g_noalloc_scratch) != cudaSuccess || fresh == nullptr) return GDN_ERR_CUDA;
+    if (fresh != p) g_scratch_addr[dev].store(fresh, std::memory_order_release);
+    p = fresh;
+  } else if (p == nullptr) {
+    return GDN_ERR_INVALID_ARG;  // first call on this device inside a capture: not supported
   }
   *out = p;
   return GDN_OK;
@@ -52,7 +63,7 @@ extern "C" int gdn_frame_fwd_noalloc(const void *q, const void *k, const void *v
   const size_t need = gdn_workspace_bytes(GDN_OP_GDN, B, H, F, L, dk, dv, opts);
   if (need > (size_t)GDN_NOALLOC_SCRATCH_BYTES) return GDN_ERR_UNSUPPORTED;
   void *scratch = nullptr;
-  const int rc = gdn::scratch_address(&scratch);
+  const int rc = gdn::scratch_address((cudaStream_t)opts->stream, &scratch);
   if (rc != GDN_OK) return rc;
   gdn_opts_t o2 = *opts;
   o2.workspace = scratch;

@@ -9,15 +9,28 @@ TOL_F32 = 1e-5   # same, fp32 inputs
 
 
 def rel_err(x, ref):
-    """max|x - ref| / max|ref| over the finite entries of ref (NaN marks uncomputed entries)."""
-    x = np.asarray(x, np.float64)
-    ref = np.asarray(ref, np.float64)
-    m = np.isfinite(ref)
-    assert m.any()
-    scale = np.abs(ref[m]).max()
-    if not np.isfinite(x[m]).all():
-        return float("inf")
-    return float(np.abs(x[m] - ref[m]).max() / max(scale, 1e-30))
+    """max|x - ref| / max|ref| over the finite entries of ref (NaN marks uncomputed entries).
+
+    Streams over the flattened arrays in blocks, so full-size outputs (about
+    5e8 elements) need no multi-gigabyte temporaries."""
+    x = np.asarray(x).reshape(-1)
+    ref = np.asarray(ref).reshape(-1)
+    assert x.size == ref.size
+    scale, err, any_ref = 0.0, 0.0, False
+    step = 1 << 24
+    for i in range(0, ref.size, step):
+        r = ref[i:i + step].astype(np.float64, copy=False)
+        m = np.isfinite(r)
+        if not m.any():
+            continue
+        any_ref = True
+        xs = x[i:i + step].astype(np.float64, copy=False)
+        if not np.isfinite(xs[m]).all():
+            return float("inf")
+        scale = max(scale, float(np.abs(r[m]).max()))
+        err = max(err, float(np.abs(xs[m] - r[m]).max()))
+    assert any_ref
+    return err / max(scale, 1e-30)
 
 
 def device_inputs(w, x, dev, torch):

@@ -36,6 +36,18 @@ def test_exports_every_declared_symbol(lib):
     assert set(names) == set(lib.EXPORTED)
 
 
+def test_boundary_names(lib):
+    """The boundary's calls: the two recurrences, the workspace query and the
+    status description (under both of its names)."""
+    raw = ctypes.CDLL(lib.LIB_PATH)
+    for n in ("gdn_frame_fwd", "relu_la_block_fwd", "gdn_workspace_bytes", "gdn_status_str", "gdn_status_string"):
+        assert hasattr(raw, n), n
+    raw.gdn_status_str.restype = ctypes.c_char_p
+    raw.gdn_status_string.restype = ctypes.c_char_p
+    for code in range(7):
+        assert raw.gdn_status_str(code) == raw.gdn_status_string(code)
+
+
 def test_header_constants_match_binding(lib):
     text = open(HEADER).read()
     consts = dict((k, int(v)) for k, v in re.findall(r"#define (GDN_\w+) (\d+)", text))
@@ -49,8 +61,8 @@ def test_header_constants_match_binding(lib):
 
 
 def test_status_strings(lib):
-    for code in range(6):
-        assert isinstance(lib.status_string(code), str) and lib.status_string(code)
+    for code in range(7):
+        assert isinstance(lib.status_string(code), str) and lib.status_string(code) != "unknown status"
     assert lib.status_string(99) == "unknown status"
 
 
@@ -70,26 +82,33 @@ def test_workspace_sizes(lib):
 
 
 def test_workspace_sizes_with_segments(lib):
-    """The tcgen05 path sizes its scratch for the most chunk segments a launch
-    may use: fp16 states and flags per segment unit, plus one bf16 high/low
-    end state per frame; one segment for many frames or one-chunk frames."""
+    """The tcgen05 path sizes its scratch for any launch the sizes may lead to:
+    with P chunk segments (residual-form kernel) fp16 states and flags per
+    segment unit plus one bf16 high/low end state per frame; with one segment
+    per frame (product-form kernel) fp16 high and low state images per frame."""
     d = 112
 
-    def need(B, H, F, L, **kw):
-        return lib.workspace_bytes(lib.OP_GDN, B, H, F, L, d, d, lib.make_opts(lib.DTYPE_BF16, impl="tc", stream=0,
+    def need(B, H, F, L, impl="tc", **kw):
+        return lib.workspace_bytes(lib.OP_GDN, B, H, F, L, d, d, lib.make_opts(lib.DTYPE_BF16, impl=impl, stream=0,
                                                                                **kw))
 
-    def layout(units, P):  # counter block, flags, fp16 states, then the end states (P > 1)
-        up = lambda x: (x + 255) // 256 * 256
+    up = lambda x: (x + 255) // 256 * 256
+
+    def residual(units, P):  # counter block, flags, fp16 states, then the end states (P > 1)
         return 256 + up(4 * units * P) + up(units * P * d * d * 2) + (up(units * d * d * 4) if P > 1 else 0)
 
+    def pform(units):  # counter block, flags, high + low images: 2 blocks of 64 columns x d rows x 2 bytes each
+        return 256 + up(4 * units) + up(units * 2 * (2 * d * 128))
+
     nch = (920 + 63) // 64
-    assert need(1, 20, 1, 920) == layout(20, min(nch, 8))                 # a streaming call: auto bound
-    assert need(1, 20, 1, 920, segments=1) == layout(20, 1)
-    assert need(1, 20, 1, 920, segments=3) == layout(20, 3)
-    assert need(1, 20, 1, 920, segments=99) == layout(20, nch)             # at most one chunk each
-    assert need(1, 20, 240, 920) == layout(4800, 1)                        # many frames: one segment
-    assert need(1, 20, 1, 64) == layout(20, 1)                             # one chunk per frame
+    assert need(1, 20, 1, 920) == max(residual(20, min(nch, 8)), pform(20))   # a streaming call: auto bound
+    assert need(1, 20, 1, 920, segments=1) == pform(20)
+    assert need(1, 20, 1, 920, segments=1, impl="tc_residual") == residual(20, 1)
+    assert need(1, 20, 1, 920, segments=3) == max(residual(20, 3), pform(20))
+    assert need(1, 20, 1, 920, segments=99) == max(residual(20, nch), pform(20))  # at most one chunk each
+    assert need(1, 20, 240, 920) == pform(4800)                                # many frames: one segment
+    assert need(1, 20, 240, 920, impl="tc_residual") == residual(4800, 1)
+    assert need(1, 20, 1, 64) == pform(20)                                     # one chunk per frame
     simt = lib.make_opts(lib.DTYPE_BF16, impl="frame_simt", stream=0, segments=4)
     assert lib.workspace_bytes(lib.OP_GDN, 1, 20, 1, 920, d, d, simt) == 256 + 256 + 20 * d * d * 4
 

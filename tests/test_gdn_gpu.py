@@ -8,7 +8,7 @@ tol = 2e-3 for bf16 inputs and 1e-5 for fp32 inputs.
 import numpy as np
 import pytest
 
-from helpers import device_inputs, oracle_gdn, rel_err, synth, tol_for
+from helpers import device_inputs, oracle, oracle_gdn, rel_err, synth, tol_for
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
@@ -69,29 +69,43 @@ def test_480p_5s(lib, dev, impl):
 
 
 @pytest.mark.parametrize("impl", ["frame_simt", "tc"])
-def test_720p_60s_sampled(lib, dev, impl):
-    """Full 720p-60s size in the benchmark's launch configuration; the oracle
-    recomputes two heads on a subset of d_v columns (columns evolve independently)."""
+def test_720p_60s_full(lib, dev, impl):
+    """Full 720p-60s workload in the benchmark's launch configuration, every
+    head and every d_v column (including columns 64-111, which come from the
+    second, zero-padded 64-wide tile) and the final state, against the oracle
+    run over all heads on every host core."""
     w = W["gdn_720p_60s"]
     x = synth.inputs(w)
     t, h = device_inputs(w, x, dev, torch)
     o, s = run_gdn(lib, w, t, dev, impl)
-    heads = [0, 13]
-    cols = (40, 56)
-    sub = {n: h[n].reshape((w.B * w.H,) + h[n].shape[2:])[heads] for n in "qkvab"}
-    o_ref, s_ref = synth_free_oracle(sub, w, cols)
-    o_g = o.reshape((w.B * w.H,) + o.shape[2:])[heads]
-    s_g = s.reshape((w.B * w.H,) + s.shape[2:])[heads]
-    eo, es = rel_err(o_g[..., cols[0]:cols[1]], o_ref[..., cols[0]:cols[1]]), \
-        rel_err(s_g[..., cols[0]:cols[1]], s_ref[..., cols[0]:cols[1]])
-    print(f"720p {impl}: err_o={eo:.3e} err_s={es:.3e}")
-    assert eo <= 2e-3 and es <= 2e-3
-    assert np.isfinite(o).all() and np.isfinite(s).all()
+    o_ref, s_ref = oracle_gdn(h, w)
+    eo, es = rel_err(o, o_ref), rel_err(s, s_ref)
+    eo_hi = rel_err(o[..., 64:], o_ref[..., 64:])
+    print(f"720p {impl}: err_o={eo:.3e} (cols 64-111: {eo_hi:.3e}) err_s={es:.3e}")
+    assert eo <= 2e-3 and es <= 2e-3 and eo_hi <= 2e-3
 
 
-def synth_free_oracle(sub, w, cols):
-    from helpers import oracle
-    return oracle.gdn(sub["q"], sub["k"], sub["v"], sub["a"], sub["b"], F=w.F, L=w.L, cols=cols)
+def test_alpha_one_long_sequence_drift(lib, dev):
+    """No forgetting (alpha = 1 given as values) over 240 frames of 128 tokens:
+    the state is carried from frame to frame by the tensor-core chain for the
+    whole sequence, so rounding in the carried state would accumulate here."""
+    w = W["gdn_480p_5s"].with_(F=240, L=128, H=4, seed=21)
+    x = synth.inputs(w)
+    t, h = device_inputs(w, x, dev, torch)
+    ones = torch.ones_like(t["a"])
+    beta = torch.sigmoid(t["b"])
+    h1 = dict(h)
+    h1["a"] = np.ones_like(h["a"])
+    h1["b"] = beta.cpu().numpy()
+    o_ref, s_ref = oracle.gdn(h1["q"], h1["k"], h1["v"], h1["a"], h1["b"], F=w.F, L=w.L, gates_are_logits=False)
+    for impl in ("tc", "frame_simt"):
+        s_out = torch.empty((w.B, w.H, w.dk, w.dv), dtype=torch.float32, device=dev)
+        o = lib.gdn_frame_fwd(t["q"], t["k"], t["v"], ones, beta, F=w.F, gates_are_logits=False,
+                              state_out=s_out, impl=impl)
+        torch.cuda.synchronize()
+        eo, es = rel_err(o.cpu().numpy(), o_ref), rel_err(s_out.cpu().numpy(), s_ref)
+        print(f"alpha=1 drift {impl}: err_o={eo:.3e} err_s={es:.3e}")
+        assert eo <= 2e-3 and es <= 2e-3, impl
 
 
 # ------------------------------------------------------------------ shapes and tails
@@ -317,3 +331,53 @@ def test_segment_timeout_status_is_reported(lib, dev):
     o_ref, s_ref = oracle_gdn(h, w)
     assert rel_err(o, o_ref) <= 2e-3
     assert rel_err(s, s_ref) <= 2e-3
+
+
+# ------------------------------------------------------------------ streaming block-cache protocol
+
+def _stream_call_inputs(w, c, dev):
+    x = synth.inputs(w, call=c)
+    t = {n: torch.from_numpy(x[n]).to(torch.bfloat16) for n in "qkv"}
+    host = {n: t[n].float().numpy() for n in "qkv"}
+    host.update(a=x["a"], b=x["b"])
+    dv_ = {n: t[n].to(dev).contiguous() for n in "qkv"}
+    dv_.update(a=torch.from_numpy(x["a"]).to(dev), b=torch.from_numpy(x["b"]).to(dev))
+    return dv_, host
+
+
+@pytest.mark.parametrize("segments", [0, 1])
+def test_streaming_protocol_720p(lib, dev, segments):
+    """The streaming block-cache decode at the 720p frame shape (20 heads, one
+    920-token frame per call): 8 frames x 4 denoising steps, fresh q, k, v and
+    gates on every call, state_out = NULL on steps 1-3 and the committed state
+    on step 4, which becomes the next frame's state_in.  Every call's o and
+    every committed state are compared with the streaming oracle, and a
+    non-committing call must leave state_in byte for byte as it was."""
+    steps, frames = 4, 8
+    w = W["gdn_stream_720p"]
+    calls = [_stream_call_inputs(w, c, dev) for c in range(frames * steps)]
+    outs_ref, _, committed_ref = oracle.gdn_stream(lambda c: calls[c][1] if c < len(calls) else None,
+                                                   steps=steps, L=w.L)
+    shape_s = (w.B, w.H, w.dk, w.dv)
+    s_cur = None
+    worst_o = worst_s = 0.0
+    for f in range(frames):
+        s_next = torch.empty(shape_s, dtype=torch.float32, device=dev)
+        before = None if s_cur is None else s_cur.clone()
+        for st in range(steps):
+            c = f * steps + st
+            t = calls[c][0]
+            commit = st == steps - 1
+            o = lib.gdn_frame_fwd(t["q"], t["k"], t["v"], t["a"], t["b"], F=1, state_in=s_cur,
+                                  state_out=s_next if commit else None, segments=segments)
+            torch.cuda.synchronize()
+            e = rel_err(o.cpu().numpy(), outs_ref[c])
+            worst_o = max(worst_o, e)
+            assert e <= 2e-3, (f, st, e)
+            if not commit and before is not None:
+                assert torch.equal(s_cur, before), (f, st)  # state_in untouched
+        e = rel_err(s_next.cpu().numpy(), committed_ref[f])
+        worst_s = max(worst_s, e)
+        assert e <= 2e-3, (f, e)
+        s_cur = s_next
+    print(f"streaming protocol segments={segments}: worst err_o={worst_o:.3e} err_s={worst_s:.3e}")

@@ -50,22 +50,17 @@ def run(lib, w, t, dev, impl, kv_in=None, z_in=None, **kw):
 
 
 @pytest.mark.parametrize("impl", ["frame_simt", "tc"])
-def test_relu_720p_81f_sampled(lib, dev, impl):
-    """Full-size workload (B=2, H=20, F=81, L=920); the oracle recomputes 3 heads."""
+def test_relu_720p_81f_full(lib, dev, impl):
+    """Full-size workload (B=2, H=20, F=81, L=920): every head, o, kv_out and
+    z_out against the oracle (heads spread over the host cores)."""
     w = W["relu_720p_81f"]
     x = synth.inputs(w)
     t, h = prep(w, x, dev)
     o, kv, z = run(lib, w, t, dev, impl)
-    heads = [0, 21, 39]
-    flat = lambda a: a.reshape((w.B * w.H,) + a.shape[2:])
-    sub = {n: flat(h[n])[heads] for n in "qkv"}
-    o_ref, kv_ref, z_ref = oracle.relu_la(sub["q"], sub["k"], sub["v"], F=w.F, L=w.L)
-    eo = rel_err(flat(o)[heads], o_ref)
-    ek = rel_err(flat(kv)[heads], kv_ref)
-    ez = rel_err(flat(z)[heads], z_ref)
+    o_ref, kv_ref, z_ref = oracle.relu_la(h["q"], h["k"], h["v"], F=w.F, L=w.L)
+    eo, ek, ez = rel_err(o, o_ref), rel_err(kv, kv_ref), rel_err(z, z_ref)
     print(f"relu 720p {impl}: err_o={eo:.3e} err_kv={ek:.3e} err_z={ez:.3e}")
     assert eo <= 2e-3 and ek <= 2e-3 and ez <= 2e-3
-    assert np.isfinite(o).all()
 
 
 SHAPES = [(1, 1, 32, 32, 1), (3, 63, 112, 112, 2), (2, 64, 64, 64, 1), (2, 65, 112, 112, 1), (5, 20, 128, 128, 1),

@@ -5,16 +5,16 @@ of their own (a plugin inside a host program that owns all device memory, a
 runtime with a fixed memory plan).  For them the library keeps its own
 fixed-size scratch array; this file checks, through the C ABI, that the
 no-allocation call gives the same result as the regular call with a
-caller workspace, on two calls in a row (the shared scratch keeps the previous
-call's contents, which must not leak into the next), and that sizes beyond the
-scratch limit are refused.  It is named so that pytest collects it last.
+caller workspace and as the fp64 oracle, on two calls in a row (the shared
+scratch keeps the previous call's contents, which must not leak into the next),
+and that sizes beyond the scratch limit are refused.  It is named so that pytest collects it last.
 """
 import ctypes
 
 import numpy as np
 import pytest
 
-from helpers import device_inputs, rel_err, synth
+from helpers import device_inputs, oracle_gdn, rel_err, synth
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
@@ -50,13 +50,18 @@ def test_noalloc_matches_regular_on_two_calls(lib):
              synth.WORKLOADS["gdn_480p_5s"].with_(F=3, L=200, seed=77)]   # different sizes and inputs
     for i, w in enumerate(cases):
         x = synth.inputs(w)
-        t, _ = device_inputs(w, x, dev, torch)
-        S0 = torch.from_numpy(np.random.default_rng(i).standard_normal((w.B, w.H, w.dk, w.dv)).astype(np.float32)).to(dev)
-        o_ref, s_ref = _regular(lib, w, t, dev, S0)
+        t, h = device_inputs(w, x, dev, torch)
+        S0h = np.random.default_rng(i).standard_normal((w.B, w.H, w.dk, w.dv)).astype(np.float32)
+        S0 = torch.from_numpy(S0h).to(dev)
+        o_reg, s_reg = _regular(lib, w, t, dev, S0)
         o, s = _noalloc_via_cabi(lib, w, t, dev, S0)
         torch.cuda.synchronize()
-        assert rel_err(o.cpu().numpy(), o_ref.cpu().numpy()) <= 2e-3
-        assert rel_err(s.cpu().numpy(), s_ref.cpu().numpy()) <= 2e-3
+        o, s = o.cpu().numpy(), s.cpu().numpy()
+        assert rel_err(o, o_reg.cpu().numpy()) <= 2e-3
+        assert rel_err(s, s_reg.cpu().numpy()) <= 2e-3
+        o_ref, s_ref = oracle_gdn(h, w, state_in=S0h)
+        assert rel_err(o, o_ref) <= 2e-3
+        assert rel_err(s, s_ref) <= 2e-3
 
 
 def test_noalloc_refuses_sizes_beyond_its_scratch(lib):
