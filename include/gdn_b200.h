@@ -76,11 +76,12 @@ extern "C" {
 #define GDN_IMPL_AUTO 0
 #define GDN_IMPL_SEQ 1          /* per-token SIMT recurrence, one CTA per head (reference-simple) */
 #define GDN_IMPL_FRAME_SIMT 2   /* frame maps + ticketed frame chain, CUDA cores, fp32 arithmetic */
-#define GDN_IMPL_TC 3           /* frame maps + chain on tcgen05/TMEM tensor cores (bf16 inputs): the
-                                   product-form kernel where its sizes allow it and frames are not
-                                   split into segments, else the residual-form kernel */
-#define GDN_IMPL_TC_RESIDUAL 4  /* the residual-form tensor-core kernel only (any d_k, d_v multiple of
-                                   16 up to 128; also splits frames into chunk segments) */
+#define GDN_IMPL_TC 3           /* frame maps + chain on tcgen05/TMEM tensor cores (bf16 inputs),
+                                   residual form (any d_k, d_v multiple of 16 up to 128; splits frames
+                                   into chunk segments when frames are few) */
+#define GDN_IMPL_TC_PFORM 4     /* tcgen05 kernel with the chunk map in product form, one CTA per
+                                   frame (sizes where its shared-memory and TMEM maps fit; see
+                                   gdn_pform_supported in the library); GDN_ERR_UNSUPPORTED otherwise */
 
 /* operation ids for gdn_workspace_bytes() */
 #define GDN_OP_GDN 0

@@ -25,10 +25,10 @@ _lib = ctypes.CDLL(LIB_PATH)
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_NO_DEVICE, ERR_RANGE = range(7)
 DTYPE_F32, DTYPE_BF16 = 0, 1
-IMPL_AUTO, IMPL_SEQ, IMPL_FRAME_SIMT, IMPL_TC, IMPL_TC_RESIDUAL = 0, 1, 2, 3, 4
+IMPL_AUTO, IMPL_SEQ, IMPL_FRAME_SIMT, IMPL_TC, IMPL_TC_PFORM = 0, 1, 2, 3, 4
 OP_GDN, OP_RELU_LA = 0, 1
 IMPLS = {"auto": IMPL_AUTO, "seq": IMPL_SEQ, "frame_simt": IMPL_FRAME_SIMT, "tc": IMPL_TC,
-         "tc_residual": IMPL_TC_RESIDUAL}
+         "tc_pform": IMPL_TC_PFORM}
 
 EXPORTED = ("gdn_frame_fwd", "relu_la_block_fwd", "gdn_frame_fwd_host", "gdn_frame_fwd_noalloc",
             "gdn_workspace_bytes", "gdn_workspace_bytes_host", "gdn_status_string", "gdn_status_str",

@@ -46,7 +46,7 @@ int check_sizes(int B, int H, int F, int L, int dk, int dv) {
 }
 
 int pick_gdn_impl(const gdn_opts_t *o, int dk, int dv) {
-  if (o->impl == GDN_IMPL_TC_RESIDUAL) return GDN_IMPL_TC;
+  if (o->impl == GDN_IMPL_TC_PFORM) return GDN_IMPL_TC;
   if (o->impl != GDN_IMPL_AUTO) return o->impl;
   if (o->in_dtype == GDN_DTYPE_BF16 && gdn_tc_supported(dk, dv)) return GDN_IMPL_TC;
   return GDN_IMPL_FRAME_SIMT;
@@ -65,10 +65,9 @@ size_t gdn_state_elems(int impl, int dk, int dv) {
   return (size_t)dk * dv;
 }
 
-// The product-form tensor-core kernel runs for GDN_IMPL_TC launches with one
-// segment per frame whose sizes it supports.
+// The product-form tensor-core kernel runs when it is asked for (one segment per frame).
 bool use_pform(int impl, const gdn_opts_t *o, int P, int dk, int dv) {
-  return impl == GDN_IMPL_TC && P == 1 && o->impl != GDN_IMPL_TC_RESIDUAL && gdn_pform_supported(dk, dv);
+  return impl == GDN_IMPL_TC && o->impl == GDN_IMPL_TC_PFORM && P == 1 && gdn_pform_supported(dk, dv);
 }
 
 // Chunk segments per frame (GDN_IMPL_TC).  The automatic choice considers
@@ -80,7 +79,7 @@ constexpr int kMaxSegs = 8;
 // The most segments a launch with these sizes and options may use; sizes the
 // workspace without asking the device.
 int gdn_seg_bound(int impl, const gdn_opts_t *o, long units, int L) {
-  if (impl != GDN_IMPL_TC) return 1;
+  if (impl != GDN_IMPL_TC || o->impl == GDN_IMPL_TC_PFORM) return 1;
   const int nch = (L + 63) / 64;
   if (o->segments > 0) return o->segments < nch ? o->segments : nch;
   if (units > kSegUnitsMax) return 1;
@@ -189,7 +188,7 @@ extern "C" int gdn_frame_fwd(const void *q, const void *k, const void *v, const 
   if (!opts) return GDN_ERR_INVALID_ARG;
   if (!q || !k || !v || !alpha || !beta || !o) return GDN_ERR_INVALID_ARG;
   if (opts->in_dtype != GDN_DTYPE_F32 && opts->in_dtype != GDN_DTYPE_BF16) return GDN_ERR_INVALID_ARG;
-  if (opts->impl < GDN_IMPL_AUTO || opts->impl > GDN_IMPL_TC_RESIDUAL) return GDN_ERR_INVALID_ARG;
+  if (opts->impl < GDN_IMPL_AUTO || opts->impl > GDN_IMPL_TC_PFORM) return GDN_ERR_INVALID_ARG;
   int rc = check_sizes(B, H, F, L, dk, dv);
   if (rc != GDN_OK) return rc;
   const void *ptrs[] = {q, k, v, alpha, beta, state_in, state_out, o, opts->workspace, opts->status};
@@ -202,6 +201,7 @@ extern "C" int gdn_frame_fwd(const void *q, const void *k, const void *v, const 
   const int impl = pick_gdn_impl(opts, dk, dv);
   if (impl == GDN_IMPL_TC && (opts->in_dtype != GDN_DTYPE_BF16 || !gdn_tc_supported(dk, dv)))
     return GDN_ERR_UNSUPPORTED;
+  if (opts->impl == GDN_IMPL_TC_PFORM && !gdn_pform_supported(dk, dv)) return GDN_ERR_UNSUPPORTED;
 
   cudaStream_t st = (cudaStream_t)opts->stream;
   GdnParams p;

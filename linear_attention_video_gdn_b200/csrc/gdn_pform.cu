@@ -55,12 +55,14 @@ constexpr int kThreads = 512;
 constexpr int kChain = 256;
 constexpr int kC = 64;               // tokens per chunk
 constexpr int kSlots = 3;            // chunks of k, v in flight
-constexpr int kQT = 128;             // tokens per read-out tile
+constexpr int kMaxQT = 64;           // most tokens per read-out tile
+constexpr int kQBuf = 3;             // q tiles in flight in the read-out
+constexpr int kStageTok = 32;        // tokens per bulk store of o
 constexpr uint32_t kSlotBytes = 32768;
 constexpr uint32_t kSlK = 0;         // khat: [col block][64 t][128 B] (TMA'd bf16, fp16 in place)
 constexpr uint32_t kSlV = 16384;     // v:    [col block][64 t][128 B]
 constexpr uint32_t kPrepBytes = 16384;   // per prep group: N (fp32 64 x 64), then T (fp16, 64 rows t x 128 B)
-constexpr uint32_t kQTileBytes = 32768;  // q tile: [col block][128 t][128 B]
+
 constexpr int kMaxSmem = 232448;
 
 struct Bars {
@@ -72,8 +74,7 @@ struct Bars {
   uint64_t y_mma;              // chain: the chunk's MMAs are done
   uint64_t fr_bar;             // chain step MMAs
   uint64_t s_full[2];          // bulk copies of S_{f-1}: low, high image
-  uint64_t q_full[2];          // read-out: q tile in buffer b (TMA)
-  uint64_t q_conv[2];          // read-out: q tile b converted to fp16
+  uint64_t q_full[kQBuf];      // read-out: q tile in buffer b (TMA)
   uint64_t o_full[2];          // read-out: the MMAs into O buffer b are done
   uint64_t o_free[2];          // read-out: the epilogue has read O buffer b
   uint64_t tkt_bar[2];         // chain -> prep groups: next frame's ticket
@@ -104,6 +105,10 @@ struct Layout {
   uint32_t off_slo;   // low image of S_{f-1}
   uint32_t off_sf;    // read-out: S_f image (fp16) over the A blocks of the copy
   uint32_t off_q;     // read-out: two q tiles
+  uint32_t qt;        // tokens per read-out tile: two O^T buffers of qt TMEM columns fit in Y's columns
+  uint32_t qtile;     // bytes of one q tile: [col block][qt t][128 B]
+  uint32_t off_stage; // read-out: o staging, kStageTok rows of d_v fp32 (the bulk store's source)
+  uint32_t stage;     // bytes of the staging area
   uint32_t ny;        // d_k + d_v: TMEM columns of Y
   uint32_t prep_cols; // TMEM columns of one prep group: 32 (W^T pairs) + d_k (M^T, fp32 then pairs)
 };
@@ -115,6 +120,10 @@ __host__ __device__ inline Layout make_layout(int dk, int dv) {
   l.ny = (uint32_t)(dk + dv);
   l.prep_cols = 32u + (uint32_t)dk;
   if (l.ny + 2 * l.prep_cols > 512) return l;                 // TMEM
+  l.qt = (l.ny / 2) / kStageTok * kStageTok;                  // whole bulk stores per tile
+  if (l.qt > (uint32_t)kMaxQT) l.qt = kMaxQT;
+  if (l.qt == 0) return l;
+  l.qtile = 2u * l.qt * 128u;
   l.yb = (uint32_t)dk * 128u;
   l.nyb = (l.ny + 63) / 64;
   l.nab = (uint32_t)(dk + 63) / 64;
@@ -122,7 +131,8 @@ __host__ __device__ inline Layout make_layout(int dk, int dv) {
   if (l.nyb < l.nab + l.nvb) return l;                        // room for the high image after A
   l.s_img = l.nvb * l.yb;
   const uint32_t ycopy = l.nyb * l.yb;
-  const uint32_t ro = l.s_img + 2 * kQTileBytes;               // read-out: S_f image + two q tiles
+  l.stage = (uint32_t)kStageTok * (uint32_t)dv * 4u;
+  const uint32_t ro = l.s_img + kQBuf * l.qtile + l.stage;     // read-out: S_f image, q tiles, staging
   uint32_t fr = l.s_img;
   if (ro > ycopy + fr) fr = ro - ycopy;
   fr = (fr + 1023) / 1024 * 1024;
@@ -137,6 +147,7 @@ __host__ __device__ inline Layout make_layout(int dk, int dv) {
   l.off_slo = l.off_fr;
   l.off_sf = l.off_y;
   l.off_q = l.off_y + l.s_img;
+  l.off_stage = l.off_q + kQBuf * l.qtile;
   l.ok = 1;
   return l;
 }
@@ -193,6 +204,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nkd = dk / 16;            // k-steps over d_k
   const int nvc = dv / 16;            // 16-column chunks of d_v
   const int nch = (L + kC - 1) / kC;  // chunks per frame
+  const int qt = (int)lay.qt;         // tokens per read-out tile
   volatile int *abort_flag = &bar.abort;
 
   // ---------------------------------------------------------------- set-up
@@ -207,11 +219,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bar.chain_done[s], 1);
       mbar_init(&bar.s_full[s], 1);
       mbar_init(&bar.q_full[s], 1);
-      mbar_init(&bar.q_conv[s], 1);
       mbar_init(&bar.o_full[s], 1);
       mbar_init(&bar.o_free[s], 1);
       mbar_init(&bar.tkt_bar[s], 1);
     }
+    mbar_init(&bar.q_full[2], 1);
     mbar_init(&bar.y_mma, 1);
     mbar_init(&bar.fr_bar, 1);
     mbar_init(&bar.drain, 3);
@@ -246,6 +258,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_load_4d(slot + kSlV, &tmap_v, &bar.kv_full[s], 0, t0, f, bh);
     tma_load_4d(slot + kSlV + 8192, &tmap_v, &bar.kv_full[s], 64, t0, f, bh);
     bar.loads = gg + 1;
+    if (c + 2 < nch) {  // two chunks further on towards L2, so that their loads find them there
+      const int t2 = t0 + 2 * kC;
+      tma_prefetch_l2_4d(&tmap_k, 0, t2, f, bh);
+      tma_prefetch_l2_4d(&tmap_k, 64, t2, f, bh);
+      tma_prefetch_l2_4d(&tmap_v, 0, t2, f, bh);
+      tma_prefetch_l2_4d(&tmap_v, 64, t2, f, bh);
+    }
     return true;
   };
   auto issue_frame_kv = [&](int tk, uint32_t g0) -> bool {
@@ -299,10 +318,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t ph = (g / kSlots) & 1u;
         uint8_t *slot = sm + lay.off_slot + s * kSlotBytes;
         // gate of token pt of the chunk (used from the N step on, so its load latency is hidden)
+        // (threads pt and pt + 64 both hold token pt % 64's: one makes N's row, the other, in
+        // group 1, T's column)
         float bt = 0.f;
-        if (pt < kC && c * kC + pt < L) {
+        if (c * kC + (pt & 63) < L) {
           const int f = tk / BH, bh = tk - (tk / BH) * BH;
-          const float braw = p.beta[(long)bh * N + (long)f * L + c * kC + pt];
+          const float braw = p.beta[(long)bh * N + (long)f * L + c * kC + (pt & 63)];
           bt = p.gates_are_logits ? gate_beta(braw) : braw;
         }
         {
@@ -397,37 +418,96 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_before();
         named_bar(pbar, 128);
-        // 4. column pt of (I + N)^-1 by forward substitution (one thread per column, the
-        //    column in registers, each row of N read as a broadcast); then T = (I + N)^-1
-        //    diag(beta): column pt of T is row pt of the K-major B operand of the W product
-        if (pt < kC) {
-          const int cc = pt;
-          float x[64];
+        // 4. (I + N)^-1 = [[Ai, 0], [X, Bi]] from its 32 x 32 blocks: Ai = (I + N_aa)^-1 and
+        //    Bi = (I + N_bb)^-1 by forward substitution (one thread per column, the column in
+        //    registers, each row of N read as a shared-memory broadcast; the two blocks on two
+        //    warps at once), then X = -Bi (N_ba Ai) by two 32 x 32 products on all 128 threads.
+        //    Every block is written over N's own block once no thread reads it.  Then
+        //    T = (I + N)^-1 diag(beta): column t of T is row t of the K-major B operand of the W
+        //    product.  Group 0 substitutes on its warps 0-1, group 1 on its warps 2-3, so the
+        //    two groups' substitutions issue from different SM sub-partitions.
+        const int inv0 = grp ? kC : 0;
+        auto nrow = [&](int r, int col) -> float * {  // address of N[r][col] (col % 4 == 0)
+          return nsm + r * 64 + 4 * ((col >> 2) ^ (r & 7));
+        };
+        if (pt >= inv0 && pt < inv0 + kC) {
+          const int sb = (pt - inv0) >> 5, cc = (pt - inv0) & 31, r0 = 32 * sb;
+          // element (r0 + i, r0 + 4 q) of the block at a constant offset from one base
+          // (r0 is a multiple of 32: (8 sb + q) ^ (i & 7) = 8 sb + (q ^ (i & 7)) for q < 8)
+          const float *blk = nsm + r0 * 64 + 32 * sb;
+          float x[32];
 #pragma unroll
-          for (int r = 0; r < 64; ++r) x[r] = (r == cc) ? 1.f : 0.f;
+          for (int i = 0; i < 32; ++i) x[i] = (i == cc) ? 1.f : 0.f;
 #pragma unroll
-          for (int r = 1; r < 64; ++r) {
-            const float *nr = nsm + r * 64;
+          for (int i = 1; i < 32; ++i) {
             float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
-            for (int q = 0; q < (r + 3) / 4; ++q) {
-              const float4 n4 = *reinterpret_cast<const float4 *>(nr + 4 * (q ^ (r & 7)));
-              if (4 * q + 0 < r) a0 = fmaf(n4.x, x[4 * q + 0], a0);
-              if (4 * q + 1 < r) a1 = fmaf(n4.y, x[4 * q + 1], a1);
-              if (4 * q + 2 < r) a2 = fmaf(n4.z, x[4 * q + 2], a2);
-              if (4 * q + 3 < r) a3 = fmaf(n4.w, x[4 * q + 3], a3);
+            for (int q = 0; q < (i + 3) / 4; ++q) {
+              const float4 n4 = *reinterpret_cast<const float4 *>(blk + i * 64 + 4 * (q ^ (i & 7)));
+              if (4 * q + 0 < i) a0 = fmaf(n4.x, x[4 * q + 0], a0);
+              if (4 * q + 1 < i) a1 = fmaf(n4.y, x[4 * q + 1], a1);
+              if (4 * q + 2 < i) a2 = fmaf(n4.z, x[4 * q + 2], a2);
+              if (4 * q + 3 < i) a3 = fmaf(n4.w, x[4 * q + 3], a3);
             }
-            const float sum = (a0 + a1) + (a2 + a3);
-            x[r] = (r == cc) ? 1.f : -sum;  // rows above the diagonal stay 0: every term is 0 there
+            // rows above the diagonal come out 0: every term there multiplies a 0
+            x[i] = (i == cc) ? 1.f : -((a0 + a1) + (a2 + a3));
           }
-          named_bar(4 + grp, kC);  // every row of N has been read: T may overwrite it
+          __syncwarp();  // the warp's 32 columns are done with N's diagonal block
 #pragma unroll
-          for (int ch = 0; ch < 8; ++ch) {
+          for (int i = 0; i < 32; ++i) nrow(r0 + i, r0 + (cc & ~3))[cc & 3] = x[i];
+        }
+        named_bar(pbar, 128);
+        {
+          // P = N_ba Ai, then X = -Bi P: thread (row i, columns 8 jg .. 8 jg + 7); the thread's
+          // own row is read a float4 at a time, the 8 columns as broadcasts
+          const int i = pt & 31, jg = pt >> 5;
+          auto row_times = [&](int arow_r, int arow_c0, int brow0, float (&acc)[8]) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+#pragma unroll 2
+            for (int kq = 0; kq < 8; ++kq) {
+              const float4 a4 = *reinterpret_cast<const float4 *>(nrow(arow_r, arow_c0 + 4 * kq));
+              const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int kk = 4 * kq + e;
+                const float4 b0 = *reinterpret_cast<const float4 *>(nrow(brow0 + kk, 8 * jg));
+                const float4 b1 = *reinterpret_cast<const float4 *>(nrow(brow0 + kk, 8 * jg + 4));
+                acc[0] = fmaf(av[e], b0.x, acc[0]); acc[1] = fmaf(av[e], b0.y, acc[1]);
+                acc[2] = fmaf(av[e], b0.z, acc[2]); acc[3] = fmaf(av[e], b0.w, acc[3]);
+                acc[4] = fmaf(av[e], b1.x, acc[4]); acc[5] = fmaf(av[e], b1.y, acc[5]);
+                acc[6] = fmaf(av[e], b1.z, acc[6]); acc[7] = fmaf(av[e], b1.w, acc[7]);
+              }
+            }
+          };
+          float acc[8];
+          row_times(32 + i, 0, 0, acc);  // P[i][.] = N_ba[i][.] Ai
+          named_bar(pbar, 128);          // every row of N_ba has been read: P goes over it
+          *reinterpret_cast<float4 *>(nrow(32 + i, 8 * jg)) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+          *reinterpret_cast<float4 *>(nrow(32 + i, 8 * jg + 4)) = make_float4(acc[4], acc[5], acc[6], acc[7]);
+          named_bar(pbar, 128);          // P complete
+          row_times(32 + i, 32, 32, acc);  // (Bi P)[i][.] = Bi[i][.] P
+          named_bar(pbar, 128);          // every row of P has been read: X goes over it
+          *reinterpret_cast<float4 *>(nrow(32 + i, 8 * jg)) = make_float4(-acc[0], -acc[1], -acc[2], -acc[3]);
+          *reinterpret_cast<float4 *>(nrow(32 + i, 8 * jg + 4)) = make_float4(-acc[4], -acc[5], -acc[6], -acc[7]);
+        }
+        named_bar(pbar, 128);
+        {
+          // T: thread (column t, half h of the rows u) reads its half column of (I + N)^-1
+          // (rows 0..31 of columns 32..63 hold N's zeros), then writes it as half of the
+          // K-major row t once every thread has read (T takes N's first 8 KB)
+          const int t = pt & 63, h = pt >> 6;
+          float x[32];
+#pragma unroll
+          for (int u = 0; u < 32; ++u) x[u] = nrow(32 * h + u, t & ~3)[t & 3];
+          named_bar(pbar, 128);
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch) {
             const uint4 u = make_uint4(pack_h2(x[8 * ch + 0] * bt, x[8 * ch + 1] * bt),
                                        pack_h2(x[8 * ch + 2] * bt, x[8 * ch + 3] * bt),
                                        pack_h2(x[8 * ch + 4] * bt, x[8 * ch + 5] * bt),
                                        pack_h2(x[8 * ch + 6] * bt, x[8 * ch + 7] * bt));
-            *reinterpret_cast<uint4 *>(scr + sw128_offset(cc, ch * 8)) = u;
+            *reinterpret_cast<uint4 *>(scr + sw128_offset(t, 32 * h + ch * 8)) = u;
           }
         }
         fence_async_smem();
@@ -520,17 +600,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t id_y = idesc_f16(128, (int)lay.ny, 0, 0, 1);   // M^T (TMEM) x Ycopy (MN-major)
     const uint32_t id_wv = idesc_f16(128, dv, 0, 0, 1);           // W^T (TMEM) x V (MN-major)
     const uint32_t id_s = idesc_f16(128, dv, 0, 0, 1);            // alpha A (K-major) x S image (MN-major)
-    const uint32_t id_o = idesc_f16(128, dv, 0, 0, 1);            // q (K-major) x S_f image (MN-major)
+    const uint32_t id_o = idesc_f16(128, qt, 0, 1, 0);            // S_f image (MN-major) x q (K-major): O^T
     const int h = (nvc + 1) / 2;                                  // S column chunks of warps 0-3
     const int sc0 = right ? h : 0, sc1 = right ? nvc : h;
     float ymax = 0.f;  // largest |value| written as an fp16 operand (range check)
 
-    auto issue_q = [&](int f, int bh, int t0) {  // thread 0: q tile (128 tokens, both column blocks)
-      const int bq = qi & 1;
-      uint8_t *qb = sm + lay.off_q + bq * kQTileBytes;
-      mbar_expect_tx(&bar.q_full[bq], kQTileBytes);
+    auto issue_q = [&](int f, int bh, int t0) {  // thread 0: q tile (qt tokens, both column blocks)
+      const int bq = qi % kQBuf;
+      uint8_t *qb = sm + lay.off_q + bq * lay.qtile;
+      mbar_expect_tx(&bar.q_full[bq], lay.qtile);
       tma_load_4d(qb, &tmap_q, &bar.q_full[bq], 0, t0, f, bh);
-      tma_load_4d(qb + 16384, &tmap_q, &bar.q_full[bq], 64, t0, f, bh);
+      tma_load_4d(qb + lay.qtile / 2, &tmap_q, &bar.q_full[bq], 64, t0, f, bh);
       ++qi;
     };
 
@@ -591,7 +671,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_commit(&bar.slot_free[s]);
           mma_commit(&bar.chain_done[grp]);
           if (c == (nch > 4 ? nch - 4 : 0)) {  // the frame's q tiles towards L2 for the read-out
-            for (int t0 = 0; t0 < L; t0 += kQT) {
+            for (int t0 = 0; t0 < L; t0 += qt) {
               tma_prefetch_l2_4d(&tmap_q, 0, t0, f, bh);
               tma_prefetch_l2_4d(&tmap_q, 64, t0, f, bh);
             }
@@ -788,48 +868,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
 
-      // ---- read-out O_f = Q_f S_f in 128-token tiles (O buffers b at TMEM columns [b d_v, (b+1) d_v))
-      const int nt = (L + kQT - 1) / kQT;
-      if (warp == 0) {
+      // ---- read-out O_f = Q_f S_f in qt-token tiles: O^T = S_f^T Q^T into TMEM buffer n & 1
+      //      (columns [b qt, (b+1) qt)); q tiles come through kQBuf shared-memory buffers
+      const int nt = (L + qt - 1) / qt;
+      if (warp < 4) {
+        // warps 0-3 convert each q tile to fp16 in place (8 16-byte chunks per thread); thread 0
+        // also issues the q loads (kQBuf ahead) and each tile's MMAs
         if (tid == 0) {
           tc_fence_after();
-          issue_q(f, bh, 0);
-          if (nt > 1) issue_q(f, bh, kQT);
-          int bad = 0;
-          for (int n = 0; n < nt && !bad; ++n) {
-            const uint32_t gt = rt + n, b = gt & 1u, ph = (gt >> 1) & 1u;
-            if (!mbar_wait(&bar.q_conv[b], ph, lim)) bad = 1;
-            if (!bad && gt >= 2 && !mbar_wait(&bar.o_free[b], ph ^ 1u, lim)) bad = 1;  // tile n - 2 has left buffer b
-            if (bad) break;
-            tc_fence_after();
-            const uint32_t q0 = smem_u32(sm + lay.off_q + b * kQTileBytes), sf = smem_u32(sm + lay.off_sf);
-            for (int kk = 0; kk < nkd; ++kk)
-              mma_f16_ss(tmem + b * dv, sdesc_sw128(q0 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                         sdesc_sw128(sf + kk * 2048, lay.yb, 1024), id_o, kk > 0 ? 1u : 0u);
-            mma_commit(&bar.o_full[b]);
-            // tile n - 1's MMAs done: its q buffer takes tile n + 1
-            if (n >= 1 && n + 1 < nt) {
-              const uint32_t gp = gt - 1;
-              if (!mbar_wait(&bar.o_full[gp & 1u], (gp >> 1) & 1u, lim)) {
-                bad = 1;
-                break;
-              }
-              issue_q(f, bh, (n + 1) * kQT);
-            }
-          }
-          if (bad) {
-            *abort_flag = 1;
-            latch_status(p.status, GDN_ERR_TIMEOUT);
-          }
+          for (int n = 0; n < nt && n < kQBuf; ++n) issue_q(f, bh, n * qt);
         }
-      } else if (warp < 4) {
-        // q tiles bf16 -> fp16 in place (96 threads)
-        const int ct = tid - 32;
         for (int n = 0; n < nt; ++n) {
-          const uint32_t gt = rt + n, b = gt & 1u, ph = (gt >> 1) & 1u;
+          const uint32_t gt = rt + n, qb = gt % kQBuf, qph = (gt / kQBuf) & 1u;
+          const uint32_t b = gt & 1u, ph = (gt >> 1) & 1u;
           {
-            const int bad = ct == 0 ? !mbar_wait(&bar.q_full[b], ph, lim) : 0;
-            if (bar_sync_or(6, 96, bad || *abort_flag)) {
+            const int bad = tid == 0 ? !mbar_wait(&bar.q_full[qb], qph, lim) : 0;
+            if (bar_sync_or(6, 128, bad || *abort_flag)) {
               if (bad) {
                 *abort_flag = 1;
                 latch_status(p.status, GDN_ERR_TIMEOUT);
@@ -837,58 +891,97 @@ __global__ void __launch_bounds__(kThreads, 1)
               break;
             }
           }
-          if (ct == 0) bar.q_used = gt + 1;
-          uint4 *qb = reinterpret_cast<uint4 *>(sm + lay.off_q + b * kQTileBytes);
+          if (tid == 0) bar.q_used = gt + 1;
+          uint4 *qv = reinterpret_cast<uint4 *>(sm + lay.off_q + qb * lay.qtile);
           float qmax = 0.f;
-#pragma unroll 4
-          for (int i = ct; i < (int)(kQTileBytes / 16); i += 96) qb[i] = bf16x8_to_f16x8(qb[i], qmax);
+          const int nq16 = (int)(lay.qtile / 16);
+#pragma unroll 2
+          for (int i0 = 0; i0 < nq16; i0 += 4 * 128) {
+            uint4 u[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              if (i0 + e * 128 + tid < nq16) u[e] = qv[i0 + e * 128 + tid];
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              if (i0 + e * 128 + tid < nq16) qv[i0 + e * 128 + tid] = bf16x8_to_f16x8(u[e], qmax);
+          }
           if (out_of_f16_range(qmax)) latch_status(p.status, GDN_ERR_RANGE);
           fence_async_smem();
-          named_bar(6, 96);
-          if (ct == 0) mbar_arrive_only(&bar.q_conv[b]);
+          named_bar(6, 128);
+          if (tid == 0) {
+            int bad = gt >= 2 && !mbar_wait(&bar.o_free[b], ph ^ 1u, lim);  // tile n - 2 has left buffer b
+            if (!bad) {
+              tc_fence_after();
+              const uint32_t q0 = smem_u32(sm + lay.off_q + qb * lay.qtile), sf = smem_u32(sm + lay.off_sf);
+              for (int kk = 0; kk < nkd; ++kk)
+                mma_f16_ss(tmem + b * qt, sdesc_sw128(sf + kk * 2048, lay.yb, 1024),
+                           sdesc_sw128(q0 + (kk >> 2) * (lay.qtile / 2) + (kk & 3) * 32, 16, 1024), id_o,
+                           kk > 0 ? 1u : 0u);
+              mma_commit(&bar.o_full[b]);
+              // tile n - 1's MMAs done: its q buffer takes tile n - 1 + kQBuf
+              if (n >= 1 && n - 1 + kQBuf < nt) {
+                const uint32_t gp = gt - 1;
+                bad = !mbar_wait(&bar.o_full[gp & 1u], (gp >> 1) & 1u, lim);
+                if (!bad) issue_q(f, bh, (n - 1 + kQBuf) * qt);
+              }
+            }
+            if (bad) {
+              *abort_flag = 1;
+              latch_status(p.status, GDN_ERR_TIMEOUT);
+            }
+          }
         }
       } else {
-        // epilogue: O rows (lane = token of the tile) straight from TMEM to o
+        // epilogue: O^T (lane = column j of o, TMEM columns = tokens of the tile) through the
+        // staging rows into o's row-major layout (for each token the 32 lanes of a warp write
+        // 32 consecutive floats), kStageTok tokens per bulk store of contiguous rows
         const int et = tid - 128;
+        float *stg = reinterpret_cast<float *>(sm + lay.off_stage);
         for (int n = 0; n < nt; ++n) {
           const uint32_t gt = rt + n, b = gt & 1u, ph = (gt >> 1) & 1u;
-          {
-            const int bad = et == 0 ? !mbar_wait(&bar.o_full[b], ph, lim) : 0;
-            if (bar_sync_or(7, 128, bad || *abort_flag)) {
-              if (bad) {
-                *abort_flag = 1;
-                latch_status(p.status, GDN_ERR_TIMEOUT);
-              }
-              break;
-            }
-          }
-          tc_fence_after();
-          const int t = n * kQT + row;
-          float *orow = p.o + ((long)bh * N + (long)f * L + t) * dv;
-#pragma unroll 1
-          for (int cb = 0; cb < nvc; cb += 2) {
-            const bool two = cb + 1 < nvc;
-            float r[2][16];
-            tmem_ld16(tmem + lane_off + b * dv + cb * 16, r[0]);
-            if (two) tmem_ld16(tmem + lane_off + b * dv + cb * 16 + 16, r[1]);
-            tmem_ld_wait();
-            if (t < L) {
-#pragma unroll
-              for (int e = 0; e < 2; ++e) {
-                if (e == 1 && !two) break;
-#pragma unroll
-                for (int z = 0; z < 16; z += 4)
-                  *reinterpret_cast<float4 *>(orow + (cb + e) * 16 + z) =
-                      make_float4(r[e][z], r[e][z + 1], r[e][z + 2], r[e][z + 3]);
+          bool stop_ro = false;
+          for (int hh = 0; hh < qt / kStageTok && !stop_ro; ++hh) {
+            {
+              int bad = (et == 0 && hh == 0) ? !mbar_wait(&bar.o_full[b], ph, lim) : 0;
+              if (et == 0) bulk_wait_read();  // the previous bulk store has read the staging rows
+              if (bar_sync_or(7, 128, bad || *abort_flag)) {
+                if (bad) {
+                  *abort_flag = 1;
+                  latch_status(p.status, GDN_ERR_TIMEOUT);
+                }
+                stop_ro = true;
+                break;
               }
             }
+            tc_fence_after();
+#pragma unroll
+            for (int cb = 0; cb < kStageTok / 16; ++cb) {
+              float r[16];
+              tmem_ld16(tmem + lane_off + b * qt + hh * kStageTok + cb * 16, r);
+              tmem_ld_wait();
+              if (row < dv) {
+#pragma unroll
+                for (int z = 0; z < 16; ++z) stg[(cb * 16 + z) * dv + row] = r[z];
+              }
+            }
+            tc_fence_before();
+            fence_async_smem();
+            named_bar(7, 128);
+            if (et == 0) {
+              if (hh + 1 == qt / kStageTok) mbar_arrive_only(&bar.o_free[b]);
+              const int t0 = n * qt + hh * kStageTok;
+              const int nv = L - t0 < kStageTok ? L - t0 : kStageTok;  // tokens inside the frame
+              if (nv > 0) {
+                bulk_store(p.o + ((long)bh * N + (long)f * L + t0) * dv, stg, (uint32_t)(nv * dv * 4));
+                bulk_commit();
+              }
+            }
           }
-          tc_fence_before();
-          named_bar(7, 128);
-          if (et == 0) mbar_arrive_only(&bar.o_free[b]);
+          if (stop_ro) break;
         }
       }
       rt += (uint32_t)nt;
+      if (tid == 128) bulk_wait_read();  // the next frame's Y copy overwrites the staging rows
       if (bar_sync_or(1, kChain, *abort_flag)) {
         failed = true;
         break;
@@ -898,6 +991,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (tid == 0) latch_status(p.status, GDN_ERR_TIMEOUT);  // the first code latched wins
       *abort_flag = 1;
     }
+    if (tid == 128) bulk_wait_all();  // o rows written before the CTA exits
     named_bar(1, kChain);
     if (tid == 0) {
       // loads still in flight complete before the CTA exits: the last k, v load of each
@@ -905,7 +999,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t n = bar.loads;
       for (uint32_t gg = n > (uint32_t)kSlots ? n - kSlots : 0u; gg < n; ++gg)
         mbar_wait(&bar.kv_full[gg % kSlots], (gg / kSlots) & 1u, lim);
-      for (uint32_t gq = bar.q_used; gq < qi; ++gq) mbar_wait(&bar.q_full[gq & 1u], (gq >> 1) & 1u, lim);
+      for (uint32_t gq = bar.q_used; gq < qi; ++gq) mbar_wait(&bar.q_full[gq % kQBuf], (gq / kQBuf) & 1u, lim);
       if (s_pending) {
         mbar_wait(&bar.s_full[0], sph, lim);
         mbar_wait(&bar.s_full[1], sph, lim);
@@ -937,7 +1031,7 @@ cudaError_t launch_gdn_pform(const GdnParams &p, int grid, cudaStream_t st) {
   if (!lay.ok) return cudaErrorInvalidValue;
   CUtensorMap mq, mk, mv;
   const int BH = p.B * p.H;
-  if (!tc::make_bf16_map(&mq, p.q, p.dk, p.L, p.F, BH, kQT) || !tc::make_bf16_map(&mk, p.k, p.dk, p.L, p.F, BH, 64) ||
+  if (!tc::make_bf16_map(&mq, p.q, p.dk, p.L, p.F, BH, (int)lay.qt) || !tc::make_bf16_map(&mk, p.k, p.dk, p.L, p.F, BH, 64) ||
       !tc::make_bf16_map(&mv, p.v, p.dv, p.L, p.F, BH, 64))
     return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(gdn_pform_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lay.smem);

@@ -83,9 +83,10 @@ def test_workspace_sizes(lib):
 
 def test_workspace_sizes_with_segments(lib):
     """The tcgen05 path sizes its scratch for any launch the sizes may lead to:
-    with P chunk segments (residual-form kernel) fp16 states and flags per
-    segment unit plus one bf16 high/low end state per frame; with one segment
-    per frame (product-form kernel) fp16 high and low state images per frame."""
+    with P chunk segments (residual-form kernel, the default) fp16 states and
+    flags per segment unit plus one bf16 high/low end state per frame; the
+    product-form kernel (one segment per frame) fp16 high and low state images
+    per frame."""
     d = 112
 
     def need(B, H, F, L, impl="tc", **kw):
@@ -101,14 +102,14 @@ def test_workspace_sizes_with_segments(lib):
         return 256 + up(4 * units) + up(units * 2 * (2 * d * 128))
 
     nch = (920 + 63) // 64
-    assert need(1, 20, 1, 920) == max(residual(20, min(nch, 8)), pform(20))   # a streaming call: auto bound
-    assert need(1, 20, 1, 920, segments=1) == pform(20)
-    assert need(1, 20, 1, 920, segments=1, impl="tc_residual") == residual(20, 1)
-    assert need(1, 20, 1, 920, segments=3) == max(residual(20, 3), pform(20))
-    assert need(1, 20, 1, 920, segments=99) == max(residual(20, nch), pform(20))  # at most one chunk each
-    assert need(1, 20, 240, 920) == pform(4800)                                # many frames: one segment
-    assert need(1, 20, 240, 920, impl="tc_residual") == residual(4800, 1)
-    assert need(1, 20, 1, 64) == pform(20)                                     # one chunk per frame
+    assert need(1, 20, 1, 920) == residual(20, min(nch, 8))                   # a streaming call: auto bound
+    assert need(1, 20, 1, 920, segments=1) == residual(20, 1)
+    assert need(1, 20, 1, 920, segments=3) == residual(20, 3)
+    assert need(1, 20, 1, 920, segments=99) == residual(20, nch)              # at most one chunk each
+    assert need(1, 20, 240, 920) == residual(4800, 1)                         # many frames: one segment
+    assert need(1, 20, 1, 64) == residual(20, 1)                              # one chunk per frame
+    assert need(1, 20, 240, 920, impl="tc_pform") == pform(4800)              # product form: one segment
+    assert need(1, 20, 1, 920, impl="tc_pform") == pform(20)
     simt = lib.make_opts(lib.DTYPE_BF16, impl="frame_simt", stream=0, segments=4)
     assert lib.workspace_bytes(lib.OP_GDN, 1, 20, 1, 920, d, d, simt) == 256 + 256 + 20 * d * d * 4
 

@@ -36,10 +36,21 @@ def run_gdn(lib, w, t, dev, impl, state_in=None, want_state=True, **kw):
     return o.cpu().numpy(), (None if s_out is None else s_out.cpu().numpy())
 
 
+def pform_ok(dk, dv):
+    """Sizes the product-form tensor-core kernel takes (its shared-memory and TMEM maps fit)."""
+    ny = dk + dv
+    if dk % 16 or dv % 16 or dv > dk or dk > 128 or ny + 2 * (32 + dk) > 512 or (ny // 2) // 32 == 0:
+        return False
+    nyb, nab, nvb = (ny + 63) // 64, (dk + 63) // 64, (dv + 63) // 64
+    return nyb >= nab + nvb
+
+
 def impls_for(w):
     out = ["seq", "frame_simt"]
     if w.dtype == "bf16" and w.dk % 16 == 0 and w.dv % 16 == 0:
         out.append("tc")
+        if pform_ok(w.dk, w.dv):
+            out.append("tc_pform")
     return out
 
 
@@ -56,7 +67,7 @@ def test_tiny_fp32(lib, dev, impl):
     assert rel_err(s, s_ref) <= 1e-5
 
 
-@pytest.mark.parametrize("impl", ["frame_simt", "tc"])
+@pytest.mark.parametrize("impl", ["frame_simt", "tc", "tc_pform"])
 def test_480p_5s(lib, dev, impl):
     w = W["gdn_480p_5s"]
     x = synth.inputs(w)
@@ -68,7 +79,7 @@ def test_480p_5s(lib, dev, impl):
     assert eo <= 2e-3 and es <= 2e-3
 
 
-@pytest.mark.parametrize("impl", ["frame_simt", "tc"])
+@pytest.mark.parametrize("impl", ["frame_simt", "tc", "tc_pform"])
 def test_720p_60s_full(lib, dev, impl):
     """Full 720p-60s workload in the benchmark's launch configuration, every
     head and every d_v column (including columns 64-111, which come from the
@@ -98,7 +109,7 @@ def test_alpha_one_long_sequence_drift(lib, dev):
     h1["a"] = np.ones_like(h["a"])
     h1["b"] = beta.cpu().numpy()
     o_ref, s_ref = oracle.gdn(h1["q"], h1["k"], h1["v"], h1["a"], h1["b"], F=w.F, L=w.L, gates_are_logits=False)
-    for impl in ("tc", "frame_simt"):
+    for impl in ("tc", "tc_pform", "frame_simt"):
         s_out = torch.empty((w.B, w.H, w.dk, w.dv), dtype=torch.float32, device=dev)
         o = lib.gdn_frame_fwd(t["q"], t["k"], t["v"], ones, beta, F=w.F, gates_are_logits=False,
                               state_out=s_out, impl=impl)
