@@ -208,7 +208,7 @@ GDN_API int gdn_frame_fwd_host(const void *q, const void *k, const void *v, cons
  * Each call clears the part of the array that must start at zero before its
  * kernel runs.  The call allocates no memory.
  */
-#define GDN_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+#define GDN_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
 GDN_API int gdn_frame_fwd_noalloc(const void *q, const void *k, const void *v, const float *alpha,
                                   const float *beta, const float *state_in, float *state_out, float *o, int B,
                                   int H, int F, int L, int dk, int dv, const gdn_opts_t *opts);

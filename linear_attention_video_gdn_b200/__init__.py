@@ -33,7 +33,7 @@ IMPLS = {"auto": IMPL_AUTO, "seq": IMPL_SEQ, "frame_simt": IMPL_FRAME_SIMT, "tc"
 EXPORTED = ("gdn_frame_fwd", "relu_la_block_fwd", "gdn_frame_fwd_host", "gdn_frame_fwd_noalloc",
             "gdn_workspace_bytes", "gdn_workspace_bytes_host", "gdn_status_string", "gdn_status_str",
             "gdn_abi_version")
-NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
+NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
 
 
 class GdnOpts(ctypes.Structure):

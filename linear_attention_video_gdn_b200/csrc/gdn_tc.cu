@@ -122,17 +122,21 @@ __device__ __forceinline__ void store_row16_f16(uint8_t *tile, uint32_t row, uin
   *reinterpret_cast<uint4 *>(tile + sw128_offset(row, col0 + 8)) = b;
 }
 
-// bf16 x 8 -> fp16 x 8 (one 16-byte chunk)
-__device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 u) {
+// bf16 x 8 -> fp16 x 8 (one 16-byte chunk); amax takes the largest |value|
+__device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 u, float &amax) {
   const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
   uint32_t o[4];
 #pragma unroll
   for (int e = 0; e < 4; ++e) {
     const float2 v2 = __bfloat1622float2(h[e]);
+    amax = fmaxf(amax, fmaxf(fabsf(v2.x), fabsf(v2.y)));
     o[e] = pack_h2(v2.x, v2.y);
   }
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
+
+// Largest finite fp16 value: an operand at or beyond it (or NaN) leaves the fp16 range.
+constexpr float kF16Max = 65504.0f;
 
 // ---------------------------------------------------------------- blocked inversion
 // The 64 x 64 unit lower triangular I + N is handled as 4 x 4 blocks of 16 x 16.
@@ -392,11 +396,13 @@ __global__ void __launch_bounds__(kGThreads, 1)
           const int t = pt >> 1, kb = pt & 1;
           uint8_t *vrow = slot + SL_V + kb * 8192;
           uint4 vu[8];
+          float vmax = 0.f;
 #pragma unroll
           for (int ch = 0; ch < 8; ++ch) vu[ch] = *reinterpret_cast<const uint4 *>(vrow + sw128_offset(t, ch * 8));
 #pragma unroll
           for (int ch = 0; ch < 8; ++ch)
-            *reinterpret_cast<uint4 *>(vrow + sw128_offset(t, ch * 8)) = bf16x8_to_f16x8(vu[ch]);
+            *reinterpret_cast<uint4 *>(vrow + sw128_offset(t, ch * 8)) = bf16x8_to_f16x8(vu[ch], vmax);
+          if (!(vmax < kF16Max)) latch_status(p.status, GDN_ERR_RANGE);
         }
         {
           const int bad = pt == 0 ? !mbar_wait(&bar.g_bar[grp], gph, lim) : 0;
@@ -795,42 +801,53 @@ __global__ void __launch_bounds__(kGThreads, 1)
       const int l0 = tile * 64;                                        // this thread's half of the d_k columns
       const int nl = dk - l0 < 64 ? (dk - l0 > 0 ? dk - l0 : 0) : 64;  // columns in it (a multiple of 16)
       if (have_prev) {
-        // S_{f-1}^T row j as fp16 pairs into TMEM columns [256, 256 + d_k / 2) (A operand)
+        // S_{f-1}^T row j as fp16 pairs into TMEM columns [256, 256 + d_k / 2) (the A operand
+        // of the chain product); the caller's fp32 state_in also as the fp16 low parts of its
+        // values into [320, 320 + d_k / 2), for a second product
         if (nl > 0) {
           if (chained) {
             // published rows S^T[j][l] (fp16, d_k per row): the pairs are the loaded words
-            const uint4 *src = reinterpret_cast<const uint4 *>(
-                reinterpret_cast<const __half *>(p.ws.states) + (uidx - 1) * (long)dk * dv + (long)j * dk + l0);
-            uint4 u[8];
+            const __half *base = reinterpret_cast<const __half *>(p.ws.states) + (uidx - 1) * (long)dk * dv;
+            {
+              const uint4 *src = reinterpret_cast<const uint4 *>(base + (long)j * dk + l0);
+              uint4 u[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e)
-              u[e] = (j < dv && 8 * e < nl) ? __ldcg(src + e) : make_uint4(0u, 0u, 0u, 0u);
+              for (int e = 0; e < 8; ++e)
+                u[e] = (j < dv && 8 * e < nl) ? __ldcg(src + e) : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
-              if (32 * h2 < nl) {
-                const uint32_t w[16] = {u[4 * h2].x,     u[4 * h2].y,     u[4 * h2].z,     u[4 * h2].w,
-                                        u[4 * h2 + 1].x, u[4 * h2 + 1].y, u[4 * h2 + 1].z, u[4 * h2 + 1].w,
-                                        u[4 * h2 + 2].x, u[4 * h2 + 2].y, u[4 * h2 + 2].z, u[4 * h2 + 2].w,
-                                        u[4 * h2 + 3].x, u[4 * h2 + 3].y, u[4 * h2 + 3].z, u[4 * h2 + 3].w};
-                tmem_st16u(tmem + TM_R + lane_off + (l0 + 32 * h2) / 2, w);
+              for (int h2 = 0; h2 < 2; ++h2) {
+                if (32 * h2 < nl) {
+                  const uint32_t w[16] = {u[4 * h2].x,     u[4 * h2].y,     u[4 * h2].z,     u[4 * h2].w,
+                                          u[4 * h2 + 1].x, u[4 * h2 + 1].y, u[4 * h2 + 1].z, u[4 * h2 + 1].w,
+                                          u[4 * h2 + 2].x, u[4 * h2 + 2].y, u[4 * h2 + 2].z, u[4 * h2 + 2].w,
+                                          u[4 * h2 + 3].x, u[4 * h2 + 3].y, u[4 * h2 + 3].z, u[4 * h2 + 3].w};
+                  tmem_st16u(tmem + TM_R + lane_off + (l0 + 32 * h2) / 2, w);
+                }
               }
             }
           } else {
-            // the caller's fp32 state S[l][j] (d_v contiguous: lanes j read consecutive addresses)
+            // the caller's fp32 state S[l][j] (d_v contiguous: lanes j read consecutive addresses),
+            // split into fp16 high and low parts
             const float *prev = p.state_in + (long)bh * dk * dv;
+            float smax = 0.f;
 #pragma unroll 1
             for (int h2 = 0; h2 < 2; ++h2) {
               if (32 * h2 >= nl) break;
-              uint32_t w[16];
+              uint32_t wh[16], wl[16];
 #pragma unroll
               for (int e = 0; e < 16; ++e) {
                 const int l = l0 + 32 * h2 + 2 * e;
                 const float v0 = (j < dv && l < dk) ? __ldcg(prev + (long)l * dv + j) : 0.f;
                 const float v1 = (j < dv && l + 1 < dk) ? __ldcg(prev + (long)(l + 1) * dv + j) : 0.f;
-                w[e] = pack_h2(v0, v1);
+                smax = fmaxf(smax, fmaxf(fabsf(v0), fabsf(v1)));
+                const float h0 = __half2float(__float2half_rn(v0)), h1 = __half2float(__float2half_rn(v1));
+                wh[e] = pack_h2(h0, h1);
+                wl[e] = pack_h2(v0 - h0, v1 - h1);
               }
-              tmem_st16u(tmem + TM_R + lane_off + (l0 + 32 * h2) / 2, w);
+              tmem_st16u(tmem + TM_R + lane_off + (l0 + 32 * h2) / 2, wh);
+              tmem_st16u(tmem + TM_R + 64 + lane_off + (l0 + 32 * h2) / 2, wl);
             }
+            if (!(smax < kF16Max)) latch_status(p.status, GDN_ERR_RANGE);
           }
         }
         tmem_st_wait();
@@ -839,8 +856,10 @@ __global__ void __launch_bounds__(kGThreads, 1)
         if (tid == 0) {
           tc_fence_after();
           const uint32_t ab = smem_u32(sm + OFF_MIRROR);  // tile A of the mirror = alpha A_f^T rows, read MN-major
-          for (int kk = 0; kk < nkd; ++kk)
-            mma_f16_ts(tmem + TM_Y + 128, tmem + TM_R + kk * 8, sdesc_sw128(ab + kk * 2048, 16384, 1024), id_s, 1u);
+          for (int part = 0; part < (chained ? 1 : 2); ++part)  // state_in: high + low parts
+            for (int kk = 0; kk < nkd; ++kk)
+              mma_f16_ts(tmem + TM_Y + 128, tmem + TM_R + 64 * part + kk * 8, sdesc_sw128(ab + kk * 2048, 16384, 1024),
+                         id_s, 1u);
           mma_commit(&bar.fr_bar);
         }
         const bool ok = group_wait(&bar.fr_bar, fphase);
@@ -861,6 +880,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
       {
         float *sout = (f == F - 1 && last_seg && p.state_out) ? p.state_out + (long)bh * dk * dv : nullptr;
         __half *srow = reinterpret_cast<__half *>(sm + OFF_STAGE) + (long)j * dk + l0;
+        float smax = 0.f;
 #pragma unroll 1
         for (int h2 = 0; h2 < 4; ++h2) {  // 16 columns l at a time
           if (16 * h2 >= nl) break;
@@ -871,7 +891,10 @@ __global__ void __launch_bounds__(kGThreads, 1)
           if (j < dv) {
             uint32_t hf[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) hf[e] = pack_h2(r[2 * e], r[2 * e + 1]);
+            for (int e = 0; e < 8; ++e) {
+              smax = fmaxf(smax, fmaxf(fabsf(r[2 * e]), fabsf(r[2 * e + 1])));
+              hf[e] = pack_h2(r[2 * e], r[2 * e + 1]);
+            }
             *reinterpret_cast<uint4 *>(srow + 16 * h2) = make_uint4(hf[0], hf[1], hf[2], hf[3]);
             *reinterpret_cast<uint4 *>(srow + 16 * h2 + 8) = make_uint4(hf[4], hf[5], hf[6], hf[7]);
             if (sout) {
@@ -880,6 +903,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
             }
           }
         }
+        if (!(smax < kF16Max)) latch_status(p.status, GDN_ERR_RANGE);
       }
       fence_async_smem();
       named_bar(1, kChain);

@@ -222,6 +222,53 @@ def test_zero_keys_and_large_values(lib, dev):
         assert rel_err(s, s_ref) <= 2e-3, impl
 
 
+def test_alpha_one_720p_60s(lib, dev):
+    """The 720p-60s workload with no forgetting (alpha = 1 as values) and beta =
+    sigmoid of the workload's logits: 240 frames of 920 tokens chained through
+    the tensor-core kernels' fp16 frame hand-off, every head and column against
+    the oracle."""
+    w = W["gdn_720p_60s"]
+    x = synth.inputs(w)
+    t, h = device_inputs(w, x, dev, torch)
+    ones = torch.ones_like(t["a"])
+    beta = torch.sigmoid(t["b"])
+    o_ref, s_ref = oracle.gdn(h["q"], h["k"], h["v"], np.ones_like(h["a"]), beta.cpu().numpy(), F=w.F, L=w.L,
+                              gates_are_logits=False)
+    for impl in ("tc", "tc_pform"):
+        s_out = torch.empty((w.B, w.H, w.dk, w.dv), dtype=torch.float32, device=dev)
+        o = lib.gdn_frame_fwd(t["q"], t["k"], t["v"], ones, beta, F=w.F, gates_are_logits=False,
+                              state_out=s_out, impl=impl)
+        torch.cuda.synchronize()
+        eo, es = rel_err(o.cpu().numpy(), o_ref), rel_err(s_out.cpu().numpy(), s_ref)
+        print(f"720p alpha=1 {impl}: err_o={eo:.3e} err_s={es:.3e}")
+        assert eo <= 2e-3 and es <= 2e-3, impl
+
+
+def test_fp16_range_is_reported(lib, dev):
+    """Values the fp16 tensor-core operands cannot hold (|v| or |state_in| >= 65504) end
+    with GDN_ERR_RANGE in *status instead of passing silently; in-range inputs do not."""
+    w = W["gdn_480p_5s"].with_(F=2, L=80, H=2)
+    x = synth.inputs(w)
+    x["v"][0, 1, 17] *= 1e5
+    t, h = device_inputs(w, x, dev, torch)
+    for impl in ("tc", "tc_pform"):
+        status = torch.zeros(4, dtype=torch.int32, device=dev)
+        run_gdn(lib, w, t, dev, impl, status=status)
+        assert int(status[0].item()) == lib.ERR_RANGE, impl
+    w2 = w.with_(seed=5)
+    x2 = synth.inputs(w2)
+    t2, _ = device_inputs(w2, x2, dev, torch)
+    big = np.zeros((w.B, w.H, w.dk, w.dv), np.float32)
+    big[0, 0, 3, 4] = 1e5
+    for impl in ("tc", "tc_pform"):
+        status = torch.zeros(4, dtype=torch.int32, device=dev)
+        run_gdn(lib, w2, t2, dev, impl, state_in=big, status=status)
+        assert int(status[0].item()) == lib.ERR_RANGE, impl
+        status.zero_()
+        run_gdn(lib, w2, t2, dev, impl, status=status)
+        assert int(status[0].item()) == 0, impl
+
+
 def test_few_ctas_many_frames(lib, dev):
     """A persistent grid far smaller than the frame count still completes the chain."""
     w = W["gdn_480p_5s"].with_(F=30, L=33, H=3)
