@@ -42,7 +42,9 @@ def _load():
         P = ctypes.c_void_p
         I64 = ctypes.c_int64
         lib.oracle_gdn.argtypes = [P, P, P, P, P, ctypes.c_int, P, P, P, I64, I64, I64, I64, I64, I64,
-                                   I64, I64, P, I64, I64, ctypes.c_int]
+                                   I64, I64, P, I64, I64, ctypes.c_int, I64, I64, ctypes.c_double]
+        lib.oracle_rope3d.argtypes = [P, P, I64, I64, I64, I64, I64, I64, ctypes.c_double]
+        lib.oracle_rope3d.restype = ctypes.c_int
         lib.oracle_gdn.restype = ctypes.c_int
         lib.oracle_relu_la.argtypes = [P, P, P, P, P, P, P, P, I64, I64, I64, I64, I64, I64, ctypes.c_double,
                                        ctypes.c_int]
@@ -78,14 +80,16 @@ def gate_beta(b: float) -> float:
 
 
 def gdn(q, k, v, alpha, beta, *, F: int, L: int, gates_are_logits: bool = True, state_in=None,
-        cols=None, heads=None, want_o: bool = True, nthreads: int | None = None):
+        cols=None, heads=None, want_o: bool = True, nthreads: int | None = None, rope=None):
     """Gated DeltaNet frame recurrence in fp64.
 
     q, k: [..., F*L, dk]; v: [..., F*L, dv]; alpha: [..., F]; beta: [..., F*L];
     leading dims are flattened into heads.  state_in: [..., dk, dv] or None.
     cols: (lo, hi) range of d_v columns to compute (others left as NaN).
     heads: optional subset of flat head indices (outputs still full-sized,
-    other heads NaN).  Returns (o, state_out) as float64 arrays.
+    other heads NaN).  rope: None, or dict(grid_w, frame_offset=0, base=1e4)
+    to apply the 3D RoPE (see ``rope3d``) to q and to k before its
+    normalisation.  Returns (o, state_out) as float64 arrays.
     """
     q, k, v, alpha, beta = map(_f32, (q, k, v, alpha, beta))
     lead = q.shape[:-2]
@@ -103,12 +107,38 @@ def gdn(q, k, v, alpha, beta, *, F: int, L: int, gates_are_logits: bool = True, 
     hl = None if heads is None else np.ascontiguousarray(np.asarray(heads, dtype=np.int64))
     nthreads = nthreads or (os.cpu_count() or 1)
     col_block = max(1, min(hi - lo, 16)) if hi > lo else 1
+    rp = _rope_args(rope)
     rc = _load().oracle_gdn(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), int(gates_are_logits),
                             _ptr(s_in), _ptr(s_out), _ptr(o), 1, nh, F, L, dk, dv, lo, hi,
-                            _ptr(hl), 0 if hl is None else hl.size, col_block, nthreads)
+                            _ptr(hl), 0 if hl is None else hl.size, col_block, nthreads, *rp)
     if rc != 0:
         raise ValueError("oracle_gdn: invalid arguments")
     return o, s_out
+
+
+def _rope_args(rope):
+    if rope is None:
+        return (0, 0, 1e4)
+    return (int(rope["grid_w"]), int(rope.get("frame_offset", 0)), float(rope.get("base", 1e4)))
+
+
+def rope3d(x, *, F: int, L: int, grid_w: int, frame_offset: int = 0, base: float = 1e4):
+    """The 3D rotary position embedding alone, in fp64: x [..., F*L, d] -> rotated x.
+
+    The d dimensions are a time part (d - 4*floor(d/6)), then a height and a
+    width part (2*floor(d/6) each); in each part the pair (2i, 2i+1) turns by
+    pos * base**(-2i / part_length), pos being the token's frame (plus
+    frame_offset), row (t // grid_w) or column (t % grid_w)."""
+    x = _f32(x)
+    lead = x.shape[:-2]
+    N, d = x.shape[-2:]
+    assert N == F * L
+    nh = int(np.prod(lead)) if lead else 1
+    out = np.empty(x.shape, np.float64)
+    rc = _load().oracle_rope3d(_ptr(x), _ptr(out), nh, F, L, d, grid_w, frame_offset, float(base))
+    if rc != 0:
+        raise ValueError("oracle_rope3d: invalid arguments")
+    return out
 
 
 def relu_la(q, k, v, *, F: int, L: int, kv_in=None, z_in=None, eps: float = 1e-6, nthreads: int | None = None):

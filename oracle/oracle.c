@@ -64,6 +64,53 @@ static double gate_beta(double b) { return 1.0 / (1.0 + exp(-b)); }
 double oracle_gate_alpha(double a) { return gate_alpha(a); }
 double oracle_gate_beta(double b) { return gate_beta(b); }
 
+/*
+ * 3D rotary position embedding (SANA-Video talk, "3D RoPE for the linear
+ * attention"; the talk gives no formula, this is the library's reading): a
+ * d-vector at latent position (frame, row, column) is split into a time part
+ * of dt dimensions, then a height and a width part of dh = dw = 2 * floor(d / 6)
+ * each (dt = d - dh - dw); in each part the pair (2i, 2i + 1) is rotated by
+ * the angle pos * base^(-2i / part_length), pos being that part's coordinate.
+ * The token at index t of a frame of a grid_w-wide latent grid sits at row
+ * t / grid_w and column t % grid_w.
+ */
+typedef struct {
+  int on;
+  int64_t grid_w;       /* latent grid width (tokens per row) */
+  int64_t frame_offset; /* time coordinate of the first frame */
+  double base;
+} rope_t;
+
+static void rope3d(const float *x, int64_t d, int64_t frame, int64_t row, int64_t col, double base, double *out) {
+  const int64_t dh = 2 * (d / 6), dw = dh, dt = d - dh - dw;
+  const int64_t len[3] = {dt, dh, dw}, pos[3] = {frame, row, col};
+  int64_t o = 0;
+  for (int a = 0; a < 3; ++a) {
+    for (int64_t i = 0; i < len[a] / 2; ++i) {
+      const double theta = pow(base, -2.0 * (double)i / (double)len[a]);
+      const double phi = (double)pos[a] * theta;
+      const double c = cos(phi), sn = sin(phi);
+      const double x0 = (double)x[o + 2 * i], x1 = (double)x[o + 2 * i + 1];
+      out[o + 2 * i] = x0 * c - x1 * sn;
+      out[o + 2 * i + 1] = x0 * sn + x1 * c;
+    }
+    o += len[a];
+  }
+}
+
+/* The embedding alone: x [n_heads, F*L, d] -> out (double), for tests. */
+int oracle_rope3d(const float *x, double *out, int64_t nh, int64_t F, int64_t L, int64_t d, int64_t grid_w,
+                  int64_t frame_offset, double base) {
+  if (d <= 0 || d % 2 || grid_w <= 0 || L % grid_w) return 1;
+  for (int64_t h = 0; h < nh; ++h)
+    for (int64_t f = 0; f < F; ++f)
+      for (int64_t t = 0; t < L; ++t) {
+        const int64_t n = (h * F + f) * L + t;
+        rope3d(x + n * d, d, frame_offset + f, t / grid_w, t % grid_w, base, out + n * d);
+      }
+  return 0;
+}
+
 typedef struct {
   const float *q, *k, *v, *alpha, *beta;
   int logits;
@@ -72,6 +119,7 @@ typedef struct {
   int64_t F, L, dk, dv;
   int64_t bh;          /* flat head index */
   int64_t c0, c1;      /* column range [c0, c1) of d_v */
+  rope_t rope;         /* 3D RoPE on q and k (k before its normalisation) */
 } gdn_unit_t;
 
 static void gdn_unit(const gdn_unit_t *u) {
@@ -84,6 +132,7 @@ static void gdn_unit(const gdn_unit_t *u) {
   const float *be = u->beta + u->bh * N;
   double *S = (double *)calloc((size_t)(dk * nc), sizeof(double)); /* S[i][j - c0] */
   double *kh = (double *)malloc(sizeof(double) * (size_t)dk);
+  double *qr = (double *)malloc(sizeof(double) * (size_t)dk);
   double *r = (double *)malloc(sizeof(double) * (size_t)nc);
   if (u->s_in)
     for (int64_t i = 0; i < dk; ++i)
@@ -92,11 +141,17 @@ static void gdn_unit(const gdn_unit_t *u) {
     const double alpha = u->logits ? gate_alpha((double)al[f]) : (double)al[f];
     for (int64_t e = 0; e < dk * nc; ++e) S[e] *= alpha;
     for (int64_t t = f * L; t < (f + 1) * L; ++t) {
+      if (u->rope.on) {
+        rope3d(k + t * dk, dk, u->rope.frame_offset + f, (t - f * L) / u->rope.grid_w, (t - f * L) % u->rope.grid_w,
+               u->rope.base, kh);
+      } else {
+        for (int64_t i = 0; i < dk; ++i) kh[i] = (double)k[t * dk + i];
+      }
       double ss = 0.0;
-      for (int64_t i = 0; i < dk; ++i) ss += (double)k[t * dk + i] * (double)k[t * dk + i];
+      for (int64_t i = 0; i < dk; ++i) ss += kh[i] * kh[i];
       double nrm = sqrt(ss);
       double den = nrm > GDN_KEY_NORM_EPS ? nrm : GDN_KEY_NORM_EPS;
-      for (int64_t i = 0; i < dk; ++i) kh[i] = (double)k[t * dk + i] / den;
+      for (int64_t i = 0; i < dk; ++i) kh[i] = kh[i] / den;
       const double beta = u->logits ? gate_beta((double)be[t]) : (double)be[t];
       for (int64_t j = 0; j < nc; ++j) {
         double p = 0.0;
@@ -107,18 +162,26 @@ static void gdn_unit(const gdn_unit_t *u) {
         for (int64_t j = 0; j < nc; ++j) S[i * nc + j] -= beta * kh[i] * r[j];
     }
     if (u->o)
-      for (int64_t t = f * L; t < (f + 1) * L; ++t)
+      for (int64_t t = f * L; t < (f + 1) * L; ++t) {
+        if (u->rope.on) {
+          rope3d(q + t * dk, dk, u->rope.frame_offset + f, (t - f * L) / u->rope.grid_w,
+                 (t - f * L) % u->rope.grid_w, u->rope.base, qr);
+        } else {
+          for (int64_t i = 0; i < dk; ++i) qr[i] = (double)q[t * dk + i];
+        }
         for (int64_t j = 0; j < nc; ++j) {
           double acc = 0.0;
-          for (int64_t i = 0; i < dk; ++i) acc += S[i * nc + j] * (double)q[t * dk + i];
+          for (int64_t i = 0; i < dk; ++i) acc += S[i * nc + j] * qr[i];
           u->o[(u->bh * N + t) * dv + u->c0 + j] = acc;
         }
+      }
   }
   if (u->s_out)
     for (int64_t i = 0; i < dk; ++i)
       for (int64_t j = 0; j < nc; ++j) u->s_out[u->bh * dk * dv + i * dv + u->c0 + j] = S[i * nc + j];
   free(S);
   free(kh);
+  free(qr);
   free(r);
 }
 
@@ -141,7 +204,8 @@ static void *gdn_worker(void *p) {
 }
 
 /*
- * Gated DeltaNet frame recurrence.  Layouts (row-major, contiguous):
+ * Gated DeltaNet frame recurrence (optionally with the 3D RoPE on q and k).
+ * Layouts (row-major, contiguous):
  *   q, k [B,H,F*L,dk]; v [B,H,F*L,dv]; alpha [B,H,F]; beta [B,H,F*L];
  *   state_in/state_out [B,H,dk,dv] (nullable); o [B,H,F*L,dv] (nullable).
  * Only d_v columns [col_lo, col_hi) of o and state_out are written.
@@ -151,8 +215,11 @@ int oracle_gdn(const float *q, const float *k, const float *v, const float *alph
                int gates_are_logits, const double *state_in, double *state_out, double *o,
                int64_t B, int64_t H, int64_t F, int64_t L, int64_t dk, int64_t dv,
                int64_t col_lo, int64_t col_hi, const int64_t *heads, int64_t nheads,
-               int64_t col_block, int nthreads) {
+               int64_t col_block, int nthreads, int64_t rope_grid_w, int64_t rope_frame_offset,
+               double rope_base) {
   if (B < 0 || H < 0 || F < 0 || L < 0 || dk <= 0 || dv <= 0) return 1;
+  /* rope_grid_w > 0 turns the 3D RoPE on (q and k; needs even d_k and L a multiple of it) */
+  if (rope_grid_w > 0 && (dk % 2 || L % rope_grid_w)) return 1;
   if (col_lo < 0 || col_hi > dv || col_lo > col_hi) return 1;
   if (col_block <= 0) col_block = dv;
   int64_t nh = heads ? nheads : B * H;
@@ -169,6 +236,10 @@ int oracle_gdn(const float *q, const float *k, const float *v, const float *alph
       u->bh = heads ? heads[h] : h;
       u->c0 = col_lo + c * col_block;
       u->c1 = u->c0 + col_block < col_hi ? u->c0 + col_block : col_hi;
+      u->rope.on = rope_grid_w > 0;
+      u->rope.grid_w = rope_grid_w > 0 ? rope_grid_w : 1;
+      u->rope.frame_offset = rope_frame_offset;
+      u->rope.base = rope_base;
     }
   pool_t pl;
   pl.units = units; pl.n = n; pl.next = 0;

@@ -423,6 +423,76 @@ def test_gdn_stream_refuses_a_frame_cut_short():
     assert outs == [] and S is None and committed == []
 
 
+# ---------------------------------------------------------------- 3D RoPE
+
+def _rope_complex(x, F, L, grid_w, frame_offset=0, base=1e4):
+    """Independent construction: each rotated pair as a complex number times
+    exp(i * angle), the parts laid out as time, height, width."""
+    x = np.asarray(x, np.float64)
+    d = x.shape[-1]
+    dh = 2 * (d // 6)
+    dt = d - 2 * dh
+    t = np.arange(F * L)
+    frame, tl = t // L + frame_offset, t % L
+    out = np.empty_like(x)
+    for (o, n), pos in zip([(0, dt), (dt, dh), (dt + dh, dh)], [frame, tl // grid_w, tl % grid_w]):
+        z = x[..., o:o + n:2] + 1j * x[..., o + 1:o + n:2]
+        z = z * np.exp(1j * np.outer(pos, base ** (-np.arange(0, n, 2) / n)))
+        out[..., o:o + n:2], out[..., o + 1:o + n:2] = z.real, z.imag
+    return out
+
+
+@pytest.mark.parametrize("d,grid_w,off", [(12, 3, 0), (112, 40, 7), (32, 4, 100)])
+def test_rope3d_matches_complex_rotation(d, grid_w, off):
+    F, L = 3, 2 * grid_w
+    x = np.random.default_rng(d).standard_normal((2, F * L, d)).astype(np.float32)
+    got = oracle.rope3d(x, F=F, L=L, grid_w=grid_w, frame_offset=off)
+    np.testing.assert_allclose(got, _rope_complex(x, F, L, grid_w, off), rtol=0, atol=1e-12)
+
+
+def test_rope3d_invariants():
+    """Rotations keep norms (per token and per part), position (0, 0, 0) is the
+    identity, and the score of two rotated vectors depends only on their
+    relative position: shifting both in time by the same amount leaves it."""
+    d, grid_w, F, L = 24, 3, 4, 6
+    rng = np.random.default_rng(3)
+    q = rng.standard_normal((1, F * L, d)).astype(np.float32)
+    k = rng.standard_normal((1, F * L, d)).astype(np.float32)
+    rq = oracle.rope3d(q, F=F, L=L, grid_w=grid_w)
+    np.testing.assert_allclose(np.linalg.norm(rq, axis=-1), np.linalg.norm(q.astype(np.float64), axis=-1),
+                               rtol=1e-13)
+    np.testing.assert_array_equal(rq[0, 0], q[0, 0].astype(np.float64))  # frame 0, row 0, column 0
+    rk = oracle.rope3d(k, F=F, L=L, grid_w=grid_w)
+    rq5 = oracle.rope3d(q, F=F, L=L, grid_w=grid_w, frame_offset=5)
+    rk5 = oracle.rope3d(k, F=F, L=L, grid_w=grid_w, frame_offset=5)
+    np.testing.assert_allclose(rq[0] @ rk[0].T, rq5[0] @ rk5[0].T, rtol=1e-10, atol=1e-10)
+    # a vector that lives only in the height part ignores frame and column
+    dh = 2 * (d // 6)
+    dt = d - 2 * dh
+    hv = np.zeros((1, F * L, d), np.float32)
+    hv[..., dt:dt + dh] = 1.0
+    r = oracle.rope3d(hv, F=F, L=L, grid_w=grid_w)
+    rows = (np.arange(F * L) % L) // grid_w
+    for i in range(F * L):
+        j = np.where(rows == rows[i])[0][0]  # first token on the same row (another column or frame)
+        np.testing.assert_allclose(r[0, i], r[0, j], rtol=0, atol=1e-14)
+
+
+def test_gdn_with_rope_equals_gdn_on_rotated_inputs():
+    """RoPE enters the recurrence only through q and k: the RoPE run equals a
+    plain run fed q and k rotated by the independent complex construction."""
+    F, L, d, dv, grid_w = 3, 6, 12, 5, 3
+    q, k, v, a, b = _rand_case(2, F, L, d, dv, np.random.default_rng(21), unit=False)
+    o_r, s_r = oracle.gdn(q, k, v, a, b, F=F, L=L, rope=dict(grid_w=grid_w, frame_offset=2))
+    qr = _rope_complex(q, F, L, grid_w, 2).astype(np.float32)
+    kr = _rope_complex(k, F, L, grid_w, 2).astype(np.float32)
+    o_p, s_p = oracle.gdn(qr, kr, v, a, b, F=F, L=L)
+    np.testing.assert_allclose(o_r, o_p, rtol=1e-5, atol=1e-6)
+    np.testing.assert_allclose(s_r, s_p, rtol=1e-5, atol=1e-6)
+    o_n, _ = oracle.gdn(q, k, v, a, b, F=F, L=L)
+    assert np.abs(o_n - o_r).max() > 1e-2  # and it does change the result
+
+
 # ---------------------------------------------------------------- ReLU mode
 
 def _quadratic_masked_attention(q, k, v, F, L, eps):
