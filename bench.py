@@ -39,8 +39,9 @@ SPEC_HBM_GBS = 8000.0  # B200 HBM3e figure quoted as "about 8 TB/s"
 # algorithmic bytes per token-head: q, k, v bf16 (3 * 112 * 2) + o fp32 (112 * 4) + beta fp32
 BYTES_PER_TOKEN_HEAD = 3 * 112 * 2 + 112 * 4 + 4
 FLOPS_PER_TOKEN_HEAD = 6 * 112 * 112
-PRECISION = ("bf16 q/k/v; fp16 tensor-core operands with fp32 accumulation; the state is carried from frame to "
-             "frame, and taken from state_in, as fp16; fp32 o and state_out")
+PRECISION = ("bf16 q/k/v; fp16 tensor-core operands with fp32 accumulation; the state passes from frame to "
+             "frame as fp16 (each frame's map contracts; alpha = 1 over 240 frames is tested) and is taken "
+             "from state_in as fp16 high + low parts; fp32 o and state_out")
 
 
 def parse():

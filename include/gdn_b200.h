@@ -56,7 +56,7 @@ extern "C" {
 #define GDN_API
 #endif
 
-#define GDN_ABI_VERSION 3
+#define GDN_ABI_VERSION 4
 
 /* return / status codes */
 #define GDN_OK 0
@@ -106,6 +106,13 @@ typedef struct gdn_opts {
   int segments;           /* gdn on GDN_IMPL_TC.  0 = automatic; P >= 1: split every frame into P
                              runs of whole 64-token chunks handled by P CTAs (see gdn_frame_fwd);
                              P is lowered to the chunk count and to what fits one resident grid */
+  int rope_grid_w;        /* gdn only.  0: no position embedding.  > 0: the 3D rotary position
+                             embedding on q and k (k before its normalisation): a frame's L tokens
+                             are a grid of L / rope_grid_w rows of rope_grid_w tokens (L must be a
+                             multiple); see gdn_frame_fwd.  Not taken by GDN_IMPL_TC_PFORM */
+  int rope_frame_offset;  /* time coordinate of the call's first frame (a streaming call: its
+                             frame index in the video) */
+  float rope_base;        /* frequency base; 0 = 10000 */
 } gdn_opts_t;
 
 /*
@@ -139,10 +146,25 @@ typedef struct gdn_opts {
  * launch), so no CTA waits for work that has not started.  The automatic
  * choice takes P > 1 only when at most half the SMs would otherwise be busy.
  *
+ * 3D position embedding (opts->rope_grid_w > 0; SANA-Video's "3D RoPE for
+ * the linear attention", which the talk names without a formula; this is the
+ * library's reading): q_t and k_t are rotated before use, k_t before its
+ * normalisation.  With d = d_k, a time part of dt = d - 4 floor(d/6)
+ * dimensions comes first, then a height and a width part of 2 floor(d/6)
+ * each; in each part the pair (2i, 2i+1) turns by pos * base^(-2i/part_length)
+ * with pos the token's frame (f + rope_frame_offset), row (t / rope_grid_w)
+ * or column (t % rope_grid_w), t its index in the frame.  The workspace then
+ * also holds a table of the angles' cosines and sines (gdn_workspace_bytes
+ * counts it); d_k must be even and L a multiple of rope_grid_w.
+ *
  * Precision: fp32 inputs use fp32 arithmetic throughout (GDN_IMPL_SEQ /
  * FRAME_SIMT).  bf16 inputs on GDN_IMPL_TC multiply on tensor cores with
  * fp16 operands (11-bit significands) and fp32 accumulation; state and
- * outputs are fp32.  Its fp16 operands need |q|, |v| and |S| below 6.5e4.
+ * outputs are fp32.  The frame state passes from frame to frame as fp16 (each
+ * frame's map contracts, so the rounding does not accumulate); state_in is
+ * taken as fp16 high and low parts (about 22 significant bits).  The fp16
+ * operands need |q|, |v| and |S| below 65504: the kernels report
+ * GDN_ERR_RANGE otherwise.
  *
  * Returns GDN_OK or GDN_ERR_*.
  */
@@ -177,8 +199,11 @@ GDN_API int relu_la_block_fwd(const void *q, const void *k, const void *v, const
  * group are copied in and the output of the previous group is copied out
  * while a group runs, on two streams the call creates and destroys, ordered
  * after the work already queued on opts->stream.  The state passes from group
- * to group in fp32, so the result equals that of gdn_frame_fwd over the whole
- * sequence.  The call synchronises opts->stream before returning.
+ * to group through state_out / state_in in fp32 (the tensor-core kernel takes
+ * it as fp16 high and low parts, a little finer than its fp16 frame hand-off
+ * inside one call), so the result agrees with gdn_frame_fwd over the whole
+ * sequence to that rounding.  The call synchronises opts->stream before
+ * returning.
  * opts->workspace must hold gdn_workspace_bytes_host() bytes (two groups'
  * inputs and outputs, four states and one group's kernel workspace).
  */

@@ -40,7 +40,8 @@ class GdnOpts(ctypes.Structure):
     _fields_ = [("in_dtype", ctypes.c_int), ("gates_are_logits", ctypes.c_int), ("impl", ctypes.c_int),
                 ("stream", ctypes.c_void_p), ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
                 ("status", ctypes.c_void_p), ("max_ctas", ctypes.c_int), ("spin_limit_us", ctypes.c_int),
-                ("test_withhold_unit", ctypes.c_int), ("segments", ctypes.c_int)]
+                ("test_withhold_unit", ctypes.c_int), ("segments", ctypes.c_int), ("rope_grid_w", ctypes.c_int),
+                ("rope_frame_offset", ctypes.c_int), ("rope_base", ctypes.c_float)]
 
 
 _P = ctypes.c_void_p
@@ -97,7 +98,7 @@ def _stream_handle(stream) -> int:
 
 def make_opts(in_dtype: int, *, gates_are_logits: bool = True, impl="auto", stream=None, workspace=None,
               status=None, max_ctas: int = 0, spin_limit_us: int = 0, test_withhold_unit: int = -1,
-              segments: int = 0) -> GdnOpts:
+              segments: int = 0, rope=None) -> GdnOpts:
     o = GdnOpts()
     o.in_dtype = in_dtype
     o.gates_are_logits = int(bool(gates_are_logits))
@@ -111,6 +112,10 @@ def make_opts(in_dtype: int, *, gates_are_logits: bool = True, impl="auto", stre
     o.spin_limit_us = int(spin_limit_us)
     o.test_withhold_unit = int(test_withhold_unit) + 1 if test_withhold_unit >= 0 else 0
     o.segments = int(segments)
+    if rope is not None:  # dict(grid_w, frame_offset=0, base=1e4): the 3D RoPE on q and k
+        o.rope_grid_w = int(rope["grid_w"])
+        o.rope_frame_offset = int(rope.get("frame_offset", 0))
+        o.rope_base = float(rope.get("base", 1e4))
     return o
 
 
@@ -140,14 +145,17 @@ def _check(t, name, shape, dtype, device, allow_none=False):
 
 def gdn_frame_fwd(q, k, v, alpha, beta, *, F: int, state_in=None, state_out=None, o=None,
                   gates_are_logits: bool = True, impl="auto", workspace=None, stream=None, status=None,
-                  max_ctas: int = 0, spin_limit_us: int = 0, test_withhold_unit: int = -1, segments: int = 0):
+                  max_ctas: int = 0, spin_limit_us: int = 0, test_withhold_unit: int = -1, segments: int = 0,
+                  rope=None):
     """Frame-wise Gated DeltaNet forward on the GPU (see include/gdn_b200.h).
 
     q, k: [B, H, F*L, dk]; v: [B, H, F*L, dv] (float32 or bfloat16, same dtype);
     alpha: [B, H, F] float32; beta: [B, H, F*L] float32; state_in/state_out:
     [B, H, dk, dv] float32 or None.  Returns o [B, H, F*L, dv] float32.
     ``segments``: chunk segments per frame for the tensor-core kernel (0 =
-    automatic; see ``gdn_opts.segments``).
+    automatic; see ``gdn_opts.segments``).  ``rope``: None, or
+    dict(grid_w, frame_offset=0, base=1e4) for the 3D rotary position
+    embedding on q and k (see ``gdn_opts.rope_grid_w``).
     """
     B, H, N, dk = q.shape
     dv = v.shape[-1]
@@ -167,7 +175,7 @@ def gdn_frame_fwd(q, k, v, alpha, beta, *, F: int, state_in=None, state_out=None
     _check(o, "o", (B, H, N, dv), torch.float32, dev)
     opts = make_opts(_dtype_code(q), gates_are_logits=gates_are_logits, impl=impl, stream=stream,
                      status=status, max_ctas=max_ctas, spin_limit_us=spin_limit_us,
-                     test_withhold_unit=test_withhold_unit, segments=segments)
+                     test_withhold_unit=test_withhold_unit, segments=segments, rope=rope)
     need = workspace_bytes(OP_GDN, B, H, F, L, dk, dv, opts)
     if workspace is None and need > 0:
         workspace = alloc_workspace(need, dev)
@@ -215,7 +223,8 @@ def relu_la_block_fwd(q, k, v, *, F: int, kv_in=None, z_in=None, kv_out=None, z_
 
 
 def gdn_frame_fwd_host(q, k, v, alpha, beta, *, F: int, o, state_in=None, state_out=None,
-                       gates_are_logits: bool = True, impl="auto", workspace=None, stream=None, status=None):
+                       gates_are_logits: bool = True, impl="auto", workspace=None, stream=None, status=None,
+                       rope=None):
     """gdn_frame_fwd with HOST (CPU, ideally pinned) tensors; synchronous.
 
     Copies inputs into ``workspace`` (a device uint8 tensor of at least
@@ -227,7 +236,8 @@ def gdn_frame_fwd_host(q, k, v, alpha, beta, *, F: int, o, state_in=None, state_
     for t in (q, k, v, alpha, beta, o, state_in, state_out):
         if t is not None and (t.device.type != "cpu" or not t.is_contiguous()):
             raise ValueError("gdn_frame_fwd_host takes contiguous CPU tensors")
-    opts = make_opts(_dtype_code(q), gates_are_logits=gates_are_logits, impl=impl, stream=stream, status=status)
+    opts = make_opts(_dtype_code(q), gates_are_logits=gates_are_logits, impl=impl, stream=stream, status=status,
+                     rope=rope)
     need = host_workspace_bytes(B, H, F, L, dk, dv, opts)
     if workspace is None:
         workspace = alloc_workspace(need, torch.device("cuda", torch.cuda.current_device()))

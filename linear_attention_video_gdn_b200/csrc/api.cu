@@ -122,10 +122,16 @@ size_t gdn_ws_bytes_p(int impl, const gdn_opts_t *o, int B, int H, int F, int dk
   return b;
 }
 
+// Bytes of the 3D RoPE table (after the chain scratch in the workspace).
+size_t gdn_rope_bytes(const gdn_opts_t *o, int F, int L, int dk) {
+  if (o->rope_grid_w <= 0 || L % o->rope_grid_w) return 0;
+  return align_up(sizeof(float2) * rope_table_entries(F, L, o->rope_grid_w, dk), 256);
+}
+
 // Workspace for any launch these sizes and options may lead to: the segment
 // count is chosen on the device, so both the most segments and one segment
-// (the product-form kernel) are covered.
-size_t gdn_ws_bytes(int impl, const gdn_opts_t *o, int B, int H, int F, int L, int dk, int dv) {
+// (the product-form kernel) are covered; then the RoPE table.
+size_t gdn_ws_chain_bytes(int impl, const gdn_opts_t *o, int B, int H, int F, int L, int dk, int dv) {
   const int bound = gdn_seg_bound(impl, o, (long)B * H * F, L);
   size_t b = gdn_ws_bytes_p(impl, o, B, H, F, dk, dv, bound);
   if (bound > 1) {
@@ -133,6 +139,10 @@ size_t gdn_ws_bytes(int impl, const gdn_opts_t *o, int B, int H, int F, int L, i
     if (b1 > b) b = b1;
   }
   return b;
+}
+
+size_t gdn_ws_bytes(int impl, const gdn_opts_t *o, int B, int H, int F, int L, int dk, int dv) {
+  return gdn_ws_chain_bytes(impl, o, B, H, F, L, dk, dv) + gdn_rope_bytes(o, F, L, dk);
 }
 
 size_t relu_ws_bytes(int B, int H, int F, int dk, int dv) {
@@ -202,6 +212,13 @@ extern "C" int gdn_frame_fwd(const void *q, const void *k, const void *v, const 
   if (impl == GDN_IMPL_TC && (opts->in_dtype != GDN_DTYPE_BF16 || !gdn_tc_supported(dk, dv)))
     return GDN_ERR_UNSUPPORTED;
   if (opts->impl == GDN_IMPL_TC_PFORM && !gdn_pform_supported(dk, dv)) return GDN_ERR_UNSUPPORTED;
+  const bool rope = opts->rope_grid_w != 0;
+  if (rope) {
+    if (opts->rope_grid_w < 0 || L % opts->rope_grid_w || dk % 2 || !(opts->rope_base >= 0.0f) ||
+        opts->rope_frame_offset < 0)
+      return GDN_ERR_INVALID_ARG;
+    if (opts->impl == GDN_IMPL_TC_PFORM) return GDN_ERR_UNSUPPORTED;
+  }
 
   cudaStream_t st = (cudaStream_t)opts->stream;
   GdnParams p;
@@ -216,6 +233,20 @@ extern "C" int gdn_frame_fwd(const void *q, const void *k, const void *v, const 
   p.segs = 1;
 
   cudaError_t e;
+  if (rope) {
+    // the table after the chain scratch; filled on the stream before the recurrence
+    const size_t chain = impl == GDN_IMPL_SEQ ? 0 : gdn_ws_chain_bytes(impl, opts, B, H, F, L, dk, dv);
+    const size_t need = chain + gdn_rope_bytes(opts, F, L, dk);
+    if (!opts->workspace || opts->workspace_bytes < need) return GDN_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(opts->workspace) & 255u) != 0) return GDN_ERR_INVALID_ARG;
+    p.rope_on = 1;
+    p.rope_gw = opts->rope_grid_w;
+    p.rope_dh = 2 * (dk / 6);
+    p.rope_dt = dk - 2 * p.rope_dh;
+    p.rope_tab = reinterpret_cast<const float2 *>((char *)opts->workspace + chain);
+    e = launch_rope_table(p, opts->rope_frame_offset, opts->rope_base > 0.0f ? opts->rope_base : 10000.0f, st);
+    if (e != cudaSuccess) return GDN_ERR_CUDA;
+  }
   if (impl == GDN_IMPL_SEQ) {
     e = launch_gdn_seq(p, opts->in_dtype, st);
   } else {
@@ -223,6 +254,7 @@ extern "C" int gdn_frame_fwd(const void *q, const void *k, const void *v, const 
     const int P = gdn_segs(impl, opts, sms, units, L);
     const size_t need = gdn_ws_bytes_p(impl, opts, B, H, F, dk, dv, P);
     if (!opts->workspace || opts->workspace_bytes < need) return GDN_ERR_INVALID_ARG;
+    // (with RoPE the table follows the scratch of the most segments; checked above)
     if ((reinterpret_cast<uintptr_t>(opts->workspace) & 255u) != 0) return GDN_ERR_INVALID_ARG;
     p.ws = chain_workspace(opts->workspace, units * P);
     p.segs = P;
@@ -251,6 +283,7 @@ extern "C" int relu_la_block_fwd(const void *q, const void *k, const void *v, co
   if (opts->impl != GDN_IMPL_AUTO && opts->impl != GDN_IMPL_FRAME_SIMT && opts->impl != GDN_IMPL_TC)
     return GDN_ERR_INVALID_ARG;
   if (!(eps >= 0.0f)) return GDN_ERR_INVALID_ARG;
+  if (opts->rope_grid_w != 0) return GDN_ERR_UNSUPPORTED;  // the position embedding is built for gdn only
   int rc = check_sizes(B, H, F, L, dk, dv);
   if (rc != GDN_OK) return rc;
   const void *ptrs[] = {q, k, v, kv_in, z_in, kv_out, z_out, o, opts->workspace, opts->status};
@@ -289,9 +322,7 @@ extern "C" int relu_la_block_fwd(const void *q, const void *k, const void *v, co
 // gdn_frame_fwd_host streams the sequence through the device in groups of
 // frames: while group g runs, the inputs of group g + 1 are copied in and the
 // output of group g - 1 is copied out, on three streams.  The state passes
-// from group to group through state_out / state_in in fp32, which is how the
-// kernels hand it from frame to frame inside one call, so the result equals
-// that of one gdn_frame_fwd over the whole sequence.
+// from group to group through state_out / state_in in fp32.
 
 namespace {
 
@@ -419,6 +450,7 @@ extern "C" int gdn_frame_fwd_host(const void *q, const void *k, const void *v, c
                                : (const float *)(base + ((gi - 1) & 1 ? h.s_b : h.s_a));
     float *sout = gi == G - 1 ? (state_out ? (float *)(base + h.s_out) : nullptr)
                               : (float *)(base + (gi & 1 ? h.s_b : h.s_a));
+    inner.rope_frame_offset = opts->rope_frame_offset + f0;  // the group's first frame in the sequence
     rc = gdn_frame_fwd(slot + h.q, slot + h.k, slot + h.v, (const float *)(slot + h.alpha),
                        (const float *)(slot + h.beta), sin, sout, (float *)(slot + h.o), B, H, Fn, L, dk, dv,
                        &inner);

@@ -106,7 +106,55 @@ struct GdnParams {
   Workspace ws;   // flags and published states per segment unit ((b, h, f), then segment)
   int segs;       // chunk segments per frame (tcgen05 kernel; 1 elsewhere)
   uint32_t *ro_states;  // segs > 1: per (b, h, f) the end-of-frame S^T rows as bf16 high/low pairs
+  // 3D rotary position embedding of q and k (rope_on != 0): cos/sin of the angle of every
+  // (axis position, pair) as float2, time part [F][dt/2], then height [L/gw][dh/2], then width [gw][dh/2]
+  const float2 *rope_tab;
+  int rope_on, rope_gw, rope_dt, rope_dh;
 };
+
+// Rotated element i of the d_k-vector x (i's pair is i ^ 1) of the token at
+// index tf of frame f, with the table of the 3D rotary position embedding.
+template <typename T>
+__device__ __forceinline__ float rope_elem(const T *x, int i, int f, int tf, const GdnParams &p) {
+  const int pr = i & ~1;
+  int a_off, idx;
+  if (pr < p.rope_dt) {
+    a_off = f * (p.rope_dt / 2);
+    idx = pr / 2;
+  } else if (pr < p.rope_dt + p.rope_dh) {
+    a_off = p.F * (p.rope_dt / 2) + (tf / p.rope_gw) * (p.rope_dh / 2);
+    idx = (pr - p.rope_dt) / 2;
+  } else {
+    a_off = p.F * (p.rope_dt / 2) + (p.L / p.rope_gw) * (p.rope_dh / 2) + (tf % p.rope_gw) * (p.rope_dh / 2);
+    idx = (pr - p.rope_dt - p.rope_dh) / 2;
+  }
+  const float2 cs = __ldg(p.rope_tab + a_off + idx);
+  const float x0 = to_f32(x[pr]), x1 = to_f32(x[pr + 1]);
+  return (i & 1) ? fmaf(x0, cs.y, x1 * cs.x) : fmaf(x0, cs.x, -x1 * cs.y);
+}
+
+// The pair (dd, dd + 1) (dd even) of a token at index tf of frame f, rotated.
+__device__ __forceinline__ float2 rope_pair(float2 x, int dd, int f, int tf, const GdnParams &p) {
+  int a_off, idx;
+  if (dd < p.rope_dt) {
+    a_off = f * (p.rope_dt / 2);
+    idx = dd / 2;
+  } else if (dd < p.rope_dt + p.rope_dh) {
+    a_off = p.F * (p.rope_dt / 2) + (tf / p.rope_gw) * (p.rope_dh / 2);
+    idx = (dd - p.rope_dt) / 2;
+  } else {
+    a_off = p.F * (p.rope_dt / 2) + (p.L / p.rope_gw) * (p.rope_dh / 2) + (tf % p.rope_gw) * (p.rope_dh / 2);
+    idx = (dd - p.rope_dt - p.rope_dh) / 2;
+  }
+  const float2 cs = __ldg(p.rope_tab + a_off + idx);
+  return make_float2(fmaf(x.x, cs.x, -x.y * cs.y), fmaf(x.x, cs.y, x.y * cs.x));
+}
+
+// Entries of the RoPE table for these sizes (float2 each).
+inline size_t rope_table_entries(int F, int L, int gw, int dk) {
+  const int dh = 2 * (dk / 6), dt = dk - 2 * dh;
+  return (size_t)F * (dt / 2) + (size_t)(L / gw) * (dh / 2) + (size_t)gw * (dh / 2);
+}
 
 struct ReluParams {
   const void *q, *k, *v;

@@ -58,7 +58,9 @@ __global__ void __launch_bounds__(128) gdn_seq_kernel(GdnParams p) {
       __syncthreads();
       for (int e = j; e < kTile * DK; e += nthr) {
         const int tt = e / DK, i = e % DK;
-        sk[tt][i] = (tt < nt && i < dk) ? to_f32(k[(t0 + tt) * dk + i]) : 0.f;
+        sk[tt][i] = (tt < nt && i < dk) ? (p.rope_on ? rope_elem(k + (t0 + tt) * dk, i, f, (int)(t0 + tt - (long)f * L), p)
+                                                      : to_f32(k[(t0 + tt) * dk + i]))
+                                        : 0.f;
       }
       for (int e = j; e < kTile * 128; e += nthr) {
         const int tt = e / 128, c = e % 128;
@@ -93,7 +95,9 @@ __global__ void __launch_bounds__(128) gdn_seq_kernel(GdnParams p) {
       __syncthreads();
       for (int e = j; e < kTile * DK; e += nthr) {
         const int tt = e / DK, i = e % DK;
-        sk[tt][i] = (tt < nt && i < dk) ? to_f32(q[(t0 + tt) * dk + i]) : 0.f;
+        sk[tt][i] = (tt < nt && i < dk) ? (p.rope_on ? rope_elem(q + (t0 + tt) * dk, i, f, (int)(t0 + tt - (long)f * L), p)
+                                                      : to_f32(q[(t0 + tt) * dk + i]))
+                                        : 0.f;
       }
       __syncthreads();
       if (j < dv) {
@@ -168,7 +172,9 @@ __global__ void __launch_bounds__(256) gdn_frame_simt_kernel(GdnParams p) {
       __syncthreads();
       for (int e = c; e < kTile * DK; e += 256) {
         const int tt = e / DK, i = e % DK;
-        sm.sk[tt][i] = (tt < nt && i < dk) ? to_f32(k[(t0 + tt) * dk + i]) : 0.f;
+        sm.sk[tt][i] = (tt < nt && i < dk) ? (p.rope_on ? rope_elem(k + (t0 + tt) * dk, i, f, (int)(t0 + tt - t_beg), p)
+                                                         : to_f32(k[(t0 + tt) * dk + i]))
+                                           : 0.f;
       }
       for (int e = c; e < kTile * 128; e += 256) {
         const int tt = e / 128, x = e % 128;
@@ -268,7 +274,9 @@ __global__ void __launch_bounds__(256) gdn_frame_simt_kernel(GdnParams p) {
       __syncthreads();
       for (int e = c; e < kTile * DK; e += 256) {
         const int tt = e / DK, i = e % DK;
-        sm.sk[tt][i] = (tt < nt && i < dk) ? to_f32(q[(t0 + tt) * dk + i]) : 0.f;
+        sm.sk[tt][i] = (tt < nt && i < dk) ? (p.rope_on ? rope_elem(q + (t0 + tt) * dk, i, f, (int)(t0 + tt - t_beg), p)
+                                                         : to_f32(q[(t0 + tt) * dk + i]))
+                                           : 0.f;
       }
       __syncthreads();
       if (is_b) {

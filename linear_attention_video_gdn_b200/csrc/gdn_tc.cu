@@ -85,6 +85,7 @@ struct Bars {
   uint64_t mma_bar[2];          // per tile chain
   uint64_t fr_bar;              // frame-level MMAs (chain step)
   uint64_t q_full[2];           // read-out: q tile in buffer b
+  uint64_t q_conv[2];           // read-out with the position embedding: q tile b rotated, as fp16
   uint64_t o_full[2];           // read-out: the MMAs into O buffer b are done
   uint64_t o_free[2];           // read-out: the epilogue has read O buffer b
   uint64_t tkt_bar[2];          // chain group -> prep groups: next frame's ticket
@@ -197,7 +198,9 @@ __device__ __forceinline__ float4 neg4(float4 v) { return make_float4(-v.x, -v.y
 
 // kSeg: frames split into p.segs chunk segments (else one unit per frame; the
 // segment arithmetic folds away)
-template <bool kSeg>
+// kRope: the 3D rotary position embedding on q and k (a separate instantiation,
+// so that the kernel without it carries none of its code)
+template <bool kSeg, bool kRope>
 __global__ void __launch_bounds__(kGThreads, 1)
     gdn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                   const __grid_constant__ CUtensorMap tmap_v, GdnParams p) {
@@ -251,6 +254,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
       mbar_init(&bar.g_bar[s], 1);
       mbar_init(&bar.mma_bar[s], 1);
       mbar_init(&bar.q_full[s], 1);
+      mbar_init(&bar.q_conv[s], 1);
       mbar_init(&bar.o_full[s], 1);
       mbar_init(&bar.o_free[s], 1);
       mbar_init(&bar.tkt_bar[s], 1);
@@ -363,14 +367,19 @@ __global__ void __launch_bounds__(kGThreads, 1)
           }
           float ss = (ssp[0] + ssp[1]) + (ssp[2] + ssp[3]);
           ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-          const float inv = 1.0f / fmaxf(sqrtf(ss), kKeyNormEps);
+          const float inv = 1.0f / fmaxf(sqrtf(ss), kKeyNormEps);  // the rotation keeps the norm
+          const int tf = c * kC + t;  // token index in the frame
+          const bool rot = kRope && tf < L;
+          const int fr = rot ? unit_of(tk).f : 0;
 #pragma unroll
           for (int ch = 0; ch < 8; ++ch) {
             const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&ku[ch]);
             uint32_t o[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const float2 v2 = __bfloat1622float2(h[e]);
+              float2 v2 = __bfloat1622float2(h[e]);
+              const int dd = kb * 64 + ch * 8 + 2 * e;  // this pair's first dimension
+              if (rot && dd < dk) v2 = rope_pair(v2, dd, fr, tf, p);
               o[e] = pack_h2(v2.x * inv, v2.y * inv);
             }
             *reinterpret_cast<uint4 *>(krow + sw128_offset(t, ch * 8)) = make_uint4(o[0], o[1], o[2], o[3]);
@@ -595,7 +604,8 @@ __global__ void __launch_bounds__(kGThreads, 1)
     const uint32_t id_vw = idesc_f16(128, dk, 0, 1, 0);         // V^T (MN) x W
     const uint32_t id_kw = idesc_f16(128, dk, 0, 1, 0, 1, 0);   // -(Khat^T) (MN) x W
     const uint32_t id_s = idesc_f16(128, dk, 0, 0, 1);          // (alpha S^T, TMEM) x A^T (MN)
-    const uint32_t id_o = idesc_f16(128, kQTok, 1, 0, 0);       // S^T (bf16 pairs, TMEM) x Q^T (bf16)
+    // S^T (bf16 pairs, TMEM) x Q^T (bf16); with the position embedding fp16 pairs x rotated fp16 q
+    const uint32_t id_o = idesc_f16(128, kQTok, kRope ? 0 : 1, 0, 0);
     uint8_t *qbuf = sm + OFF_QB;                                 // q buffers, 16 KB each
     const uint32_t tmO = tmem + TM_R;                            // O buffers, 64 columns each
 
@@ -925,11 +935,19 @@ __global__ void __launch_bounds__(kGThreads, 1)
         for (int e = 0; e < 8; ++e) {
           const float a = j < dv ? r[2 * e] : 0.f;
           const float b = j < dv ? r[2 * e + 1] : 0.f;
-          const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-          const float2 hb = __bfloat1622float2(h);
-          const __nv_bfloat162 lw = __floats2bfloat162_rn(a - hb.x, b - hb.y);
-          hi[e] = *reinterpret_cast<const uint32_t *>(&h);
-          lo[e] = *reinterpret_cast<const uint32_t *>(&lw);
+          if (kRope) {  // the read-out's q is fp16 (rotated): fp16 pairs
+            const __half2 h = __floats2half2_rn(a, b);
+            const float2 hb = __half22float2(h);
+            const __half2 lw = __floats2half2_rn(a - hb.x, b - hb.y);
+            hi[e] = *reinterpret_cast<const uint32_t *>(&h);
+            lo[e] = *reinterpret_cast<const uint32_t *>(&lw);
+          } else {
+            const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+            const float2 hb = __bfloat1622float2(h);
+            const __nv_bfloat162 lw = __floats2bfloat162_rn(a - hb.x, b - hb.y);
+            hi[e] = *reinterpret_cast<const uint32_t *>(&h);
+            lo[e] = *reinterpret_cast<const uint32_t *>(&lw);
+          }
         }
         tmem_st8u(tmem + TM_Y + lane_off + lb / 2, hi);
         tmem_st8u(tmem + TM_Y + 64 + lane_off + lb / 2, lo);
@@ -1007,7 +1025,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
         int bad = 0;
         for (int n = 0; n < nt; ++n) {
           const uint32_t gt = rt + n, b = gt & 1u, ph = (gt >> 1) & 1u;
-          if (!mbar_wait(&bar.q_full[b], ph, lim)) {
+          if (!mbar_wait(kRope ? &bar.q_conv[b] : &bar.q_full[b], ph, lim)) {
             bad = 1;
             break;
           }
@@ -1037,6 +1055,47 @@ __global__ void __launch_bounds__(kGThreads, 1)
           *abort_flag = 1;
           latch_status(p.status, GDN_ERR_TIMEOUT);
           failed = true;
+        }
+      } else if (kRope && warp >= 1 && warp < 4) {
+        // position embedding: warps 1-3 rotate each q tile and convert it to fp16 in place
+        const int ct = tid - 32;
+        for (int n = 0; n < nt; ++n) {
+          const uint32_t gt = rt + n, b = gt & 1u, ph = (gt >> 1) & 1u;
+          {
+            const int bad = ct == 0 ? !mbar_wait(&bar.q_full[b], ph, lim) : 0;
+            if (bar_sync_or(6, 96, bad || *abort_flag)) {
+              if (bad) {
+                *abort_flag = 1;
+                latch_status(p.status, GDN_ERR_TIMEOUT);
+              }
+              failed = true;
+              break;
+            }
+          }
+          uint8_t *qb = qbuf + b * 16384;
+          float qmax = 0.f;
+          for (int i = ct; i < 1024; i += 96) {  // [column block][64 rows][8 x 16 B], swizzled
+            const int kb = i >> 9, rw = (i >> 3) & 63, pc = i & 7;
+            const int ch = pc ^ (rw & 7);
+            const int tf = tb0 + n * kQTok + rw;  // token index in the frame
+            uint4 *cp = reinterpret_cast<uint4 *>(qb + kb * 8192 + rw * 128 + pc * 16);
+            const uint4 u = *cp;
+            const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+            uint32_t o4[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              float2 v2 = __bfloat1622float2(h[e]);
+              const int dd = kb * 64 + ch * 8 + 2 * e;
+              if (tf < L && dd < dk) v2 = rope_pair(v2, dd, f, tf, p);
+              qmax = fmaxf(qmax, fmaxf(fabsf(v2.x), fabsf(v2.y)));
+              o4[e] = pack_h2(v2.x, v2.y);
+            }
+            *cp = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+          }
+          if (!(qmax < kF16Max)) latch_status(p.status, GDN_ERR_RANGE);
+          fence_async_smem();
+          named_bar(6, 96);
+          if (ct == 0) mbar_arrive_only(&bar.q_conv[b]);
         }
       } else if (tile == 1) {
         float *stg = reinterpret_cast<float *>(sm + OFF_STAGE);
@@ -1116,22 +1175,19 @@ bool gdn_tc_supported(int dk, int dv) {
 // published frame states are fp16 rows S^T[j][l]: d_k * d_v halves = d_k * d_v / 2 floats
 size_t gdn_tc_state_elems(int dk, int dv) { return (size_t)dk * dv / 2; }
 
-cudaError_t launch_gdn_tc(const GdnParams &p, int grid, bool cooperative, cudaStream_t st) {
+template <bool kRope>
+static cudaError_t launch_tc(const GdnParams &p, int grid, bool cooperative, cudaStream_t st, const CUtensorMap &mq,
+                             const CUtensorMap &mk, const CUtensorMap &mv) {
   using namespace tc;
-  CUtensorMap mq, mk, mv;
-  const int BH = p.B * p.H;
-  if (!make_bf16_map(&mq, p.q, p.dk, p.L, p.F, BH, kQTok) || !make_bf16_map(&mk, p.k, p.dk, p.L, p.F, BH, 64) ||
-      !make_bf16_map(&mv, p.v, p.dv, p.L, p.F, BH, 64))
-    return cudaErrorInvalidValue;
   if (!cooperative) {  // one unit per frame
-    cudaError_t e =
-        cudaFuncSetAttribute(gdn_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGdnSmemBytes);
+    cudaError_t e = cudaFuncSetAttribute(gdn_tc_kernel<false, kRope>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kGdnSmemBytes);
     if (e != cudaSuccess) return e;
-    gdn_tc_kernel<false><<<grid, kGThreads, kGdnSmemBytes, st>>>(mq, mk, mv, p);
+    gdn_tc_kernel<false, kRope><<<grid, kGThreads, kGdnSmemBytes, st>>>(mq, mk, mv, p);
     return cudaGetLastError();
   }
-  cudaError_t e =
-      cudaFuncSetAttribute(gdn_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGdnSmemBytes);
+  cudaError_t e = cudaFuncSetAttribute(gdn_tc_kernel<true, kRope>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)kGdnSmemBytes);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid);
@@ -1143,7 +1199,18 @@ cudaError_t launch_gdn_tc(const GdnParams &p, int grid, bool cooperative, cudaSt
   at[0].val.cooperative = 1;
   cfg.attrs = at;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, gdn_tc_kernel<true>, mq, mk, mv, p);
+  return cudaLaunchKernelEx(&cfg, gdn_tc_kernel<true, kRope>, mq, mk, mv, p);
+}
+
+cudaError_t launch_gdn_tc(const GdnParams &p, int grid, bool cooperative, cudaStream_t st) {
+  using namespace tc;
+  CUtensorMap mq, mk, mv;
+  const int BH = p.B * p.H;
+  if (!make_bf16_map(&mq, p.q, p.dk, p.L, p.F, BH, kQTok) || !make_bf16_map(&mk, p.k, p.dk, p.L, p.F, BH, 64) ||
+      !make_bf16_map(&mv, p.v, p.dv, p.L, p.F, BH, 64))
+    return cudaErrorInvalidValue;
+  return p.rope_on ? launch_tc<true>(p, grid, cooperative, st, mq, mk, mv)
+                   : launch_tc<false>(p, grid, cooperative, st, mq, mk, mv);
 }
 
 }  // namespace gdn

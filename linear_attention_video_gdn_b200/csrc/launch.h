@@ -8,6 +8,8 @@ namespace gdn {
 cudaError_t launch_gdn_seq(const GdnParams &p, int in_dtype, cudaStream_t st);
 cudaError_t launch_gdn_frame_simt(const GdnParams &p, int in_dtype, int grid, cudaStream_t st);
 cudaError_t launch_relu_frame_simt(const ReluParams &p, int in_dtype, int grid, cudaStream_t st);
+// fills p.rope_tab (the 3D RoPE table) on the stream
+cudaError_t launch_rope_table(const GdnParams &p, int frame_offset, float base, cudaStream_t st);
 
 // tcgen05 / TMEM / TMA kernels (bf16 inputs, dk = dv in {16..128} multiples of 16).
 bool gdn_tc_supported(int dk, int dv);

@@ -56,7 +56,7 @@ def test_header_constants_match_binding(lib):
     assert consts["GDN_DTYPE_BF16"] == lib.DTYPE_BF16 and consts["GDN_OP_RELU_LA"] == lib.OP_RELU_LA
     # the ctypes mirror of gdn_opts_t has the C layout (ints, pointers, size_t in declaration order)
     fields = re.search(r"typedef struct gdn_opts \{(.*?)\} gdn_opts_t;", text, re.S).group(1)
-    names = re.findall(r"^\s*(?:int|void|size_t)\s*\*?\s*(\w+);", fields, re.M)
+    names = re.findall(r"^\s*(?:int|void|size_t|float)\s*\*?\s*(\w+);", fields, re.M)
     assert names == [f[0] for f in lib.GdnOpts._fields_]
 
 

@@ -143,7 +143,8 @@ def test_shapes_all_impls(lib, dev, F, L, dk, dv, H, dtype):
 
 
 def test_streaming_equals_whole_sequence(lib, dev):
-    """F=1 calls that carry the state reproduce one call over all frames."""
+    """F=1 calls that carry the state reproduce one call over all frames (exactly up to
+    the fp32 kernels' rounding; within the state hand-off's rounding on tensor cores)."""
     w = W["gdn_480p_5s"].with_(F=4, L=90, H=3)
     x = synth.inputs(w)
     t, h = device_inputs(w, x, dev, torch)
@@ -161,8 +162,13 @@ def test_streaming_equals_whole_sequence(lib, dev):
             S = s_out
         torch.cuda.synchronize()
         o_str = torch.cat(outs, dim=2).cpu().numpy()
-        assert rel_err(o_str, o_all) <= 1e-5, impl
-        assert rel_err(S.cpu().numpy(), s_all) <= 1e-5, impl
+        # the fp32 kernels hand the state on in fp32 either way; the tensor-core kernel takes
+        # state_in as fp16 high + low parts but hands it from frame to frame as one fp16 image
+        tol = 1e-5 if impl in ("seq", "frame_simt") else 1e-3
+        assert rel_err(o_str, o_all) <= tol, impl
+        assert rel_err(S.cpu().numpy(), s_all) <= tol, impl
+    o_ref, s_ref = oracle_gdn(h, w)
+    assert rel_err(o_str, o_ref) <= 2e-3 and rel_err(S.cpu().numpy(), s_ref) <= 2e-3
 
 
 def test_in_place_state_carry(lib, dev):
@@ -305,8 +311,11 @@ def test_host_entry_point(lib, dev):
     o_h = torch.empty((w.B, w.H, w.N, w.dv), dtype=torch.float32).pin_memory()
     s_h = torch.empty((w.B, w.H, w.dk, w.dv), dtype=torch.float32).pin_memory()
     lib.gdn_frame_fwd_host(qh, kh, vh, ah, bh, F=w.F, o=o_h, state_out=s_h)
-    np.testing.assert_array_equal(o_h.numpy(), o_dev)
-    np.testing.assert_array_equal(s_h.numpy(), s_dev)
+    # frame groups pass the state through fp32 state_in (high + low fp16 parts), inside
+    # one call it passes as one fp16 image: equal within that rounding, and both parity
+    o_ref, s_ref = oracle_gdn(h, w)
+    assert rel_err(o_h.numpy(), o_ref) <= 2e-3 and rel_err(s_h.numpy(), s_ref) <= 2e-3
+    assert rel_err(o_h.numpy(), o_dev) <= 1e-3 and rel_err(s_h.numpy(), s_dev) <= 1e-3
 
 
 def test_device_timeout_status_is_reported(lib, dev):
@@ -439,3 +448,84 @@ def test_streaming_protocol_720p(lib, dev, segments):
         assert e <= 2e-3, (f, e)
         s_cur = s_next
     print(f"streaming protocol segments={segments}: worst err_o={worst_o:.3e} err_s={worst_s:.3e}")
+
+
+# ------------------------------------------------------------------ 3D rotary position embedding
+
+ROPE_SHAPES = [  # (F, L, grid_w, dk, dv, H, frame_offset)
+    (3, 40, 8, 112, 112, 2, 0), (2, 129, 43, 64, 64, 1, 5), (4, 30, 6, 48, 80, 2, 11), (1, 920, 40, 112, 112, 3, 17),
+]
+
+
+@pytest.mark.parametrize("F,L,gw,dk,dv,H,off", ROPE_SHAPES)
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_rope_matches_oracle(lib, dev, F, L, gw, dk, dv, H, off, dtype):
+    """q and k rotated by the 3D position embedding (latent grid L / gw x gw,
+    frames numbered from off) against the oracle, on every kernel that takes it."""
+    w = W["gdn_480p_5s"].with_(F=F, L=L, dk=dk, dv=dv, H=H, dtype=dtype, seed=300 + L + dk)
+    x = synth.inputs(w)
+    t, h = device_inputs(w, x, dev, torch)
+    rope = dict(grid_w=gw, frame_offset=off)
+    S0 = np.random.default_rng(L).standard_normal((w.B, w.H, dk, dv)).astype(np.float32)
+    o_ref, s_ref = oracle.gdn(h["q"], h["k"], h["v"], h["a"], h["b"], F=w.F, L=w.L, state_in=S0, rope=rope)
+    tol = tol_for(w)
+    for impl in [i for i in impls_for(w) if i != "tc_pform"]:
+        o, s = run_gdn(lib, w, t, dev, impl, state_in=S0, rope=rope)
+        eo, es = rel_err(o, o_ref), rel_err(s, s_ref)
+        print(f"rope {F}x{L} gw={gw} d={dk}/{dv} {dtype} {impl}: err_o={eo:.3e} err_s={es:.3e}")
+        assert eo <= tol and es <= tol, impl
+    if dtype == "bf16":  # the tensor-core kernel with chunk segments (several CTAs per frame)
+        o, s = run_gdn(lib, w, t, dev, "tc", state_in=S0, rope=rope, segments=3)
+        assert rel_err(o, o_ref) <= tol and rel_err(s, s_ref) <= tol
+
+
+def test_rope_resumed_call_and_host_entry(lib, dev):
+    """A sequence cut in two calls, the second with frame_offset = the frames of
+    the first, gives the one-call result; the host-buffer call (which streams
+    frame groups with their offsets) equals the device call."""
+    w = W["gdn_480p_5s"].with_(F=6, L=60, H=2, seed=41)
+    x = synth.inputs(w)
+    t, h = device_inputs(w, x, dev, torch)
+    rope = dict(grid_w=10, frame_offset=3)
+    o_all, s_all = run_gdn(lib, w, t, dev, "tc", rope=rope)
+    cut = 4 * w.L
+    w1, w2 = w.with_(F=4), w.with_(F=2)
+    t1 = {n: (t[n][:, :, :cut] if n != "a" else t[n][:, :, :4]).contiguous() for n in "qkvab"}
+    t2 = {n: (t[n][:, :, cut:] if n != "a" else t[n][:, :, 4:]).contiguous() for n in "qkvab"}
+    _, s1 = run_gdn(lib, w1, t1, dev, "tc", rope=rope)
+    o2, s2 = run_gdn(lib, w2, t2, dev, "tc", state_in=s1, rope=dict(grid_w=10, frame_offset=7))
+    assert rel_err(o2, o_all[:, :, cut:]) <= 2e-3 and rel_err(s2, s_all) <= 2e-3
+    o_ref, s_ref = oracle.gdn(h["q"], h["k"], h["v"], h["a"], h["b"], F=w.F, L=w.L, rope=rope)
+    assert rel_err(o_all, o_ref) <= 2e-3
+    qh, kh, vh = (t[n].cpu().pin_memory() for n in "qkv")
+    ah, bh = t["a"].cpu().pin_memory(), t["b"].cpu().pin_memory()
+    o_h = torch.empty((w.B, w.H, w.N, w.dv), dtype=torch.float32).pin_memory()
+    lib.gdn_frame_fwd_host(qh, kh, vh, ah, bh, F=w.F, o=o_h, rope=rope)
+    assert rel_err(o_h.numpy(), o_ref) <= 2e-3
+    assert rel_err(o_h.numpy(), o_all) <= 1e-3
+
+
+def test_rope_720p_60s_full(lib, dev):
+    """The 720p-60s workload with the 3D position embedding on its 23 x 40 latent
+    grid: every head and column against the oracle."""
+    w = W["gdn_720p_60s"]
+    x = synth.inputs(w)
+    t, h = device_inputs(w, x, dev, torch)
+    rope = dict(grid_w=40)
+    o, s = run_gdn(lib, w, t, dev, "tc", rope=rope)
+    o_ref, s_ref = oracle.gdn(h["q"], h["k"], h["v"], h["a"], h["b"], F=w.F, L=w.L, rope=rope)
+    eo, es = rel_err(o, o_ref), rel_err(s, s_ref)
+    print(f"rope 720p tc: err_o={eo:.3e} err_s={es:.3e}")
+    assert eo <= 2e-3 and es <= 2e-3
+
+
+def test_rope_refusals(lib, dev):
+    w = W["gdn_480p_5s"].with_(F=2, L=64, H=1)
+    x = synth.inputs(w)
+    t, _ = device_inputs(w, x, dev, torch)
+    with pytest.raises(lib.GdnError) as e:
+        run_gdn(lib, w, t, dev, "tc_pform", rope=dict(grid_w=8))
+    assert e.value.code == lib.ERR_UNSUPPORTED
+    with pytest.raises(lib.GdnError) as e:
+        run_gdn(lib, w, t, dev, "tc", rope=dict(grid_w=7))  # L is not a multiple of the grid width
+    assert e.value.code == lib.ERR_INVALID_ARG
