@@ -45,6 +45,8 @@ def _load():
                                    I64, I64, P, I64, I64, ctypes.c_int, I64, I64, ctypes.c_double]
         lib.oracle_rope3d.argtypes = [P, P, I64, I64, I64, I64, I64, I64, ctypes.c_double]
         lib.oracle_rope3d.restype = ctypes.c_int
+        lib.oracle_temporal_conv.argtypes = [P, P, P, P, P, P, I64, I64, I64, I64]
+        lib.oracle_temporal_conv.restype = ctypes.c_int
         lib.oracle_gdn.restype = ctypes.c_int
         lib.oracle_relu_la.argtypes = [P, P, P, P, P, P, P, P, I64, I64, I64, I64, I64, I64, ctypes.c_double,
                                        ctypes.c_int]
@@ -201,3 +203,22 @@ def gdn_stream(step_inputs, *, steps: int, L: int, state_in=None, cols=None):
         S = last_state
         committed.append(S)
     return outs, S, committed
+
+
+def temporal_conv(x, w, *, bias=None, cache_in=None):
+    """Causal temporal convolution of one block of frames with the block-boundary
+    cache, in fp64 (see oracle.c): x [B, F, HW, C]; w [C, 3]; bias [C] or None;
+    cache_in [B, HW, C] or None (zero).  Returns (y [B, F, HW, C], cache_out
+    [B, HW, C] = the block's last frame)."""
+    x = _f32(x)
+    B, F, HW, C = x.shape
+    w = _f32(w)
+    assert w.shape == (C, 3)
+    b = None if bias is None else _f32(bias)
+    ci = None if cache_in is None else _f32(cache_in)
+    y = np.empty(x.shape, np.float64)
+    co = np.empty((B, HW, C), np.float64)
+    rc = _load().oracle_temporal_conv(_ptr(x), _ptr(w), _ptr(b), _ptr(ci), _ptr(y), _ptr(co), B, F, HW, C)
+    if rc != 0:
+        raise ValueError("oracle_temporal_conv: invalid arguments")
+    return y, co

@@ -358,3 +358,38 @@ int oracle_relu_la(const float *q, const float *k, const float *v, const double 
   free(units);
   return 0;
 }
+
+/*
+ * Causal temporal convolution of one block of frames with the block-boundary
+ * cache (SANA-Video talk, causal Mix-FFN passage: in training a zero token
+ * separates two blocks so that block one cannot see block two, and block
+ * two is prefixed with block one's last token; both are removed after the
+ * convolution).  The library's reading: a depthwise convolution of kernel 3
+ * along the frame axis, per latent position n and channel c,
+ *   y[f][n][c] = w[c][0] x[f-1][n][c] + w[c][1] x[f][n][c] + w[c][2] x[f+1][n][c] + bias[c]
+ * where x[-1] is the cached last frame of the previous block (zero without
+ * one) and x[F] is zero (the block cannot see the next one).  cache_out is
+ * the block's last frame.  Layouts: x, y [B, F, HW, C]; cache [B, HW, C];
+ * w [C][3]; bias [C] (nullable).
+ */
+int oracle_temporal_conv(const float *x, const float *w, const float *bias, const float *cache_in, double *y,
+                         double *cache_out, int64_t B, int64_t F, int64_t HW, int64_t C) {
+  if (B < 0 || F <= 0 || HW <= 0 || C <= 0) return 1;
+  for (int64_t b = 0; b < B; ++b)
+    for (int64_t f = 0; f < F; ++f)
+      for (int64_t n = 0; n < HW; ++n)
+        for (int64_t c = 0; c < C; ++c) {
+          const int64_t at = ((b * F + f) * HW + n) * C + c;
+          const double prev = f > 0 ? (double)x[at - HW * C] : (cache_in ? (double)cache_in[(b * HW + n) * C + c] : 0.0);
+          const double next = f + 1 < F ? (double)x[at + HW * C] : 0.0;
+          double acc = (double)w[c * 3 + 0] * prev + (double)w[c * 3 + 1] * (double)x[at] + (double)w[c * 3 + 2] * next;
+          if (bias) acc += (double)bias[c];
+          y[at] = acc;
+        }
+  if (cache_out)
+    for (int64_t b = 0; b < B; ++b)
+      for (int64_t n = 0; n < HW; ++n)
+        for (int64_t c = 0; c < C; ++c)
+          cache_out[(b * HW + n) * C + c] = (double)x[((b * F + F - 1) * HW + n) * C + c];
+  return 0;
+}

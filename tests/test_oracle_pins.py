@@ -493,6 +493,69 @@ def test_gdn_with_rope_equals_gdn_on_rotated_inputs():
     assert np.abs(o_n - o_r).max() > 1e-2  # and it does change the result
 
 
+# ---------------------------------------------------------------- causal temporal conv with block cache
+
+def _training_construction(blocks, w, bias):
+    """The talk's training-time construction, through a library convolution: the
+    blocks laid end to end along time with a zero token and then a copy of the
+    previous block's last frame before every later block, one depthwise
+    kernel-3 convolution (zero padding at both ends) over the whole sequence,
+    and the inserted positions dropped."""
+    import torch
+    seq, keep = [], []
+    for i, blk in enumerate(blocks):
+        if i > 0:
+            seq += [np.zeros_like(blk[:, :1]), blocks[i - 1][:, -1:]]
+            keep += [False, False]
+        seq.append(blk)
+        keep += [True] * blk.shape[1]
+    x = np.concatenate(seq, axis=1).astype(np.float64)           # [B, T, HW, C]
+    B, T, HW, C = x.shape
+    xt = torch.from_numpy(x).permute(0, 2, 3, 1).reshape(B * HW, C, T)
+    wt = torch.from_numpy(np.asarray(w, np.float64)).reshape(C, 1, 3)
+    bt = None if bias is None else torch.from_numpy(np.asarray(bias, np.float64))
+    yt = torch.nn.functional.conv1d(xt, wt, bt, padding=1, groups=C)
+    y = yt.reshape(B, HW, C, T).permute(0, 3, 1, 2).numpy()
+    return y[:, np.array(keep)]
+
+
+@pytest.mark.parametrize("with_bias", [False, True])
+def test_temporal_conv_stream_equals_training_construction(with_bias):
+    rng = np.random.default_rng(31)
+    B, HW, C = 2, 5, 6
+    blocks = [rng.standard_normal((B, F, HW, C)).astype(np.float32) for F in (3, 1, 4)]
+    w = rng.standard_normal((C, 3)).astype(np.float32)
+    bias = rng.standard_normal(C).astype(np.float32) if with_bias else None
+    outs, cache = [], None
+    for blk in blocks:
+        y, cache = oracle.temporal_conv(blk, w, bias=bias, cache_in=cache)
+        outs.append(y)
+        np.testing.assert_array_equal(cache, blk[:, -1].astype(np.float64))
+    np.testing.assert_allclose(np.concatenate(outs, axis=1), _training_construction(blocks, w, bias),
+                               rtol=1e-12, atol=1e-12)
+
+
+def test_temporal_conv_impulse_and_block_boundaries():
+    """An impulse at frame f of a block spreads to frames f-1, f, f+1 of the same
+    block only (through the cache, to the first frame of the next block when f
+    is the last frame; never back into the previous block)."""
+    B, F, HW, C = 1, 4, 1, 3
+    w = np.array([[1., 2., 3.], [4., 5., 6.], [7., 8., 9.]], np.float32)
+    for f in range(F):
+        x = np.zeros((B, F, HW, C), np.float32)
+        x[0, f, 0, :] = 1.0
+        y, cache = oracle.temporal_conv(x, w)
+        expect = np.zeros((B, F, HW, C))
+        expect[0, f, 0] = w[:, 1]
+        if f > 0:
+            expect[0, f - 1, 0] = w[:, 2]
+        if f + 1 < F:
+            expect[0, f + 1, 0] = w[:, 0]
+        np.testing.assert_array_equal(y, expect)
+        y2, _ = oracle.temporal_conv(np.zeros_like(x), w, cache_in=cache)
+        np.testing.assert_array_equal(y2[0, 0, 0], w[:, 0] * (1.0 if f == F - 1 else 0.0))
+
+
 # ---------------------------------------------------------------- ReLU mode
 
 def _quadratic_masked_attention(q, k, v, F, L, eps):
