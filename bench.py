@@ -283,6 +283,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         if not args.no_streaming:
             extra["streaming"] = streaming_leg(args, lib, synth, torch, dev, stream, cpu_on)
         extra["configs_other"] = small_configs_leg(args, lib, synth, torch, dev, stream, cpu_on)
+        extra["temporal_conv"] = temporal_conv_leg(args, lib, synth, torch, dev, stream, cpu_on)
     peak, peak_src = measured_peaks()
     alg_bytes = token_heads * BYTES_PER_TOKEN_HEAD + w.B * w.H * (w.F * 4 + w.dk * w.dv * 4)
     achieved = alg_bytes / (ms / 1e3) / 1e9
@@ -537,6 +538,68 @@ def streaming_leg(args, lib, synth, torch, dev, stream, cpu_baseline_on):
         out["cpu_baseline"] = {"value": tps, "unit": "step tokens/s", "cores": nthreads, "kind": "oracle",
                                "sample": f"one streaming call (20 heads, 920 tokens) repeated {runs} times in "
                                          f"{secs:.1f} s"}
+    return out
+
+
+def temporal_conv_leg(args, lib, synth, torch, dev, stream, cpu_baseline_on):
+    """The causal temporal convolution with the block-boundary cache at the 720p
+    latent grid and model width (HW = 920, C = 2240, bf16): the whole 60 s clip
+    as one block of 240 frames, and the clip generated as 24 blocks of 10
+    frames with the cache carried in place from block to block."""
+    peak, src = measured_peaks()
+    out = {}
+    cw = synth.CONV_WORKLOADS["tconv_720p_60s"]
+    inp = synth.conv_inputs(cw)
+    x = torch.from_numpy(inp["x"]).to(torch.bfloat16).to(dev)
+    del inp["x"]
+    w_, b_ = torch.from_numpy(inp["w"]).to(dev), torch.from_numpy(inp["bias"]).to(dev)
+    cache = torch.zeros((cw.B, cw.HW, cw.C), dtype=torch.bfloat16, device=dev)
+    y = torch.empty_like(x)
+    call = lambda: lib.temporal_conv_fwd(x, w_, bias=b_, cache_in=cache, cache_out=cache, y=y)
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    ms = _events_ms(call, max(10, args.steps), stream)
+    es = 2
+    nb = 2 * es * x.numel() + 2 * es * cache.numel()
+    out["whole_clip"] = {"workload": cw.name, "B": cw.B, "F": cw.F, "HW": cw.HW, "C": cw.C, "dtype": cw.dtype,
+                         "ms": ms, "frames_per_s": cw.B * cw.F / (ms / 1e3),
+                         "tokens_per_s": cw.B * cw.F * cw.HW / (ms / 1e3),
+                         "roofline": _roofline(nb, ms, peak, src),
+                         "l2": "x and y 0.99 GB each, larger than L2; no flush needed"}
+    del x, y
+    sw = synth.CONV_WORKLOADS["tconv_stream_720p"]
+    pool_n = 8
+    pool = [torch.from_numpy(synth.conv_inputs(sw, block=i)["x"]).to(torch.bfloat16).to(dev) for i in range(pool_n)]
+    ys = torch.empty_like(pool[0])
+    sc = torch.zeros((sw.B, sw.HW, sw.C), dtype=torch.bfloat16, device=dev)
+
+    def blocks():
+        for i in range(sw.blocks):
+            lib.temporal_conv_fwd(pool[i % pool_n], w_, bias=b_, cache_in=sc if i else None, cache_out=sc, y=ys)
+
+    blocks()
+    torch.cuda.synchronize()
+    ms_s = _events_ms(blocks, 3, stream)
+    nbs = sw.blocks * (2 * es * pool[0].numel() + es * sc.numel()) + (sw.blocks - 1) * es * sc.numel()
+    out["streaming_blocks"] = {"workload": sw.name, "B": sw.B, "F_per_block": sw.F, "blocks": sw.blocks,
+                               "HW": sw.HW, "C": sw.C, "ms_all_blocks": ms_s, "us_per_block": ms_s * 1e3 / sw.blocks,
+                               "frames_per_s": sw.B * sw.F * sw.blocks / (ms_s / 1e3),
+                               "roofline": _roofline(nbs, ms_s, peak, src),
+                               "l2": f"blocks cycled from a pool of {pool_n} distinct blocks (330 MB, more than "
+                                     f"L2)"}
+    del pool, ys, sc
+    if cpu_baseline_on:
+        import oracle
+        n_pos = 92
+        xs = synth.conv_inputs(sw, frames=sw.F)["x"][:, :, :n_pos]
+        xs = torch.from_numpy(np.ascontiguousarray(xs)).to(torch.bfloat16).float().numpy()
+        tps, runs, secs = _oracle_tokens_per_s(lambda: oracle.temporal_conv(xs, inp["w"], bias=inp["bias"]),
+                                               sw.B * sw.F * n_pos)
+        out["cpu_baseline"] = {"value": tps, "unit": "tokens/s (latent positions x frames, all 2240 channels)",
+                               "cores": 1, "kind": "oracle",
+                               "sample": f"one block of {sw.F} frames x {n_pos} of {sw.HW} latent positions, "
+                                         f"{runs} runs in {secs:.1f} s"}
     return out
 
 

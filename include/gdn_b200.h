@@ -56,7 +56,7 @@ extern "C" {
 #define GDN_API
 #endif
 
-#define GDN_ABI_VERSION 4
+#define GDN_ABI_VERSION 5
 
 /* return / status codes */
 #define GDN_OK 0
@@ -188,6 +188,39 @@ GDN_API int gdn_frame_fwd(const void *q, const void *k, const void *v, const flo
 GDN_API int relu_la_block_fwd(const void *q, const void *k, const void *v, const float *kv_in, const float *z_in,
                       float *kv_out, float *z_out, float *o, int B, int H, int F, int L, int dk, int dv,
                       float eps, const gdn_opts_t *opts);
+
+/*
+ * temporal_conv_fwd -- causal temporal convolution of one block of latent
+ * frames with the block-boundary cache.
+ *
+ * SANA-Video's causal feed-forward network convolves along time (talk
+ * transcript, causal FFN passage): in training a zero token separates two
+ * blocks, so the first block cannot see the second, and the second block is
+ * prefixed with the first block's last frame; both inserted tokens are
+ * dropped after the convolution.  Generated block by block, the same result
+ * comes from carrying the last frame of each block in a cache.  The talk gives
+ * no kernel size; this library's reading is a depthwise convolution of kernel
+ * 3, centred on the frame (one zero token is exactly the separation a kernel
+ * of 3 needs).  For every batch b, latent position n < HW and channel c < C:
+ *
+ *   y[b,f,n,c] = w[c][0] x[b,f-1,n,c] + w[c][1] x[b,f,n,c] + w[c][2] x[b,f+1,n,c] + bias[c]
+ *
+ * with x[b,-1,n,c] = cache_in[b,n,c] (zero if cache_in == NULL: the first
+ * block) and x[b,F,n,c] = 0 (a block never sees the next one); then
+ * cache_out[b,n,c] <- x[b,F-1,n,c] (skipped if cache_out == NULL).  Calling
+ * this once per block with cache_in = the previous call's cache_out gives the
+ * training construction's result over the whole video.
+ *
+ * x, y: [B, F, HW, C], element type opts->in_dtype; cache_in, cache_out:
+ * [B, HW, C], the same type (a copy of a frame, exact); w: [C, 3] float32;
+ * bias: [C] float32 or NULL.  The arithmetic is fp32 and y is rounded once
+ * to the element type (nearest even for bf16).  cache_in may equal cache_out
+ * (in-place carry); no other two of x, y and the caches may overlap
+ * (GDN_ERR_INVALID_ARG).  Sizes: B, F, HW, C >= 1.  Options used: in_dtype,
+ * stream, max_ctas; no workspace.  Returns GDN_OK or GDN_ERR_*.
+ */
+GDN_API int temporal_conv_fwd(const void *x, const float *w, const float *bias, const void *cache_in,
+                              void *cache_out, void *y, int B, int F, int HW, int C, const gdn_opts_t *opts);
 
 /*
  * gdn_frame_fwd_host -- gdn_frame_fwd with HOST tensors.

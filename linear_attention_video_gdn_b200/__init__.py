@@ -32,7 +32,7 @@ IMPLS = {"auto": IMPL_AUTO, "seq": IMPL_SEQ, "frame_simt": IMPL_FRAME_SIMT, "tc"
 
 EXPORTED = ("gdn_frame_fwd", "relu_la_block_fwd", "gdn_frame_fwd_host", "gdn_frame_fwd_noalloc",
             "gdn_workspace_bytes", "gdn_workspace_bytes_host", "gdn_status_string", "gdn_status_str",
-            "gdn_abi_version")
+            "gdn_abi_version", "temporal_conv_fwd")
 NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
 
 
@@ -54,6 +54,8 @@ _lib.gdn_frame_fwd_noalloc.argtypes = [_P] * 8 + [_I] * 6 + [ctypes.POINTER(GdnO
 _lib.gdn_frame_fwd_noalloc.restype = _I
 _lib.relu_la_block_fwd.argtypes = [_P] * 8 + [_I] * 6 + [ctypes.c_float, ctypes.POINTER(GdnOpts)]
 _lib.relu_la_block_fwd.restype = _I
+_lib.temporal_conv_fwd.argtypes = [_P] * 6 + [_I] * 4 + [ctypes.POINTER(GdnOpts)]
+_lib.temporal_conv_fwd.restype = _I
 _lib.gdn_workspace_bytes.argtypes = [_I] * 7 + [ctypes.POINTER(GdnOpts)]
 _lib.gdn_workspace_bytes.restype = ctypes.c_size_t
 _lib.gdn_workspace_bytes_host.argtypes = [_I] * 6 + [ctypes.POINTER(GdnOpts)]
@@ -220,6 +222,29 @@ def relu_la_block_fwd(q, k, v, *, F: int, kv_in=None, z_in=None, kv_out=None, z_
     if rc != OK:
         raise GdnError(rc, "relu_la_block_fwd")
     return o
+
+
+def temporal_conv_fwd(x, w, *, bias=None, cache_in=None, cache_out=None, y=None, stream=None, max_ctas: int = 0):
+    """Causal temporal convolution of one block of frames with the block-boundary
+    cache on the GPU (see include/gdn_b200.h).  x: [B, F, HW, C] float32 or
+    bfloat16; w: [C, 3] float32; bias: [C] float32 or None; cache_in /
+    cache_out: [B, HW, C] of x's dtype or None.  Returns y (x's shape and dtype)."""
+    B, F, HW, C = x.shape
+    dev = x.device
+    _check(x, "x", (B, F, HW, C), x.dtype, dev)
+    _check(w, "w", (C, 3), torch.float32, dev)
+    _check(bias, "bias", (C,), torch.float32, dev, allow_none=True)
+    _check(cache_in, "cache_in", (B, HW, C), x.dtype, dev, allow_none=True)
+    _check(cache_out, "cache_out", (B, HW, C), x.dtype, dev, allow_none=True)
+    if y is None:
+        y = torch.empty_like(x)
+    _check(y, "y", (B, F, HW, C), x.dtype, dev)
+    opts = make_opts(_dtype_code(x), stream=stream, max_ctas=max_ctas)
+    rc = _lib.temporal_conv_fwd(_ptr(x), _ptr(w), _ptr(bias), _ptr(cache_in), _ptr(cache_out), _ptr(y),
+                                B, F, HW, C, ctypes.byref(opts))
+    if rc != OK:
+        raise GdnError(rc, "temporal_conv_fwd")
+    return y
 
 
 def gdn_frame_fwd_host(q, k, v, alpha, beta, *, F: int, o, state_in=None, state_out=None,

@@ -317,6 +317,40 @@ extern "C" int relu_la_block_fwd(const void *q, const void *k, const void *v, co
   return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
+namespace gdn {
+namespace {
+bool overlap(const void *a, size_t na, const void *b, size_t nb) {
+  if (!a || !b) return false;
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+}  // namespace
+}  // namespace gdn
+
+extern "C" int temporal_conv_fwd(const void *x, const float *w, const float *bias, const void *cache_in,
+                                 void *cache_out, void *y, int B, int F, int HW, int C, const gdn_opts_t *opts) {
+  using namespace gdn;
+  if (!opts || !x || !w || !y) return GDN_ERR_INVALID_ARG;
+  if (opts->in_dtype != GDN_DTYPE_F32 && opts->in_dtype != GDN_DTYPE_BF16) return GDN_ERR_INVALID_ARG;
+  if (B < 1 || F < 1 || HW < 1 || C < 1) return GDN_ERR_INVALID_ARG;
+  if ((long long)B * F * HW * C > (1LL << 40)) return GDN_ERR_UNSUPPORTED;
+  const void *ptrs[] = {x, w, bias, cache_in, cache_out, y};
+  for (const void *ptr : ptrs)
+    if (!aligned16(ptr)) return GDN_ERR_INVALID_ARG;
+  const size_t es = opts->in_dtype == GDN_DTYPE_BF16 ? 2 : 4;
+  const size_t nx = es * (size_t)B * F * HW * C, nc = es * (size_t)B * HW * C;
+  if (overlap(x, nx, y, nx) || overlap(cache_in, nc, y, nx) || overlap(cache_out, nc, y, nx) ||
+      overlap(cache_out, nc, x, nx) || (cache_in != cache_out && overlap(cache_in, nc, cache_out, nc)))
+    return GDN_ERR_INVALID_ARG;
+  int sms = 0, cc = 0;
+  int rc = device_info(&sms, &cc);
+  if (rc != GDN_OK) return rc;
+  if (cc != 100) return GDN_ERR_NO_DEVICE;
+  const cudaError_t e = launch_temporal_conv(x, w, bias, cache_in, cache_out, y, B, F, HW, C, opts->in_dtype, sms,
+                                             opts->max_ctas, (cudaStream_t)opts->stream);
+  return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
 // ---------------------------------------------------------------- host I/O
 //
 // gdn_frame_fwd_host streams the sequence through the device in groups of

@@ -171,3 +171,51 @@ def inputs(w: Workload, heads=None, call: int = 0, frames: int | None = None) ->
         a = a.reshape(w.B, w.H, F)
         b = b.reshape(w.B, w.H, N)
     return dict(q=q, k=k, v=v, a=a, b=b)
+
+
+# ---------------------------------------------------------------- temporal convolution inputs
+
+@dataclass(frozen=True)
+class ConvWorkload:
+    """Shape and input distribution of a causal temporal convolution workload:
+    x [B, F, HW, C] per block of F latent frames, depthwise kernel-3 weights
+    w [C, 3] and bias [C]; ``blocks`` consecutive blocks (streaming)."""
+    name: str
+    B: int
+    F: int
+    HW: int
+    C: int
+    dtype: str
+    seed: int
+    blocks: int = 1
+
+
+# tensor ids of the temporal convolution draws (block c uses ids base + 8 * c)
+TID_X, TID_W, TID_BIAS = 0, 1, 2
+
+# The 720p latent grid (23x40 = 920 positions) at the model width of 20 heads
+# of 112 channels: the whole 60 s clip (240 latent frames) as one block, and
+# the same clip generated in 24 blocks of 10 frames with the cache carried.
+CONV_WORKLOADS = {
+    "tconv_720p_60s": ConvWorkload("tconv_720p_60s", 1, 240, 920, 2240, "bf16", seed=5),
+    "tconv_stream_720p": ConvWorkload("tconv_stream_720p", 1, 10, 920, 2240, "bf16", seed=6, blocks=24),
+}
+
+
+def conv_inputs(cw: ConvWorkload, block: int = 0, frames: int | None = None) -> dict:
+    """Draw x (block ``block``; its first ``frames`` frames when given), w and
+    bias for ``cw`` as float32 numpy arrays.  x ~ N(0, 1); w ~ N(0, 1/3) so that
+    the output keeps about unit variance; bias ~ N(0, 0.1^2).  w and bias are
+    shared by all blocks."""
+    F = cw.F if frames is None else min(frames, cw.F)
+    off = TID_STRIDE_PER_CALL * block
+    x = normal(cw.seed, TID_X + off, 0, cw.B * cw.F * cw.HW * cw.C).reshape(cw.B, cw.F, cw.HW, cw.C) \
+        if F == cw.F else None
+    if x is None:  # a prefix of every batch's frames
+        x = np.empty((cw.B, F, cw.HW, cw.C), np.float32)
+        per_b = cw.F * cw.HW * cw.C
+        for b in range(cw.B):
+            normal(cw.seed, TID_X + off, b * per_b, F * cw.HW * cw.C, out=x[b].reshape(-1))
+    w = normal(cw.seed, TID_W, 0, cw.C * 3, std=3.0 ** -0.5).reshape(cw.C, 3)
+    bias = normal(cw.seed, TID_BIAS, 0, cw.C, std=0.1)
+    return dict(x=x, w=w, bias=bias)

@@ -143,6 +143,28 @@ def test_host_argument_validation(lib):
                                  ctypes.c_float(-1.0), ctypes.byref(o)) == lib.ERR_INVALID_ARG
 
 
+def test_temporal_conv_argument_validation(lib):
+    raw = lib._lib
+    o = lib.make_opts(lib.DTYPE_BF16, stream=0)
+    P = ctypes.c_void_p
+    x, w, y, c = P(0x100000), P(0x200000), P(0x300000), P(0x400000)  # never dereferenced
+    call = lambda *a: raw.temporal_conv_fwd(*a, ctypes.byref(o))
+    assert call(None, w, None, None, None, y, 1, 4, 8, 16) == lib.ERR_INVALID_ARG       # null x
+    assert call(x, w, None, None, None, None, 1, 4, 8, 16) == lib.ERR_INVALID_ARG       # null y
+    assert call(x, P(0x200004), None, None, None, y, 1, 4, 8, 16) == lib.ERR_INVALID_ARG  # misaligned w
+    assert call(x, w, None, None, None, y, 1, 0, 8, 16) == lib.ERR_INVALID_ARG          # F = 0
+    assert call(x, w, None, None, None, P(0x100010), 1, 4, 8, 16) == lib.ERR_INVALID_ARG  # y overlaps x
+    assert call(x, w, None, None, P(0x100000 + 512), y, 1, 4, 8, 16) == lib.ERR_INVALID_ARG   # cache in x
+    assert call(x, w, None, c, P(0x400010), y, 1, 4, 8, 16) == lib.ERR_INVALID_ARG      # caches overlap
+    o.in_dtype = 5
+    assert call(x, w, None, None, None, y, 1, 4, 8, 16) == lib.ERR_INVALID_ARG          # bad dtype
+    o.in_dtype = lib.DTYPE_BF16
+    assert raw.temporal_conv_fwd(x, w, None, None, None, y, 1, 4, 8, 16, None) == lib.ERR_INVALID_ARG
+    import torch
+    if not torch.cuda.is_available():  # valid arguments, in-place cache: the device check comes last
+        assert call(x, w, None, c, c, y, 1, 4, 8, 16) == lib.ERR_NO_DEVICE
+
+
 def test_no_device_is_reported_without_gpu(lib):
     import torch
     if torch.cuda.is_available():
