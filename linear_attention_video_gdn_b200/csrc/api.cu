@@ -346,7 +346,7 @@ extern "C" int temporal_conv_fwd(const void *x, const float *w, const float *bia
   int rc = device_info(&sms, &cc);
   if (rc != GDN_OK) return rc;
   if (cc != 100) return GDN_ERR_NO_DEVICE;
-  const cudaError_t e = launch_temporal_conv(x, w, bias, cache_in, cache_out, y, B, F, HW, C, opts->in_dtype, sms,
+  const cudaError_t e = launch_temporal_conv(x, w, bias, cache_in, cache_out, y, B, F, HW, C, opts->in_dtype,
                                              opts->max_ctas, (cudaStream_t)opts->stream);
   return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }

@@ -21,10 +21,10 @@ cudaError_t launch_gdn_tc(const GdnParams &p, int grid, bool cooperative, cudaSt
 bool gdn_pform_supported(int dk, int dv);
 size_t gdn_pform_state_bytes(int dk, int dv);  // published bytes per frame
 cudaError_t launch_gdn_pform(const GdnParams &p, int grid, cudaStream_t st);
-// causal temporal convolution with the block-boundary cache (one resident wave)
+// causal temporal convolution with the block-boundary cache (one CTA per run of frames of a column tile)
 cudaError_t launch_temporal_conv(const void *x, const float *w, const float *bias, const void *cache_in,
-                                 void *cache_out, void *y, int B, int F, int HW, int C, int in_dtype, int sms,
-                                 int max_ctas, cudaStream_t st);
+                                 void *cache_out, void *y, int B, int F, int HW, int C, int in_dtype, int max_ctas,
+                                 cudaStream_t st);
 bool relu_tc_supported(int dk, int dv);
 cudaError_t launch_relu_tc(const ReluParams &p, int grid, cudaStream_t st);
 

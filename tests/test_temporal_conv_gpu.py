@@ -83,11 +83,13 @@ def run_case(lib, dev, B, F, HW, C, dtype, *, seed=11, bias=True, cache=True, ma
     return y
 
 
-# B, F, HW, C: vector columns (C % 8 == 0), several tiles of 256 columns with a
+# B, F, HW, C: vector columns (C % 8 == 0), several tiles of 128 columns with a
 # ragged last tile, single-element columns (C not a multiple of the vector),
-# one frame, and frame counts around the load step of 4.
+# one frame, frame counts around the prefetch depths, and frame counts above
+# the 32-frame run of one CTA (runs that start and end inside a column, with
+# a halo frame on each side), exactly two runs, and one frame past a run.
 SHAPES = [(1, 5, 7, 16), (2, 13, 300, 64), (1, 1, 9, 24), (2, 6, 5, 12), (1, 9, 33, 6), (3, 4, 2, 8),
-          (1, 8, 130, 40)]
+          (1, 8, 130, 40), (1, 70, 33, 16), (2, 64, 9, 24), (1, 33, 20, 8), (1, 100, 5, 6), (2, 45, 7, 12)]
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
@@ -103,15 +105,17 @@ def test_optional_arguments(lib, dev, dtype, bias, cache):
 
 
 @pytest.mark.parametrize("max_ctas", [1, 3, 7, 50])
-def test_frame_runs_split_across_ctas(lib, dev, max_ctas):
-    """Few CTAs: every CTA covers several frame runs of several column tiles, so
-    runs start and end inside a column (halo frames on both sides)."""
-    run_case(lib, dev, 2, 23, 150, 32, "bf16", max_ctas=max_ctas)
-    run_case(lib, dev, 1, 17, 45, 12, "f32", max_ctas=max_ctas)
+def test_few_ctas_loop_over_runs(lib, dev, max_ctas):
+    """A capped grid: every CTA loops over several runs of several column tiles,
+    including runs that start and end inside a column (halo frames)."""
+    run_case(lib, dev, 2, 75, 40, 32, "bf16", max_ctas=max_ctas)
+    run_case(lib, dev, 1, 41, 45, 12, "f32", max_ctas=max_ctas)
 
 
 def test_in_place_cache(lib, dev):
     run_case(lib, dev, 2, 9, 40, 48, "bf16", inplace=True, max_ctas=5)
+    run_case(lib, dev, 1, 70, 30, 16, "bf16", inplace=True)
+    run_case(lib, dev, 1, 40, 30, 20, "f32", inplace=True)
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
