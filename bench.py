@@ -57,7 +57,46 @@ def parse():
                     help="use only the first N latent frames (a smaller case of the same kernel, for profiling)")
     ap.add_argument("--quick", action="store_true",
                     help="kernel leg only: no end-to-end leg, no ReLU-mode line, no CPU baseline")
+    ap.add_argument("--profile-case", choices=["gdn", "relu", "tconv", "stream"], default=None,
+                    help="run three launches of one kernel on a small case (inputs larger than L2, under 1 GB) "
+                         "and exit: the command profiled with ncu --set full")
     return ap.parse_args()
+
+
+def profile_case(name: str):
+    """Three launches of one kernel at a reduced size of its workload: gdn_tc_kernel
+    on the first 48 frames of the 720p 60 s shape, relu_tc_kernel on 16 of the 81
+    frames, the temporal convolution on 60 of the 240 frames, and one streaming
+    call (F = 1, all 20 heads, 920 tokens; 12 MB, L2-resident as in the protocol)."""
+    import torch
+
+    import linear_attention_video_gdn_b200 as lib
+    import synth
+    dev = torch.device("cuda", 0)
+    if name in ("gdn", "stream"):
+        w = synth.WORKLOADS["gdn_720p_60s"].with_(F=48) if name == "gdn" else synth.WORKLOADS["gdn_stream_720p"]
+        x = synth.inputs(w)
+        q, k, v = (torch.from_numpy(x[n]).to(torch.bfloat16).to(dev) for n in "qkv")
+        a, b = (torch.from_numpy(x[n]).to(dev) for n in "ab")
+        F = w.F if name == "gdn" else 1
+        s_in = torch.zeros((w.B, w.H, w.dk, w.dv), dtype=torch.float32, device=dev) if name == "stream" else None
+        call = lambda: lib.gdn_frame_fwd(q, k, v, a, b, F=F, state_in=s_in)
+    elif name == "relu":
+        w = synth.WORKLOADS["relu_720p_81f"].with_(F=16)
+        x = synth.inputs(w)
+        q, k, v = (torch.from_numpy(x[n]).to(torch.bfloat16).to(dev) for n in "qkv")
+        call = lambda: lib.relu_la_block_fwd(q, k, v, F=w.F)
+    else:
+        cw = synth.CONV_WORKLOADS["tconv_720p_60s"]
+        inp = synth.conv_inputs(cw, frames=60)
+        xc = torch.from_numpy(inp["x"]).to(torch.bfloat16).to(dev)
+        wc, bc = torch.from_numpy(inp["w"]).to(dev), torch.from_numpy(inp["bias"]).to(dev)
+        cache = torch.zeros((cw.B, cw.HW, cw.C), dtype=torch.bfloat16, device=dev)
+        call = lambda: lib.temporal_conv_fwd(xc, wc, bias=bc, cache_in=cache, cache_out=cache)
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    print(f"profile case {name}: 3 launches done", flush=True)
 
 
 def measured_peaks():
@@ -610,6 +649,9 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", 0))
     if args.impl == "reference":
         run_reference(args, rank)
+        return
+    if args.profile_case:
+        profile_case(args.profile_case)
         return
     if world > 1:
         import datetime
