@@ -109,22 +109,32 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_source_hash() -> str:
+# source files each profiled kernel is built from: a committed traffic figure
+# counts only while their hash matches the figure's
+KERNEL_SOURCES = {
+    "gdn_tc": ("gdn_tc.cu", "tc_ptx.cuh", "common.cuh"),
+    "relu_tc": ("relu_tc.cu", "tc_ptx.cuh", "common.cuh"),
+    "temporal_conv": ("temporal_conv.cu", "tc_ptx.cuh", "common.cuh"),
+}
+
+
+def kernel_source_hash(kernel: str = "gdn_tc") -> str:
     h = hashlib.sha256()
-    for name in ("gdn_tc.cu", "tc_ptx.cuh", "common.cuh"):
+    for name in KERNEL_SOURCES[kernel]:
         with open(os.path.join(ROOT, "linear_attention_video_gdn_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def ncu_traffic():
-    """DRAM bytes per launch of the GDN kernel from the committed ncu summary, if it
-    was taken on the current kernel source (else None)."""
-    path = os.path.join(ROOT, "profiles", "gdn_tc_traffic.json")
+def ncu_traffic(kernel: str = "gdn_tc"):
+    """DRAM bytes per launch of a kernel from its committed ncu summary
+    (profiles/<kernel>_traffic.json), if it was taken on the current kernel
+    source (else None)."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}_traffic.json")
     try:
         with open(path) as f:
             d = json.load(f)
-        if d.get("kernel_source_sha") == kernel_source_hash():
+        if d.get("kernel_source_sha") == kernel_source_hash(kernel):
             return d
     except Exception:
         pass
@@ -326,7 +336,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     peak, peak_src = measured_peaks()
     alg_bytes = token_heads * BYTES_PER_TOKEN_HEAD + w.B * w.H * (w.F * 4 + w.dk * w.dv * 4)
     achieved = alg_bytes / (ms / 1e3) / 1e9
-    tr = ncu_traffic() if w.F == 240 else None
+    tr = ncu_traffic("gdn_tc") if w.F == 240 else None
     line = {
         "metric": METRIC,
         "value": whole_job_tokens_per_s(tokens, world, ms),
@@ -440,8 +450,12 @@ def relu_leg(args, lib, synth, torch, dev, stream, cpu_baseline_on):
     rms = _events_ms(call, max(5, args.steps // 2), stream)
     rbytes = wr.B * wr.H * wr.N * (3 * wr.dk * 2 + wr.dv * 4) + wr.B * wr.H * wr.dk * (wr.dv + 1) * 4
     peak, src = measured_peaks()
+    roof = _roofline(rbytes, rms, peak, src)
+    tr = ncu_traffic("relu_tc")
+    roof["traffic"] = None if tr is None else tr["dram_bytes_per_launch"]
+    roof["traffic_source"] = None if tr is None else tr["source"]
     out = {"workload": "relu_720p_81f", "B": wr.B, "H": wr.H, "F": wr.F, "L": wr.L, "d": wr.dk, "ms": rms,
-           "tokens_per_s": wr.B * wr.N / (rms / 1e3), "roofline": _roofline(rbytes, rms, peak, src),
+           "tokens_per_s": wr.B * wr.N / (rms / 1e3), "roofline": roof,
            "achieved_gbs": rbytes / (rms / 1e3) / 1e9, "frac_hbm": rbytes / (rms / 1e3) / 1e9 / peak,
            "l2": "inputs 2.0 GB, larger than L2; no flush needed"}
     del rq, rk, rv, ro, rws
@@ -601,10 +615,14 @@ def temporal_conv_leg(args, lib, synth, torch, dev, stream, cpu_baseline_on):
     ms = _events_ms(call, max(10, args.steps), stream)
     es = 2
     nb = 2 * es * x.numel() + 2 * es * cache.numel()
+    roof = _roofline(nb, ms, peak, src)
+    tr = ncu_traffic("temporal_conv")
+    roof["traffic"] = None if tr is None else tr["dram_bytes_per_launch"]
+    roof["traffic_source"] = None if tr is None else tr["source"]
     out["whole_clip"] = {"workload": cw.name, "B": cw.B, "F": cw.F, "HW": cw.HW, "C": cw.C, "dtype": cw.dtype,
                          "ms": ms, "frames_per_s": cw.B * cw.F / (ms / 1e3),
                          "tokens_per_s": cw.B * cw.F * cw.HW / (ms / 1e3),
-                         "roofline": _roofline(nb, ms, peak, src),
+                         "roofline": roof,
                          "l2": "x and y 0.99 GB each, larger than L2; no flush needed"}
     del x, y
     sw = synth.CONV_WORKLOADS["tconv_stream_720p"]
