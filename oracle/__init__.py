@@ -45,6 +45,9 @@ def _load():
                                    I64, I64, P, I64, I64, ctypes.c_int, I64, I64, ctypes.c_double]
         lib.oracle_rope3d.argtypes = [P, P, I64, I64, I64, I64, I64, I64, ctypes.c_double]
         lib.oracle_rope3d.restype = ctypes.c_int
+        lib.oracle_softmax_window.argtypes = [P, P, P, P, I64, I64, I64, I64, I64, I64, I64, ctypes.c_double, P,
+                                              ctypes.c_int]
+        lib.oracle_softmax_window.restype = ctypes.c_int
         lib.oracle_temporal_conv.argtypes = [P, P, P, P, P, P, I64, I64, I64, I64]
         lib.oracle_temporal_conv.restype = ctypes.c_int
         lib.oracle_gdn.restype = ctypes.c_int
@@ -222,3 +225,27 @@ def temporal_conv(x, w, *, bias=None, cache_in=None):
     if rc != 0:
         raise ValueError("oracle_temporal_conv: invalid arguments")
     return y, co
+
+
+def softmax_window(q, k, v, *, F: int, L: int, W: int, scale=None, frames=None, nthreads=None):
+    """Windowed block-causal softmax attention in fp64 (see oracle.c): q, k
+    [B, H, F*L, dk], v [B, H, F*L, dv]; token t of frame f attends to all tokens
+    of frames max(0, f-W+1) .. f with weights softmax(scale q_t . k_s), scale
+    defaulting to 1/sqrt(dk).  ``frames``: compute only these query frames (the
+    other rows of o are NaN)."""
+    q, k, v = _f32(q), _f32(k), _f32(v)
+    B, H, N, dk = q.shape
+    dv = v.shape[-1]
+    assert N == F * L and k.shape == q.shape and v.shape[:3] == (B, H, N)
+    sc = float(dk) ** -0.5 if scale is None else float(scale)
+    mask = None
+    o = np.empty((B, H, N, dv), np.float64)
+    if frames is not None:
+        mask = np.zeros(F, np.uint8)
+        mask[list(frames)] = 1
+        o.fill(np.nan)
+    nt = nthreads or max(1, min(64, os.cpu_count() or 1))
+    rc = _load().oracle_softmax_window(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, H, F, L, dk, dv, W, sc, _ptr(mask), nt)
+    if rc != 0:
+        raise ValueError("oracle_softmax_window: invalid arguments")
+    return o

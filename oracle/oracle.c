@@ -393,3 +393,85 @@ int oracle_temporal_conv(const float *x, const float *w, const float *bias, cons
           cache_out[(b * HW + n) * C + c] = (double)x[((b * F + F - 1) * HW + n) * C + c];
   return 0;
 }
+
+/*
+ * Windowed block-causal softmax attention: the softmax layers that SANA-WM's
+ * hybrid interleaves with the frame-wise Gated DeltaNet (GeekNews summary of
+ * SANA-WM, "Core design and generation pipeline": periodic softmax; the
+ * Vietnamese post: Gated DeltaNet for most of the sequence, softmax windows
+ * in between; SANA-Video talk: long videos keep softmax inside a sliding
+ * window).  The library's reading: token t of frame f attends to every token
+ * of frames max(0, f-W+1) .. f (its own frame in full, as in the linear
+ * modes), o_t = sum_s softmax_s(scale q_t . k_s) v_s.  Per (b, h) and per
+ * frame f the key set is shared; rows of o outside frame_mask (if given, one
+ * byte per frame) are left untouched.  q, k: [B, H, F*L, dk]; v, o: [B, H, F*L, dv].
+ */
+typedef struct {
+  const float *q, *k, *v;
+  double *o;
+  int64_t BH, F, L, dk, dv, W;
+  double scale;
+  const unsigned char *frame_mask;
+  int64_t next; /* shared work counter over (bh, f) */
+  pthread_mutex_t mu;
+} sw_job_t;
+
+static void sw_unit(sw_job_t *j, int64_t bh, int64_t f) {
+  const int64_t N = j->F * j->L;
+  const int64_t f0 = f - j->W + 1 < 0 ? 0 : f - j->W + 1;
+  const int64_t nk = (f - f0 + 1) * j->L;
+  double *sc = (double *)malloc(sizeof(double) * (size_t)nk);
+  for (int64_t t = f * j->L; t < (f + 1) * j->L; ++t) {
+    const float *qt = j->q + (bh * N + t) * j->dk;
+    double m = -INFINITY;
+    for (int64_t s = 0; s < nk; ++s) {
+      const float *ks = j->k + (bh * N + f0 * j->L + s) * j->dk;
+      double acc = 0.0;
+      for (int64_t i = 0; i < j->dk; ++i) acc += (double)qt[i] * (double)ks[i];
+      sc[s] = acc * j->scale;
+      if (sc[s] > m) m = sc[s];
+    }
+    double den = 0.0;
+    for (int64_t s = 0; s < nk; ++s) {
+      sc[s] = exp(sc[s] - m);
+      den += sc[s];
+    }
+    double *ot = j->o + (bh * N + t) * j->dv;
+    for (int64_t c = 0; c < j->dv; ++c) ot[c] = 0.0;
+    for (int64_t s = 0; s < nk; ++s) {
+      const float *vs = j->v + (bh * N + f0 * j->L + s) * j->dv;
+      const double p = sc[s] / den;
+      for (int64_t c = 0; c < j->dv; ++c) ot[c] += p * (double)vs[c];
+    }
+  }
+  free(sc);
+}
+
+static void *sw_worker(void *arg) {
+  sw_job_t *j = (sw_job_t *)arg;
+  for (;;) {
+    pthread_mutex_lock(&j->mu);
+    const int64_t u = j->next++;
+    pthread_mutex_unlock(&j->mu);
+    if (u >= j->BH * j->F) break;
+    const int64_t bh = u / j->F, f = u % j->F;
+    if (j->frame_mask && !j->frame_mask[f]) continue;
+    sw_unit(j, bh, f);
+  }
+  return NULL;
+}
+
+int oracle_softmax_window(const float *q, const float *k, const float *v, double *o, int64_t B, int64_t H, int64_t F,
+                          int64_t L, int64_t dk, int64_t dv, int64_t W, double scale,
+                          const unsigned char *frame_mask, int nthreads) {
+  if (B <= 0 || H <= 0 || F <= 0 || L <= 0 || dk <= 0 || dv <= 0 || W <= 0) return 1;
+  sw_job_t j = {q, k, v, o, B * H, F, L, dk, dv, W, scale, frame_mask, 0};
+  pthread_mutex_init(&j.mu, NULL);
+  if (nthreads < 1) nthreads = 1;
+  if (nthreads > 256) nthreads = 256;
+  pthread_t th[256];
+  for (int i = 0; i < nthreads; ++i) pthread_create(&th[i], NULL, sw_worker, &j);
+  for (int i = 0; i < nthreads; ++i) pthread_join(th[i], NULL);
+  pthread_mutex_destroy(&j.mu);
+  return 0;
+}

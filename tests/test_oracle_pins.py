@@ -556,6 +556,87 @@ def test_temporal_conv_impulse_and_block_boundaries():
         np.testing.assert_array_equal(y2[0, 0, 0], w[:, 0] * (1.0 if f == F - 1 else 0.0))
 
 
+# ---------------------------------------------------------------- windowed softmax attention
+
+def _sdpa_window(q, k, v, F, L, W, scale=None):
+    """The windowed layer through the library's attention primitive: one fp64
+    scaled_dot_product_attention over the whole sequence with a boolean mask
+    (key frame within [query frame - W + 1, query frame])."""
+    import torch
+    fr = np.arange(F * L) // L
+    allowed = (fr[None, :] <= fr[:, None]) & (fr[None, :] >= fr[:, None] - W + 1)
+    qt, kt, vt = (torch.from_numpy(np.asarray(x, np.float64)) for x in (q, k, v))
+    out = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, attn_mask=torch.from_numpy(allowed),
+                                                           scale=scale)
+    return out.numpy()
+
+
+@pytest.mark.parametrize("F,L,W,dk,dv", [(5, 3, 2, 4, 3), (4, 6, 1, 8, 8), (3, 5, 4, 6, 2), (6, 2, 3, 5, 7)])
+def test_softmax_window_equals_masked_library_attention(F, L, W, dk, dv):
+    rng = np.random.default_rng(40 + F)
+    q = rng.standard_normal((2, 3, F * L, dk)).astype(np.float32)
+    k = rng.standard_normal((2, 3, F * L, dk)).astype(np.float32)
+    v = rng.standard_normal((2, 3, F * L, dv)).astype(np.float32)
+    o = oracle.softmax_window(q, k, v, F=F, L=L, W=W)
+    np.testing.assert_allclose(o, _sdpa_window(q, k, v, F, L, W), rtol=1e-12, atol=1e-12)
+    o2 = oracle.softmax_window(q, k, v, F=F, L=L, W=W, scale=0.3)
+    np.testing.assert_allclose(o2, _sdpa_window(q, k, v, F, L, W, scale=0.3), rtol=1e-12, atol=1e-12)
+
+
+def test_softmax_window_closed_forms():
+    rng = np.random.default_rng(5)
+    F, L, d = 4, 3, 4
+    q = rng.standard_normal((1, 1, F * L, d)).astype(np.float32)
+    k = rng.standard_normal((1, 1, F * L, d)).astype(np.float32)
+    # constant values: every output row is that value
+    v = np.tile(np.array([1.5, -2.0, 0.25], np.float32), (1, 1, F * L, 1))
+    np.testing.assert_allclose(oracle.softmax_window(q, k, v, F=F, L=L, W=2), v.astype(np.float64), rtol=1e-14)
+    # zero queries: the plain mean of the window's values (frames f-W+1 .. f, clipped at 0)
+    v = rng.standard_normal((1, 1, F * L, 3)).astype(np.float32)
+    o = oracle.softmax_window(np.zeros_like(q), k, v, F=F, L=L, W=2)
+    for f in range(F):
+        lo = max(0, f - 1) * L
+        np.testing.assert_allclose(o[0, 0, f * L:(f + 1) * L], np.tile(v[0, 0, lo:(f + 1) * L].astype(np.float64).mean(0), (L, 1)),
+                                   rtol=1e-12, atol=1e-14)
+    # one dominant key inside the window picks its value; the same key just outside the window is ignored
+    qd = np.zeros((1, 1, F * L, d), np.float32)
+    kd = np.zeros((1, 1, F * L, d), np.float32)
+    qd[..., 0] = 1.0
+    kd[0, 0, 4, 0] = 60.0  # frame 1, token 1
+    o = oracle.softmax_window(qd, kd, v, F=F, L=L, W=2, scale=1.0)
+    np.testing.assert_allclose(o[0, 0, 3 * 1:3 * 3], np.tile(v[0, 0, 4], (6, 1)), rtol=1e-12, atol=1e-12)  # frames 1, 2
+    uniform = o[0, 0, 9:12]  # frame 3 sees frames 2, 3 only: no dominant key, zero scores
+    np.testing.assert_allclose(uniform, np.tile(v[0, 0, 6:12].astype(np.float64).mean(0), (3, 1)), rtol=1e-12, atol=1e-14)
+    # W >= F: block-causal attention over all earlier frames; W = 1: within the frame only
+    v = rng.standard_normal((1, 1, F * L, 3)).astype(np.float32)
+    full = oracle.softmax_window(q, k, v, F=F, L=L, W=F + 3)
+    np.testing.assert_allclose(full, oracle.softmax_window(q, k, v, F=F, L=L, W=F), rtol=0, atol=0)
+    own = oracle.softmax_window(q, k, v, F=F, L=L, W=1)
+    for f in range(F):
+        sl = slice(f * L, (f + 1) * L)
+        np.testing.assert_allclose(own[0, 0, sl], oracle.softmax_window(q[:, :, sl], k[:, :, sl], v[:, :, sl], F=1,
+                                                                         L=L, W=1)[0, 0], rtol=1e-14)
+
+
+def test_softmax_window_frame_subset_and_permutation():
+    rng = np.random.default_rng(6)
+    F, L, d = 5, 4, 6
+    q, k = (rng.standard_normal((1, 2, F * L, d)).astype(np.float32) for _ in range(2))
+    v = rng.standard_normal((1, 2, F * L, 5)).astype(np.float32)
+    full = oracle.softmax_window(q, k, v, F=F, L=L, W=3)
+    part = oracle.softmax_window(q, k, v, F=F, L=L, W=3, frames=[1, 4])
+    for f in range(F):
+        sl = slice(f * L, (f + 1) * L)
+        if f in (1, 4):
+            np.testing.assert_array_equal(part[:, :, sl], full[:, :, sl])
+        else:
+            assert np.isnan(part[:, :, sl]).all()
+    # permuting the tokens inside every frame permutes the outputs the same way
+    perm = np.concatenate([f * L + rng.permutation(L) for f in range(F)])
+    outp = oracle.softmax_window(q[:, :, perm], k[:, :, perm], v[:, :, perm], F=F, L=L, W=3)
+    np.testing.assert_allclose(outp, full[:, :, perm], rtol=1e-12, atol=1e-13)
+
+
 # ---------------------------------------------------------------- ReLU mode
 
 def _quadratic_masked_attention(q, k, v, F, L, eps):
