@@ -36,6 +36,7 @@ METRIC = "GDN frame-recurrence tokens/s (720p-60s shape, bf16) and % of roofline
 WORKLOAD = "gdn_720p_60s"
 FALLBACK_HBM_GBS = 6650.0
 SPEC_HBM_GBS = 8000.0  # B200 HBM3e figure quoted as "about 8 TB/s"
+FALLBACK_BF16_TFLOPS = 1590.0  # dense bf16 GEMM (burst) measured earlier on this machine
 # algorithmic bytes per token-head: q, k, v bf16 (3 * 112 * 2) + o fp32 (112 * 4) + beta fp32
 BYTES_PER_TOKEN_HEAD = 3 * 112 * 2 + 112 * 4 + 4
 FLOPS_PER_TOKEN_HEAD = 6 * 112 * 112
@@ -57,7 +58,7 @@ def parse():
                     help="use only the first N latent frames (a smaller case of the same kernel, for profiling)")
     ap.add_argument("--quick", action="store_true",
                     help="kernel leg only: no end-to-end leg, no ReLU-mode line, no CPU baseline")
-    ap.add_argument("--profile-case", choices=["gdn", "relu", "tconv", "stream"], default=None,
+    ap.add_argument("--profile-case", choices=["gdn", "relu", "tconv", "stream", "swa"], default=None,
                     help="run three launches of one kernel on a small case (inputs larger than L2, under 1 GB) "
                          "and exit: the command profiled with ncu --set full")
     return ap.parse_args()
@@ -86,6 +87,11 @@ def profile_case(name: str):
         x = synth.inputs(w)
         q, k, v = (torch.from_numpy(x[n]).to(torch.bfloat16).to(dev) for n in "qkv")
         call = lambda: lib.relu_la_block_fwd(q, k, v, F=w.F)
+    elif name == "swa":  # windowed softmax layer, first 24 of the 240 frames, W = 4
+        F, L, d = 24, 920, 112
+        q, k, v = (torch.from_numpy(synth.normal(7, t, 0, 20 * F * L * d).reshape(1, 20, F * L, d))
+                   .to(torch.bfloat16).to(dev) for t in range(3))
+        call = lambda: lib.softmax_window_fwd(q, k, v, F=F, W=4)
     else:
         cw = synth.CONV_WORKLOADS["tconv_720p_60s"]
         inp = synth.conv_inputs(cw, frames=60)
@@ -333,6 +339,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
             extra["streaming"] = streaming_leg(args, lib, synth, torch, dev, stream, cpu_on)
         extra["configs_other"] = small_configs_leg(args, lib, synth, torch, dev, stream, cpu_on)
         extra["temporal_conv"] = temporal_conv_leg(args, lib, synth, torch, dev, stream, cpu_on)
+        extra["softmax_window"] = softmax_window_leg(args, lib, synth, torch, dev, stream, cpu_on)
     peak, peak_src = measured_peaks()
     alg_bytes = token_heads * BYTES_PER_TOKEN_HEAD + w.B * w.H * (w.F * 4 + w.dk * w.dv * 4)
     achieved = alg_bytes / (ms / 1e3) / 1e9
@@ -657,6 +664,55 @@ def temporal_conv_leg(args, lib, synth, torch, dev, stream, cpu_baseline_on):
                                "cores": 1, "kind": "oracle",
                                "sample": f"one block of {sw.F} frames x {n_pos} of {sw.HW} latent positions, "
                                          f"{runs} runs in {secs:.1f} s"}
+    return out
+
+
+def softmax_window_leg(args, lib, synth, torch, dev, stream, cpu_baseline_on):
+    """The windowed softmax layer at the 720p 60 s shape (B=1, H=20, F=240, L=920,
+    d=112, bf16), window W = 4 latent frames (the current one and three before:
+    about one second of the clip).  Bound: tensor cores."""
+    B, H, F, L, d, W = 1, 20, 240, 920, 112, 4
+    N = F * L
+    q, k, v = (torch.from_numpy(synth.normal(7, t, 0, B * H * N * d).reshape(B, H, N, d)).to(torch.bfloat16).to(dev)
+               for t in range(3))
+    o = torch.empty((B, H, N, d), dtype=torch.float32, device=dev)
+    call = lambda: lib.softmax_window_fwd(q, k, v, F=F, W=W, o=o)
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    ms = _events_ms(call, 5, stream)
+    keys = sum(min(f + 1, W) * L for f in range(F))  # keys seen by one query row, summed over a head's frames
+    flops = 4.0 * d * B * H * L * keys               # q.k and p.v, 2 flops per multiply-add
+    tf = flops / (ms / 1e3) / 1e12
+    peak = FALLBACK_BF16_TFLOPS
+    mp = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    src = "fallback bf16_tflops (burst)"
+    if os.path.exists(mp):
+        try:
+            with open(mp) as f:
+                peak = float(json.load(f)["bf16_tflops"])
+            src = "measured bf16_tflops (burst)"
+        except Exception:
+            pass
+    out = {"workload": "swa_720p_60s_w4", "B": B, "H": H, "F": F, "L": L, "d": d, "W": W, "ms": ms,
+           "tokens_per_s": B * N / (ms / 1e3),
+           "roofline": {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
+                        "peak_source": src, "alg_flops_per_launch": flops},
+           "l2": "q, k, v 1.48 GB and o 1.98 GB, larger than L2; no flush needed"}
+    del q, k, v, o
+    if cpu_baseline_on:
+        import oracle
+        Fs = 5  # the first five frames of every head (frames 0-3 fill the window)
+        def head_prefix(t):  # frames 0..Fs-1 of every head: one contiguous run of the draw per head
+            x = np.stack([synth.normal(7, t, h * N * d, Fs * L * d) for h in range(H)]).reshape(B, H, Fs * L, d)
+            return torch.from_numpy(x).to(torch.bfloat16).float().numpy()
+        qs, ks, vs = (head_prefix(t) for t in range(3))
+        nthreads = os.cpu_count() or 1
+        tps, runs, secs = _oracle_tokens_per_s(
+            lambda: oracle.softmax_window(qs, ks, vs, F=Fs, L=L, W=W, nthreads=nthreads), B * Fs * L, target_s=4.0)
+        out["cpu_baseline"] = {"value": tps, "unit": "tokens/s", "cores": nthreads, "kind": "oracle",
+                               "sample": f"all {H} heads x first {Fs} of {F} frames (windows of 1-4 frames, "
+                                         f"below the 4-frame average), {runs} runs in {secs:.1f} s"}
     return out
 
 

@@ -56,7 +56,7 @@ extern "C" {
 #define GDN_API
 #endif
 
-#define GDN_ABI_VERSION 5
+#define GDN_ABI_VERSION 6
 
 /* return / status codes */
 #define GDN_OK 0
@@ -221,6 +221,33 @@ GDN_API int relu_la_block_fwd(const void *q, const void *k, const void *v, const
  */
 GDN_API int temporal_conv_fwd(const void *x, const float *w, const float *bias, const void *cache_in,
                               void *cache_out, void *y, int B, int F, int HW, int C, const gdn_opts_t *opts);
+
+/*
+ * softmax_window_fwd -- windowed block-causal softmax attention.
+ *
+ * SANA-WM's hybrid transformer interleaves the frame-wise Gated DeltaNet with
+ * softmax attention layers ("SANA-WM, an open-source 2.6B world model for
+ * 1-minute 720p video", GeekNews, "Core design and generation pipeline":
+ * periodic softmax; the Vietnamese post on SANA-WM: softmax windows between
+ * the Gated DeltaNet layers keep long rollouts coherent; the SANA-Video talk:
+ * minute-long video needs softmax kept inside a sliding window).  The pages
+ * give no window shape; this library's reading, per head (b, h): token t of
+ * frame f attends to every token of frames max(0, f-W+1) .. f (its own frame
+ * in full, block-causal like the linear modes),
+ *
+ *   o_t = sum_s softmax_s(scale * q_t . k_s) v_s,   scale = 1/sqrt(dk) if 0.
+ *
+ * q, k: [B, H, F*L, dk]; v: [B, H, F*L, dv] (opts->in_dtype must be
+ * GDN_DTYPE_BF16); o: [B, H, F*L, dv] float32, not overlapping the inputs.
+ * dk, dv multiples of 16 up to 128; W >= 1 (W >= F: all earlier frames).
+ * The scores are formed on tensor cores from the bf16 inputs with fp32
+ * accumulation; the probabilities and v enter the second product as fp16
+ * (11-bit significands), |v| < 65504 (GDN_ERR_RANGE otherwise), and o is
+ * accumulated in fp32.  Options used: in_dtype, stream, status,
+ * spin_limit_us; no workspace.  Returns GDN_OK or GDN_ERR_*.
+ */
+GDN_API int softmax_window_fwd(const void *q, const void *k, const void *v, float *o, int B, int H, int F, int L,
+                               int dk, int dv, int W, float scale, const gdn_opts_t *opts);
 
 /*
  * gdn_frame_fwd_host -- gdn_frame_fwd with HOST tensors.

@@ -32,7 +32,7 @@ IMPLS = {"auto": IMPL_AUTO, "seq": IMPL_SEQ, "frame_simt": IMPL_FRAME_SIMT, "tc"
 
 EXPORTED = ("gdn_frame_fwd", "relu_la_block_fwd", "gdn_frame_fwd_host", "gdn_frame_fwd_noalloc",
             "gdn_workspace_bytes", "gdn_workspace_bytes_host", "gdn_status_string", "gdn_status_str",
-            "gdn_abi_version", "temporal_conv_fwd")
+            "gdn_abi_version", "temporal_conv_fwd", "softmax_window_fwd")
 NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
 
 
@@ -56,6 +56,8 @@ _lib.relu_la_block_fwd.argtypes = [_P] * 8 + [_I] * 6 + [ctypes.c_float, ctypes.
 _lib.relu_la_block_fwd.restype = _I
 _lib.temporal_conv_fwd.argtypes = [_P] * 6 + [_I] * 4 + [ctypes.POINTER(GdnOpts)]
 _lib.temporal_conv_fwd.restype = _I
+_lib.softmax_window_fwd.argtypes = [_P] * 4 + [_I] * 7 + [ctypes.c_float, ctypes.POINTER(GdnOpts)]
+_lib.softmax_window_fwd.restype = _I
 _lib.gdn_workspace_bytes.argtypes = [_I] * 7 + [ctypes.POINTER(GdnOpts)]
 _lib.gdn_workspace_bytes.restype = ctypes.c_size_t
 _lib.gdn_workspace_bytes_host.argtypes = [_I] * 6 + [ctypes.POINTER(GdnOpts)]
@@ -245,6 +247,31 @@ def temporal_conv_fwd(x, w, *, bias=None, cache_in=None, cache_out=None, y=None,
     if rc != OK:
         raise GdnError(rc, "temporal_conv_fwd")
     return y
+
+
+def softmax_window_fwd(q, k, v, *, F: int, W: int, scale: float = 0.0, o=None, stream=None, status=None,
+                       spin_limit_us: int = 0):
+    """Windowed block-causal softmax attention on the GPU (see include/gdn_b200.h):
+    q, k [B, H, F*L, dk] and v [B, H, F*L, dv] bfloat16; token t of frame f attends
+    to frames max(0, f-W+1) .. f.  Returns o [B, H, F*L, dv] float32."""
+    B, H, N, dk = q.shape
+    dv = v.shape[-1]
+    if N % F:
+        raise ValueError(f"token count {N} is not a multiple of F={F}")
+    L = N // F
+    dev = q.device
+    _check(q, "q", (B, H, N, dk), q.dtype, dev)
+    _check(k, "k", (B, H, N, dk), q.dtype, dev)
+    _check(v, "v", (B, H, N, dv), q.dtype, dev)
+    if o is None:
+        o = torch.empty((B, H, N, dv), dtype=torch.float32, device=dev)
+    _check(o, "o", (B, H, N, dv), torch.float32, dev)
+    opts = make_opts(_dtype_code(q), stream=stream, status=status, spin_limit_us=spin_limit_us)
+    rc = _lib.softmax_window_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, H, F, L, dk, dv, int(W), float(scale),
+                                 ctypes.byref(opts))
+    if rc != OK:
+        raise GdnError(rc, "softmax_window_fwd")
+    return o
 
 
 def gdn_frame_fwd_host(q, k, v, alpha, beta, *, F: int, o, state_in=None, state_out=None,

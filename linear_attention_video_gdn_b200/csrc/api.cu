@@ -351,6 +351,32 @@ extern "C" int temporal_conv_fwd(const void *x, const float *w, const float *bia
   return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
+extern "C" int softmax_window_fwd(const void *q, const void *k, const void *v, float *o, int B, int H, int F, int L,
+                                  int dk, int dv, int W, float scale, const gdn_opts_t *opts) {
+  using namespace gdn;
+  if (!opts || !q || !k || !v || !o) return GDN_ERR_INVALID_ARG;
+  if (opts->in_dtype != GDN_DTYPE_F32 && opts->in_dtype != GDN_DTYPE_BF16) return GDN_ERR_INVALID_ARG;
+  if (W < 1 || !(scale >= 0.0f)) return GDN_ERR_INVALID_ARG;
+  int rc = check_sizes(B, H, F, L, dk, dv);
+  if (rc != GDN_OK) return rc;
+  if (opts->in_dtype != GDN_DTYPE_BF16 || !softmax_window_supported(dk, dv)) return GDN_ERR_UNSUPPORTED;
+  const void *ptrs[] = {q, k, v, o, opts->status};
+  for (const void *ptr : ptrs)
+    if (!aligned16(ptr)) return GDN_ERR_INVALID_ARG;
+  const size_t N = (size_t)B * H * F * L;
+  if (overlap(o, N * dv * 4, q, N * dk * 2) || overlap(o, N * dv * 4, k, N * dk * 2) ||
+      overlap(o, N * dv * 4, v, N * dv * 2))
+    return GDN_ERR_INVALID_ARG;
+  int sms = 0, cc = 0;
+  rc = device_info(&sms, &cc);
+  if (rc != GDN_OK) return rc;
+  if (cc != 100) return GDN_ERR_NO_DEVICE;
+  const float sc = scale > 0.0f ? scale : 1.0f / sqrtf((float)dk);
+  const cudaError_t e = launch_softmax_window(q, k, v, o, B, H, F, L, dk, dv, W, sc, opts->status, spin_ns(opts),
+                                              (cudaStream_t)opts->stream);
+  return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
 // ---------------------------------------------------------------- host I/O
 //
 // gdn_frame_fwd_host streams the sequence through the device in groups of

@@ -25,6 +25,11 @@ cudaError_t launch_gdn_pform(const GdnParams &p, int grid, cudaStream_t st);
 cudaError_t launch_temporal_conv(const void *x, const float *w, const float *bias, const void *cache_in,
                                  void *cache_out, void *y, int B, int F, int HW, int C, int in_dtype, int max_ctas,
                                  cudaStream_t st);
+// windowed block-causal softmax attention (bf16 q, k, v on tcgen05; fp32 o)
+bool softmax_window_supported(int dk, int dv);
+cudaError_t launch_softmax_window(const void *q, const void *k, const void *v, float *o, int B, int H, int F, int L,
+                                  int dk, int dv, int W, float scale, int *status, unsigned long long spin_limit_ns,
+                                  cudaStream_t st);
 bool relu_tc_supported(int dk, int dv);
 cudaError_t launch_relu_tc(const ReluParams &p, int grid, cudaStream_t st);
 
