@@ -120,7 +120,7 @@ def measured_peaks():
 KERNEL_SOURCES = {
     "gdn_tc": ("gdn_tc.cu", "tc_ptx.cuh", "common.cuh"),
     "relu_tc": ("relu_tc.cu", "tc_ptx.cuh", "common.cuh"),
-    "temporal_conv": ("temporal_conv.cu", "tc_ptx.cuh", "common.cuh"),
+    "temporal_conv": ("temporal_conv.cu", "f32x2.cuh", "tc_ptx.cuh", "common.cuh"),
 }
 
 

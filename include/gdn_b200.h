@@ -241,8 +241,8 @@ GDN_API int temporal_conv_fwd(const void *x, const float *w, const float *bias, 
  * GDN_DTYPE_BF16); o: [B, H, F*L, dv] float32, not overlapping the inputs.
  * dk, dv multiples of 16 up to 128; W >= 1 (W >= F: all earlier frames).
  * The scores are formed on tensor cores from the bf16 inputs with fp32
- * accumulation; the probabilities and v enter the second product as fp16
- * (11-bit significands), |v| < 65504 (GDN_ERR_RANGE otherwise), and o is
+ * accumulation; the probabilities enter the second product as bf16 high and
+ * low parts (about 16 significant bits) against v as given, and o is
  * accumulated in fp32.  Options used: in_dtype, stream, status,
  * spin_limit_us; no workspace.  Returns GDN_OK or GDN_ERR_*.
  */

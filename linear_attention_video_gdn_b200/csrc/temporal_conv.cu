@@ -23,6 +23,7 @@
 // other CTAs' transfers.
 #include <cuda_bf16.h>
 
+#include "f32x2.cuh"
 #include "launch.h"
 #include "tc_ptx.cuh"
 
@@ -35,15 +36,6 @@ constexpr int kAhead = 4;  // frames loaded ahead per step (single-element colum
 // frames prefetched per thread into shared memory (16-byte columns): deeper
 // where fewer CTAs fit an SM (bf16 columns hold more registers)
 template <int V> __host__ __device__ constexpr int ring_depth() { return V == 8 ? 12 : 8; }
-
-__device__ __forceinline__ uint64_t pack2(uint32_t lo, uint32_t hi) { return ((uint64_t)hi << 32) | lo; }
-
-// Two fp32 fused multiply-adds in one instruction (each lane rounded as fmaf).
-__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
 
 // A vector of V channels as it sits in memory (Raw) and in registers (float[V]).
 template <typename T, int V> struct Col;
