@@ -121,6 +121,7 @@ KERNEL_SOURCES = {
     "gdn_tc": ("gdn_tc.cu", "tc_ptx.cuh", "common.cuh"),
     "relu_tc": ("relu_tc.cu", "tc_ptx.cuh", "common.cuh"),
     "temporal_conv": ("temporal_conv.cu", "f32x2.cuh", "tc_ptx.cuh", "common.cuh"),
+    "softmax_window": ("softmax_window.cu", "f32x2.cuh", "tc_ptx.cuh", "common.cuh"),
 }
 
 
@@ -697,7 +698,9 @@ def softmax_window_leg(args, lib, synth, torch, dev, stream, cpu_baseline_on):
     out = {"workload": "swa_720p_60s_w4", "B": B, "H": H, "F": F, "L": L, "d": d, "W": W, "ms": ms,
            "tokens_per_s": B * N / (ms / 1e3),
            "roofline": {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
-                        "peak_source": src, "alg_flops_per_launch": flops},
+                        "peak_source": src, "alg_flops_per_launch": flops,
+                        "traffic": None if ncu_traffic("softmax_window") is None
+                        else ncu_traffic("softmax_window")["dram_bytes_per_launch"]},
            "l2": "q, k, v 1.48 GB and o 1.98 GB, larger than L2; no flush needed"}
     del q, k, v, o
     if cpu_baseline_on:
