@@ -237,14 +237,16 @@ GDN_API int temporal_conv_fwd(const void *x, const float *w, const float *bias, 
  *
  *   o_t = sum_s softmax_s(scale * q_t . k_s) v_s,   scale = 1/sqrt(dk) if 0.
  *
- * q, k: [B, H, F*L, dk]; v: [B, H, F*L, dv] (opts->in_dtype must be
- * GDN_DTYPE_BF16); o: [B, H, F*L, dv] float32, not overlapping the inputs.
- * dk, dv multiples of 16 up to 128; W >= 1 (W >= F: all earlier frames).
- * The scores are formed on tensor cores from the bf16 inputs with fp32
- * accumulation; the probabilities enter the second product as bf16 high and
- * low parts (about 16 significant bits) against v as given, and o is
- * accumulated in fp32.  Options used: in_dtype, stream, status,
- * spin_limit_us; no workspace.  Returns GDN_OK or GDN_ERR_*.
+ * q, k: [B, H, F*L, dk]; v: [B, H, F*L, dv] (element type opts->in_dtype);
+ * o: [B, H, F*L, dv] float32, not overlapping the inputs.  dk, dv <= 128;
+ * W >= 1 (W >= F: all earlier frames).  Kernels (opts->impl): GDN_IMPL_TC
+ * (bf16 inputs, dk and dv multiples of 16) forms the scores on tensor cores
+ * with fp32 accumulation and feeds the probabilities to the second product as
+ * bf16 high and low parts (about 16 significant bits) against v as given, o
+ * accumulated in fp32; GDN_IMPL_FRAME_SIMT runs in fp32 on CUDA cores (any
+ * shape, fp32 or bf16 inputs); GDN_IMPL_AUTO takes the tensor cores when they
+ * apply.  Options used: in_dtype, impl, stream, status, spin_limit_us; no
+ * workspace.  Returns GDN_OK or GDN_ERR_*.
  */
 GDN_API int softmax_window_fwd(const void *q, const void *k, const void *v, float *o, int B, int H, int F, int L,
                                int dk, int dv, int W, float scale, const gdn_opts_t *opts);

@@ -249,11 +249,11 @@ def temporal_conv_fwd(x, w, *, bias=None, cache_in=None, cache_out=None, y=None,
     return y
 
 
-def softmax_window_fwd(q, k, v, *, F: int, W: int, scale: float = 0.0, o=None, stream=None, status=None,
-                       spin_limit_us: int = 0):
+def softmax_window_fwd(q, k, v, *, F: int, W: int, scale: float = 0.0, o=None, impl="auto", stream=None,
+                       status=None, spin_limit_us: int = 0):
     """Windowed block-causal softmax attention on the GPU (see include/gdn_b200.h):
-    q, k [B, H, F*L, dk] and v [B, H, F*L, dv] bfloat16; token t of frame f attends
-    to frames max(0, f-W+1) .. f.  Returns o [B, H, F*L, dv] float32."""
+    q, k [B, H, F*L, dk] and v [B, H, F*L, dv] bfloat16 or float32; token t of
+    frame f attends to frames max(0, f-W+1) .. f.  Returns o [B, H, F*L, dv] float32."""
     B, H, N, dk = q.shape
     dv = v.shape[-1]
     if N % F:
@@ -266,7 +266,7 @@ def softmax_window_fwd(q, k, v, *, F: int, W: int, scale: float = 0.0, o=None, s
     if o is None:
         o = torch.empty((B, H, N, dv), dtype=torch.float32, device=dev)
     _check(o, "o", (B, H, N, dv), torch.float32, dev)
-    opts = make_opts(_dtype_code(q), stream=stream, status=status, spin_limit_us=spin_limit_us)
+    opts = make_opts(_dtype_code(q), impl=impl, stream=stream, status=status, spin_limit_us=spin_limit_us)
     rc = _lib.softmax_window_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, H, F, L, dk, dv, int(W), float(scale),
                                  ctypes.byref(opts))
     if rc != OK:

@@ -359,21 +359,28 @@ extern "C" int softmax_window_fwd(const void *q, const void *k, const void *v, f
   if (W < 1 || !(scale >= 0.0f)) return GDN_ERR_INVALID_ARG;
   int rc = check_sizes(B, H, F, L, dk, dv);
   if (rc != GDN_OK) return rc;
-  if (opts->in_dtype != GDN_DTYPE_BF16 || !softmax_window_supported(dk, dv)) return GDN_ERR_UNSUPPORTED;
+  if (opts->impl != GDN_IMPL_AUTO && opts->impl != GDN_IMPL_FRAME_SIMT && opts->impl != GDN_IMPL_TC)
+    return GDN_ERR_INVALID_ARG;
+  const bool tc_ok = opts->in_dtype == GDN_DTYPE_BF16 && softmax_window_supported(dk, dv);
+  if (opts->impl == GDN_IMPL_TC && !tc_ok) return GDN_ERR_UNSUPPORTED;
+  const bool use_tc = tc_ok && opts->impl != GDN_IMPL_FRAME_SIMT;
   const void *ptrs[] = {q, k, v, o, opts->status};
   for (const void *ptr : ptrs)
     if (!aligned16(ptr)) return GDN_ERR_INVALID_ARG;
-  const size_t N = (size_t)B * H * F * L;
-  if (overlap(o, N * dv * 4, q, N * dk * 2) || overlap(o, N * dv * 4, k, N * dk * 2) ||
-      overlap(o, N * dv * 4, v, N * dv * 2))
+  const size_t N = (size_t)B * H * F * L, es = opts->in_dtype == GDN_DTYPE_BF16 ? 2 : 4;
+  if (overlap(o, N * dv * 4, q, N * dk * es) || overlap(o, N * dv * 4, k, N * dk * es) ||
+      overlap(o, N * dv * 4, v, N * dv * es))
     return GDN_ERR_INVALID_ARG;
   int sms = 0, cc = 0;
   rc = device_info(&sms, &cc);
   if (rc != GDN_OK) return rc;
   if (cc != 100) return GDN_ERR_NO_DEVICE;
   const float sc = scale > 0.0f ? scale : 1.0f / sqrtf((float)dk);
-  const cudaError_t e = launch_softmax_window(q, k, v, o, B, H, F, L, dk, dv, W, sc, opts->status, spin_ns(opts),
-                                              (cudaStream_t)opts->stream);
+  const cudaError_t e =
+      use_tc ? launch_softmax_window(q, k, v, o, B, H, F, L, dk, dv, W, sc, opts->status, spin_ns(opts),
+                                     (cudaStream_t)opts->stream)
+             : launch_softmax_window_simt(q, k, v, o, B, H, F, L, dk, dv, W, sc, opts->in_dtype,
+                                          (cudaStream_t)opts->stream);
   return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 

@@ -111,12 +111,27 @@ def test_large_values_and_refusals(lib, dev):
     o = lib.softmax_window_fwd(q, k, big, F=3, W=2)
     torch.cuda.synchronize()
     assert rel_err(o.cpu().numpy(), oracle.softmax_window(qh, kh, big.float().cpu().numpy(), F=3, L=40, W=2)) <= TOL
-    with pytest.raises(lib.GdnError) as e:  # fp32 inputs: tensor-core path only
-        lib.softmax_window_fwd(q.float(), k.float(), v.float(), F=3, W=1)
+    with pytest.raises(lib.GdnError) as e:  # the tensor-core kernel takes bf16 only
+        lib.softmax_window_fwd(q.float(), k.float(), v.float(), F=3, W=1, impl="tc")
     assert e.value.code == lib.ERR_UNSUPPORTED
-    with pytest.raises(lib.GdnError) as e:  # d not a multiple of 16
-        lib.softmax_window_fwd(q[..., :24].contiguous(), k[..., :24].contiguous(), v, F=3, W=1)
+    with pytest.raises(lib.GdnError) as e:  # ... and d a multiple of 16
+        lib.softmax_window_fwd(q[..., :24].contiguous(), k[..., :24].contiguous(), v, F=3, W=1, impl="tc")
     assert e.value.code == lib.ERR_UNSUPPORTED
     with pytest.raises(lib.GdnError) as e:
         lib.softmax_window_fwd(q, k, v, F=3, W=0)
     assert e.value.code == lib.ERR_INVALID_ARG
+
+
+# fp32 inputs (CUDA cores, bar 1e-5) and bf16 shapes the tensor cores do not take
+@pytest.mark.parametrize("B,H,F,L,dk,dv,W,dtype", [(1, 2, 3, 37, 32, 32, 2, "f32"), (2, 1, 5, 20, 24, 40, 3, "f32"),
+                                                   (1, 1, 4, 9, 128, 100, 10, "f32"), (1, 2, 3, 50, 24, 24, 2, "bf16"),
+                                                   (1, 2, 3, 64, 64, 64, 2, "bf16")])
+def test_cuda_core_path(lib, dev, B, H, F, L, dk, dv, W, dtype):
+    N = F * L
+    x = [synth.normal(70 + L, t, 0, B * H * N * d).reshape(B, H, N, d) for t, d in enumerate((dk, dk, dv))]
+    dt = torch.float32 if dtype == "f32" else torch.bfloat16
+    q, k, v = (torch.from_numpy(a).to(dt).to(dev) for a in x)
+    o = lib.softmax_window_fwd(q, k, v, F=F, W=W, impl="frame_simt")
+    torch.cuda.synchronize()
+    ref = oracle.softmax_window(*(t.float().cpu().numpy() for t in (q, k, v)), F=F, L=L, W=W)
+    assert rel_err(o.cpu().numpy(), ref) <= (1e-5 if dtype == "f32" else TOL)
