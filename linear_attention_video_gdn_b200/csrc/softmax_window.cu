@@ -94,6 +94,47 @@ __device__ __forceinline__ KeyTile key_tile(int j, int f0, int tpf, int L) {
   return t;
 }
 
+// Maximum of the raw scores over the first nvalid keys (kFull: all 64), four
+// partial maxima to shorten the dependent chain.
+template <bool kFull>
+__device__ __forceinline__ float tile_max(const float (&sc)[kKeys], int nvalid) {
+  float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+  for (int c = 0; c < kKeys; ++c)
+    if (kFull || c < nvalid) mx[c & 3] = fmaxf(mx[c & 3], sc[c]);
+  return fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+}
+
+// p = exp2(s * c - m) over the row's 64 keys (zero past nvalid), written to the
+// K-major P tiles as bf16 high and low parts 8 keys at a time; returns the sum.
+template <bool kFull>
+__device__ __forceinline__ float tile_exp(const float (&sc)[kKeys], int nvalid, float c, float m, int row,
+                                          uint8_t *p_hi, uint8_t *p_lo) {
+  const uint64_t c2 = pack2(__float_as_uint(c), __float_as_uint(c));
+  const uint64_t nm2 = pack2(__float_as_uint(-m), __float_as_uint(-m));
+  float rs[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+  for (int c8 = 0; c8 < kKeys / 8; ++c8) {
+    uint32_t hi[4], lo[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int k0 = c8 * 8 + 2 * e;
+      const uint64_t arg = fma2(pack2(__float_as_uint(sc[k0]), __float_as_uint(sc[k0 + 1])), c2, nm2);
+      float p0 = ex2(__uint_as_float((uint32_t)arg)), p1 = ex2(__uint_as_float((uint32_t)(arg >> 32)));
+      if (!kFull) {
+        p0 = k0 < nvalid ? p0 : 0.0f;
+        p1 = k0 + 1 < nvalid ? p1 : 0.0f;
+      }
+      rs[e] += p0 + p1;
+      split_bf16x2(p0, p1, hi[e], lo[e]);
+    }
+    const uint32_t off = sw128_offset((uint32_t)row, (uint32_t)(c8 * 8));
+    *reinterpret_cast<uint4 *>(p_hi + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+    *reinterpret_cast<uint4 *>(p_lo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+  }
+  return (rs[0] + rs[1]) + (rs[2] + rs[3]);
+}
+
 struct SwParams {
   float *o;
   int BH, F, L, dk, dv, W;
@@ -262,12 +303,9 @@ __global__ void __launch_bounds__(kSwThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_only(&sm.s_free[x][b]);  // this warp's rows of S buffer b are read
-      // the maximum of the raw scores over the keys inside the frame
-      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-      for (int c = 0; c < kKeys; ++c)
-        if (c < t.valid) mx[c & 3] = fmaxf(mx[c & 3], sc[c]);
-      const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * p.scale_log2;
+      // the maximum of the raw scores over the keys inside the frame (most tiles are full)
+      const bool full = t.valid == kKeys;
+      const float mt = (full ? tile_max<true>(sc, kKeys) : tile_max<false>(sc, t.valid)) * p.scale_log2;
       // P_x (one buffer) and O_x: the previous key tile's PV MMAs must be done
       bad = j >= 1 && !mbar_wait(&sm.o_done[x], (uint32_t)(j - 1) & 1u, lim);
       // move the running maximum only when this tile exceeds it by more than 2^kRescale;
@@ -292,26 +330,8 @@ __global__ void __launch_bounds__(kSwThreads, 1)
         m = m_new;
       }
       // p = exp2(s * scale_log2 - m), written 8 keys at a time as bf16 high and low parts
-      const uint64_t c2 = pack2(__float_as_uint(p.scale_log2), __float_as_uint(p.scale_log2));
-      const uint64_t nm2 = pack2(__float_as_uint(-m), __float_as_uint(-m));
-      float rs[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll
-      for (int c8 = 0; c8 < kKeys / 8; ++c8) {
-        uint32_t hi[4], lo[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int c = c8 * 8 + 2 * e;
-          const uint64_t arg = fma2(pack2(__float_as_uint(sc[c]), __float_as_uint(sc[c + 1])), c2, nm2);
-          const float p0 = c < t.valid ? ex2(__uint_as_float((uint32_t)arg)) : 0.0f;
-          const float p1 = c + 1 < t.valid ? ex2(__uint_as_float((uint32_t)(arg >> 32))) : 0.0f;
-          rs[e] += p0 + p1;
-          split_bf16x2(p0, p1, hi[e], lo[e]);
-        }
-        const uint32_t off = sw128_offset((uint32_t)row, (uint32_t)(c8 * 8));
-        *reinterpret_cast<uint4 *>(sm.p[x][0] + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-        *reinterpret_cast<uint4 *>(sm.p[x][1] + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-      }
-      l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
+      l += full ? tile_exp<true>(sc, kKeys, p.scale_log2, m, row, sm.p[x][0], sm.p[x][1])
+                : tile_exp<false>(sc, t.valid, p.scale_log2, m, row, sm.p[x][0], sm.p[x][1]);
       fence_async_smem();
       tc_fence_before();
       if (bar_sync_or(hb, 128, bad)) { failed = true; break; }
