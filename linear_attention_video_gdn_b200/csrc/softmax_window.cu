@@ -52,7 +52,7 @@ struct __align__(1024) SwSmem {
   uint64_t v_empty[kRing];   // both query tiles' PV MMAs reading the V half have completed
   uint64_t s_full[2][2];     // [X][b]: S buffer b of tile X holds its scores
   uint64_t s_free[2][2];     // [X][b]: tile X's four softmax warps have read it
-  uint64_t p_full[2];        // [X]: P_X holds the current key tile's probabilities
+  uint64_t p_full[2];        // [X]: P_X holds the current key tile's probabilities (one arrival per warp)
   uint64_t o_done[2];        // [X]: the PV MMAs of tile X's latest key tile have completed
   uint64_t fin;              // every MMA of the CTA has completed (teardown)
   uint32_t tmem_base;
@@ -174,7 +174,7 @@ __global__ void __launch_bounds__(kSwThreads, 1)
         mbar_init(&sm.s_full[x][b], 1);
         mbar_init(&sm.s_free[x][b], 4);  // one arrival per softmax warp of the tile
       }
-      mbar_init(&sm.p_full[x], 1);
+      mbar_init(&sm.p_full[x], 4);
       mbar_init(&sm.o_done[x], 1);
     }
     mbar_init(&sm.fin, 2);
@@ -284,7 +284,6 @@ __global__ void __launch_bounds__(kSwThreads, 1)
     // ---------------- softmax: query tile x = warp / 4, one query row per thread ----------------
     const int x = warp >> 2, quarter = warp & 3;
     const int row = quarter * 32 + lane;
-    const int hb = 1 + x;  // the tile's named barrier
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const int qrow = (2 * qp + x) * kQRows + row;
     float m = -INFINITY, l = 0.0f;  // running maximum (exp2 units) and row sum
@@ -292,8 +291,9 @@ __global__ void __launch_bounds__(kSwThreads, 1)
     for (int j = 0; j < nt; ++j) {
       const int b = j & 1;
       const KeyTile t = key_tile(j, f0, tpf, L);
+      // each warp runs its own rows: mbarriers only, no barrier with the tile's other warps
       int bad = !mbar_wait(&sm.s_full[x][b], (uint32_t)(j >> 1) & 1u, lim);
-      if (bar_sync_or(hb, 128, bad)) { failed = true; break; }
+      if (__any_sync(0xffffffffu, bad)) { failed = true; break; }
       tc_fence_after();
       float sc[kKeys];
 #pragma unroll
@@ -334,12 +334,12 @@ __global__ void __launch_bounds__(kSwThreads, 1)
                 : tile_exp<false>(sc, t.valid, p.scale_log2, m, row, sm.p[x][0], sm.p[x][1]);
       fence_async_smem();
       tc_fence_before();
-      if (bar_sync_or(hb, 128, bad)) { failed = true; break; }
-      if (row == 0) mbar_arrive_only(&sm.p_full[x]);
+      if (__any_sync(0xffffffffu, bad)) { failed = true; break; }
+      if (lane == 0) mbar_arrive_only(&sm.p_full[x]);  // this warp's rows of P_x are written
     }
     if (!failed && nt >= 1) {
       const int bad = !mbar_wait(&sm.o_done[x], (uint32_t)(nt - 1) & 1u, lim);
-      if (bar_sync_or(hb, 128, bad)) failed = true;
+      if (__any_sync(0xffffffffu, bad)) failed = true;
     }
     if (!failed) {
       tc_fence_after();
@@ -363,7 +363,7 @@ __global__ void __launch_bounds__(kSwThreads, 1)
           }
         }
       }
-    } else if (row == 0) {
+    } else if (lane == 0) {
       latch_status(p.status, GDN_ERR_TIMEOUT);
     }
   }
