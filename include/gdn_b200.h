@@ -241,8 +241,8 @@ GDN_API int temporal_conv_fwd(const void *x, const float *w, const float *bias, 
  * o: [B, H, F*L, dv] float32, not overlapping the inputs.  dk, dv <= 128;
  * W >= 1 (W >= F: all earlier frames).  Kernels (opts->impl): GDN_IMPL_TC
  * (bf16 inputs, dk and dv multiples of 16) forms the scores on tensor cores
- * with fp32 accumulation and feeds the probabilities to the second product as
- * bf16 high and low parts (about 16 significant bits) against v as given, o
+ * with fp32 accumulation and feeds the probabilities and v to the second
+ * product as fp16 (11-bit significands; |v| < 65504, else GDN_ERR_RANGE), o
  * accumulated in fp32; GDN_IMPL_FRAME_SIMT runs in fp32 on CUDA cores (any
  * shape, fp32 or bf16 inputs); GDN_IMPL_AUTO takes the tensor cores when they
  * apply.  Options used: in_dtype, impl, stream, status, spin_limit_us; no

@@ -16,10 +16,10 @@
 //   S_X = Q_X K^T     tcgen05, M=128 queries x N=64 keys, bf16 operands, into
 //                     one of two TMEM buffers of tile X;
 //   P_X = exp(S - m)  warps 4X .. 4X+3, one query row per thread, written to
-//                     shared memory as bf16 high and low parts (truncated
-//                     upper halves, about 16 significant bits);
-//   O_X += P_X V      tcgen05, M=128 x N=dv, two MMAs per 16 keys (high and low
-//                     parts against the bf16 V tile as loaded), fp32 in TMEM.
+//                     shared memory as fp16 (11-bit significands); warps
+//                     12-13 convert the V tile to fp16 in place (exact for
+//                     bf16 values inside the fp16 range);
+//   O_X += P_X V      tcgen05, M=128 x N=dv, fp16 operands, fp32 in TMEM.
 // While one query tile's warps exponentiate, the tensor pipe runs the other
 // tile's products.  The running maximum m moves only when a tile's maximum
 // exceeds it by more than 2^8 in exp2 units; then the row of O (in TMEM) and
@@ -35,21 +35,22 @@ namespace gdn {
 namespace tc {
 namespace {
 
-constexpr int kSwThreads = 384;  // warps 0-3: query tile 0; 4-7: query tile 1; 8-11: S, PV, K, V
+constexpr int kSwThreads = 448;  // warps 0-3: query tile 0; 4-7: query tile 1; 8-11: S, PV, K, V; 12-13: V to fp16
 constexpr int kQRows = 128;      // queries per query tile
 constexpr int kKeys = 64;        // keys per key tile
-constexpr int kRing = 3;         // K/V tiles in flight
+constexpr int kRing = 4;         // K/V tiles in flight
 constexpr uint32_t kHalfBytes = 16384;  // the K (or V) half of a ring slot: 64 keys x 2 atoms
 constexpr float kRescale = 8.0f;        // exp2 units the running maximum may lag behind
 
 struct __align__(1024) SwSmem {
   uint8_t q[2][2][16384];          // query tile X: two 64-column atoms of 128 rows (K-major A operand)
   uint8_t kv[kRing][2][16384];     // slot: K half, V half (64 keys x 2 atoms each)
-  uint8_t p[2][2][16384];          // query tile X, high / low part: bf16, 128 rows x 64 keys (K-major)
+  uint8_t p[2][16384];             // query tile X: fp16 probabilities, 128 rows x 64 keys (K-major)
   uint64_t q_full;
   uint64_t k_full[kRing], v_full[kRing];
   uint64_t k_empty[kRing];   // both query tiles' S MMAs reading the K half have completed
   uint64_t v_empty[kRing];   // both query tiles' PV MMAs reading the V half have completed
+  uint64_t v_conv[kRing];    // the V half has been converted to fp16 (one arrival per converting warp)
   uint64_t s_full[2][2];     // [X][b]: S buffer b of tile X holds its scores
   uint64_t s_free[2][2];     // [X][b]: tile X's four softmax warps have read it
   uint64_t p_full[2];        // [X]: P_X holds the current key tile's probabilities (one arrival per warp)
@@ -64,15 +65,10 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// Two values as bf16 high parts (the upper 16 bits) and bf16 low parts (the upper
-// 16 bits of what the high part leaves, formed exactly in fp32): about 16
-// significant bits in all, with integer and add instructions only, so the
-// conversion unit stays free for the exponentials.
-__device__ __forceinline__ void split_bf16x2(float a, float b, uint32_t &hi, uint32_t &lo) {
-  const uint32_t ua = __float_as_uint(a), ub = __float_as_uint(b);
-  const float ra = a - __uint_as_float(ua & 0xffff0000u), rb = b - __uint_as_float(ub & 0xffff0000u);
-  hi = __byte_perm(ua, ub, 0x7632);  // (b's upper half << 16) | a's upper half
-  lo = __byte_perm(__float_as_uint(ra), __float_as_uint(rb), 0x7632);
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
 }
 
 __device__ __forceinline__ void sw_st_v8(float *p, const float *v, float scale) {
@@ -106,16 +102,16 @@ __device__ __forceinline__ float tile_max(const float (&sc)[kKeys], int nvalid) 
 }
 
 // p = exp2(s * c - m) over the row's 64 keys (zero past nvalid), written to the
-// K-major P tiles as bf16 high and low parts 8 keys at a time; returns the sum.
+// K-major P tile as fp16 8 keys at a time; returns the sum.
 template <bool kFull>
 __device__ __forceinline__ float tile_exp(const float (&sc)[kKeys], int nvalid, float c, float m, int row,
-                                          uint8_t *p_hi, uint8_t *p_lo) {
+                                          uint8_t *p_tile) {
   const uint64_t c2 = pack2(__float_as_uint(c), __float_as_uint(c));
   const uint64_t nm2 = pack2(__float_as_uint(-m), __float_as_uint(-m));
   float rs[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
   for (int c8 = 0; c8 < kKeys / 8; ++c8) {
-    uint32_t hi[4], lo[4];
+    uint32_t h[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const int k0 = c8 * 8 + 2 * e;
@@ -126,11 +122,10 @@ __device__ __forceinline__ float tile_exp(const float (&sc)[kKeys], int nvalid, 
         p1 = k0 + 1 < nvalid ? p1 : 0.0f;
       }
       rs[e] += p0 + p1;
-      split_bf16x2(p0, p1, hi[e], lo[e]);
+      h[e] = pack_f16x2(p0, p1);
     }
     const uint32_t off = sw128_offset((uint32_t)row, (uint32_t)(c8 * 8));
-    *reinterpret_cast<uint4 *>(p_hi + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-    *reinterpret_cast<uint4 *>(p_lo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+    *reinterpret_cast<uint4 *>(p_tile + off) = make_uint4(h[0], h[1], h[2], h[3]);
   }
   return (rs[0] + rs[1]) + (rs[2] + rs[3]);
 }
@@ -168,6 +163,7 @@ __global__ void __launch_bounds__(kSwThreads, 1)
       mbar_init(&sm.v_full[s], 1);
       mbar_init(&sm.k_empty[s], 1);
       mbar_init(&sm.v_empty[s], 1);
+      mbar_init(&sm.v_conv[s], 2);
     }
     for (int x = 0; x < 2; ++x) {
       for (int b = 0; b < 2; ++b) {
@@ -192,7 +188,7 @@ __global__ void __launch_bounds__(kSwThreads, 1)
   auto tS = [&](int x, int b) { return tmem + (uint32_t)(x * 128 + b * 64); };
   auto tO = [&](int x) { return tmem + 256u + (uint32_t)(x * 128); };
 
-  if (warp >= 8) {
+  if (warp >= 8 && warp < 12) {
     // ---------------- one thread per role: S MMAs, PV MMAs, Q and K loads, V loads ----------------
     const bool lead = lane == 0;
     bool ok = true;
@@ -220,24 +216,21 @@ __global__ void __launch_bounds__(kSwThreads, 1)
         if (ok) mma_commit(&sm.k_empty[s]);
       }
       mma_commit(&sm.fin);  // TMEM is released only after every MMA of both issuers
-    } else if (warp == 9 && lead) {  // O_X += P_X V_j, high then low part of P
-      const uint32_t idesc_pv = idesc_f16(kQRows, dv, 1, 0, 1);  // bf16; P K-major, V MN-major
+    } else if (warp == 9 && lead) {  // O_X += P_X V_j
+      const uint32_t idesc_pv = idesc_f16(kQRows, dv, 0, 0, 1);  // fp16; P K-major, V MN-major
       for (int j = 0; j < nt && ok; ++j) {
         const int s = j % kRing;
-        ok = mbar_wait(&sm.v_full[s], (uint32_t)(j / kRing) & 1u, lim);
+        ok = mbar_wait(&sm.v_conv[s], (uint32_t)(j / kRing) & 1u, lim);
         const uint64_t vd = sdesc_sw128(smem_u32(sm.kv[s][1]), 8192, 1024);
         for (int x = 0; x < 2 && ok; ++x) {
           ok = mbar_wait(&sm.p_full[x], (uint32_t)j & 1u, lim);
           if (!ok) break;
           tc_fence_after();
+          const uint64_t pd = sdesc_sw128(smem_u32(sm.p[x]), 16, 1024);
 #pragma unroll
-          for (int part = 0; part < 2; ++part) {
-            const uint64_t pd = sdesc_sw128(smem_u32(sm.p[x][part]), 16, 1024);
-#pragma unroll
-            for (int kk = 0; kk < kKeys / 16; ++kk)
-              mma_f16_ss(tO(x), pd + (uint64_t)(kk * 32 / 16), vd + (uint64_t)(kk * 2048 / 16), idesc_pv,
-                         (j > 0 || part > 0 || kk > 0) ? 1u : 0u);
-          }
+          for (int kk = 0; kk < kKeys / 16; ++kk)
+            mma_f16_ss(tO(x), pd + (uint64_t)(kk * 32 / 16), vd + (uint64_t)(kk * 2048 / 16), idesc_pv,
+                       (j > 0 || kk > 0) ? 1u : 0u);
           mma_commit(&sm.o_done[x]);
         }
         if (ok) mma_commit(&sm.v_empty[s]);
@@ -280,6 +273,36 @@ __global__ void __launch_bounds__(kSwThreads, 1)
         ok = mbar_wait(&sm.v_full[j % kRing], (uint32_t)(j / kRing) & 1u, lim);
     }
     if (lead && !ok) latch_status(p.status, GDN_ERR_TIMEOUT);
+  } else if (warp >= 12) {
+    // ---------------- V halves to fp16 in place, each warp half of the 16 KB ----------------
+    const int part = warp - 12;
+    bool range_bad = false, failed = false;
+    for (int j = 0; j < nt; ++j) {
+      const int s = j % kRing;
+      if (__any_sync(0xffffffffu, !mbar_wait(&sm.v_full[s], (uint32_t)(j / kRing) & 1u, lim))) {
+        failed = true;
+        break;
+      }
+      uint4 *vt = reinterpret_cast<uint4 *>(sm.kv[s][1]) + part * 512;
+#pragma unroll 4
+      for (int e = 0; e < 16; ++e) {
+        const uint4 w = vt[lane + 32 * e];
+        const uint32_t in[4] = {w.x, w.y, w.z, w.w};
+        uint32_t out[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float lo = __uint_as_float(in[i] << 16), hi = __uint_as_float(in[i] & 0xffff0000u);
+          range_bad |= !(fmaxf(fabsf(lo), fabsf(hi)) < 65504.0f);
+          out[i] = pack_f16x2(lo, hi);
+        }
+        vt[lane + 32 * e] = make_uint4(out[0], out[1], out[2], out[3]);
+      }
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_only(&sm.v_conv[s]);
+    }
+    if (__any_sync(0xffffffffu, range_bad) && lane == 0) latch_status(p.status, GDN_ERR_RANGE);
+    if (failed && lane == 0) latch_status(p.status, GDN_ERR_TIMEOUT);
   } else {
     // ---------------- softmax: query tile x = warp / 4, one query row per thread ----------------
     const int x = warp >> 2, quarter = warp & 3;
@@ -330,8 +353,8 @@ __global__ void __launch_bounds__(kSwThreads, 1)
         m = m_new;
       }
       // p = exp2(s * scale_log2 - m), written 8 keys at a time as bf16 high and low parts
-      l += full ? tile_exp<true>(sc, kKeys, p.scale_log2, m, row, sm.p[x][0], sm.p[x][1])
-                : tile_exp<false>(sc, t.valid, p.scale_log2, m, row, sm.p[x][0], sm.p[x][1]);
+      l += full ? tile_exp<true>(sc, kKeys, p.scale_log2, m, row, sm.p[x])
+                : tile_exp<false>(sc, t.valid, p.scale_log2, m, row, sm.p[x]);
       fence_async_smem();
       tc_fence_before();
       if (__any_sync(0xffffffffu, bad)) { failed = true; break; }

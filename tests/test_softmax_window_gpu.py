@@ -3,9 +3,8 @@ CPU oracle, called through the C ABI.
 
 Bar: max|o - o_ref| <= 2e-3 * max|o_ref| (bf16 inputs), the bound every mode of
 the library meets.  The kernel forms the scores exactly (bf16 products, fp32
-sums) and splits the probabilities into bf16 high and low parts for the second
-product (about 16 significant bits), so
-its error sits far below the bar.
+sums) and rounds the probabilities and v to fp16 (11-bit significands) for the
+second product, so its error sits far below the bar.
 """
 import numpy as np
 import pytest
@@ -107,10 +106,18 @@ def test_720p_60s_window4_sampled_frames(lib, dev):
 
 def test_large_values_and_refusals(lib, dev):
     (q, k, v), (qh, kh, vh) = inputs(1, 2, 3, 40, 32, 32, seed=64, dev=dev)
-    big = (v.float() * 3000.0).to(torch.bfloat16)  # |v| beyond the fp16 range: v enters the product as bf16
+    big = (v.float() * 3000.0).to(torch.bfloat16)  # large values inside the fp16 range of the second product
     o = lib.softmax_window_fwd(q, k, big, F=3, W=2)
     torch.cuda.synchronize()
     assert rel_err(o.cpu().numpy(), oracle.softmax_window(qh, kh, big.float().cpu().numpy(), F=3, L=40, W=2)) <= TOL
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    huge = v.clone()
+    huge[0, 1, 17, 5] = 70000.0  # past the fp16 range: reported, not silently wrong
+    lib.softmax_window_fwd(q, k, huge, F=3, W=2, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == lib.ERR_RANGE
+    lib.softmax_window_fwd(q, k, huge, F=3, W=2, impl="frame_simt")  # the fp32 path takes it
+    torch.cuda.synchronize()
     with pytest.raises(lib.GdnError) as e:  # the tensor-core kernel takes bf16 only
         lib.softmax_window_fwd(q.float(), k.float(), v.float(), F=3, W=1, impl="tc")
     assert e.value.code == lib.ERR_UNSUPPORTED
