@@ -165,6 +165,32 @@ def test_temporal_conv_argument_validation(lib):
         assert call(x, w, None, c, c, y, 1, 4, 8, 16) == lib.ERR_NO_DEVICE
 
 
+def test_softmax_window_argument_validation(lib):
+    raw = lib._lib
+    o = lib.make_opts(lib.DTYPE_BF16, stream=0)
+    P = ctypes.c_void_p
+    q, k, v, out = P(0x100000), P(0x200000), P(0x300000), P(0x400000)  # never dereferenced
+    f32 = ctypes.c_float
+    call = lambda *a: raw.softmax_window_fwd(*a, ctypes.byref(o))
+    assert call(None, k, v, out, 1, 2, 3, 16, 32, 32, 2, f32(0)) == lib.ERR_INVALID_ARG     # null q
+    assert call(q, k, v, None, 1, 2, 3, 16, 32, 32, 2, f32(0)) == lib.ERR_INVALID_ARG       # null o
+    assert call(q, k, v, out, 1, 2, 3, 16, 32, 32, 0, f32(0)) == lib.ERR_INVALID_ARG        # W = 0
+    assert call(q, k, v, out, 1, 2, 3, 16, 32, 32, 2, f32(-1)) == lib.ERR_INVALID_ARG       # negative scale
+    assert call(q, k, v, out, 1, 2, 3, 16, 256, 32, 2, f32(0)) == lib.ERR_UNSUPPORTED       # dk > 128
+    assert call(P(0x100004), k, v, out, 1, 2, 3, 16, 32, 32, 2, f32(0)) == lib.ERR_INVALID_ARG  # misaligned
+    assert call(q, k, v, P(0x100000 + 512), 1, 2, 3, 16, 32, 32, 2, f32(0)) == lib.ERR_INVALID_ARG  # o inside q
+    o.impl = lib.IMPL_TC
+    assert call(q, k, v, out, 1, 2, 3, 16, 24, 32, 2, f32(0)) == lib.ERR_UNSUPPORTED        # tc: d % 16
+    o.in_dtype = lib.DTYPE_F32
+    assert call(q, k, v, out, 1, 2, 3, 16, 32, 32, 2, f32(0)) == lib.ERR_UNSUPPORTED        # tc: bf16 only
+    o.impl = 9
+    assert call(q, k, v, out, 1, 2, 3, 16, 32, 32, 2, f32(0)) == lib.ERR_INVALID_ARG        # unknown kernel
+    o.impl = 0
+    import torch
+    if not torch.cuda.is_available():  # valid arguments: the device check comes last
+        assert call(q, k, v, out, 1, 2, 3, 16, 24, 40, 2, f32(0)) == lib.ERR_NO_DEVICE
+
+
 def test_no_device_is_reported_without_gpu(lib):
     import torch
     if torch.cuda.is_available():
