@@ -8,7 +8,9 @@ CUDA path.
 What is computed, and the passages it follows, is stated at the top of
 ``oracle.c``.  Parity is pinned by the ``-m "not gpu"`` tests in
 ``tests/test_oracle_pins.py`` (brute-force dense products, closed forms,
-invariants, O(N^2) masked attention).
+invariants, O(N^2) masked attention) and, for the backward ``gdn_bwd``, by
+``tests/test_oracle_bwd_pins.py`` (finite differences of the forward, torch
+autograd through an independent loop, closed forms).
 """
 from __future__ import annotations
 
@@ -51,6 +53,9 @@ def _load():
         lib.oracle_temporal_conv.argtypes = [P, P, P, P, P, P, I64, I64, I64, I64]
         lib.oracle_temporal_conv.restype = ctypes.c_int
         lib.oracle_gdn.restype = ctypes.c_int
+        lib.oracle_gdn_bwd.argtypes = [P, P, P, P, P, ctypes.c_int, P, P, P, P, P, P, P, P, P,
+                                       I64, I64, I64, I64, I64, I64, P, I64, ctypes.c_int]
+        lib.oracle_gdn_bwd.restype = ctypes.c_int
         lib.oracle_relu_la.argtypes = [P, P, P, P, P, P, P, P, I64, I64, I64, I64, I64, I64, ctypes.c_double,
                                        ctypes.c_int]
         lib.oracle_relu_la.restype = ctypes.c_int
@@ -119,6 +124,40 @@ def gdn(q, k, v, alpha, beta, *, F: int, L: int, gates_are_logits: bool = True, 
     if rc != 0:
         raise ValueError("oracle_gdn: invalid arguments")
     return o, s_out
+
+
+def gdn_bwd(q, k, v, alpha, beta, d_o, *, F: int, L: int, gates_are_logits: bool = True, state_in=None,
+            dstate_out=None, heads=None, nthreads: int | None = None):
+    """Backward of the Gated DeltaNet frame recurrence in fp64 (see oracle.c).
+
+    Shapes as in ``gdn``; d_o: [..., F*L, dv] (dL/do), dstate_out: [..., dk, dv]
+    or None (zero).  Returns a dict of float64 arrays: dq, dk [..., F*L, dk],
+    dv [..., F*L, dv], dalpha [..., F] and dbeta [..., F*L] (with respect to the
+    logits when ``gates_are_logits``, else the gate values) and dstate_in
+    [..., dk, dv].  heads: optional subset of flat head indices (the others'
+    entries are NaN)."""
+    q, k, v, alpha, beta, d_o = map(_f32, (q, k, v, alpha, beta, d_o))
+    lead = q.shape[:-2]
+    N, dk = q.shape[-2:]
+    dv = v.shape[-1]
+    assert N == F * L and k.shape == q.shape and v.shape[:-1] == q.shape[:-1] and d_o.shape == v.shape
+    nh = int(np.prod(lead)) if lead else 1
+    assert alpha.size == nh * F and beta.size == nh * N
+    s_in, ds_out = _f64(state_in), _f64(dstate_out)
+    for x in (s_in, ds_out):
+        assert x is None or x.size == nh * dk * dv
+    out = dict(dq=np.full(lead + (N, dk), np.nan), dk=np.full(lead + (N, dk), np.nan),
+               dv=np.full(lead + (N, dv), np.nan), dalpha=np.full(lead + (F,), np.nan),
+               dbeta=np.full(lead + (N,), np.nan), dstate_in=np.full(lead + (dk, dv), np.nan))
+    hl = None if heads is None else np.ascontiguousarray(np.asarray(heads, dtype=np.int64))
+    nthreads = nthreads or (os.cpu_count() or 1)
+    rc = _load().oracle_gdn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), int(gates_are_logits),
+                                _ptr(s_in), _ptr(d_o), _ptr(ds_out), _ptr(out["dq"]), _ptr(out["dk"]),
+                                _ptr(out["dv"]), _ptr(out["dalpha"]), _ptr(out["dbeta"]), _ptr(out["dstate_in"]),
+                                1, nh, F, L, dk, dv, _ptr(hl), 0 if hl is None else hl.size, nthreads)
+    if rc != 0:
+        raise ValueError("oracle_gdn_bwd: invalid arguments")
+    return out
 
 
 def _rope_args(rope):

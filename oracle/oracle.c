@@ -47,6 +47,10 @@
  * Threads split the work over independent (b, h) heads and blocks of d_v
  * columns (column j of S and o depends only on column j of v and S0), which
  * changes no arithmetic.
+ *
+ * The backward of the Gated DeltaNet recurrence (oracle_gdn_bwd, below) is its
+ * reverse-mode derivative, token by token in fp64; its pins are finite
+ * differences of the forward and torch autograd through a separate loop.
  */
 #include <math.h>
 #include <pthread.h>
@@ -250,6 +254,231 @@ int oracle_gdn(const float *q, const float *k, const float *v, const float *alph
   pthread_t th[512];
   for (int t = 1; t < nthreads; ++t) pthread_create(&th[t], NULL, gdn_worker, &pl);
   gdn_worker(&pl);
+  for (int t = 1; t < nthreads; ++t) pthread_join(th[t], NULL);
+  pthread_mutex_destroy(&pl.mu);
+  free(units);
+  return 0;
+}
+
+/*
+ * Backward of the Gated DeltaNet frame recurrence (no position embedding).
+ *
+ * The model is trained (SANA-WM GeekNews summary, "Core design and generation
+ * pipeline": 64 H100 GPUs over 15 days), so the recurrence above needs its
+ * gradient.  Given dL/do [B,H,F*L,dv] (do) and dL/dstate_out [B,H,dk,dv]
+ * (dstate_out, nullable = 0) for a loss L, this returns dL/dq, dL/dk, dL/dv,
+ * dL/d(alpha input) [B,H,F] and dL/d(beta input) [B,H,F*L] (with respect to
+ * the logits a, b when gates_are_logits, else the gate values), and
+ * dL/dstate_in [B,H,dk,dv] (also when state_in is NULL: the gradient with
+ * respect to the zero start state).
+ *
+ * Reverse-mode differentiation of the forward above, one head at a time:
+ *   1. Forward over the frames, keeping S_{f-1} (the state before frame f's
+ *      decay) for every frame.
+ *   2. Frames in reverse.  Frame f is run forward again from alpha_f S_{f-1},
+ *      keeping each token's r_t = S^T khat_t - v_t; with S_f its end state,
+ *      the read-out o_t = S_f^T q_t gives dq_t = S_f do_t and adds
+ *      sum_t q_t do_t^T to H = dL/dS_f.  Tokens in reverse: with
+ *      H = dL/dS after token t and S the state after it,
+ *        S    <- S + beta khat r^T           (the state before token t: the
+ *                                             update undone, exact in real
+ *                                             arithmetic)
+ *        g     = H^T khat                    (length d_v)
+ *        dv_t  = beta g
+ *        dbeta = -(g . r)
+ *        dkhat = -beta (H r + S g)
+ *        H    <- H - beta khat g^T           (dL/dS before token t)
+ *      then dk_t from dkhat through khat = k / max(||k||, eps):
+ *        dk = (dkhat - khat (khat . dkhat)) / ||k||   if ||k|| > eps,
+ *        dk = dkhat / eps                             otherwise.
+ *      At the frame start H = dL/d(alpha_f S_{f-1}):
+ *        dalpha_f = <H, S_{f-1}>,  dL/dS_{f-1} = alpha_f H  (carried to frame f-1).
+ *   3. Gate logits: dalpha/da = -alpha (1 - alpha) (alpha = 1 / (1 + e^a)),
+ *      dbeta/db = beta (1 - beta).
+ * The derivation is pinned by central finite differences of the forward.
+ * heads: optional list of nheads flat head indices (NULL = all); only their
+ * outputs are written.
+ */
+typedef struct {
+  const float *q, *k, *v, *alpha, *beta, *d_o;
+  int logits;
+  const double *s_in, *ds_out;
+  double *dq, *dk, *dv, *dal, *dbe, *ds_in;
+  int64_t F, L, dk_, dv_, bh;
+} gdn_bwd_unit_t;
+
+static void gdn_bwd_unit(const gdn_bwd_unit_t *u) {
+  const int64_t F = u->F, L = u->L, dk = u->dk_, dv = u->dv_, N = F * L, bh = u->bh;
+  const int64_t SS = dk * dv;
+  const float *q = u->q + bh * N * dk, *k = u->k + bh * N * dk, *v = u->v + bh * N * dv;
+  const float *al = u->alpha + bh * F, *be = u->beta + bh * N, *d_o = u->d_o + bh * N * dv;
+  double *Sprev = (double *)calloc((size_t)(F * SS), sizeof(double)); /* S_{f-1} for each frame f */
+  double *S = (double *)calloc((size_t)SS, sizeof(double));
+  double *H = (double *)calloc((size_t)SS, sizeof(double));
+  double *kh = (double *)malloc(sizeof(double) * (size_t)(L * dk)); /* the frame's khat rows */
+  double *nrm = (double *)malloc(sizeof(double) * (size_t)L);
+  double *r = (double *)malloc(sizeof(double) * (size_t)(L * dv));   /* the frame's residuals */
+  double *g = (double *)malloc(sizeof(double) * (size_t)dv);
+  double *dkh = (double *)malloc(sizeof(double) * (size_t)dk);
+  if (u->s_in)
+    for (int64_t e = 0; e < SS; ++e) S[e] = u->s_in[bh * SS + e];
+  /* khat_t and ||k_t|| for token t of frame f (index tl in the frame) */
+#define GDN_BWD_KEY(f, tl)                                                        \
+  do {                                                                            \
+    const float *kt = k + ((f) * L + (tl)) * dk;                                  \
+    double ss = 0.0;                                                              \
+    for (int64_t i = 0; i < dk; ++i) ss += (double)kt[i] * (double)kt[i];         \
+    const double n_ = sqrt(ss);                                                   \
+    const double den = n_ > GDN_KEY_NORM_EPS ? n_ : GDN_KEY_NORM_EPS;             \
+    nrm[tl] = n_;                                                                 \
+    for (int64_t i = 0; i < dk; ++i) kh[(tl) * dk + i] = (double)kt[i] / den;     \
+  } while (0)
+  /* 1. forward over the frames */
+  for (int64_t f = 0; f < F; ++f) {
+    memcpy(Sprev + f * SS, S, sizeof(double) * (size_t)SS);
+    const double alpha = u->logits ? gate_alpha((double)al[f]) : (double)al[f];
+    for (int64_t e = 0; e < SS; ++e) S[e] *= alpha;
+    for (int64_t tl = 0; tl < L; ++tl) {
+      GDN_BWD_KEY(f, tl);
+      const double *x = kh + tl * dk;
+      const double beta = u->logits ? gate_beta((double)be[f * L + tl]) : (double)be[f * L + tl];
+      for (int64_t j = 0; j < dv; ++j) {
+        double p = 0.0;
+        for (int64_t i = 0; i < dk; ++i) p += S[i * dv + j] * x[i];
+        r[j] = p - (double)v[(f * L + tl) * dv + j];
+      }
+      for (int64_t i = 0; i < dk; ++i)
+        for (int64_t j = 0; j < dv; ++j) S[i * dv + j] -= beta * x[i] * r[j];
+    }
+  }
+  /* 2. frames in reverse; H = dL/dS after the last frame */
+  if (u->ds_out)
+    for (int64_t e = 0; e < SS; ++e) H[e] = u->ds_out[bh * SS + e];
+  for (int64_t f = F - 1; f >= 0; --f) {
+    const double alpha = u->logits ? gate_alpha((double)al[f]) : (double)al[f];
+    for (int64_t e = 0; e < SS; ++e) S[e] = alpha * Sprev[f * SS + e];
+    for (int64_t tl = 0; tl < L; ++tl) { /* the frame again, keeping khat and r */
+      GDN_BWD_KEY(f, tl);
+      const double *x = kh + tl * dk;
+      double *rt = r + tl * dv;
+      const double beta = u->logits ? gate_beta((double)be[f * L + tl]) : (double)be[f * L + tl];
+      for (int64_t j = 0; j < dv; ++j) {
+        double p = 0.0;
+        for (int64_t i = 0; i < dk; ++i) p += S[i * dv + j] * x[i];
+        rt[j] = p - (double)v[(f * L + tl) * dv + j];
+      }
+      for (int64_t i = 0; i < dk; ++i)
+        for (int64_t j = 0; j < dv; ++j) S[i * dv + j] -= beta * x[i] * rt[j];
+    }
+    /* read-out: o_t = S_f^T q_t */
+    for (int64_t tl = 0; tl < L; ++tl) {
+      const int64_t t = f * L + tl;
+      for (int64_t i = 0; i < dk; ++i) {
+        double acc = 0.0;
+        for (int64_t j = 0; j < dv; ++j) acc += S[i * dv + j] * (double)d_o[t * dv + j];
+        u->dq[(bh * N + t) * dk + i] = acc;
+      }
+      for (int64_t i = 0; i < dk; ++i)
+        for (int64_t j = 0; j < dv; ++j) H[i * dv + j] += (double)q[t * dk + i] * (double)d_o[t * dv + j];
+    }
+    /* tokens in reverse */
+    for (int64_t tl = L - 1; tl >= 0; --tl) {
+      const int64_t t = f * L + tl;
+      const double *x = kh + tl * dk, *rt = r + tl * dv;
+      const double beta = u->logits ? gate_beta((double)be[t]) : (double)be[t];
+      for (int64_t i = 0; i < dk; ++i)
+        for (int64_t j = 0; j < dv; ++j) S[i * dv + j] += beta * x[i] * rt[j];
+      for (int64_t j = 0; j < dv; ++j) {
+        double p = 0.0;
+        for (int64_t i = 0; i < dk; ++i) p += H[i * dv + j] * x[i];
+        g[j] = p;
+        u->dv[(bh * N + t) * dv + j] = beta * p;
+      }
+      double gr = 0.0;
+      for (int64_t j = 0; j < dv; ++j) gr += g[j] * rt[j];
+      const double dbeta = -gr;
+      for (int64_t i = 0; i < dk; ++i) {
+        double hr = 0.0, sg = 0.0;
+        for (int64_t j = 0; j < dv; ++j) {
+          hr += H[i * dv + j] * rt[j];
+          sg += S[i * dv + j] * g[j];
+        }
+        dkh[i] = -beta * (hr + sg);
+      }
+      for (int64_t i = 0; i < dk; ++i)
+        for (int64_t j = 0; j < dv; ++j) H[i * dv + j] -= beta * x[i] * g[j];
+      if (nrm[tl] > GDN_KEY_NORM_EPS) {
+        double kd = 0.0;
+        for (int64_t i = 0; i < dk; ++i) kd += x[i] * dkh[i];
+        for (int64_t i = 0; i < dk; ++i) u->dk[(bh * N + t) * dk + i] = (dkh[i] - x[i] * kd) / nrm[tl];
+      } else {
+        for (int64_t i = 0; i < dk; ++i) u->dk[(bh * N + t) * dk + i] = dkh[i] / GDN_KEY_NORM_EPS;
+      }
+      u->dbe[bh * N + t] = u->logits ? dbeta * beta * (1.0 - beta) : dbeta;
+    }
+    /* frame start: H = dL/d(alpha_f S_{f-1}) */
+    double da = 0.0;
+    for (int64_t e = 0; e < SS; ++e) da += H[e] * Sprev[f * SS + e];
+    u->dal[bh * F + f] = u->logits ? da * (-alpha * (1.0 - alpha)) : da;
+    for (int64_t e = 0; e < SS; ++e) H[e] *= alpha;
+  }
+#undef GDN_BWD_KEY
+  if (u->ds_in)
+    for (int64_t e = 0; e < SS; ++e) u->ds_in[bh * SS + e] = H[e];
+  free(Sprev);
+  free(S);
+  free(H);
+  free(kh);
+  free(nrm);
+  free(r);
+  free(g);
+  free(dkh);
+}
+
+typedef struct {
+  gdn_bwd_unit_t *units;
+  int64_t n, next;
+  pthread_mutex_t mu;
+} bwd_pool_t;
+
+static void *gdn_bwd_worker(void *p) {
+  bwd_pool_t *pl = (bwd_pool_t *)p;
+  for (;;) {
+    pthread_mutex_lock(&pl->mu);
+    int64_t i = pl->next++;
+    pthread_mutex_unlock(&pl->mu);
+    if (i >= pl->n) return NULL;
+    gdn_bwd_unit(&pl->units[i]);
+  }
+}
+
+int oracle_gdn_bwd(const float *q, const float *k, const float *v, const float *alpha, const float *beta,
+                   int gates_are_logits, const double *state_in, const float *d_o, const double *dstate_out,
+                   double *dq, double *dk, double *dv, double *dalpha, double *dbeta, double *dstate_in,
+                   int64_t B, int64_t H, int64_t F, int64_t L, int64_t dk_, int64_t dv_,
+                   const int64_t *heads, int64_t nheads, int nthreads) {
+  if (B < 0 || H < 0 || F < 0 || L < 0 || dk_ <= 0 || dv_ <= 0) return 1;
+  if (!dq || !dk || !dv || !dalpha || !dbeta) return 1;
+  const int64_t n = heads ? nheads : B * H;
+  if (n <= 0) return 0;
+  gdn_bwd_unit_t *units = (gdn_bwd_unit_t *)calloc((size_t)n, sizeof(gdn_bwd_unit_t));
+  for (int64_t h = 0; h < n; ++h) {
+    gdn_bwd_unit_t *u = &units[h];
+    u->q = q; u->k = k; u->v = v; u->alpha = alpha; u->beta = beta; u->d_o = d_o;
+    u->logits = gates_are_logits; u->s_in = state_in; u->ds_out = dstate_out;
+    u->dq = dq; u->dk = dk; u->dv = dv; u->dal = dalpha; u->dbe = dbeta; u->ds_in = dstate_in;
+    u->F = F; u->L = L; u->dk_ = dk_; u->dv_ = dv_;
+    u->bh = heads ? heads[h] : h;
+  }
+  bwd_pool_t pl;
+  pl.units = units; pl.n = n; pl.next = 0;
+  pthread_mutex_init(&pl.mu, NULL);
+  if (nthreads < 1) nthreads = 1;
+  if (nthreads > n) nthreads = (int)n;
+  if (nthreads > 512) nthreads = 512;
+  pthread_t th[512];
+  for (int t = 1; t < nthreads; ++t) pthread_create(&th[t], NULL, gdn_bwd_worker, &pl);
+  gdn_bwd_worker(&pl);
   for (int t = 1; t < nthreads; ++t) pthread_join(th[t], NULL);
   pthread_mutex_destroy(&pl.mu);
   free(units);
