@@ -56,7 +56,7 @@ extern "C" {
 #define GDN_API
 #endif
 
-#define GDN_ABI_VERSION 6
+#define GDN_ABI_VERSION 7
 
 /* return / status codes */
 #define GDN_OK 0
@@ -86,6 +86,7 @@ extern "C" {
 /* operation ids for gdn_workspace_bytes() */
 #define GDN_OP_GDN 0
 #define GDN_OP_RELU_LA 1
+#define GDN_OP_GDN_BWD 2
 
 typedef struct gdn_opts {
   int in_dtype;           /* GDN_DTYPE_F32 or GDN_DTYPE_BF16: element type of q, k, v */
@@ -170,6 +171,50 @@ typedef struct gdn_opts {
  */
 GDN_API int gdn_frame_fwd(const void *q, const void *k, const void *v, const float *alpha, const float *beta,
                   const float *state_in, float *state_out, float *o, int B, int H, int F, int L,
+                  int dk, int dv, const gdn_opts_t *opts);
+
+/*
+ * gdn_frame_bwd -- backward of gdn_frame_fwd (without the position embedding).
+ *
+ * The model is trained (SANA-WM GeekNews summary, "Core design and generation
+ * pipeline": 64 H100 GPUs over 15 days), so the recurrence needs its
+ * gradient.  For a loss L, given d_o = dL/do [B, H, N, dv] and d_state_out =
+ * dL/dstate_out [B, H, dk, dv] (zero if NULL), this writes
+ *   d_q, d_k  [B, H, N, dk]  dL/dq, dL/dk
+ *   d_v       [B, H, N, dv]  dL/dv
+ *   d_alpha   [B, H, F]      dL/d(alpha input): with respect to the logit a when
+ *                            opts->gates_are_logits (alpha = exp(-softplus(a))),
+ *                            else to the gate value
+ *   d_beta    [B, H, N]      the same for beta (beta = sigmoid(b) with logits)
+ *   d_state_in [B, H, dk, dv]  dL/dstate_in (skipped if NULL; with state_in ==
+ *                            NULL, the gradient at the zero start state)
+ * all float32.  The inputs q, k, v, alpha, beta, state_in are those of the
+ * forward call (the forward is recomputed; nothing is kept between calls).
+ * The outputs may overlap neither one another nor the inputs.
+ *
+ * Method: with G_f = dL/dS_f, the gradient at frame f's end state,
+ *   G_{F-1} = dS_out + Q_{F-1}^T dO_{F-1},  G_{f-1} = Q_{f-1}^T dO_{f-1} + alpha_f A_f^T G_f,
+ * A_f being the frame's transition (ordered product of I - beta khat khat^T),
+ * and d_alpha_f = <A_f^T G_f, S_{f-1}>, d_state_in = alpha_0 A_0^T G_0.  Inside a
+ * frame the token gradients come from two sweeps over chunks of 48 tokens in
+ * the UT form: forward from alpha_f S_{f-1}, then in reverse from G_f.  Three
+ * launches on opts->stream: the forward recompute keeping every frame's A_f
+ * and S_f (GDN_IMPL_TC for bf16 inputs where it applies, else FRAME_SIMT in
+ * fp32; opts->impl may force either), the chain over frames, and one CTA per
+ * frame for the token gradients (fp32 on CUDA cores).
+ *
+ * Sizes: as gdn_frame_fwd, with dk, dv <= 112.  Workspace:
+ * gdn_workspace_bytes(GDN_OP_GDN_BWD, ...) (four fp32 d x d matrices per frame
+ * plus the recompute's scratch).  opts->rope_grid_w must be 0
+ * (GDN_ERR_UNSUPPORTED otherwise).
+ *
+ * Precision: with bf16 inputs the recomputed A_f and S_f carry the tensor-core
+ * forward's rounding (see gdn_frame_fwd); everything else is fp32.  Returns
+ * GDN_OK or GDN_ERR_*.
+ */
+GDN_API int gdn_frame_bwd(const void *q, const void *k, const void *v, const float *alpha, const float *beta,
+                  const float *state_in, const float *d_o, const float *d_state_out, float *d_q, float *d_k,
+                  float *d_v, float *d_alpha, float *d_beta, float *d_state_in, int B, int H, int F, int L,
                   int dk, int dv, const gdn_opts_t *opts);
 
 /*

@@ -26,13 +26,13 @@ _lib = ctypes.CDLL(LIB_PATH)
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_NO_DEVICE, ERR_RANGE = range(7)
 DTYPE_F32, DTYPE_BF16 = 0, 1
 IMPL_AUTO, IMPL_SEQ, IMPL_FRAME_SIMT, IMPL_TC, IMPL_TC_PFORM = 0, 1, 2, 3, 4
-OP_GDN, OP_RELU_LA = 0, 1
+OP_GDN, OP_RELU_LA, OP_GDN_BWD = 0, 1, 2
 IMPLS = {"auto": IMPL_AUTO, "seq": IMPL_SEQ, "frame_simt": IMPL_FRAME_SIMT, "tc": IMPL_TC,
          "tc_pform": IMPL_TC_PFORM}
 
 EXPORTED = ("gdn_frame_fwd", "relu_la_block_fwd", "gdn_frame_fwd_host", "gdn_frame_fwd_noalloc",
             "gdn_workspace_bytes", "gdn_workspace_bytes_host", "gdn_status_string", "gdn_status_str",
-            "gdn_abi_version", "temporal_conv_fwd", "softmax_window_fwd")
+            "gdn_abi_version", "temporal_conv_fwd", "softmax_window_fwd", "gdn_frame_bwd")
 NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
 
 
@@ -48,6 +48,8 @@ _P = ctypes.c_void_p
 _I = ctypes.c_int
 _lib.gdn_frame_fwd.argtypes = [_P] * 8 + [_I] * 6 + [ctypes.POINTER(GdnOpts)]
 _lib.gdn_frame_fwd.restype = _I
+_lib.gdn_frame_bwd.argtypes = [_P] * 14 + [_I] * 6 + [ctypes.POINTER(GdnOpts)]
+_lib.gdn_frame_bwd.restype = _I
 _lib.gdn_frame_fwd_host.argtypes = [_P] * 8 + [_I] * 6 + [ctypes.POINTER(GdnOpts)]
 _lib.gdn_frame_fwd_host.restype = _I
 _lib.gdn_frame_fwd_noalloc.argtypes = [_P] * 8 + [_I] * 6 + [ctypes.POINTER(GdnOpts)]
@@ -191,6 +193,55 @@ def gdn_frame_fwd(q, k, v, alpha, beta, *, F: int, state_in=None, state_out=None
     if rc != OK:
         raise GdnError(rc, "gdn_frame_fwd")
     return o
+
+
+def gdn_frame_bwd(q, k, v, alpha, beta, d_o, *, F: int, state_in=None, d_state_out=None, out=None,
+                  gates_are_logits: bool = True, impl="auto", workspace=None, stream=None, status=None,
+                  max_ctas: int = 0, spin_limit_us: int = 0, test_withhold_unit: int = -1):
+    """Backward of ``gdn_frame_fwd`` on the GPU (see include/gdn_b200.h).
+
+    q, k, v, alpha, beta, state_in: the forward call's inputs; d_o: [B, H, F*L, dv]
+    float32 (dL/do); d_state_out: [B, H, dk, dv] float32 or None (zero).  Returns
+    a dict of float32 tensors dq, dk [B, H, F*L, dk], dv [B, H, F*L, dv],
+    dalpha [B, H, F], dbeta [B, H, F*L] (with respect to the logits when
+    ``gates_are_logits``) and dstate_in [B, H, dk, dv].  ``out``: an optional
+    dict of preallocated tensors with those names.
+    """
+    B, H, N, dk = q.shape
+    dv = v.shape[-1]
+    if N % F:
+        raise ValueError(f"token count {N} is not a multiple of F={F}")
+    L = N // F
+    dev = q.device
+    _check(k, "k", (B, H, N, dk), q.dtype, dev)
+    _check(v, "v", (B, H, N, dv), q.dtype, dev)
+    _check(q, "q", (B, H, N, dk), q.dtype, dev)
+    _check(alpha, "alpha", (B, H, F), torch.float32, dev)
+    _check(beta, "beta", (B, H, N), torch.float32, dev)
+    _check(state_in, "state_in", (B, H, dk, dv), torch.float32, dev, allow_none=True)
+    _check(d_o, "d_o", (B, H, N, dv), torch.float32, dev)
+    _check(d_state_out, "d_state_out", (B, H, dk, dv), torch.float32, dev, allow_none=True)
+    shapes = dict(dq=(B, H, N, dk), dk=(B, H, N, dk), dv=(B, H, N, dv), dalpha=(B, H, F), dbeta=(B, H, N),
+                  dstate_in=(B, H, dk, dv))
+    out = dict(out or {})
+    for name, shp in shapes.items():
+        if out.get(name) is None:
+            out[name] = torch.empty(shp, dtype=torch.float32, device=dev)
+        _check(out[name], name, shp, torch.float32, dev)
+    opts = make_opts(_dtype_code(q), gates_are_logits=gates_are_logits, impl=impl, stream=stream,
+                     status=status, max_ctas=max_ctas, spin_limit_us=spin_limit_us,
+                     test_withhold_unit=test_withhold_unit)
+    need = workspace_bytes(OP_GDN_BWD, B, H, F, L, dk, dv, opts)
+    if workspace is None:
+        workspace = alloc_workspace(need, dev)
+    opts.workspace = workspace.data_ptr()
+    opts.workspace_bytes = workspace.numel() * workspace.element_size()
+    rc = _lib.gdn_frame_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(state_in), _ptr(d_o),
+                            _ptr(d_state_out), *(_ptr(out[n]) for n in shapes), B, H, F, L, dk, dv,
+                            ctypes.byref(opts))
+    if rc != OK:
+        raise GdnError(rc, "gdn_frame_bwd")
+    return out
 
 
 def relu_la_block_fwd(q, k, v, *, F: int, kv_in=None, z_in=None, kv_out=None, z_out=None, o=None,

@@ -164,6 +164,16 @@ int grid_for(const gdn_opts_t *o, int sms, long units) {
 }  // namespace
 }  // namespace gdn
 
+namespace gdn {
+namespace {
+bool overlap(const void *a, size_t na, const void *b, size_t nb) {
+  if (!a || !b) return false;
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+}  // namespace
+}  // namespace gdn
+
 using namespace gdn;
 
 extern "C" int gdn_abi_version(void) { return GDN_ABI_VERSION; }
@@ -185,12 +195,124 @@ extern "C" const char *gdn_status_string(int s) {
 
 extern "C" const char *gdn_status_str(int s) { return gdn_status_string(s); }
 
+namespace gdn {
+namespace {
+// The backward's forward recompute: the tensor-core kernel for bf16 inputs where it
+// applies (one unit per frame), else the fp32 CUDA-core frame kernel.
+int pick_bwd_fwd_impl(const gdn_opts_t *o, int dk, int dv) {
+  if (o->impl == GDN_IMPL_FRAME_SIMT) return GDN_IMPL_FRAME_SIMT;
+  if (o->impl == GDN_IMPL_TC) return GDN_IMPL_TC;
+  return o->in_dtype == GDN_DTYPE_BF16 && gdn_tc_supported(dk, dv) ? GDN_IMPL_TC : GDN_IMPL_FRAME_SIMT;
+}
+
+// Backward workspace: the recompute's chain scratch, then A_f^T and S_f of every
+// frame, G_f of every frame, and the per-column-group dalpha partial sums.
+struct BwdLayout {
+  size_t maps, states, gbuf, part, total;
+};
+BwdLayout bwd_layout(const gdn_opts_t *o, int B, int H, int F, int dk, int dv) {
+  BwdLayout w;
+  const size_t fr = (size_t)B * H * F;
+  w.maps = align_up(gdn_ws_bytes_p(pick_bwd_fwd_impl(o, dk, dv), o, B, H, F, dk, dv, 1), 256);
+  w.states = w.maps + align_up(sizeof(float) * fr * dk * dk, 256);
+  w.gbuf = w.states + align_up(sizeof(float) * fr * dk * dv, 256);
+  w.part = w.gbuf + align_up(sizeof(float) * fr * dk * dv, 256);
+  w.total = w.part + align_up(sizeof(float) * fr * ((dv + 15) / 16), 256);
+  return w;
+}
+}  // namespace
+}  // namespace gdn
+
 extern "C" size_t gdn_workspace_bytes(int op, int B, int H, int F, int L, int dk, int dv, const gdn_opts_t *opts) {
   if (!opts || check_sizes(B, H, F, L, dk, dv) != GDN_OK) return 0;
   if (op == GDN_OP_GDN) return gdn_ws_bytes(pick_gdn_impl(opts, dk, dv), opts, B, H, F, L, dk, dv);
   if (op == GDN_OP_RELU_LA) return relu_ws_bytes(B, H, F, dk, dv);
+  if (op == GDN_OP_GDN_BWD) return bwd_layout(opts, B, H, F, dk, dv).total;
   return 0;
 }
+
+extern "C" int gdn_frame_bwd(const void *q, const void *k, const void *v, const float *alpha, const float *beta,
+                             const float *state_in, const float *d_o, const float *dstate_out, float *dq,
+                             float *dk_out, float *dv_out, float *dalpha, float *dbeta, float *dstate_in, int B,
+                             int H, int F, int L, int dk, int dv, const gdn_opts_t *opts) {
+  if (!opts) return GDN_ERR_INVALID_ARG;
+  if (!q || !k || !v || !alpha || !beta || !d_o || !dq || !dk_out || !dv_out || !dalpha || !dbeta)
+    return GDN_ERR_INVALID_ARG;
+  if (opts->in_dtype != GDN_DTYPE_F32 && opts->in_dtype != GDN_DTYPE_BF16) return GDN_ERR_INVALID_ARG;
+  if (opts->impl != GDN_IMPL_AUTO && opts->impl != GDN_IMPL_FRAME_SIMT && opts->impl != GDN_IMPL_TC)
+    return GDN_ERR_INVALID_ARG;
+  if (opts->rope_grid_w != 0) return GDN_ERR_UNSUPPORTED;  // the backward covers gdn without the embedding
+  int rc = check_sizes(B, H, F, L, dk, dv);
+  if (rc != GDN_OK) return rc;
+  if (!gdn_bwd_supported(dk, dv)) return GDN_ERR_UNSUPPORTED;
+  const void *ptrs[] = {q, k, v, alpha, beta, state_in, d_o, dstate_out, dq, dk_out, dv_out, dalpha, dbeta,
+                        dstate_in, opts->workspace, opts->status};
+  for (const void *ptr : ptrs)
+    if (!aligned16(ptr)) return GDN_ERR_INVALID_ARG;
+  // the outputs overlap neither one another nor the inputs
+  const size_t N = (size_t)B * H * F * L, nsq = (size_t)B * H * dk * dv, nf = (size_t)B * H * F;
+  const size_t isz = opts->in_dtype == GDN_DTYPE_F32 ? 4 : 2;
+  const void *outs[] = {dq, dk_out, dv_out, dalpha, dbeta, dstate_in};
+  const size_t osz[] = {N * dk * 4, N * dk * 4, N * dv * 4, nf * 4, N * 4, nsq * 4};
+  const void *ins[] = {q, k, v, alpha, beta, state_in, d_o, dstate_out};
+  const size_t insz[] = {N * dk * isz, N * dk * isz, N * dv * isz, nf * 4, N * 4, nsq * 4, N * dv * 4, nsq * 4};
+  for (int a = 0; a < 6; ++a) {
+    for (int c = a + 1; c < 6; ++c)
+      if (overlap(outs[a], osz[a], outs[c], osz[c])) return GDN_ERR_INVALID_ARG;
+    for (int c = 0; c < 8; ++c)
+      if (overlap(outs[a], osz[a], ins[c], insz[c])) return GDN_ERR_INVALID_ARG;
+  }
+  int sms = 0, cc = 0;
+  rc = device_info(&sms, &cc);
+  if (rc != GDN_OK) return rc;
+  if (cc != 100) return GDN_ERR_NO_DEVICE;
+  const int fimpl = pick_bwd_fwd_impl(opts, dk, dv);
+  if (fimpl == GDN_IMPL_TC && (opts->in_dtype != GDN_DTYPE_BF16 || !gdn_tc_supported(dk, dv)))
+    return GDN_ERR_UNSUPPORTED;
+  const BwdLayout w = bwd_layout(opts, B, H, F, dk, dv);
+  if (!opts->workspace || opts->workspace_bytes < w.total) return GDN_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(opts->workspace) & 255u) != 0) return GDN_ERR_INVALID_ARG;
+  char *ws = static_cast<char *>(opts->workspace);
+  float *maps = reinterpret_cast<float *>(ws + w.maps);
+  float *states = reinterpret_cast<float *>(ws + w.states);
+  cudaStream_t st = (cudaStream_t)opts->stream;
+
+  // 1. forward recompute: every frame's A_f^T and S_f (no read-out)
+  GdnParams p;
+  memset(&p, 0, sizeof(p));
+  p.q = q; p.k = k; p.v = v; p.alpha = alpha; p.beta = beta;
+  p.state_in = state_in;
+  p.B = B; p.H = H; p.F = F; p.L = L; p.dk = dk; p.dv = dv;
+  p.gates_are_logits = opts->gates_are_logits ? 1 : 0;
+  p.status = opts->status;
+  p.spin_limit_ns = spin_ns(opts);
+  p.withhold = opts->test_withhold_unit > 0 ? (long)opts->test_withhold_unit - 1 : -1;
+  p.segs = 1;
+  p.save_maps = maps;
+  p.save_states = states;
+  const long units = (long)B * H * F;
+  p.ws = chain_workspace(ws, units);
+  cudaError_t e = cudaMemsetAsync(ws, 0, chain_workspace_zero_bytes(units), st);
+  if (e != cudaSuccess) return GDN_ERR_CUDA;
+  const int grid = grid_for(opts, sms, units);
+  e = fimpl == GDN_IMPL_TC ? launch_gdn_tc(p, grid, false, st) : launch_gdn_frame_simt(p, opts->in_dtype, grid, st);
+  if (e != cudaSuccess) return GDN_ERR_CUDA;
+
+  // 2-3. the adjoint frame chain, then the frame-parallel backward
+  BwdParams b;
+  memset(&b, 0, sizeof(b));
+  b.q = q; b.k = k; b.v = v; b.alpha = alpha; b.beta = beta; b.state_in = state_in;
+  b.d_o = d_o; b.dstate_out = dstate_out;
+  b.maps = maps; b.states = states;
+  b.gbuf = reinterpret_cast<float *>(ws + w.gbuf);
+  b.dal_part = reinterpret_cast<float *>(ws + w.part);
+  b.dq = dq; b.dk_out = dk_out; b.dv_out = dv_out; b.dalpha = dalpha; b.dbeta = dbeta; b.dstate_in = dstate_in;
+  b.B = B; b.H = H; b.F = F; b.L = L; b.dk = dk; b.dv = dv;
+  b.gates_are_logits = p.gates_are_logits;
+  e = launch_gdn_bwd(b, opts->in_dtype, st);
+  return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
 
 extern "C" int gdn_frame_fwd(const void *q, const void *k, const void *v, const float *alpha, const float *beta,
                              const float *state_in, float *state_out, float *o, int B, int H, int F, int L,
@@ -317,15 +439,6 @@ extern "C" int relu_la_block_fwd(const void *q, const void *k, const void *v, co
   return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
-namespace gdn {
-namespace {
-bool overlap(const void *a, size_t na, const void *b, size_t nb) {
-  if (!a || !b) return false;
-  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
-  return x < y + nb && y < x + na;
-}
-}  // namespace
-}  // namespace gdn
 
 extern "C" int temporal_conv_fwd(const void *x, const float *w, const float *bias, const void *cache_in,
                                  void *cache_out, void *y, int B, int F, int HW, int C, const gdn_opts_t *opts) {

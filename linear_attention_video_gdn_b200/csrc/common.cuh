@@ -110,6 +110,28 @@ struct GdnParams {
   // (axis position, pair) as float2, time part [F][dt/2], then height [L/gw][dh/2], then width [gw][dh/2]
   const float2 *rope_tab;
   int rope_on, rope_gw, rope_dt, rope_dh;
+  // backward recompute (non-null together, one unit per frame, no position embedding):
+  // every frame's map A_f^T [b, h, f][r][i] = A_f[i][r] and end state S_f [b, h, f][l][j], fp32
+  float *save_maps;
+  float *save_states;
+};
+
+// Backward of the Gated DeltaNet (gdn_bwd.cu).  Buffers are [b, h] then as named.
+struct BwdParams {
+  const void *q, *k, *v;        // [N][dk], [N][dk], [N][dv] (bf16 or fp32)
+  const float *alpha, *beta;    // [F], [N] (logits when gates_are_logits)
+  const float *state_in;        // [dk][dv] or null (zero)
+  const float *d_o;             // [N][dv]
+  const float *dstate_out;      // [dk][dv] or null (zero)
+  const float *maps;            // [F][dk][dk]: A_f^T (recomputed forward)
+  const float *states;          // [F][dk][dv]: S_f, the end state of every frame
+  float *gbuf;                  // [F][dk][dv]: G_f = dL/dS_f (adjoint chain -> frame kernel)
+  float *dal_part;              // [F][ceil(dv / 16)]: dalpha_f per column group
+  float *dq, *dk_out, *dv_out;  // [N][dk], [N][dk], [N][dv]; dv_out is also scratch
+  float *dalpha, *dbeta;        // [F], [N]
+  float *dstate_in;             // [dk][dv] or null
+  int B, H, F, L, dk, dv;
+  int gates_are_logits;
 };
 
 // Rotated element i of the d_k-vector x (i's pair is i ^ 1) of the token at

@@ -216,6 +216,11 @@ __global__ void __launch_bounds__(256) gdn_frame_simt_kernel(GdnParams p) {
       const int l = e / DK, i = e % DK;
       if (i >= dk) sm.sAt[l][i] = 0.f;
     }
+    if (p.save_maps) {  // A_f^T rows for the backward (written by threads c < dk above)
+      __syncthreads();
+      float *mp = p.save_maps + ((long)bh * F + f) * (long)dk * dk;
+      for (int e = c; e < dk * dk; e += 256) mp[e] = sm.sAt[e / dk][e % dk];
+    }
     const float a = p.alpha[(long)bh * F + f];
     const float al = p.gates_are_logits ? gate_alpha(a) : a;
     bool have_prev = true;
@@ -261,6 +266,12 @@ __global__ void __launch_bounds__(256) gdn_frame_simt_kernel(GdnParams p) {
         for (int i = 0; i < DK; ++i)
           if (i < dk) p.state_out[(long)bh * dk * dv + (long)i * dv + j] = y[i];
       }
+      if (p.save_states) {
+        float *sp = p.save_states + ((long)bh * F + f) * (long)dk * dv;
+#pragma unroll
+        for (int i = 0; i < DK; ++i)
+          if (i < dk) sp[(long)i * dv + j] = y[i];
+      }
     }
     __syncthreads();
     if (c == 0 && ticket != p.withhold) {
@@ -268,8 +279,8 @@ __global__ void __launch_bounds__(256) gdn_frame_simt_kernel(GdnParams p) {
       st_release(p.ws.flags + (long)bh * F + f, 1);
     }
 
-    // ---- read-out: o_t = S_f^T q_t for the frame's tokens ----
-    for (long t0 = t_beg; t0 < t_end; t0 += kTile) {
+    // ---- read-out: o_t = S_f^T q_t for the frame's tokens (none for the backward's recompute) ----
+    for (long t0 = t_beg; p.o && t0 < t_end; t0 += kTile) {
       const int nt = (int)min((long)kTile, t_end - t0);
       __syncthreads();
       for (int e = c; e < kTile * DK; e += 256) {

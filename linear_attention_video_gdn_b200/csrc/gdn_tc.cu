@@ -200,7 +200,9 @@ __device__ __forceinline__ float4 neg4(float4 v) { return make_float4(-v.x, -v.y
 // segment arithmetic folds away)
 // kRope: the 3D rotary position embedding on q and k (a separate instantiation,
 // so that the kernel without it carries none of its code)
-template <bool kSeg, bool kRope>
+// kSave: the backward's recompute: every frame's map A_f^T and end state S_f
+// go to p.save_maps / p.save_states (fp32) and there is no read-out
+template <bool kSeg, bool kRope, bool kSave = false>
 __global__ void __launch_bounds__(kGThreads, 1)
     gdn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                   const __grid_constant__ CUtensorMap tmap_v, GdnParams p) {
@@ -785,13 +787,28 @@ __global__ void __launch_bounds__(kGThreads, 1)
         failed = true;
         break;
       }
+      if (kSave && tile == 0) {  // A_f^T row `row` (TMEM lane) -> the backward's frame maps
+        tc_fence_after();
+        float *mrow = p.save_maps + (((long)bh * F + f) * dk + row) * dk;
+#pragma unroll 1
+        for (int cb = 0; cb < nkd; ++cb) {
+          float r[16];
+          tmem_ld16(tmY + lane_off + cb * 16, r);
+          tmem_ld_wait();
+          if (row < dk) {
+#pragma unroll
+            for (int e = 0; e < 16; e += 4)
+              *reinterpret_cast<float4 *>(mrow + cb * 16 + e) = make_float4(r[e], r[e + 1], r[e + 2], r[e + 3]);
+          }
+        }
+      }
 
       // ---- chain step: S_f^T = B_f^T + S_{f-1}^T (alpha A_f^T)
       const long uidx = ((long)bh * F + f) * P + seg;  // this unit's flag and published state
       // read-out tiles of this chain: tile-chain A takes tiles 0, 2, 4, ...; B 1, 3, 5, ...
       const int tb0 = c0 * kC, tb1 = (kSeg && c1 * kC < L) ? c1 * kC : L;  // the unit's tokens
-      const int nt = (tb1 - tb0 + kQTok - 1) / kQTok;  // read-out tiles
-      if (tid == 0) {  // the first q tiles -> the tile-B half of the mirror (free now)
+      const int nt = kSave ? 0 : (tb1 - tb0 + kQTok - 1) / kQTok;  // read-out tiles
+      if (!kSave && tid == 0) {  // the first q tiles -> the tile-B half of the mirror (free now)
         issue_q(f, bh, tb0);
         if (nt > 1) issue_q(f, bh, tb0 + kQTok);
       }
@@ -889,6 +906,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
       const bool last_seg = seg == P - 1;
       {
         float *sout = (f == F - 1 && last_seg && p.state_out) ? p.state_out + (long)bh * dk * dv : nullptr;
+        float *sall = kSave ? p.save_states + ((long)bh * F + f) * dk * dv : nullptr;
         __half *srow = reinterpret_cast<__half *>(sm + OFF_STAGE) + (long)j * dk + l0;
         float smax = 0.f;
 #pragma unroll 1
@@ -910,6 +928,10 @@ __global__ void __launch_bounds__(kGThreads, 1)
             if (sout) {
 #pragma unroll
               for (int e = 0; e < 16; ++e) sout[(long)(lb + e) * dv + j] = r[e];
+            }
+            if (kSave) {
+#pragma unroll
+              for (int e = 0; e < 16; ++e) sall[(long)(lb + e) * dv + j] = r[e];
             }
           }
         }
@@ -1209,6 +1231,14 @@ cudaError_t launch_gdn_tc(const GdnParams &p, int grid, bool cooperative, cudaSt
   if (!make_bf16_map(&mq, p.q, p.dk, p.L, p.F, BH, kQTok) || !make_bf16_map(&mk, p.k, p.dk, p.L, p.F, BH, 64) ||
       !make_bf16_map(&mv, p.v, p.dv, p.L, p.F, BH, 64))
     return cudaErrorInvalidValue;
+  if (p.save_maps) {  // the backward's recompute: one unit per frame, no position embedding
+    if (cooperative || p.rope_on || !p.save_states) return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(gdn_tc_kernel<false, false, true>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGdnSmemBytes);
+    if (e != cudaSuccess) return e;
+    gdn_tc_kernel<false, false, true><<<grid, kGThreads, kGdnSmemBytes, st>>>(mq, mk, mv, p);
+    return cudaGetLastError();
+  }
   return p.rope_on ? launch_tc<true>(p, grid, cooperative, st, mq, mk, mv)
                    : launch_tc<false>(p, grid, cooperative, st, mq, mk, mv);
 }

@@ -27,6 +27,7 @@ _lib = None
 # tensor ids: the draw order q, k, v, a, b
 TID_Q, TID_K, TID_V, TID_A, TID_B = 0, 1, 2, 3, 4
 TID_STRIDE_PER_CALL = 8  # streaming call c uses ids base + 8 * c
+TID_DO, TID_STATE_IN, TID_DSTATE_OUT = 5, 6, 7  # the backward's upstream gradients and start state
 
 
 def build(force: bool = False) -> str:
@@ -171,6 +172,19 @@ def inputs(w: Workload, heads=None, call: int = 0, frames: int | None = None) ->
         a = a.reshape(w.B, w.H, F)
         b = b.reshape(w.B, w.H, N)
     return dict(q=q, k=k, v=v, a=a, b=b)
+
+
+
+def grad_inputs(w: Workload, state_in: bool = False, dstate_out: bool = False) -> dict:
+    """Inputs of the backward beyond ``inputs(w)``: dL/do [B, H, N, dv] ~ N(0, 1),
+    and optionally a start state and dL/dstate_out [B, H, dk, dv] ~ N(0, 1)."""
+    nh = w.B * w.H
+    out = dict(d_o=normal(w.seed, TID_DO, 0, nh * w.N * w.dv).reshape(w.B, w.H, w.N, w.dv))
+    out["state_in"] = (normal(w.seed, TID_STATE_IN, 0, nh * w.dk * w.dv).reshape(w.B, w.H, w.dk, w.dv)
+                       if state_in else None)
+    out["dstate_out"] = (normal(w.seed, TID_DSTATE_OUT, 0, nh * w.dk * w.dv).reshape(w.B, w.H, w.dk, w.dv)
+                         if dstate_out else None)
+    return out
 
 
 # ---------------------------------------------------------------- temporal convolution inputs

@@ -199,3 +199,46 @@ def test_no_device_is_reported_without_gpu(lib):
     p16 = ctypes.c_void_p(0x10000)
     rc = lib._lib.gdn_frame_fwd(p16, p16, p16, p16, p16, None, None, p16, 1, 1, 1, 1, 16, 16, ctypes.byref(o))
     assert rc == lib.ERR_NO_DEVICE
+
+
+def test_backward_workspace_and_argument_validation(lib):
+    """gdn_frame_bwd: the workspace holds the recompute's chain scratch, then
+    A_f^T, S_f and G_f of every frame and the dalpha partial sums; host checks
+    come before any device work."""
+    up = lambda x: (x + 255) // 256 * 256
+    B, H, F, L, d = 1, 20, 240, 920, 112
+    fr = B * H * F
+    tc = lib.make_opts(lib.DTYPE_BF16, stream=0)
+    chain = lib.workspace_bytes(lib.OP_GDN, B, H, F, L, d, d, lib.make_opts(lib.DTYPE_BF16, stream=0, segments=1))
+    want = up(chain) + 3 * up(fr * d * d * 4) + up(fr * 7 * 4)
+    assert lib.workspace_bytes(lib.OP_GDN_BWD, B, H, F, L, d, d, tc) == want
+    f32 = lib.make_opts(lib.DTYPE_F32, stream=0)  # the fp32 recompute publishes fp32 states
+    chain32 = 256 + up(fr * 4) + up(fr * d * d * 4)
+    assert lib.workspace_bytes(lib.OP_GDN_BWD, B, H, F, L, d, d, f32) == up(chain32) + 3 * up(fr * d * d * 4) + \
+        up(fr * 7 * 4)
+    raw = lib._lib
+    P = ctypes.c_void_p
+    q, k, v, a, b, do = (P(0x1000000 * (i + 1)) for i in range(6))
+    outs = [P(0x10000000 * (i + 1)) for i in range(6)]
+    ws = P(0x70000000)
+    o = lib.make_opts(lib.DTYPE_BF16, stream=0)
+    o.workspace = 0x70000000
+    o.workspace_bytes = 1 << 40
+    call = lambda *args, sizes=(1, 2, 3, 16, 32, 32): raw.gdn_frame_bwd(*args, *sizes, ctypes.byref(o))
+    assert call(q, k, v, a, b, None, None, None, *outs) == lib.ERR_INVALID_ARG            # null d_o
+    assert call(q, k, v, a, b, None, do, None, None, *outs[1:]) == lib.ERR_INVALID_ARG    # null dq
+    assert call(q, k, v, a, b, None, do, None, *outs, sizes=(1, 2, 3, 16, 128, 32)) == lib.ERR_UNSUPPORTED
+    assert call(q, k, v, a, b, None, do, None, P(0x1000000 + 64), *outs[1:]) == lib.ERR_INVALID_ARG  # dq in q
+    assert call(q, k, v, a, b, None, do, None, outs[0], outs[0], *outs[2:]) == lib.ERR_INVALID_ARG  # dq = dk
+    assert call(P(0x1000004), k, v, a, b, None, do, None, *outs) == lib.ERR_INVALID_ARG  # misaligned
+    o.rope_grid_w = 4
+    assert call(q, k, v, a, b, None, do, None, *outs) == lib.ERR_UNSUPPORTED              # no RoPE backward
+    o.rope_grid_w = 0
+    o.impl = lib.IMPL_SEQ
+    assert call(q, k, v, a, b, None, do, None, *outs) == lib.ERR_INVALID_ARG              # no such recompute
+    o.impl = lib.IMPL_AUTO
+    assert raw.gdn_frame_bwd(q, k, v, a, b, None, do, None, *outs, 1, 2, 3, 16, 32, 32, None) == lib.ERR_INVALID_ARG
+    import torch
+    if not torch.cuda.is_available():  # valid arguments: the device check comes last
+        assert call(q, k, v, a, b, None, do, None, *outs) == lib.ERR_NO_DEVICE
+    del ws
