@@ -341,6 +341,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         extra["configs_other"] = small_configs_leg(args, lib, synth, torch, dev, stream, cpu_on)
         extra["temporal_conv"] = temporal_conv_leg(args, lib, synth, torch, dev, stream, cpu_on)
         extra["softmax_window"] = softmax_window_leg(args, lib, synth, torch, dev, stream, cpu_on)
+        extra["backward"] = backward_leg(args, lib, synth, torch, dev, stream, cpu_on)
     peak, peak_src = measured_peaks()
     alg_bytes = token_heads * BYTES_PER_TOKEN_HEAD + w.B * w.H * (w.F * 4 + w.dk * w.dv * 4)
     achieved = alg_bytes / (ms / 1e3) / 1e9
@@ -729,6 +730,50 @@ def softmax_window_leg(args, lib, synth, torch, dev, stream, cpu_baseline_on):
                                "sample": f"all {H} heads x first {Fs} of {F} frames (windows of 1-4 frames, "
                                          f"below the 4-frame average), {runs} runs in {secs:.1f} s"}
     return out
+
+
+def backward_leg(args, lib, synth, torch, dev, stream, cpu_baseline_on):
+    """gdn_frame_bwd on the headline workload (720p 60 s: B=1, H=20, F=240, L=920,
+    d=112, bf16 q, k, v; fp32 dL/do ~ N(0, 1), no start state).  One call =
+    the forward recompute, the adjoint frame chain and the frame kernel."""
+    w = synth.WORKLOADS["gdn_720p_60s"]
+    x = synth.inputs(w)
+    q, k, v = (torch.from_numpy(x[n]).to(torch.bfloat16).to(dev) for n in "qkv")
+    a, b = (torch.from_numpy(x[n]).to(dev) for n in "ab")
+    d_o = torch.from_numpy(synth.grad_inputs(w)["d_o"]).to(dev)
+    del x
+    opts = lib.make_opts(lib.DTYPE_BF16)
+    ws = lib.alloc_workspace(lib.workspace_bytes(lib.OP_GDN_BWD, w.B, w.H, w.F, w.L, w.dk, w.dv, opts), dev)
+    out = lib.gdn_frame_bwd(q, k, v, a, b, d_o, F=w.F, workspace=ws)
+    call = lambda: lib.gdn_frame_bwd(q, k, v, a, b, d_o, F=w.F, workspace=ws, out=out)
+    for _ in range(2):
+        call()
+    torch.cuda.synchronize()
+    ms = _events_ms(call, 3, stream)
+    th, fh = w.B * w.H * w.N, w.B * w.H * w.F
+    # read q, k, v (bf16), beta and dL/do; write dq, dk, dv and dbeta (fp32); alpha and dalpha per frame
+    alg_bytes = th * (2 * (2 * w.dk + w.dv) + 4 + 4 * w.dv + 4 * (2 * w.dk + w.dv) + 4) + fh * 8
+    peak, peak_src = measured_peaks()
+    res = {"workload": WORKLOAD, "B": w.B, "H": w.H, "F": w.F, "L": w.L, "d": w.dk, "ms": ms,
+           "tokens_per_s": w.B * w.N / (ms / 1e3),
+           "roofline": dict(_roofline(alg_bytes, ms, peak, peak_src), scope="the whole call (three launches)"),
+           "launches_per_call": 3,
+           "l2": "inputs 2.97 GB and dL/do 1.98 GB, larger than L2; no flush needed"}
+    del q, k, v, a, b, d_o, out, ws
+    if cpu_baseline_on:
+        import oracle
+        Fs = 4
+        xs = synth.inputs(w, frames=Fs)
+        ds = synth.normal(w.seed, synth.TID_DO, 0, w.B * w.H * w.N * w.dv).reshape(w.B, w.H, w.N, w.dv)[:, :, :Fs * w.L]
+        qs, ks, vs = (torch.from_numpy(xs[n]).to(torch.bfloat16).float().numpy() for n in "qkv")
+        nthreads = os.cpu_count() or 1
+        tps, runs, secs = _oracle_tokens_per_s(
+            lambda: oracle.gdn_bwd(qs, ks, vs, xs["a"], xs["b"], ds, F=Fs, L=w.L, nthreads=nthreads),
+            w.B * Fs * w.L, target_s=4.0)
+        res["cpu_baseline"] = {"value": tps, "unit": "tokens/s", "cores": nthreads, "kind": "oracle",
+                               "sample": f"the backward of the first {Fs} of {w.F} frames of all {w.H} heads, "
+                                         f"{runs} runs in {secs:.1f} s"}
+    return res
 
 
 def main():

@@ -10,10 +10,10 @@
 //  1. (gdn_tc / gdn_frame_simt, recompute) every frame's map A_f (the ordered
 //     product of the frame's I - beta khat khat^T factors, saved as A_f^T) and
 //     end state S_f, fp32.
-//  2. gdn_bwd_adjoint_kernel: the frame chain in reverse.  With
+//  2. gdn_bwd_qdo_kernel: C_f = Q_f^T dO_f for every frame (frame-parallel);
+//     gdn_bwd_adjoint_kernel: the frame chain in reverse.  With
 //     G_f = dL/dS_f (end of frame f),
-//        G_{F-1} = dS_out + Q_{F-1}^T dO_{F-1},
-//        G_{f-1} = Q_{f-1}^T dO_{f-1} + alpha_f A_f^T G_f,
+//        G_{F-1} = dS_out + C_{F-1},   G_{f-1} = C_{f-1} + alpha_f A_f^T G_f,
 //     dalpha_f = <A_f^T G_f, S_{f-1}>, dS_in = alpha_0 A_0^T G_0.  Columns j
 //     of G are independent: one CTA per (head, 16 columns), serial over
 //     frames.
@@ -33,7 +33,12 @@
 //                      (the in-chunk terms of H_t r_t and S_{t-1} g_t),
 //                      H -= Khat^T diag(beta) Gm;
 //     dk from dkhat through the normalisation.
-// Products run on CUDA cores in fp32 (register tiles over shared memory).
+// Products: bf16 inputs on the tensor cores through warp-level mma.sync
+// (tf32 operands, fp32 accumulation); fp32 inputs on CUDA cores in fp32
+// (register tiles over shared memory), except Q^T dO, on the tensor cores with
+// tf32 high/low operand splits (about fp32).
+#include <type_traits>
+
 #include "launch.h"
 
 namespace gdn {
@@ -41,13 +46,7 @@ namespace bwd {
 
 constexpr int kThreads = 256;
 constexpr int kC = 48;      // tokens per chunk (frame kernel)
-constexpr int kLdC = kC + 1;
-constexpr int kQt = 64;     // tokens per tile (adjoint kernel)
-
-template <typename T>
-__device__ __forceinline__ float ldf(const T *p) {
-  return to_f32(*p);
-}
+constexpr int kQt = 64;     // tokens per tile (Q^T dO kernel)
 
 // acc[i][j] += sum_{k < K} fa(ty + 16 i, k) * fb(k, tx + 16 j): the thread's
 // rows and columns interleave with stride 16, so that a warp reads two rows
@@ -69,6 +68,70 @@ __device__ __forceinline__ void mm(float (&acc)[TM][TN], int K, int ty, int tx, 
   }
 }
 
+// Global -> shared copies of fp32 tiles: dst[r * ldd + c] = scale * src[r * gs + c]
+// for r < rows, c < cols (rows >= nvalid read as zero).  Each thread keeps eight
+// loads in flight before storing, four elements per load where the rows allow
+// it (cols % 4 == 0); loads go through L2 (__ldcg), so that data this kernel
+// wrote earlier is seen.
+__device__ __forceinline__ float4 ld4(const float *p) { return __ldcg(reinterpret_cast<const float4 *>(p)); }
+__device__ __forceinline__ float4 ld4(const __nv_bfloat16 *p) {
+  const uint2 u = __ldcg(reinterpret_cast<const uint2 *>(p));
+  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
+  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
+  return make_float4(a.x, a.y, b.x, b.y);
+}
+__device__ __forceinline__ float ld1(const float *p) { return __ldcg(p); }
+__device__ __forceinline__ float ld1(const __nv_bfloat16 *p) { return __bfloat162float(*p); }
+
+template <typename T>
+__device__ __forceinline__ void tile_load(float *dst, int ldd, const T *src, long gs, int rows, int nvalid, int cols,
+                                          float scale = 1.f) {
+  constexpr int kB = 8;
+  if ((cols & 3) == 0 && (gs & 3) == 0) {
+    const int cv = cols >> 2, nv = rows * cv;
+    for (int base = threadIdx.x; base < nv; base += kB * kThreads) {
+      float4 r[kB];
+#pragma unroll
+      for (int b = 0; b < kB; ++b) {
+        const int e = base + b * kThreads;
+        const int row = e / cv, c4 = e - row * cv;
+        r[b] = (e < nv && row < nvalid) ? ld4(src + row * gs + 4 * c4) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int b = 0; b < kB; ++b) {
+        const int e = base + b * kThreads;
+        if (e < nv) {
+          const int row = e / cv, c4 = e - row * cv;
+          float *d = dst + row * ldd + 4 * c4;
+          d[0] = scale * r[b].x;
+          d[1] = scale * r[b].y;
+          d[2] = scale * r[b].z;
+          d[3] = scale * r[b].w;
+        }
+      }
+    }
+  } else {
+    const int nv = rows * cols;
+    for (int base = threadIdx.x; base < nv; base += kB * kThreads) {
+      float r[kB];
+#pragma unroll
+      for (int b = 0; b < kB; ++b) {
+        const int e = base + b * kThreads;
+        const int row = e / cols, c = e - row * cols;
+        r[b] = (e < nv && row < nvalid) ? ld1(src + row * gs + c) : 0.f;
+      }
+#pragma unroll
+      for (int b = 0; b < kB; ++b) {
+        const int e = base + b * kThreads;
+        if (e < nv) {
+          const int row = e / cols, c = e - row * cols;
+          dst[row * ldd + c] = scale * r[b];
+        }
+      }
+    }
+  }
+}
+
 template <int TM, int TN>
 __device__ __forceinline__ void zero(float (&acc)[TM][TN]) {
 #pragma unroll
@@ -78,14 +141,12 @@ __device__ __forceinline__ void zero(float (&acc)[TM][TN]) {
 }
 
 // ---------------------------------------------------------------- pass 2
-// Shared memory: A_f^T [DP][DP + 1], G [DP][17], q tile [kQt][DP + 1], dO tile [kQt][17].
+// Shared memory: A_f^T [DP][DP + 1], G [DP][17].
 template <int ND>
 struct AdjSmem {
   static constexpr int DP = 16 * ND, LD = DP + 1;
   float a[DP * LD];
   float g[DP * 17];
-  float q[kQt * LD];
-  float d[kQt * 17];
   float red[kThreads / 32];
 };
 
@@ -103,8 +164,6 @@ __global__ void __launch_bounds__(kThreads) gdn_bwd_adjoint_kernel(BwdParams p) 
   const int j = cg * 16 + tx;  // this thread's column of G
   const bool jok = j < dv;
   const long SS = (long)dk * dv;
-  const T *q = static_cast<const T *>(p.q) + (long)bh * N * dk;
-  const float *d_o = p.d_o + (long)bh * N * dv;
 
   for (int e = tid; e < (int)(sizeof(SM) / 4); e += kThreads) reinterpret_cast<float *>(&sm)[e] = 0.f;
   float carry[ND];  // alpha_{f+1} A_{f+1}^T G_{f+1} (or dS_out), rows ty + 16 r
@@ -116,29 +175,13 @@ __global__ void __launch_bounds__(kThreads) gdn_bwd_adjoint_kernel(BwdParams p) 
   __syncthreads();
   for (int f = F - 1; f >= 0; --f) {
     // A_f^T into shared memory
-    const float *mp = p.maps + ((long)bh * F + f) * (long)dk * dk;
-    for (int e = tid; e < dk * dk; e += kThreads) sm.a[(e / dk) * LD + e % dk] = __ldg(mp + e);
-    // C = Q_f^T dO_f (columns of this CTA)
-    float c[ND][1];
-    zero(c);
-    for (int t0 = 0; t0 < L; t0 += kQt) {
-      const int nt = min(kQt, L - t0);
-      const long base = (long)f * L + t0;
-      for (int e = tid; e < nt * dk; e += kThreads) sm.q[(e / dk) * LD + e % dk] = ldf(q + base * dk + e);
-      for (int e = tid; e < nt * 16; e += kThreads) {
-        const int jj = cg * 16 + (e & 15);
-        sm.d[(e >> 4) * 17 + (e & 15)] = jj < dv ? __ldg(d_o + (base + (e >> 4)) * dv + jj) : 0.f;
-      }
-      __syncthreads();
-      mm(c, nt, ty, tx, [&](int m, int k) { return sm.q[k * LD + m]; }, [&](int k, int n) { return sm.d[k * 17 + n]; });
-      __syncthreads();
-    }
-    // G_f = C + carry -> global (for the frame kernel) and shared memory
+    tile_load(sm.a, LD, p.maps + ((long)bh * F + f) * (long)dk * dk, dk, dk, dk, dk);
+    // G_f = C_f + carry (C_f = Q_f^T dO_f, from gdn_bwd_qdo_kernel in gbuf) -> gbuf and shared memory
     float *gout = p.gbuf + ((long)bh * F + f) * SS;
 #pragma unroll
     for (int r = 0; r < ND; ++r) {
       const int i = ty + 16 * r;
-      const float gv = c[r][0] + carry[r];
+      const float gv = (jok && i < dk ? __ldcg(gout + (long)i * dv + j) : 0.f) + carry[r];
       sm.g[i * 17 + tx] = gv;
       if (jok && i < dk) gout[(long)i * dv + j] = gv;
     }
@@ -182,34 +225,33 @@ __global__ void __launch_bounds__(kThreads) gdn_bwd_adjoint_kernel(BwdParams p) 
 }
 
 // ---------------------------------------------------------------- pass 3
-template <int ND>
-struct FrameSmem {
-  static constexpr int DP = 16 * ND, LD = DP + 1;
+// Row-major fp32 tiles with padded rows: LD = DP + PAD for d-wide rows, LDC =
+// kC + PAD for chunk-wide rows (PAD 1 for the CUDA-core products, 4 for the
+// warp-MMA fragments).
+template <int ND, int PAD>
+struct FrameSmemT {
+  static constexpr int DP = 16 * ND, LD = DP + PAD, LDC = kC + PAD;
   float S[DP * LD];   // S[i][j]
   float H[DP * LD];   // H[i][j]
   float K[kC * LD];   // khat rows
   float E[kC * LD];   // v -> E -> R rows
-  float U[kC * LD];   // U rows
+  float U[kC * LD];   // U rows; dkhat rows (warp-MMA kernel)
   float G[kC * LD];   // Khat H -> Gm rows; dO rows for dq
-  float M[kC * kLdC]; // Gram (upper, with diagonal) | Linv (strict lower); then the dkhat coupling M
+  float M[kC * LDC];  // Gram (upper, with diagonal) | Linv (strict lower); then the dkhat coupling M
   float T[3 * 16 * 17];  // inverse scratch
   float b[kC], inv[kC], nrm[kC], red[kC];
 };
+template <int ND>
+using FrameSmem = FrameSmemT<ND, 1>;
 
 // Rows t0 .. t0 + nc - 1 of the frame: khat (normalised), beta, v.
-template <int ND, typename T>
-__device__ __forceinline__ void load_chunk(FrameSmem<ND> &sm, const BwdParams &p, const T *k, const T *v,
-                                           const float *beta, long t0, int nc, int tid) {
-  constexpr int LD = FrameSmem<ND>::LD;
+template <class SM, typename T>
+__device__ __forceinline__ void load_chunk(SM &sm, const BwdParams &p, const T *k, const T *v, const float *beta,
+                                           long t0, int nc, int tid) {
+  constexpr int LD = SM::LD;
   const int dk = p.dk, dv = p.dv;
-  for (int e = tid; e < kC * dk; e += kThreads) {
-    const int t = e / dk, i = e % dk;
-    sm.K[t * LD + i] = t < nc ? ldf(k + (t0 + t) * dk + i) : 0.f;
-  }
-  for (int e = tid; e < kC * dv; e += kThreads) {
-    const int t = e / dv, jj = e % dv;
-    sm.E[t * LD + jj] = t < nc ? ldf(v + (t0 + t) * dv + jj) : 0.f;
-  }
+  tile_load(sm.K, LD, k + t0 * dk, dk, kC, nc, dk);
+  tile_load(sm.E, LD, v + t0 * dv, dv, kC, nc, dv);
   if (tid < kC) {
     const float braw = tid < nc ? beta[t0 + tid] : 0.f;
     sm.b[tid] = tid < nc ? (p.gates_are_logits ? gate_beta(braw) : braw) : 0.f;
@@ -235,28 +277,13 @@ __device__ __forceinline__ void load_chunk(FrameSmem<ND> &sm, const BwdParams &p
   __syncthreads();
 }
 
-// Gram matrix into the upper triangle (with the diagonal) of M, then
 // Linv = (I + N)^-1, N[t][s] = beta_t (khat_t . khat_s) for s < t, into the
-// strict lower triangle (its unit diagonal implied): 16 x 16 blocks, the
-// diagonal ones by forward substitution, the others by block substitution.
-template <int ND>
-__device__ __forceinline__ void gram_inverse(FrameSmem<ND> &sm, int nc, int dk, int tid) {
-  constexpr int LD = FrameSmem<ND>::LD;
-  const int ty = tid >> 4, tx = tid & 15;
-  {
-    float g[3][3];
-    zero(g);
-    mm(g, dk, ty, tx, [&](int m, int k) { return sm.K[m * LD + k]; },
-       [&](int k, int n) { return sm.K[n * LD + k]; });
-#pragma unroll
-    for (int i = 0; i < 3; ++i)
-#pragma unroll
-      for (int jj = 0; jj < 3; ++jj) {
-        const int t = ty + 16 * i, s = tx + 16 * jj;
-        if (s >= t) sm.M[t * kLdC + s] = g[i][jj];
-      }
-  }
-  __syncthreads();
+// strict lower triangle of M (its unit diagonal implied), from the Gram matrix
+// in the upper triangle: 16 x 16 blocks, the diagonal ones by forward
+// substitution, the others by block substitution.
+template <class SM>
+__device__ __forceinline__ void inverse(SM &sm, int nc, int tid) {
+  constexpr int kLdC = SM::LDC;
   // N[t][s] (s < t) = beta_t M[s][t]
   auto Nv = [&](int t, int s) { return sm.b[t] * sm.M[s * kLdC + t]; };
   const int nb = (nc + 15) / 16;
@@ -303,16 +330,38 @@ __device__ __forceinline__ void gram_inverse(FrameSmem<ND> &sm, int nc, int dk, 
   }
 }
 
-// Linv[t][s] with its unit diagonal and zero upper part
+// Gram matrix (CUDA cores) into the upper triangle of M, with the diagonal; then the inverse.
 template <int ND>
-__device__ __forceinline__ float linv(const FrameSmem<ND> &sm, int t, int s) {
-  return s < t ? sm.M[t * kLdC + s] : (s == t ? 1.f : 0.f);
+__device__ __forceinline__ void gram_inverse(FrameSmem<ND> &sm, int nc, int dk, int tid) {
+  constexpr int LD = FrameSmem<ND>::LD, kLdC = FrameSmem<ND>::LDC;
+  const int ty = tid >> 4, tx = tid & 15;
+  {
+    float g[3][3];
+    zero(g);
+    mm(g, dk, ty, tx, [&](int m, int k) { return sm.K[m * LD + k]; },
+       [&](int k, int n) { return sm.K[n * LD + k]; });
+#pragma unroll
+    for (int i = 0; i < 3; ++i)
+#pragma unroll
+      for (int jj = 0; jj < 3; ++jj) {
+        const int t = ty + 16 * i, s = tx + 16 * jj;
+        if (s >= t) sm.M[t * kLdC + s] = g[i][jj];
+      }
+  }
+  __syncthreads();
+  inverse(sm, nc, tid);
+}
+
+// Linv[t][s] with its unit diagonal and zero upper part
+template <class SM>
+__device__ __forceinline__ float linv(const SM &sm, int t, int s) {
+  return s < t ? sm.M[t * SM::LDC + s] : (s == t ? 1.f : 0.f);
 }
 
 template <int ND, typename T>
 __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_frame_kernel(BwdParams p) {
   using SM = FrameSmem<ND>;
-  constexpr int LD = SM::LD;
+  constexpr int LD = SM::LD, kLdC = SM::LDC;
   extern __shared__ __align__(16) unsigned char smem_raw[];
   SM &sm = *reinterpret_cast<SM *>(smem_raw);
   const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
@@ -337,12 +386,8 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_frame_kernel(BwdParams p)
   {
     const float *sprev = f > 0 ? p.states + ((long)bh * F + f - 1) * SS
                                : (p.state_in ? p.state_in + (long)bh * SS : nullptr);
-    const float *gf = p.gbuf + ((long)bh * F + f) * SS;
-    for (int e = tid; e < dk * dv; e += kThreads) {
-      const int i = e / dv, jj = e % dv;
-      sm.S[i * LD + jj] = sprev ? al * __ldg(sprev + e) : 0.f;
-      sm.H[i * LD + jj] = __ldg(gf + e);
-    }
+    if (sprev) tile_load(sm.S, LD, sprev, dv, dk, dk, dv, al);
+    tile_load(sm.H, LD, p.gbuf + ((long)bh * F + f) * SS, dv, dk, dk, dv);
   }
   __syncthreads();
 
@@ -350,7 +395,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_frame_kernel(BwdParams p)
   for (int c = 0; c < nch; ++c) {
     const long t0 = (long)f * L + c * kC;
     const int nc = min(kC, L - c * kC);
-    load_chunk<ND, T>(sm, p, k, v, beta, t0, nc, tid);
+    load_chunk(sm, p, k, v, beta, t0, nc, tid);
     gram_inverse<ND>(sm, nc, dk, tid);
     {  // E = V - Khat S
       float a[3][ND];
@@ -395,10 +440,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_frame_kernel(BwdParams p)
   for (int c = 0; c < nch; ++c) {
     const long t0 = (long)f * L + c * kC;
     const int nc = min(kC, L - c * kC);
-    for (int e = tid; e < kC * dv; e += kThreads) {
-      const int t = e / dv, jj = e % dv;
-      sm.G[t * LD + jj] = t < nc ? __ldg(d_o + (t0 + t) * dv + jj) : 0.f;
-    }
+    tile_load(sm.G, LD, d_o + t0 * dv, dv, kC, nc, dv);
     __syncthreads();
     float a[3][ND];
     zero(a);
@@ -418,11 +460,8 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_frame_kernel(BwdParams p)
   for (int c = nch - 1; c >= 0; --c) {
     const long t0 = (long)f * L + c * kC;
     const int nc = min(kC, L - c * kC);
-    for (int e = tid; e < kC * dv; e += kThreads) {
-      const int t = e / dv, jj = e % dv;
-      sm.U[t * LD + jj] = t < nc ? dvg[(t0 + t) * dv + jj] : 0.f;
-    }
-    load_chunk<ND, T>(sm, p, k, v, beta, t0, nc, tid);  // (its barriers order the U loads too)
+    tile_load(sm.U, LD, dvg + t0 * dv, dv, kC, nc, dv);
+    load_chunk(sm, p, k, v, beta, t0, nc, tid);  // (its barriers order the U loads too)
     {  // S -= Khat^T U: the chunk's start state
       float a[ND][ND];
       zero(a);
@@ -577,20 +616,380 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_frame_kernel(BwdParams p)
   }
 }
 
+// ---------------------------------------------------------------- pass 3 on warp MMAs (bf16 inputs)
+// The same frame kernel with every product on the tensor cores through
+// mma.sync m16n8k8 (tf32 operands, fp32 accumulation).  NP = 1: operands
+// rounded to tf32 (10-bit significands); NP = 3: each operand split into tf32
+// high and low parts and the three leading products summed (about fp32).
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return r;
+}
+__device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+// acc += the (16 MT) x (8 NT) block at (m0, n0) of sum_{k < K} fa(m, k) fb(k, n),
+// in the m16n8 accumulator layout (lane: g = lane / 4 rows g, g + 8; t = lane % 4
+// columns 2t, 2t + 1).  A fragments: rows g, g + 8, k = t, t + 4; B: k = t, t + 4, column g.
+template <int MT, int NT, int NP, class FA, class FB>
+__device__ __forceinline__ void wmm(float (&acc)[MT][NT][4], int m0, int n0, int K, FA fa, FB fb) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+#pragma unroll 1
+  for (int k0 = 0; k0 < K; k0 += 8) {
+    const int ka = k0 + t, kb = k0 + t + 4;
+    const bool va = ka < K, vb = kb < K;
+    uint32_t ah[MT][4], al[MT][4], bh[NT][2], bl[NT][2];
+#pragma unroll
+    for (int i = 0; i < MT; ++i) {
+      const int r = m0 + 16 * i + g;
+      const float x[4] = {va ? fa(r, ka) : 0.f, va ? fa(r + 8, ka) : 0.f, vb ? fa(r, kb) : 0.f,
+                          vb ? fa(r + 8, kb) : 0.f};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        ah[i][e] = to_tf32(x[e]);
+        if (NP == 3) al[i][e] = to_tf32(x[e] - __uint_as_float(ah[i][e]));
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < NT; ++j) {
+      const int n = n0 + 8 * j + g;
+      const float y[2] = {va ? fb(ka, n) : 0.f, vb ? fb(kb, n) : 0.f};
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        bh[j][e] = to_tf32(y[e]);
+        if (NP == 3) bl[j][e] = to_tf32(y[e] - __uint_as_float(bh[j][e]));
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < MT; ++i)
+#pragma unroll
+      for (int j = 0; j < NT; ++j) {
+        mma_tf32(acc[i][j], ah[i], bh[j]);
+        if (NP == 3) {
+          mma_tf32(acc[i][j], ah[i], bl[j]);
+          mma_tf32(acc[i][j], al[i], bh[j]);
+        }
+      }
+  }
+}
+
+template <int MT, int NT, class EP>
+__device__ __forceinline__ void each(const float (&acc)[MT][NT][4], int m0, int n0, EP ep) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int i = 0; i < MT; ++i)
+#pragma unroll
+    for (int j = 0; j < NT; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) ep(m0 + 16 * i + g + 8 * (e >> 1), n0 + 8 * j + 2 * t + (e & 1), acc[i][j][e]);
+}
+
+// An M x N product over all warps, blocks of (16 MT) x (8 NT) taken round-robin;
+// ep(m, n, value) for every element inside M x N.
+template <int MT, int NT, int NP, class FA, class FB, class EP>
+__device__ __forceinline__ void wrun(int M, int N, int K, FA fa, FB fb, EP ep) {
+  const int warp = threadIdx.x >> 5;
+  const int nmb = (M + 16 * MT - 1) / (16 * MT), nnb = (N + 8 * NT - 1) / (8 * NT);
+  for (int blk = warp; blk < nmb * nnb; blk += kThreads / 32) {
+    const int m0 = (blk % nmb) * 16 * MT, n0 = (blk / nmb) * 8 * NT;
+    float acc[MT][NT][4];
+#pragma unroll
+    for (int i = 0; i < MT; ++i)
+#pragma unroll
+      for (int j = 0; j < NT; ++j)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[i][j][e] = 0.f;
+    wmm<MT, NT, NP>(acc, m0, n0, K, fa, fb);
+    each(acc, m0, n0, [&](int m, int n, float v) {
+      if (m < M && n < N) ep(m, n, v);
+    });
+  }
+}
+
+// The same with at most one block per warp and a barrier between the products
+// and the epilogue (for results written over an operand).  All threads call it.
+template <int MT, int NT, int NP, class FA, class FB, class EP>
+__device__ __forceinline__ void wrun_sync(int M, int N, int K, FA fa, FB fb, EP ep) {
+  const int warp = threadIdx.x >> 5;
+  const int nmb = (M + 16 * MT - 1) / (16 * MT), nnb = (N + 8 * NT - 1) / (8 * NT);
+  const bool has = warp < nmb * nnb;
+  const int m0 = (warp % nmb) * 16 * MT, n0 = (warp / nmb) * 8 * NT;
+  float acc[MT][NT][4];
+#pragma unroll
+  for (int i = 0; i < MT; ++i)
+#pragma unroll
+    for (int j = 0; j < NT; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[i][j][e] = 0.f;
+  if (has) wmm<MT, NT, NP>(acc, m0, n0, K, fa, fb);
+  __syncthreads();
+  if (has)
+    each(acc, m0, n0, [&](int m, int n, float v) {
+      if (m < M && n < N) ep(m, n, v);
+    });
+}
+
+template <int ND, typename T, int NP>
+__global__ void __launch_bounds__(kThreads, 1) gdn_bwd_frame_mma_kernel(BwdParams p) {
+  using SM = FrameSmemT<ND, 4>;
+  constexpr int LD = SM::LD, LDC = SM::LDC;
+  static_assert(ND <= 8, "one 16-column block per warp");
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  SM &sm = *reinterpret_cast<SM *>(smem_raw);
+  const int tid = threadIdx.x;
+  const int dk = p.dk, dv = p.dv, L = p.L, F = p.F;
+  const long N = (long)F * L;
+  const long SS = (long)dk * dv;
+  const int f = blockIdx.x % F, bh = blockIdx.x / F;
+  const T *k = static_cast<const T *>(p.k) + (long)bh * N * dk;
+  const T *v = static_cast<const T *>(p.v) + (long)bh * N * dv;
+  const float *beta = p.beta + (long)bh * N;
+  const float *d_o = p.d_o + (long)bh * N * dv;
+  float *dq = p.dq + (long)bh * N * dk;
+  float *dkg = p.dk_out + (long)bh * N * dk;
+  float *dvg = p.dv_out + (long)bh * N * dv;  // also the U scratch of the forward sweep
+  float *dbg = p.dbeta + (long)bh * N;
+  const int nch = (L + kC - 1) / kC;
+  const int warp = tid >> 5, lane = tid & 31;
+
+  for (int e = tid; e < (int)(sizeof(SM) / 4); e += kThreads) reinterpret_cast<float *>(&sm)[e] = 0.f;
+  __syncthreads();
+  const float araw = p.alpha[(long)bh * F + f];
+  const float al = p.gates_are_logits ? gate_alpha(araw) : araw;
+  {
+    const float *sprev = f > 0 ? p.states + ((long)bh * F + f - 1) * SS
+                               : (p.state_in ? p.state_in + (long)bh * SS : nullptr);
+    if (sprev) tile_load(sm.S, LD, sprev, dv, dk, dk, dv, al);
+    tile_load(sm.H, LD, p.gbuf + ((long)bh * F + f) * SS, dv, dk, dk, dv);
+  }
+  __syncthreads();
+  auto Krow = [&](int m, int kk) { return sm.K[m * LD + kk]; };  // Khat (t, i)
+  auto Kcol = [&](int m, int kk) { return sm.K[kk * LD + m]; };  // Khat^T (i, t)
+  auto gram = [&]() {
+    wrun<1, 2, NP>(kC, kC, dk, Krow, [&](int kk, int n) { return sm.K[n * LD + kk]; }, [&](int m, int n, float x) {
+      if (n >= m) sm.M[m * LDC + n] = x;
+    });
+  };
+
+  // ---- forward sweep
+  for (int c = 0; c < nch; ++c) {
+    const long t0 = (long)f * L + c * kC;
+    const int nc = min(kC, L - c * kC);
+    load_chunk(sm, p, k, v, beta, t0, nc, tid);
+    gram();
+    __syncthreads();
+    inverse(sm, nc, tid);
+    wrun<3, 2, NP>(kC, dv, dk, Krow, [&](int kk, int n) { return sm.S[kk * LD + n]; },
+                   [&](int m, int n, float x) { sm.E[m * LD + n] -= x; });  // E = V - Khat S
+    __syncthreads();
+    wrun<3, 2, NP>(kC, dv, nc, [&](int m, int s2) { return linv(sm, m, s2) * sm.b[s2]; },
+                   [&](int s2, int n) { return sm.E[s2 * LD + n]; }, [&](int m, int n, float x) {
+                     sm.U[m * LD + n] = x;  // U = Linv diag(beta) E
+                     if (m < nc) dvg[(t0 + m) * dv + n] = x;
+                   });
+    __syncthreads();
+    wrun<ND, 2, NP>(dk, dv, nc, Kcol, [&](int t, int n) { return sm.U[t * LD + n]; },
+                    [&](int m, int n, float x) { sm.S[m * LD + n] += x; });  // S += Khat^T U
+    __syncthreads();
+  }
+
+  // ---- dq = dO S_f^T
+  for (int c = 0; c < nch; ++c) {
+    const long t0 = (long)f * L + c * kC;
+    const int nc = min(kC, L - c * kC);
+    tile_load(sm.G, LD, d_o + t0 * dv, dv, kC, nc, dv);
+    __syncthreads();
+    wrun<3, 2, NP>(kC, dk, dv, [&](int m, int jj) { return sm.G[m * LD + jj]; },
+                   [&](int jj, int n) { return sm.S[n * LD + jj]; }, [&](int m, int n, float x) {
+                     if (m < nc) dq[(t0 + m) * dk + n] = x;
+                   });
+    __syncthreads();
+  }
+
+  // ---- reverse sweep
+  for (int c = nch - 1; c >= 0; --c) {
+    const long t0 = (long)f * L + c * kC;
+    const int nc = min(kC, L - c * kC);
+    tile_load(sm.U, LD, dvg + t0 * dv, dv, kC, nc, dv);
+    load_chunk(sm, p, k, v, beta, t0, nc, tid);
+    wrun<ND, 2, NP>(dk, dv, nc, Kcol, [&](int t, int n) { return sm.U[t * LD + n]; },
+                    [&](int m, int n, float x) { sm.S[m * LD + n] -= x; });  // the chunk's start state
+    gram();
+    __syncthreads();
+    inverse(sm, nc, tid);
+    wrun<3, 2, NP>(kC, dv, dk, Krow, [&](int kk, int n) { return sm.S[kk * LD + n]; },
+                   [&](int m, int n, float x) { sm.E[m * LD + n] -= x; });  // E = V - Khat S
+    __syncthreads();
+    wrun<3, 2, NP>(kC, dv, nc, [&](int m, int s2) { return s2 < m ? sm.M[s2 * LDC + m] : 0.f; },
+                   [&](int s2, int n) { return sm.U[s2 * LD + n]; },
+                   [&](int m, int n, float x) { sm.E[m * LD + n] -= x; });  // R = E - strict_lower(Gram) U
+    wrun<3, 2, NP>(kC, dv, dk, Krow, [&](int kk, int n) { return sm.H[kk * LD + n]; },
+                   [&](int m, int n, float x) { sm.G[m * LD + n] = x; });  // Khat H
+    __syncthreads();
+    wrun_sync<3, 2, NP>(kC, dv, nc, [&](int m, int s2) { return linv(sm, s2, m); },
+                        [&](int s2, int n) { return sm.G[s2 * LD + n]; }, [&](int m, int n, float x) {
+                          sm.G[m * LD + n] = x;  // Gm = Linv^T (Khat H)
+                          if (m < nc) dvg[(t0 + m) * dv + n] = sm.b[m] * x;
+                        });
+    __syncthreads();
+    for (int t = warp; t < nc; t += kThreads / 32) {  // dbeta_t = g_t . R_t
+      float s2 = 0.f;
+      for (int jj = lane; jj < dv; jj += 32) s2 = fmaf(sm.G[t * LD + jj], sm.E[t * LD + jj], s2);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) s2 += __shfl_xor_sync(0xffffffffu, s2, off);
+      if (lane == 0) {
+        const float bt = sm.b[t];
+        dbg[t0 + t] = p.gates_are_logits ? s2 * bt * (1.f - bt) : s2;
+      }
+    }
+    {  // M: upper beta_s R_t . g_s, lower g_t . u_s (Gram and Linv are dead)
+      for (int blk = warp; blk < 9; blk += kThreads / 32) {
+        const int m0 = (blk % 3) * 16, n0 = (blk / 3) * 16;
+        float r1[1][2][4] = {}, r2[1][2][4] = {};
+        wmm<1, 2, NP>(r1, m0, n0, dv, [&](int m, int jj) { return sm.E[m * LD + jj]; },
+                      [&](int jj, int n) { return sm.G[n * LD + jj]; });
+        wmm<1, 2, NP>(r2, m0, n0, dv, [&](int m, int jj) { return sm.G[m * LD + jj]; },
+                      [&](int jj, int n) { return sm.U[n * LD + jj]; });
+        each(r1, m0, n0, [&](int m, int n, float x) {
+          if (n > m) sm.M[m * LDC + n] = sm.b[n] * x;
+          else if (n == m) sm.M[m * LDC + n] = 0.f;
+        });
+        each(r2, m0, n0, [&](int m, int n, float x) {
+          if (n < m) sm.M[m * LDC + n] = x;
+        });
+      }
+    }
+    __syncthreads();
+    {  // dkhat = diag(beta) (R H^T - Gm S^T - M Khat) -> U rows (U is dead)
+      const bool has = warp < ND;
+      float a[3][2][4] = {};
+      if (has) {
+        const int n0 = warp * 16;
+        wmm<3, 2, NP>(a, 0, n0, dv, [&](int m, int jj) { return sm.E[m * LD + jj]; },
+                      [&](int jj, int n) { return sm.H[n * LD + jj]; });
+        wmm<3, 2, NP>(a, 0, n0, dv, [&](int m, int jj) { return -sm.G[m * LD + jj]; },
+                      [&](int jj, int n) { return sm.S[n * LD + jj]; });
+        wmm<3, 2, NP>(a, 0, n0, nc, [&](int m, int s2) { return -sm.M[m * LDC + s2]; },
+                      [&](int s2, int n) { return sm.K[s2 * LD + n]; });
+      }
+      __syncthreads();
+      if (has)
+        each(a, 0, warp * 16, [&](int m, int n, float x) { sm.U[m * LD + n] = sm.b[m] * x; });
+    }
+    __syncthreads();
+    for (int t = warp; t < nc; t += kThreads / 32) {
+      // dk = (dkhat - khat (khat . dkhat)) / ||k|| (||k|| > eps), dkhat / eps (otherwise)
+      float dot = 0.f;
+      for (int i = lane; i < dk; i += 32) dot = fmaf(sm.K[t * LD + i], sm.U[t * LD + i], dot);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
+      const bool proj = sm.nrm[t] > kKeyNormEps;
+      const float sc = sm.inv[t];
+      for (int i = lane; i < dk; i += 32) {
+        const float gk = proj ? sm.U[t * LD + i] - sm.K[t * LD + i] * dot : sm.U[t * LD + i];
+        dkg[(t0 + t) * dk + i] = gk * sc;
+      }
+    }
+    wrun<ND, 2, NP>(dk, dv, nc, [&](int m, int t) { return sm.K[t * LD + m] * sm.b[t]; },
+                    [&](int t, int n) { return sm.G[t * LD + n]; },
+                    [&](int m, int n, float x) { sm.H[m * LD + n] -= x; });  // H -= Khat^T diag(beta) Gm
+    __syncthreads();
+  }
+  if (tid == 0) {
+    const int ncg = (dv + 15) / 16;
+    float s2 = 0.f;
+    for (int cg = 0; cg < ncg; ++cg) s2 += p.dal_part[((long)bh * F + f) * ncg + cg];
+    p.dalpha[(long)bh * F + f] = p.gates_are_logits ? s2 * (-al * (1.f - al)) : s2;
+  }
+}
+
+// ---------------------------------------------------------------- pass 2a
+// C_f = Q_f^T dO_f for every frame, into gbuf (the adjoint chain adds its carry
+// there): one CTA per frame, 64-token tiles of q and dO in shared memory, warp
+// MMAs (tf32 operands with NP passes) over all d_k rows and 16 columns per warp.
+template <int ND>
+struct QdoSmem {
+  static constexpr int DP = 16 * ND, LD = DP + 8;  // LD % 32 in {8, 24}: conflict-free k-major fragments
+  float q[kQt * LD];
+  float d[kQt * LD];
+};
+
+template <int ND, typename T, int NP>
+__global__ void __launch_bounds__(kThreads) gdn_bwd_qdo_kernel(BwdParams p) {
+  using SM = QdoSmem<ND>;
+  constexpr int LD = SM::LD;
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  SM &sm = *reinterpret_cast<SM *>(smem_raw);
+  const int dk = p.dk, dv = p.dv, L = p.L, F = p.F;
+  const long N = (long)F * L;
+  const int f = blockIdx.x % F, bh = blockIdx.x / F;
+  const T *q = static_cast<const T *>(p.q) + (long)bh * N * dk + (long)f * L * dk;
+  const float *d_o = p.d_o + (long)bh * N * dv + (long)f * L * dv;
+  const int warp = threadIdx.x >> 5;
+  const bool has = warp < (dv + 15) / 16;
+  float acc[ND][2][4];
+#pragma unroll
+  for (int i = 0; i < ND; ++i)
+#pragma unroll
+    for (int j = 0; j < 2; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[i][j][e] = 0.f;
+  for (int t0 = 0; t0 < L; t0 += kQt) {
+    const int nt = min(kQt, L - t0);
+    tile_load(sm.q, LD, q + (long)t0 * dk, dk, nt, nt, dk);
+    tile_load(sm.d, LD, d_o + (long)t0 * dv, dv, nt, nt, dv);
+    __syncthreads();
+    if (has)
+      wmm<ND, 2, NP>(acc, 0, warp * 16, nt, [&](int m, int t) { return sm.q[t * LD + m]; },
+                     [&](int t, int n) { return sm.d[t * LD + n]; });
+    __syncthreads();
+  }
+  float *c = p.gbuf + ((long)bh * F + f) * (long)dk * dv;
+  if (has)
+    each(acc, 0, warp * 16, [&](int m, int n, float x) {
+      if (m < dk && n < dv) c[(long)m * dv + n] = x;
+    });
+}
+
+// tf32 passes of the warp-MMA frame kernel (bf16 inputs): 3 = high/low split
+constexpr int kMmaPasses = 1;
+
 template <int ND, typename T>
 cudaError_t launch_nd(const BwdParams &p, cudaStream_t st) {
-  const size_t sa = sizeof(AdjSmem<ND>), sf = sizeof(FrameSmem<ND>);
-  cudaError_t e = cudaFuncSetAttribute(gdn_bwd_adjoint_kernel<ND, T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)sa);
+  constexpr bool mma = std::is_same<T, __nv_bfloat16>::value;
+  const size_t sa = sizeof(AdjSmem<ND>);
+  const size_t sf = mma ? sizeof(FrameSmemT<ND, 4>) : sizeof(FrameSmem<ND>);
+  const size_t sq = sizeof(QdoSmem<ND>);
+  constexpr int qnp = mma ? kMmaPasses : 3;  // fp32 inputs: high/low split (about fp32)
+  cudaError_t e = cudaFuncSetAttribute(gdn_bwd_qdo_kernel<ND, T, qnp>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)sq);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(gdn_bwd_frame_kernel<ND, T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sf);
+  e = cudaFuncSetAttribute(gdn_bwd_adjoint_kernel<ND, T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sa);
   if (e != cudaSuccess) return e;
   const int BH = p.B * p.H;
   const int ncg = (p.dv + 15) / 16;
+  gdn_bwd_qdo_kernel<ND, T, qnp><<<(unsigned)((long)BH * p.F), kThreads, sq, st>>>(p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
   gdn_bwd_adjoint_kernel<ND, T><<<BH * ncg, kThreads, sa, st>>>(p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  gdn_bwd_frame_kernel<ND, T><<<(unsigned)((long)BH * p.F), kThreads, sf, st>>>(p);
+  const unsigned grid = (unsigned)((long)BH * p.F);
+  if constexpr (mma) {
+    e = cudaFuncSetAttribute(gdn_bwd_frame_mma_kernel<ND, T, kMmaPasses>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sf);
+    if (e != cudaSuccess) return e;
+    gdn_bwd_frame_mma_kernel<ND, T, kMmaPasses><<<grid, kThreads, sf, st>>>(p);
+  } else {
+    e = cudaFuncSetAttribute(gdn_bwd_frame_kernel<ND, T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sf);
+    if (e != cudaSuccess) return e;
+    gdn_bwd_frame_kernel<ND, T><<<grid, kThreads, sf, st>>>(p);
+  }
   return cudaGetLastError();
 }
 
