@@ -208,16 +208,22 @@ int pick_bwd_fwd_impl(const gdn_opts_t *o, int dk, int dv) {
 // Backward workspace: the recompute's chain scratch, then A_f^T and S_f of every
 // frame, G_f of every frame, and the per-column-group dalpha partial sums.
 struct BwdLayout {
-  size_t maps, states, gbuf, part, total;
+  size_t maps, states, gbuf, part, linv, rbuf, total;
 };
-BwdLayout bwd_layout(const gdn_opts_t *o, int B, int H, int F, int dk, int dv) {
+BwdLayout bwd_layout(const gdn_opts_t *o, int B, int H, int F, int L, int dk, int dv) {
   BwdLayout w;
   const size_t fr = (size_t)B * H * F;
   w.maps = align_up(gdn_ws_bytes_p(pick_bwd_fwd_impl(o, dk, dv), o, B, H, F, dk, dv, 1), 256);
   w.states = w.maps + align_up(sizeof(float) * fr * dk * dk, 256);
   w.gbuf = w.states + align_up(sizeof(float) * fr * dk * dv, 256);
   w.part = w.gbuf + align_up(sizeof(float) * fr * dk * dv, 256);
-  w.total = w.part + align_up(sizeof(float) * fr * ((dv + 15) / 16), 256);
+  w.linv = w.part + align_up(sizeof(float) * fr * ((dv + 15) / 16), 256);
+  w.rbuf = w.linv;
+  w.total = w.linv;
+  if (o->in_dtype == GDN_DTYPE_BF16) {  // the tensor-core frame kernel keeps each chunk's Linv and residuals
+    w.rbuf = w.linv + align_up(sizeof(float) * fr * gdn_bwd_chunks(L) * 48 * 48, 256);
+    w.total = w.rbuf + (dv > dk ? align_up(sizeof(float) * fr * L * dv, 256) : 0);
+  }
   return w;
 }
 }  // namespace
@@ -227,7 +233,7 @@ extern "C" size_t gdn_workspace_bytes(int op, int B, int H, int F, int L, int dk
   if (!opts || check_sizes(B, H, F, L, dk, dv) != GDN_OK) return 0;
   if (op == GDN_OP_GDN) return gdn_ws_bytes(pick_gdn_impl(opts, dk, dv), opts, B, H, F, L, dk, dv);
   if (op == GDN_OP_RELU_LA) return relu_ws_bytes(B, H, F, dk, dv);
-  if (op == GDN_OP_GDN_BWD) return bwd_layout(opts, B, H, F, dk, dv).total;
+  if (op == GDN_OP_GDN_BWD) return bwd_layout(opts, B, H, F, L, dk, dv).total;
   return 0;
 }
 
@@ -269,7 +275,7 @@ extern "C" int gdn_frame_bwd(const void *q, const void *k, const void *v, const 
   const int fimpl = pick_bwd_fwd_impl(opts, dk, dv);
   if (fimpl == GDN_IMPL_TC && (opts->in_dtype != GDN_DTYPE_BF16 || !gdn_tc_supported(dk, dv)))
     return GDN_ERR_UNSUPPORTED;
-  const BwdLayout w = bwd_layout(opts, B, H, F, dk, dv);
+  const BwdLayout w = bwd_layout(opts, B, H, F, L, dk, dv);
   if (!opts->workspace || opts->workspace_bytes < w.total) return GDN_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(opts->workspace) & 255u) != 0) return GDN_ERR_INVALID_ARG;
   char *ws = static_cast<char *>(opts->workspace);
@@ -306,6 +312,8 @@ extern "C" int gdn_frame_bwd(const void *q, const void *k, const void *v, const 
   b.maps = maps; b.states = states;
   b.gbuf = reinterpret_cast<float *>(ws + w.gbuf);
   b.dal_part = reinterpret_cast<float *>(ws + w.part);
+  b.linv_buf = reinterpret_cast<float *>(ws + w.linv);
+  b.rbuf = w.total > w.rbuf ? reinterpret_cast<float *>(ws + w.rbuf) : nullptr;
   b.dq = dq; b.dk_out = dk_out; b.dv_out = dv_out; b.dalpha = dalpha; b.dbeta = dbeta; b.dstate_in = dstate_in;
   b.B = B; b.H = H; b.F = F; b.L = L; b.dk = dk; b.dv = dv;
   b.gates_are_logits = p.gates_are_logits;

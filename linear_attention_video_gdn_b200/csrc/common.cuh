@@ -127,6 +127,8 @@ struct BwdParams {
   const float *states;          // [F][dk][dv]: S_f, the end state of every frame
   float *gbuf;                  // [F][dk][dv]: G_f = dL/dS_f (adjoint chain -> frame kernel)
   float *dal_part;              // [F][ceil(dv / 16)]: dalpha_f per column group
+  float *linv_buf;              // [F][chunks][48][48]: each chunk's Linv (bf16-input frame kernel)
+  float *rbuf;                  // [N][dv]: each token's residual, or null (then kept in dk_out's rows, dv <= dk)
   float *dq, *dk_out, *dv_out;  // [N][dk], [N][dk], [N][dv]; dv_out is also scratch
   float *dalpha, *dbeta;        // [F], [N]
   float *dstate_in;             // [dk][dv] or null

@@ -132,6 +132,13 @@ __device__ __forceinline__ void tile_load(float *dst, int ldd, const T *src, lon
   }
 }
 
+// Ask L2 for [base, base + bytes) (128-byte lines spread over the block's threads).
+__device__ __forceinline__ void prefetch_l2(const void *base, long bytes) {
+  const char *b = static_cast<const char *>(base);
+  for (long off = (long)threadIdx.x * 128; off < bytes; off += (long)kThreads * 128)
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(b + off));
+}
+
 template <int TM, int TN>
 __device__ __forceinline__ void zero(float (&acc)[TM][TN]) {
 #pragma unroll
@@ -150,15 +157,14 @@ struct AdjSmem {
   float red[kThreads / 32];
 };
 
-template <int ND, typename T>
+template <int ND>
 __global__ void __launch_bounds__(kThreads) gdn_bwd_adjoint_kernel(BwdParams p) {
   using SM = AdjSmem<ND>;
   constexpr int LD = SM::LD;
   extern __shared__ __align__(16) unsigned char smem_raw[];
   SM &sm = *reinterpret_cast<SM *>(smem_raw);
   const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
-  const int dk = p.dk, dv = p.dv, L = p.L, F = p.F;
-  const long N = (long)F * L;
+  const int dk = p.dk, dv = p.dv, F = p.F;
   const int ncg = (dv + 15) / 16;
   const int bh = blockIdx.x / ncg, cg = blockIdx.x % ncg;
   const int j = cg * 16 + tx;  // this thread's column of G
@@ -244,14 +250,14 @@ struct FrameSmemT {
 template <int ND>
 using FrameSmem = FrameSmemT<ND, 1>;
 
-// Rows t0 .. t0 + nc - 1 of the frame: khat (normalised), beta, v.
-template <class SM, typename T>
+// Rows t0 .. t0 + nc - 1 of the frame: khat (normalised), beta and (kV) v.
+template <class SM, typename T, bool kV = true>
 __device__ __forceinline__ void load_chunk(SM &sm, const BwdParams &p, const T *k, const T *v, const float *beta,
                                            long t0, int nc, int tid) {
   constexpr int LD = SM::LD;
   const int dk = p.dk, dv = p.dv;
   tile_load(sm.K, LD, k + t0 * dk, dk, kC, nc, dk);
-  tile_load(sm.E, LD, v + t0 * dv, dv, kC, nc, dv);
+  if (kV) tile_load(sm.E, LD, v + t0 * dv, dv, kC, nc, dv);
   if (tid < kC) {
     const float braw = tid < nc ? beta[t0 + tid] : 0.f;
     sm.b[tid] = tid < nc ? (p.gates_are_logits ? gate_beta(braw) : braw) : 0.f;
@@ -756,6 +762,11 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_frame_mma_kernel(BwdParam
   float *dbg = p.dbeta + (long)bh * N;
   const int nch = (L + kC - 1) / kC;
   const int warp = tid >> 5, lane = tid & 31;
+  // each token's residual R (kept by the forward sweep for the reverse one): in the
+  // workspace, or in dk_out's rows (dv <= dk), which the reverse sweep overwrites after reading
+  float *rdst = p.rbuf ? p.rbuf + (long)bh * N * dv : dkg;
+  const int rld = p.rbuf ? dv : dk;
+  float *lbuf = p.linv_buf + ((long)bh * F + f) * nch * (kC * kC);  // each chunk's Linv, [48][48]
 
   for (int e = tid; e < (int)(sizeof(SM) / 4); e += kThreads) reinterpret_cast<float *>(&sm)[e] = 0.f;
   __syncthreads();
@@ -780,6 +791,11 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_frame_mma_kernel(BwdParam
   for (int c = 0; c < nch; ++c) {
     const long t0 = (long)f * L + c * kC;
     const int nc = min(kC, L - c * kC);
+    if (c + 1 < nch) {
+      const int nn = min(kC, L - (c + 1) * kC);
+      prefetch_l2(k + (t0 + kC) * dk, (long)nn * dk * sizeof(T));
+      prefetch_l2(v + (t0 + kC) * dv, (long)nn * dv * sizeof(T));
+    }
     load_chunk(sm, p, k, v, beta, t0, nc, tid);
     gram();
     __syncthreads();
@@ -795,6 +811,12 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_frame_mma_kernel(BwdParam
     __syncthreads();
     wrun<ND, 2, NP>(dk, dv, nc, Kcol, [&](int t, int n) { return sm.U[t * LD + n]; },
                     [&](int m, int n, float x) { sm.S[m * LD + n] += x; });  // S += Khat^T U
+    // R = E - strict_lower(Gram) U, and Linv, kept for the reverse sweep
+    wrun<3, 2, NP>(kC, dv, nc, [&](int m, int s2) { return s2 < m ? sm.M[s2 * LDC + m] : 0.f; },
+                   [&](int s2, int n) { return sm.U[s2 * LD + n]; }, [&](int m, int n, float x) {
+                     if (m < nc) rdst[(t0 + m) * rld + n] = sm.E[m * LD + n] - x;
+                   });
+    for (int e = tid; e < kC * kC; e += kThreads) lbuf[c * (kC * kC) + e] = sm.M[(e / kC) * LDC + e % kC];
     __syncthreads();
   }
 
@@ -811,23 +833,22 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_frame_mma_kernel(BwdParam
     __syncthreads();
   }
 
-  // ---- reverse sweep
+  // ---- reverse sweep (U, R and Linv kept by the forward sweep)
   for (int c = nch - 1; c >= 0; --c) {
     const long t0 = (long)f * L + c * kC;
     const int nc = min(kC, L - c * kC);
+    if (c > 0) {
+      prefetch_l2(k + (t0 - kC) * dk, (long)kC * dk * sizeof(T));
+      prefetch_l2(dvg + (t0 - kC) * dv, (long)kC * dv * sizeof(float));
+      prefetch_l2(rdst + (t0 - kC) * rld, (long)kC * rld * sizeof(float));
+      prefetch_l2(lbuf + (c - 1) * (kC * kC), (long)kC * kC * sizeof(float));
+    }
     tile_load(sm.U, LD, dvg + t0 * dv, dv, kC, nc, dv);
-    load_chunk(sm, p, k, v, beta, t0, nc, tid);
+    tile_load(sm.E, LD, rdst + t0 * rld, rld, kC, nc, dv);
+    tile_load(sm.M, LDC, lbuf + c * (kC * kC), kC, kC, kC, kC);
+    load_chunk<SM, T, false>(sm, p, k, v, beta, t0, nc, tid);
     wrun<ND, 2, NP>(dk, dv, nc, Kcol, [&](int t, int n) { return sm.U[t * LD + n]; },
                     [&](int m, int n, float x) { sm.S[m * LD + n] -= x; });  // the chunk's start state
-    gram();
-    __syncthreads();
-    inverse(sm, nc, tid);
-    wrun<3, 2, NP>(kC, dv, dk, Krow, [&](int kk, int n) { return sm.S[kk * LD + n]; },
-                   [&](int m, int n, float x) { sm.E[m * LD + n] -= x; });  // E = V - Khat S
-    __syncthreads();
-    wrun<3, 2, NP>(kC, dv, nc, [&](int m, int s2) { return s2 < m ? sm.M[s2 * LDC + m] : 0.f; },
-                   [&](int s2, int n) { return sm.U[s2 * LD + n]; },
-                   [&](int m, int n, float x) { sm.E[m * LD + n] -= x; });  // R = E - strict_lower(Gram) U
     wrun<3, 2, NP>(kC, dv, dk, Krow, [&](int kk, int n) { return sm.H[kk * LD + n]; },
                    [&](int m, int n, float x) { sm.G[m * LD + n] = x; });  // Khat H
     __syncthreads();
@@ -969,14 +990,14 @@ cudaError_t launch_nd(const BwdParams &p, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(gdn_bwd_qdo_kernel<ND, T, qnp>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)sq);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(gdn_bwd_adjoint_kernel<ND, T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sa);
+  e = cudaFuncSetAttribute(gdn_bwd_adjoint_kernel<ND>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sa);
   if (e != cudaSuccess) return e;
   const int BH = p.B * p.H;
   const int ncg = (p.dv + 15) / 16;
   gdn_bwd_qdo_kernel<ND, T, qnp><<<(unsigned)((long)BH * p.F), kThreads, sq, st>>>(p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  gdn_bwd_adjoint_kernel<ND, T><<<BH * ncg, kThreads, sa, st>>>(p);
+  gdn_bwd_adjoint_kernel<ND><<<BH * ncg, kThreads, sa, st>>>(p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const unsigned grid = (unsigned)((long)BH * p.F);
@@ -1004,6 +1025,7 @@ cudaError_t launch_t(const BwdParams &p, cudaStream_t st) {
 }  // namespace bwd
 
 bool gdn_bwd_supported(int dk, int dv) { return dk >= 1 && dv >= 1 && dk <= 112 && dv <= 112; }
+int gdn_bwd_chunks(int L) { return (L + bwd::kC - 1) / bwd::kC; }
 
 cudaError_t launch_gdn_bwd(const BwdParams &p, int in_dtype, cudaStream_t st) {
   if (!gdn_bwd_supported(p.dk, p.dv)) return cudaErrorInvalidValue;

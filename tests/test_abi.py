@@ -210,8 +210,14 @@ def test_backward_workspace_and_argument_validation(lib):
     fr = B * H * F
     tc = lib.make_opts(lib.DTYPE_BF16, stream=0)
     chain = lib.workspace_bytes(lib.OP_GDN, B, H, F, L, d, d, lib.make_opts(lib.DTYPE_BF16, stream=0, segments=1))
-    want = up(chain) + 3 * up(fr * d * d * 4) + up(fr * 7 * 4)
+    nch = (L + 47) // 48  # the tensor-core frame kernel keeps each 48-token chunk's Linv
+    want = up(chain) + 3 * up(fr * d * d * 4) + up(fr * 7 * 4) + up(fr * nch * 48 * 48 * 4)
     assert lib.workspace_bytes(lib.OP_GDN_BWD, B, H, F, L, d, d, tc) == want
+    # d_v > d_k: the residuals need their own rows (d_k's rows hold them otherwise)
+    assert lib.workspace_bytes(lib.OP_GDN_BWD, B, H, F, L, 48, 112, tc) == \
+        up(lib.workspace_bytes(lib.OP_GDN, B, H, F, L, 48, 112, lib.make_opts(lib.DTYPE_BF16, stream=0, segments=1))) + \
+        up(fr * 48 * 48 * 4) + 2 * up(fr * 48 * 112 * 4) + up(fr * 7 * 4) + up(fr * nch * 48 * 48 * 4) + \
+        up(fr * L * 112 * 4)
     f32 = lib.make_opts(lib.DTYPE_F32, stream=0)  # the fp32 recompute publishes fp32 states
     chain32 = 256 + up(fr * 4) + up(fr * d * d * 4)
     assert lib.workspace_bytes(lib.OP_GDN_BWD, B, H, F, L, d, d, f32) == up(chain32) + 3 * up(fr * d * d * 4) + \
