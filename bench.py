@@ -58,7 +58,7 @@ def parse():
                     help="use only the first N latent frames (a smaller case of the same kernel, for profiling)")
     ap.add_argument("--quick", action="store_true",
                     help="kernel leg only: no end-to-end leg, no ReLU-mode line, no CPU baseline")
-    ap.add_argument("--profile-case", choices=["gdn", "relu", "tconv", "stream", "swa"], default=None,
+    ap.add_argument("--profile-case", choices=["gdn", "relu", "tconv", "stream", "swa", "bwd"], default=None,
                     help="run three launches of one kernel on a small case (inputs larger than L2, under 1 GB) "
                          "and exit: the command profiled with ncu --set full")
     return ap.parse_args()
@@ -87,6 +87,13 @@ def profile_case(name: str):
         x = synth.inputs(w)
         q, k, v = (torch.from_numpy(x[n]).to(torch.bfloat16).to(dev) for n in "qkv")
         call = lambda: lib.relu_la_block_fwd(q, k, v, F=w.F)
+    elif name == "bwd":  # the backward, first 24 of the 240 frames of the 720p 60 s shape
+        w = synth.WORKLOADS["gdn_720p_60s"].with_(F=24)
+        x = synth.inputs(w)
+        q, k, v = (torch.from_numpy(x[n]).to(torch.bfloat16).to(dev) for n in "qkv")
+        a, b = (torch.from_numpy(x[n]).to(dev) for n in "ab")
+        d_o = torch.from_numpy(synth.grad_inputs(w)["d_o"]).to(dev)
+        call = lambda: lib.gdn_frame_bwd(q, k, v, a, b, d_o, F=w.F)
     elif name == "swa":  # windowed softmax layer, first 24 of the 240 frames, W = 4
         F, L, d = 24, 920, 112
         q, k, v = (torch.from_numpy(synth.normal(7, t, 0, 20 * F * L * d).reshape(1, 20, F * L, d))
@@ -122,6 +129,7 @@ KERNEL_SOURCES = {
     "relu_tc": ("relu_tc.cu", "tc_ptx.cuh", "common.cuh"),
     "temporal_conv": ("temporal_conv.cu", "f32x2.cuh", "tc_ptx.cuh", "common.cuh"),
     "softmax_window": ("softmax_window.cu", "f32x2.cuh", "tc_ptx.cuh", "common.cuh"),
+    "gdn_bwd": ("gdn_bwd.cu", "common.cuh"),
 }
 
 
@@ -735,7 +743,8 @@ def softmax_window_leg(args, lib, synth, torch, dev, stream, cpu_baseline_on):
 def backward_leg(args, lib, synth, torch, dev, stream, cpu_baseline_on):
     """gdn_frame_bwd on the headline workload (720p 60 s: B=1, H=20, F=240, L=920,
     d=112, bf16 q, k, v; fp32 dL/do ~ N(0, 1), no start state).  One call =
-    the forward recompute, the adjoint frame chain and the frame kernel."""
+    the forward recompute, Q^T dO per frame, the adjoint frame chain and the
+    frame kernel."""
     w = synth.WORKLOADS["gdn_720p_60s"]
     x = synth.inputs(w)
     q, k, v = (torch.from_numpy(x[n]).to(torch.bfloat16).to(dev) for n in "qkv")
@@ -756,8 +765,10 @@ def backward_leg(args, lib, synth, torch, dev, stream, cpu_baseline_on):
     peak, peak_src = measured_peaks()
     res = {"workload": WORKLOAD, "B": w.B, "H": w.H, "F": w.F, "L": w.L, "d": w.dk, "ms": ms,
            "tokens_per_s": w.B * w.N / (ms / 1e3),
-           "roofline": dict(_roofline(alg_bytes, ms, peak, peak_src), scope="the whole call (three launches)"),
-           "launches_per_call": 3,
+           "roofline": dict(_roofline(alg_bytes, ms, peak, peak_src), scope="the whole call (four launches)",
+                            frame_kernel_traffic=None if ncu_traffic("gdn_bwd") is None
+                            else ncu_traffic("gdn_bwd")["dram_bytes_per_launch"]),
+           "launches_per_call": 4,
            "l2": "inputs 2.97 GB and dL/do 1.98 GB, larger than L2; no flush needed"}
     del q, k, v, a, b, d_o, out, ws
     if cpu_baseline_on:

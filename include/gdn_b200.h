@@ -197,20 +197,23 @@ GDN_API int gdn_frame_fwd(const void *q, const void *k, const void *v, const flo
  * A_f being the frame's transition (ordered product of I - beta khat khat^T),
  * and d_alpha_f = <A_f^T G_f, S_{f-1}>, d_state_in = alpha_0 A_0^T G_0.  Inside a
  * frame the token gradients come from two sweeps over chunks of 48 tokens in
- * the UT form: forward from alpha_f S_{f-1}, then in reverse from G_f.  Three
+ * the UT form: forward from alpha_f S_{f-1}, then in reverse from G_f.  Four
  * launches on opts->stream: the forward recompute keeping every frame's A_f
  * and S_f (GDN_IMPL_TC for bf16 inputs where it applies, else FRAME_SIMT in
- * fp32; opts->impl may force either), the chain over frames, and one CTA per
- * frame for the token gradients (fp32 on CUDA cores).
+ * fp32; opts->impl may force either), Q_f^T dO_f for every frame, the chain
+ * over frames, and one CTA per frame for the token gradients.
  *
  * Sizes: as gdn_frame_fwd, with dk, dv <= 112.  Workspace:
- * gdn_workspace_bytes(GDN_OP_GDN_BWD, ...) (four fp32 d x d matrices per frame
- * plus the recompute's scratch).  opts->rope_grid_w must be 0
+ * gdn_workspace_bytes(GDN_OP_GDN_BWD, ...) (four fp32 d x d matrices per frame,
+ * with bf16 inputs a 48 x 48 matrix per 48-token chunk and, when dv > dk, a
+ * row per token, plus the recompute's scratch).  opts->rope_grid_w must be 0
  * (GDN_ERR_UNSUPPORTED otherwise).
  *
  * Precision: with bf16 inputs the recomputed A_f and S_f carry the tensor-core
- * forward's rounding (see gdn_frame_fwd); everything else is fp32.  Returns
- * GDN_OK or GDN_ERR_*.
+ * forward's rounding (see gdn_frame_fwd), and the products of Q_f^T dO_f and of
+ * the token gradients take tf32 operands (10-bit significands) with fp32
+ * accumulation; with fp32 inputs everything is fp32 (Q_f^T dO_f with tf32
+ * high/low operand splits, about fp32).  Returns GDN_OK or GDN_ERR_*.
  */
 GDN_API int gdn_frame_bwd(const void *q, const void *k, const void *v, const float *alpha, const float *beta,
                   const float *state_in, const float *d_o, const float *d_state_out, float *d_q, float *d_k,
