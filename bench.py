@@ -334,9 +334,10 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         dist.barrier()
     torch.cuda.synchronize()
 
-    ms_e2e, h2d, d2h = None, 0, 0
+    ms_e2e, h2d, d2h, cbound = None, 0, 0, None
     if not args.quick:
-        ms_e2e, h2d, d2h = end_to_end_leg(args, lib, torch, dist, w, dev, stream, world, (hq, hk, hv, ha, hb))
+        ms_e2e, h2d, d2h, cbound = end_to_end_leg(args, lib, torch, dist, w, dev, stream, world,
+                                                  (hq, hk, hv, ha, hb))
     if rank != 0:
         return
     cpu_on = world == 1 and not args.no_cpu_baseline
@@ -386,7 +387,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     if ms_e2e is not None:
         line["e2e"] = {"value": whole_job_tokens_per_s(tokens, world, ms_e2e), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                        "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e,
-                       "call": "gdn_frame_fwd_host (C ABI, pinned host buffers, copies + kernel + sync)"}
+                       "call": "gdn_frame_fwd_host (C ABI, pinned host buffers, copies + kernel + sync)",
+                       "pcie_floor": cbound}
     line.update(extra)
     if cpu_on and not args.quick:
         line["cpu_baseline"] = cpu_baseline(w)
@@ -449,7 +451,41 @@ def end_to_end_leg(args, lib, torch, dist, w, dev, stream, world, host):
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, ha, hb))
     d2h = ho.numel() * ho.element_size()
     del hws
-    return ms_e2e, h2d, d2h
+    return ms_e2e, h2d, d2h, copy_bound(torch, dev, (hq, hk, hv, ha, hb), ho)
+
+
+def copy_bound(torch, dev, host_in, host_out):
+    """The PCIe floor of the end-to-end leg: the same bytes as plain pinned copies
+    (cudaMemcpyAsync through torch), host -> device alone, device -> host alone,
+    and both at once on two streams (the link is full duplex)."""
+    dins = [torch.empty_like(t, device=dev) for t in host_in]
+    dout = torch.empty_like(host_out, device=dev)
+    s1, s2 = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+
+    def h2d():
+        with torch.cuda.stream(s1):
+            for d, h in zip(dins, host_in):
+                d.copy_(h, non_blocking=True)
+
+    def d2h():
+        with torch.cuda.stream(s2):
+            host_out.copy_(dout, non_blocking=True)
+
+    def timed(fns):
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        for fn in fns:
+            fn()
+        torch.cuda.synchronize()
+        return (time.perf_counter() - t0) * 1e3
+
+    h2d(), d2h()
+    res = {"h2d_only_ms": min(timed([h2d]) for _ in range(2)), "d2h_only_ms": min(timed([d2h]) for _ in range(2)),
+           "both_ms": min(timed([h2d, d2h]) for _ in range(2)),
+           "method": "the same bytes as plain pinned cudaMemcpyAsync copies on two streams, host wall clock "
+                     "around device syncs, best of 2"}
+    del dins, dout
+    return res
 
 
 def relu_leg(args, lib, synth, torch, dev, stream, cpu_baseline_on):
