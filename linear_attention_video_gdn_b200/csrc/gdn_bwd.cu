@@ -24,7 +24,9 @@
 //                      (U kept for the reverse sweep); then dq = dO S_f^T;
 //       reverse sweep: S -= Khat^T U (the chunk's start state again),
 //                      E = V - Khat S, R = E - strict_lower(Khat Khat^T) U
-//                      (row t: the token's residual v_t - S_{t-1}^T khat_t),
+//                      (row t: the token's residual v_t - S_{t-1}^T khat_t;
+//                      the warp-MMA kernel keeps R and Linv from the forward
+//                      sweep instead),
 //                      Gm = Linv^T Khat H (row t: g_t = H_t^T khat_t with H_t
 //                      the gradient after token t),
 //                      dv = diag(beta) Gm, dbeta_t = g_t . R_t,
@@ -89,17 +91,17 @@ __device__ __forceinline__ void tile_load(float *dst, int ldd, const T *src, lon
   constexpr int kB = 8;
   if ((cols & 3) == 0 && (gs & 3) == 0) {
     const int cv = cols >> 2, nv = rows * cv;
-    for (int base = threadIdx.x; base < nv; base += kB * kThreads) {
+    for (int base = threadIdx.x; base < nv; base += kB * (int)blockDim.x) {
       float4 r[kB];
 #pragma unroll
       for (int b = 0; b < kB; ++b) {
-        const int e = base + b * kThreads;
+        const int e = base + b * (int)blockDim.x;
         const int row = e / cv, c4 = e - row * cv;
         r[b] = (e < nv && row < nvalid) ? ld4(src + row * gs + 4 * c4) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
 #pragma unroll
       for (int b = 0; b < kB; ++b) {
-        const int e = base + b * kThreads;
+        const int e = base + b * (int)blockDim.x;
         if (e < nv) {
           const int row = e / cv, c4 = e - row * cv;
           float *d = dst + row * ldd + 4 * c4;
@@ -112,17 +114,17 @@ __device__ __forceinline__ void tile_load(float *dst, int ldd, const T *src, lon
     }
   } else {
     const int nv = rows * cols;
-    for (int base = threadIdx.x; base < nv; base += kB * kThreads) {
+    for (int base = threadIdx.x; base < nv; base += kB * (int)blockDim.x) {
       float r[kB];
 #pragma unroll
       for (int b = 0; b < kB; ++b) {
-        const int e = base + b * kThreads;
+        const int e = base + b * (int)blockDim.x;
         const int row = e / cols, c = e - row * cols;
         r[b] = (e < nv && row < nvalid) ? ld1(src + row * gs + c) : 0.f;
       }
 #pragma unroll
       for (int b = 0; b < kB; ++b) {
-        const int e = base + b * kThreads;
+        const int e = base + b * (int)blockDim.x;
         if (e < nv) {
           const int row = e / cols, c = e - row * cols;
           dst[row * ldd + c] = scale * r[b];
@@ -135,7 +137,7 @@ __device__ __forceinline__ void tile_load(float *dst, int ldd, const T *src, lon
 // Ask L2 for [base, base + bytes) (128-byte lines spread over the block's threads).
 __device__ __forceinline__ void prefetch_l2(const void *base, long bytes) {
   const char *b = static_cast<const char *>(base);
-  for (long off = (long)threadIdx.x * 128; off < bytes; off += (long)kThreads * 128)
+  for (long off = (long)threadIdx.x * 128; off < bytes; off += (long)blockDim.x * 128)
     asm volatile("prefetch.global.L2 [%0];" ::"l"(b + off));
 }
 
@@ -264,7 +266,7 @@ __device__ __forceinline__ void load_chunk(SM &sm, const BwdParams &p, const T *
   }
   __syncthreads();
   const int warp = tid >> 5, lane = tid & 31;
-  for (int t = warp; t < kC; t += kThreads / 32) {
+  for (int t = warp; t < kC; t += (int)(blockDim.x >> 5)) {
     float ss = 0.f;
     for (int i = lane; i < dk; i += 32) ss = fmaf(sm.K[t * LD + i], sm.K[t * LD + i], ss);
 #pragma unroll
@@ -276,7 +278,7 @@ __device__ __forceinline__ void load_chunk(SM &sm, const BwdParams &p, const T *
     }
   }
   __syncthreads();
-  for (int e = tid; e < kC * dk; e += kThreads) {
+  for (int e = tid; e < kC * dk; e += (int)blockDim.x) {
     const int t = e / dk, i = e % dk;
     sm.K[t * LD + i] *= sm.inv[t];
   }
@@ -313,7 +315,7 @@ __device__ __forceinline__ void inverse(SM &sm, int nc, int tid) {
   // off-diagonal blocks, by distance: Linv_{i,j} = -D_i sum_{m=j}^{i-1} N_{i,m} Linv_{m,j}
   for (int d = 1; d < nb; ++d) {
     // T_{i,j} = sum_m N_{i,m} Linv_{m,j}  (Linv_{m,m} = D_m with its unit diagonal)
-    for (int e = tid; e < (nb - d) * 256; e += kThreads) {
+    for (int e = tid; e < (nb - d) * 256; e += (int)blockDim.x) {
       const int jb = e >> 8, r = (e >> 4) & 15, c = e & 15, ib = jb + d;
       float a = 0.f;
       for (int mb = jb; mb < ib; ++mb)
@@ -326,7 +328,7 @@ __device__ __forceinline__ void inverse(SM &sm, int nc, int tid) {
     }
     __syncthreads();
     // Linv_{i,j} = -D_i T_{i,j}
-    for (int e = tid; e < (nb - d) * 256; e += kThreads) {
+    for (int e = tid; e < (nb - d) * 256; e += (int)blockDim.x) {
       const int jb = e >> 8, r = (e >> 4) & 15, c = e & 15, ib = jb + d;
       float a = sm.T[jb * 272 + r * 17 + c];  // D_i's unit diagonal
       for (int u = 0; u < r; ++u) a = fmaf(sm.M[(16 * ib + r) * kLdC + 16 * ib + u], sm.T[jb * 272 + u * 17 + c], a);
@@ -701,7 +703,7 @@ template <int MT, int NT, int NP, class FA, class FB, class EP>
 __device__ __forceinline__ void wrun(int M, int N, int K, FA fa, FB fb, EP ep) {
   const int warp = threadIdx.x >> 5;
   const int nmb = (M + 16 * MT - 1) / (16 * MT), nnb = (N + 8 * NT - 1) / (8 * NT);
-  for (int blk = warp; blk < nmb * nnb; blk += kThreads / 32) {
+  for (int blk = warp; blk < nmb * nnb; blk += (int)(blockDim.x >> 5)) {
     const int m0 = (blk % nmb) * 16 * MT, n0 = (blk / nmb) * 8 * NT;
     float acc[MT][NT][4];
 #pragma unroll
@@ -740,11 +742,13 @@ __device__ __forceinline__ void wrun_sync(int M, int N, int K, FA fa, FB fb, EP 
     });
 }
 
-template <int ND, typename T, int NP>
-__global__ void __launch_bounds__(kThreads, 1) gdn_bwd_frame_mma_kernel(BwdParams p) {
+template <int ND, typename T, int NP, int NW>
+__global__ void __launch_bounds__(32 * NW, 1) gdn_bwd_frame_mma_kernel(BwdParams p) {
+  constexpr int kTh = 32 * NW;
+  constexpr int NB = NW >= 16 ? 1 : 2;  // 8-column tiles per warp block: more warps, narrower blocks
   using SM = FrameSmemT<ND, 4>;
   constexpr int LD = SM::LD, LDC = SM::LDC;
-  static_assert(ND <= 8, "one 16-column block per warp");
+  static_assert(2 * ND <= NB * NW, "one block per warp");
   extern __shared__ __align__(16) unsigned char smem_raw[];
   SM &sm = *reinterpret_cast<SM *>(smem_raw);
   const int tid = threadIdx.x;
@@ -768,7 +772,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_frame_mma_kernel(BwdParam
   const int rld = p.rbuf ? dv : dk;
   float *lbuf = p.linv_buf + ((long)bh * F + f) * nch * (kC * kC);  // each chunk's Linv, [48][48]
 
-  for (int e = tid; e < (int)(sizeof(SM) / 4); e += kThreads) reinterpret_cast<float *>(&sm)[e] = 0.f;
+  for (int e = tid; e < (int)(sizeof(SM) / 4); e += kTh) reinterpret_cast<float *>(&sm)[e] = 0.f;
   __syncthreads();
   const float araw = p.alpha[(long)bh * F + f];
   const float al = p.gates_are_logits ? gate_alpha(araw) : araw;
@@ -782,7 +786,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_frame_mma_kernel(BwdParam
   auto Krow = [&](int m, int kk) { return sm.K[m * LD + kk]; };  // Khat (t, i)
   auto Kcol = [&](int m, int kk) { return sm.K[kk * LD + m]; };  // Khat^T (i, t)
   auto gram = [&]() {
-    wrun<1, 2, NP>(kC, kC, dk, Krow, [&](int kk, int n) { return sm.K[n * LD + kk]; }, [&](int m, int n, float x) {
+    wrun<3, NB, NP>(kC, kC, dk, Krow, [&](int kk, int n) { return sm.K[n * LD + kk]; }, [&](int m, int n, float x) {
       if (n >= m) sm.M[m * LDC + n] = x;
     });
   };
@@ -800,23 +804,23 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_frame_mma_kernel(BwdParam
     gram();
     __syncthreads();
     inverse(sm, nc, tid);
-    wrun<3, 2, NP>(kC, dv, dk, Krow, [&](int kk, int n) { return sm.S[kk * LD + n]; },
+    wrun<3, NB, NP>(kC, dv, dk, Krow, [&](int kk, int n) { return sm.S[kk * LD + n]; },
                    [&](int m, int n, float x) { sm.E[m * LD + n] -= x; });  // E = V - Khat S
     __syncthreads();
-    wrun<3, 2, NP>(kC, dv, nc, [&](int m, int s2) { return linv(sm, m, s2) * sm.b[s2]; },
+    wrun<3, NB, NP>(kC, dv, nc, [&](int m, int s2) { return linv(sm, m, s2) * sm.b[s2]; },
                    [&](int s2, int n) { return sm.E[s2 * LD + n]; }, [&](int m, int n, float x) {
                      sm.U[m * LD + n] = x;  // U = Linv diag(beta) E
                      if (m < nc) dvg[(t0 + m) * dv + n] = x;
                    });
     __syncthreads();
-    wrun<ND, 2, NP>(dk, dv, nc, Kcol, [&](int t, int n) { return sm.U[t * LD + n]; },
+    wrun<ND, NB, NP>(dk, dv, nc, Kcol, [&](int t, int n) { return sm.U[t * LD + n]; },
                     [&](int m, int n, float x) { sm.S[m * LD + n] += x; });  // S += Khat^T U
     // R = E - strict_lower(Gram) U, and Linv, kept for the reverse sweep
-    wrun<3, 2, NP>(kC, dv, nc, [&](int m, int s2) { return s2 < m ? sm.M[s2 * LDC + m] : 0.f; },
+    wrun<3, NB, NP>(kC, dv, nc, [&](int m, int s2) { return s2 < m ? sm.M[s2 * LDC + m] : 0.f; },
                    [&](int s2, int n) { return sm.U[s2 * LD + n]; }, [&](int m, int n, float x) {
                      if (m < nc) rdst[(t0 + m) * rld + n] = sm.E[m * LD + n] - x;
                    });
-    for (int e = tid; e < kC * kC; e += kThreads) lbuf[c * (kC * kC) + e] = sm.M[(e / kC) * LDC + e % kC];
+    for (int e = tid; e < kC * kC; e += kTh) lbuf[c * (kC * kC) + e] = sm.M[(e / kC) * LDC + e % kC];
     __syncthreads();
   }
 
@@ -826,7 +830,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_frame_mma_kernel(BwdParam
     const int nc = min(kC, L - c * kC);
     tile_load(sm.G, LD, d_o + t0 * dv, dv, kC, nc, dv);
     __syncthreads();
-    wrun<3, 2, NP>(kC, dk, dv, [&](int m, int jj) { return sm.G[m * LD + jj]; },
+    wrun<3, NB, NP>(kC, dk, dv, [&](int m, int jj) { return sm.G[m * LD + jj]; },
                    [&](int jj, int n) { return sm.S[n * LD + jj]; }, [&](int m, int n, float x) {
                      if (m < nc) dq[(t0 + m) * dk + n] = x;
                    });
@@ -847,18 +851,18 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_frame_mma_kernel(BwdParam
     tile_load(sm.E, LD, rdst + t0 * rld, rld, kC, nc, dv);
     tile_load(sm.M, LDC, lbuf + c * (kC * kC), kC, kC, kC, kC);
     load_chunk<SM, T, false>(sm, p, k, v, beta, t0, nc, tid);
-    wrun<ND, 2, NP>(dk, dv, nc, Kcol, [&](int t, int n) { return sm.U[t * LD + n]; },
+    wrun<ND, NB, NP>(dk, dv, nc, Kcol, [&](int t, int n) { return sm.U[t * LD + n]; },
                     [&](int m, int n, float x) { sm.S[m * LD + n] -= x; });  // the chunk's start state
-    wrun<3, 2, NP>(kC, dv, dk, Krow, [&](int kk, int n) { return sm.H[kk * LD + n]; },
+    wrun<3, NB, NP>(kC, dv, dk, Krow, [&](int kk, int n) { return sm.H[kk * LD + n]; },
                    [&](int m, int n, float x) { sm.G[m * LD + n] = x; });  // Khat H
     __syncthreads();
-    wrun_sync<3, 2, NP>(kC, dv, nc, [&](int m, int s2) { return linv(sm, s2, m); },
+    wrun_sync<3, NB, NP>(kC, dv, nc, [&](int m, int s2) { return linv(sm, s2, m); },
                         [&](int s2, int n) { return sm.G[s2 * LD + n]; }, [&](int m, int n, float x) {
                           sm.G[m * LD + n] = x;  // Gm = Linv^T (Khat H)
                           if (m < nc) dvg[(t0 + m) * dv + n] = sm.b[m] * x;
                         });
     __syncthreads();
-    for (int t = warp; t < nc; t += kThreads / 32) {  // dbeta_t = g_t . R_t
+    for (int t = warp; t < nc; t += NW) {  // dbeta_t = g_t . R_t
       float s2 = 0.f;
       for (int jj = lane; jj < dv; jj += 32) s2 = fmaf(sm.G[t * LD + jj], sm.E[t * LD + jj], s2);
 #pragma unroll
@@ -868,42 +872,43 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_frame_mma_kernel(BwdParam
         dbg[t0 + t] = p.gates_are_logits ? s2 * bt * (1.f - bt) : s2;
       }
     }
-    {  // M: upper beta_s R_t . g_s, lower g_t . u_s (Gram and Linv are dead)
-      for (int blk = warp; blk < 9; blk += kThreads / 32) {
-        const int m0 = (blk % 3) * 16, n0 = (blk / 3) * 16;
-        float r1[1][2][4] = {}, r2[1][2][4] = {};
-        wmm<1, 2, NP>(r1, m0, n0, dv, [&](int m, int jj) { return sm.E[m * LD + jj]; },
-                      [&](int jj, int n) { return sm.G[n * LD + jj]; });
-        wmm<1, 2, NP>(r2, m0, n0, dv, [&](int m, int jj) { return sm.G[m * LD + jj]; },
-                      [&](int jj, int n) { return sm.U[n * LD + jj]; });
-        each(r1, m0, n0, [&](int m, int n, float x) {
-          if (n > m) sm.M[m * LDC + n] = sm.b[n] * x;
-          else if (n == m) sm.M[m * LDC + n] = 0.f;
+    // M: upper beta_s R_t . g_s, lower g_t . u_s (Gram and Linv are dead): 8 NB columns of
+    // all 48 rows per warp, the first 6 / NB warps for R Gm^T, the next for Gm U^T
+    if (warp < 12 / NB) {
+      const int half = warp / (6 / NB), n0 = (warp % (6 / NB)) * 8 * NB;
+      float r[3][NB][4] = {};
+      if (half == 0) {
+        wmm<3, NB, NP>(r, 0, n0, dv, [&](int m, int jj) { return sm.E[m * LD + jj]; },
+                       [&](int jj, int n) { return sm.G[n * LD + jj]; });
+        each(r, 0, n0, [&](int m, int n, float x) {
+          if (n >= m) sm.M[m * LDC + n] = n > m ? sm.b[n] * x : 0.f;
         });
-        each(r2, m0, n0, [&](int m, int n, float x) {
+      } else {
+        wmm<3, NB, NP>(r, 0, n0, dv, [&](int m, int jj) { return sm.G[m * LD + jj]; },
+                       [&](int jj, int n) { return sm.U[n * LD + jj]; });
+        each(r, 0, n0, [&](int m, int n, float x) {
           if (n < m) sm.M[m * LDC + n] = x;
         });
       }
     }
     __syncthreads();
     {  // dkhat = diag(beta) (R H^T - Gm S^T - M Khat) -> U rows (U is dead)
-      const bool has = warp < ND;
-      float a[3][2][4] = {};
+      const int n0 = warp * 8 * NB;
+      const bool has = n0 < dk;
+      float a[3][NB][4] = {};
       if (has) {
-        const int n0 = warp * 16;
-        wmm<3, 2, NP>(a, 0, n0, dv, [&](int m, int jj) { return sm.E[m * LD + jj]; },
-                      [&](int jj, int n) { return sm.H[n * LD + jj]; });
-        wmm<3, 2, NP>(a, 0, n0, dv, [&](int m, int jj) { return -sm.G[m * LD + jj]; },
-                      [&](int jj, int n) { return sm.S[n * LD + jj]; });
-        wmm<3, 2, NP>(a, 0, n0, nc, [&](int m, int s2) { return -sm.M[m * LDC + s2]; },
-                      [&](int s2, int n) { return sm.K[s2 * LD + n]; });
+        wmm<3, NB, NP>(a, 0, n0, dv, [&](int m, int jj) { return sm.E[m * LD + jj]; },
+                       [&](int jj, int n) { return sm.H[n * LD + jj]; });
+        wmm<3, NB, NP>(a, 0, n0, dv, [&](int m, int jj) { return -sm.G[m * LD + jj]; },
+                       [&](int jj, int n) { return sm.S[n * LD + jj]; });
+        wmm<3, NB, NP>(a, 0, n0, nc, [&](int m, int s2) { return -sm.M[m * LDC + s2]; },
+                       [&](int s2, int n) { return sm.K[s2 * LD + n]; });
       }
       __syncthreads();
-      if (has)
-        each(a, 0, warp * 16, [&](int m, int n, float x) { sm.U[m * LD + n] = sm.b[m] * x; });
+      if (has) each(a, 0, n0, [&](int m, int n, float x) { sm.U[m * LD + n] = sm.b[m] * x; });
     }
     __syncthreads();
-    for (int t = warp; t < nc; t += kThreads / 32) {
+    for (int t = warp; t < nc; t += NW) {
       // dk = (dkhat - khat (khat . dkhat)) / ||k|| (||k|| > eps), dkhat / eps (otherwise)
       float dot = 0.f;
       for (int i = lane; i < dk; i += 32) dot = fmaf(sm.K[t * LD + i], sm.U[t * LD + i], dot);
@@ -916,7 +921,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_frame_mma_kernel(BwdParam
         dkg[(t0 + t) * dk + i] = gk * sc;
       }
     }
-    wrun<ND, 2, NP>(dk, dv, nc, [&](int m, int t) { return sm.K[t * LD + m] * sm.b[t]; },
+    wrun<ND, NB, NP>(dk, dv, nc, [&](int m, int t) { return sm.K[t * LD + m] * sm.b[t]; },
                     [&](int t, int n) { return sm.G[t * LD + n]; },
                     [&](int m, int n, float x) { sm.H[m * LD + n] -= x; });  // H -= Khat^T diag(beta) Gm
     __syncthreads();
@@ -979,6 +984,7 @@ __global__ void __launch_bounds__(kThreads) gdn_bwd_qdo_kernel(BwdParams p) {
 
 // tf32 passes of the warp-MMA frame kernel (bf16 inputs): 3 = high/low split
 constexpr int kMmaPasses = 1;
+constexpr int kMmaWarps = 8;  // warps of the warp-MMA frame kernel (16 measured slower: a phase is as long as its k-loop)
 
 template <int ND, typename T>
 cudaError_t launch_nd(const BwdParams &p, cudaStream_t st) {
@@ -1002,10 +1008,10 @@ cudaError_t launch_nd(const BwdParams &p, cudaStream_t st) {
   if (e != cudaSuccess) return e;
   const unsigned grid = (unsigned)((long)BH * p.F);
   if constexpr (mma) {
-    e = cudaFuncSetAttribute(gdn_bwd_frame_mma_kernel<ND, T, kMmaPasses>,
+    e = cudaFuncSetAttribute(gdn_bwd_frame_mma_kernel<ND, T, kMmaPasses, kMmaWarps>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sf);
     if (e != cudaSuccess) return e;
-    gdn_bwd_frame_mma_kernel<ND, T, kMmaPasses><<<grid, kThreads, sf, st>>>(p);
+    gdn_bwd_frame_mma_kernel<ND, T, kMmaPasses, kMmaWarps><<<grid, 32 * kMmaWarps, sf, st>>>(p);
   } else {
     e = cudaFuncSetAttribute(gdn_bwd_frame_kernel<ND, T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sf);
     if (e != cudaSuccess) return e;
