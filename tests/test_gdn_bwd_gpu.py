@@ -112,3 +112,22 @@ def test_720p_60s_two_heads(lib, dev):
     heads = [0, 13]
     out, ref = run(lib, dev, w, x, d_o, None, None, heads=heads)
     check(out, ref, TOL_BF16)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_recompute_timeout_status_is_reported(lib, dev, dtype):
+    """A frame of the forward recompute that never publishes its state (the
+    test option withholds frame 0 of head 0): the next frame's bounded wait runs
+    out after 2 ms, GDN_ERR_TIMEOUT is latched, the call returns, and the next
+    call on the same context is correct."""
+    w, x, d_o, si, dso = case(1, 1, 3, 40, 32, 32, dtype, seed=91)
+    t, _ = device_inputs(w, x, dev, torch)
+    st = torch.zeros(4, dtype=torch.int32, device=dev)
+    lib.gdn_frame_bwd(t["q"], t["k"], t["v"], t["a"], t["b"], torch.from_numpy(d_o).to(dev), F=w.F,
+                      state_in=torch.from_numpy(si).to(dev), status=st, spin_limit_us=2000, test_withhold_unit=0)
+    torch.cuda.synchronize()
+    assert int(st[0].item()) == lib.ERR_TIMEOUT
+    st.zero_()
+    out, ref = run(lib, dev, w, x, d_o, si, dso, status=st)
+    assert int(st[0].item()) == 0
+    check(out, ref, TOL_F32 if dtype == "f32" else TOL_BF16)
