@@ -70,6 +70,13 @@ __device__ __forceinline__ void mm(float (&acc)[TM][TN], int K, int ty, int tx, 
   }
 }
 
+// x rounded to the nearest tf32 value (10-bit significand), as a float
+__device__ __forceinline__ float tf32_round(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return __uint_as_float(r);
+}
+
 // Global -> shared copies of fp32 tiles: dst[r * ldd + c] = scale * src[r * gs + c]
 // for r < rows, c < cols (rows >= nvalid read as zero).  Each thread keeps eight
 // loads in flight before storing, four elements per load where the rows allow
@@ -85,9 +92,11 @@ __device__ __forceinline__ float4 ld4(const __nv_bfloat16 *p) {
 __device__ __forceinline__ float ld1(const float *p) { return __ldcg(p); }
 __device__ __forceinline__ float ld1(const __nv_bfloat16 *p) { return __bfloat162float(*p); }
 
-template <typename T>
+// kTf32: the stored values rounded to tf32 (tiles used only as warp-MMA operands).
+template <bool kTf32 = false, typename T>
 __device__ __forceinline__ void tile_load(float *dst, int ldd, const T *src, long gs, int rows, int nvalid, int cols,
                                           float scale = 1.f) {
+  auto rnd = [](float x) { return kTf32 ? tf32_round(x) : x; };
   constexpr int kB = 8;
   if ((cols & 3) == 0 && (gs & 3) == 0) {
     const int cv = cols >> 2, nv = rows * cv;
@@ -105,10 +114,10 @@ __device__ __forceinline__ void tile_load(float *dst, int ldd, const T *src, lon
         if (e < nv) {
           const int row = e / cv, c4 = e - row * cv;
           float *d = dst + row * ldd + 4 * c4;
-          d[0] = scale * r[b].x;
-          d[1] = scale * r[b].y;
-          d[2] = scale * r[b].z;
-          d[3] = scale * r[b].w;
+          d[0] = rnd(scale * r[b].x);
+          d[1] = rnd(scale * r[b].y);
+          d[2] = rnd(scale * r[b].z);
+          d[3] = rnd(scale * r[b].w);
         }
       }
     }
@@ -127,7 +136,7 @@ __device__ __forceinline__ void tile_load(float *dst, int ldd, const T *src, lon
         const int e = base + b * (int)blockDim.x;
         if (e < nv) {
           const int row = e / cols, c = e - row * cols;
-          dst[row * ldd + c] = scale * r[b];
+          dst[row * ldd + c] = rnd(scale * r[b]);
         }
       }
     }
@@ -253,7 +262,7 @@ template <int ND>
 using FrameSmem = FrameSmemT<ND, 1>;
 
 // Rows t0 .. t0 + nc - 1 of the frame: khat (normalised), beta and (kV) v.
-template <class SM, typename T, bool kV = true>
+template <class SM, typename T, bool kV = true, bool kTf32 = false>
 __device__ __forceinline__ void load_chunk(SM &sm, const BwdParams &p, const T *k, const T *v, const float *beta,
                                            long t0, int nc, int tid) {
   constexpr int LD = SM::LD;
@@ -280,7 +289,8 @@ __device__ __forceinline__ void load_chunk(SM &sm, const BwdParams &p, const T *
   __syncthreads();
   for (int e = tid; e < kC * dk; e += (int)blockDim.x) {
     const int t = e / dk, i = e % dk;
-    sm.K[t * LD + i] *= sm.inv[t];
+    const float x = sm.K[t * LD + i] * sm.inv[t];
+    sm.K[t * LD + i] = kTf32 ? tf32_round(x) : x;
   }
   __syncthreads();
 }
@@ -644,8 +654,11 @@ __device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], 
 // acc += the (16 MT) x (8 NT) block at (m0, n0) of sum_{k < K} fa(m, k) fb(k, n),
 // in the m16n8 accumulator layout (lane: g = lane / 4 rows g, g + 8; t = lane % 4
 // columns 2t, 2t + 1).  A fragments: rows g, g + 8, k = t, t + 4; B: k = t, t + 4, column g.
-template <int MT, int NT, int NP, class FA, class FB>
+// RA / RB false: that operand already holds tf32 values (rounded where it was
+// written), so its fragments skip the conversion (one-pass products only).
+template <int MT, int NT, int NP, bool RA = true, bool RB = true, class FA, class FB>
 __device__ __forceinline__ void wmm(float (&acc)[MT][NT][4], int m0, int n0, int K, FA fa, FB fb) {
+  constexpr bool ca = RA || NP != 1, cb = RB || NP != 1;
   const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
 #pragma unroll 1
   for (int k0 = 0; k0 < K; k0 += 8) {
@@ -659,7 +672,7 @@ __device__ __forceinline__ void wmm(float (&acc)[MT][NT][4], int m0, int n0, int
                           vb ? fa(r + 8, kb) : 0.f};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        ah[i][e] = to_tf32(x[e]);
+        ah[i][e] = ca ? to_tf32(x[e]) : __float_as_uint(x[e]);
         if (NP == 3) al[i][e] = to_tf32(x[e] - __uint_as_float(ah[i][e]));
       }
     }
@@ -669,7 +682,7 @@ __device__ __forceinline__ void wmm(float (&acc)[MT][NT][4], int m0, int n0, int
       const float y[2] = {va ? fb(ka, n) : 0.f, vb ? fb(kb, n) : 0.f};
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
-        bh[j][e] = to_tf32(y[e]);
+        bh[j][e] = cb ? to_tf32(y[e]) : __float_as_uint(y[e]);
         if (NP == 3) bl[j][e] = to_tf32(y[e] - __uint_as_float(bh[j][e]));
       }
     }
@@ -699,7 +712,7 @@ __device__ __forceinline__ void each(const float (&acc)[MT][NT][4], int m0, int 
 
 // An M x N product over all warps, blocks of (16 MT) x (8 NT) taken round-robin;
 // ep(m, n, value) for every element inside M x N.
-template <int MT, int NT, int NP, class FA, class FB, class EP>
+template <int MT, int NT, int NP, bool RA = true, bool RB = true, class FA, class FB, class EP>
 __device__ __forceinline__ void wrun(int M, int N, int K, FA fa, FB fb, EP ep) {
   const int warp = threadIdx.x >> 5;
   const int nmb = (M + 16 * MT - 1) / (16 * MT), nnb = (N + 8 * NT - 1) / (8 * NT);
@@ -712,7 +725,7 @@ __device__ __forceinline__ void wrun(int M, int N, int K, FA fa, FB fb, EP ep) {
       for (int j = 0; j < NT; ++j)
 #pragma unroll
         for (int e = 0; e < 4; ++e) acc[i][j][e] = 0.f;
-    wmm<MT, NT, NP>(acc, m0, n0, K, fa, fb);
+    wmm<MT, NT, NP, RA, RB>(acc, m0, n0, K, fa, fb);
     each(acc, m0, n0, [&](int m, int n, float v) {
       if (m < M && n < N) ep(m, n, v);
     });
@@ -721,7 +734,7 @@ __device__ __forceinline__ void wrun(int M, int N, int K, FA fa, FB fb, EP ep) {
 
 // The same with at most one block per warp and a barrier between the products
 // and the epilogue (for results written over an operand).  All threads call it.
-template <int MT, int NT, int NP, class FA, class FB, class EP>
+template <int MT, int NT, int NP, bool RA = true, bool RB = true, class FA, class FB, class EP>
 __device__ __forceinline__ void wrun_sync(int M, int N, int K, FA fa, FB fb, EP ep) {
   const int warp = threadIdx.x >> 5;
   const int nmb = (M + 16 * MT - 1) / (16 * MT), nnb = (N + 8 * NT - 1) / (8 * NT);
@@ -734,7 +747,7 @@ __device__ __forceinline__ void wrun_sync(int M, int N, int K, FA fa, FB fb, EP 
     for (int j = 0; j < NT; ++j)
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[i][j][e] = 0.f;
-  if (has) wmm<MT, NT, NP>(acc, m0, n0, K, fa, fb);
+  if (has) wmm<MT, NT, NP, RA, RB>(acc, m0, n0, K, fa, fb);
   __syncthreads();
   if (has)
     each(acc, m0, n0, [&](int m, int n, float v) {
@@ -786,9 +799,10 @@ __global__ void __launch_bounds__(32 * NW, 1) gdn_bwd_frame_mma_kernel(BwdParams
   auto Krow = [&](int m, int kk) { return sm.K[m * LD + kk]; };  // Khat (t, i)
   auto Kcol = [&](int m, int kk) { return sm.K[kk * LD + m]; };  // Khat^T (i, t)
   auto gram = [&]() {
-    wrun<3, NB, NP>(kC, kC, dk, Krow, [&](int kk, int n) { return sm.K[n * LD + kk]; }, [&](int m, int n, float x) {
-      if (n >= m) sm.M[m * LDC + n] = x;
-    });
+    wrun<3, NB, NP, false, false>(kC, kC, dk, Krow, [&](int kk, int n) { return sm.K[n * LD + kk]; },
+                                  [&](int m, int n, float x) {
+                                    if (n >= m) sm.M[m * LDC + n] = x;
+                                  });
   };
 
   // ---- forward sweep
@@ -800,26 +814,27 @@ __global__ void __launch_bounds__(32 * NW, 1) gdn_bwd_frame_mma_kernel(BwdParams
       prefetch_l2(k + (t0 + kC) * dk, (long)nn * dk * sizeof(T));
       prefetch_l2(v + (t0 + kC) * dv, (long)nn * dv * sizeof(T));
     }
-    load_chunk(sm, p, k, v, beta, t0, nc, tid);
+    load_chunk<SM, T, true, true>(sm, p, k, v, beta, t0, nc, tid);
     gram();
     __syncthreads();
     inverse(sm, nc, tid);
-    wrun<3, NB, NP>(kC, dv, dk, Krow, [&](int kk, int n) { return sm.S[kk * LD + n]; },
-                   [&](int m, int n, float x) { sm.E[m * LD + n] -= x; });  // E = V - Khat S
+    wrun<3, NB, NP, false, true>(kC, dv, dk, Krow, [&](int kk, int n) { return sm.S[kk * LD + n]; },
+                                 [&](int m, int n, float x) { sm.E[m * LD + n] -= x; });  // E = V - Khat S
     __syncthreads();
     wrun<3, NB, NP>(kC, dv, nc, [&](int m, int s2) { return linv(sm, m, s2) * sm.b[s2]; },
                    [&](int s2, int n) { return sm.E[s2 * LD + n]; }, [&](int m, int n, float x) {
-                     sm.U[m * LD + n] = x;  // U = Linv diag(beta) E
-                     if (m < nc) dvg[(t0 + m) * dv + n] = x;
+                     const float xr = tf32_round(x);  // U = Linv diag(beta) E (an operand from here on)
+                     sm.U[m * LD + n] = xr;
+                     if (m < nc) dvg[(t0 + m) * dv + n] = xr;
                    });
     __syncthreads();
-    wrun<ND, NB, NP>(dk, dv, nc, Kcol, [&](int t, int n) { return sm.U[t * LD + n]; },
-                    [&](int m, int n, float x) { sm.S[m * LD + n] += x; });  // S += Khat^T U
+    wrun<ND, NB, NP, false, false>(dk, dv, nc, Kcol, [&](int t, int n) { return sm.U[t * LD + n]; },
+                                   [&](int m, int n, float x) { sm.S[m * LD + n] += x; });  // S += Khat^T U
     // R = E - strict_lower(Gram) U, and Linv, kept for the reverse sweep
-    wrun<3, NB, NP>(kC, dv, nc, [&](int m, int s2) { return s2 < m ? sm.M[s2 * LDC + m] : 0.f; },
-                   [&](int s2, int n) { return sm.U[s2 * LD + n]; }, [&](int m, int n, float x) {
-                     if (m < nc) rdst[(t0 + m) * rld + n] = sm.E[m * LD + n] - x;
-                   });
+    wrun<3, NB, NP, true, false>(kC, dv, nc, [&](int m, int s2) { return s2 < m ? sm.M[s2 * LDC + m] : 0.f; },
+                                 [&](int s2, int n) { return sm.U[s2 * LD + n]; }, [&](int m, int n, float x) {
+                                   if (m < nc) rdst[(t0 + m) * rld + n] = tf32_round(sm.E[m * LD + n] - x);
+                                 });
     for (int e = tid; e < kC * kC; e += kTh) lbuf[c * (kC * kC) + e] = sm.M[(e / kC) * LDC + e % kC];
     __syncthreads();
   }
@@ -828,9 +843,9 @@ __global__ void __launch_bounds__(32 * NW, 1) gdn_bwd_frame_mma_kernel(BwdParams
   for (int c = 0; c < nch; ++c) {
     const long t0 = (long)f * L + c * kC;
     const int nc = min(kC, L - c * kC);
-    tile_load(sm.G, LD, d_o + t0 * dv, dv, kC, nc, dv);
+    tile_load<true>(sm.G, LD, d_o + t0 * dv, dv, kC, nc, dv);  // dO rows, rounded to tf32 once
     __syncthreads();
-    wrun<3, NB, NP>(kC, dk, dv, [&](int m, int jj) { return sm.G[m * LD + jj]; },
+    wrun<3, NB, NP, false, true>(kC, dk, dv, [&](int m, int jj) { return sm.G[m * LD + jj]; },
                    [&](int jj, int n) { return sm.S[n * LD + jj]; }, [&](int m, int n, float x) {
                      if (m < nc) dq[(t0 + m) * dk + n] = x;
                    });
@@ -850,15 +865,15 @@ __global__ void __launch_bounds__(32 * NW, 1) gdn_bwd_frame_mma_kernel(BwdParams
     tile_load(sm.U, LD, dvg + t0 * dv, dv, kC, nc, dv);
     tile_load(sm.E, LD, rdst + t0 * rld, rld, kC, nc, dv);
     tile_load(sm.M, LDC, lbuf + c * (kC * kC), kC, kC, kC, kC);
-    load_chunk<SM, T, false>(sm, p, k, v, beta, t0, nc, tid);
-    wrun<ND, NB, NP>(dk, dv, nc, Kcol, [&](int t, int n) { return sm.U[t * LD + n]; },
-                    [&](int m, int n, float x) { sm.S[m * LD + n] -= x; });  // the chunk's start state
-    wrun<3, NB, NP>(kC, dv, dk, Krow, [&](int kk, int n) { return sm.H[kk * LD + n]; },
-                   [&](int m, int n, float x) { sm.G[m * LD + n] = x; });  // Khat H
+    load_chunk<SM, T, false, true>(sm, p, k, v, beta, t0, nc, tid);
+    wrun<ND, NB, NP, false, false>(dk, dv, nc, Kcol, [&](int t, int n) { return sm.U[t * LD + n]; },
+                                   [&](int m, int n, float x) { sm.S[m * LD + n] -= x; });  // the chunk's start state
+    wrun<3, NB, NP, false, true>(kC, dv, dk, Krow, [&](int kk, int n) { return sm.H[kk * LD + n]; },
+                                 [&](int m, int n, float x) { sm.G[m * LD + n] = tf32_round(x); });  // Khat H
     __syncthreads();
-    wrun_sync<3, NB, NP>(kC, dv, nc, [&](int m, int s2) { return linv(sm, s2, m); },
-                        [&](int s2, int n) { return sm.G[s2 * LD + n]; }, [&](int m, int n, float x) {
-                          sm.G[m * LD + n] = x;  // Gm = Linv^T (Khat H)
+    wrun_sync<3, NB, NP, true, false>(kC, dv, nc, [&](int m, int s2) { return linv(sm, s2, m); },
+                                      [&](int s2, int n) { return sm.G[s2 * LD + n]; }, [&](int m, int n, float x) {
+                          sm.G[m * LD + n] = tf32_round(x);  // Gm = Linv^T (Khat H), an operand from here on
                           if (m < nc) dvg[(t0 + m) * dv + n] = sm.b[m] * x;
                         });
     __syncthreads();
@@ -878,14 +893,14 @@ __global__ void __launch_bounds__(32 * NW, 1) gdn_bwd_frame_mma_kernel(BwdParams
       const int half = warp / (6 / NB), n0 = (warp % (6 / NB)) * 8 * NB;
       float r[3][NB][4] = {};
       if (half == 0) {
-        wmm<3, NB, NP>(r, 0, n0, dv, [&](int m, int jj) { return sm.E[m * LD + jj]; },
-                       [&](int jj, int n) { return sm.G[n * LD + jj]; });
+        wmm<3, NB, NP, false, false>(r, 0, n0, dv, [&](int m, int jj) { return sm.E[m * LD + jj]; },
+                                     [&](int jj, int n) { return sm.G[n * LD + jj]; });
         each(r, 0, n0, [&](int m, int n, float x) {
           if (n >= m) sm.M[m * LDC + n] = n > m ? sm.b[n] * x : 0.f;
         });
       } else {
-        wmm<3, NB, NP>(r, 0, n0, dv, [&](int m, int jj) { return sm.G[m * LD + jj]; },
-                       [&](int jj, int n) { return sm.U[n * LD + jj]; });
+        wmm<3, NB, NP, false, false>(r, 0, n0, dv, [&](int m, int jj) { return sm.G[m * LD + jj]; },
+                                     [&](int jj, int n) { return sm.U[n * LD + jj]; });
         each(r, 0, n0, [&](int m, int n, float x) {
           if (n < m) sm.M[m * LDC + n] = x;
         });
@@ -897,12 +912,12 @@ __global__ void __launch_bounds__(32 * NW, 1) gdn_bwd_frame_mma_kernel(BwdParams
       const bool has = n0 < dk;
       float a[3][NB][4] = {};
       if (has) {
-        wmm<3, NB, NP>(a, 0, n0, dv, [&](int m, int jj) { return sm.E[m * LD + jj]; },
-                       [&](int jj, int n) { return sm.H[n * LD + jj]; });
-        wmm<3, NB, NP>(a, 0, n0, dv, [&](int m, int jj) { return -sm.G[m * LD + jj]; },
-                       [&](int jj, int n) { return sm.S[n * LD + jj]; });
-        wmm<3, NB, NP>(a, 0, n0, nc, [&](int m, int s2) { return -sm.M[m * LDC + s2]; },
-                       [&](int s2, int n) { return sm.K[s2 * LD + n]; });
+        wmm<3, NB, NP, false, true>(a, 0, n0, dv, [&](int m, int jj) { return sm.E[m * LD + jj]; },
+                                    [&](int jj, int n) { return sm.H[n * LD + jj]; });
+        wmm<3, NB, NP, false, true>(a, 0, n0, dv, [&](int m, int jj) { return -sm.G[m * LD + jj]; },
+                                    [&](int jj, int n) { return sm.S[n * LD + jj]; });
+        wmm<3, NB, NP, true, false>(a, 0, n0, nc, [&](int m, int s2) { return -sm.M[m * LDC + s2]; },
+                                    [&](int s2, int n) { return sm.K[s2 * LD + n]; });
       }
       __syncthreads();
       if (has) each(a, 0, n0, [&](int m, int n, float x) { sm.U[m * LD + n] = sm.b[m] * x; });
@@ -921,8 +936,8 @@ __global__ void __launch_bounds__(32 * NW, 1) gdn_bwd_frame_mma_kernel(BwdParams
         dkg[(t0 + t) * dk + i] = gk * sc;
       }
     }
-    wrun<ND, NB, NP>(dk, dv, nc, [&](int m, int t) { return sm.K[t * LD + m] * sm.b[t]; },
-                    [&](int t, int n) { return sm.G[t * LD + n]; },
+    wrun<ND, NB, NP, true, false>(dk, dv, nc, [&](int m, int t) { return sm.K[t * LD + m] * sm.b[t]; },
+                                  [&](int t, int n) { return sm.G[t * LD + n]; },
                     [&](int m, int n, float x) { sm.H[m * LD + n] -= x; });  // H -= Khat^T diag(beta) Gm
     __syncthreads();
   }
