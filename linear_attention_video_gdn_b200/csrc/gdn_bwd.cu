@@ -143,6 +143,19 @@ __device__ __forceinline__ void tile_load(float *dst, int ldd, const T *src, lon
   }
 }
 
+// Asynchronous global -> shared copies of fp32 rows, 16 bytes per cp.async:
+// dst[r * ldd + c] = src[r * gs + c] for r < rows, c < cols (cols, gs and ldd
+// multiples of 4, both bases 16-byte aligned).  The caller commits the group,
+// waits for it and then synchronises the block before the rows are read.
+__device__ __forceinline__ void tile_load_async(float *dst, int ldd, const float *src, long gs, int rows, int cols) {
+  const int cv = cols >> 2, nv = rows * cv;
+  for (int e = threadIdx.x; e < nv; e += blockDim.x) {
+    const int row = e / cv, c4 = e - row * cv;
+    const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst + row * ldd + 4 * c4);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(src + row * gs + 4 * c4) : "memory");
+  }
+}
+
 // Ask L2 for [base, base + bytes) (128-byte lines spread over the block's threads).
 __device__ __forceinline__ void prefetch_l2(const void *base, long bytes) {
   const char *b = static_cast<const char *>(base);
@@ -852,19 +865,34 @@ __global__ void __launch_bounds__(32 * NW, 1) gdn_bwd_frame_mma_kernel(BwdParams
     __syncthreads();
   }
 
-  // ---- reverse sweep (U, R and Linv kept by the forward sweep)
+  // ---- reverse sweep (U, R and Linv kept by the forward sweep).  Chunk c's U, R and
+  // Linv arrive by asynchronous copies issued during chunk c + 1's H update.
+  const bool async_rows = dv % 4 == 0 && rld % 4 == 0;
+  auto fetch = [&](int cc) {  // U, R and Linv of chunk cc -> U, E and M (rows past the frame zero)
+    const long tt = (long)f * L + cc * kC;
+    const int n = min(kC, L - cc * kC);
+    if (async_rows) {
+      tile_load_async(sm.U, LD, dvg + tt * dv, dv, n, dv);
+      tile_load_async(sm.E, LD, rdst + tt * rld, rld, n, dv);
+      tile_load_async(sm.M, LDC, lbuf + cc * (kC * kC), kC, kC, kC);
+      asm volatile("cp.async.commit_group;" ::: "memory");
+      for (int e = tid; e < (kC - n) * dv; e += kTh) {
+        const int row = n + e / dv, col = e % dv;
+        sm.U[row * LD + col] = 0.f;
+        sm.E[row * LD + col] = 0.f;
+      }
+    } else {
+      tile_load(sm.U, LD, dvg + tt * dv, dv, kC, n, dv);
+      tile_load(sm.E, LD, rdst + tt * rld, rld, kC, n, dv);
+      tile_load(sm.M, LDC, lbuf + cc * (kC * kC), kC, kC, kC, kC);
+    }
+  };
+  fetch(nch - 1);
   for (int c = nch - 1; c >= 0; --c) {
     const long t0 = (long)f * L + c * kC;
     const int nc = min(kC, L - c * kC);
-    if (c > 0) {
-      prefetch_l2(k + (t0 - kC) * dk, (long)kC * dk * sizeof(T));
-      prefetch_l2(dvg + (t0 - kC) * dv, (long)kC * dv * sizeof(float));
-      prefetch_l2(rdst + (t0 - kC) * rld, (long)kC * rld * sizeof(float));
-      prefetch_l2(lbuf + (c - 1) * (kC * kC), (long)kC * kC * sizeof(float));
-    }
-    tile_load(sm.U, LD, dvg + t0 * dv, dv, kC, nc, dv);
-    tile_load(sm.E, LD, rdst + t0 * rld, rld, kC, nc, dv);
-    tile_load(sm.M, LDC, lbuf + c * (kC * kC), kC, kC, kC, kC);
+    if (c > 0) prefetch_l2(k + (t0 - kC) * dk, (long)kC * dk * sizeof(T));
+    asm volatile("cp.async.wait_all;" ::: "memory");  // this thread's copies; load_chunk's barrier publishes them
     load_chunk<SM, T, false, true>(sm, p, k, v, beta, t0, nc, tid);
     wrun<ND, NB, NP, false, false>(dk, dv, nc, Kcol, [&](int t, int n) { return sm.U[t * LD + n]; },
                                    [&](int m, int n, float x) { sm.S[m * LD + n] -= x; });  // the chunk's start state
@@ -936,6 +964,8 @@ __global__ void __launch_bounds__(32 * NW, 1) gdn_bwd_frame_mma_kernel(BwdParams
         dkg[(t0 + t) * dk + i] = gk * sc;
       }
     }
+    __syncthreads();  // U (dkhat), E (R) and M are dead: the next chunk's arrive under the H update
+    if (c > 0) fetch(c - 1);
     wrun<ND, NB, NP, true, false>(dk, dv, nc, [&](int m, int t) { return sm.K[t * LD + m] * sm.b[t]; },
                                   [&](int t, int n) { return sm.G[t * LD + n]; },
                     [&](int m, int n, float x) { sm.H[m * LD + n] -= x; });  // H -= Khat^T diag(beta) Gm
