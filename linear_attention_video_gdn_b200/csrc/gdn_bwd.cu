@@ -852,18 +852,34 @@ __global__ void __launch_bounds__(32 * NW, 1) gdn_bwd_frame_mma_kernel(BwdParams
     __syncthreads();
   }
 
-  // ---- dq = dO S_f^T
+  // ---- dq = dO S_f^T, the dO rows double-buffered in G and U (free here): the next
+  // chunk's arrive by asynchronous copies while this chunk's product runs
+  auto fetch_do = [&](int cc) {
+    const long tt = (long)f * L + cc * kC;
+    const int n = min(kC, L - cc * kC);
+    float *dst = (cc & 1) ? sm.U : sm.G;
+    if (dv % 4 == 0) {
+      tile_load_async(dst, LD, d_o + tt * dv, dv, n, dv);
+      asm volatile("cp.async.commit_group;" ::: "memory");
+      for (int e = tid; e < (kC - n) * dv; e += kTh) dst[(n + e / dv) * LD + e % dv] = 0.f;
+    } else {
+      tile_load(dst, LD, d_o + tt * dv, dv, kC, n, dv);
+    }
+  };
+  fetch_do(0);
   for (int c = 0; c < nch; ++c) {
     const long t0 = (long)f * L + c * kC;
     const int nc = min(kC, L - c * kC);
-    tile_load<true>(sm.G, LD, d_o + t0 * dv, dv, kC, nc, dv);  // dO rows, rounded to tf32 once
-    __syncthreads();
-    wrun<3, NB, NP, false, true>(kC, dk, dv, [&](int m, int jj) { return sm.G[m * LD + jj]; },
-                   [&](int jj, int n) { return sm.S[n * LD + jj]; }, [&](int m, int n, float x) {
-                     if (m < nc) dq[(t0 + m) * dk + n] = x;
-                   });
-    __syncthreads();
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    __syncthreads();  // chunk c's rows are visible; chunk c - 1's product is done with the other buffer
+    if (c + 1 < nch) fetch_do(c + 1);
+    const float *dcur = (c & 1) ? sm.U : sm.G;
+    wrun<3, NB, NP>(kC, dk, dv, [&](int m, int jj) { return dcur[m * LD + jj]; },
+                    [&](int jj, int n) { return sm.S[n * LD + jj]; }, [&](int m, int n, float x) {
+                      if (m < nc) dq[(t0 + m) * dk + n] = x;
+                    });
   }
+  __syncthreads();
 
   // ---- reverse sweep (U, R and Linv kept by the forward sweep).  Chunk c's U, R and
   // Linv arrive by asynchronous copies issued during chunk c + 1's H update.
