@@ -131,3 +131,14 @@ def test_recompute_timeout_status_is_reported(lib, dev, dtype):
     out, ref = run(lib, dev, w, x, d_o, si, dso, status=st)
     assert int(st[0].item()) == 0
     check(out, ref, TOL_F32 if dtype == "f32" else TOL_BF16)
+
+
+def test_480p_5s_all_heads(lib, dev):
+    """The 480p 5 s workload (B=1, H=20, F=21, L=390, d=112, bf16) with a start
+    state and dL/dstate_out: every head, frame, token and column against the
+    oracle."""
+    w = synth.WORKLOADS["gdn_480p_5s"]
+    x = synth.inputs(w)
+    g = synth.grad_inputs(w, state_in=True, dstate_out=True)
+    out, ref = run(lib, dev, w, x, g["d_o"], g["state_in"], g["dstate_out"])
+    check(out, ref, TOL_BF16)
