@@ -54,7 +54,7 @@ def _load():
         lib.oracle_temporal_conv.restype = ctypes.c_int
         lib.oracle_gdn.restype = ctypes.c_int
         lib.oracle_gdn_bwd.argtypes = [P, P, P, P, P, ctypes.c_int, P, P, P, P, P, P, P, P, P,
-                                       I64, I64, I64, I64, I64, I64, P, I64, ctypes.c_int]
+                                       I64, I64, I64, I64, I64, I64, P, I64, ctypes.c_int, I64, I64, ctypes.c_double]
         lib.oracle_gdn_bwd.restype = ctypes.c_int
         lib.oracle_relu_la.argtypes = [P, P, P, P, P, P, P, P, I64, I64, I64, I64, I64, I64, ctypes.c_double,
                                        ctypes.c_int]
@@ -127,7 +127,7 @@ def gdn(q, k, v, alpha, beta, *, F: int, L: int, gates_are_logits: bool = True, 
 
 
 def gdn_bwd(q, k, v, alpha, beta, d_o, *, F: int, L: int, gates_are_logits: bool = True, state_in=None,
-            dstate_out=None, heads=None, nthreads: int | None = None):
+            dstate_out=None, heads=None, nthreads: int | None = None, rope=None):
     """Backward of the Gated DeltaNet frame recurrence in fp64 (see oracle.c).
 
     Shapes as in ``gdn``; d_o: [..., F*L, dv] (dL/do), dstate_out: [..., dk, dv]
@@ -135,7 +135,8 @@ def gdn_bwd(q, k, v, alpha, beta, d_o, *, F: int, L: int, gates_are_logits: bool
     dv [..., F*L, dv], dalpha [..., F] and dbeta [..., F*L] (with respect to the
     logits when ``gates_are_logits``, else the gate values) and dstate_in
     [..., dk, dv].  heads: optional subset of flat head indices (the others'
-    entries are NaN)."""
+    entries are NaN).  rope: as in ``gdn`` (the gradients are with respect to
+    the unrotated q and k)."""
     q, k, v, alpha, beta, d_o = map(_f32, (q, k, v, alpha, beta, d_o))
     lead = q.shape[:-2]
     N, dk = q.shape[-2:]
@@ -154,7 +155,8 @@ def gdn_bwd(q, k, v, alpha, beta, d_o, *, F: int, L: int, gates_are_logits: bool
     rc = _load().oracle_gdn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), int(gates_are_logits),
                                 _ptr(s_in), _ptr(d_o), _ptr(ds_out), _ptr(out["dq"]), _ptr(out["dk"]),
                                 _ptr(out["dv"]), _ptr(out["dalpha"]), _ptr(out["dbeta"]), _ptr(out["dstate_in"]),
-                                1, nh, F, L, dk, dv, _ptr(hl), 0 if hl is None else hl.size, nthreads)
+                                1, nh, F, L, dk, dv, _ptr(hl), 0 if hl is None else hl.size, nthreads,
+                                *_rope_args(rope))
     if rc != 0:
         raise ValueError("oracle_gdn_bwd: invalid arguments")
     return out

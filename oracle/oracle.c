@@ -102,6 +102,26 @@ static void rope3d(const float *x, int64_t d, int64_t frame, int64_t row, int64_
   }
 }
 
+/* The rotation of a double d-vector by sign times rope3d's angles (sign = -1:
+ * the transpose, which maps a gradient with respect to the rotated vector to
+ * one with respect to the vector). */
+static void rope3d_rot(const double *x, int64_t d, int64_t frame, int64_t row, int64_t col, double base, double sign,
+                       double *out) {
+  const int64_t dh = 2 * (d / 6), dw = dh, dt = d - dh - dw;
+  const int64_t len[3] = {dt, dh, dw}, pos[3] = {frame, row, col};
+  int64_t o = 0;
+  for (int a = 0; a < 3; ++a) {
+    for (int64_t i = 0; i < len[a] / 2; ++i) {
+      const double phi = sign * (double)pos[a] * pow(base, -2.0 * (double)i / (double)len[a]);
+      const double c = cos(phi), sn = sin(phi);
+      const double x0 = x[o + 2 * i], x1 = x[o + 2 * i + 1];
+      out[o + 2 * i] = x0 * c - x1 * sn;
+      out[o + 2 * i + 1] = x0 * sn + x1 * c;
+    }
+    o += len[a];
+  }
+}
+
 /* The embedding alone: x [n_heads, F*L, d] -> out (double), for tests. */
 int oracle_rope3d(const float *x, double *out, int64_t nh, int64_t F, int64_t L, int64_t d, int64_t grid_w,
                   int64_t frame_offset, double base) {
@@ -261,7 +281,7 @@ int oracle_gdn(const float *q, const float *k, const float *v, const float *alph
 }
 
 /*
- * Backward of the Gated DeltaNet frame recurrence (no position embedding).
+ * Backward of the Gated DeltaNet frame recurrence.
  *
  * The model is trained (SANA-WM GeekNews summary, "Core design and generation
  * pipeline": 64 H100 GPUs over 15 days), so the recurrence above needs its
@@ -271,6 +291,10 @@ int oracle_gdn(const float *q, const float *k, const float *v, const float *alph
  * the logits a, b when gates_are_logits, else the gate values), and
  * dL/dstate_in [B,H,dk,dv] (also when state_in is NULL: the gradient with
  * respect to the zero start state).
+ *
+ * With the 3D RoPE (rope_grid_w > 0), q_t and k_t are rotated as in the
+ * forward (k before its normalisation) and the gradients with respect to the
+ * rotated vectors are rotated back by the transpose rotation.
  *
  * Reverse-mode differentiation of the forward above, one head at a time:
  *   1. Forward over the frames, keeping S_{f-1} (the state before frame f's
@@ -305,6 +329,7 @@ typedef struct {
   const double *s_in, *ds_out;
   double *dq, *dk, *dv, *dal, *dbe, *ds_in;
   int64_t F, L, dk_, dv_, bh;
+  rope_t rope;         /* 3D RoPE on q and k (k before its normalisation) */
 } gdn_bwd_unit_t;
 
 static void gdn_bwd_unit(const gdn_bwd_unit_t *u) {
@@ -320,18 +345,26 @@ static void gdn_bwd_unit(const gdn_bwd_unit_t *u) {
   double *r = (double *)malloc(sizeof(double) * (size_t)(L * dv));   /* the frame's residuals */
   double *g = (double *)malloc(sizeof(double) * (size_t)dv);
   double *dkh = (double *)malloc(sizeof(double) * (size_t)dk);
+  double *qr = (double *)malloc(sizeof(double) * (size_t)dk); /* q_t (rotated with the embedding) */
+  double *grot = (double *)malloc(sizeof(double) * (size_t)dk); /* a gradient with respect to a rotated vector */
   if (u->s_in)
     for (int64_t e = 0; e < SS; ++e) S[e] = u->s_in[bh * SS + e];
   /* khat_t and ||k_t|| for token t of frame f (index tl in the frame) */
 #define GDN_BWD_KEY(f, tl)                                                        \
   do {                                                                            \
     const float *kt = k + ((f) * L + (tl)) * dk;                                  \
+    double *kx = kh + (tl) * dk;                                                  \
+    if (u->rope.on)                                                               \
+      rope3d(kt, dk, u->rope.frame_offset + (f), (tl) / u->rope.grid_w,           \
+             (tl) % u->rope.grid_w, u->rope.base, kx);                            \
+    else                                                                          \
+      for (int64_t i = 0; i < dk; ++i) kx[i] = (double)kt[i];                     \
     double ss = 0.0;                                                              \
-    for (int64_t i = 0; i < dk; ++i) ss += (double)kt[i] * (double)kt[i];         \
+    for (int64_t i = 0; i < dk; ++i) ss += kx[i] * kx[i];                         \
     const double n_ = sqrt(ss);                                                   \
     const double den = n_ > GDN_KEY_NORM_EPS ? n_ : GDN_KEY_NORM_EPS;             \
     nrm[tl] = n_;                                                                 \
-    for (int64_t i = 0; i < dk; ++i) kh[(tl) * dk + i] = (double)kt[i] / den;     \
+    for (int64_t i = 0; i < dk; ++i) kx[i] = kx[i] / den;                         \
   } while (0)
   /* 1. forward over the frames */
   for (int64_t f = 0; f < F; ++f) {
@@ -370,16 +403,25 @@ static void gdn_bwd_unit(const gdn_bwd_unit_t *u) {
       for (int64_t i = 0; i < dk; ++i)
         for (int64_t j = 0; j < dv; ++j) S[i * dv + j] -= beta * x[i] * rt[j];
     }
-    /* read-out: o_t = S_f^T q_t */
+    /* read-out: o_t = S_f^T q_t (q_t rotated with the embedding; its gradient rotated back) */
     for (int64_t tl = 0; tl < L; ++tl) {
       const int64_t t = f * L + tl;
+      if (u->rope.on)
+        rope3d(q + t * dk, dk, u->rope.frame_offset + f, tl / u->rope.grid_w, tl % u->rope.grid_w, u->rope.base, qr);
+      else
+        for (int64_t i = 0; i < dk; ++i) qr[i] = (double)q[t * dk + i];
       for (int64_t i = 0; i < dk; ++i) {
         double acc = 0.0;
         for (int64_t j = 0; j < dv; ++j) acc += S[i * dv + j] * (double)d_o[t * dv + j];
-        u->dq[(bh * N + t) * dk + i] = acc;
+        grot[i] = acc;
       }
+      if (u->rope.on)
+        rope3d_rot(grot, dk, u->rope.frame_offset + f, tl / u->rope.grid_w, tl % u->rope.grid_w, u->rope.base, -1.0,
+                   u->dq + (bh * N + t) * dk);
+      else
+        for (int64_t i = 0; i < dk; ++i) u->dq[(bh * N + t) * dk + i] = grot[i];
       for (int64_t i = 0; i < dk; ++i)
-        for (int64_t j = 0; j < dv; ++j) H[i * dv + j] += (double)q[t * dk + i] * (double)d_o[t * dv + j];
+        for (int64_t j = 0; j < dv; ++j) H[i * dv + j] += qr[i] * (double)d_o[t * dv + j];
     }
     /* tokens in reverse */
     for (int64_t tl = L - 1; tl >= 0; --tl) {
@@ -410,10 +452,16 @@ static void gdn_bwd_unit(const gdn_bwd_unit_t *u) {
       if (nrm[tl] > GDN_KEY_NORM_EPS) {
         double kd = 0.0;
         for (int64_t i = 0; i < dk; ++i) kd += x[i] * dkh[i];
-        for (int64_t i = 0; i < dk; ++i) u->dk[(bh * N + t) * dk + i] = (dkh[i] - x[i] * kd) / nrm[tl];
+        for (int64_t i = 0; i < dk; ++i) grot[i] = (dkh[i] - x[i] * kd) / nrm[tl];
       } else {
-        for (int64_t i = 0; i < dk; ++i) u->dk[(bh * N + t) * dk + i] = dkh[i] / GDN_KEY_NORM_EPS;
+        for (int64_t i = 0; i < dk; ++i) grot[i] = dkh[i] / GDN_KEY_NORM_EPS;
       }
+      /* grot = dL/d(the rotated key); the key's own gradient is its transpose rotation */
+      if (u->rope.on)
+        rope3d_rot(grot, dk, u->rope.frame_offset + f, tl / u->rope.grid_w, tl % u->rope.grid_w, u->rope.base, -1.0,
+                   u->dk + (bh * N + t) * dk);
+      else
+        for (int64_t i = 0; i < dk; ++i) u->dk[(bh * N + t) * dk + i] = grot[i];
       u->dbe[bh * N + t] = u->logits ? dbeta * beta * (1.0 - beta) : dbeta;
     }
     /* frame start: H = dL/d(alpha_f S_{f-1}) */
@@ -433,6 +481,8 @@ static void gdn_bwd_unit(const gdn_bwd_unit_t *u) {
   free(r);
   free(g);
   free(dkh);
+  free(qr);
+  free(grot);
 }
 
 typedef struct {
@@ -456,9 +506,11 @@ int oracle_gdn_bwd(const float *q, const float *k, const float *v, const float *
                    int gates_are_logits, const double *state_in, const float *d_o, const double *dstate_out,
                    double *dq, double *dk, double *dv, double *dalpha, double *dbeta, double *dstate_in,
                    int64_t B, int64_t H, int64_t F, int64_t L, int64_t dk_, int64_t dv_,
-                   const int64_t *heads, int64_t nheads, int nthreads) {
+                   const int64_t *heads, int64_t nheads, int nthreads, int64_t rope_grid_w,
+                   int64_t rope_frame_offset, double rope_base) {
   if (B < 0 || H < 0 || F < 0 || L < 0 || dk_ <= 0 || dv_ <= 0) return 1;
   if (!dq || !dk || !dv || !dalpha || !dbeta) return 1;
+  if (rope_grid_w > 0 && (dk_ % 2 || L % rope_grid_w)) return 1;
   const int64_t n = heads ? nheads : B * H;
   if (n <= 0) return 0;
   gdn_bwd_unit_t *units = (gdn_bwd_unit_t *)calloc((size_t)n, sizeof(gdn_bwd_unit_t));
@@ -469,6 +521,10 @@ int oracle_gdn_bwd(const float *q, const float *k, const float *v, const float *
     u->dq = dq; u->dk = dk; u->dv = dv; u->dal = dalpha; u->dbe = dbeta; u->ds_in = dstate_in;
     u->F = F; u->L = L; u->dk_ = dk_; u->dv_ = dv_;
     u->bh = heads ? heads[h] : h;
+    u->rope.on = rope_grid_w > 0;
+    u->rope.grid_w = rope_grid_w > 0 ? rope_grid_w : 1;
+    u->rope.frame_offset = rope_frame_offset;
+    u->rope.base = rope_base;
   }
   bwd_pool_t pl;
   pl.units = units; pl.n = n; pl.next = 0;

@@ -44,7 +44,7 @@ def _case(rng, nh, F, L, dk, dv, logits=True):
 def _loss(c, F, L, logits, **over):
     x = dict(c, **over)
     o, s = oracle.gdn(x["q"], x["k"], x["v"], x["a"], x["b"], F=F, L=L, gates_are_logits=logits,
-                      state_in=x["s_in"], nthreads=1)
+                      state_in=x["s_in"], nthreads=1, rope=x.get("rope"))
     return float(np.sum(o * x["d_o"].astype(np.float64)) + np.sum(s * x["ds_out"]))
 
 
@@ -74,7 +74,7 @@ def _check_fd(c, g, F, L, logits, names=GRAD, h=2.0 ** -10, rtol=1e-7):
 
 def _bwd(c, F, L, logits, **kw):
     return oracle.gdn_bwd(c["q"], c["k"], c["v"], c["a"], c["b"], c["d_o"], F=F, L=L, gates_are_logits=logits,
-                          state_in=c["s_in"], dstate_out=c["ds_out"], nthreads=1, **kw)
+                          state_in=c["s_in"], dstate_out=c["ds_out"], nthreads=1, rope=c.get("rope"), **kw)
 
 
 @pytest.mark.parametrize("F,L,dk,dv,logits", [(3, 4, 4, 3, True), (2, 3, 3, 5, False), (1, 1, 2, 2, True),
@@ -83,6 +83,22 @@ def test_bwd_matches_finite_differences(F, L, dk, dv, logits):
     rng = np.random.default_rng(100 + F * 10 + L)
     c = _case(rng, 1, F, L, dk, dv, logits)
     _check_fd(c, _bwd(c, F, L, logits), F, L, logits)
+
+
+@pytest.mark.parametrize("F,L,d,gw,off", [(3, 4, 8, 2, 0), (2, 6, 12, 3, 5)])
+def test_bwd_with_rope_matches_finite_differences(F, L, d, gw, off):
+    """With the 3D RoPE on q and k: the gradients with respect to the unrotated
+    q and k (and every other input) against central differences of the forward
+    oracle with the same embedding."""
+    rng = np.random.default_rng(200 + d)
+    c = _case(rng, 1, F, L, d, 3)
+    c["rope"] = dict(grid_w=gw, frame_offset=off, base=100.0)
+    g = _bwd(c, F, L, True)
+    _check_fd(c, g, F, L, True)
+    c0 = dict(c)
+    c0.pop("rope")
+    g0 = _bwd(c0, F, L, True)
+    assert np.abs(g["dk"] - g0["dk"]).max() > 1e-3  # the embedding changes the key gradients
 
 
 def _torch_forward(c, F, L, logits, leaves):
