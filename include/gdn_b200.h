@@ -174,7 +174,8 @@ GDN_API int gdn_frame_fwd(const void *q, const void *k, const void *v, const flo
                   int dk, int dv, const gdn_opts_t *opts);
 
 /*
- * gdn_frame_bwd -- backward of gdn_frame_fwd (without the position embedding).
+ * gdn_frame_bwd -- backward of gdn_frame_fwd, with or without the 3D position
+ * embedding.
  *
  * The model is trained (SANA-WM GeekNews summary, "Core design and generation
  * pipeline": 64 H100 GPUs over 15 days), so the recurrence needs its
@@ -206,8 +207,14 @@ GDN_API int gdn_frame_fwd(const void *q, const void *k, const void *v, const flo
  * Sizes: as gdn_frame_fwd, with dk, dv <= 112.  Workspace:
  * gdn_workspace_bytes(GDN_OP_GDN_BWD, ...) (four fp32 d x d matrices per frame,
  * with bf16 inputs a 48 x 48 matrix per 48-token chunk and, when dv > dk, a
- * row per token, plus the recompute's scratch).  opts->rope_grid_w must be 0
- * (GDN_ERR_UNSUPPORTED otherwise).
+ * row per token, plus the recompute's scratch, plus the RoPE table).
+ *
+ * 3D RoPE (opts->rope_grid_w > 0, the forward call's rope_grid_w,
+ * rope_frame_offset and rope_base; the same checks): the recompute is
+ * FRAME_SIMT (GDN_IMPL_TC is refused with GDN_ERR_UNSUPPORTED); the kernels
+ * rotate q and k where they load them, and d_q, d_k are turned back through
+ * the transpose rotation, so they are gradients with respect to the unrotated
+ * inputs, as the forward receives them.
  *
  * Precision: with bf16 inputs the recomputed A_f and S_f carry the tensor-core
  * forward's rounding (see gdn_frame_fwd), and the products of Q_f^T dO_f and of

@@ -197,7 +197,7 @@ def gdn_frame_fwd(q, k, v, alpha, beta, *, F: int, state_in=None, state_out=None
 
 def gdn_frame_bwd(q, k, v, alpha, beta, d_o, *, F: int, state_in=None, d_state_out=None, out=None,
                   gates_are_logits: bool = True, impl="auto", workspace=None, stream=None, status=None,
-                  max_ctas: int = 0, spin_limit_us: int = 0, test_withhold_unit: int = -1):
+                  max_ctas: int = 0, spin_limit_us: int = 0, test_withhold_unit: int = -1, rope=None):
     """Backward of ``gdn_frame_fwd`` on the GPU (see include/gdn_b200.h).
 
     q, k, v, alpha, beta, state_in: the forward call's inputs; d_o: [B, H, F*L, dv]
@@ -205,7 +205,9 @@ def gdn_frame_bwd(q, k, v, alpha, beta, d_o, *, F: int, state_in=None, d_state_o
     a dict of float32 tensors dq, dk [B, H, F*L, dk], dv [B, H, F*L, dv],
     dalpha [B, H, F], dbeta [B, H, F*L] (with respect to the logits when
     ``gates_are_logits``) and dstate_in [B, H, dk, dv].  ``out``: an optional
-    dict of preallocated tensors with those names.
+    dict of preallocated tensors with those names.  ``rope``: the forward's 3D
+    RoPE options (dict(grid_w, frame_offset=0, base=1e4)), or None; dq and dk are
+    then with respect to the unrotated q and k.
     """
     B, H, N, dk = q.shape
     dv = v.shape[-1]
@@ -230,7 +232,7 @@ def gdn_frame_bwd(q, k, v, alpha, beta, d_o, *, F: int, state_in=None, d_state_o
         _check(out[name], name, shp, torch.float32, dev)
     opts = make_opts(_dtype_code(q), gates_are_logits=gates_are_logits, impl=impl, stream=stream,
                      status=status, max_ctas=max_ctas, spin_limit_us=spin_limit_us,
-                     test_withhold_unit=test_withhold_unit)
+                     test_withhold_unit=test_withhold_unit, rope=rope)
     need = workspace_bytes(OP_GDN_BWD, B, H, F, L, dk, dv, opts)
     if workspace is None:
         workspace = alloc_workspace(need, dev)

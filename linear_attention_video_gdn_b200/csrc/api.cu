@@ -198,17 +198,20 @@ extern "C" const char *gdn_status_str(int s) { return gdn_status_string(s); }
 namespace gdn {
 namespace {
 // The backward's forward recompute: the tensor-core kernel for bf16 inputs where it
-// applies (one unit per frame), else the fp32 CUDA-core frame kernel.
+// applies (one unit per frame, no position embedding), else the fp32 CUDA-core
+// frame kernel.
 int pick_bwd_fwd_impl(const gdn_opts_t *o, int dk, int dv) {
   if (o->impl == GDN_IMPL_FRAME_SIMT) return GDN_IMPL_FRAME_SIMT;
   if (o->impl == GDN_IMPL_TC) return GDN_IMPL_TC;
+  if (o->rope_grid_w != 0) return GDN_IMPL_FRAME_SIMT;
   return o->in_dtype == GDN_DTYPE_BF16 && gdn_tc_supported(dk, dv) ? GDN_IMPL_TC : GDN_IMPL_FRAME_SIMT;
 }
 
 // Backward workspace: the recompute's chain scratch, then A_f^T and S_f of every
-// frame, G_f of every frame, and the per-column-group dalpha partial sums.
+// frame, G_f of every frame, the per-column-group dalpha partial sums, (bf16
+// inputs) each chunk's Linv and the residuals, and (with the 3D RoPE) its table.
 struct BwdLayout {
-  size_t maps, states, gbuf, part, linv, rbuf, total;
+  size_t maps, states, gbuf, part, linv, rbuf, rope, total;
 };
 BwdLayout bwd_layout(const gdn_opts_t *o, int B, int H, int F, int L, int dk, int dv) {
   BwdLayout w;
@@ -224,6 +227,8 @@ BwdLayout bwd_layout(const gdn_opts_t *o, int B, int H, int F, int L, int dk, in
     w.rbuf = w.linv + align_up(sizeof(float) * fr * gdn_bwd_chunks(L) * 48 * 48, 256);
     w.total = w.rbuf + (dv > dk ? align_up(sizeof(float) * fr * L * dv, 256) : 0);
   }
+  w.rope = w.total;
+  w.total += gdn_rope_bytes(o, F, L, dk);
   return w;
 }
 }  // namespace
@@ -247,10 +252,13 @@ extern "C" int gdn_frame_bwd(const void *q, const void *k, const void *v, const 
   if (opts->in_dtype != GDN_DTYPE_F32 && opts->in_dtype != GDN_DTYPE_BF16) return GDN_ERR_INVALID_ARG;
   if (opts->impl != GDN_IMPL_AUTO && opts->impl != GDN_IMPL_FRAME_SIMT && opts->impl != GDN_IMPL_TC)
     return GDN_ERR_INVALID_ARG;
-  if (opts->rope_grid_w != 0) return GDN_ERR_UNSUPPORTED;  // the backward covers gdn without the embedding
   int rc = check_sizes(B, H, F, L, dk, dv);
   if (rc != GDN_OK) return rc;
   if (!gdn_bwd_supported(dk, dv)) return GDN_ERR_UNSUPPORTED;
+  const bool rope = opts->rope_grid_w != 0;
+  if (rope && (opts->rope_grid_w < 0 || L % opts->rope_grid_w || dk % 2 || !(opts->rope_base >= 0.0f) ||
+               opts->rope_frame_offset < 0))
+    return GDN_ERR_INVALID_ARG;
   const void *ptrs[] = {q, k, v, alpha, beta, state_in, d_o, dstate_out, dq, dk_out, dv_out, dalpha, dbeta,
                         dstate_in, opts->workspace, opts->status};
   for (const void *ptr : ptrs)
@@ -273,7 +281,7 @@ extern "C" int gdn_frame_bwd(const void *q, const void *k, const void *v, const 
   if (rc != GDN_OK) return rc;
   if (cc != 100) return GDN_ERR_NO_DEVICE;
   const int fimpl = pick_bwd_fwd_impl(opts, dk, dv);
-  if (fimpl == GDN_IMPL_TC && (opts->in_dtype != GDN_DTYPE_BF16 || !gdn_tc_supported(dk, dv)))
+  if (fimpl == GDN_IMPL_TC && (opts->in_dtype != GDN_DTYPE_BF16 || !gdn_tc_supported(dk, dv) || rope))
     return GDN_ERR_UNSUPPORTED;
   const BwdLayout w = bwd_layout(opts, B, H, F, L, dk, dv);
   if (!opts->workspace || opts->workspace_bytes < w.total) return GDN_ERR_INVALID_ARG;
@@ -300,6 +308,15 @@ extern "C" int gdn_frame_bwd(const void *q, const void *k, const void *v, const 
   p.ws = chain_workspace(ws, units);
   cudaError_t e = cudaMemsetAsync(ws, 0, chain_workspace_zero_bytes(units), st);
   if (e != cudaSuccess) return GDN_ERR_CUDA;
+  if (rope) {  // the table, filled on the stream before the recompute; the backward kernels read it too
+    p.rope_on = 1;
+    p.rope_gw = opts->rope_grid_w;
+    p.rope_dh = 2 * (dk / 6);
+    p.rope_dt = dk - 2 * p.rope_dh;
+    p.rope_tab = reinterpret_cast<const float2 *>(ws + w.rope);
+    e = launch_rope_table(p, opts->rope_frame_offset, opts->rope_base > 0.0f ? opts->rope_base : 10000.0f, st);
+    if (e != cudaSuccess) return GDN_ERR_CUDA;
+  }
   const int grid = grid_for(opts, sms, units);
   e = fimpl == GDN_IMPL_TC ? launch_gdn_tc(p, grid, false, st) : launch_gdn_frame_simt(p, opts->in_dtype, grid, st);
   if (e != cudaSuccess) return GDN_ERR_CUDA;
@@ -313,11 +330,11 @@ extern "C" int gdn_frame_bwd(const void *q, const void *k, const void *v, const 
   b.gbuf = reinterpret_cast<float *>(ws + w.gbuf);
   b.dal_part = reinterpret_cast<float *>(ws + w.part);
   b.linv_buf = reinterpret_cast<float *>(ws + w.linv);
-  b.rbuf = w.total > w.rbuf ? reinterpret_cast<float *>(ws + w.rbuf) : nullptr;
+  b.rbuf = w.rope > w.rbuf ? reinterpret_cast<float *>(ws + w.rbuf) : nullptr;  // own rows only when dv > dk
   b.dq = dq; b.dk_out = dk_out; b.dv_out = dv_out; b.dalpha = dalpha; b.dbeta = dbeta; b.dstate_in = dstate_in;
   b.B = B; b.H = H; b.F = F; b.L = L; b.dk = dk; b.dv = dv;
   b.gates_are_logits = p.gates_are_logits;
-  e = launch_gdn_bwd(b, opts->in_dtype, st);
+  e = launch_gdn_bwd(b, p, opts->in_dtype, st);
   return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 

@@ -274,10 +274,24 @@ struct FrameSmemT {
 template <int ND>
 using FrameSmem = FrameSmemT<ND, 1>;
 
-// Rows t0 .. t0 + nc - 1 of the frame: khat (normalised), beta and (kV) v.
+// The 3D rotary position embedding of rows [0, rows) of an fp32 tile (row t = the
+// token at index tf0 + t of frame f), in place, from the table in rp (rope_pair).
+__device__ __forceinline__ void rope_rows(float *x, int ld, int rows, int d, int f, int tf0, const GdnParams &rp) {
+  const int np = d / 2;
+  for (int e = threadIdx.x; e < rows * np; e += blockDim.x) {
+    const int t = e / np, pr = e - t * np;
+    float *px = x + t * ld + 2 * pr;
+    const float2 y = rope_pair(make_float2(px[0], px[1]), 2 * pr, f, tf0 + t, rp);
+    px[0] = y.x;
+    px[1] = y.y;
+  }
+}
+
+// Rows t0 .. t0 + nc - 1 of the frame: khat (normalised), beta and (kV) v.  With
+// the embedding (rp.rope_on), k is rotated before its normalisation.
 template <class SM, typename T, bool kV = true, bool kTf32 = false>
-__device__ __forceinline__ void load_chunk(SM &sm, const BwdParams &p, const T *k, const T *v, const float *beta,
-                                           long t0, int nc, int tid) {
+__device__ __forceinline__ void load_chunk(SM &sm, const BwdParams &p, const GdnParams &rp, const T *k, const T *v,
+                                           const float *beta, long t0, int nc, int tid) {
   constexpr int LD = SM::LD;
   const int dk = p.dk, dv = p.dv;
   tile_load(sm.K, LD, k + t0 * dk, dk, kC, nc, dk);
@@ -287,6 +301,11 @@ __device__ __forceinline__ void load_chunk(SM &sm, const BwdParams &p, const T *
     sm.b[tid] = tid < nc ? (p.gates_are_logits ? gate_beta(braw) : braw) : 0.f;
   }
   __syncthreads();
+  if (rp.rope_on) {
+    const int f = (int)(t0 / p.L);
+    rope_rows(sm.K, LD, nc, dk, f, (int)(t0 - (long)f * p.L), rp);
+    __syncthreads();
+  }
   const int warp = tid >> 5, lane = tid & 31;
   for (int t = warp; t < kC; t += (int)(blockDim.x >> 5)) {
     float ss = 0.f;
@@ -390,7 +409,7 @@ __device__ __forceinline__ float linv(const SM &sm, int t, int s) {
 }
 
 template <int ND, typename T>
-__global__ void __launch_bounds__(kThreads, 1) gdn_bwd_frame_kernel(BwdParams p) {
+__global__ void __launch_bounds__(kThreads, 1) gdn_bwd_frame_kernel(BwdParams p, GdnParams rp) {
   using SM = FrameSmem<ND>;
   constexpr int LD = SM::LD, kLdC = SM::LDC;
   extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -426,7 +445,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_frame_kernel(BwdParams p)
   for (int c = 0; c < nch; ++c) {
     const long t0 = (long)f * L + c * kC;
     const int nc = min(kC, L - c * kC);
-    load_chunk(sm, p, k, v, beta, t0, nc, tid);
+    load_chunk(sm, p, rp, k, v, beta, t0, nc, tid);
     gram_inverse<ND>(sm, nc, dk, tid);
     {  // E = V - Khat S
       float a[3][ND];
@@ -492,7 +511,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_frame_kernel(BwdParams p)
     const long t0 = (long)f * L + c * kC;
     const int nc = min(kC, L - c * kC);
     tile_load(sm.U, LD, dvg + t0 * dv, dv, kC, nc, dv);
-    load_chunk(sm, p, k, v, beta, t0, nc, tid);  // (its barriers order the U loads too)
+    load_chunk(sm, p, rp, k, v, beta, t0, nc, tid);  // (its barriers order the U loads too)
     {  // S -= Khat^T U: the chunk's start state
       float a[ND][ND];
       zero(a);
@@ -769,7 +788,7 @@ __device__ __forceinline__ void wrun_sync(int M, int N, int K, FA fa, FB fb, EP 
 }
 
 template <int ND, typename T, int NP, int NW>
-__global__ void __launch_bounds__(32 * NW, 1) gdn_bwd_frame_mma_kernel(BwdParams p) {
+__global__ void __launch_bounds__(32 * NW, 1) gdn_bwd_frame_mma_kernel(BwdParams p, GdnParams rp) {
   constexpr int kTh = 32 * NW;
   constexpr int NB = NW >= 16 ? 1 : 2;  // 8-column tiles per warp block: more warps, narrower blocks
   using SM = FrameSmemT<ND, 4>;
@@ -827,7 +846,7 @@ __global__ void __launch_bounds__(32 * NW, 1) gdn_bwd_frame_mma_kernel(BwdParams
       prefetch_l2(k + (t0 + kC) * dk, (long)nn * dk * sizeof(T));
       prefetch_l2(v + (t0 + kC) * dv, (long)nn * dv * sizeof(T));
     }
-    load_chunk<SM, T, true, true>(sm, p, k, v, beta, t0, nc, tid);
+    load_chunk<SM, T, true, true>(sm, p, rp, k, v, beta, t0, nc, tid);
     gram();
     __syncthreads();
     inverse(sm, nc, tid);
@@ -909,7 +928,7 @@ __global__ void __launch_bounds__(32 * NW, 1) gdn_bwd_frame_mma_kernel(BwdParams
     const int nc = min(kC, L - c * kC);
     if (c > 0) prefetch_l2(k + (t0 - kC) * dk, (long)kC * dk * sizeof(T));
     asm volatile("cp.async.wait_all;" ::: "memory");  // this thread's copies; load_chunk's barrier publishes them
-    load_chunk<SM, T, false, true>(sm, p, k, v, beta, t0, nc, tid);
+    load_chunk<SM, T, false, true>(sm, p, rp, k, v, beta, t0, nc, tid);
     wrun<ND, NB, NP, false, false>(dk, dv, nc, Kcol, [&](int t, int n) { return sm.U[t * LD + n]; },
                                    [&](int m, int n, float x) { sm.S[m * LD + n] -= x; });  // the chunk's start state
     wrun<3, NB, NP, false, true>(kC, dv, dk, Krow, [&](int kk, int n) { return sm.H[kk * LD + n]; },
@@ -1007,7 +1026,7 @@ struct QdoSmem {
 };
 
 template <int ND, typename T, int NP>
-__global__ void __launch_bounds__(kThreads) gdn_bwd_qdo_kernel(BwdParams p) {
+__global__ void __launch_bounds__(kThreads) gdn_bwd_qdo_kernel(BwdParams p, GdnParams rp) {
   using SM = QdoSmem<ND>;
   constexpr int LD = SM::LD;
   extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -1031,6 +1050,10 @@ __global__ void __launch_bounds__(kThreads) gdn_bwd_qdo_kernel(BwdParams p) {
     tile_load(sm.q, LD, q + (long)t0 * dk, dk, nt, nt, dk);
     tile_load(sm.d, LD, d_o + (long)t0 * dv, dv, nt, nt, dv);
     __syncthreads();
+    if (rp.rope_on) {
+      rope_rows(sm.q, LD, nt, dk, f, t0, rp);
+      __syncthreads();
+    }
     if (has)
       wmm<ND, 2, NP>(acc, 0, warp * 16, nt, [&](int m, int t) { return sm.q[t * LD + m]; },
                      [&](int t, int n) { return sm.d[t * LD + n]; });
@@ -1043,12 +1066,33 @@ __global__ void __launch_bounds__(kThreads) gdn_bwd_qdo_kernel(BwdParams p) {
     });
 }
 
+// With the embedding: dq and dk hold the gradients with respect to the rotated q
+// and k; each pair is turned back by the transpose rotation, R^T x = (y.x, -y.y)
+// with y = R (x.x, -x.y).
+__global__ void gdn_bwd_rope_back_kernel(float *dq, float *dk, long ntok, int F, int L, int d, GdnParams rp) {
+  const int np = d / 2;
+  const long total = ntok * np;
+  for (long e = blockIdx.x * (long)blockDim.x + threadIdx.x; e < total; e += (long)gridDim.x * blockDim.x) {
+    const long tok = e / np;
+    const int pr = (int)(e - tok * np);
+    const long tt = tok % ((long)F * L);  // token index in its head's sequence
+    const int f = (int)(tt / L), tf = (int)(tt - (long)f * L);
+    float *px[2] = {dq + tok * d + 2 * pr, dk + tok * d + 2 * pr};
+#pragma unroll
+    for (int w = 0; w < 2; ++w) {
+      const float2 y = rope_pair(make_float2(px[w][0], -px[w][1]), 2 * pr, f, tf, rp);
+      px[w][0] = y.x;
+      px[w][1] = -y.y;
+    }
+  }
+}
+
 // tf32 passes of the warp-MMA frame kernel (bf16 inputs): 3 = high/low split
 constexpr int kMmaPasses = 1;
 constexpr int kMmaWarps = 8;  // warps of the warp-MMA frame kernel (16 measured slower: a phase is as long as its k-loop)
 
 template <int ND, typename T>
-cudaError_t launch_nd(const BwdParams &p, cudaStream_t st) {
+cudaError_t launch_nd(const BwdParams &p, const GdnParams &rp, cudaStream_t st) {
   constexpr bool mma = std::is_same<T, __nv_bfloat16>::value;
   const size_t sa = sizeof(AdjSmem<ND>);
   const size_t sf = mma ? sizeof(FrameSmemT<ND, 4>) : sizeof(FrameSmem<ND>);
@@ -1061,7 +1105,7 @@ cudaError_t launch_nd(const BwdParams &p, cudaStream_t st) {
   if (e != cudaSuccess) return e;
   const int BH = p.B * p.H;
   const int ncg = (p.dv + 15) / 16;
-  gdn_bwd_qdo_kernel<ND, T, qnp><<<(unsigned)((long)BH * p.F), kThreads, sq, st>>>(p);
+  gdn_bwd_qdo_kernel<ND, T, qnp><<<(unsigned)((long)BH * p.F), kThreads, sq, st>>>(p, rp);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   gdn_bwd_adjoint_kernel<ND><<<BH * ncg, kThreads, sa, st>>>(p);
@@ -1072,21 +1116,25 @@ cudaError_t launch_nd(const BwdParams &p, cudaStream_t st) {
     e = cudaFuncSetAttribute(gdn_bwd_frame_mma_kernel<ND, T, kMmaPasses, kMmaWarps>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sf);
     if (e != cudaSuccess) return e;
-    gdn_bwd_frame_mma_kernel<ND, T, kMmaPasses, kMmaWarps><<<grid, 32 * kMmaWarps, sf, st>>>(p);
+    gdn_bwd_frame_mma_kernel<ND, T, kMmaPasses, kMmaWarps><<<grid, 32 * kMmaWarps, sf, st>>>(p, rp);
   } else {
     e = cudaFuncSetAttribute(gdn_bwd_frame_kernel<ND, T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sf);
     if (e != cudaSuccess) return e;
-    gdn_bwd_frame_kernel<ND, T><<<grid, kThreads, sf, st>>>(p);
+    gdn_bwd_frame_kernel<ND, T><<<grid, kThreads, sf, st>>>(p, rp);
   }
   return cudaGetLastError();
 }
 
 template <typename T>
-cudaError_t launch_t(const BwdParams &p, cudaStream_t st) {
+cudaError_t launch_t(const BwdParams &p, const GdnParams &rp, cudaStream_t st) {
   const int d = p.dk > p.dv ? p.dk : p.dv;
-  if (d <= 32) return launch_nd<2, T>(p, st);
-  if (d <= 64) return launch_nd<4, T>(p, st);
-  return launch_nd<7, T>(p, st);
+  cudaError_t e = d <= 32 ? launch_nd<2, T>(p, rp, st) : (d <= 64 ? launch_nd<4, T>(p, rp, st) : launch_nd<7, T>(p, rp, st));
+  if (e != cudaSuccess || !rp.rope_on) return e;
+  const long ntok = (long)p.B * p.H * p.F * p.L;
+  const long work = ntok * (p.dk / 2);
+  const int blocks = (int)(work / 256 + 1 < 4096 ? work / 256 + 1 : 4096);
+  gdn_bwd_rope_back_kernel<<<blocks, 256, 0, st>>>(p.dq, p.dk_out, ntok, p.F, p.L, p.dk, rp);
+  return cudaGetLastError();
 }
 
 }  // namespace bwd
@@ -1094,9 +1142,9 @@ cudaError_t launch_t(const BwdParams &p, cudaStream_t st) {
 bool gdn_bwd_supported(int dk, int dv) { return dk >= 1 && dv >= 1 && dk <= 112 && dv <= 112; }
 int gdn_bwd_chunks(int L) { return (L + bwd::kC - 1) / bwd::kC; }
 
-cudaError_t launch_gdn_bwd(const BwdParams &p, int in_dtype, cudaStream_t st) {
+cudaError_t launch_gdn_bwd(const BwdParams &p, const GdnParams &rope, int in_dtype, cudaStream_t st) {
   if (!gdn_bwd_supported(p.dk, p.dv)) return cudaErrorInvalidValue;
-  return in_dtype == GDN_DTYPE_F32 ? bwd::launch_t<float>(p, st) : bwd::launch_t<__nv_bfloat16>(p, st);
+  return in_dtype == GDN_DTYPE_F32 ? bwd::launch_t<float>(p, rope, st) : bwd::launch_t<__nv_bfloat16>(p, rope, st);
 }
 
 }  // namespace gdn

@@ -34,10 +34,11 @@ cudaError_t launch_softmax_window(const void *q, const void *k, const void *v, f
 cudaError_t launch_softmax_window_simt(const void *q, const void *k, const void *v, float *o, int B, int H, int F,
                                        int L, int dk, int dv, int W, float scale, int in_dtype, cudaStream_t st);
 // backward of the Gated DeltaNet (after the recompute has filled p.maps and p.states):
-// the adjoint frame chain, then the frame-parallel chunked backward; d_k, d_v <= 112
+// Q^T dO per frame, the adjoint frame chain, then the frame-parallel chunked backward;
+// d_k, d_v <= 112.  rope: the 3D RoPE's table fields (rope.rope_on = 0: none)
 bool gdn_bwd_supported(int dk, int dv);
 int gdn_bwd_chunks(int L);  // 48-token chunks per frame of the frame kernel
-cudaError_t launch_gdn_bwd(const BwdParams &p, int in_dtype, cudaStream_t st);
+cudaError_t launch_gdn_bwd(const BwdParams &p, const GdnParams &rope, int in_dtype, cudaStream_t st);
 bool relu_tc_supported(int dk, int dv);
 cudaError_t launch_relu_tc(const ReluParams &p, int grid, cudaStream_t st);
 

@@ -203,8 +203,8 @@ def test_no_device_is_reported_without_gpu(lib):
 
 def test_backward_workspace_and_argument_validation(lib):
     """gdn_frame_bwd: the workspace holds the recompute's chain scratch, then
-    A_f^T, S_f and G_f of every frame and the dalpha partial sums; host checks
-    come before any device work."""
+    A_f^T, S_f and G_f of every frame, the dalpha partial sums and (with the 3D
+    RoPE) its table; host checks come before any device work."""
     up = lambda x: (x + 255) // 256 * 256
     B, H, F, L, d = 1, 20, 240, 920, 112
     fr = B * H * F
@@ -222,6 +222,17 @@ def test_backward_workspace_and_argument_validation(lib):
     chain32 = 256 + up(fr * 4) + up(fr * d * d * 4)
     assert lib.workspace_bytes(lib.OP_GDN_BWD, B, H, F, L, d, d, f32) == up(chain32) + 3 * up(fr * d * d * 4) + \
         up(fr * 7 * 4)
+    # the 3D RoPE: the fp32 CUDA-core recompute (so its chain scratch), then the table
+    # (time [F][dt/2], height [L/gw][dh/2], width [gw][dh/2] cos/sin pairs)
+    rope = dict(grid_w=40)
+    dh = 2 * (d // 6)
+    dt = d - 2 * dh
+    table = up(8 * (F * (dt // 2) + (L // 40) * (dh // 2) + 40 * (dh // 2)))
+    simt = lib.make_opts(lib.DTYPE_BF16, stream=0, impl="frame_simt")
+    assert lib.workspace_bytes(lib.OP_GDN_BWD, B, H, F, L, d, d, lib.make_opts(lib.DTYPE_BF16, stream=0, rope=rope)) \
+        == lib.workspace_bytes(lib.OP_GDN_BWD, B, H, F, L, d, d, simt) + table
+    assert lib.workspace_bytes(lib.OP_GDN_BWD, B, H, F, L, d, d, lib.make_opts(lib.DTYPE_F32, stream=0, rope=rope)) \
+        == lib.workspace_bytes(lib.OP_GDN_BWD, B, H, F, L, d, d, f32) + table
     raw = lib._lib
     P = ctypes.c_void_p
     q, k, v, a, b, do = (P(0x1000000 * (i + 1)) for i in range(6))
@@ -237,9 +248,11 @@ def test_backward_workspace_and_argument_validation(lib):
     assert call(q, k, v, a, b, None, do, None, P(0x1000000 + 64), *outs[1:]) == lib.ERR_INVALID_ARG  # dq in q
     assert call(q, k, v, a, b, None, do, None, outs[0], outs[0], *outs[2:]) == lib.ERR_INVALID_ARG  # dq = dk
     assert call(P(0x1000004), k, v, a, b, None, do, None, *outs) == lib.ERR_INVALID_ARG  # misaligned
-    o.rope_grid_w = 4
-    assert call(q, k, v, a, b, None, do, None, *outs) == lib.ERR_UNSUPPORTED              # no RoPE backward
-    o.rope_grid_w = 0
+    o.rope_grid_w = 5
+    assert call(q, k, v, a, b, None, do, None, *outs) == lib.ERR_INVALID_ARG              # L % grid_w != 0
+    o.rope_grid_w, o.rope_frame_offset = 4, -1
+    assert call(q, k, v, a, b, None, do, None, *outs) == lib.ERR_INVALID_ARG              # negative offset
+    o.rope_grid_w, o.rope_frame_offset = 0, 0
     o.impl = lib.IMPL_SEQ
     assert call(q, k, v, a, b, None, do, None, *outs) == lib.ERR_INVALID_ARG              # no such recompute
     o.impl = lib.IMPL_AUTO
@@ -247,4 +260,7 @@ def test_backward_workspace_and_argument_validation(lib):
     import torch
     if not torch.cuda.is_available():  # valid arguments: the device check comes last
         assert call(q, k, v, a, b, None, do, None, *outs) == lib.ERR_NO_DEVICE
+        o.rope_grid_w = 4
+        assert call(q, k, v, a, b, None, do, None, *outs) == lib.ERR_NO_DEVICE
+        o.rope_grid_w = 0
     del ws

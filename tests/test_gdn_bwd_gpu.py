@@ -37,21 +37,22 @@ def case(B, H, F, L, dk, dv, dtype, seed, logits=True, s_in=True, ds_out=True):
     return w, x, g["d_o"], g["state_in"], g["dstate_out"]
 
 
-def run(lib, dev, w, x, d_o, si, dso, logits=True, heads=None, **kw):
+def run(lib, dev, w, x, d_o, si, dso, logits=True, heads=None, rope=None, **kw):
     """The GPU gradients and the oracle's; with ``heads`` (flat head indices, B = 1)
-    only those heads, the oracle run on them alone (heads are independent)."""
+    only those heads, the oracle run on them alone (heads are independent).
+    ``rope``: the 3D RoPE options, given to both sides."""
     t, h = device_inputs(w, x, dev, torch)
     tsi = None if si is None else torch.from_numpy(si).to(dev)
     tds = None if dso is None else torch.from_numpy(dso).to(dev)
     g = lib.gdn_frame_bwd(t["q"], t["k"], t["v"], t["a"], t["b"], torch.from_numpy(d_o).to(dev), F=w.F,
-                          state_in=tsi, d_state_out=tds, gates_are_logits=logits, **kw)
+                          state_in=tsi, d_state_out=tds, gates_are_logits=logits, rope=rope, **kw)
     torch.cuda.synchronize()
     sel = (lambda a: a) if heads is None else (lambda a: a[:, heads])
     out = {n: sel(g[n]).cpu().numpy() for n in NAMES}
     del g, t
     ref = oracle.gdn_bwd(*(sel(h[n]) for n in ("q", "k", "v", "a", "b")), sel(d_o), F=w.F, L=w.L,
                          gates_are_logits=logits, state_in=None if si is None else sel(si),
-                         dstate_out=None if dso is None else sel(dso))
+                         dstate_out=None if dso is None else sel(dso), rope=rope)
     return out, ref
 
 
@@ -142,3 +143,38 @@ def test_480p_5s_all_heads(lib, dev):
     g = synth.grad_inputs(w, state_in=True, dstate_out=True)
     out, ref = run(lib, dev, w, x, g["d_o"], g["state_in"], g["dstate_out"])
     check(out, ref, TOL_BF16)
+
+
+# B, H, F, L, dk, dv, grid_w, frame_offset: the 3D RoPE (time, height and width
+# bands of d_k) on q and k, with ragged 48-token chunks and a resumed clip's offset
+ROPE = [(1, 2, 3, 40, 32, 32, 8, 0), (1, 1, 4, 100, 112, 112, 10, 5), (2, 1, 2, 60, 48, 64, 12, 2)]
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("shape", ROPE)
+def test_rope_matches_oracle(lib, dev, shape, dtype):
+    """The forward with the embedding on q and k (the fp32 CUDA-core recompute),
+    its gradients taken back through the rotation, against the oracle's."""
+    *sz, gw, off = shape
+    w, x, d_o, si, dso = case(*sz, dtype, seed=sz[3] + 11)
+    out, ref = run(lib, dev, w, x, d_o, si, dso, rope=dict(grid_w=gw, frame_offset=off))
+    check(out, ref, TOL_F32 if dtype == "f32" else TOL_BF16)
+
+
+def test_rope_720p_60s_one_head(lib, dev):
+    """The benchmark's workload with the embedding (40 x 23 token grid per frame):
+    head 7 in full (every frame, token and column) against the oracle."""
+    w = synth.WORKLOADS["gdn_720p_60s"]
+    x = synth.inputs(w)
+    d_o = synth.grad_inputs(w)["d_o"]
+    out, ref = run(lib, dev, w, x, d_o, None, None, heads=[7], rope=dict(grid_w=40))
+    check(out, ref, TOL_BF16)
+
+
+def test_rope_tensor_core_recompute_refused(lib, dev):
+    """The tensor-core recompute has no embedding: forcing it is refused."""
+    w, x, d_o, _, _ = case(1, 1, 2, 16, 32, 32, "bf16", seed=5)
+    t, _ = device_inputs(w, x, dev, torch)
+    with pytest.raises(lib.GdnError):
+        lib.gdn_frame_bwd(t["q"], t["k"], t["v"], t["a"], t["b"], torch.from_numpy(d_o).to(dev), F=w.F,
+                          impl="tc", rope=dict(grid_w=8))
