@@ -351,6 +351,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         extra["temporal_conv"] = temporal_conv_leg(args, lib, synth, torch, dev, stream, cpu_on)
         extra["softmax_window"] = softmax_window_leg(args, lib, synth, torch, dev, stream, cpu_on)
         extra["backward"] = backward_leg(args, lib, synth, torch, dev, stream, cpu_on)
+        extra["rope"] = rope_leg(args, lib, synth, torch, dev, stream, cpu_on)
     peak, peak_src = measured_peaks()
     alg_bytes = token_heads * BYTES_PER_TOKEN_HEAD + w.B * w.H * (w.F * 4 + w.dk * w.dv * 4)
     achieved = alg_bytes / (ms / 1e3) / 1e9
@@ -819,6 +820,61 @@ def backward_leg(args, lib, synth, torch, dev, stream, cpu_baseline_on):
             w.B * Fs * w.L, target_s=4.0)
         res["cpu_baseline"] = {"value": tps, "unit": "tokens/s", "cores": nthreads, "kind": "oracle",
                                "sample": f"the backward of the first {Fs} of {w.F} frames of all {w.H} heads, "
+                                         f"{runs} runs in {secs:.1f} s"}
+    return res
+
+
+def rope_leg(args, lib, synth, torch, dev, stream, cpu_baseline_on):
+    """The headline workload (720p 60 s) with the 3D RoPE on q and k: 920 tokens
+    per frame as a 23 x 40 latent grid (grid_w = 40).  The forward is the
+    tensor-core kernel's RoPE instantiation (the rotation fused where q and k
+    are loaded) after the angle-table kernel; the backward with the embedding
+    is timed beside it (one call: table, tensor-core recompute, Q^T dO,
+    adjoint chain, frame kernel, the transpose rotation of dq and dk)."""
+    w = synth.WORKLOADS["gdn_720p_60s"]
+    x = synth.inputs(w)
+    q, k, v = (torch.from_numpy(x[n]).to(torch.bfloat16).to(dev) for n in "qkv")
+    a, b = (torch.from_numpy(x[n]).to(dev) for n in "ab")
+    rope = dict(grid_w=40)
+    opts = lib.make_opts(lib.DTYPE_BF16, rope=rope)
+    o = torch.empty((w.B, w.H, w.N, w.dv), dtype=torch.float32, device=dev)
+    s_out = torch.empty((w.B, w.H, w.dk, w.dv), dtype=torch.float32, device=dev)
+    ws = lib.alloc_workspace(lib.workspace_bytes(lib.OP_GDN, w.B, w.H, w.F, w.L, w.dk, w.dv, opts), dev)
+    call = lambda: lib.gdn_frame_fwd(q, k, v, a, b, F=w.F, o=o, state_out=s_out, workspace=ws, rope=rope)
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    ms = _events_ms(call, max(5, args.steps // 2), stream)
+    peak, src = measured_peaks()
+    # the same algorithmic bytes as without the embedding: the angle table (a few KB) stays in L2
+    roof = dict(_roofline(_gdn_alg_bytes(w), ms, peak, src), traffic=None,
+                traffic_source="not captured for the RoPE instantiation")
+    res = {"workload": f"{WORKLOAD} with the 3D RoPE (grid 23 x 40)", "B": w.B, "H": w.H, "F": w.F, "L": w.L,
+           "d": w.dk, "ms": ms, "tokens_per_s": w.B * w.N / (ms / 1e3), "roofline": roof,
+           "kernel": "gdn_tc_kernel<0,1,0> after the angle-table kernel", "launches_per_call": 2,
+           "l2": "inputs 2.97 GB, larger than L2; no flush needed"}
+    del o, s_out, ws
+    d_o = torch.from_numpy(synth.grad_inputs(w)["d_o"]).to(dev)
+    bopts = lib.make_opts(lib.DTYPE_BF16, rope=rope)
+    bws = lib.alloc_workspace(lib.workspace_bytes(lib.OP_GDN_BWD, w.B, w.H, w.F, w.L, w.dk, w.dv, bopts), dev)
+    g = lib.gdn_frame_bwd(q, k, v, a, b, d_o, F=w.F, workspace=bws, rope=rope)
+    bcall = lambda: lib.gdn_frame_bwd(q, k, v, a, b, d_o, F=w.F, workspace=bws, out=g, rope=rope)
+    bcall()
+    torch.cuda.synchronize()
+    res["backward_ms"] = _events_ms(bcall, 2, stream)
+    res["backward_launches_per_call"] = 6
+    del q, k, v, a, b, d_o, g, bws
+    if cpu_baseline_on:
+        import oracle
+        frames = 3
+        xs = synth.inputs(w, frames=frames)
+        hx = {n: torch.from_numpy(xs[n]).to(torch.bfloat16).float().numpy() for n in "qkv"}
+        nthreads = os.cpu_count() or 1
+        tps, runs, secs = _oracle_tokens_per_s(
+            lambda: oracle.gdn(hx["q"], hx["k"], hx["v"], xs["a"], xs["b"], F=frames, L=w.L, nthreads=nthreads,
+                               rope=rope), w.B * frames * w.L)
+        res["cpu_baseline"] = {"value": tps, "unit": "tokens/s", "cores": nthreads, "kind": "oracle",
+                               "sample": f"all {w.H} heads x first {frames} of {w.F} frames with the embedding, "
                                          f"{runs} runs in {secs:.1f} s"}
     return res
 

@@ -210,11 +210,11 @@ GDN_API int gdn_frame_fwd(const void *q, const void *k, const void *v, const flo
  * row per token, plus the recompute's scratch, plus the RoPE table).
  *
  * 3D RoPE (opts->rope_grid_w > 0, the forward call's rope_grid_w,
- * rope_frame_offset and rope_base; the same checks): the recompute is
- * FRAME_SIMT (GDN_IMPL_TC is refused with GDN_ERR_UNSUPPORTED); the kernels
- * rotate q and k where they load them, and d_q, d_k are turned back through
- * the transpose rotation, so they are gradients with respect to the unrotated
- * inputs, as the forward receives them.
+ * rope_frame_offset and rope_base; the same checks): every kernel rotates q
+ * and k where it loads them, and d_q, d_k are turned back through the
+ * transpose rotation, so they are gradients with respect to the unrotated
+ * inputs, as the forward receives them (one more launch, and one first for
+ * the angle table).
  *
  * Precision: with bf16 inputs the recomputed A_f and S_f carry the tensor-core
  * forward's rounding (see gdn_frame_fwd), and the products of Q_f^T dO_f and of

@@ -198,12 +198,10 @@ extern "C" const char *gdn_status_str(int s) { return gdn_status_string(s); }
 namespace gdn {
 namespace {
 // The backward's forward recompute: the tensor-core kernel for bf16 inputs where it
-// applies (one unit per frame, no position embedding), else the fp32 CUDA-core
-// frame kernel.
+// applies (one unit per frame), else the fp32 CUDA-core frame kernel.
 int pick_bwd_fwd_impl(const gdn_opts_t *o, int dk, int dv) {
   if (o->impl == GDN_IMPL_FRAME_SIMT) return GDN_IMPL_FRAME_SIMT;
   if (o->impl == GDN_IMPL_TC) return GDN_IMPL_TC;
-  if (o->rope_grid_w != 0) return GDN_IMPL_FRAME_SIMT;
   return o->in_dtype == GDN_DTYPE_BF16 && gdn_tc_supported(dk, dv) ? GDN_IMPL_TC : GDN_IMPL_FRAME_SIMT;
 }
 
@@ -281,7 +279,7 @@ extern "C" int gdn_frame_bwd(const void *q, const void *k, const void *v, const 
   if (rc != GDN_OK) return rc;
   if (cc != 100) return GDN_ERR_NO_DEVICE;
   const int fimpl = pick_bwd_fwd_impl(opts, dk, dv);
-  if (fimpl == GDN_IMPL_TC && (opts->in_dtype != GDN_DTYPE_BF16 || !gdn_tc_supported(dk, dv) || rope))
+  if (fimpl == GDN_IMPL_TC && (opts->in_dtype != GDN_DTYPE_BF16 || !gdn_tc_supported(dk, dv)))
     return GDN_ERR_UNSUPPORTED;
   const BwdLayout w = bwd_layout(opts, B, H, F, L, dk, dv);
   if (!opts->workspace || opts->workspace_bytes < w.total) return GDN_ERR_INVALID_ARG;

@@ -196,6 +196,27 @@ __device__ __forceinline__ void blk_row_mul(float4 &acc, const float *A, const f
 }
 __device__ __forceinline__ float4 neg4(float4 v) { return make_float4(-v.x, -v.y, -v.z, -v.w); }
 
+// 3D RoPE of one token: where its time, height and width rows start in the angle
+// table (time [F][dt/2], height [L/gw][dh/2], width [gw][dh/2]), each less the
+// pair index of its band's first pair, so that pair j of any band is entry off + j.
+// The division by the grid width is taken once per token, not once per pair.
+struct RopeTok {
+  int t_off, h_off, w_off;
+};
+__device__ __forceinline__ RopeTok rope_tok(int f, int tf, const GdnParams &p) {
+  const int row = tf / p.rope_gw, col = tf - row * p.rope_gw;
+  const int ht = p.F * (p.rope_dt / 2), hp = p.rope_dh / 2;
+  return {f * (p.rope_dt / 2), ht + row * hp - p.rope_dt / 2,
+          ht + (p.L / p.rope_gw) * hp + col * hp - (p.rope_dt + p.rope_dh) / 2};
+}
+// The pair (dd, dd + 1) (dd even) rotated by its angle: the band is a select, not a
+// branch (lanes of a warp hold pairs of different bands).
+__device__ __forceinline__ float2 rope_at(float2 x, int dd, const RopeTok &r, const GdnParams &p) {
+  const int off = dd < p.rope_dt ? r.t_off : (dd < p.rope_dt + p.rope_dh ? r.h_off : r.w_off);
+  const float2 cs = __ldg(p.rope_tab + off + (dd >> 1));
+  return make_float2(fmaf(x.x, cs.x, -x.y * cs.y), fmaf(x.x, cs.y, x.y * cs.x));
+}
+
 // kSeg: frames split into p.segs chunk segments (else one unit per frame; the
 // segment arithmetic folds away)
 // kRope: the 3D rotary position embedding on q and k (a separate instantiation,
@@ -372,7 +393,8 @@ __global__ void __launch_bounds__(kGThreads, 1)
           const float inv = 1.0f / fmaxf(sqrtf(ss), kKeyNormEps);  // the rotation keeps the norm
           const int tf = c * kC + t;  // token index in the frame
           const bool rot = kRope && tf < L;
-          const int fr = rot ? unit_of(tk).f : 0;
+          RopeTok rtok = {0, 0, 0};
+          if (rot) rtok = rope_tok(unit_of(tk).f, tf, p);
 #pragma unroll
           for (int ch = 0; ch < 8; ++ch) {
             const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&ku[ch]);
@@ -381,7 +403,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
             for (int e = 0; e < 4; ++e) {
               float2 v2 = __bfloat1622float2(h[e]);
               const int dd = kb * 64 + ch * 8 + 2 * e;  // this pair's first dimension
-              if (rot && dd < dk) v2 = rope_pair(v2, dd, fr, tf, p);
+              if (rot && dd < dk) v2 = rope_at(v2, dd, rtok, p);
               o[e] = pack_h2(v2.x * inv, v2.y * inv);
             }
             *reinterpret_cast<uint4 *>(krow + sw128_offset(t, ch * 8)) = make_uint4(o[0], o[1], o[2], o[3]);
@@ -1100,6 +1122,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
             const int kb = i >> 9, rw = (i >> 3) & 63, pc = i & 7;
             const int ch = pc ^ (rw & 7);
             const int tf = tb0 + n * kQTok + rw;  // token index in the frame
+            const RopeTok rtok = rope_tok(f, tf < L ? tf : 0, p);
             uint4 *cp = reinterpret_cast<uint4 *>(qb + kb * 8192 + rw * 128 + pc * 16);
             const uint4 u = *cp;
             const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
@@ -1108,7 +1131,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
             for (int e = 0; e < 4; ++e) {
               float2 v2 = __bfloat1622float2(h[e]);
               const int dd = kb * 64 + ch * 8 + 2 * e;
-              if (tf < L && dd < dk) v2 = rope_pair(v2, dd, f, tf, p);
+              if (tf < L && dd < dk) v2 = rope_at(v2, dd, rtok, p);
               qmax = fmaxf(qmax, fmaxf(fabsf(v2.x), fabsf(v2.y)));
               o4[e] = pack_h2(v2.x, v2.y);
             }
@@ -1224,6 +1247,18 @@ static cudaError_t launch_tc(const GdnParams &p, int grid, bool cooperative, cud
   return cudaLaunchKernelEx(&cfg, gdn_tc_kernel<true, kRope>, mq, mk, mv, p);
 }
 
+// the backward's recompute (kSave): maps and end states, no read-out
+template <bool kRope>
+static cudaError_t launch_save(const GdnParams &p, int grid, cudaStream_t st, const CUtensorMap &mq,
+                               const CUtensorMap &mk, const CUtensorMap &mv) {
+  using namespace tc;
+  cudaError_t e = cudaFuncSetAttribute(gdn_tc_kernel<false, kRope, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)kGdnSmemBytes);
+  if (e != cudaSuccess) return e;
+  gdn_tc_kernel<false, kRope, true><<<grid, kGThreads, kGdnSmemBytes, st>>>(mq, mk, mv, p);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_gdn_tc(const GdnParams &p, int grid, bool cooperative, cudaStream_t st) {
   using namespace tc;
   CUtensorMap mq, mk, mv;
@@ -1231,13 +1266,9 @@ cudaError_t launch_gdn_tc(const GdnParams &p, int grid, bool cooperative, cudaSt
   if (!make_bf16_map(&mq, p.q, p.dk, p.L, p.F, BH, kQTok) || !make_bf16_map(&mk, p.k, p.dk, p.L, p.F, BH, 64) ||
       !make_bf16_map(&mv, p.v, p.dv, p.L, p.F, BH, 64))
     return cudaErrorInvalidValue;
-  if (p.save_maps) {  // the backward's recompute: one unit per frame, no position embedding
-    if (cooperative || p.rope_on || !p.save_states) return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(gdn_tc_kernel<false, false, true>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGdnSmemBytes);
-    if (e != cudaSuccess) return e;
-    gdn_tc_kernel<false, false, true><<<grid, kGThreads, kGdnSmemBytes, st>>>(mq, mk, mv, p);
-    return cudaGetLastError();
+  if (p.save_maps) {  // the backward's recompute: one unit per frame
+    if (cooperative || !p.save_states) return cudaErrorInvalidValue;
+    return p.rope_on ? launch_save<true>(p, grid, st, mq, mk, mv) : launch_save<false>(p, grid, st, mq, mk, mv);
   }
   return p.rope_on ? launch_tc<true>(p, grid, cooperative, st, mq, mk, mv)
                    : launch_tc<false>(p, grid, cooperative, st, mq, mk, mv);

@@ -222,15 +222,14 @@ def test_backward_workspace_and_argument_validation(lib):
     chain32 = 256 + up(fr * 4) + up(fr * d * d * 4)
     assert lib.workspace_bytes(lib.OP_GDN_BWD, B, H, F, L, d, d, f32) == up(chain32) + 3 * up(fr * d * d * 4) + \
         up(fr * 7 * 4)
-    # the 3D RoPE: the fp32 CUDA-core recompute (so its chain scratch), then the table
-    # (time [F][dt/2], height [L/gw][dh/2], width [gw][dh/2] cos/sin pairs)
+    # the 3D RoPE: the same layout, then the table (time [F][dt/2], height [L/gw][dh/2],
+    # width [gw][dh/2] cos/sin pairs)
     rope = dict(grid_w=40)
     dh = 2 * (d // 6)
     dt = d - 2 * dh
     table = up(8 * (F * (dt // 2) + (L // 40) * (dh // 2) + 40 * (dh // 2)))
-    simt = lib.make_opts(lib.DTYPE_BF16, stream=0, impl="frame_simt")
     assert lib.workspace_bytes(lib.OP_GDN_BWD, B, H, F, L, d, d, lib.make_opts(lib.DTYPE_BF16, stream=0, rope=rope)) \
-        == lib.workspace_bytes(lib.OP_GDN_BWD, B, H, F, L, d, d, simt) + table
+        == want + table
     assert lib.workspace_bytes(lib.OP_GDN_BWD, B, H, F, L, d, d, lib.make_opts(lib.DTYPE_F32, stream=0, rope=rope)) \
         == lib.workspace_bytes(lib.OP_GDN_BWD, B, H, F, L, d, d, f32) + table
     raw = lib._lib

@@ -153,8 +153,9 @@ ROPE = [(1, 2, 3, 40, 32, 32, 8, 0), (1, 1, 4, 100, 112, 112, 10, 5), (2, 1, 2, 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("shape", ROPE)
 def test_rope_matches_oracle(lib, dev, shape, dtype):
-    """The forward with the embedding on q and k (the fp32 CUDA-core recompute),
-    its gradients taken back through the rotation, against the oracle's."""
+    """The forward with the embedding on q and k (recomputed by the tensor-core
+    kernel for bf16 inputs, the CUDA-core one for fp32), its gradients taken
+    back through the rotation, against the oracle's."""
     *sz, gw, off = shape
     w, x, d_o, si, dso = case(*sz, dtype, seed=sz[3] + 11)
     out, ref = run(lib, dev, w, x, d_o, si, dso, rope=dict(grid_w=gw, frame_offset=off))
@@ -171,10 +172,9 @@ def test_rope_720p_60s_one_head(lib, dev):
     check(out, ref, TOL_BF16)
 
 
-def test_rope_tensor_core_recompute_refused(lib, dev):
-    """The tensor-core recompute has no embedding: forcing it is refused."""
-    w, x, d_o, _, _ = case(1, 1, 2, 16, 32, 32, "bf16", seed=5)
-    t, _ = device_inputs(w, x, dev, torch)
-    with pytest.raises(lib.GdnError):
-        lib.gdn_frame_bwd(t["q"], t["k"], t["v"], t["a"], t["b"], torch.from_numpy(d_o).to(dev), F=w.F,
-                          impl="tc", rope=dict(grid_w=8))
+def test_rope_recompute_kernels_agree(lib, dev):
+    """bf16 inputs with the embedding and the fp32 CUDA-core recompute forced
+    (the default is the tensor-core one): the same gradients."""
+    w, x, d_o, si, dso = case(1, 2, 3, 70, 64, 64, "bf16", seed=79)
+    out, ref = run(lib, dev, w, x, d_o, si, dso, impl="frame_simt", rope=dict(grid_w=10, frame_offset=1))
+    check(out, ref, TOL_BF16)
