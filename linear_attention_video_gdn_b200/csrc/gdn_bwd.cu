@@ -274,16 +274,37 @@ struct FrameSmemT {
 template <int ND>
 using FrameSmem = FrameSmemT<ND, 1>;
 
+// 3D RoPE of one token: the start of its time, height and width rows in the angle
+// table (time [F][dt/2], height [L/gw][dh/2], width [gw][dh/2]), each less the pair
+// index of its band's first pair, so that pair j of any band is entry off + j.
+struct RopeRow {
+  int t_off, h_off, w_off;
+};
+__device__ __forceinline__ RopeRow rope_row(int f, int tf, const GdnParams &rp) {
+  const int row = tf / rp.rope_gw, col = tf - row * rp.rope_gw;
+  const int ht = rp.F * (rp.rope_dt / 2), hp = rp.rope_dh / 2;
+  return {f * (rp.rope_dt / 2), ht + row * hp - rp.rope_dt / 2,
+          ht + (rp.L / rp.rope_gw) * hp + col * hp - (rp.rope_dt + rp.rope_dh) / 2};
+}
+// (cos, sin) of the pair (dd, dd + 1), dd even: the band is a select, not a branch
+__device__ __forceinline__ float2 rope_cs(int dd, const RopeRow &r, const GdnParams &rp) {
+  const int off = dd < rp.rope_dt ? r.t_off : (dd < rp.rope_dt + rp.rope_dh ? r.h_off : r.w_off);
+  return __ldg(rp.rope_tab + off + (dd >> 1));
+}
+
 // The 3D rotary position embedding of rows [0, rows) of an fp32 tile (row t = the
-// token at index tf0 + t of frame f), in place, from the table in rp (rope_pair).
+// token at index tf0 + t of frame f), in place: a warp per row, its lanes over the pairs.
 __device__ __forceinline__ void rope_rows(float *x, int ld, int rows, int d, int f, int tf0, const GdnParams &rp) {
-  const int np = d / 2;
-  for (int e = threadIdx.x; e < rows * np; e += blockDim.x) {
-    const int t = e / np, pr = e - t * np;
-    float *px = x + t * ld + 2 * pr;
-    const float2 y = rope_pair(make_float2(px[0], px[1]), 2 * pr, f, tf0 + t, rp);
-    px[0] = y.x;
-    px[1] = y.y;
+  const int lane = threadIdx.x & 31, nw = (int)(blockDim.x >> 5);
+  for (int t = (int)(threadIdx.x >> 5); t < rows; t += nw) {
+    const RopeRow r = rope_row(f, tf0 + t, rp);
+    float *px = x + t * ld;
+    for (int dd = 2 * lane; dd < d; dd += 64) {
+      const float2 cs = rope_cs(dd, r, rp);
+      const float x0 = px[dd], x1 = px[dd + 1];
+      px[dd] = fmaf(x0, cs.x, -x1 * cs.y);
+      px[dd + 1] = fmaf(x0, cs.y, x1 * cs.x);
+    }
   }
 }
 
@@ -1067,22 +1088,23 @@ __global__ void __launch_bounds__(kThreads) gdn_bwd_qdo_kernel(BwdParams p, GdnP
 }
 
 // With the embedding: dq and dk hold the gradients with respect to the rotated q
-// and k; each pair is turned back by the transpose rotation, R^T x = (y.x, -y.y)
-// with y = R (x.x, -x.y).
+// and k; each pair is turned back by the transpose rotation (cos, -sin).  A warp
+// per token, its lanes over the pairs.
 __global__ void gdn_bwd_rope_back_kernel(float *dq, float *dk, long ntok, int F, int L, int d, GdnParams rp) {
-  const int np = d / 2;
-  const long total = ntok * np;
-  for (long e = blockIdx.x * (long)blockDim.x + threadIdx.x; e < total; e += (long)gridDim.x * blockDim.x) {
-    const long tok = e / np;
-    const int pr = (int)(e - tok * np);
+  const int lane = threadIdx.x & 31;
+  const long nwarps = (long)gridDim.x * (blockDim.x >> 5);
+  for (long tok = blockIdx.x * (long)(blockDim.x >> 5) + (threadIdx.x >> 5); tok < ntok; tok += nwarps) {
     const long tt = tok % ((long)F * L);  // token index in its head's sequence
     const int f = (int)(tt / L), tf = (int)(tt - (long)f * L);
-    float *px[2] = {dq + tok * d + 2 * pr, dk + tok * d + 2 * pr};
+    const RopeRow r = rope_row(f, tf, rp);
+    for (int dd = 2 * lane; dd < d; dd += 64) {
+      const float2 cs = rope_cs(dd, r, rp);
 #pragma unroll
-    for (int w = 0; w < 2; ++w) {
-      const float2 y = rope_pair(make_float2(px[w][0], -px[w][1]), 2 * pr, f, tf, rp);
-      px[w][0] = y.x;
-      px[w][1] = -y.y;
+      for (int w = 0; w < 2; ++w) {
+        float2 *px = reinterpret_cast<float2 *>((w ? dk : dq) + tok * d + dd);
+        const float2 x = *px;
+        *px = make_float2(fmaf(x.x, cs.x, x.y * cs.y), fmaf(x.y, cs.x, -x.x * cs.y));
+      }
     }
   }
 }
@@ -1131,8 +1153,7 @@ cudaError_t launch_t(const BwdParams &p, const GdnParams &rp, cudaStream_t st) {
   cudaError_t e = d <= 32 ? launch_nd<2, T>(p, rp, st) : (d <= 64 ? launch_nd<4, T>(p, rp, st) : launch_nd<7, T>(p, rp, st));
   if (e != cudaSuccess || !rp.rope_on) return e;
   const long ntok = (long)p.B * p.H * p.F * p.L;
-  const long work = ntok * (p.dk / 2);
-  const int blocks = (int)(work / 256 + 1 < 4096 ? work / 256 + 1 : 4096);
+  const int blocks = (int)(ntok / 8 + 1 < 148 * 16 ? ntok / 8 + 1 : 148 * 16);  // 8 tokens (warps) per block
   gdn_bwd_rope_back_kernel<<<blocks, 256, 0, st>>>(p.dq, p.dk_out, ntok, p.F, p.L, p.dk, rp);
   return cudaGetLastError();
 }
