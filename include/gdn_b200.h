@@ -107,10 +107,11 @@ typedef struct gdn_opts {
   int segments;           /* gdn on GDN_IMPL_TC.  0 = automatic; P >= 1: split every frame into P
                              runs of whole 64-token chunks handled by P CTAs (see gdn_frame_fwd);
                              P is lowered to the chunk count and to what fits one resident grid */
-  int rope_grid_w;        /* gdn only.  0: no position embedding.  > 0: the 3D rotary position
-                             embedding on q and k (k before its normalisation): a frame's L tokens
-                             are a grid of L / rope_grid_w rows of rope_grid_w tokens (L must be a
-                             multiple); see gdn_frame_fwd.  Not taken by GDN_IMPL_TC_PFORM */
+  int rope_grid_w;        /* gdn only (gdn_frame_fwd and gdn_frame_bwd).  0: no position
+                             embedding.  > 0: the 3D rotary position embedding on q and k (k before
+                             its normalisation): a frame's L tokens are a grid of L / rope_grid_w
+                             rows of rope_grid_w tokens (L must be a multiple); see gdn_frame_fwd.
+                             Not taken by GDN_IMPL_TC_PFORM */
   int rope_frame_offset;  /* time coordinate of the call's first frame (a streaming call: its
                              frame index in the video) */
   float rope_base;        /* frequency base; 0 = 10000 */
