@@ -327,7 +327,7 @@ extern "C" int gdn_frame_bwd(const void *q, const void *k, const void *v, const 
   b.maps = maps; b.states = states;
   b.gbuf = reinterpret_cast<float *>(ws + w.gbuf);
   b.dal_part = reinterpret_cast<float *>(ws + w.part);
-  b.linv_buf = reinterpret_cast<float *>(ws + w.linv);
+  b.linv_buf = w.rbuf > w.linv ? reinterpret_cast<float *>(ws + w.linv) : nullptr;  // bf16 inputs only
   b.rbuf = w.rope > w.rbuf ? reinterpret_cast<float *>(ws + w.rbuf) : nullptr;  // own rows only when dv > dk
   b.dq = dq; b.dk_out = dk_out; b.dv_out = dv_out; b.dalpha = dalpha; b.dbeta = dbeta; b.dstate_in = dstate_in;
   b.B = B; b.H = H; b.F = F; b.L = L; b.dk = dk; b.dv = dv;
