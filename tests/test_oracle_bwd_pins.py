@@ -6,8 +6,8 @@ recurrence.  Each gradient is checked against
     inputs and steps are dyadic so that x +- h is exact in float32 and the
     forward runs in fp64 on exactly the perturbed values),
   * torch autograd through an independent fp64 per-token loop of the forward,
-  * closed forms (no writes, alpha = 1), linearity in (do, dstate_out), and the
-    key-norm clamp,
+  * closed forms (no writes, alpha = 1), linearity in (do, dstate_out),
+    additivity over groups of d_v columns, and the key-norm clamp,
 and a Python copy of the algorithm with plausible mistakes planted in it shows
 that the finite-difference pin fails each of them.
 """
@@ -204,6 +204,31 @@ def test_bwd_linear_in_upstream_gradients_and_head_subsets():
     for n in GRAD.values():
         np.testing.assert_array_equal(gs[n][[0, 2]], g[n][[0, 2]])
         assert np.isnan(gs[n][1]).all()
+
+
+
+@pytest.mark.parametrize("rope", [None, dict(grid_w=2, frame_offset=1)])
+def test_bwd_additive_over_value_columns(rope):
+    """The recurrence never mixes d_v columns: column j of S evolves from column j
+    of v alone, and o's column j reads only it.  So the loss splits into one
+    term per column group, and the gradients of the whole problem are those of
+    its column groups: dq, dk, dalpha and dbeta summed over the groups, dv and
+    dstate_in put side by side."""
+    rng = np.random.default_rng(31)
+    F, L, dk, dv = 3, 4, 6, 5
+    c = _case(rng, 2, F, L, dk, dv)
+    c["rope"] = rope
+    g = _bwd(c, F, L, True)
+    parts = []
+    for cols in (slice(0, 2), slice(2, 5)):
+        ci = dict(c, v=np.ascontiguousarray(c["v"][..., cols]), d_o=np.ascontiguousarray(c["d_o"][..., cols]),
+                  s_in=np.ascontiguousarray(c["s_in"][..., cols]), ds_out=np.ascontiguousarray(c["ds_out"][..., cols]))
+        parts.append(_bwd(ci, F, L, True))
+    for n in ("dq", "dk", "dalpha", "dbeta"):
+        np.testing.assert_allclose(g[n], parts[0][n] + parts[1][n], rtol=1e-10, atol=1e-12, err_msg=n)
+    for n in ("dv", "dstate_in"):
+        np.testing.assert_allclose(g[n], np.concatenate([parts[0][n], parts[1][n]], axis=-1), rtol=1e-10,
+                                   atol=1e-12, err_msg=n)
 
 
 # ---------------------------------------------------------------- planted mistakes
